@@ -1,0 +1,129 @@
+"""fp64 CPU oracle of the DDTS recurrence (test infrastructure only).
+
+Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` import this package; the CUDA library never does, and the two
+share no code.  The arithmetic lives in ``rdm_oracle.c`` (plain C, double
+precision, token by token); this module only builds it with gcc, marshals
+numpy arrays and calls it.
+
+Definition followed (Rodimus*, digest.lyk-ai.com summary, section "Method",
+DDTS gates; paperhub.cn OpenReview rebuttal, "Efficient Parallelization"
+bullet and Q2 on the fixed-size recurrent state):
+
+    alpha_t = exp(-g_t * tau_t),  alpha_hat_t = g_t ** tau_t
+    S_t = diag(alpha_t) S_{t-1} + (alpha_hat_t * k_t)(beta_hat_t * v_t)^T
+    o_t = S_t^T q_t
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "rdm_oracle.c")
+_LIB = os.path.join(_HERE, "librdm_oracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile rdm_oracle.c into librdm_oracle.so next to it (gcc -O2)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c99", "-D_POSIX_C_SOURCE=200809L", "-shared",
+                               "-fPIC", "-o", tmp, _SRC, "-lm", "-lpthread"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def load_library(path: str):
+    """Open a compiled oracle library and declare its C signatures."""
+    lib = ctypes.CDLL(path)
+    P = ctypes.POINTER(ctypes.c_double)
+    I = ctypes.c_int
+    lib.rdm_oracle_fwd.argtypes = [I] * 5 + [P] * 9 + [I]
+    lib.rdm_oracle_bwd.argtypes = [I] * 5 + [P] * 16 + [I]
+    lib.rdm_oracle_decode_step.argtypes = [I] * 4 + [P] * 8 + [I]
+    for f in (lib.rdm_oracle_fwd, lib.rdm_oracle_bwd, lib.rdm_oracle_decode_step):
+        f.restype = I
+    return lib
+
+
+def _load(lib=None):
+    global _lib
+    if lib is not None:
+        return lib
+    if _lib is None:
+        _lib = load_library(build())
+    return _lib
+
+
+def default_threads() -> int:
+    return len(os.sched_getaffinity(0))
+
+
+def _f64(x):
+    """Any array-like (numpy or torch, any float dtype) -> C-contiguous float64 numpy."""
+    if x is None:
+        return None
+    if hasattr(x, "detach"):
+        x = x.detach().to("cpu")
+        import torch
+        x = x.to(torch.float64).numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _p(a):
+    if a is None:
+        return ctypes.POINTER(ctypes.c_double)()
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def fwd(q, k, v, g, tau, beta, S0=None, nthreads=None, lib=None):
+    """Token-by-token forward.  q,k,g,tau [B,H,T,dk]; v,beta [B,H,T,dv];
+    S0 [B,H,dk,dv] or None (zeros).  Returns (o [B,H,T,dv], S_T [B,H,dk,dv])."""
+    q, k, v, g, tau, beta, S0 = map(_f64, (q, k, v, g, tau, beta, S0))
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    o = np.zeros((B, H, T, dv))
+    ST = np.zeros((B, H, dk, dv))
+    rc = _load(lib).rdm_oracle_fwd(B, H, T, dk, dv, _p(q), _p(k), _p(v), _p(g), _p(tau), _p(beta),
+                                _p(S0), _p(o), _p(ST), nthreads or default_threads())
+    if rc != 0:
+        raise RuntimeError("rdm_oracle_fwd failed")
+    return o, ST
+
+
+def bwd(q, k, v, g, tau, beta, S0, dO, dST=None, nthreads=None, lib=None):
+    """Reverse mode of the token loop.  Returns dict dq, dk, dv, dg, dtau, dbeta, dS0."""
+    q, k, v, g, tau, beta, S0, dO, dST = map(_f64, (q, k, v, g, tau, beta, S0, dO, dST))
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    out = {n: np.zeros(q.shape) for n in ("dq", "dk", "dg", "dtau")}
+    out.update({n: np.zeros(v.shape) for n in ("dv", "dbeta")})
+    out["dS0"] = np.zeros((B, H, dk, dv))
+    rc = _load(lib).rdm_oracle_bwd(B, H, T, dk, dv, _p(q), _p(k), _p(v), _p(g), _p(tau), _p(beta),
+                                _p(S0), _p(dO), _p(dST), _p(out["dq"]), _p(out["dk"]),
+                                _p(out["dv"]), _p(out["dg"]), _p(out["dtau"]), _p(out["dbeta"]),
+                                _p(out["dS0"]), nthreads or default_threads())
+    if rc != 0:
+        raise RuntimeError("rdm_oracle_bwd failed")
+    return out
+
+
+def decode_step(q, k, v, g, tau, beta, S, nthreads=None, lib=None):
+    """One token per (b,h).  q,k,g,tau [B,H,dk]; v,beta [B,H,dv]; S [B,H,dk,dv]
+    float64 numpy, updated in place.  Returns o [B,H,dv]."""
+    if not (isinstance(S, np.ndarray) and S.dtype == np.float64 and S.flags.c_contiguous):
+        raise TypeError("S must be a C-contiguous float64 numpy array (updated in place)")
+    q, k, v, g, tau, beta = map(_f64, (q, k, v, g, tau, beta))
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    o = np.zeros((B, H, dv))
+    rc = _load(lib).rdm_oracle_decode_step(B, H, dk, dv, _p(q), _p(k), _p(v), _p(g), _p(tau),
+                                        _p(beta), _p(S), _p(o), nthreads or default_threads())
+    if rc != 0:
+        raise RuntimeError("rdm_oracle_decode_step failed")
+    return o

@@ -1,0 +1,246 @@
+"""Pins of the fp64 oracle against facts the definition fixes.
+
+Each check raises AssertionError on a mismatch.  They take an optional `lib`
+(an oracle library opened with ``oracle.load_library``) so that the same checks
+can be run against deliberately broken builds of the oracle (mutants): every
+plausible slip in the oracle must make at least one of them fail.
+
+Definition (Rodimus*, digest.lyk-ai.com summary, "Method": alpha = exp(-g*tau),
+alpha_hat = g^tau; state S_t = diag(alpha_t) S_{t-1} + (alpha_hat_t k_t)(beta_t v_t)^T,
+o_t = S_t^T q_t, diagonal along n = d_k per the paperhub.cn rebuttal).
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def rand_inputs(rng, B, H, T, dk, dv, g_lo=0.05, g_hi=2.0, tau_lo=0.05, tau_hi=1.0, s0=0.5):
+    return dict(
+        q=rng.standard_normal((B, H, T, dk)),
+        k=rng.standard_normal((B, H, T, dk)),
+        v=rng.standard_normal((B, H, T, dv)),
+        g=rng.uniform(g_lo, g_hi, (B, H, T, dk)),
+        tau=rng.uniform(tau_lo, tau_hi, (B, H, T, dk)),
+        beta=rng.uniform(0.1, 1.0, (B, H, T, dv)),
+        S0=s0 * rng.standard_normal((B, H, dk, dv)),
+    )
+
+
+def close(a, b, tol, what):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    assert a.shape == b.shape, (what, a.shape, b.shape)
+    scale = max(1.0, float(np.max(np.abs(b)))) if b.size else 1.0
+    err = float(np.max(np.abs(a - b))) / scale if a.size else 0.0
+    assert err <= tol, f"{what}: max abs err / max(1,|ref|) = {err:.3e} > {tol:.1e}"
+
+
+# ------------------------------------------------------------------ forward pins
+def check_worked_example(lib=None):
+    """Hand-derived T=3 example (tests/golden/ddts_worked_example_T3.json)."""
+    fx = json.load(open(os.path.join(GOLDEN, "ddts_worked_example_T3.json")))
+    shp = lambda a: np.asarray(a, dtype=np.float64)[None, None]
+    o, ST = oracle.fwd(shp(fx["q"]), shp(fx["k"]), shp(fx["v"]), shp(fx["g"]), shp(fx["tau"]),
+                       shp(fx["beta"]), shp(fx["S0"]), lib=lib)
+    close(o[0, 0], fx["expected_o"], fx["tolerance"], "worked example o")
+    close(ST[0, 0], fx["expected_ST"], fx["tolerance"], "worked example S_T")
+
+
+def check_T1_closed_form(lib=None, seed=1):
+    """T = 1: o_1 = S_0^T (alpha_1*q_1) + (khat_1 . q_1) vhat_1 and
+    S_1 = diag(alpha_1) S_0 + khat_1 vhat_1^T."""
+    rng = np.random.default_rng(seed)
+    x = rand_inputs(rng, 2, 3, 1, 5, 4)
+    o, ST = oracle.fwd(**x, lib=lib)
+    al = np.exp(-x["g"][:, :, 0] * x["tau"][:, :, 0])
+    kh = x["g"][:, :, 0] ** x["tau"][:, :, 0] * x["k"][:, :, 0]
+    vh = x["beta"][:, :, 0] * x["v"][:, :, 0]
+    q = x["q"][:, :, 0]
+    o_ref = np.einsum("bhij,bhi->bhj", x["S0"], al * q) + np.sum(kh * q, -1)[..., None] * vh
+    S_ref = al[..., None] * x["S0"] + kh[..., :, None] * vh[..., None, :]
+    close(o[:, :, 0], o_ref, 1e-13, "T=1 o")
+    close(ST, S_ref, 1e-13, "T=1 S_1")
+
+
+def check_g_zero(lib=None, seed=2):
+    """g = 0 (tau > 0): alpha = 1, alpha_hat = 0, so S_t = S_0 and o_t = S_0^T q_t;
+    with S_0 = 0 everything is zero."""
+    rng = np.random.default_rng(seed)
+    x = rand_inputs(rng, 1, 2, 9, 4, 3)
+    x["g"][:] = 0.0
+    o, ST = oracle.fwd(**x, lib=lib)
+    close(o, np.einsum("bhij,bhti->bhtj", x["S0"], x["q"]), 1e-13, "g=0 o")
+    close(ST, x["S0"], 1e-15, "g=0 S_T")
+    x["S0"] = None
+    o, ST = oracle.fwd(**x, lib=lib)
+    assert np.all(o == 0.0) and np.all(ST == 0.0)
+
+
+def check_tau_zero(lib=None, seed=3):
+    """tau -> 0: alpha = 1 and alpha_hat = 1 (0^0 = 1 too), i.e. plain
+    cumulative linear attention S_t = S_0 + sum_{s<=t} k_s vhat_s^T, checked
+    against numpy prefix sums of outer products."""
+    rng = np.random.default_rng(seed)
+    x = rand_inputs(rng, 2, 2, 11, 3, 5)
+    for tau_val, tol in ((0.0, 1e-13), (1e-8, 1e-6)):
+        x["tau"][:] = tau_val
+        # 0^0 = 1 at tau = 0 exactly; for tau > 0 the limit needs g > 0
+        x["g"][0, 0, :, 0] = 0.0 if tau_val == 0.0 else 0.3
+        o, ST = oracle.fwd(**x, lib=lib)
+        vh = x["beta"] * x["v"]
+        S = x["S0"][:, :, None] + np.cumsum(x["k"][..., :, None] * vh[..., None, :], axis=2)
+        close(o, np.einsum("bhtij,bhti->bhtj", S, x["q"]), tol, f"tau={tau_val} o")
+        close(ST, S[:, :, -1], tol, f"tau={tau_val} S_T")
+
+
+def quadratic_form(x):
+    """Brute force O(T^2):  o_t = sum_{s<=t} (prod_{r=s+1..t} alpha_r * khat_s)^T q_t vhat_s
+    + S_0^T (prod_{r<=t} alpha_r * q_t), products taken explicitly."""
+    q, k, v, g, tau, beta, S0 = (x[n] for n in ("q", "k", "v", "g", "tau", "beta", "S0"))
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    al = np.exp(-g * tau)
+    kh = g ** tau * k
+    vh = beta * v
+    o = np.zeros((B, H, T, dv))
+    for b in range(B):
+        for h in range(H):
+            for t in range(T):
+                for s in range(t + 1):
+                    w = np.ones(dk)
+                    for r in range(s + 1, t + 1):
+                        w = w * al[b, h, r]
+                    o[b, h, t] += np.dot(w * kh[b, h, s], q[b, h, t]) * vh[b, h, s]
+                w = np.ones(dk)
+                for r in range(t + 1):
+                    w = w * al[b, h, r]
+                o[b, h, t] += S0[b, h].T @ (w * q[b, h, t])
+    return o
+
+
+def check_quadratic(lib=None, seed=4):
+    rng = np.random.default_rng(seed)
+    for (T, dk, dv) in ((16, 4, 3), (7, 2, 6)):
+        x = rand_inputs(rng, 1, 2, T, dk, dv, g_lo=0.0, g_hi=3.0)
+        o, _ = oracle.fwd(**x, lib=lib)
+        close(o, quadratic_form(x), 1e-12, f"quadratic form T={T}")
+
+
+def check_linearity(lib=None, seed=5):
+    """o is linear in (vhat, S_0) jointly: scaling beta and S_0 by c scales o
+    and S_T by c; superposing two v's (with their S_0's) superposes outputs."""
+    rng = np.random.default_rng(seed)
+    x = rand_inputs(rng, 1, 2, 10, 4, 3)
+    o, ST = oracle.fwd(**x, lib=lib)
+    y = dict(x, beta=2.5 * x["beta"], S0=2.5 * x["S0"])
+    o2, ST2 = oracle.fwd(**y, lib=lib)
+    close(o2, 2.5 * o, 1e-13, "scale o")
+    close(ST2, 2.5 * ST, 1e-13, "scale S_T")
+    x2 = rand_inputs(rng, 1, 2, 10, 4, 3)
+    ya = dict(x, v=x2["v"], S0=x2["S0"])
+    oa, _ = oracle.fwd(**ya, lib=lib)
+    yb = dict(x, v=x["v"] + x2["v"], S0=x["S0"] + x2["S0"])
+    ob, _ = oracle.fwd(**yb, lib=lib)
+    close(ob, o + oa, 1e-12, "superposition")
+
+
+def check_split_and_decode(lib=None, seed=6):
+    """fwd(T1) then fwd(T2, S_0 = S_T1) == fwd(T1+T2); T decode steps == fwd(T)."""
+    rng = np.random.default_rng(seed)
+    x = rand_inputs(rng, 2, 1, 13, 3, 4)
+    o, ST = oracle.fwd(**x, lib=lib)
+    cut = lambda a, sl: a[:, :, sl]
+    seq = ("q", "k", "v", "g", "tau", "beta")
+    a = {n: cut(x[n], slice(0, 5)) for n in seq}
+    b = {n: cut(x[n], slice(5, None)) for n in seq}
+    oa, Sa = oracle.fwd(**a, S0=x["S0"], lib=lib)
+    ob, Sb = oracle.fwd(**b, S0=Sa, lib=lib)
+    close(np.concatenate([oa, ob], 2), o, 1e-13, "split o")
+    close(Sb, ST, 1e-13, "split S_T")
+    S = np.ascontiguousarray(x["S0"].copy())
+    for t in range(13):
+        ot = oracle.decode_step(*(x[n][:, :, t] for n in seq), S, lib=lib)
+        close(ot, o[:, :, t], 1e-13, f"decode step {t}")
+    close(S, ST, 1e-13, "decode final state")
+
+
+# ----------------------------------------------------------------- backward pins
+def loss_value(x, dO, dST, lib=None):
+    o, ST = oracle.fwd(**x, lib=lib)
+    return float(np.sum(o * dO) + np.sum(ST * dST))
+
+
+def check_bwd_finite_differences(lib=None, seed=7):
+    """Central differences (h = 1e-6) of L = <o, dO> + <S_T, dS_T> against the
+    oracle's reverse mode, for every input including S_0 and the upstream dS_T."""
+    rng = np.random.default_rng(seed)
+    B, H, T, dk, dv = 1, 1, 6, 3, 2
+    x = rand_inputs(rng, B, H, T, dk, dv, g_lo=0.1, g_hi=3.0, tau_lo=0.05, tau_hi=1.0)
+    dO = rng.standard_normal((B, H, T, dv))
+    dST = rng.standard_normal((B, H, dk, dv))
+    gr = oracle.bwd(**x, dO=dO, dST=dST, lib=lib)
+    names = dict(q="dq", k="dk", v="dv", g="dg", tau="dtau", beta="dbeta", S0="dS0")
+    h = 1e-6
+    for n, gn in names.items():
+        num = np.zeros_like(x[n])
+        for idx in np.ndindex(x[n].shape):
+            xp = {m: a.copy() for m, a in x.items()}
+            xp[n][idx] += h
+            lp = loss_value(xp, dO, dST, lib)
+            xp[n][idx] -= 2 * h
+            lm = loss_value(xp, dO, dST, lib)
+            num[idx] = (lp - lm) / (2 * h)
+        close(gr[gn], num, 2e-7, f"finite differences {gn}")
+    # no upstream dS_T (NULL) is the same as a zero dS_T
+    gr0 = oracle.bwd(**x, dO=dO, dST=None, lib=lib)
+    grz = oracle.bwd(**x, dO=dO, dST=np.zeros_like(dST), lib=lib)
+    for gn in names.values():
+        close(gr0[gn], grz[gn], 0.0, f"dS_T=None vs zeros {gn}")
+
+
+def torch_loop_grads(x, dO, dST):
+    """Gradients of a naive fp64 torch loop by torch.autograd (a library
+    routine independent of the oracle's hand-written reverse mode)."""
+    import torch
+    t = {n: torch.tensor(a, dtype=torch.float64, requires_grad=True) for n, a in x.items()}
+    S = t["S0"]
+    outs = []
+    T = x["q"].shape[2]
+    for s in range(T):
+        al = torch.exp(-t["g"][:, :, s] * t["tau"][:, :, s])
+        kh = torch.pow(t["g"][:, :, s], t["tau"][:, :, s]) * t["k"][:, :, s]
+        vh = t["beta"][:, :, s] * t["v"][:, :, s]
+        S = al[..., :, None] * S + kh[..., :, None] * vh[..., None, :]
+        outs.append((S * t["q"][:, :, s][..., :, None]).sum(-2))
+    o = torch.stack(outs, 2)
+    L = (o * torch.tensor(dO)).sum() + (S * torch.tensor(dST)).sum()
+    L.backward()
+    return {n: t[n].grad.numpy() for n in t}
+
+
+def check_bwd_autograd(lib=None, seed=8):
+    rng = np.random.default_rng(seed)
+    # T = 70 crosses the oracle's 64-token checkpoint boundary
+    B, H, T, dk, dv = 1, 2, 70, 4, 3
+    x = rand_inputs(rng, B, H, T, dk, dv, g_lo=0.05, g_hi=1.0)
+    dO = rng.standard_normal((B, H, T, dv))
+    dST = rng.standard_normal((B, H, dk, dv))
+    gr = oracle.bwd(**x, dO=dO, dST=dST, lib=lib)
+    ref = torch_loop_grads(x, dO, dST)
+    names = dict(q="dq", k="dk", v="dv", g="dg", tau="dtau", beta="dbeta", S0="dS0")
+    for n, gn in names.items():
+        close(gr[gn], ref[n], 1e-11, f"autograd {gn}")
+
+
+FORWARD_PINS = [check_worked_example, check_T1_closed_form, check_g_zero, check_tau_zero,
+                check_quadratic, check_linearity, check_split_and_decode]
+BACKWARD_PINS = [check_bwd_finite_differences, check_bwd_autograd]
+ALL_PINS = FORWARD_PINS + BACKWARD_PINS

@@ -1,0 +1,67 @@
+"""Mutation check of the oracle's pins: plant one plausible slip at a time in a
+copy of the oracle's C source (on the CPU), build it, and require that at least
+one pin fails.  A pin set that let a mutant through would not pin the oracle."""
+import os
+import subprocess
+
+import pytest
+
+import oracle
+from tests import oracle_pins as P
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "rdm_oracle.c")
+
+# (name, original text, planted slip, pins that must catch it)
+MUTANTS = [
+    ("decay sign", "return exp(-g * tau);", "return exp(g * tau);", P.FORWARD_PINS),
+    ("decay uses g only", "return exp(-g * tau);", "return exp(-g);", P.FORWARD_PINS),
+    ("write gate swapped pow", "return pow(g, tau);", "return pow(tau, g);", P.FORWARD_PINS),
+    ("write gate dropped", "double kh = gate_alpha_hat(g[i], tau[i]) * k[i];",
+     "double kh = k[i];", P.FORWARD_PINS),
+    ("decay dropped", "row[j] = al * row[j] + kh * (beta[j] * v[j]);",
+     "row[j] = row[j] + kh * (beta[j] * v[j]);", P.FORWARD_PINS),
+    ("input gate dropped", "row[j] = al * row[j] + kh * (beta[j] * v[j]);",
+     "row[j] = al * row[j] + kh * v[j];", P.FORWARD_PINS),
+    ("readout with k", "acc += S[(size_t)i * dv + j] * q[i];",
+     "acc += S[(size_t)i * dv + j] * k[i];", P.FORWARD_PINS),
+    ("readout before update", "    if (o) {\n        for (int j = 0; j < dv; ++j) {",
+     "    if (o && 0) {\n        for (int j = 0; j < dv; ++j) {", P.FORWARD_PINS),
+    ("bwd readout with k", "dS[(size_t)i * dv + j] += q[i] * dO[j];",
+     "dS[(size_t)i * dv + j] += k[i] * dO[j];", P.BACKWARD_PINS),
+    ("bwd decay not propagated", "dS[(size_t)i * dv + j] *= al[i];",
+     "dS[(size_t)i * dv + j] *= 1.0;", P.BACKWARD_PINS),
+    ("bwd dalpha uses S_t", "a2 += dS[(size_t)i * dv + j] * Sp[(size_t)i * dv + j];",
+     "a2 += dS[(size_t)i * dv + j] * St[(size_t)i * dv + j];", P.BACKWARD_PINS),
+    ("bwd dg sign", "J->dg[ok + i] = dal[i] * (-tau[i] * al[i]) + dah * dah_dg;",
+     "J->dg[ok + i] = dal[i] * (tau[i] * al[i]) + dah * dah_dg;", P.BACKWARD_PINS),
+    ("bwd dtau log of tau", "ah[i] * log(g[i]);", "ah[i] * log(tau[i]);", P.BACKWARD_PINS),
+    ("bwd dbeta with beta", "J->dbeta[ov + j] = v[j] * dvh[j];",
+     "J->dbeta[ov + j] = beta[j] * dvh[j];", P.BACKWARD_PINS),
+    ("bwd dk without gate", "J->dk_[ok + i] = ah[i] * dkh[i];",
+     "J->dk_[ok + i] = dkh[i];", P.BACKWARD_PINS),
+    ("bwd dq uses S_{t-1}", "acc += St[(size_t)i * dv + j] * dO[j];",
+     "acc += Sp[(size_t)i * dv + j] * dO[j];", P.BACKWARD_PINS),
+    ("bwd dv transposed gate", "J->dv_[ov + j] = beta[j] * dvh[j];",
+     "J->dv_[ov + j] = v[j] * dvh[j];", P.BACKWARD_PINS),
+    ("bwd upstream dS_T ignored", "if (J->dST) memcpy(dS, J->dST + ss, sizeof(double) * SS);",
+     "if (0) memcpy(dS, J->dST + ss, sizeof(double) * SS);", P.BACKWARD_PINS),
+]
+
+
+@pytest.mark.parametrize("name,orig,slip,pins", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_catch_mutant(tmp_path, name, orig, slip, pins):
+    src = open(SRC).read()
+    assert src.count(orig) == 1, f"mutation anchor not unique/found: {orig!r}"
+    mpath = tmp_path / "mutant.c"
+    mpath.write_text(src.replace(orig, slip))
+    so = tmp_path / "libmutant.so"
+    subprocess.check_call(["gcc", "-O1", "-std=c99", "-D_POSIX_C_SOURCE=200809L", "-shared",
+                           "-fPIC", "-o", str(so), str(mpath), "-lm", "-lpthread"])
+    lib = oracle.load_library(str(so))
+    caught = []
+    for check in pins:
+        try:
+            check(lib=lib)
+        except (AssertionError, RuntimeError, FloatingPointError, ValueError):
+            caught.append(check.__name__)
+    assert caught, f"mutant '{name}' passed every pin"
