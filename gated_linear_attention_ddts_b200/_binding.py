@@ -1,0 +1,205 @@
+"""ctypes binding of librdm_ddts.so (include/rdm_ddts.h).
+
+Argument marshalling only: torch tensors become device pointers, the current
+torch stream becomes the cudaStream_t, statuses become exceptions.  Every step
+of the computation runs in the library's CUDA kernels; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "librdm_ddts.so")
+
+RDM_OK, RDM_ERR_INVALID_ARG, RDM_ERR_UNSUPPORTED, RDM_ERR_CUDA, RDM_ERR_TIMEOUT, \
+    RDM_ERR_WORKSPACE = range(6)
+RDM_F32, RDM_BF16 = 0, 1
+IMPL = {"auto": 0, "simt": 1, "tc": 2, 0: 0, 1: 1, 2: 2}
+
+_VP = ctypes.c_void_p
+_I = ctypes.c_int
+
+
+class FwdArgs(ctypes.Structure):
+    _fields_ = [("B", _I), ("H", _I), ("T", _I), ("dk", _I), ("dv", _I), ("chunk", _I),
+                ("dtype", _I), ("impl", _I),
+                ("q", _VP), ("k", _VP), ("v", _VP), ("g", _VP), ("tau", _VP), ("beta", _VP),
+                ("S0", _VP), ("o", _VP), ("ST", _VP), ("saved_states", _VP)]
+
+
+class BwdArgs(ctypes.Structure):
+    _fields_ = [("B", _I), ("H", _I), ("T", _I), ("dk", _I), ("dv", _I), ("chunk", _I),
+                ("dtype", _I), ("impl", _I),
+                ("q", _VP), ("k", _VP), ("v", _VP), ("g", _VP), ("tau", _VP), ("beta", _VP),
+                ("S0", _VP), ("grad_o", _VP), ("grad_ST", _VP), ("saved_states", _VP),
+                ("grad_q", _VP), ("grad_k", _VP), ("grad_v", _VP), ("grad_g", _VP),
+                ("grad_tau", _VP), ("grad_beta", _VP), ("grad_S0", _VP),
+                ("workspace", _VP), ("workspace_bytes", ctypes.c_size_t)]
+
+
+class RdmError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+_lib = None
+
+EXPORTS = ["rdm_ddts_fwd", "rdm_ddts_saved_states_size", "rdm_ddts_bwd",
+           "rdm_ddts_bwd_workspace_size", "rdm_ddts_decode_step", "rdm_ddts_sync_status",
+           "rdm_status_string", "rdm_ddts_version"]
+
+
+def load():
+    """Open librdm_ddts.so and declare its signatures.  Raises if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is not built; run "
+                               "`python -m gated_linear_attention_ddts_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        lib.rdm_ddts_fwd.argtypes = [ctypes.POINTER(FwdArgs), _VP]
+        lib.rdm_ddts_fwd.restype = _I
+        lib.rdm_ddts_saved_states_size.argtypes = [_I] * 6
+        lib.rdm_ddts_saved_states_size.restype = ctypes.c_size_t
+        lib.rdm_ddts_bwd.argtypes = [ctypes.POINTER(BwdArgs), _VP]
+        lib.rdm_ddts_bwd.restype = _I
+        lib.rdm_ddts_bwd_workspace_size.argtypes = [ctypes.POINTER(BwdArgs)]
+        lib.rdm_ddts_bwd_workspace_size.restype = ctypes.c_size_t
+        lib.rdm_ddts_decode_step.argtypes = [_I] * 5 + [_VP] * 9
+        lib.rdm_ddts_decode_step.restype = _I
+        lib.rdm_ddts_sync_status.argtypes = [_VP]
+        lib.rdm_ddts_sync_status.restype = _I
+        lib.rdm_status_string.argtypes = [_I]
+        lib.rdm_status_string.restype = ctypes.c_char_p
+        lib.rdm_ddts_version.argtypes = []
+        lib.rdm_ddts_version.restype = _I
+        _lib = lib
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return load().rdm_status_string(int(status)).decode()
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("expected a torch.Tensor")
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError("tensors passed to the library must be contiguous CUDA tensors")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return RDM_BF16
+    if t.dtype == torch.float32:
+        return RDM_F32
+    raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
+
+
+def _check(status: int, where: str):
+    if status != RDM_OK:
+        raise RdmError(status, where)
+
+
+def rdm_ddts_saved_states_size(B, H, T, dk, dv, chunk=0) -> int:
+    return int(load().rdm_ddts_saved_states_size(B, H, T, dk, dv, chunk))
+
+
+def rdm_ddts_fwd(q, k, v, g, tau, beta, S0=None, o=None, ST=None, saved_states=None, *,
+                 chunk=0, impl="auto", return_state=False, stream=None):
+    """Forward over [B,H,T,D] sequences.  Allocates o (and S_T when
+    return_state) with torch if not given.  Returns (o, S_T or None)."""
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    if o is None:
+        o = torch.empty(B, H, T, dv, dtype=q.dtype, device=q.device)
+    if ST is None and return_state:
+        ST = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device)
+    a = FwdArgs(B, H, T, dk, dv, chunk, _dtype_code(q), IMPL[impl],
+                _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(tau), _ptr(beta), _ptr(S0), _ptr(o),
+                _ptr(ST), _ptr(saved_states))
+    _check(load().rdm_ddts_fwd(ctypes.byref(a), _stream(stream)), "rdm_ddts_fwd")
+    return o, ST
+
+
+def _bwd_args(q, k, v, g, tau, beta, S0, grad_o, grad_ST, saved_states, grads, ws, ws_bytes,
+              chunk, impl):
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    return BwdArgs(B, H, T, dk, dv, chunk, _dtype_code(q), IMPL[impl],
+                   _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(tau), _ptr(beta), _ptr(S0),
+                   _ptr(grad_o), _ptr(grad_ST), _ptr(saved_states),
+                   *(_ptr(grads.get(n)) for n in ("dq", "dk", "dv", "dg", "dtau", "dbeta",
+                                                    "dS0")),
+                   _ptr(ws), ws_bytes)
+
+
+def rdm_ddts_bwd_workspace_size(q, k, v, g, tau, beta, S0=None, grad_o=None, grad_ST=None,
+                                saved_states=None, *, chunk=0, impl="auto") -> int:
+    a = _bwd_args(q, k, v, g, tau, beta, S0, grad_o, grad_ST, saved_states, {}, None, 0,
+                  chunk, impl)
+    n = load().rdm_ddts_bwd_workspace_size(ctypes.byref(a))
+    if n == ctypes.c_size_t(-1).value:
+        raise RdmError(RDM_ERR_INVALID_ARG, "rdm_ddts_bwd_workspace_size")
+    return int(n)
+
+
+def rdm_ddts_bwd(q, k, v, g, tau, beta, S0, grad_o, grad_ST=None, saved_states=None, *,
+                 grads=None, workspace=None, chunk=0, impl="auto", want_dS0=True, stream=None):
+    """Backward.  `grads` may hold preallocated dq, dk, dv, dg, dtau, dbeta, dS0;
+    missing ones are allocated with torch, as is the workspace.  Returns the dict."""
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    grads = dict(grads or {})
+    for n, ref in (("dq", q), ("dk", k), ("dg", g), ("dtau", tau), ("dv", v), ("dbeta", beta)):
+        if grads.get(n) is None:
+            grads[n] = torch.empty_like(ref)
+    if want_dS0 and grads.get("dS0") is None:
+        grads["dS0"] = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        need = rdm_ddts_bwd_workspace_size(q, k, v, g, tau, beta, S0, grad_o, grad_ST,
+                                           saved_states, chunk=chunk, impl=impl)
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    a = _bwd_args(q, k, v, g, tau, beta, S0, grad_o, grad_ST, saved_states, grads, workspace,
+                  workspace.numel() * workspace.element_size(), chunk, impl)
+    _check(load().rdm_ddts_bwd(ctypes.byref(a), _stream(stream)), "rdm_ddts_bwd")
+    return grads
+
+
+def rdm_ddts_decode_step(q, k, v, g, tau, beta, S, o=None, *, stream=None):
+    """One token per (b,h): q,k,g,tau [B,H,dk], v,beta [B,H,dv]; S [B,H,dk,dv]
+    float32 updated in place.  Returns o [B,H,dv]."""
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    if o is None:
+        o = torch.empty(B, H, dv, dtype=q.dtype, device=q.device)
+    st = load().rdm_ddts_decode_step(B, H, dk, dv, _dtype_code(q), _ptr(q), _ptr(k), _ptr(v),
+                                     _ptr(g), _ptr(tau), _ptr(beta), _ptr(S), _ptr(o),
+                                     _stream(stream))
+    _check(st, "rdm_ddts_decode_step")
+    return o
+
+
+def rdm_ddts_sync_status(stream=None) -> int:
+    return int(load().rdm_ddts_sync_status(_stream(stream)))
+
+
+def rdm_status_string(status: int) -> str:
+    return status_string(status)
+
+
+def rdm_ddts_version() -> int:
+    return int(load().rdm_ddts_version())

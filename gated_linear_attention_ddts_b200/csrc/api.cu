@@ -1,0 +1,215 @@
+// api.cu -- the exported C ABI (include/rdm_ddts.h): argument validation,
+// path selection and launch.  Nothing here allocates device memory or
+// synchronises, except rdm_ddts_sync_status.
+#include <stdint.h>
+#include <string.h>
+
+#include "../../include/rdm_ddts.h"
+#include "launch.h"
+#include "rdm_common.cuh"
+
+namespace rdm {
+
+// Device status word (bit kErrTimeout: a bounded wait ran out).  One copy per
+// device the library is loaded on.
+__device__ unsigned g_status_word;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+unsigned* g_status_ptr[kMaxDevices];
+
+unsigned* status_word() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    if (!g_status_ptr[dev]) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_status_word) != cudaSuccess) return nullptr;
+        g_status_ptr[dev] = static_cast<unsigned*>(ptr);
+    }
+    return g_status_ptr[dev];
+}
+
+bool dim_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+bool aligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool opt_aligned(const void* p) { return p == nullptr || aligned(p); }
+
+rdm_status from_cuda(cudaError_t e) { return e == cudaSuccess ? RDM_OK : RDM_ERR_CUDA; }
+
+// Sizes shared by fwd and bwd.  Returns RDM_OK or the reason to refuse.
+rdm_status check_sizes(int B, int H, int T, int dk, int dv, int chunk, rdm_dtype dtype,
+                       rdm_impl impl) {
+    if (B < 1 || H < 1 || T < 0 || dk < 1 || dv < 1) return RDM_ERR_INVALID_ARG;
+    if (dtype != RDM_F32 && dtype != RDM_BF16) return RDM_ERR_INVALID_ARG;
+    if (impl != RDM_IMPL_AUTO && impl != RDM_IMPL_SIMT && impl != RDM_IMPL_TC)
+        return RDM_ERR_INVALID_ARG;
+    if (chunk < 0) return RDM_ERR_INVALID_ARG;
+    if (!dim_ok(dk) || !dim_ok(dv)) return RDM_ERR_UNSUPPORTED;
+    if (chunk != 0 && chunk != 16 && chunk != 32 && chunk != 64 && chunk != 128)
+        return RDM_ERR_UNSUPPORTED;
+    // every element offset must fit in 63 bits and the grid in 31
+    const double n = (double)B * H * (double)(T > 0 ? T : 1) * (dk > dv ? dk : dv);
+    if (n > 4.0e18 || (double)B * H > 2.0e9 || T > (1 << 30)) return RDM_ERR_INVALID_ARG;
+    return RDM_OK;
+}
+
+int eff_chunk(int chunk) { return chunk == 0 ? 64 : chunk; }
+
+// T == 0: no tokens; S_T = S_0 (or zero), no saved states.
+rdm_status empty_sequence(int B, int H, int dk, int dv, const float* S0, float* ST,
+                          cudaStream_t s) {
+    if (!ST) return RDM_OK;
+    const size_t bytes = (size_t)B * H * dk * dv * 4;
+    cudaError_t e = S0 ? cudaMemcpyAsync(ST, S0, bytes, cudaMemcpyDeviceToDevice, s)
+                       : cudaMemsetAsync(ST, 0, bytes, s);
+    return from_cuda(e);
+}
+
+bool use_tc_fwd(const SeqParams& p, rdm_impl impl) {
+    if (impl == RDM_IMPL_SIMT) return false;
+    return tc_fwd_supported(p);
+}
+
+bool use_tc_bwd(const BwdParams& p, rdm_impl impl) {
+    if (impl == RDM_IMPL_SIMT) return false;
+    return tc_bwd_supported(p);
+}
+
+BwdParams bwd_params(const rdm_bwd_args* a) {
+    BwdParams p;
+    memset(&p, 0, sizeof(p));
+    p.B = a->B; p.H = a->H; p.T = a->T; p.dk = a->dk; p.dv = a->dv;
+    p.chunk = eff_chunk(a->chunk);
+    p.bf16 = a->dtype == RDM_BF16;
+    p.q = a->q; p.k = a->k; p.v = a->v; p.g = a->g; p.tau = a->tau; p.beta = a->beta;
+    p.S0 = a->S0; p.dO = a->grad_o; p.dST = a->grad_ST; p.saved = a->saved_states;
+    p.dq = a->grad_q; p.dk_ = a->grad_k; p.dv_ = a->grad_v; p.dg = a->grad_g;
+    p.dtau = a->grad_tau; p.dbeta = a->grad_beta; p.dS0 = a->grad_S0;
+    p.ws = a->workspace; p.ws_bytes = a->workspace_bytes;
+    return p;
+}
+
+}  // namespace
+}  // namespace rdm
+
+using namespace rdm;
+
+extern "C" {
+
+size_t rdm_ddts_saved_states_size(int B, int H, int T, int dk, int dv, int chunk) {
+    if (check_sizes(B, H, T, dk, dv, chunk, RDM_F32, RDM_IMPL_AUTO) != RDM_OK) return 0;
+    const int C = eff_chunk(chunk);
+    const size_t nc = (size_t)(T + C - 1) / C;
+    return (size_t)B * H * nc * dk * dv * 4;
+}
+
+rdm_status rdm_ddts_fwd(const rdm_fwd_args* a, rdm_stream_t stream) {
+    if (!a) return RDM_ERR_INVALID_ARG;
+    rdm_status st = check_sizes(a->B, a->H, a->T, a->dk, a->dv, a->chunk, a->dtype, a->impl);
+    if (st != RDM_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (!opt_aligned(a->S0) || !opt_aligned(a->ST) || !opt_aligned(a->saved_states))
+        return RDM_ERR_INVALID_ARG;
+    if (a->T == 0) {
+        if (a->impl == RDM_IMPL_TC && a->dtype != RDM_BF16) return RDM_ERR_UNSUPPORTED;
+        return empty_sequence(a->B, a->H, a->dk, a->dv, a->S0, a->ST, s);
+    }
+    const void* in[] = {a->q, a->k, a->v, a->g, a->tau, a->beta, a->o};
+    for (const void* p : in)
+        if (!p || !aligned(p)) return RDM_ERR_INVALID_ARG;
+    SeqParams p;
+    memset(&p, 0, sizeof(p));
+    p.B = a->B; p.H = a->H; p.T = a->T; p.dk = a->dk; p.dv = a->dv;
+    p.chunk = eff_chunk(a->chunk);
+    p.bf16 = a->dtype == RDM_BF16;
+    p.q = a->q; p.k = a->k; p.v = a->v; p.g = a->g; p.tau = a->tau; p.beta = a->beta;
+    p.S0 = a->S0; p.o = a->o; p.ST = a->ST; p.saved = a->saved_states;
+    p.err = status_word();
+    if (!p.err) return RDM_ERR_CUDA;
+    const bool tc = use_tc_fwd(p, a->impl);
+    if (a->impl == RDM_IMPL_TC && !tc) return RDM_ERR_UNSUPPORTED;
+    return from_cuda(tc ? launch_tc_fwd(p, s) : launch_simt_fwd(p, s));
+}
+
+size_t rdm_ddts_bwd_workspace_size(const rdm_bwd_args* a) {
+    if (!a) return (size_t)-1;
+    if (check_sizes(a->B, a->H, a->T, a->dk, a->dv, a->chunk, a->dtype, a->impl) != RDM_OK)
+        return (size_t)-1;
+    if (a->T == 0) return 0;
+    BwdParams p = bwd_params(a);
+    if (use_tc_bwd(p, a->impl)) return tc_bwd_workspace(p);
+    return simt_bwd_workspace(p);
+}
+
+rdm_status rdm_ddts_bwd(const rdm_bwd_args* a, rdm_stream_t stream) {
+    if (!a) return RDM_ERR_INVALID_ARG;
+    rdm_status st = check_sizes(a->B, a->H, a->T, a->dk, a->dv, a->chunk, a->dtype, a->impl);
+    if (st != RDM_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (!opt_aligned(a->S0) || !opt_aligned(a->grad_ST) || !opt_aligned(a->grad_S0) ||
+        !opt_aligned(a->saved_states) || !opt_aligned(a->workspace))
+        return RDM_ERR_INVALID_ARG;
+    if (a->T == 0) {
+        if (a->impl == RDM_IMPL_TC && a->dtype != RDM_BF16) return RDM_ERR_UNSUPPORTED;
+        // no tokens: dS_0 = dS_T
+        return empty_sequence(a->B, a->H, a->dk, a->dv, a->grad_ST, a->grad_S0, s);
+    }
+    const void* in[] = {a->q, a->k, a->v, a->g, a->tau, a->beta, a->grad_o, a->grad_q,
+                        a->grad_k, a->grad_v, a->grad_g, a->grad_tau, a->grad_beta};
+    for (const void* p : in)
+        if (!p || !aligned(p)) return RDM_ERR_INVALID_ARG;
+    BwdParams p = bwd_params(a);
+    p.err = status_word();
+    if (!p.err) return RDM_ERR_CUDA;
+    const bool tc = use_tc_bwd(p, a->impl);
+    if (a->impl == RDM_IMPL_TC && !tc) return RDM_ERR_UNSUPPORTED;
+    const size_t need = tc ? tc_bwd_workspace(p) : simt_bwd_workspace(p);
+    if (need > 0 && (!a->workspace || a->workspace_bytes < need)) return RDM_ERR_WORKSPACE;
+    return from_cuda(tc ? launch_tc_bwd(p, s) : launch_simt_bwd(p, s));
+}
+
+rdm_status rdm_ddts_decode_step(int B, int H, int dk, int dv, rdm_dtype dtype, const void* q,
+                                const void* k, const void* v, const void* g, const void* tau,
+                                const void* beta, float* S, void* o, rdm_stream_t stream) {
+    rdm_status st = check_sizes(B, H, 1, dk, dv, 0, dtype, RDM_IMPL_AUTO);
+    if (st != RDM_OK) return st;
+    const void* in[] = {q, k, v, g, tau, beta, S, o};
+    for (const void* p : in)
+        if (!p || !aligned(p)) return RDM_ERR_INVALID_ARG;
+    DecodeParams p;
+    p.B = B; p.H = H; p.dk = dk; p.dv = dv; p.bf16 = dtype == RDM_BF16;
+    p.q = q; p.k = k; p.v = v; p.g = g; p.tau = tau; p.beta = beta; p.S = S; p.o = o;
+    return from_cuda(launch_decode(p, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+rdm_status rdm_ddts_sync_status(rdm_stream_t stream) {
+    cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return RDM_ERR_CUDA;
+    unsigned* w = status_word();
+    if (!w) return RDM_ERR_CUDA;
+    unsigned h = 0;
+    if (cudaMemcpy(&h, w, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return RDM_ERR_CUDA;
+    if (h != 0) {
+        const unsigned zero = 0;
+        if (cudaMemcpy(w, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+            return RDM_ERR_CUDA;
+        if (h & kErrTimeout) return RDM_ERR_TIMEOUT;
+    }
+    return RDM_OK;
+}
+
+const char* rdm_status_string(rdm_status s) {
+    switch (s) {
+        case RDM_OK: return "ok";
+        case RDM_ERR_INVALID_ARG: return "invalid argument (size, NULL or misaligned pointer)";
+        case RDM_ERR_UNSUPPORTED: return "unsupported configuration";
+        case RDM_ERR_CUDA: return "CUDA runtime error";
+        case RDM_ERR_TIMEOUT: return "a bounded on-device wait timed out";
+        case RDM_ERR_WORKSPACE: return "workspace missing or too small";
+    }
+    return "unknown status";
+}
+
+int rdm_ddts_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,58 @@
+// launch.h -- internal host launchers behind the C ABI (not exported).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+namespace rdm {
+
+struct SeqParams {
+    int B, H, T, dk, dv, chunk;
+    int bf16;  // element type of sequence tensors: 1 = bf16, 0 = float32
+    const void *q, *k, *v, *g, *tau, *beta;
+    const float* S0;
+    void* o;
+    float* ST;
+    float* saved;        // [B,H,NC,dk,dv] chunk-start states, or null
+    unsigned* err;       // device status word
+};
+
+struct BwdParams {
+    int B, H, T, dk, dv, chunk;
+    int bf16;
+    const void *q, *k, *v, *g, *tau, *beta;
+    const float* S0;
+    const void* dO;
+    const float* dST;
+    const float* saved;  // chunk-start states (tensor-core path), or null
+    void *dq, *dk_, *dv_, *dg, *dtau, *dbeta;
+    float* dS0;
+    void* ws;            // scratch
+    size_t ws_bytes;
+    unsigned* err;
+};
+
+struct DecodeParams {
+    int B, H, dk, dv;
+    int bf16;
+    const void *q, *k, *v, *g, *tau, *beta;
+    float* S;
+    void* o;
+};
+
+// exact token-serial CUDA-core path (any supported shape, float32 or bf16)
+cudaError_t launch_simt_fwd(const SeqParams& p, cudaStream_t s);
+size_t simt_bwd_workspace(const BwdParams& p);
+cudaError_t launch_simt_bwd(const BwdParams& p, cudaStream_t s);
+
+// decode step
+cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s);
+
+// tensor-core (tcgen05) chunked path
+bool tc_fwd_supported(const SeqParams& p);
+cudaError_t launch_tc_fwd(const SeqParams& p, cudaStream_t s);
+bool tc_bwd_supported(const BwdParams& p);
+size_t tc_bwd_workspace(const BwdParams& p);
+cudaError_t launch_tc_bwd(const BwdParams& p, cudaStream_t s);
+
+}  // namespace rdm

@@ -1,0 +1,176 @@
+/*
+ * rdm_ddts.h -- C ABI of the B200 (sm_100a) DDTS-gated linear-attention
+ * recurrence of Rodimus.
+ *
+ * The operation (per batch b, head h, token t; i runs over d_k, j over d_v):
+ *
+ *   alpha_t     = exp(-g_t * tau_t)        alpha_hat_t = g_t ^ tau_t
+ *   S_t         = diag(alpha_t) S_{t-1} + (alpha_hat_t * k_t)(beta_hat_t * v_t)^T
+ *   o_t         = S_t^T q_t
+ *
+ * Sources: the gate formulas are those of the DDTS mechanism in "Rodimus*:
+ * Breaking the Accuracy-Efficiency Trade-Off with Efficient Attentions"
+ * (digest.lyk-ai.com summary, section "Method", first Rodimus bullet: selection
+ * gate g_t, temperature gate tau_t).  The selection acts only along the key
+ * dimension n = d_k, which is what allows chunkwise-parallel training
+ * (paperhub.cn OpenReview rebuttal, "Efficient Parallelization" bullet, Sec.
+ * 3.1.3 / App. B3); training runs chunkwise in parallel and inference runs token
+ * by token on a fixed-size cached state (same page, answer to Q2; state size
+ * n x m, answer to Q5-3 on Table 4).  beta_hat gates the input only, never the
+ * transition (atlas.scime.ai summary, ablation rows on hat-beta and on beta in
+ * the state transition).  The pages do not print the state update itself; the
+ * form above is the plainest reading that agrees with all of these.
+ *
+ * Conventions shared by every entry point:
+ *   - Layouts are dense row-major: sequences [B,H,T,D], states [B,H,d_k,d_v],
+ *     decode inputs [B,H,D].  D is d_k for q, k, g, tau and d_v for v, beta_hat,
+ *     o and their gradients.
+ *   - Element type of every sequence tensor is `dtype` (RDM_F32 or RDM_BF16);
+ *     states, saved states and dS_0 are always float32.  Arithmetic is float32
+ *     throughout; bf16 operands feed the tensor cores with float32 accumulation.
+ *   - All pointers are DEVICE pointers of the current device, 16-byte aligned.
+ *     The caller owns every buffer.  The library allocates nothing, never
+ *     synchronises (except rdm_ddts_sync_status) and launches only on `stream`.
+ *   - Domain: g >= 0, tau >= 0.  Values are not checked on the device;
+ *     out-of-domain values give NaN as the formulas do.  0^0 = 1, 0^tau = 0.
+ *   - Host-side validation failures return a status and launch nothing.
+ *     Kernel-side failures (a bounded wait that ran out) set a device status
+ *     word that rdm_ddts_sync_status reports.
+ *   - Supported sizes: d_k, d_v in {16, 32, 64, 128}; any T >= 0; B*H >= 1.
+ *     The tensor-core path covers bf16 with d_k in {64, 128} and d_v in
+ *     {64, 128} (d_v a multiple of the per-CTA tile); every other supported
+ *     shape, and all float32 calls, run the exact-recurrence CUDA-core path.
+ */
+#ifndef RDM_DDTS_H
+#define RDM_DDTS_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st *rdm_stream_t;
+
+typedef enum {
+    RDM_OK = 0,
+    RDM_ERR_INVALID_ARG = 1,  /* bad size, NULL or misaligned pointer      */
+    RDM_ERR_UNSUPPORTED = 2,  /* valid request this build does not handle  */
+    RDM_ERR_CUDA = 3,         /* a CUDA runtime call failed                 */
+    RDM_ERR_TIMEOUT = 4,      /* a bounded on-device wait ran out           */
+    RDM_ERR_WORKSPACE = 5     /* workspace missing or too small             */
+} rdm_status;
+
+typedef enum { RDM_F32 = 0, RDM_BF16 = 1 } rdm_dtype;
+
+/* Which kernels to use.  AUTO picks the tensor-core path when the shape and
+ * dtype allow it.  SIMT forces the exact token-serial CUDA-core path.  TC
+ * forces the tensor-core path and fails with RDM_ERR_UNSUPPORTED where it does
+ * not apply. */
+typedef enum { RDM_IMPL_AUTO = 0, RDM_IMPL_SIMT = 1, RDM_IMPL_TC = 2 } rdm_impl;
+
+/* ------------------------------------------------------------------ forward
+ * Chunkwise-parallel forward over whole sequences (the training / prefill
+ * form named in the rebuttal's answer to Q2).
+ *
+ *   q, k, g, tau : [B,H,T,d_k] dtype      v, beta : [B,H,T,d_v] dtype
+ *   S0           : [B,H,d_k,d_v] float32, or NULL for a zero initial state
+ *   o            : [B,H,T,d_v] dtype, written
+ *   ST           : [B,H,d_k,d_v] float32 final state, written; NULL = skip
+ *   saved_states : [B,H,ceil(T/chunk),d_k,d_v] float32, written with the state
+ *                  in force before each chunk (S_0 for chunk 0); NULL = skip.
+ *                  rdm_ddts_bwd can reuse it instead of recomputing.
+ *   chunk        : tokens per chunk; 0 selects 64.  Allowed: 64.
+ */
+typedef struct {
+    int B, H, T, dk, dv;
+    int chunk;
+    rdm_dtype dtype;
+    rdm_impl impl;
+    const void *q, *k, *v, *g, *tau, *beta;
+    const float *S0;
+    void *o;
+    float *ST;
+    float *saved_states;
+} rdm_fwd_args;
+
+rdm_status rdm_ddts_fwd(const rdm_fwd_args *args, rdm_stream_t stream);
+
+/* Bytes of `saved_states` that rdm_ddts_fwd writes for these sizes
+ * (B*H*ceil(T/chunk)*d_k*d_v*4); 0 on invalid sizes. */
+size_t rdm_ddts_saved_states_size(int B, int H, int T, int dk, int dv, int chunk);
+
+/* ----------------------------------------------------------------- backward
+ * Reverse mode of the forward for the loss L with dL/do = grad_o and
+ * dL/dS_T = grad_ST.  The pages print no backward; this is the exact gradient
+ * of the recurrence above.
+ *
+ *   inputs as in rdm_fwd_args (q..beta, S0)
+ *   grad_o       : [B,H,T,d_v] dtype
+ *   grad_ST      : [B,H,d_k,d_v] float32, or NULL for zero
+ *   saved_states : states written by rdm_ddts_fwd with the same inputs and
+ *                  chunk, or NULL to recompute them (into the workspace)
+ *   grad_q, grad_k, grad_g, grad_tau : [B,H,T,d_k] dtype, written
+ *   grad_v, grad_beta                : [B,H,T,d_v] dtype, written
+ *   grad_S0      : [B,H,d_k,d_v] float32, written; NULL = skip
+ *   workspace    : device scratch of at least rdm_ddts_bwd_workspace_size()
+ *                  bytes (may be NULL when that size is 0); contents on entry
+ *                  are ignored and on exit are unspecified.
+ * Gradients with respect to g are undefined where g = 0 (g^(tau-1) is
+ * unbounded there); d/dtau uses alpha_hat * ln g = 0 where alpha_hat = 0.
+ */
+typedef struct {
+    int B, H, T, dk, dv;
+    int chunk;
+    rdm_dtype dtype;
+    rdm_impl impl;
+    const void *q, *k, *v, *g, *tau, *beta;
+    const float *S0;
+    const void *grad_o;
+    const float *grad_ST;
+    const float *saved_states;
+    void *grad_q, *grad_k, *grad_v, *grad_g, *grad_tau, *grad_beta;
+    float *grad_S0;
+    void *workspace;
+    size_t workspace_bytes;
+} rdm_bwd_args;
+
+rdm_status rdm_ddts_bwd(const rdm_bwd_args *args, rdm_stream_t stream);
+
+/* Scratch bytes rdm_ddts_bwd needs for `args` (depends on sizes, dtype, impl
+ * and whether saved_states is given); (size_t)-1 on invalid sizes. */
+size_t rdm_ddts_bwd_workspace_size(const rdm_bwd_args *args);
+
+/* ------------------------------------------------------------ decode step
+ * One token of sequential inference on a cached fixed-size state, O(1) per
+ * token (rebuttal answers to Q1 and Q2).  For every (b,h):
+ *   S <- diag(alpha) S + (alpha_hat * k)(beta_hat * v)^T ;  o = S^T q
+ *
+ *   q, k, g, tau : [B,H,d_k] dtype     v, beta : [B,H,d_v] dtype
+ *   S            : [B,H,d_k,d_v] float32, read and updated in place
+ *   o            : [B,H,d_v] dtype, written
+ */
+rdm_status rdm_ddts_decode_step(int B, int H, int dk, int dv, rdm_dtype dtype,
+                                const void *q, const void *k, const void *v,
+                                const void *g, const void *tau, const void *beta,
+                                float *S, void *o, rdm_stream_t stream);
+
+/* ------------------------------------------------------------------ status */
+
+/* Synchronises `stream`, then reports (and clears) the device status word of
+ * the current device: RDM_ERR_TIMEOUT if a bounded wait in a kernel ran out,
+ * RDM_ERR_CUDA if the stream holds a CUDA error, RDM_OK otherwise. */
+rdm_status rdm_ddts_sync_status(rdm_stream_t stream);
+
+/* Static, NUL-terminated description of a status code. */
+const char *rdm_status_string(rdm_status status);
+
+/* Library ABI version (major*10000 + minor*100 + patch). */
+int rdm_ddts_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RDM_DDTS_H */
