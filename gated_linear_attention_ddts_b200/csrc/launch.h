@@ -56,3 +56,13 @@ size_t tc_bwd_workspace(const BwdParams& p);
 cudaError_t launch_tc_bwd(const BwdParams& p, cudaStream_t s);
 
 }  // namespace rdm
+
+// ---------------------------------------------------------------- TMA maps
+#include <cuda.h>
+namespace rdm {
+// 3-D bf16 tensor [n2][n1][n0] (n0 innermost, dense) as a TMA map with box
+// {b0, b1, 1} and 128-byte swizzle (b0 * 2 must be 128).  Returns false if the
+// driver refuses the map.
+bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t n0, uint64_t n1,
+                       uint64_t n2, uint32_t b0, uint32_t b1);
+}  // namespace rdm

@@ -1,7 +1,570 @@
-// tc_fwd.cu -- tensor-core chunked forward (placeholder until the kernel lands).
+// tc_fwd.cu -- chunkwise-parallel DDTS forward on the sm_100a tensor cores.
+//
+// Rodimus trains the DDTS recurrence chunk by chunk (paperhub.cn rebuttal,
+// answer to Q2 and "Efficient Parallelization": selection only along d_k makes
+// the chunkwise form possible).  Per (b,h) and chunk of C = 64 tokens, with
+// b_t the inclusive running sum of log(alpha) = -g*tau inside the window and
+// m a per-channel reference (the midpoint of the window's b range):
+//
+//   Qt = q * exp(b_t - m)              Kt = k * alpha_hat * exp(m - b_s)
+//   A  = mask_{s<=t}(Qt Kt^T)          Vh = beta_hat * v
+//   o  = A Vh + Qt (diag(exp(m)) S_prev)                 (intra + inter chunk)
+//   S  = diag(exp(b_last)) S_prev + diag(exp(b_last - m)) Kt^T Vh
+//
+// Every factor stays inside exp(+-span/2) with span = b_first - b_last of the
+// window, so products are exact in fp32 range whenever span <= kSpanMax.  A
+// chunk whose span is larger is processed as windows of 16 tokens, or of 1
+// token, each window being one pass of the same pipeline (exact for any decay).
+//
+// One CTA owns one (b,h) and a 64-wide slice of d_v.  Warp roles:
+//   warps 0-3  epilogue: A -> masked bf16 operand, state (fp32 registers),
+//              S_hat operand, o store (TMEM lanes = rows)
+//   warps 4-7  gates: TMA tiles -> log-decay scan, Qt, Kt, Vh operands (bf16)
+//   warp  8    TMA producer (q, k, g, tau, v, beta tiles, 128B-swizzled)
+//   warp  9    TMEM allocator and single-thread tcgen05.mma issuer
+// All hand-offs are mbarriers with bounded waits (a timeout sets the device
+// status word and the CTA exits cleanly).
+#include <cuda.h>
+
 #include "launch.h"
+#include "rdm_common.cuh"
+#include "tc_ptx.cuh"
 
 namespace rdm {
-bool tc_fwd_supported(const SeqParams&) { return false; }
-cudaError_t launch_tc_fwd(const SeqParams&, cudaStream_t) { return cudaErrorNotSupported; }
+namespace {
+using namespace tc;
+
+constexpr int C = 64;                        // tokens per chunk (tile rows)
+constexpr int kThreads = 320;
+constexpr float kSpanMax = 120.0f;           // largest in-window log-decay span
+constexpr long long kWaitLimit = 2000000000LL;  // ~1 s of SM clocks
+constexpr int kEpiWarp0 = 0, kGateWarp0 = 4, kProdWarp = 8, kMmaWarp = 9;
+constexpr int kBarPair = 1;  // +half: the two gate warps of one channel half (64 threads)
+constexpr int kBarGate = 3;  // the four gate warps (128 threads)
+constexpr int kBox = 64 * 64 * 2;  // bytes of one 64x64 bf16 TMA box
+
+template <int DK, int DVT>
+struct Cfg {
+    static constexpr int NS = DK == 128 ? 1 : 2;   // raw TMA stages
+    static constexpr int NB = 2;                   // operand buffers
+    static constexpr int KB = DK / 64;             // boxes per key-side tile
+    static constexpr int VB = DVT / 64;            // boxes per value-side tile
+    static constexpr int RAW = (4 * KB + 2 * VB) * kBox;
+    static constexpr int G = DK / 8;               // 8-channel groups
+    static constexpr int COL_A = 0, COL_S = 64, COL_O = 64 + DVT;
+    static constexpr int TMEM_COLS = (64 + 2 * DVT) <= 256 ? 256 : 512;
+};
+
+template <int DK, int DVT>
+struct alignas(1024) FwdSmem {
+    using K = Cfg<DK, DVT>;
+    uint8_t raw[K::NS][K::RAW];
+    uint8_t qt[K::NB][C * DK * 2];
+    uint8_t kt[K::NB][C * DK * 2];
+    uint8_t vh[K::NB][C * DVT * 2];
+    uint8_t abf[C * C * 2];
+    uint8_t shat[DK * DVT * 2];
+    float em[K::NB][DK], cf[K::NB][DK], gm[K::NB][DK];
+    int info[K::NB][4];  // chunk, w0, w1, last
+    float xf[3][DK];     // gate exchange: scan carry, b at window start, b at window end
+    uint64_t raw_full[K::NS], raw_empty[K::NS], ops_full[K::NB], ops_empty[K::NB];
+    uint64_t mma1_done, as_free, abf_full, mmao_done, o_free;
+    int need16[2], need1[2];
+    uint32_t tmem_base;
+    int fail;
+};
+
+struct FwdKernelArgs {
+    CUtensorMap mq, mk, mg, mt, mv, mb;
+    SeqParams p;
+};
+
+// ---- shared-memory operand offsets (bytes), canonical no-swizzle UMMA layouts
+// Qt, Kt, A_bf16: K-major, rows x (8-row groups 128 B apart), K groups 1024 B apart
+__device__ __forceinline__ uint32_t off_rowmajor64(int r, int k) {
+    return (uint32_t)((r >> 3) * 128 + (k >> 3) * 1024 + (r & 7) * 16 + (k & 7) * 2);
+}
+// Vh [s][j] stored MN-major for N = j: j groups 1024 B apart, s groups 128 B apart
+__device__ __forceinline__ uint32_t off_vh(int s, int j) {
+    return (uint32_t)((j >> 3) * 1024 + (s >> 3) * 128 + (s & 7) * 16 + (j & 7) * 2);
+}
+// S_hat [i][j] stored MN-major for N = j: j groups DK*16 B apart, i groups 128 B apart
+template <int DK>
+__device__ __forceinline__ uint32_t off_shat(int i, int j) {
+    return (uint32_t)((j >> 3) * (DK * 16) + (i >> 3) * 128 + (i & 7) * 16 + (j & 7) * 2);
+}
+// 8 consecutive bf16 of row t, column group cg, in a tile of 64-wide 128B-swizzled boxes
+__device__ __forceinline__ uint32_t off_raw(int t, int cg) {
+    return (uint32_t)((cg >> 3) * kBox + t * 128 + (((cg & 7) ^ (t & 7)) << 4));
+}
+
+__device__ __forceinline__ void unpack8(uint4 u, float* f) {
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float2 x = __bfloat1622float2(h[e]);
+        f[2 * e] = x.x;
+        f[2 * e + 1] = x.y;
+    }
+}
+__device__ __forceinline__ uint4 pack8(const float* f) {
+    uint4 u;
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) h[e] = __floats2bfloat162_rn(f[2 * e], f[2 * e + 1]);
+    return u;
+}
+
+__device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity))
+        if (clock64() - t0 > kWaitLimit) return false;
+    return true;
+}
+
+template <int DK, int DVT>
+__global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_constant__ FwdKernelArgs A) {
+    using K = Cfg<DK, DVT>;
+    constexpr int NS = K::NS, NB = K::NB, KB = K::KB, VB = K::VB;
+    extern __shared__ uint8_t smem_dyn[];
+    FwdSmem<DK, DVT>& sm = *reinterpret_cast<FwdSmem<DK, DVT>*>(
+        (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+    const SeqParams& p = A.p;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int NJ = p.dv / DVT;
+    const int bh = blockIdx.x / NJ, j0 = (blockIdx.x % NJ) * DVT;
+    const int T = p.T, NC = (T + C - 1) / C;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(&sm.raw_full[s], 1);
+            mbar_init(&sm.raw_empty[s], 4);
+        }
+        for (int b = 0; b < NB; ++b) {
+            mbar_init(&sm.ops_full[b], 4);
+            mbar_init(&sm.ops_empty[b], 1 + 4);
+        }
+        mbar_init(&sm.mma1_done, 1);
+        mbar_init(&sm.as_free, 4);
+        mbar_init(&sm.abf_full, 4);
+        mbar_init(&sm.mmao_done, 1);
+        mbar_init(&sm.o_free, 4);
+        sm.need16[0] = sm.need16[1] = sm.need1[0] = sm.need1[1] = 0;
+        sm.fail = 0;
+        fence_mbar_init();
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc(&sm.tmem_base, K::TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (warp == kProdWarp && lane == 0) {
+        prefetch_tmap(&A.mq); prefetch_tmap(&A.mk); prefetch_tmap(&A.mg);
+        prefetch_tmap(&A.mt); prefetch_tmap(&A.mv); prefetch_tmap(&A.mb);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    volatile int* fail = &sm.fail;
+
+    if (warp == kProdWarp) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            int issued = 0;
+            for (int c = 0; c < NC; ++c) {
+                const int st = c % NS;
+                if (c >= NS && !mbar_wait(&sm.raw_empty[st], ((c / NS) - 1) & 1, fail, kWaitLimit))
+                    break;
+                mbar_expect_tx(&sm.raw_full[st], K::RAW);
+                uint8_t* raw = sm.raw[st];
+                for (int kb = 0; kb < KB; ++kb) {
+                    tma_load_3d(raw + (0 * KB + kb) * kBox, &A.mq, &sm.raw_full[st], 64 * kb, c * C, bh);
+                    tma_load_3d(raw + (1 * KB + kb) * kBox, &A.mk, &sm.raw_full[st], 64 * kb, c * C, bh);
+                    tma_load_3d(raw + (2 * KB + kb) * kBox, &A.mg, &sm.raw_full[st], 64 * kb, c * C, bh);
+                    tma_load_3d(raw + (3 * KB + kb) * kBox, &A.mt, &sm.raw_full[st], 64 * kb, c * C, bh);
+                }
+                for (int vb = 0; vb < VB; ++vb) {
+                    tma_load_3d(raw + (4 * KB + vb) * kBox, &A.mv, &sm.raw_full[st], j0 + 64 * vb, c * C, bh);
+                    tma_load_3d(raw + (4 * KB + VB + vb) * kBox, &A.mb, &sm.raw_full[st], j0 + 64 * vb, c * C, bh);
+                }
+                ++issued;
+            }
+            // never leave the CTA with copies in flight
+            for (int c = issued - NS < 0 ? 0 : issued - NS; c < issued; ++c)
+                drain_wait(&sm.raw_full[c % NS], (c / NS) & 1);
+        }
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t tA = tmem + K::COL_A, tS = tmem + K::COL_S, tO = tmem + K::COL_O;
+            constexpr uint32_t id1 = idesc_bf16(64, 64, 0, 0);    // A  = Qt Kt^T
+            constexpr uint32_t idS = idesc_bf16(DK, DVT, 1, 1);   // dS = Kt^T Vh
+            constexpr uint32_t idO = idesc_bf16(64, DVT, 0, 1);   // O  = A Vh + Qt S_hat
+            int item = 0, n1 = 0, nO = 0;
+            while (true) {
+                const int ob = item % NB;
+                if (!mbar_wait(&sm.ops_full[ob], (item / NB) & 1, fail, kWaitLimit)) break;
+                const int last = sm.info[ob][3];
+                if (item > 0 && !mbar_wait(&sm.as_free, (item - 1) & 1, fail, kWaitLimit)) break;
+                tc_fence_after();
+                const uint32_t q = smem_u32(sm.qt[ob]), k = smem_u32(sm.kt[ob]);
+                const uint32_t v = smem_u32(sm.vh[ob]);
+#pragma unroll
+                for (int ks = 0; ks < DK / 16; ++ks)
+                    mma_bf16(tA, sdesc(q + ks * 2048, 1024, 128), sdesc(k + ks * 2048, 1024, 128),
+                             id1, ks > 0);
+#pragma unroll
+                for (int ks = 0; ks < C / 16; ++ks)
+                    mma_bf16(tS, sdesc(k + ks * 256, 128, 1024), sdesc(v + ks * 256, 128, 1024), idS,
+                             ks > 0);
+                mma_commit(&sm.mma1_done);
+                ++n1;
+                if (!mbar_wait(&sm.abf_full, item & 1, fail, kWaitLimit)) break;
+                if (item > 0 && !mbar_wait(&sm.o_free, (item - 1) & 1, fail, kWaitLimit)) break;
+                tc_fence_after();
+                const uint32_t a = smem_u32(sm.abf), sh = smem_u32(sm.shat);
+#pragma unroll
+                for (int ks = 0; ks < C / 16; ++ks)
+                    mma_bf16(tO, sdesc(a + ks * 2048, 1024, 128), sdesc(v + ks * 256, 128, 1024), idO,
+                             ks > 0);
+#pragma unroll
+                for (int ks = 0; ks < DK / 16; ++ks)
+                    mma_bf16(tO, sdesc(q + ks * 2048, 1024, 128), sdesc(sh + ks * 256, 128, DK * 16),
+                             idO, 1);
+                mma_commit(&sm.mmao_done);
+                mma_commit(&sm.ops_empty[ob]);
+                ++nO;
+                if (last) break;
+                ++item;
+            }
+            // let issued MMAs finish before TMEM is released
+            if (n1 > 0) drain_wait(&sm.mma1_done, (n1 - 1) & 1);
+            if (nO > 0) drain_wait(&sm.mmao_done, (nO - 1) & 1);
+        }
+        __syncwarp();
+    } else if (warp >= kGateWarp0) {
+        // ------------------------------------------------------------ gates
+        const int gw = warp - kGateWarp0, half = gw >> 1;
+        const int t = ((gw & 1) << 5) | lane;  // token row of the chunk
+        const int gtid = gw * 32 + lane;
+        constexpr int GH = K::G / 2;    // channel groups per half
+        constexpr int VGH = DVT / 16;   // value column groups per half
+        const uint32_t full = 0xffffffffu;
+        int item = 0;
+        for (int c = 0; c < NC; ++c) {
+            const int st = c % NS;
+            if (!mbar_wait(&sm.raw_full[st], (c / NS) & 1, fail, kWaitLimit)) break;
+            const uint8_t* raw = sm.raw[st];
+            const int nval = min(C, T - c * C);
+            // b <- log(alpha) for my channels at token t (rows past T: 0)
+            float b[GH][8];
+            auto load_log_alpha = [&]() {
+#pragma unroll
+                for (int gg = 0; gg < GH; ++gg) {
+                    const int cg = half * GH + gg;
+                    float g8[8], t8[8];
+                    unpack8(*reinterpret_cast<const uint4*>(raw + 2 * KB * kBox + off_raw(t, cg)), g8);
+                    unpack8(*reinterpret_cast<const uint4*>(raw + 3 * KB * kBox + off_raw(t, cg)), t8);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) b[gg][e] = (t < nval) ? log_alpha(g8[e], t8[e]) : 0.0f;
+                }
+            };
+            load_log_alpha();
+            // chunk-wide inclusive scan over tokens (lanes, then carry across the warp pair)
+#pragma unroll
+            for (int gg = 0; gg < GH; ++gg)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    float x = b[gg][e];
+#pragma unroll
+                    for (int d = 1; d < 32; d <<= 1) {
+                        const float y = __shfl_up_sync(full, x, d);
+                        if (lane >= d) x += y;
+                    }
+                    b[gg][e] = x;
+                }
+            if ((gw & 1) == 0 && lane == 31) {
+#pragma unroll
+                for (int gg = 0; gg < GH; ++gg)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) sm.xf[0][(half * GH + gg) * 8 + e] = b[gg][e];
+            }
+            named_bar(kBarPair + half, 64);
+            if (gw & 1) {
+#pragma unroll
+                for (int gg = 0; gg < GH; ++gg)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) b[gg][e] += sm.xf[0][(half * GH + gg) * 8 + e];
+            }
+            if (t == 0 || t == nval - 1) {
+#pragma unroll
+                for (int gg = 0; gg < GH; ++gg)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int ch = (half * GH + gg) * 8 + e;
+                        if (t == 0) sm.xf[1][ch] = b[gg][e];
+                        if (t == nval - 1) sm.xf[2][ch] = b[gg][e];
+                    }
+            }
+            named_bar(kBarPair + half, 64);
+            // window size: 64, or 16 / 1 when the decay span is too wide for one reference
+            float span = 0.0f;
+#pragma unroll
+            for (int gg = 0; gg < GH; ++gg)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int ch = (half * GH + gg) * 8 + e;
+                    span = fmaxf(span, sm.xf[1][ch] - sm.xf[2][ch]);
+                }
+            if (__any_sync(full, !(span <= kSpanMax)) && lane == 0) sm.need16[c & 1] = c + 1;
+            named_bar(kBarGate, 128);
+            int W = sm.need16[c & 1] == c + 1 ? 16 : C;
+            // lanes holding the first / last valid token of this thread's 16-token window
+            const int wl0 = lane & ~15;
+            const int wlast = max(wl0, min(wl0 + 15, nval - 1 - ((gw & 1) << 5)));
+            if (W == 16) {
+                load_log_alpha();
+                float sp16 = 0.0f;
+#pragma unroll
+                for (int gg = 0; gg < GH; ++gg)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        float x = b[gg][e];
+#pragma unroll
+                        for (int d = 1; d < 16; d <<= 1) {
+                            const float y = __shfl_up_sync(full, x, d);
+                            if ((lane & 15) >= d) x += y;
+                        }
+                        b[gg][e] = x;
+                        const float bf = __shfl_sync(full, x, wl0), bl = __shfl_sync(full, x, wlast);
+                        if (t < nval) sp16 = fmaxf(sp16, bf - bl);
+                    }
+                if (__any_sync(full, !(sp16 <= kSpanMax)) && lane == 0) sm.need1[c & 1] = c + 1;
+                named_bar(kBarGate, 128);
+                if (sm.need1[c & 1] == c + 1) {
+                    W = 1;
+                    load_log_alpha();
+                }
+            }
+
+            for (int w0 = 0; w0 < nval; w0 += W) {
+                const int w1 = min(w0 + W, nval);
+                const int ob = item % NB;
+                if (item >= NB && !mbar_wait(&sm.ops_empty[ob], ((item / NB) - 1) & 1, fail, kWaitLimit))
+                    break;
+                const bool in = t >= w0 && t < w1;
+#pragma unroll
+                for (int gg = 0; gg < GH; ++gg) {
+                    const int cg = half * GH + gg;
+                    float q8[8], k8[8], g8[8], t8[8], oq[8], ok[8], mm[8], bl[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        // reference m = midpoint of the window's b range; bl = b at its last token
+                        if (W == C) {
+                            const int ch = cg * 8 + e;
+                            bl[e] = sm.xf[2][ch];
+                            mm[e] = 0.5f * (sm.xf[1][ch] + bl[e]);
+                        } else if (W == 16) {
+                            const float bf = __shfl_sync(full, b[gg][e], wl0);
+                            bl[e] = __shfl_sync(full, b[gg][e], wlast);
+                            mm[e] = 0.5f * (bf + bl[e]);
+                        } else {
+                            bl[e] = mm[e] = b[gg][e];
+                        }
+                    }
+                    unpack8(*reinterpret_cast<const uint4*>(raw + 0 * KB * kBox + off_raw(t, cg)), q8);
+                    unpack8(*reinterpret_cast<const uint4*>(raw + 1 * KB * kBox + off_raw(t, cg)), k8);
+                    unpack8(*reinterpret_cast<const uint4*>(raw + 2 * KB * kBox + off_raw(t, cg)), g8);
+                    unpack8(*reinterpret_cast<const uint4*>(raw + 3 * KB * kBox + off_raw(t, cg)), t8);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float bb = b[gg][e];
+                        oq[e] = in ? q8[e] * exp2f((bb - mm[e]) * kLog2e) : 0.0f;
+                        ok[e] = in ? k8[e] * exp2f(log2_alpha_hat(g8[e], t8[e]) + (mm[e] - bb) * kLog2e)
+                                   : 0.0f;
+                    }
+                    *reinterpret_cast<uint4*>(sm.qt[ob] + off_rowmajor64(t, cg * 8)) = pack8(oq);
+                    *reinterpret_cast<uint4*>(sm.kt[ob] + off_rowmajor64(t, cg * 8)) = pack8(ok);
+                    if (t == w0) {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const int ch = cg * 8 + e;
+                            sm.em[ob][ch] = exp2f(mm[e] * kLog2e);
+                            sm.cf[ob][ch] = exp2f((bl[e] - mm[e]) * kLog2e);
+                            sm.gm[ob][ch] = exp2f(bl[e] * kLog2e);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int vg = 0; vg < VGH; ++vg) {
+                    const int jg = half * VGH + vg;
+                    float v8[8], b8[8], o8[8];
+                    unpack8(*reinterpret_cast<const uint4*>(raw + 4 * KB * kBox + off_raw(t, jg)), v8);
+                    unpack8(*reinterpret_cast<const uint4*>(raw + (4 * KB + VB) * kBox + off_raw(t, jg)), b8);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) o8[e] = in ? v8[e] * b8[e] : 0.0f;
+                    *reinterpret_cast<uint4*>(sm.vh[ob] + off_vh(t, jg * 8)) = pack8(o8);
+                }
+                if (gtid == 0) {
+                    sm.info[ob][0] = c;
+                    sm.info[ob][1] = w0;
+                    sm.info[ob][2] = w1;
+                    sm.info[ob][3] = (c == NC - 1) && (w1 == nval);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.ops_full[ob]);
+                ++item;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.raw_empty[st]);
+            if (*fail) break;
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int ew = warp - kEpiWarp0;
+        const bool rowA = lane < 16;                      // valid rows of A and O (M = 64)
+        const int tA = 16 * ew + lane;
+        const bool rowS = (DK == 128) || lane < 16;        // valid state rows (M = DK)
+        const int iS = (DK == 128) ? 32 * ew + lane : 16 * ew + lane;
+        const uint32_t lb = (uint32_t)(32 * ew) << 16;
+        float S[DVT];
+#pragma unroll
+        for (int j = 0; j < DVT; ++j)
+            S[j] = (rowS && p.S0) ? p.S0[((size_t)bh * DK + iS) * p.dv + j0 + j] : 0.0f;
+        int item = 0;
+        while (true) {
+            const int ob = item % NB;
+            if (!mbar_wait(&sm.ops_full[ob], (item / NB) & 1, fail, kWaitLimit)) break;
+            const int c = sm.info[ob][0], w0 = sm.info[ob][1], w1 = sm.info[ob][2];
+            const int last = sm.info[ob][3];
+            if (!mbar_wait(&sm.mma1_done, item & 1, fail, kWaitLimit)) break;
+            tc_fence_after();
+            // A -> causal mask -> bf16 operand (row t = tA, columns s)
+#pragma unroll
+            for (int qd = 0; qd < 4; ++qd) {
+                float v[16];
+                tmem_ld16(tmem + lb + K::COL_A + 16 * qd, v);
+                tmem_ld_wait();
+                if (rowA) {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) v[e] = (16 * qd + e <= tA) ? v[e] : 0.0f;
+                    *reinterpret_cast<uint4*>(sm.abf + off_rowmajor64(tA, 16 * qd)) = pack8(v);
+                    *reinterpret_cast<uint4*>(sm.abf + off_rowmajor64(tA, 16 * qd + 8)) = pack8(v + 8);
+                }
+            }
+            // S_hat = diag(exp(m)) S_prev, and the chunk-start state if requested
+            if (rowS) {
+                const float em = sm.em[ob][iS];
+#pragma unroll
+                for (int jg = 0; jg < DVT / 8; ++jg) {
+                    float x[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) x[e] = S[jg * 8 + e] * em;
+                    *reinterpret_cast<uint4*>(sm.shat + off_shat<DK>(iS, jg * 8)) = pack8(x);
+                }
+                if (p.saved && w0 == 0) {
+                    float4* dst = reinterpret_cast<float4*>(
+                        p.saved + (((size_t)bh * NC + c) * DK + iS) * p.dv + j0);
+#pragma unroll
+                    for (int j4 = 0; j4 < DVT / 4; ++j4)
+                        dst[j4] = make_float4(S[4 * j4], S[4 * j4 + 1], S[4 * j4 + 2], S[4 * j4 + 3]);
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.abf_full);
+            // state update S = diag(gamma) S + diag(cfac) (Kt^T Vh)
+            {
+                const float gmv = rowS ? sm.gm[ob][iS] : 0.0f, cfv = rowS ? sm.cf[ob][iS] : 0.0f;
+#pragma unroll
+                for (int qd = 0; qd < DVT / 16; ++qd) {
+                    float v[16];
+                    tmem_ld16(tmem + lb + K::COL_S + 16 * qd, v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) S[16 * qd + e] = fmaf(gmv, S[16 * qd + e], cfv * v[e]);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.as_free);
+            // o rows of this window
+            if (!mbar_wait(&sm.mmao_done, item & 1, fail, kWaitLimit)) break;
+            tc_fence_after();
+            {
+                const bool st_row = rowA && tA >= w0 && tA < w1;
+                __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.o) +
+                                      ((size_t)bh * T + (size_t)c * C + tA) * p.dv + j0;
+#pragma unroll
+                for (int qd = 0; qd < DVT / 16; ++qd) {
+                    float v[16];
+                    tmem_ld16(tmem + lb + K::COL_O + 16 * qd, v);
+                    tmem_ld_wait();
+                    if (st_row) {
+                        reinterpret_cast<uint4*>(orow + 16 * qd)[0] = pack8(v);
+                        reinterpret_cast<uint4*>(orow + 16 * qd)[1] = pack8(v + 8);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&sm.o_free);
+                mbar_arrive(&sm.ops_empty[ob]);
+            }
+            if (last) break;
+            ++item;
+        }
+        if (!*fail && rowS && p.ST) {
+            float4* dst = reinterpret_cast<float4*>(p.ST + ((size_t)bh * DK + iS) * p.dv + j0);
+#pragma unroll
+            for (int j4 = 0; j4 < DVT / 4; ++j4)
+                dst[j4] = make_float4(S[4 * j4], S[4 * j4 + 1], S[4 * j4 + 2], S[4 * j4 + 3]);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, K::TMEM_COLS);
+    }
+    if (threadIdx.x == 0 && sm.fail) atomicOr(p.err, kErrTimeout);
+}
+
+template <int DK, int DVT>
+cudaError_t launch_cfg(const SeqParams& p, cudaStream_t s) {
+    FwdKernelArgs a;
+    a.p = p;
+    const uint64_t BH = (uint64_t)p.B * p.H;
+    if (!make_tmap_bf16_3d(&a.mq, p.q, p.dk, p.T, BH, 64, 64) ||
+        !make_tmap_bf16_3d(&a.mk, p.k, p.dk, p.T, BH, 64, 64) ||
+        !make_tmap_bf16_3d(&a.mg, p.g, p.dk, p.T, BH, 64, 64) ||
+        !make_tmap_bf16_3d(&a.mt, p.tau, p.dk, p.T, BH, 64, 64) ||
+        !make_tmap_bf16_3d(&a.mv, p.v, p.dv, p.T, BH, 64, 64) ||
+        !make_tmap_bf16_3d(&a.mb, p.beta, p.dv, p.T, BH, 64, 64))
+        return cudaErrorInvalidValue;
+    const size_t smem = sizeof(FwdSmem<DK, DVT>) + 1024;
+    auto kern = tc_fwd_kernel<DK, DVT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int grid = (int)(BH * (p.dv / DVT));
+    kern<<<grid, kThreads, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool tc_fwd_supported(const SeqParams& p) {
+    return p.bf16 && p.chunk == C && p.T >= 1 && (p.dk == 64 || p.dk == 128) &&
+           (p.dv == 64 || p.dv == 128);
+}
+
+cudaError_t launch_tc_fwd(const SeqParams& p, cudaStream_t s) {
+    if (!tc_fwd_supported(p)) return cudaErrorNotSupported;
+    if (p.dk == 64) return launch_cfg<64, 64>(p, s);
+    return launch_cfg<128, 64>(p, s);
+}
+
 }  // namespace rdm
