@@ -35,6 +35,20 @@ __device__ __forceinline__ float alpha(float g, float tau) {
     return exp2f(log_alpha(g, tau) * kLog2e);
 }
 
+// Single MUFU instructions (PTX ex2.approx / lg2.approx, flush-to-zero): 2^x
+// and log2(x) to about 22 bits, with ex2(-inf) = 0 and lg2(0) = -inf.  Used on
+// the bf16 tensor-core path, where every result is rounded to 8 bits anyway.
+__device__ __forceinline__ float ex2_fast(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float lg2_fast(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // Device status word bits (set with atomicOr by kernels, read by the host).
 constexpr unsigned kErrTimeout = 1u;
 

@@ -42,6 +42,9 @@ constexpr int kEpiWarp0 = 0, kGateWarp0 = 4, kProdWarp = 8, kMmaWarp = 9;
 constexpr int kBarPair = 1;  // +half: the two gate warps of one channel half (64 threads)
 constexpr int kBarGate = 3;  // the four gate warps (128 threads)
 constexpr int kBox = 64 * 64 * 2;  // bytes of one 64x64 bf16 TMA box
+// channel-group stride of the Qt / Kt operand tiles: 1024 + 16 bytes, the skew
+// spreads the channel groups a warp writes for one token over all banks
+constexpr int kQK = 1040;
 
 template <int DK, int DVT>
 struct Cfg {
@@ -59,14 +62,15 @@ template <int DK, int DVT>
 struct alignas(1024) FwdSmem {
     using K = Cfg<DK, DVT>;
     uint8_t raw[K::NS][K::RAW];
-    uint8_t qt[K::NB][C * DK * 2];
-    uint8_t kt[K::NB][C * DK * 2];
+    uint8_t qt[K::NB][K::G * kQK];
+    uint8_t kt[K::NB][K::G * kQK];
     uint8_t vh[K::NB][C * DVT * 2];
     uint8_t abf[C * C * 2];
     uint8_t shat[DK * DVT * 2];
     float em[K::NB][DK], cf[K::NB][DK], gm[K::NB][DK];
     int info[K::NB][4];  // chunk, w0, w1, last
-    float xf[3][DK];     // gate exchange: scan carry, b at window start, b at window end
+    float xf[2][DK];     // gate exchange: b at the first and at the last token of the chunk
+    float wtot[4][DK];   // gate exchange: per-warp scan totals
     uint64_t raw_full[K::NS], raw_empty[K::NS], ops_full[K::NB], ops_empty[K::NB];
     uint64_t mma1_done, as_free, abf_full, mmao_done, o_free;
     int need16[2], need1[2];
@@ -80,9 +84,14 @@ struct FwdKernelArgs {
 };
 
 // ---- shared-memory operand offsets (bytes), canonical no-swizzle UMMA layouts
-// Qt, Kt, A_bf16: K-major, rows x (8-row groups 128 B apart), K groups 1024 B apart
+// A_bf16: K-major, 8-row groups 128 B apart, K groups 1024 B apart
 __device__ __forceinline__ uint32_t off_rowmajor64(int r, int k) {
     return (uint32_t)((r >> 3) * 128 + (k >> 3) * 1024 + (r & 7) * 16 + (k & 7) * 2);
+}
+// Qt, Kt: K-major [token][channel], 8-token groups 128 B apart, channel groups
+// kQK B apart
+__device__ __forceinline__ uint32_t off_qk(int t, int i) {
+    return (uint32_t)((t >> 3) * 128 + (i >> 3) * kQK + (t & 7) * 16 + (i & 7) * 2);
 }
 // Vh [s][j] stored MN-major for N = j: j groups 1024 B apart, s groups 128 B apart
 __device__ __forceinline__ uint32_t off_vh(int s, int j) {
@@ -211,11 +220,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                 const uint32_t v = smem_u32(sm.vh[ob]);
 #pragma unroll
                 for (int ks = 0; ks < DK / 16; ++ks)
-                    mma_bf16(tA, sdesc(q + ks * 2048, 1024, 128), sdesc(k + ks * 2048, 1024, 128),
+                    mma_bf16(tA, sdesc(q + ks * 2 * kQK, kQK, 128), sdesc(k + ks * 2 * kQK, kQK, 128),
                              id1, ks > 0);
 #pragma unroll
                 for (int ks = 0; ks < C / 16; ++ks)
-                    mma_bf16(tS, sdesc(k + ks * 256, 128, 1024), sdesc(v + ks * 256, 128, 1024), idS,
+                    mma_bf16(tS, sdesc(k + ks * 256, 128, kQK), sdesc(v + ks * 256, 128, 1024), idS,
                              ks > 0);
                 mma_commit(&sm.mma1_done);
                 ++n1;
@@ -229,7 +238,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                              ks > 0);
 #pragma unroll
                 for (int ks = 0; ks < DK / 16; ++ks)
-                    mma_bf16(tO, sdesc(q + ks * 2048, 1024, 128), sdesc(sh + ks * 256, 128, DK * 16),
+                    mma_bf16(tO, sdesc(q + ks * 2 * kQK, kQK, 128), sdesc(sh + ks * 256, 128, DK * 16),
                              idO, 1);
                 mma_commit(&sm.mmao_done);
                 mma_commit(&sm.ops_empty[ob]);
@@ -244,11 +253,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
         __syncwarp();
     } else if (warp >= kGateWarp0) {
         // ------------------------------------------------------------ gates
-        const int gw = warp - kGateWarp0, half = gw >> 1;
-        const int t = ((gw & 1) << 5) | lane;  // token row of the chunk
-        const int gtid = gw * 32 + lane;
-        constexpr int GH = K::G / 2;    // channel groups per half
-        constexpr int VGH = DVT / 16;   // value column groups per half
+        // thread -> (8-channel group cg, segment of SEGT consecutive tokens); a warp
+        // covers 16 consecutive tokens, so a 16-token window never leaves a warp
+        constexpr int G = K::G, NSEG = 128 / G, SEGT = C / NSEG, SPW = 32 / G;
+        constexpr int VG = DVT / 8, TPG = 128 / VG, VIT = C / TPG;
+        const int gt = (warp - kGateWarp0) * 32 + lane, gw = gt >> 5;
+        const int cg = gt % G, seg = gt / G;
+        const int tb = seg * SEGT;  // first token of my segment
         const uint32_t full = 0xffffffffu;
         int item = 0;
         for (int c = 0; c < NC; ++c) {
@@ -256,165 +267,228 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             if (!mbar_wait(&sm.raw_full[st], (c / NS) & 1, fail, kWaitLimit)) break;
             const uint8_t* raw = sm.raw[st];
             const int nval = min(C, T - c * C);
-            // b <- log(alpha) for my channels at token t (rows past T: 0)
-            float b[GH][8];
-            auto load_log_alpha = [&]() {
+            float b[SEGT][8];
+            // b <- log(alpha) = -g*tau of my tokens (0 past T), then its running sum
+            auto load_scan = [&]() {
 #pragma unroll
-                for (int gg = 0; gg < GH; ++gg) {
-                    const int cg = half * GH + gg;
+                for (int u = 0; u < SEGT; ++u) {
                     float g8[8], t8[8];
-                    unpack8(*reinterpret_cast<const uint4*>(raw + 2 * KB * kBox + off_raw(t, cg)), g8);
-                    unpack8(*reinterpret_cast<const uint4*>(raw + 3 * KB * kBox + off_raw(t, cg)), t8);
+                    unpack8(*reinterpret_cast<const uint4*>(raw + 2 * KB * kBox + off_raw(tb + u, cg)), g8);
+                    unpack8(*reinterpret_cast<const uint4*>(raw + 3 * KB * kBox + off_raw(tb + u, cg)), t8);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) b[gg][e] = (t < nval) ? log_alpha(g8[e], t8[e]) : 0.0f;
+                    for (int e = 0; e < 8; ++e) {
+                        const float la = (tb + u < nval) ? log_alpha(g8[e], t8[e]) : 0.0f;
+                        b[u][e] = u == 0 ? la : b[u - 1][e] + la;
+                    }
                 }
             };
-            load_log_alpha();
-            // chunk-wide inclusive scan over tokens (lanes, then carry across the warp pair)
-#pragma unroll
-            for (int gg = 0; gg < GH; ++gg)
+            // exclusive prefix of segment totals over the segments of this warp
+            auto warp_prefix = [&](float* excl, float* wsum) {
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    float x = b[gg][e];
+                    const float tot = b[SEGT - 1][e];
+                    float x = tot;
 #pragma unroll
-                    for (int d = 1; d < 32; d <<= 1) {
+                    for (int d = G; d < 32; d <<= 1) {
                         const float y = __shfl_up_sync(full, x, d);
                         if (lane >= d) x += y;
                     }
-                    b[gg][e] = x;
+                    excl[e] = x - tot;
+                    wsum[e] = __shfl_sync(full, x, cg + G * (SPW - 1));
                 }
-            if ((gw & 1) == 0 && lane == 31) {
+            };
+            load_scan();
+            {
+                float excl[8], wsum[8];
+                warp_prefix(excl, wsum);
+                if (lane < G) {
 #pragma unroll
-                for (int gg = 0; gg < GH; ++gg)
+                    for (int e = 0; e < 8; ++e) sm.wtot[gw][cg * 8 + e] = wsum[e];
+                }
+                named_bar(kBarGate, 128);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) sm.xf[0][(half * GH + gg) * 8 + e] = b[gg][e];
+                for (int e = 0; e < 8; ++e) {
+                    float off = excl[e];
+                    for (int w2 = 0; w2 < gw; ++w2) off += sm.wtot[w2][cg * 8 + e];
+#pragma unroll
+                    for (int u = 0; u < SEGT; ++u) b[u][e] += off;
+                }
             }
-            named_bar(kBarPair + half, 64);
-            if (gw & 1) {
+            if (tb == 0) {
 #pragma unroll
-                for (int gg = 0; gg < GH; ++gg)
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) b[gg][e] += sm.xf[0][(half * GH + gg) * 8 + e];
+                for (int e = 0; e < 8; ++e) sm.xf[0][cg * 8 + e] = b[0][e];
             }
-            if (t == 0 || t == nval - 1) {
+            if (tb <= nval - 1 && nval - 1 < tb + SEGT) {
 #pragma unroll
-                for (int gg = 0; gg < GH; ++gg)
+                for (int u = 0; u < SEGT; ++u)
+                    if (tb + u == nval - 1) {
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int ch = (half * GH + gg) * 8 + e;
-                        if (t == 0) sm.xf[1][ch] = b[gg][e];
-                        if (t == nval - 1) sm.xf[2][ch] = b[gg][e];
+                        for (int e = 0; e < 8; ++e) sm.xf[1][cg * 8 + e] = b[u][e];
                     }
             }
-            named_bar(kBarPair + half, 64);
+            named_bar(kBarGate, 128);
             // window size: 64, or 16 / 1 when the decay span is too wide for one reference
             float span = 0.0f;
 #pragma unroll
-            for (int gg = 0; gg < GH; ++gg)
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int ch = (half * GH + gg) * 8 + e;
-                    span = fmaxf(span, sm.xf[1][ch] - sm.xf[2][ch]);
-                }
+            for (int e = 0; e < 8; ++e) span = fmaxf(span, sm.xf[0][cg * 8 + e] - sm.xf[1][cg * 8 + e]);
             if (__any_sync(full, !(span <= kSpanMax)) && lane == 0) sm.need16[c & 1] = c + 1;
             named_bar(kBarGate, 128);
             int W = sm.need16[c & 1] == c + 1 ? 16 : C;
-            // lanes holding the first / last valid token of this thread's 16-token window
-            const int wl0 = lane & ~15;
-            const int wlast = max(wl0, min(wl0 + 15, nval - 1 - ((gw & 1) << 5)));
-            if (W == 16) {
-                load_log_alpha();
-                float sp16 = 0.0f;
-#pragma unroll
-                for (int gg = 0; gg < GH; ++gg)
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        float x = b[gg][e];
-#pragma unroll
-                        for (int d = 1; d < 16; d <<= 1) {
-                            const float y = __shfl_up_sync(full, x, d);
-                            if ((lane & 15) >= d) x += y;
-                        }
-                        b[gg][e] = x;
-                        const float bf = __shfl_sync(full, x, wl0), bl = __shfl_sync(full, x, wlast);
-                        if (t < nval) sp16 = fmaxf(sp16, bf - bl);
-                    }
-                if (__any_sync(full, !(sp16 <= kSpanMax)) && lane == 0) sm.need1[c & 1] = c + 1;
-                named_bar(kBarGate, 128);
-                if (sm.need1[c & 1] == c + 1) {
-                    W = 1;
-                    load_log_alpha();
-                }
-            }
 
-            for (int w0 = 0; w0 < nval; w0 += W) {
-                const int w1 = min(w0 + W, nval);
+            if (W == C) {
+                // ---- hot path: one window = the whole chunk
                 const int ob = item % NB;
                 if (item >= NB && !mbar_wait(&sm.ops_empty[ob], ((item / NB) - 1) & 1, fail, kWaitLimit))
                     break;
-                const bool in = t >= w0 && t < w1;
+                float mm[8], bl[8];
 #pragma unroll
-                for (int gg = 0; gg < GH; ++gg) {
-                    const int cg = half * GH + gg;
-                    float q8[8], k8[8], g8[8], t8[8], oq[8], ok[8], mm[8], bl[8];
+                for (int e = 0; e < 8; ++e) {
+                    bl[e] = sm.xf[1][cg * 8 + e];
+                    mm[e] = 0.5f * (sm.xf[0][cg * 8 + e] + bl[e]);
+                }
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        // reference m = midpoint of the window's b range; bl = b at its last token
-                        if (W == C) {
-                            const int ch = cg * 8 + e;
-                            bl[e] = sm.xf[2][ch];
-                            mm[e] = 0.5f * (sm.xf[1][ch] + bl[e]);
-                        } else if (W == 16) {
-                            const float bf = __shfl_sync(full, b[gg][e], wl0);
-                            bl[e] = __shfl_sync(full, b[gg][e], wlast);
-                            mm[e] = 0.5f * (bf + bl[e]);
-                        } else {
-                            bl[e] = mm[e] = b[gg][e];
-                        }
-                    }
+                for (int u = 0; u < SEGT; ++u) {
+                    const int t = tb + u;
+                    float q8[8], k8[8], g8[8], t8[8], oq[8], ok[8];
                     unpack8(*reinterpret_cast<const uint4*>(raw + 0 * KB * kBox + off_raw(t, cg)), q8);
                     unpack8(*reinterpret_cast<const uint4*>(raw + 1 * KB * kBox + off_raw(t, cg)), k8);
                     unpack8(*reinterpret_cast<const uint4*>(raw + 2 * KB * kBox + off_raw(t, cg)), g8);
                     unpack8(*reinterpret_cast<const uint4*>(raw + 3 * KB * kBox + off_raw(t, cg)), t8);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        const float bb = b[gg][e];
-                        oq[e] = in ? q8[e] * exp2f((bb - mm[e]) * kLog2e) : 0.0f;
-                        ok[e] = in ? k8[e] * exp2f(log2_alpha_hat(g8[e], t8[e]) + (mm[e] - bb) * kLog2e)
-                                   : 0.0f;
+                        const float d = (b[u][e] - mm[e]) * kLog2e;
+                        const float lah = t8[e] == 0.0f ? 0.0f : t8[e] * lg2_fast(g8[e]);
+                        oq[e] = q8[e] * ex2_fast(d);
+                        ok[e] = k8[e] * ex2_fast(lah - d);
                     }
-                    *reinterpret_cast<uint4*>(sm.qt[ob] + off_rowmajor64(t, cg * 8)) = pack8(oq);
-                    *reinterpret_cast<uint4*>(sm.kt[ob] + off_rowmajor64(t, cg * 8)) = pack8(ok);
-                    if (t == w0) {
+                    *reinterpret_cast<uint4*>(sm.qt[ob] + off_qk(t, cg * 8)) = pack8(oq);
+                    *reinterpret_cast<uint4*>(sm.kt[ob] + off_qk(t, cg * 8)) = pack8(ok);
+                }
+                if (tb == 0) {
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const int ch = cg * 8 + e;
-                            sm.em[ob][ch] = exp2f(mm[e] * kLog2e);
-                            sm.cf[ob][ch] = exp2f((bl[e] - mm[e]) * kLog2e);
-                            sm.gm[ob][ch] = exp2f(bl[e] * kLog2e);
-                        }
+                    for (int e = 0; e < 8; ++e) {
+                        sm.em[ob][cg * 8 + e] = ex2_fast(mm[e] * kLog2e);
+                        sm.cf[ob][cg * 8 + e] = ex2_fast((bl[e] - mm[e]) * kLog2e);
+                        sm.gm[ob][cg * 8 + e] = ex2_fast(bl[e] * kLog2e);
                     }
                 }
 #pragma unroll
-                for (int vg = 0; vg < VGH; ++vg) {
-                    const int jg = half * VGH + vg;
+                for (int it = 0; it < VIT; ++it) {
+                    const int jg = gt / TPG, t = (gt % TPG) + TPG * it;
                     float v8[8], b8[8], o8[8];
                     unpack8(*reinterpret_cast<const uint4*>(raw + 4 * KB * kBox + off_raw(t, jg)), v8);
                     unpack8(*reinterpret_cast<const uint4*>(raw + (4 * KB + VB) * kBox + off_raw(t, jg)), b8);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) o8[e] = in ? v8[e] * b8[e] : 0.0f;
+                    for (int e = 0; e < 8; ++e) o8[e] = v8[e] * b8[e];
                     *reinterpret_cast<uint4*>(sm.vh[ob] + off_vh(t, jg * 8)) = pack8(o8);
                 }
-                if (gtid == 0) {
+                if (gt == 0) {
                     sm.info[ob][0] = c;
-                    sm.info[ob][1] = w0;
-                    sm.info[ob][2] = w1;
-                    sm.info[ob][3] = (c == NC - 1) && (w1 == nval);
+                    sm.info[ob][1] = 0;
+                    sm.info[ob][2] = nval;
+                    sm.info[ob][3] = (c == NC - 1);
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm.ops_full[ob]);
                 ++item;
+            } else {
+                // ---- exact fallback: windows of 16 tokens (one warp each), or of 1 token
+                load_scan();
+                {
+                    float excl[8], wsum[8];
+                    warp_prefix(excl, wsum);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+#pragma unroll
+                        for (int u = 0; u < SEGT; ++u) b[u][e] += excl[e];
+                }
+                // first / last valid token of my warp's 16-token window
+                const int wf = gw * 16, wlst = min(wf + 15, nval - 1);
+                const int lsrc = cg + G * (((wlst - wf) / SEGT) & (SPW - 1));
+                float bf16w[8], bl16w[8], sp16 = 0.0f;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    float mine = 0.0f;
+#pragma unroll
+                    for (int u = 0; u < SEGT; ++u)
+                        if (tb + u == wlst) mine = b[u][e];
+                    bf16w[e] = __shfl_sync(full, b[0][e], cg);
+                    bl16w[e] = __shfl_sync(full, mine, lsrc);
+                    if (wf < nval) sp16 = fmaxf(sp16, bf16w[e] - bl16w[e]);
+                }
+                if (__any_sync(full, !(sp16 <= kSpanMax)) && lane == 0) sm.need1[c & 1] = c + 1;
+                named_bar(kBarGate, 128);
+                if (sm.need1[c & 1] == c + 1) W = 1;
+                if (W == 1) {
+#pragma unroll
+                    for (int u = 0; u < SEGT; ++u) {
+                        float g8[8], t8[8];
+                        unpack8(*reinterpret_cast<const uint4*>(raw + 2 * KB * kBox + off_raw(tb + u, cg)), g8);
+                        unpack8(*reinterpret_cast<const uint4*>(raw + 3 * KB * kBox + off_raw(tb + u, cg)), t8);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            b[u][e] = (tb + u < nval) ? log_alpha(g8[e], t8[e]) : 0.0f;
+                    }
+                }
+                bool ok_loop = true;
+                for (int w0 = 0; w0 < nval && ok_loop; w0 += W) {
+                    const int w1 = min(w0 + W, nval);
+                    const int ob = item % NB;
+                    if (item >= NB &&
+                        !mbar_wait(&sm.ops_empty[ob], ((item / NB) - 1) & 1, fail, kWaitLimit)) {
+                        ok_loop = false;
+                        break;
+                    }
+#pragma unroll
+                    for (int u = 0; u < SEGT; ++u) {
+                        const int t = tb + u;
+                        const bool in = t >= w0 && t < w1;
+                        float q8[8], k8[8], g8[8], t8[8], oq[8], ok[8];
+                        unpack8(*reinterpret_cast<const uint4*>(raw + 0 * KB * kBox + off_raw(t, cg)), q8);
+                        unpack8(*reinterpret_cast<const uint4*>(raw + 1 * KB * kBox + off_raw(t, cg)), k8);
+                        unpack8(*reinterpret_cast<const uint4*>(raw + 2 * KB * kBox + off_raw(t, cg)), g8);
+                        unpack8(*reinterpret_cast<const uint4*>(raw + 3 * KB * kBox + off_raw(t, cg)), t8);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const float bl = W == 1 ? b[u][e] : bl16w[e];
+                            const float m = W == 1 ? b[u][e] : 0.5f * (bf16w[e] + bl);
+                            const float d = (b[u][e] - m) * kLog2e;
+                            const float lah = t8[e] == 0.0f ? 0.0f : t8[e] * lg2_fast(g8[e]);
+                            oq[e] = in ? q8[e] * ex2_fast(d) : 0.0f;
+                            ok[e] = in ? k8[e] * ex2_fast(lah - d) : 0.0f;
+                            if (t == w0) {
+                                sm.em[ob][cg * 8 + e] = ex2_fast(m * kLog2e);
+                                sm.cf[ob][cg * 8 + e] = ex2_fast((bl - m) * kLog2e);
+                                sm.gm[ob][cg * 8 + e] = ex2_fast(bl * kLog2e);
+                            }
+                        }
+                        *reinterpret_cast<uint4*>(sm.qt[ob] + off_qk(t, cg * 8)) = pack8(oq);
+                        *reinterpret_cast<uint4*>(sm.kt[ob] + off_qk(t, cg * 8)) = pack8(ok);
+                    }
+#pragma unroll
+                    for (int it = 0; it < VIT; ++it) {
+                        const int jg = gt / TPG, t = (gt % TPG) + TPG * it;
+                        const bool in = t >= w0 && t < w1;
+                        float v8[8], b8[8], o8[8];
+                        unpack8(*reinterpret_cast<const uint4*>(raw + 4 * KB * kBox + off_raw(t, jg)), v8);
+                        unpack8(*reinterpret_cast<const uint4*>(raw + (4 * KB + VB) * kBox + off_raw(t, jg)), b8);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) o8[e] = in ? v8[e] * b8[e] : 0.0f;
+                        *reinterpret_cast<uint4*>(sm.vh[ob] + off_vh(t, jg * 8)) = pack8(o8);
+                    }
+                    if (gt == 0) {
+                        sm.info[ob][0] = c;
+                        sm.info[ob][1] = w0;
+                        sm.info[ob][2] = w1;
+                        sm.info[ob][3] = (c == NC - 1) && (w1 == nval);
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sm.ops_full[ob]);
+                    ++item;
+                }
+                if (!ok_loop) break;
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.raw_empty[st]);
@@ -441,16 +515,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             if (!mbar_wait(&sm.mma1_done, item & 1, fail, kWaitLimit)) break;
             tc_fence_after();
             // A -> causal mask -> bf16 operand (row t = tA, columns s)
-#pragma unroll
-            for (int qd = 0; qd < 4; ++qd) {
-                float v[16];
-                tmem_ld16(tmem + lb + K::COL_A + 16 * qd, v);
+            {
+                float v[64];
+                tmem_ld32(tmem + lb + K::COL_A, v);
+                tmem_ld32(tmem + lb + K::COL_A + 32, v + 32);
                 tmem_ld_wait();
                 if (rowA) {
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) v[e] = (16 * qd + e <= tA) ? v[e] : 0.0f;
-                    *reinterpret_cast<uint4*>(sm.abf + off_rowmajor64(tA, 16 * qd)) = pack8(v);
-                    *reinterpret_cast<uint4*>(sm.abf + off_rowmajor64(tA, 16 * qd + 8)) = pack8(v + 8);
+                    for (int e = 0; e < 64; ++e) v[e] = (e <= tA) ? v[e] : 0.0f;
+#pragma unroll
+                    for (int sg = 0; sg < 8; ++sg)
+                        *reinterpret_cast<uint4*>(sm.abf + off_rowmajor64(tA, 8 * sg)) = pack8(v + 8 * sg);
                 }
             }
             // S_hat = diag(exp(m)) S_prev, and the chunk-start state if requested
@@ -477,14 +552,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             // state update S = diag(gamma) S + diag(cfac) (Kt^T Vh)
             {
                 const float gmv = rowS ? sm.gm[ob][iS] : 0.0f, cfv = rowS ? sm.cf[ob][iS] : 0.0f;
+                float v[DVT];
 #pragma unroll
-                for (int qd = 0; qd < DVT / 16; ++qd) {
-                    float v[16];
-                    tmem_ld16(tmem + lb + K::COL_S + 16 * qd, v);
-                    tmem_ld_wait();
+                for (int qd = 0; qd < DVT / 32; ++qd) tmem_ld32(tmem + lb + K::COL_S + 32 * qd, v + 32 * qd);
+                tmem_ld_wait();
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) S[16 * qd + e] = fmaf(gmv, S[16 * qd + e], cfv * v[e]);
-                }
+                for (int e = 0; e < DVT; ++e) S[e] = fmaf(gmv, S[e], cfv * v[e]);
             }
             tc_fence_before();
             __syncwarp();
@@ -496,15 +569,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                 const bool st_row = rowA && tA >= w0 && tA < w1;
                 __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.o) +
                                       ((size_t)bh * T + (size_t)c * C + tA) * p.dv + j0;
+                float v[DVT];
 #pragma unroll
-                for (int qd = 0; qd < DVT / 16; ++qd) {
-                    float v[16];
-                    tmem_ld16(tmem + lb + K::COL_O + 16 * qd, v);
-                    tmem_ld_wait();
-                    if (st_row) {
-                        reinterpret_cast<uint4*>(orow + 16 * qd)[0] = pack8(v);
-                        reinterpret_cast<uint4*>(orow + 16 * qd)[1] = pack8(v + 8);
-                    }
+                for (int qd = 0; qd < DVT / 32; ++qd) tmem_ld32(tmem + lb + K::COL_O + 32 * qd, v + 32 * qd);
+                tmem_ld_wait();
+                if (st_row) {
+#pragma unroll
+                    for (int sg = 0; sg < DVT / 8; ++sg)
+                        reinterpret_cast<uint4*>(orow)[sg] = pack8(v + 8 * sg);
                 }
             }
             tc_fence_before();
