@@ -135,9 +135,11 @@ template <int DK, int DVT>
 __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_constant__ FwdKernelArgs A) {
     using K = Cfg<DK, DVT>;
     constexpr int NS = K::NS, NB = K::NB, KB = K::KB, VB = K::VB;
-    extern __shared__ uint8_t smem_dyn[];
+    // align by pointer arithmetic on the __shared__ array so that every access
+    // below stays a shared-memory access (an integer round trip would make it generic)
+    extern __shared__ __align__(1024) uint8_t smem_dyn[];
     FwdSmem<DK, DVT>& sm = *reinterpret_cast<FwdSmem<DK, DVT>*>(
-        (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+        smem_dyn + ((1024u - (smem_u32(smem_dyn) & 1023u)) & 1023u));
     const SeqParams& p = A.p;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int NJ = p.dv / DVT;
