@@ -49,7 +49,7 @@ class RdmError(RuntimeError):
 _lib = None
 
 EXPORTS = ["rdm_ddts_fwd", "rdm_ddts_saved_states_size", "rdm_ddts_bwd",
-           "rdm_ddts_bwd_workspace_size", "rdm_ddts_decode_step", "rdm_ddts_sync_status",
+           "rdm_ddts_bwd_workspace_size", "rdm_ddts_bwd_noalloc", "rdm_ddts_decode_step", "rdm_ddts_sync_status",
            "rdm_status_string", "rdm_ddts_version"]
 
 
@@ -69,6 +69,8 @@ def load():
         lib.rdm_ddts_bwd.restype = _I
         lib.rdm_ddts_bwd_workspace_size.argtypes = [ctypes.POINTER(BwdArgs)]
         lib.rdm_ddts_bwd_workspace_size.restype = ctypes.c_size_t
+        lib.rdm_ddts_bwd_noalloc.argtypes = [ctypes.POINTER(BwdArgs), _VP]
+        lib.rdm_ddts_bwd_noalloc.restype = _I
         lib.rdm_ddts_decode_step.argtypes = [_I] * 5 + [_VP] * 9
         lib.rdm_ddts_decode_step.restype = _I
         lib.rdm_ddts_sync_status.argtypes = [_VP]
@@ -176,6 +178,24 @@ def rdm_ddts_bwd(q, k, v, g, tau, beta, S0, grad_o, grad_ST=None, saved_states=N
     a = _bwd_args(q, k, v, g, tau, beta, S0, grad_o, grad_ST, saved_states, grads, workspace,
                   workspace.numel() * workspace.element_size(), chunk, impl)
     _check(load().rdm_ddts_bwd(ctypes.byref(a), _stream(stream)), "rdm_ddts_bwd")
+    return grads
+
+
+def rdm_ddts_bwd_noalloc(q, k, v, g, tau, beta, S0, grad_o, grad_ST=None, *, grads=None,
+                         chunk=0, want_dS0=True, stream=None):
+    """Backward through the library's own fixed scratch (no workspace
+    argument).  Gradient tensors are allocated with torch if not given;
+    returns the dict of gradients."""
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    grads = dict(grads or {})
+    for n, ref in (("dq", q), ("dk", k), ("dg", g), ("dtau", tau), ("dv", v), ("dbeta", beta)):
+        if grads.get(n) is None:
+            grads[n] = torch.empty_like(ref)
+    if want_dS0 and grads.get("dS0") is None:
+        grads["dS0"] = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device)
+    a = _bwd_args(q, k, v, g, tau, beta, S0, grad_o, grad_ST, None, grads, None, 0, chunk, "simt")
+    _check(load().rdm_ddts_bwd_noalloc(ctypes.byref(a), _stream(stream)), "rdm_ddts_bwd_noalloc")
     return grads
 
 

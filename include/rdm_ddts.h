@@ -142,6 +142,28 @@ rdm_status rdm_ddts_bwd(const rdm_bwd_args *args, rdm_stream_t stream);
  * and whether saved_states is given); (size_t)-1 on invalid sizes. */
 size_t rdm_ddts_bwd_workspace_size(const rdm_bwd_args *args);
 
+/* Backward without a caller-provided workspace.  The pages have no
+ * counterpart of this: it exists for callers that cannot allocate device
+ * memory when they need the gradient (a process that reserved its device
+ * memory once at start-up and may not grow it, or a callback that must not
+ * call cudaMalloc / cudaFree because those can synchronise the device).
+ *
+ * Same arguments and results as rdm_ddts_bwd computed by the exact CUDA-core
+ * path (args->impl, args->workspace and args->workspace_bytes are ignored).
+ * The scratch comes from one 16 MiB array inside the library, allocated on
+ * every device that loads it and held until the process exits.
+ *   - The first call on a device, with that device current, looks up the
+ *     array's device address; make that first call before any stream capture.
+ *   - Problems needing more scratch than 16 MiB (B*H*T*d_k*4 + B*H*d_k*4
+ *     bytes) return RDM_ERR_WORKSPACE and launch nothing.
+ *   - All calls share the one array and it keeps whatever the last call left;
+ *     nothing in it has to start at zero (each call writes every scratch
+ *     element before reading it).  Calls whose kernels overlap on the GPU
+ *     (several streams, or several host threads on one device) race on it:
+ *     serialise them.
+ */
+rdm_status rdm_ddts_bwd_noalloc(const rdm_bwd_args *args, rdm_stream_t stream);
+
 /* ------------------------------------------------------------ decode step
  * One token of sequential inference on a cached fixed-size state, O(1) per
  * token (rebuttal answers to Q1 and Q2).  For every (b,h):
