@@ -276,11 +276,14 @@ def run_extras(rdm, dev, pk, K):
     fb = fwd_bytes(w, False)  # the saved chunk states are scratch, not algorithmic traffic
     out["training_fwd_bwd"] = {
         "workload": w.name, "value": w.B * w.T / ((msf + msb) / 1e3), "unit": "tokens/s",
-        "ms_per_step": msf + msb, "ms_fwd": msf, "ms_bwd": msb, "gpu_launches_per_step": None,
+        "ms_per_step": msf + msb, "ms_fwd": msf, "ms_bwd": msb,
+        # forward kernel; backward kernel + the two exact re-run kernels (they exit at
+        # once for heads the tensor-core kernel handled)
+        "gpu_launches_per_step": 4,
         "roofline_fwd": roofline(fb, chunk_flops_fwd(w), msf, pk,
                                  ncu_traffic("tc_fwd_kernel", ["tc_fwd.cu"], 3)),
         "roofline_bwd": roofline(bwd_bytes(w), chunk_flops_bwd(w), msb, pk,
-                                 ncu_traffic("bwd", ["tc_bwd.cu", "simt.cu"], 3)),
+                                 ncu_traffic("tc_bwd_kernel", ["tc_bwd.cu"], 3)),
         "roofline_step": roofline(fb + bwd_bytes(w), chunk_flops_fwd(w) + chunk_flops_bwd(w),
                                   msf + msb, pk, None)}
     del x, o, saved, grads, ws

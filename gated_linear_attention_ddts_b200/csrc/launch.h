@@ -44,6 +44,8 @@ struct DecodeParams {
 cudaError_t launch_simt_fwd(const SeqParams& p, cudaStream_t s);
 size_t simt_bwd_workspace(const BwdParams& p);
 cudaError_t launch_simt_bwd(const BwdParams& p, cudaStream_t s);
+// same, for the heads with flags[b*H + h] != 0 only (the others return at once)
+cudaError_t launch_simt_bwd_flagged(const BwdParams& p, const int* flags, cudaStream_t s);
 
 // decode step
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s);

@@ -83,8 +83,10 @@ __global__ void __launch_bounds__(128) simt_fwd_kernel(SeqParams p) {
 
 // ------------------------------------------------ backward, forward sweep F
 template <typename T, int DV>
-__global__ void __launch_bounds__(128) simt_bwd_fsweep(BwdParams p, float* qdq, float* fin) {
+__global__ void __launch_bounds__(128) simt_bwd_fsweep(BwdParams p, float* qdq, float* fin,
+                                                       const int* only) {
     const int bh = blockIdx.x;
+    if (only && only[bh] == 0) return;  // head already handled by the tensor-core path
     const int T_ = p.T, dk = p.dk;
     const bool act = (int)threadIdx.x < dk;  // block padded to whole warps
     const int i = act ? threadIdx.x : 0;      // row of the state owned by this thread
@@ -141,8 +143,9 @@ __global__ void __launch_bounds__(128) simt_bwd_fsweep(BwdParams p, float* qdq, 
 // ------------------------------------------------ backward, reverse sweep R
 template <typename T, int DV>
 __global__ void __launch_bounds__(128) simt_bwd_rsweep(BwdParams p, const float* qdq,
-                                                       const float* fin) {
+                                                       const float* fin, const int* only) {
     const int bh = blockIdx.x;
+    if (only && only[bh] == 0) return;
     const int T_ = p.T, dk = p.dk;
     // the block is padded to whole warps; rows past d_k carry zeros
     const bool act = (int)threadIdx.x < dk;
@@ -244,22 +247,22 @@ cudaError_t fwd_t(const SeqParams& p, cudaStream_t s) {
 }
 
 template <typename T, int DV>
-cudaError_t bwd_tv(const BwdParams& p, float* qdq, float* fin, cudaStream_t s) {
+cudaError_t bwd_tv(const BwdParams& p, float* qdq, float* fin, const int* only, cudaStream_t s) {
     const int grid = p.B * p.H, block = (p.dk + 31) / 32 * 32;
-    simt_bwd_fsweep<T, DV><<<grid, block, 0, s>>>(p, qdq, fin);
+    simt_bwd_fsweep<T, DV><<<grid, block, 0, s>>>(p, qdq, fin, only);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    simt_bwd_rsweep<T, DV><<<grid, block, 0, s>>>(p, qdq, fin);
+    simt_bwd_rsweep<T, DV><<<grid, block, 0, s>>>(p, qdq, fin, only);
     return cudaGetLastError();
 }
 
 template <typename T>
-cudaError_t bwd_t(const BwdParams& p, float* qdq, float* fin, cudaStream_t s) {
+cudaError_t bwd_t(const BwdParams& p, float* qdq, float* fin, const int* only, cudaStream_t s) {
     switch (p.dv) {
-        case 16: return bwd_tv<T, 16>(p, qdq, fin, s);
-        case 32: return bwd_tv<T, 32>(p, qdq, fin, s);
-        case 64: return bwd_tv<T, 64>(p, qdq, fin, s);
-        case 128: return bwd_tv<T, 128>(p, qdq, fin, s);
+        case 16: return bwd_tv<T, 16>(p, qdq, fin, only, s);
+        case 32: return bwd_tv<T, 32>(p, qdq, fin, only, s);
+        case 64: return bwd_tv<T, 64>(p, qdq, fin, only, s);
+        case 128: return bwd_tv<T, 128>(p, qdq, fin, only, s);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -278,13 +281,19 @@ size_t simt_bwd_workspace(const BwdParams& p) {
     return a + rows * 4;
 }
 
-cudaError_t launch_simt_bwd(const BwdParams& p, cudaStream_t s) {
+static cudaError_t simt_bwd(const BwdParams& p, const int* only, cudaStream_t s) {
     if (p.B * p.H == 0) return cudaSuccess;
     const size_t rows = (size_t)p.B * p.H * p.dk;
     const size_t a = ((rows * (size_t)p.T * 4) + 255) / 256 * 256;
     float* qdq = static_cast<float*>(p.ws);
     float* fin = reinterpret_cast<float*>(static_cast<char*>(p.ws) + a);
-    return p.bf16 ? bwd_t<__nv_bfloat16>(p, qdq, fin, s) : bwd_t<float>(p, qdq, fin, s);
+    return p.bf16 ? bwd_t<__nv_bfloat16>(p, qdq, fin, only, s) : bwd_t<float>(p, qdq, fin, only, s);
+}
+
+cudaError_t launch_simt_bwd(const BwdParams& p, cudaStream_t s) { return simt_bwd(p, nullptr, s); }
+
+cudaError_t launch_simt_bwd_flagged(const BwdParams& p, const int* flags, cudaStream_t s) {
+    return simt_bwd(p, flags, s);
 }
 
 }  // namespace rdm

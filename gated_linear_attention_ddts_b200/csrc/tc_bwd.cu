@@ -1,8 +1,716 @@
-// tc_bwd.cu -- tensor-core chunked backward (placeholder until the kernel lands).
+// tc_bwd.cu -- chunkwise DDTS backward on the sm_100a tensor cores.
+//
+// The pages print no backward; this is the exact reverse mode of
+//   S_t = diag(alpha_t) S_{t-1} + khat_t vhat_t^T,  o_t = S_t^T q_t,
+// (alpha = exp(-g*tau), khat = g^tau * k, vhat = beta_hat * v; Rodimus*,
+// digest.lyk-ai.com summary, "Method") organised by chunks of 64 tokens, last
+// chunk first.  With b_t the inclusive running sum of log(alpha) in the chunk,
+// m the per-channel reference of the forward (midpoint of the b range),
+// Qt = q e^{b-m}, Kt = khat e^{m-b}, S_prev the state before the chunk (saved by
+// the forward) and R = dL/dS at the end of the chunk (flowing backwards):
+//
+//   A  = mask_{s<=t}(Qt Kt^T)          B  = mask_{s<=t}(dO Vh^T)
+//   dQ = B Kt + dO (diag(e^m) S_prev)^T          dq_t    = e^{b_t-m}  dQ_t
+//   dK = B^T Qt + Vh (diag(e^{b_last-m}) R)^T    dkhat_s = e^{m-b_s}  dK_s
+//   dV = A^T dO + Kt (diag(e^{b_last-m}) R)      dvhat_s = dV_s
+//   R <- diag(e^{b_last}) R + diag(e^m) Qt^T dO  (becomes dL/dS_0 after chunk 0)
+//
+// and the decay gradient through the identity, exact for the closed form
+// S_t = sum_s diag(e^{G_t-G_s}) khat_s vhat_s^T + diag(e^{G_t}) S_0:
+//   d log(alpha_t) = sum_{u>=t} (q_u dq_u - khat_u dkhat_u)  [+ rowsum(dS_T o S_T)]
+//   dk = alpha_hat dkhat,  dg = -tau dla + tau g^(tau-1) k dkhat,
+//   dtau = -g dla + alpha_hat ln(g) k dkhat,  dv = beta dvhat,  dbeta = v dvhat.
+//
+// One CTA per (b,h) (d_k = 64, d_v = 64 or 128), 320 threads:
+//   warps 0-3 epilogue (TMEM rows; R in fp32 registers), warps 4-7 gates
+//   (operands before the MMAs, final gate gradients and the suffix scan after),
+//   warp 8 TMA producer, warp 9 TMEM allocator + single-thread MMA issuer.
+// A chunk whose log-decay span exceeds the range one reference can hold flags
+// its head; those heads are recomputed afterwards by the exact CUDA-core
+// backward (launched behind this kernel, it skips unflagged heads).
+#include <cuda.h>
+
 #include "launch.h"
+#include "rdm_common.cuh"
+#include "tc_common.cuh"
 
 namespace rdm {
-bool tc_bwd_supported(const BwdParams&) { return false; }
-size_t tc_bwd_workspace(const BwdParams&) { return 0; }
-cudaError_t launch_tc_bwd(const BwdParams&, cudaStream_t) { return cudaErrorNotSupported; }
+namespace {
+using namespace tc;
+
+constexpr int C = 64;
+constexpr int DK = 64;
+constexpr int kThreads = 320;
+constexpr int kEpiWarp0 = 0, kGateWarp0 = 4, kProdWarp = 8, kMmaWarp = 9;
+constexpr int kBarGate = 3;  // the four gate warps
+constexpr int kStg = 68;     // row stride (floats) of the dQ / dK staging tiles
+
+template <int DV>
+struct BCfg {
+    static constexpr int VB = DV / 64;
+    static constexpr int RAW = (4 + 3 * VB) * kBox;  // q k g tau | v beta dO
+    static constexpr int OFF_V = 4 * kBox, OFF_B = (4 + VB) * kBox, OFF_DO = (4 + 2 * VB) * kBox;
+    static constexpr int COL_A = 0, COL_B = 64, COL_DQ = 128, COL_DK = 192, COL_DV = 256,
+                         COL_DR = 256 + DV;
+    static constexpr int TMEM_COLS = 512;
+};
+
+template <int DV>
+struct alignas(1024) BwdSmem {
+    uint8_t raw[BCfg<DV>::RAW];
+    uint8_t qt[8 * kQK];       // [t][i]
+    uint8_t kt[8 * kQK];       // [s][i]
+    uint8_t qtl[8 * kQK];      // bf16 remainders Qt - bf16(Qt), Kt - bf16(Kt): the
+    uint8_t ktl[8 * kQK];      // pair products of dQ and dK reach ~16 mantissa bits
+    uint8_t vh[C * DV * 2];    // [s][j], column groups 1024 B apart
+    uint8_t dot[C * DV * 2];   // [t][j]
+    // A, B, S_hat and R_hat operands of the second MMA group; once that group
+    // has completed, the same bytes hold the fp32 dQ / dK staging tiles
+    union {
+        struct {
+            uint8_t abf[C * C * 2];       // [t][s]
+            uint8_t bmb[C * C * 2];       // [t][s]
+            uint8_t shat[DK * DV * 2];    // [i][j], e^m S_prev
+            uint8_t rhat[DK * DV * 2];    // [i][j], e^{b_last-m} R
+        } op;
+        struct {
+            float dqs[C][kStg], dks[C][kStg];
+        } st;
+    } u;
+    float em[DK], cf[DK], gm[DK], fin[DK], carry[DK];
+    float bdiag[C];  // B_tt = vhat_t . dO_t (the diagonal kept out of the dQ / dK MMAs)
+    float xf[2][DK];
+    float wtot[4][DK];
+    uint64_t raw_full, raw_empty, ops_full, ops_empty, g1_done, g2_ready, tm1_free, g2_done,
+        tm2_free, post_ready, post_done;
+    uint32_t tmem_base;
+    int fail;
+};
+
+struct BwdKernelArgs {
+    CUtensorMap mq, mk, mg, mt, mv, mb, mdo;
+    BwdParams p;
+    int* flags;
+};
+
+// [row][col] tile with 8-row groups 128 B apart and 8-column groups 1024 B
+// apart (64 rows): K-major for (rows = M/N, K = cols), MN-major for (MN = cols,
+// K = rows).
+__device__ __forceinline__ uint32_t off_rc(int r, int c) {
+    return (uint32_t)((r >> 3) * 128 + (c >> 3) * 1024 + (r & 7) * 16 + (c & 7) * 2);
+}
+
+template <int DV>
+__global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_constant__ BwdKernelArgs A) {
+    using K = BCfg<DV>;
+    constexpr int VB = K::VB;
+    extern __shared__ __align__(1024) uint8_t smem_dyn[];
+    BwdSmem<DV>& sm = *reinterpret_cast<BwdSmem<DV>*>(
+        smem_dyn + ((1024u - (smem_u32(smem_dyn) & 1023u)) & 1023u));
+    const BwdParams& p = A.p;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bh = blockIdx.x;
+    const int T = p.T, NC = (T + C - 1) / C;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&sm.raw_full, 1);
+        mbar_init(&sm.raw_empty, 4);
+        mbar_init(&sm.ops_full, 4);
+        mbar_init(&sm.ops_empty, 1);
+        mbar_init(&sm.g1_done, 1);
+        mbar_init(&sm.g2_ready, 4);
+        mbar_init(&sm.tm1_free, 4);
+        mbar_init(&sm.g2_done, 1);
+        mbar_init(&sm.tm2_free, 4);
+        mbar_init(&sm.post_ready, 4);
+        mbar_init(&sm.post_done, 4);
+        sm.fail = 0;
+        fence_mbar_init();
+    }
+    if (threadIdx.x < DK) {
+        sm.fin[threadIdx.x] = 0.0f;
+        sm.carry[threadIdx.x] = 0.0f;
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc(&sm.tmem_base, K::TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (warp == kProdWarp && lane == 0) {
+        prefetch_tmap(&A.mq); prefetch_tmap(&A.mk); prefetch_tmap(&A.mg); prefetch_tmap(&A.mt);
+        prefetch_tmap(&A.mv); prefetch_tmap(&A.mb); prefetch_tmap(&A.mdo);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    volatile int* fail = &sm.fail;
+
+    if (warp == kProdWarp) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            int issued = 0;
+            for (int it = 0; it < NC; ++it) {
+                const int c = NC - 1 - it;
+                if (it > 0 && !mbar_wait(&sm.raw_empty, (it - 1) & 1, fail, kWaitLimit)) break;
+                mbar_expect_tx(&sm.raw_full, K::RAW);
+                tma_load_3d(sm.raw + 0 * kBox, &A.mq, &sm.raw_full, 0, c * C, bh);
+                tma_load_3d(sm.raw + 1 * kBox, &A.mk, &sm.raw_full, 0, c * C, bh);
+                tma_load_3d(sm.raw + 2 * kBox, &A.mg, &sm.raw_full, 0, c * C, bh);
+                tma_load_3d(sm.raw + 3 * kBox, &A.mt, &sm.raw_full, 0, c * C, bh);
+                for (int vb = 0; vb < VB; ++vb) {
+                    tma_load_3d(sm.raw + K::OFF_V + vb * kBox, &A.mv, &sm.raw_full, 64 * vb, c * C, bh);
+                    tma_load_3d(sm.raw + K::OFF_B + vb * kBox, &A.mb, &sm.raw_full, 64 * vb, c * C, bh);
+                    tma_load_3d(sm.raw + K::OFF_DO + vb * kBox, &A.mdo, &sm.raw_full, 64 * vb, c * C, bh);
+                }
+                ++issued;
+            }
+            if (issued > 0) drain_wait(&sm.raw_full, (issued - 1) & 1);
+        }
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t q = smem_u32(sm.qt), k = smem_u32(sm.kt), v = smem_u32(sm.vh);
+            const uint32_t d = smem_u32(sm.dot), a = smem_u32(sm.u.op.abf), bm = smem_u32(sm.u.op.bmb);
+            const uint32_t sh = smem_u32(sm.u.op.shat), rh = smem_u32(sm.u.op.rhat);
+            const uint32_t ql = smem_u32(sm.qtl), kl = smem_u32(sm.ktl);
+            constexpr uint32_t id_a = idesc_bf16(64, 64, 0, 0);    // A = Qt Kt^T, B = dO Vh^T
+            constexpr uint32_t id_r = idesc_bf16(DK, DV, 1, 1);    // Qt^T dO, Kt^T Vh
+            constexpr uint32_t id_q1 = idesc_bf16(64, DK, 0, 1);   // B Kt
+            constexpr uint32_t id_q2 = idesc_bf16(64, DK, 0, 0);   // dO S_hat^T
+            constexpr uint32_t id_k1 = idesc_bf16(64, DK, 1, 1);   // B^T Qt
+            constexpr uint32_t id_k2 = idesc_bf16(64, DK, 0, 0);   // Vh R_hat^T
+            constexpr uint32_t id_v1 = idesc_bf16(64, DV, 1, 1);   // A^T dO
+            constexpr uint32_t id_v2 = idesc_bf16(64, DV, 0, 1);   // Kt R_hat
+            int n1 = 0, n2 = 0;
+            for (int it = 0; it < NC; ++it) {
+                if (!mbar_wait(&sm.ops_full, it & 1, fail, kWaitLimit)) break;
+                if (it > 0 && !mbar_wait(&sm.tm1_free, (it - 1) & 1, fail, kWaitLimit)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < DK / 16; ++ks)
+                    mma_bf16(tmem + K::COL_A, sdesc(q + ks * 2 * kQK, kQK, 128),
+                             sdesc(k + ks * 2 * kQK, kQK, 128), id_a, ks > 0);
+#pragma unroll
+                for (int ks = 0; ks < DV / 16; ++ks)
+                    mma_bf16(tmem + K::COL_B, sdesc(d + ks * 2048, 1024, 128),
+                             sdesc(v + ks * 2048, 1024, 128), id_a, ks > 0);
+#pragma unroll
+                for (int ks = 0; ks < C / 16; ++ks)
+                    mma_bf16(tmem + K::COL_DR, sdesc(q + ks * 256, 128, kQK),
+                             sdesc(d + ks * 256, 128, 1024), id_r, ks > 0);
+                if (it == 0 && p.dST) {
+                    // Kt^T Vh of the last chunk, for S_T (only the final-state gradient needs it)
+#pragma unroll
+                    for (int ks = 0; ks < C / 16; ++ks)
+                        mma_bf16(tmem + K::COL_DV, sdesc(k + ks * 256, 128, kQK),
+                                 sdesc(v + ks * 256, 128, 1024), id_r, ks > 0);
+                }
+                mma_commit(&sm.g1_done);
+                ++n1;
+                if (!mbar_wait(&sm.g2_ready, it & 1, fail, kWaitLimit)) break;
+                if (it > 0 && !mbar_wait(&sm.tm2_free, (it - 1) & 1, fail, kWaitLimit)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < C / 16; ++ks)
+                    mma_bf16(tmem + K::COL_DQ, sdesc(bm + ks * 2048, 1024, 128),
+                             sdesc(k + ks * 256, 128, kQK), id_q1, ks > 0);
+#pragma unroll
+                for (int ks = 0; ks < C / 16; ++ks)
+                    mma_bf16(tmem + K::COL_DQ, sdesc(bm + ks * 2048, 1024, 128),
+                             sdesc(kl + ks * 256, 128, kQK), id_q1, 1);
+#pragma unroll
+                for (int ks = 0; ks < DV / 16; ++ks)
+                    mma_bf16(tmem + K::COL_DQ, sdesc(d + ks * 2048, 1024, 128),
+                             sdesc(sh + ks * 2048, 1024, 128), id_q2, 1);
+#pragma unroll
+                for (int ks = 0; ks < C / 16; ++ks)
+                    mma_bf16(tmem + K::COL_DK, sdesc(bm + ks * 256, 128, 1024),
+                             sdesc(q + ks * 256, 128, kQK), id_k1, ks > 0);
+#pragma unroll
+                for (int ks = 0; ks < C / 16; ++ks)
+                    mma_bf16(tmem + K::COL_DK, sdesc(bm + ks * 256, 128, 1024),
+                             sdesc(ql + ks * 256, 128, kQK), id_k1, 1);
+#pragma unroll
+                for (int ks = 0; ks < DV / 16; ++ks)
+                    mma_bf16(tmem + K::COL_DK, sdesc(v + ks * 2048, 1024, 128),
+                             sdesc(rh + ks * 2048, 1024, 128), id_k2, 1);
+#pragma unroll
+                for (int ks = 0; ks < C / 16; ++ks)
+                    mma_bf16(tmem + K::COL_DV, sdesc(a + ks * 256, 128, 1024),
+                             sdesc(d + ks * 256, 128, 1024), id_v1, ks > 0);
+#pragma unroll
+                for (int ks = 0; ks < DK / 16; ++ks)
+                    mma_bf16(tmem + K::COL_DV, sdesc(k + ks * 2 * kQK, kQK, 128),
+                             sdesc(rh + ks * 256, 128, 1024), id_v2, 1);
+                mma_commit(&sm.g2_done);
+                mma_commit(&sm.ops_empty);
+                ++n2;
+            }
+            if (n1 > 0) drain_wait(&sm.g1_done, (n1 - 1) & 1);
+            if (n2 > 0) drain_wait(&sm.g2_done, (n2 - 1) & 1);
+        }
+        __syncwarp();
+    } else if (warp >= kGateWarp0) {
+        // ------------------------------------------------------------ gates
+        constexpr int G = DK / 8, NSEG = 128 / G, SEGT = C / NSEG, SPW = 32 / G;
+        constexpr int VG = DV / 8, TPG = 128 / VG, VIT = C / TPG;
+        const int gt = (warp - kGateWarp0) * 32 + lane, gw = gt >> 5;
+        const int cg = gt % G, seg = gt / G;
+        const int tb = seg * SEGT;
+        const uint32_t full = 0xffffffffu;
+        const uint8_t* raw = sm.raw;
+        for (int it = 0; it < NC; ++it) {
+            const int c = NC - 1 - it;
+            if (!mbar_wait(&sm.raw_full, it & 1, fail, kWaitLimit)) break;
+            const int nval = min(C, T - c * C);
+            // ---- pre: running log-decay, reference, operands
+            float b[SEGT][8], mm[8];
+#pragma unroll
+            for (int u = 0; u < SEGT; ++u) {
+                float g8[8], t8[8];
+                unpack8(*reinterpret_cast<const uint4*>(raw + 2 * kBox + off_raw(tb + u, cg)), g8);
+                unpack8(*reinterpret_cast<const uint4*>(raw + 3 * kBox + off_raw(tb + u, cg)), t8);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float la = (tb + u < nval) ? log_alpha(g8[e], t8[e]) : 0.0f;
+                    b[u][e] = u == 0 ? la : b[u - 1][e] + la;
+                }
+            }
+            {
+                float excl[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float tot = b[SEGT - 1][e];
+                    float x = tot;
+#pragma unroll
+                    for (int dd = G; dd < 32; dd <<= 1) {
+                        const float y = __shfl_up_sync(full, x, dd);
+                        if (lane >= dd) x += y;
+                    }
+                    excl[e] = x - tot;
+                    const float ws = __shfl_sync(full, x, cg + G * (SPW - 1));
+                    if (lane < G) sm.wtot[gw][cg * 8 + e] = ws;
+                }
+                named_bar(kBarGate, 128);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    float off = excl[e];
+                    for (int w2 = 0; w2 < gw; ++w2) off += sm.wtot[w2][cg * 8 + e];
+#pragma unroll
+                    for (int u = 0; u < SEGT; ++u) b[u][e] += off;
+                }
+            }
+            if (tb == 0) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) sm.xf[0][cg * 8 + e] = b[0][e];
+            }
+#pragma unroll
+            for (int u = 0; u < SEGT; ++u)
+                if (tb + u == nval - 1) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) sm.xf[1][cg * 8 + e] = b[u][e];
+                }
+            named_bar(kBarGate, 128);
+            float span = 0.0f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float bl = sm.xf[1][cg * 8 + e];
+                mm[e] = 0.5f * (sm.xf[0][cg * 8 + e] + bl);
+                span = fmaxf(span, sm.xf[0][cg * 8 + e] - bl);
+            }
+            if (__any_sync(full, !(span <= kSpanMax)) && lane == 0) A.flags[bh] = 1;
+            if (it > 0 && !mbar_wait(&sm.ops_empty, (it - 1) & 1, fail, kWaitLimit)) break;
+#pragma unroll
+            for (int u = 0; u < SEGT; ++u) {
+                const int t = tb + u;
+                float q8[8], k8[8], g8[8], t8[8], oq[8], ok[8];
+                unpack8(*reinterpret_cast<const uint4*>(raw + 0 * kBox + off_raw(t, cg)), q8);
+                unpack8(*reinterpret_cast<const uint4*>(raw + 1 * kBox + off_raw(t, cg)), k8);
+                unpack8(*reinterpret_cast<const uint4*>(raw + 2 * kBox + off_raw(t, cg)), g8);
+                unpack8(*reinterpret_cast<const uint4*>(raw + 3 * kBox + off_raw(t, cg)), t8);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float dd = (b[u][e] - mm[e]) * kLog2e;
+                    const float lah = t8[e] == 0.0f ? 0.0f : t8[e] * lg2_fast(g8[e]);
+                    oq[e] = q8[e] * ex2_fast(dd);
+                    ok[e] = k8[e] * ex2_fast(lah - dd);
+                }
+                const uint4 hq = pack8(oq), hk = pack8(ok);
+                float fq[8], fk[8];
+                unpack8(hq, fq);
+                unpack8(hk, fk);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    oq[e] -= fq[e];
+                    ok[e] -= fk[e];
+                }
+                *reinterpret_cast<uint4*>(sm.qt + off_qk(t, cg * 8)) = hq;
+                *reinterpret_cast<uint4*>(sm.kt + off_qk(t, cg * 8)) = hk;
+                *reinterpret_cast<uint4*>(sm.qtl + off_qk(t, cg * 8)) = pack8(oq);
+                *reinterpret_cast<uint4*>(sm.ktl + off_qk(t, cg * 8)) = pack8(ok);
+            }
+            if (tb == 0) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float bl = sm.xf[1][cg * 8 + e];
+                    sm.em[cg * 8 + e] = ex2_fast(mm[e] * kLog2e);
+                    sm.cf[cg * 8 + e] = ex2_fast((bl - mm[e]) * kLog2e);
+                    sm.gm[cg * 8 + e] = ex2_fast(bl * kLog2e);
+                }
+            }
+#pragma unroll
+            for (int iv = 0; iv < VIT; ++iv) {
+                const int jg = gt / TPG, t = (gt % TPG) + TPG * iv;
+                float v8[8], b8[8], o8[8];
+                unpack8(*reinterpret_cast<const uint4*>(raw + K::OFF_V + off_raw(t, jg)), v8);
+                unpack8(*reinterpret_cast<const uint4*>(raw + K::OFF_B + off_raw(t, jg)), b8);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) o8[e] = v8[e] * b8[e];
+                *reinterpret_cast<uint4*>(sm.vh + off_rc(t, jg * 8)) = pack8(o8);
+                *reinterpret_cast<uint4*>(sm.dot + off_rc(t, jg * 8)) =
+                    *reinterpret_cast<const uint4*>(raw + K::OFF_DO + off_raw(t, jg));
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.ops_full);
+
+            // ---- post: final gate gradients once dQ, dK of this chunk are staged
+            if (!mbar_wait(&sm.post_ready, it & 1, fail, kWaitLimit)) break;
+            float dG[SEGT][8], dkh[SEGT][8];
+#pragma unroll
+            for (int u = 0; u < SEGT; ++u) {
+                const int t = tb + u;
+                float q8[8], k8[8], g8[8], t8[8], dqo[8];
+                unpack8(*reinterpret_cast<const uint4*>(raw + 0 * kBox + off_raw(t, cg)), q8);
+                unpack8(*reinterpret_cast<const uint4*>(raw + 1 * kBox + off_raw(t, cg)), k8);
+                unpack8(*reinterpret_cast<const uint4*>(raw + 2 * kBox + off_raw(t, cg)), g8);
+                unpack8(*reinterpret_cast<const uint4*>(raw + 3 * kBox + off_raw(t, cg)), t8);
+                const float4* dq4 = reinterpret_cast<const float4*>(&sm.u.st.dqs[t][cg * 8]);
+                const float4* dk4 = reinterpret_cast<const float4*>(&sm.u.st.dks[t][cg * 8]);
+                const float4 qa = dq4[0], qb = dq4[1], ka = dk4[0], kb4 = dk4[1];
+                const float dQv[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+                const float dKv[8] = {ka.x, ka.y, ka.z, ka.w, kb4.x, kb4.y, kb4.z, kb4.w};
+                const float bd = sm.bdiag[t];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float dd = (b[u][e] - mm[e]) * kLog2e;
+                    const float lah = t8[e] == 0.0f ? 0.0f : t8[e] * lg2_fast(g8[e]);
+                    const float kh = ex2_fast(lah) * k8[e];
+                    const float dq_off = ex2_fast(dd) * dQv[e];    // pairs s < t
+                    const float dk_off = ex2_fast(-dd) * dKv[e];   // pairs t > s
+                    dG[u][e] = q8[e] * dq_off - kh * dk_off;        // the s = t pair cancels
+                    dqo[e] = dq_off + kh * bd;
+                    dkh[u][e] = dk_off + q8[e] * bd;
+                }
+                if (c * C + t < T) {
+                    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.dq) +
+                                         ((size_t)bh * T + (size_t)c * C + t) * DK + cg * 8;
+                    *reinterpret_cast<uint4*>(dst) = pack8(dqo);
+                }
+            }
+            // suffix sums of dG: inside the segment, over later segments, later chunks
+#pragma unroll
+            for (int u = SEGT - 2; u >= 0; --u)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) dG[u][e] += dG[u + 1][e];
+            float later[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float tot = dG[0][e];
+                float x = tot;
+#pragma unroll
+                for (int dd = G; dd < 32; dd <<= 1) {
+                    const float y = __shfl_down_sync(full, x, dd);
+                    if (lane + dd < 32) x += y;
+                }
+                later[e] = x - tot;
+                const float ws = __shfl_sync(full, x, cg);  // first segment of the warp: warp total
+                if (lane < G) sm.wtot[gw][cg * 8 + e] = ws;
+            }
+            named_bar(kBarGate, 128);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                float off = later[e] + sm.carry[cg * 8 + e] + (it == 0 ? sm.fin[cg * 8 + e] : 0.0f);
+                for (int w2 = gw + 1; w2 < 4; ++w2) off += sm.wtot[w2][cg * 8 + e];
+#pragma unroll
+                for (int u = 0; u < SEGT; ++u) dG[u][e] += off;  // now d log(alpha) at token tb+u
+            }
+#pragma unroll
+            for (int u = 0; u < SEGT; ++u) {
+                const int t = tb + u;
+                float k8[8], g8[8], t8[8], odk[8], odg[8], odt[8];
+                unpack8(*reinterpret_cast<const uint4*>(raw + 1 * kBox + off_raw(t, cg)), k8);
+                unpack8(*reinterpret_cast<const uint4*>(raw + 2 * kBox + off_raw(t, cg)), g8);
+                unpack8(*reinterpret_cast<const uint4*>(raw + 3 * kBox + off_raw(t, cg)), t8);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float gg = g8[e], ta = t8[e];
+                    const float l2g = lg2_fast(gg);
+                    const float ah = ta == 0.0f ? 1.0f : ex2_fast(ta * l2g);
+                    const float dah = k8[e] * dkh[u][e];
+                    const float dah_dg = ta == 0.0f ? 0.0f : ta * ex2_fast((ta - 1.0f) * l2g);
+                    const float dah_dt = ah == 0.0f ? 0.0f : ah * l2g * kLn2;
+                    odk[e] = ah * dkh[u][e];
+                    odg[e] = -ta * dG[u][e] + dah_dg * dah;
+                    odt[e] = -gg * dG[u][e] + dah_dt * dah;
+                }
+                if (c * C + t < T) {
+                    const size_t o = ((size_t)bh * T + (size_t)c * C + t) * DK + cg * 8;
+                    *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dk_) + o) = pack8(odk);
+                    *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dg) + o) = pack8(odg);
+                    *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dtau) + o) = pack8(odt);
+                }
+            }
+            named_bar(kBarGate, 128);  // everyone has read the old carry
+            if (tb == 0) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) sm.carry[cg * 8 + e] = dG[0][e];
+            }
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&sm.post_done);
+                mbar_arrive(&sm.raw_empty);
+            }
+            if (*fail) break;
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int ew = warp - kEpiWarp0;
+        const bool row = lane < 16;  // M = 64 tiles: rows in lanes 0-15 of each sub-partition
+        const int r = 16 * ew + lane;
+        const uint32_t lb = (uint32_t)(32 * ew) << 16;
+        float R[DV];
+#pragma unroll
+        for (int j = 0; j < DV; ++j) R[j] = (row && p.dST) ? p.dST[((size_t)bh * DK + r) * DV + j] : 0.0f;
+        for (int it = 0; it < NC; ++it) {
+            const int c = NC - 1 - it;
+            if (!mbar_wait(&sm.ops_full, it & 1, fail, kWaitLimit)) break;
+            if (!mbar_wait(&sm.g1_done, it & 1, fail, kWaitLimit)) break;
+            tc_fence_after();
+            // A and B -> causal mask -> bf16 operands (row t = r)
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {
+                float v[64];
+                const uint32_t col = which == 0 ? K::COL_A : K::COL_B;
+                tmem_ld32(tmem + lb + col, v);
+                tmem_ld32(tmem + lb + col + 32, v + 32);
+                tmem_ld_wait();
+                if (row) {
+                    uint8_t* dst = which == 0 ? sm.u.op.abf : sm.u.op.bmb;
+                    // A keeps s <= t.  B keeps s < t: its diagonal contributes the
+                    // same product to q.dq and to khat.dkhat, which cancel exactly in
+                    // the decay gradient, so it is added back in fp32 after the MMAs
+                    // instead of passing through two differently rounded operands.
+                    if (which == 1) {
+                        float dg = 0.0f;
+#pragma unroll
+                        for (int e = 0; e < 64; ++e) dg = (e == r) ? v[e] : dg;
+                        sm.bdiag[r] = dg;
+                    }
+                    const int lim = which == 0 ? r : r - 1;
+#pragma unroll
+                    for (int e = 0; e < 64; ++e) v[e] = (e <= lim) ? v[e] : 0.0f;
+#pragma unroll
+                    for (int sg = 0; sg < 8; ++sg)
+                        *reinterpret_cast<uint4*>(dst + off_rc(r, 8 * sg)) = pack8(v + 8 * sg);
+                }
+            }
+            const float emv = row ? sm.em[r] : 0.0f, cfv = row ? sm.cf[r] : 0.0f;
+            const float gmv = row ? sm.gm[r] : 0.0f;
+            const float* Sprev = p.saved + (((size_t)bh * NC + c) * DK + r) * DV;
+            if (it == 0 && p.dST) {
+                // final-state term rowsum(dS_T o S_T) with S_T = diag(gm) S_prev + diag(cf) Kt^T Vh
+                float f = 0.0f;
+#pragma unroll
+                for (int qd = 0; qd < DV / 32; ++qd) {
+                    float v[32];
+                    tmem_ld32(tmem + lb + K::COL_DV + 32 * qd, v);
+                    tmem_ld_wait();
+                    if (row) {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            const int j = 32 * qd + e;
+                            f = fmaf(R[j], fmaf(gmv, Sprev[j], cfv * v[e]), f);  // R = dS_T here
+                        }
+                    }
+                }
+                if (row) sm.fin[r] = f;
+            }
+            if (row) {
+                // S_hat = diag(e^m) S_prev ; R_hat = diag(cf) R
+#pragma unroll
+                for (int jg = 0; jg < DV / 8; ++jg) {
+                    const float4 s0 = reinterpret_cast<const float4*>(Sprev)[2 * jg];
+                    const float4 s1 = reinterpret_cast<const float4*>(Sprev)[2 * jg + 1];
+                    const float xs[8] = {s0.x * emv, s0.y * emv, s0.z * emv, s0.w * emv,
+                                         s1.x * emv, s1.y * emv, s1.z * emv, s1.w * emv};
+                    *reinterpret_cast<uint4*>(sm.u.op.shat + off_rc(r, 8 * jg)) = pack8(xs);
+                    float xr[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) xr[e] = R[8 * jg + e] * cfv;
+                    *reinterpret_cast<uint4*>(sm.u.op.rhat + off_rc(r, 8 * jg)) = pack8(xr);
+                }
+            }
+            // R <- diag(e^{b_last}) R + diag(e^m) Qt^T dO
+#pragma unroll
+            for (int qd = 0; qd < DV / 32; ++qd) {
+                float v[32];
+                tmem_ld32(tmem + lb + K::COL_DR + 32 * qd, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) R[32 * qd + e] = fmaf(gmv, R[32 * qd + e], emv * v[e]);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&sm.g2_ready);
+                mbar_arrive(&sm.tm1_free);
+            }
+            if (!mbar_wait(&sm.g2_done, it & 1, fail, kWaitLimit)) break;
+            tc_fence_after();
+            // dV -> dv = beta dvhat, dbeta = v dvhat (row s = r)
+            {
+                const bool st = row && c * C + r < T;
+                const size_t o = ((size_t)bh * T + (size_t)c * C + r) * DV;
+#pragma unroll
+                for (int qd = 0; qd < DV / 32; ++qd) {
+                    float v[32];
+                    tmem_ld32(tmem + lb + K::COL_DV + 32 * qd, v);
+                    tmem_ld_wait();
+                    if (st) {
+#pragma unroll
+                        for (int h4 = 0; h4 < 4; ++h4) {
+                            const int jg = qd * 4 + h4;
+                            float v8[8], b8[8], ov[8], ob[8];
+                            unpack8(*reinterpret_cast<const uint4*>(sm.raw + K::OFF_V + off_raw(r, jg)), v8);
+                            unpack8(*reinterpret_cast<const uint4*>(sm.raw + K::OFF_B + off_raw(r, jg)), b8);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                ov[e] = b8[e] * v[8 * h4 + e];
+                                ob[e] = v8[e] * v[8 * h4 + e];
+                            }
+                            *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dv_) + o + 8 * jg) = pack8(ov);
+                            *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dbeta) + o + 8 * jg) = pack8(ob);
+                        }
+                    }
+                }
+            }
+            // dQ, dK -> fp32 staging for the gate warps
+            if (it > 0 && !mbar_wait(&sm.post_done, (it - 1) & 1, fail, kWaitLimit)) break;
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {
+                float v[64];
+                const uint32_t col = which == 0 ? K::COL_DQ : K::COL_DK;
+                tmem_ld32(tmem + lb + col, v);
+                tmem_ld32(tmem + lb + col + 32, v + 32);
+                tmem_ld_wait();
+                if (row) {
+                    float4* dst = reinterpret_cast<float4*>(which == 0 ? &sm.u.st.dqs[r][0] : &sm.u.st.dks[r][0]);
+#pragma unroll
+                    for (int e4 = 0; e4 < 16; ++e4)
+                        dst[e4] = make_float4(v[4 * e4], v[4 * e4 + 1], v[4 * e4 + 2], v[4 * e4 + 3]);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&sm.post_ready);
+                mbar_arrive(&sm.tm2_free);
+            }
+        }
+        if (!*fail && row && p.dS0) {
+            float4* dst = reinterpret_cast<float4*>(p.dS0 + ((size_t)bh * DK + r) * DV);
+#pragma unroll
+            for (int j4 = 0; j4 < DV / 4; ++j4)
+                dst[j4] = make_float4(R[4 * j4], R[4 * j4 + 1], R[4 * j4 + 2], R[4 * j4 + 3]);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, K::TMEM_COLS);
+    }
+    if (threadIdx.x == 0 && sm.fail) atomicOr(p.err, kErrTimeout);
+}
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+struct WsLayout {
+    size_t states, oscr, flags, simt, total;
+};
+
+WsLayout ws_layout(const BwdParams& p) {
+    WsLayout w;
+    const size_t bh = (size_t)p.B * p.H, nc = (size_t)(p.T + C - 1) / C;
+    w.states = p.saved ? 0 : align256(bh * nc * p.dk * p.dv * 4);
+    w.oscr = p.saved ? 0 : align256(bh * (size_t)p.T * p.dv * 2);
+    w.flags = align256(bh * 4);
+    w.simt = align256(simt_bwd_workspace(p));
+    w.total = w.states + w.oscr + w.flags + w.simt;
+    return w;
+}
+
+template <int DV>
+cudaError_t launch_dv(const BwdParams& p, const float* saved, int* flags, cudaStream_t s) {
+    BwdKernelArgs a;
+    a.p = p;
+    a.p.saved = saved;
+    a.flags = flags;
+    const uint64_t BH = (uint64_t)p.B * p.H;
+    if (!make_tmap_bf16_3d(&a.mq, p.q, DK, p.T, BH, 64, 64) ||
+        !make_tmap_bf16_3d(&a.mk, p.k, DK, p.T, BH, 64, 64) ||
+        !make_tmap_bf16_3d(&a.mg, p.g, DK, p.T, BH, 64, 64) ||
+        !make_tmap_bf16_3d(&a.mt, p.tau, DK, p.T, BH, 64, 64) ||
+        !make_tmap_bf16_3d(&a.mv, p.v, DV, p.T, BH, 64, 64) ||
+        !make_tmap_bf16_3d(&a.mb, p.beta, DV, p.T, BH, 64, 64) ||
+        !make_tmap_bf16_3d(&a.mdo, p.dO, DV, p.T, BH, 64, 64))
+        return cudaErrorInvalidValue;
+    const size_t smem = sizeof(BwdSmem<DV>) + 1024;
+    auto kern = tc_bwd_kernel<DV>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<(int)BH, kThreads, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool tc_bwd_supported(const BwdParams& p) {
+    return p.bf16 && p.chunk == C && p.T >= 1 && p.dk == DK && (p.dv == 64 || p.dv == 128);
+}
+
+size_t tc_bwd_workspace(const BwdParams& p) { return ws_layout(p).total; }
+
+cudaError_t launch_tc_bwd(const BwdParams& p, cudaStream_t s) {
+    if (!tc_bwd_supported(p)) return cudaErrorNotSupported;
+    const WsLayout w = ws_layout(p);
+    char* ws = static_cast<char*>(p.ws);
+    const float* saved = p.saved;
+    cudaError_t e;
+    if (!saved) {
+        // recompute the chunk-start states with the forward kernel
+        SeqParams f;
+        f.B = p.B; f.H = p.H; f.T = p.T; f.dk = p.dk; f.dv = p.dv; f.chunk = p.chunk; f.bf16 = 1;
+        f.q = p.q; f.k = p.k; f.v = p.v; f.g = p.g; f.tau = p.tau; f.beta = p.beta; f.S0 = p.S0;
+        f.o = ws + w.states;
+        f.ST = nullptr;
+        f.saved = reinterpret_cast<float*>(ws);
+        f.err = p.err;
+        if ((e = launch_tc_fwd(f, s)) != cudaSuccess) return e;
+        saved = f.saved;
+    }
+    int* flags = reinterpret_cast<int*>(ws + w.states + w.oscr);
+    if ((e = cudaMemsetAsync(flags, 0, (size_t)p.B * p.H * 4, s)) != cudaSuccess) return e;
+    e = p.dv == 64 ? launch_dv<64>(p, saved, flags, s) : launch_dv<128>(p, saved, flags, s);
+    if (e != cudaSuccess) return e;
+    // heads whose decay span needs narrower windows: exact CUDA-core backward
+    BwdParams q = p;
+    q.ws = ws + w.states + w.oscr + w.flags;
+    q.ws_bytes = w.simt;
+    return launch_simt_bwd_flagged(q, flags, s);
+}
+
 }  // namespace rdm

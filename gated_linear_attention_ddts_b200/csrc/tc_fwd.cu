@@ -28,7 +28,7 @@
 
 #include "launch.h"
 #include "rdm_common.cuh"
-#include "tc_ptx.cuh"
+#include "tc_common.cuh"
 
 namespace rdm {
 namespace {
@@ -36,15 +36,9 @@ using namespace tc;
 
 constexpr int C = 64;                        // tokens per chunk (tile rows)
 constexpr int kThreads = 320;
-constexpr float kSpanMax = 120.0f;           // largest in-window log-decay span
-constexpr long long kWaitLimit = 2000000000LL;  // ~1 s of SM clocks
 constexpr int kEpiWarp0 = 0, kGateWarp0 = 4, kProdWarp = 8, kMmaWarp = 9;
 constexpr int kBarPair = 1;  // +half: the two gate warps of one channel half (64 threads)
 constexpr int kBarGate = 3;  // the four gate warps (128 threads)
-constexpr int kBox = 64 * 64 * 2;  // bytes of one 64x64 bf16 TMA box
-// channel-group stride of the Qt / Kt operand tiles: 1024 + 16 bytes, the skew
-// spreads the channel groups a warp writes for one token over all banks
-constexpr int kQK = 1040;
 
 template <int DK, int DVT>
 struct Cfg {
@@ -82,54 +76,6 @@ struct FwdKernelArgs {
     CUtensorMap mq, mk, mg, mt, mv, mb;
     SeqParams p;
 };
-
-// ---- shared-memory operand offsets (bytes), canonical no-swizzle UMMA layouts
-// A_bf16: K-major, 8-row groups 128 B apart, K groups 1024 B apart
-__device__ __forceinline__ uint32_t off_rowmajor64(int r, int k) {
-    return (uint32_t)((r >> 3) * 128 + (k >> 3) * 1024 + (r & 7) * 16 + (k & 7) * 2);
-}
-// Qt, Kt: K-major [token][channel], 8-token groups 128 B apart, channel groups
-// kQK B apart
-__device__ __forceinline__ uint32_t off_qk(int t, int i) {
-    return (uint32_t)((t >> 3) * 128 + (i >> 3) * kQK + (t & 7) * 16 + (i & 7) * 2);
-}
-// Vh [s][j] stored MN-major for N = j: j groups 1024 B apart, s groups 128 B apart
-__device__ __forceinline__ uint32_t off_vh(int s, int j) {
-    return (uint32_t)((j >> 3) * 1024 + (s >> 3) * 128 + (s & 7) * 16 + (j & 7) * 2);
-}
-// S_hat [i][j] stored MN-major for N = j: j groups DK*16 B apart, i groups 128 B apart
-template <int DK>
-__device__ __forceinline__ uint32_t off_shat(int i, int j) {
-    return (uint32_t)((j >> 3) * (DK * 16) + (i >> 3) * 128 + (i & 7) * 16 + (j & 7) * 2);
-}
-// 8 consecutive bf16 of row t, column group cg, in a tile of 64-wide 128B-swizzled boxes
-__device__ __forceinline__ uint32_t off_raw(int t, int cg) {
-    return (uint32_t)((cg >> 3) * kBox + t * 128 + (((cg & 7) ^ (t & 7)) << 4));
-}
-
-__device__ __forceinline__ void unpack8(uint4 u, float* f) {
-    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        const float2 x = __bfloat1622float2(h[e]);
-        f[2 * e] = x.x;
-        f[2 * e + 1] = x.y;
-    }
-}
-__device__ __forceinline__ uint4 pack8(const float* f) {
-    uint4 u;
-    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) h[e] = __floats2bfloat162_rn(f[2 * e], f[2 * e + 1]);
-    return u;
-}
-
-__device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
-    const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity))
-        if (clock64() - t0 > kWaitLimit) return false;
-    return true;
-}
 
 template <int DK, int DVT>
 __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_constant__ FwdKernelArgs A) {
