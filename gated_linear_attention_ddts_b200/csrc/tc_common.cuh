@@ -42,13 +42,14 @@ __device__ __forceinline__ uint32_t off_raw(int t, int cg) {
     return (uint32_t)((cg >> 3) * kBox + t * 128 + (((cg & 7) ^ (t & 7)) << 4));
 }
 
+// bf16 -> fp32 is a 16-bit shift of the bit pattern; doing it with integer
+// ops keeps it off the conversion pipe that the exp2/log2 instructions need.
 __device__ __forceinline__ void unpack8(uint4 u, float* f) {
-    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-        const float2 x = __bfloat1622float2(h[e]);
-        f[2 * e] = x.x;
-        f[2 * e + 1] = x.y;
+        f[2 * e] = __uint_as_float(w[e] << 16);
+        f[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
     }
 }
 __device__ __forceinline__ uint4 pack8(const float* f) {

@@ -37,7 +37,6 @@ using namespace tc;
 constexpr int C = 64;                        // tokens per chunk (tile rows)
 constexpr int kThreads = 320;
 constexpr int kEpiWarp0 = 0, kGateWarp0 = 4, kProdWarp = 8, kMmaWarp = 9;
-constexpr int kBarPair = 1;  // +half: the two gate warps of one channel half (64 threads)
 constexpr int kBarGate = 3;  // the four gate warps (128 threads)
 
 template <int DK, int DVT>
@@ -63,8 +62,6 @@ struct alignas(1024) FwdSmem {
     uint8_t shat[DK * DVT * 2];
     float em[K::NB][DK], cf[K::NB][DK], gm[K::NB][DK];
     int info[K::NB][4];  // chunk, w0, w1, last
-    float xf[2][DK];     // gate exchange: b at the first and at the last token of the chunk
-    float wtot[4][DK];   // gate exchange: per-warp scan totals
     uint64_t raw_full[K::NS], raw_empty[K::NS], ops_full[K::NB], ops_empty[K::NB];
     uint64_t mma1_done, as_free, abf_full, mmao_done, o_free;
     int need16[2], need1[2];
@@ -201,12 +198,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
         __syncwarp();
     } else if (warp >= kGateWarp0) {
         // ------------------------------------------------------------ gates
-        // thread -> (8-channel group cg, segment of SEGT consecutive tokens); a warp
-        // covers 16 consecutive tokens, so a 16-token window never leaves a warp
-        constexpr int G = K::G, NSEG = 128 / G, SEGT = C / NSEG, SPW = 32 / G;
+        // warp gw owns channel groups [gw*GW, gw*GW + GW) (8 channels each) for all
+        // 64 tokens; lane -> (group cgl, segment of SEGT consecutive tokens).  The
+        // running sum of log(alpha) is an in-thread scan plus a shuffle scan over
+        // the segments: no data crosses warps.  The chunk is cut into windows of W
+        // tokens (64, or 16 / 1 when the decay span is too wide for one
+        // reference); only that choice is agreed across the gate warps.
+        constexpr int G = K::G, GW = G / 4, NSW = 32 / GW, SEGT = C / NSW;
         constexpr int VG = DVT / 8, TPG = 128 / VG, VIT = C / TPG;
-        const int gt = (warp - kGateWarp0) * 32 + lane, gw = gt >> 5;
-        const int cg = gt % G, seg = gt / G;
+        const int gw = warp - kGateWarp0, gt = gw * 32 + lane;
+        const int cgl = lane % GW, seg = lane / GW;
+        const int cg = gw * GW + cgl;
         const int tb = seg * SEGT;  // first token of my segment
         const uint32_t full = 0xffffffffu;
         int item = 0;
@@ -215,9 +217,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             if (!mbar_wait(&sm.raw_full[st], (c / NS) & 1, fail, kWaitLimit)) break;
             const uint8_t* raw = sm.raw[st];
             const int nval = min(C, T - c * C);
-            float b[SEGT][8];
-            // b <- log(alpha) = -g*tau of my tokens (0 past T), then its running sum
-            auto load_scan = [&]() {
+            float b[SEGT][8], bf[8], bl[8];
+            // window-relative inclusive running sum of log(alpha) over my tokens, and
+            // b at the first / last valid token of my window (W in {64, 16})
+            auto scan = [&](int W) {
 #pragma unroll
                 for (int u = 0; u < SEGT; ++u) {
                     float g8[8], t8[8];
@@ -226,77 +229,70 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const float la = (tb + u < nval) ? log_alpha(g8[e], t8[e]) : 0.0f;
-                        b[u][e] = u == 0 ? la : b[u - 1][e] + la;
+                        b[u][e] = (u == 0 || W == 1) ? la : b[u - 1][e] + la;
                     }
                 }
-            };
-            // exclusive prefix of segment totals over the segments of this warp
-            auto warp_prefix = [&](float* excl, float* wsum) {
+                if (W == 1) return;
+                const int WL = W / SEGT * GW;        // lanes per window
+                const int l0 = lane & ~(WL - 1);     // first lane of my window
+                const int tw0 = (l0 / GW) * SEGT;    // first token of my window
+                const int tl = min(tw0 + W, nval) - 1;  // last valid token of my window
+                const int lsrc = cgl + GW * (max(tl, tw0) / SEGT);
+                const int usrc = max(tl, tw0) % SEGT;
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const float tot = b[SEGT - 1][e];
                     float x = tot;
 #pragma unroll
-                    for (int d = G; d < 32; d <<= 1) {
+                    for (int d = GW; d < 32; d <<= 1) {
                         const float y = __shfl_up_sync(full, x, d);
-                        if (lane >= d) x += y;
+                        if ((lane & (WL - 1)) >= d) x += y;
                     }
-                    excl[e] = x - tot;
-                    wsum[e] = __shfl_sync(full, x, cg + G * (SPW - 1));
+                    const float excl = x - tot;
+                    float mine = 0.0f;
+#pragma unroll
+                    for (int u = 0; u < SEGT; ++u) {
+                        b[u][e] += excl;
+                        if (u == usrc) mine = b[u][e];
+                    }
+                    bf[e] = __shfl_sync(full, b[0][e], l0 + cgl);
+                    bl[e] = __shfl_sync(full, mine, lsrc);
                 }
             };
-            load_scan();
-            {
-                float excl[8], wsum[8];
-                warp_prefix(excl, wsum);
-                if (lane < G) {
+            // true when some window of this chunk spans more log-decay than one
+            // reference holds; every gate warp takes the same answer
+            auto too_wide = [&](int* flag) {
+                float span = 0.0f;
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) sm.wtot[gw][cg * 8 + e] = wsum[e];
-                }
+                for (int e = 0; e < 8; ++e) span = fmaxf(span, bf[e] - bl[e]);
+                if (tb >= nval) span = 0.0f;
+                if (__any_sync(full, !(span <= kSpanMax)) && lane == 0) *flag = c + 1;
                 named_bar(kBarGate, 128);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    float off = excl[e];
-                    for (int w2 = 0; w2 < gw; ++w2) off += sm.wtot[w2][cg * 8 + e];
-#pragma unroll
-                    for (int u = 0; u < SEGT; ++u) b[u][e] += off;
+                return *flag == c + 1;
+            };
+            int W = C;
+            scan(C);
+            if (too_wide(&sm.need16[c & 1])) {
+                W = 16;
+                scan(16);
+                if (too_wide(&sm.need1[c & 1])) {
+                    W = 1;
+                    scan(1);
                 }
             }
-            if (tb == 0) {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) sm.xf[0][cg * 8 + e] = b[0][e];
-            }
-            if (tb <= nval - 1 && nval - 1 < tb + SEGT) {
-#pragma unroll
-                for (int u = 0; u < SEGT; ++u)
-                    if (tb + u == nval - 1) {
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) sm.xf[1][cg * 8 + e] = b[u][e];
-                    }
-            }
-            named_bar(kBarGate, 128);
-            // window size: 64, or 16 / 1 when the decay span is too wide for one reference
-            float span = 0.0f;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) span = fmaxf(span, sm.xf[0][cg * 8 + e] - sm.xf[1][cg * 8 + e]);
-            if (__any_sync(full, !(span <= kSpanMax)) && lane == 0) sm.need16[c & 1] = c + 1;
-            named_bar(kBarGate, 128);
-            int W = sm.need16[c & 1] == c + 1 ? 16 : C;
-
-            if (W == C) {
-                // ---- hot path: one window = the whole chunk
+            bool ok_loop = true;
+            for (int w0 = 0; w0 < nval; w0 += W) {
+                const int w1 = min(w0 + W, nval);
                 const int ob = item % NB;
-                if (item >= NB && !mbar_wait(&sm.ops_empty[ob], ((item / NB) - 1) & 1, fail, kWaitLimit))
+                if (item >= NB &&
+                    !mbar_wait(&sm.ops_empty[ob], ((item / NB) - 1) & 1, fail, kWaitLimit)) {
+                    ok_loop = false;
                     break;
-                float mm[8], bl[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    bl[e] = sm.xf[1][cg * 8 + e];
-                    mm[e] = 0.5f * (sm.xf[0][cg * 8 + e] + bl[e]);
                 }
 #pragma unroll
                 for (int u = 0; u < SEGT; ++u) {
                     const int t = tb + u;
+                    const bool in = t >= w0 && t < w1;
                     float q8[8], k8[8], g8[8], t8[8], oq[8], ok[8];
                     unpack8(*reinterpret_cast<const uint4*>(raw + 0 * KB * kBox + off_raw(t, cg)), q8);
                     unpack8(*reinterpret_cast<const uint4*>(raw + 1 * KB * kBox + off_raw(t, cg)), k8);
@@ -304,140 +300,45 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                     unpack8(*reinterpret_cast<const uint4*>(raw + 3 * KB * kBox + off_raw(t, cg)), t8);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        const float d = (b[u][e] - mm[e]) * kLog2e;
+                        // reference m = midpoint of the window's b range, blast = b at its end
+                        const float blast = W == 1 ? b[u][e] : bl[e];
+                        const float m = W == 1 ? b[u][e] : 0.5f * (bf[e] + bl[e]);
+                        const float d = (b[u][e] - m) * kLog2e;
                         const float lah = t8[e] == 0.0f ? 0.0f : t8[e] * lg2_fast(g8[e]);
-                        oq[e] = q8[e] * ex2_fast(d);
-                        ok[e] = k8[e] * ex2_fast(lah - d);
+                        oq[e] = in ? q8[e] * ex2_fast(d) : 0.0f;
+                        ok[e] = in ? k8[e] * ex2_fast(lah - d) : 0.0f;
+                        if (t == w0) {
+                            sm.em[ob][cg * 8 + e] = ex2_fast(m * kLog2e);
+                            sm.cf[ob][cg * 8 + e] = ex2_fast((blast - m) * kLog2e);
+                            sm.gm[ob][cg * 8 + e] = ex2_fast(blast * kLog2e);
+                        }
                     }
                     *reinterpret_cast<uint4*>(sm.qt[ob] + off_qk(t, cg * 8)) = pack8(oq);
                     *reinterpret_cast<uint4*>(sm.kt[ob] + off_qk(t, cg * 8)) = pack8(ok);
                 }
-                if (tb == 0) {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        sm.em[ob][cg * 8 + e] = ex2_fast(mm[e] * kLog2e);
-                        sm.cf[ob][cg * 8 + e] = ex2_fast((bl[e] - mm[e]) * kLog2e);
-                        sm.gm[ob][cg * 8 + e] = ex2_fast(bl[e] * kLog2e);
-                    }
-                }
 #pragma unroll
                 for (int it = 0; it < VIT; ++it) {
                     const int jg = gt / TPG, t = (gt % TPG) + TPG * it;
+                    const bool in = t >= w0 && t < w1;
                     float v8[8], b8[8], o8[8];
                     unpack8(*reinterpret_cast<const uint4*>(raw + 4 * KB * kBox + off_raw(t, jg)), v8);
                     unpack8(*reinterpret_cast<const uint4*>(raw + (4 * KB + VB) * kBox + off_raw(t, jg)), b8);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) o8[e] = v8[e] * b8[e];
+                    for (int e = 0; e < 8; ++e) o8[e] = in ? v8[e] * b8[e] : 0.0f;
                     *reinterpret_cast<uint4*>(sm.vh[ob] + off_vh(t, jg * 8)) = pack8(o8);
                 }
                 if (gt == 0) {
                     sm.info[ob][0] = c;
-                    sm.info[ob][1] = 0;
-                    sm.info[ob][2] = nval;
-                    sm.info[ob][3] = (c == NC - 1);
+                    sm.info[ob][1] = w0;
+                    sm.info[ob][2] = w1;
+                    sm.info[ob][3] = (c == NC - 1) && (w1 == nval);
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm.ops_full[ob]);
                 ++item;
-            } else {
-                // ---- exact fallback: windows of 16 tokens (one warp each), or of 1 token
-                load_scan();
-                {
-                    float excl[8], wsum[8];
-                    warp_prefix(excl, wsum);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-#pragma unroll
-                        for (int u = 0; u < SEGT; ++u) b[u][e] += excl[e];
-                }
-                // first / last valid token of my warp's 16-token window
-                const int wf = gw * 16, wlst = min(wf + 15, nval - 1);
-                const int lsrc = cg + G * (((wlst - wf) / SEGT) & (SPW - 1));
-                float bf16w[8], bl16w[8], sp16 = 0.0f;
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    float mine = 0.0f;
-#pragma unroll
-                    for (int u = 0; u < SEGT; ++u)
-                        if (tb + u == wlst) mine = b[u][e];
-                    bf16w[e] = __shfl_sync(full, b[0][e], cg);
-                    bl16w[e] = __shfl_sync(full, mine, lsrc);
-                    if (wf < nval) sp16 = fmaxf(sp16, bf16w[e] - bl16w[e]);
-                }
-                if (__any_sync(full, !(sp16 <= kSpanMax)) && lane == 0) sm.need1[c & 1] = c + 1;
-                named_bar(kBarGate, 128);
-                if (sm.need1[c & 1] == c + 1) W = 1;
-                if (W == 1) {
-#pragma unroll
-                    for (int u = 0; u < SEGT; ++u) {
-                        float g8[8], t8[8];
-                        unpack8(*reinterpret_cast<const uint4*>(raw + 2 * KB * kBox + off_raw(tb + u, cg)), g8);
-                        unpack8(*reinterpret_cast<const uint4*>(raw + 3 * KB * kBox + off_raw(tb + u, cg)), t8);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            b[u][e] = (tb + u < nval) ? log_alpha(g8[e], t8[e]) : 0.0f;
-                    }
-                }
-                bool ok_loop = true;
-                for (int w0 = 0; w0 < nval && ok_loop; w0 += W) {
-                    const int w1 = min(w0 + W, nval);
-                    const int ob = item % NB;
-                    if (item >= NB &&
-                        !mbar_wait(&sm.ops_empty[ob], ((item / NB) - 1) & 1, fail, kWaitLimit)) {
-                        ok_loop = false;
-                        break;
-                    }
-#pragma unroll
-                    for (int u = 0; u < SEGT; ++u) {
-                        const int t = tb + u;
-                        const bool in = t >= w0 && t < w1;
-                        float q8[8], k8[8], g8[8], t8[8], oq[8], ok[8];
-                        unpack8(*reinterpret_cast<const uint4*>(raw + 0 * KB * kBox + off_raw(t, cg)), q8);
-                        unpack8(*reinterpret_cast<const uint4*>(raw + 1 * KB * kBox + off_raw(t, cg)), k8);
-                        unpack8(*reinterpret_cast<const uint4*>(raw + 2 * KB * kBox + off_raw(t, cg)), g8);
-                        unpack8(*reinterpret_cast<const uint4*>(raw + 3 * KB * kBox + off_raw(t, cg)), t8);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const float bl = W == 1 ? b[u][e] : bl16w[e];
-                            const float m = W == 1 ? b[u][e] : 0.5f * (bf16w[e] + bl);
-                            const float d = (b[u][e] - m) * kLog2e;
-                            const float lah = t8[e] == 0.0f ? 0.0f : t8[e] * lg2_fast(g8[e]);
-                            oq[e] = in ? q8[e] * ex2_fast(d) : 0.0f;
-                            ok[e] = in ? k8[e] * ex2_fast(lah - d) : 0.0f;
-                            if (t == w0) {
-                                sm.em[ob][cg * 8 + e] = ex2_fast(m * kLog2e);
-                                sm.cf[ob][cg * 8 + e] = ex2_fast((bl - m) * kLog2e);
-                                sm.gm[ob][cg * 8 + e] = ex2_fast(bl * kLog2e);
-                            }
-                        }
-                        *reinterpret_cast<uint4*>(sm.qt[ob] + off_qk(t, cg * 8)) = pack8(oq);
-                        *reinterpret_cast<uint4*>(sm.kt[ob] + off_qk(t, cg * 8)) = pack8(ok);
-                    }
-#pragma unroll
-                    for (int it = 0; it < VIT; ++it) {
-                        const int jg = gt / TPG, t = (gt % TPG) + TPG * it;
-                        const bool in = t >= w0 && t < w1;
-                        float v8[8], b8[8], o8[8];
-                        unpack8(*reinterpret_cast<const uint4*>(raw + 4 * KB * kBox + off_raw(t, jg)), v8);
-                        unpack8(*reinterpret_cast<const uint4*>(raw + (4 * KB + VB) * kBox + off_raw(t, jg)), b8);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) o8[e] = in ? v8[e] * b8[e] : 0.0f;
-                        *reinterpret_cast<uint4*>(sm.vh[ob] + off_vh(t, jg * 8)) = pack8(o8);
-                    }
-                    if (gt == 0) {
-                        sm.info[ob][0] = c;
-                        sm.info[ob][1] = w0;
-                        sm.info[ob][2] = w1;
-                        sm.info[ob][3] = (c == NC - 1) && (w1 == nval);
-                    }
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&sm.ops_full[ob]);
-                    ++item;
-                }
-                if (!ok_loop) break;
             }
+            if (!ok_loop) break;
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.raw_empty[st]);
             if (*fail) break;
