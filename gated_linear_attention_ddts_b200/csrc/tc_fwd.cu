@@ -280,42 +280,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                     scan(1);
                 }
             }
-            bool ok_loop = true;
-            for (int w0 = 0; w0 < nval; w0 += W) {
-                const int w1 = min(w0 + W, nval);
-                const int ob = item % NB;
-                if (item >= NB &&
-                    !mbar_wait(&sm.ops_empty[ob], ((item / NB) - 1) & 1, fail, kWaitLimit)) {
-                    ok_loop = false;
-                    break;
-                }
-#pragma unroll
-                for (int u = 0; u < SEGT; ++u) {
-                    const int t = tb + u;
-                    const bool in = t >= w0 && t < w1;
-                    float q8[8], k8[8], g8[8], t8[8], oq[8], ok[8];
-                    unpack8(*reinterpret_cast<const uint4*>(raw + 0 * KB * kBox + off_raw(t, cg)), q8);
-                    unpack8(*reinterpret_cast<const uint4*>(raw + 1 * KB * kBox + off_raw(t, cg)), k8);
-                    unpack8(*reinterpret_cast<const uint4*>(raw + 2 * KB * kBox + off_raw(t, cg)), g8);
-                    unpack8(*reinterpret_cast<const uint4*>(raw + 3 * KB * kBox + off_raw(t, cg)), t8);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        // reference m = midpoint of the window's b range, blast = b at its end
-                        const float blast = W == 1 ? b[u][e] : bl[e];
-                        const float m = W == 1 ? b[u][e] : 0.5f * (bf[e] + bl[e]);
-                        const float d = (b[u][e] - m) * kLog2e;
-                        const float lah = t8[e] == 0.0f ? 0.0f : t8[e] * lg2_fast(g8[e]);
-                        oq[e] = in ? q8[e] * ex2_fast(d) : 0.0f;
-                        ok[e] = in ? k8[e] * ex2_fast(lah - d) : 0.0f;
-                        if (t == w0) {
-                            sm.em[ob][cg * 8 + e] = ex2_fast(m * kLog2e);
-                            sm.cf[ob][cg * 8 + e] = ex2_fast((blast - m) * kLog2e);
-                            sm.gm[ob][cg * 8 + e] = ex2_fast(blast * kLog2e);
-                        }
-                    }
-                    *reinterpret_cast<uint4*>(sm.qt[ob] + off_qk(t, cg * 8)) = pack8(oq);
-                    *reinterpret_cast<uint4*>(sm.kt[ob] + off_qk(t, cg * 8)) = pack8(ok);
-                }
+            // Vh = beta_hat * v for the rows of [w0, w1), zero elsewhere
+            auto write_vh = [&](int ob, int w0, int w1) {
 #pragma unroll
                 for (int it = 0; it < VIT; ++it) {
                     const int jg = gt / TPG, t = (gt % TPG) + TPG * it;
@@ -327,6 +293,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                     for (int e = 0; e < 8; ++e) o8[e] = in ? v8[e] * b8[e] : 0.0f;
                     *reinterpret_cast<uint4*>(sm.vh[ob] + off_vh(t, jg * 8)) = pack8(o8);
                 }
+            };
+            auto publish = [&](int ob, int w0, int w1) {
                 if (gt == 0) {
                     sm.info[ob][0] = c;
                     sm.info[ob][1] = w0;
@@ -336,9 +304,88 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm.ops_full[ob]);
+            };
+            if (W == C) {
+                // ---- one window = the whole chunk (rows past T hold zeros from the
+                // TMA fill, so every row can be computed unmasked)
+                const int ob = item % NB;
+                if (item >= NB && !mbar_wait(&sm.ops_empty[ob], ((item / NB) - 1) & 1, fail, kWaitLimit))
+                    break;
+                float mL[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) mL[e] = 0.5f * (bf[e] + bl[e]) * kLog2e;
+#pragma unroll
+                for (int u = 0; u < SEGT; ++u) {
+                    const int t = tb + u;
+                    float q8[8], k8[8], g8[8], t8[8], oq[8], ok[8];
+                    unpack8(*reinterpret_cast<const uint4*>(raw + 0 * KB * kBox + off_raw(t, cg)), q8);
+                    unpack8(*reinterpret_cast<const uint4*>(raw + 1 * KB * kBox + off_raw(t, cg)), k8);
+                    unpack8(*reinterpret_cast<const uint4*>(raw + 2 * KB * kBox + off_raw(t, cg)), g8);
+                    unpack8(*reinterpret_cast<const uint4*>(raw + 3 * KB * kBox + off_raw(t, cg)), t8);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float d = fmaf(b[u][e], kLog2e, -mL[e]);
+                        const float lah = t8[e] == 0.0f ? 0.0f : t8[e] * lg2_fast(g8[e]);
+                        oq[e] = q8[e] * ex2_fast(d);
+                        ok[e] = k8[e] * ex2_fast(lah - d);
+                    }
+                    *reinterpret_cast<uint4*>(sm.qt[ob] + off_qk(t, cg * 8)) = pack8(oq);
+                    *reinterpret_cast<uint4*>(sm.kt[ob] + off_qk(t, cg * 8)) = pack8(ok);
+                }
+                if (tb == 0) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        sm.em[ob][cg * 8 + e] = ex2_fast(mL[e]);
+                        sm.cf[ob][cg * 8 + e] = ex2_fast(bl[e] * kLog2e - mL[e]);
+                        sm.gm[ob][cg * 8 + e] = ex2_fast(bl[e] * kLog2e);
+                    }
+                }
+                write_vh(ob, 0, C);
+                publish(ob, 0, nval);
                 ++item;
+            } else {
+                bool ok_loop = true;
+                for (int w0 = 0; w0 < nval; w0 += W) {
+                    const int w1 = min(w0 + W, nval);
+                    const int ob = item % NB;
+                    if (item >= NB &&
+                        !mbar_wait(&sm.ops_empty[ob], ((item / NB) - 1) & 1, fail, kWaitLimit)) {
+                        ok_loop = false;
+                        break;
+                    }
+#pragma unroll 1
+                    for (int u = 0; u < SEGT; ++u) {
+                        const int t = tb + u;
+                        const bool in = t >= w0 && t < w1;
+                        float q8[8], k8[8], g8[8], t8[8], oq[8], ok[8];
+                        unpack8(*reinterpret_cast<const uint4*>(raw + 0 * KB * kBox + off_raw(t, cg)), q8);
+                        unpack8(*reinterpret_cast<const uint4*>(raw + 1 * KB * kBox + off_raw(t, cg)), k8);
+                        unpack8(*reinterpret_cast<const uint4*>(raw + 2 * KB * kBox + off_raw(t, cg)), g8);
+                        unpack8(*reinterpret_cast<const uint4*>(raw + 3 * KB * kBox + off_raw(t, cg)), t8);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            // reference m = midpoint of the window's b range, blast = b at its end
+                            const float blast = W == 1 ? b[u][e] : bl[e];
+                            const float m = W == 1 ? b[u][e] : 0.5f * (bf[e] + bl[e]);
+                            const float d = (b[u][e] - m) * kLog2e;
+                            const float lah = t8[e] == 0.0f ? 0.0f : t8[e] * lg2_fast(g8[e]);
+                            oq[e] = in ? q8[e] * ex2_fast(d) : 0.0f;
+                            ok[e] = in ? k8[e] * ex2_fast(lah - d) : 0.0f;
+                            if (t == w0) {
+                                sm.em[ob][cg * 8 + e] = ex2_fast(m * kLog2e);
+                                sm.cf[ob][cg * 8 + e] = ex2_fast((blast - m) * kLog2e);
+                                sm.gm[ob][cg * 8 + e] = ex2_fast(blast * kLog2e);
+                            }
+                        }
+                        *reinterpret_cast<uint4*>(sm.qt[ob] + off_qk(t, cg * 8)) = pack8(oq);
+                        *reinterpret_cast<uint4*>(sm.kt[ob] + off_qk(t, cg * 8)) = pack8(ok);
+                    }
+                    write_vh(ob, w0, w1);
+                    publish(ob, w0, w1);
+                    ++item;
+                }
+                if (!ok_loop) break;
             }
-            if (!ok_loop) break;
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.raw_empty[st]);
             if (*fail) break;
