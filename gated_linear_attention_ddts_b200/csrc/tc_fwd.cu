@@ -47,8 +47,10 @@ struct Cfg {
     static constexpr int VB = DVT / 64;            // boxes per value-side tile
     static constexpr int RAW = (4 * KB + 2 * VB) * kBox;
     static constexpr int G = DK / 8;               // 8-channel groups
+    // A | dS | O (double-buffered: the epilogue reads O of one chunk while the
+    // tensor core writes the next)
     static constexpr int COL_A = 0, COL_S = 64, COL_O = 64 + DVT;
-    static constexpr int TMEM_COLS = (64 + 2 * DVT) <= 256 ? 256 : 512;
+    static constexpr int TMEM_COLS = (64 + 3 * DVT) <= 256 ? 256 : 512;
 };
 
 template <int DK, int DVT>
@@ -63,7 +65,7 @@ struct alignas(1024) FwdSmem {
     float em[K::NB][DK], cf[K::NB][DK], gm[K::NB][DK];
     int info[K::NB][4];  // chunk, w0, w1, last
     uint64_t raw_full[K::NS], raw_empty[K::NS], ops_full[K::NB], ops_empty[K::NB];
-    uint64_t mma1_done, as_free, abf_full, mmao_done, o_free;
+    uint64_t mma1_done, as_free, abf_full, mmao_done[2], o_free[2];
     int need16[2], need1[2];
     uint32_t tmem_base;
     int fail;
@@ -101,8 +103,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
         mbar_init(&sm.mma1_done, 1);
         mbar_init(&sm.as_free, 4);
         mbar_init(&sm.abf_full, 4);
-        mbar_init(&sm.mmao_done, 1);
-        mbar_init(&sm.o_free, 4);
+        mbar_init(&sm.mmao_done[0], 1);
+        mbar_init(&sm.mmao_done[1], 1);
+        mbar_init(&sm.o_free[0], 4);
+        mbar_init(&sm.o_free[1], 4);
         sm.need16[0] = sm.need16[1] = sm.need1[0] = sm.need1[1] = 0;
         sm.fail = 0;
         fence_mbar_init();
@@ -174,18 +178,19 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                 mma_commit(&sm.mma1_done);
                 ++n1;
                 if (!mbar_wait(&sm.abf_full, item & 1, fail, kWaitLimit)) break;
-                if (item > 0 && !mbar_wait(&sm.o_free, (item - 1) & 1, fail, kWaitLimit)) break;
+                const int obuf = item & 1;
+                if (item >= 2 && !mbar_wait(&sm.o_free[obuf], ((item >> 1) - 1) & 1, fail, kWaitLimit)) break;
                 tc_fence_after();
                 const uint32_t a = smem_u32(sm.abf), sh = smem_u32(sm.shat);
 #pragma unroll
                 for (int ks = 0; ks < C / 16; ++ks)
-                    mma_bf16(tO, sdesc(a + ks * 2048, 1024, 128), sdesc(v + ks * 256, 128, 1024), idO,
-                             ks > 0);
+                    mma_bf16(tO + obuf * DVT, sdesc(a + ks * 2048, 1024, 128),
+                             sdesc(v + ks * 256, 128, 1024), idO, ks > 0);
 #pragma unroll
                 for (int ks = 0; ks < DK / 16; ++ks)
-                    mma_bf16(tO, sdesc(q + ks * 2 * kQK, kQK, 128), sdesc(sh + ks * 256, 128, DK * 16),
-                             idO, 1);
-                mma_commit(&sm.mmao_done);
+                    mma_bf16(tO + obuf * DVT, sdesc(q + ks * 2 * kQK, kQK, 128),
+                             sdesc(sh + ks * 256, 128, DK * 16), idO, 1);
+                mma_commit(&sm.mmao_done[obuf]);
                 mma_commit(&sm.ops_empty[ob]);
                 ++nO;
                 if (last) break;
@@ -193,7 +198,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             }
             // let issued MMAs finish before TMEM is released
             if (n1 > 0) drain_wait(&sm.mma1_done, (n1 - 1) & 1);
-            if (nO > 0) drain_wait(&sm.mmao_done, (nO - 1) & 1);
+            if (nO > 0) drain_wait(&sm.mmao_done[(nO - 1) & 1], ((nO - 1) >> 1) & 1);
         }
         __syncwarp();
     } else if (warp >= kGateWarp0) {
@@ -402,7 +407,31 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
 #pragma unroll
         for (int j = 0; j < DVT; ++j)
             S[j] = (rowS && p.S0) ? p.S0[((size_t)bh * DK + iS) * p.dv + j0 + j] : 0.0f;
-        int item = 0;
+        // o rows [w0, w1) of chunk c from the O buffer of item `it`
+        auto store_o = [&](int it, int c, int w0, int w1) -> bool {
+            const int obuf = it & 1;
+            if (!mbar_wait(&sm.mmao_done[obuf], (it >> 1) & 1, fail, kWaitLimit)) return false;
+            tc_fence_after();
+            const bool st_row = rowA && tA >= w0 && tA < w1;
+            __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.o) +
+                                  ((size_t)bh * T + (size_t)c * C + tA) * p.dv + j0;
+#pragma unroll
+            for (int qd = 0; qd < DVT / 32; ++qd) {
+                float v[32];
+                tmem_ld32(tmem + lb + K::COL_O + obuf * DVT + 32 * qd, v);
+                tmem_ld_wait();
+                if (st_row) {
+#pragma unroll
+                    for (int sg = 0; sg < 4; ++sg)
+                        reinterpret_cast<uint4*>(orow)[4 * qd + sg] = pack8(v + 8 * sg);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.o_free[obuf]);
+            return true;
+        };
+        int item = 0, pc = 0, pw0 = 0, pw1 = 0;
         while (true) {
             const int ob = item % NB;
             if (!mbar_wait(&sm.ops_full[ob], (item / NB) & 1, fail, kWaitLimit)) break;
@@ -458,30 +487,20 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.as_free);
-            // o rows of this window
-            if (!mbar_wait(&sm.mmao_done, item & 1, fail, kWaitLimit)) break;
-            tc_fence_after();
-            {
-                const bool st_row = rowA && tA >= w0 && tA < w1;
-                __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.o) +
-                                      ((size_t)bh * T + (size_t)c * C + tA) * p.dv + j0;
-                float v[DVT];
-#pragma unroll
-                for (int qd = 0; qd < DVT / 32; ++qd) tmem_ld32(tmem + lb + K::COL_O + 32 * qd, v + 32 * qd);
-                tmem_ld_wait();
-                if (st_row) {
-#pragma unroll
-                    for (int sg = 0; sg < DVT / 8; ++sg)
-                        reinterpret_cast<uint4*>(orow)[sg] = pack8(v + 8 * sg);
-                }
-            }
-            tc_fence_before();
+            // the constants of this item are consumed: its operand slot can refill
+            // once the tensor core is done with it too
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&sm.o_free);
-                mbar_arrive(&sm.ops_empty[ob]);
+            if (lane == 0) mbar_arrive(&sm.ops_empty[ob]);
+            // o of the previous item (its MMA finished while this item's A and state
+            // were processed), then of this one if it is the last
+            if (item > 0 && !store_o(item - 1, pc, pw0, pw1)) break;
+            if (last) {
+                store_o(item, c, w0, w1);
+                break;
             }
-            if (last) break;
+            pc = c;
+            pw0 = w0;
+            pw1 = w1;
             ++item;
         }
         if (!*fail && rowS && p.ST) {
