@@ -35,9 +35,10 @@ namespace {
 using namespace tc;
 
 constexpr int C = 64;                        // tokens per chunk (tile rows)
-constexpr int kThreads = 320;
-constexpr int kEpiWarp0 = 0, kGateWarp0 = 4, kProdWarp = 8, kMmaWarp = 9;
-constexpr int kBarGate = 3;  // the four gate warps (128 threads)
+constexpr int kGateWarps = 8;  // two per SM sub-partition
+constexpr int kThreads = 32 * (4 + kGateWarps + 2);
+constexpr int kEpiWarp0 = 0, kGateWarp0 = 4, kProdWarp = 4 + kGateWarps, kMmaWarp = 5 + kGateWarps;
+constexpr int kBarGate = 3;  // all gate warps
 
 template <int DK, int DVT>
 struct Cfg {
@@ -94,10 +95,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
             mbar_init(&sm.raw_full[s], 1);
-            mbar_init(&sm.raw_empty[s], 4);
+            mbar_init(&sm.raw_empty[s], kGateWarps);
         }
         for (int b = 0; b < NB; ++b) {
-            mbar_init(&sm.ops_full[b], 4);
+            mbar_init(&sm.ops_full[b], kGateWarps);
             mbar_init(&sm.ops_empty[b], 1 + 4);
         }
         mbar_init(&sm.mma1_done, 1);
@@ -209,8 +210,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
         // the segments: no data crosses warps.  The chunk is cut into windows of W
         // tokens (64, or 16 / 1 when the decay span is too wide for one
         // reference); only that choice is agreed across the gate warps.
-        constexpr int G = K::G, GW = G / 4, NSW = 32 / GW, SEGT = C / NSW;
-        constexpr int VG = DVT / 8, TPG = 128 / VG, VIT = C / TPG;
+        constexpr int G = K::G, GW = G / kGateWarps, NSW = 32 / GW, SEGT = C / NSW;
+        constexpr int VG = DVT / 8, TPG = 32 * kGateWarps / VG, VIT = C / TPG;
         const int gw = warp - kGateWarp0, gt = gw * 32 + lane;
         const int cgl = lane % GW, seg = lane / GW;
         const int cg = gw * GW + cgl;
@@ -272,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                 for (int e = 0; e < 8; ++e) span = fmaxf(span, bf[e] - bl[e]);
                 if (tb >= nval) span = 0.0f;
                 if (__any_sync(full, !(span <= kSpanMax)) && lane == 0) *flag = c + 1;
-                named_bar(kBarGate, 128);
+                named_bar(kBarGate, 32 * kGateWarps);
                 return *flag == c + 1;
             };
             int W = C;
@@ -440,17 +441,18 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             if (!mbar_wait(&sm.mma1_done, item & 1, fail, kWaitLimit)) break;
             tc_fence_after();
             // A -> causal mask -> bf16 operand (row t = tA, columns s)
-            {
-                float v[64];
-                tmem_ld32(tmem + lb + K::COL_A, v);
-                tmem_ld32(tmem + lb + K::COL_A + 32, v + 32);
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                float v[32];
+                tmem_ld32(tmem + lb + K::COL_A + 32 * hf, v);
                 tmem_ld_wait();
                 if (rowA) {
 #pragma unroll
-                    for (int e = 0; e < 64; ++e) v[e] = (e <= tA) ? v[e] : 0.0f;
+                    for (int e = 0; e < 32; ++e) v[e] = (32 * hf + e <= tA) ? v[e] : 0.0f;
 #pragma unroll
-                    for (int sg = 0; sg < 8; ++sg)
-                        *reinterpret_cast<uint4*>(sm.abf + off_rowmajor64(tA, 8 * sg)) = pack8(v + 8 * sg);
+                    for (int sg = 0; sg < 4; ++sg)
+                        *reinterpret_cast<uint4*>(sm.abf + off_rowmajor64(tA, 32 * hf + 8 * sg)) =
+                            pack8(v + 8 * sg);
                 }
             }
             // S_hat = diag(exp(m)) S_prev, and the chunk-start state if requested
@@ -477,12 +479,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             // state update S = diag(gamma) S + diag(cfac) (Kt^T Vh)
             {
                 const float gmv = rowS ? sm.gm[ob][iS] : 0.0f, cfv = rowS ? sm.cf[ob][iS] : 0.0f;
-                float v[DVT];
 #pragma unroll
-                for (int qd = 0; qd < DVT / 32; ++qd) tmem_ld32(tmem + lb + K::COL_S + 32 * qd, v + 32 * qd);
-                tmem_ld_wait();
+                for (int qd = 0; qd < DVT / 32; ++qd) {
+                    float v[32];
+                    tmem_ld32(tmem + lb + K::COL_S + 32 * qd, v);
+                    tmem_ld_wait();
 #pragma unroll
-                for (int e = 0; e < DVT; ++e) S[e] = fmaf(gmv, S[e], cfv * v[e]);
+                    for (int e = 0; e < 32; ++e) S[32 * qd + e] = fmaf(gmv, S[32 * qd + e], cfv * v[e]);
+                }
             }
             tc_fence_before();
             __syncwarp();
