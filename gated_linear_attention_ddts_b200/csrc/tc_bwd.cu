@@ -40,9 +40,9 @@ using namespace tc;
 
 constexpr int C = 64;
 constexpr int DK = 64;
-constexpr int kThreads = 320;
-constexpr int kEpiWarp0 = 0, kGateWarp0 = 4, kProdWarp = 8, kMmaWarp = 9;
-constexpr int kBarGate = 3;  // the four gate warps
+constexpr int kGateWarps = 8;  // one 8-channel group each
+constexpr int kThreads = 32 * (4 + kGateWarps + 2);
+constexpr int kEpiWarp0 = 0, kGateWarp0 = 4, kProdWarp = 4 + kGateWarps, kMmaWarp = 5 + kGateWarps;
 constexpr int kStg = 68;     // row stride (floats) of the dQ / dK staging tiles
 
 template <int DV>
@@ -70,19 +70,17 @@ struct alignas(1024) BwdSmem {
         struct {
             uint8_t abf[C * C * 2];       // [t][s]
             uint8_t bmb[C * C * 2];       // [t][s]
-            uint8_t shat[DK * DV * 2];    // [i][j], e^m S_prev
             uint8_t rhat[DK * DV * 2];    // [i][j], e^{b_last-m} R
         } op;
         struct {
             float dqs[C][kStg], dks[C][kStg];
         } st;
     } u;
+    uint8_t shat[DK * DV * 2];  // [i][j], e^m S_prev (written by the gate warps)
     float em[DK], cf[DK], gm[DK], fin[DK], carry[DK];
     float bdiag[C];  // B_tt = vhat_t . dO_t (the diagonal kept out of the dQ / dK MMAs)
-    float xf[2][DK];
-    float wtot[4][DK];
-    uint64_t raw_full, raw_empty, ops_full, ops_empty, g1_done, g2_ready, tm1_free, g2_done,
-        tm2_free, post_ready, post_done;
+    uint64_t raw_full, raw_empty, ops_full, shat_full, ops_empty, g1_done, g2_ready, tm1_free,
+        g2_done, tm2_free, post_ready, post_done;
     uint32_t tmem_base;
     int fail;
 };
@@ -114,8 +112,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
 
     if (threadIdx.x == 0) {
         mbar_init(&sm.raw_full, 1);
-        mbar_init(&sm.raw_empty, 4);
-        mbar_init(&sm.ops_full, 4);
+        mbar_init(&sm.raw_empty, kGateWarps);
+        mbar_init(&sm.ops_full, kGateWarps);
+        mbar_init(&sm.shat_full, kGateWarps);
         mbar_init(&sm.ops_empty, 1);
         mbar_init(&sm.g1_done, 1);
         mbar_init(&sm.g2_ready, 4);
@@ -123,7 +122,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
         mbar_init(&sm.g2_done, 1);
         mbar_init(&sm.tm2_free, 4);
         mbar_init(&sm.post_ready, 4);
-        mbar_init(&sm.post_done, 4);
+        mbar_init(&sm.post_done, kGateWarps);
         sm.fail = 0;
         fence_mbar_init();
     }
@@ -171,7 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
         if (lane == 0) {
             const uint32_t q = smem_u32(sm.qt), k = smem_u32(sm.kt), v = smem_u32(sm.vh);
             const uint32_t d = smem_u32(sm.dot), a = smem_u32(sm.u.op.abf), bm = smem_u32(sm.u.op.bmb);
-            const uint32_t sh = smem_u32(sm.u.op.shat), rh = smem_u32(sm.u.op.rhat);
+            const uint32_t sh = smem_u32(sm.shat), rh = smem_u32(sm.u.op.rhat);
             const uint32_t ql = smem_u32(sm.qtl), kl = smem_u32(sm.ktl);
             constexpr uint32_t id_a = idesc_bf16(64, 64, 0, 0);    // A = Qt Kt^T, B = dO Vh^T
             constexpr uint32_t id_r = idesc_bf16(DK, DV, 1, 1);    // Qt^T dO, Kt^T Vh
@@ -208,6 +207,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 mma_commit(&sm.g1_done);
                 ++n1;
                 if (!mbar_wait(&sm.g2_ready, it & 1, fail, kWaitLimit)) break;
+                if (!mbar_wait(&sm.shat_full, it & 1, fail, kWaitLimit)) break;
                 if (it > 0 && !mbar_wait(&sm.tm2_free, (it - 1) & 1, fail, kWaitLimit)) break;
                 tc_fence_after();
 #pragma unroll
@@ -252,10 +252,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
         __syncwarp();
     } else if (warp >= kGateWarp0) {
         // ------------------------------------------------------------ gates
-        constexpr int G = DK / 8, NSEG = 128 / G, SEGT = C / NSEG, SPW = 32 / G;
-        constexpr int VG = DV / 8, TPG = 128 / VG, VIT = C / TPG;
-        const int gt = (warp - kGateWarp0) * 32 + lane, gw = gt >> 5;
-        const int cg = gt % G, seg = gt / G;
+        // warp gw owns channel group gw (8 channels) for all 64 tokens; lane ->
+        // segment of SEGT tokens.  Prefix (running log-decay) and suffix (decay
+        // gradient) scans are in-thread plus shuffles: no data crosses warps.
+        constexpr int G = DK / 8, GW = G / kGateWarps, NSW = 32 / GW, SEGT = C / NSW;
+        constexpr int VG = DV / 8, TPG = 32 * kGateWarps / VG, VIT = C / TPG;
+        const int gw = warp - kGateWarp0, gt = gw * 32 + lane;
+        const int cgl = lane % GW, seg = lane / GW;
+        const int cg = gw * GW + cgl;
         const int tb = seg * SEGT;
         const uint32_t full = 0xffffffffu;
         const uint8_t* raw = sm.raw;
@@ -264,7 +268,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             if (!mbar_wait(&sm.raw_full, it & 1, fail, kWaitLimit)) break;
             const int nval = min(C, T - c * C);
             // ---- pre: running log-decay, reference, operands
-            float b[SEGT][8], mm[8];
+            float b[SEGT][8], mL[8], blL[8];
 #pragma unroll
             for (int u = 0; u < SEGT; ++u) {
                 float g8[8], t8[8];
@@ -277,48 +281,33 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 }
             }
             {
-                float excl[8];
+                const int tl = nval - 1;
+                const int lsrc = cgl + GW * (tl / SEGT), usrc = tl % SEGT;
+                float span = 0.0f;
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const float tot = b[SEGT - 1][e];
                     float x = tot;
 #pragma unroll
-                    for (int dd = G; dd < 32; dd <<= 1) {
-                        const float y = __shfl_up_sync(full, x, dd);
-                        if (lane >= dd) x += y;
+                    for (int d = GW; d < 32; d <<= 1) {
+                        const float y = __shfl_up_sync(full, x, d);
+                        if (lane >= d) x += y;
                     }
-                    excl[e] = x - tot;
-                    const float ws = __shfl_sync(full, x, cg + G * (SPW - 1));
-                    if (lane < G) sm.wtot[gw][cg * 8 + e] = ws;
+                    float mine = 0.0f;
+#pragma unroll
+                    for (int u = 0; u < SEGT; ++u) {
+                        b[u][e] += x - tot;
+                        if (u == usrc) mine = b[u][e];
+                    }
+                    const float bf = __shfl_sync(full, b[0][e], cgl);
+                    const float bl = __shfl_sync(full, mine, lsrc);
+                    mL[e] = 0.5f * (bf + bl) * kLog2e;
+                    blL[e] = bl * kLog2e;
+                    span = fmaxf(span, bf - bl);
                 }
-                named_bar(kBarGate, 128);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    float off = excl[e];
-                    for (int w2 = 0; w2 < gw; ++w2) off += sm.wtot[w2][cg * 8 + e];
-#pragma unroll
-                    for (int u = 0; u < SEGT; ++u) b[u][e] += off;
-                }
+                // too wide for one reference: the exact path recomputes this head
+                if (__any_sync(full, !(span <= kSpanMax)) && lane == 0) A.flags[bh] = 1;
             }
-            if (tb == 0) {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) sm.xf[0][cg * 8 + e] = b[0][e];
-            }
-#pragma unroll
-            for (int u = 0; u < SEGT; ++u)
-                if (tb + u == nval - 1) {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) sm.xf[1][cg * 8 + e] = b[u][e];
-                }
-            named_bar(kBarGate, 128);
-            float span = 0.0f;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float bl = sm.xf[1][cg * 8 + e];
-                mm[e] = 0.5f * (sm.xf[0][cg * 8 + e] + bl);
-                span = fmaxf(span, sm.xf[0][cg * 8 + e] - bl);
-            }
-            if (__any_sync(full, !(span <= kSpanMax)) && lane == 0) A.flags[bh] = 1;
             if (it > 0 && !mbar_wait(&sm.ops_empty, (it - 1) & 1, fail, kWaitLimit)) break;
 #pragma unroll
             for (int u = 0; u < SEGT; ++u) {
@@ -330,7 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 unpack8(*reinterpret_cast<const uint4*>(raw + 3 * kBox + off_raw(t, cg)), t8);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    const float dd = (b[u][e] - mm[e]) * kLog2e;
+                    const float dd = fmaf(b[u][e], kLog2e, -mL[e]);
                     const float lah = t8[e] == 0.0f ? 0.0f : t8[e] * lg2_fast(g8[e]);
                     oq[e] = q8[e] * ex2_fast(dd);
                     ok[e] = k8[e] * ex2_fast(lah - dd);
@@ -352,10 +341,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             if (tb == 0) {
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    const float bl = sm.xf[1][cg * 8 + e];
-                    sm.em[cg * 8 + e] = ex2_fast(mm[e] * kLog2e);
-                    sm.cf[cg * 8 + e] = ex2_fast((bl - mm[e]) * kLog2e);
-                    sm.gm[cg * 8 + e] = ex2_fast(bl * kLog2e);
+                    sm.em[cg * 8 + e] = ex2_fast(mL[e]);
+                    sm.cf[cg * 8 + e] = ex2_fast(blL[e] - mL[e]);
+                    sm.gm[cg * 8 + e] = ex2_fast(blL[e]);
                 }
             }
 #pragma unroll
@@ -373,6 +361,27 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.ops_full);
+            // S_hat = diag(e^m) S_prev for this warp's rows (channels), while the
+            // first MMA group runs
+#pragma unroll
+            for (int gi = 0; gi < GW; ++gi) {
+                const int i = (gw * GW + gi) * 8 + (lane >> 2);
+                const float* Sp = p.saved + (((size_t)bh * NC + c) * DK + i) * DV;
+                constexpr int CPT = DV / 4;  // 8 rows x DV columns over 32 lanes
+                const int c0 = (lane & 3) * CPT;
+                const float emr = sm.em[i];
+#pragma unroll
+                for (int j8 = 0; j8 < CPT / 8; ++j8) {
+                    const float4 s0 = *reinterpret_cast<const float4*>(Sp + c0 + 8 * j8);
+                    const float4 s1 = *reinterpret_cast<const float4*>(Sp + c0 + 8 * j8 + 4);
+                    const float xs[8] = {s0.x * emr, s0.y * emr, s0.z * emr, s0.w * emr,
+                                         s1.x * emr, s1.y * emr, s1.z * emr, s1.w * emr};
+                    *reinterpret_cast<uint4*>(sm.shat + off_rc(i, c0 + 8 * j8)) = pack8(xs);
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.shat_full);
 
             // ---- post: final gate gradients once dQ, dK of this chunk are staged
             if (!mbar_wait(&sm.post_ready, it & 1, fail, kWaitLimit)) break;
@@ -393,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 const float bd = sm.bdiag[t];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    const float dd = (b[u][e] - mm[e]) * kLog2e;
+                    const float dd = fmaf(b[u][e], kLog2e, -mL[e]);
                     const float lah = t8[e] == 0.0f ? 0.0f : t8[e] * lg2_fast(g8[e]);
                     const float kh = ex2_fast(lah) * k8[e];
                     const float dq_off = ex2_fast(dd) * dQv[e];    // pairs s < t
@@ -408,32 +417,24 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                     *reinterpret_cast<uint4*>(dst) = pack8(dqo);
                 }
             }
-            // suffix sums of dG: inside the segment, over later segments, later chunks
+            // d log(alpha) = suffix sum of dG: in the segment, over later segments of
+            // this warp (= later tokens of the chunk), over later chunks (carry)
 #pragma unroll
             for (int u = SEGT - 2; u >= 0; --u)
 #pragma unroll
                 for (int e = 0; e < 8; ++e) dG[u][e] += dG[u + 1][e];
-            float later[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 const float tot = dG[0][e];
                 float x = tot;
 #pragma unroll
-                for (int dd = G; dd < 32; dd <<= 1) {
-                    const float y = __shfl_down_sync(full, x, dd);
-                    if (lane + dd < 32) x += y;
+                for (int d = GW; d < 32; d <<= 1) {
+                    const float y = __shfl_down_sync(full, x, d);
+                    if (lane + d < 32) x += y;
                 }
-                later[e] = x - tot;
-                const float ws = __shfl_sync(full, x, cg);  // first segment of the warp: warp total
-                if (lane < G) sm.wtot[gw][cg * 8 + e] = ws;
-            }
-            named_bar(kBarGate, 128);
+                const float off = (x - tot) + sm.carry[cg * 8 + e] + (it == 0 ? sm.fin[cg * 8 + e] : 0.0f);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                float off = later[e] + sm.carry[cg * 8 + e] + (it == 0 ? sm.fin[cg * 8 + e] : 0.0f);
-                for (int w2 = gw + 1; w2 < 4; ++w2) off += sm.wtot[w2][cg * 8 + e];
-#pragma unroll
-                for (int u = 0; u < SEGT; ++u) dG[u][e] += off;  // now d log(alpha) at token tb+u
+                for (int u = 0; u < SEGT; ++u) dG[u][e] += off;
             }
 #pragma unroll
             for (int u = 0; u < SEGT; ++u) {
@@ -461,7 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                     *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dtau) + o) = pack8(odt);
                 }
             }
-            named_bar(kBarGate, 128);  // everyone has read the old carry
+            __syncwarp();  // every lane has read the old carry
             if (tb == 0) {
 #pragma unroll
                 for (int e = 0; e < 8; ++e) sm.carry[cg * 8 + e] = dG[0][e];
@@ -537,14 +538,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 if (row) sm.fin[r] = f;
             }
             if (row) {
-                // S_hat = diag(e^m) S_prev ; R_hat = diag(cf) R
+                // R_hat = diag(cf) R  (S_hat is written by the gate warps)
 #pragma unroll
                 for (int jg = 0; jg < DV / 8; ++jg) {
-                    const float4 s0 = reinterpret_cast<const float4*>(Sprev)[2 * jg];
-                    const float4 s1 = reinterpret_cast<const float4*>(Sprev)[2 * jg + 1];
-                    const float xs[8] = {s0.x * emv, s0.y * emv, s0.z * emv, s0.w * emv,
-                                         s1.x * emv, s1.y * emv, s1.z * emv, s1.w * emv};
-                    *reinterpret_cast<uint4*>(sm.u.op.shat + off_rc(r, 8 * jg)) = pack8(xs);
                     float xr[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) xr[e] = R[8 * jg + e] * cfv;
