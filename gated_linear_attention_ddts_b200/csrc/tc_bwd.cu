@@ -21,10 +21,10 @@
 //   dk = alpha_hat dkhat,  dg = -tau dla + tau g^(tau-1) k dkhat,
 //   dtau = -g dla + alpha_hat ln(g) k dkhat,  dv = beta dvhat,  dbeta = v dvhat.
 //
-// One CTA per (b,h) (d_k = 64, d_v = 64 or 128), 320 threads:
-//   warps 0-3 epilogue (TMEM rows; R in fp32 registers), warps 4-7 gates
+// One CTA per (b,h) (d_k = 64, d_v = 64 or 128), 448 threads:
+//   warps 0-3 epilogue (TMEM rows; R in fp32 registers), warps 4-11 gates
 //   (operands before the MMAs, final gate gradients and the suffix scan after),
-//   warp 8 TMA producer, warp 9 TMEM allocator + single-thread MMA issuer.
+//   warp 12 TMA producer, warp 13 TMEM allocator + single-thread MMA issuer.
 // A chunk whose log-decay span exceeds the range one reference can hold flags
 // its head; those heads are recomputed afterwards by the exact CUDA-core
 // backward (launched behind this kernel, it skips unflagged heads).
@@ -476,82 +476,78 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
         }
     } else {
         // ------------------------------------------------------------ epilogue
+        // M = 64 accumulators sit in TMEM lanes 0-15 of each sub-partition; the
+        // split load hands row r = 16 ew + (lane & 15) to two threads, lane >> 4
+        // selecting which half of the columns each one holds.
+        constexpr int HV = DV / 2;  // state columns per thread
         const int ew = warp - kEpiWarp0;
-        const bool row = lane < 16;  // M = 64 tiles: rows in lanes 0-15 of each sub-partition
-        const int r = 16 * ew + lane;
+        const int hf = lane >> 4;
+        const int r = 16 * ew + (lane & 15);
         const uint32_t lb = (uint32_t)(32 * ew) << 16;
-        float R[DV];
+        float R[HV];  // R[r][hf*HV .. hf*HV + HV)
 #pragma unroll
-        for (int j = 0; j < DV; ++j) R[j] = (row && p.dST) ? p.dST[((size_t)bh * DK + r) * DV + j] : 0.0f;
+        for (int j = 0; j < HV; ++j) R[j] = p.dST ? p.dST[((size_t)bh * DK + r) * DV + hf * HV + j] : 0.0f;
         for (int it = 0; it < NC; ++it) {
             const int c = NC - 1 - it;
             if (!mbar_wait(&sm.ops_full, it & 1, fail, kWaitLimit)) break;
             if (!mbar_wait(&sm.g1_done, it & 1, fail, kWaitLimit)) break;
             tc_fence_after();
-            // A and B -> causal mask -> bf16 operands (row t = r)
+            // A and B -> causal mask -> bf16 operands (row t = r, columns s = 32 hf + e)
 #pragma unroll
             for (int which = 0; which < 2; ++which) {
-                float v[64];
-                const uint32_t col = which == 0 ? K::COL_A : K::COL_B;
-                tmem_ld32(tmem + lb + col, v);
-                tmem_ld32(tmem + lb + col + 32, v + 32);
+                float v[32];
+                tmem_ld32_split<32>(tmem + lb + (which == 0 ? K::COL_A : K::COL_B), v);
                 tmem_ld_wait();
-                if (row) {
-                    uint8_t* dst = which == 0 ? sm.u.op.abf : sm.u.op.bmb;
-                    // A keeps s <= t.  B keeps s < t: its diagonal contributes the
-                    // same product to q.dq and to khat.dkhat, which cancel exactly in
-                    // the decay gradient, so it is added back in fp32 after the MMAs
-                    // instead of passing through two differently rounded operands.
-                    if (which == 1) {
-                        float dg = 0.0f;
+                uint8_t* dst = which == 0 ? sm.u.op.abf : sm.u.op.bmb;
+                // A keeps s <= t.  B keeps s < t: its diagonal contributes the same
+                // product to q.dq and to khat.dkhat, which cancel exactly in the
+                // decay gradient, so it is added back in fp32 after the MMAs
+                // instead of passing through two differently rounded operands.
+                if (which == 1 && (r >> 5) == hf) {
+                    float dg = 0.0f;
 #pragma unroll
-                        for (int e = 0; e < 64; ++e) dg = (e == r) ? v[e] : dg;
-                        sm.bdiag[r] = dg;
-                    }
-                    const int lim = which == 0 ? r : r - 1;
-#pragma unroll
-                    for (int e = 0; e < 64; ++e) v[e] = (e <= lim) ? v[e] : 0.0f;
-#pragma unroll
-                    for (int sg = 0; sg < 8; ++sg)
-                        *reinterpret_cast<uint4*>(dst + off_rc(r, 8 * sg)) = pack8(v + 8 * sg);
+                    for (int e = 0; e < 32; ++e) dg = (32 * hf + e == r) ? v[e] : dg;
+                    sm.bdiag[r] = dg;
                 }
+                const int lim = (which == 0 ? r : r - 1) - 32 * hf;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) v[e] = (e <= lim) ? v[e] : 0.0f;
+#pragma unroll
+                for (int sg = 0; sg < 4; ++sg)
+                    *reinterpret_cast<uint4*>(dst + off_rc(r, 32 * hf + 8 * sg)) = pack8(v + 8 * sg);
             }
-            const float emv = row ? sm.em[r] : 0.0f, cfv = row ? sm.cf[r] : 0.0f;
-            const float gmv = row ? sm.gm[r] : 0.0f;
-            const float* Sprev = p.saved + (((size_t)bh * NC + c) * DK + r) * DV;
+            const float emv = sm.em[r], cfv = sm.cf[r], gmv = sm.gm[r];
             if (it == 0 && p.dST) {
                 // final-state term rowsum(dS_T o S_T) with S_T = diag(gm) S_prev + diag(cf) Kt^T Vh
+                const float* Sprev = p.saved + (((size_t)bh * NC + c) * DK + r) * DV + hf * HV;
                 float f = 0.0f;
 #pragma unroll
-                for (int qd = 0; qd < DV / 32; ++qd) {
+                for (int qd = 0; qd < HV / 32; ++qd) {
                     float v[32];
-                    tmem_ld32(tmem + lb + K::COL_DV + 32 * qd, v);
+                    tmem_ld32_split<HV>(tmem + lb + K::COL_DV + 32 * qd, v);
                     tmem_ld_wait();
-                    if (row) {
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            const int j = 32 * qd + e;
-                            f = fmaf(R[j], fmaf(gmv, Sprev[j], cfv * v[e]), f);  // R = dS_T here
-                        }
+                    for (int e = 0; e < 32; ++e) {
+                        const int j = 32 * qd + e;
+                        f = fmaf(R[j], fmaf(gmv, Sprev[j], cfv * v[e]), f);  // R = dS_T here
                     }
                 }
-                if (row) sm.fin[r] = f;
+                f += __shfl_xor_sync(0xffffffffu, f, 16);
+                if (hf == 0) sm.fin[r] = f;
             }
-            if (row) {
-                // R_hat = diag(cf) R  (S_hat is written by the gate warps)
+            // R_hat = diag(cf) R  (S_hat is written by the gate warps)
 #pragma unroll
-                for (int jg = 0; jg < DV / 8; ++jg) {
-                    float xr[8];
+            for (int jg = 0; jg < HV / 8; ++jg) {
+                float xr[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) xr[e] = R[8 * jg + e] * cfv;
-                    *reinterpret_cast<uint4*>(sm.u.op.rhat + off_rc(r, 8 * jg)) = pack8(xr);
-                }
+                for (int e = 0; e < 8; ++e) xr[e] = R[8 * jg + e] * cfv;
+                *reinterpret_cast<uint4*>(sm.u.op.rhat + off_rc(r, hf * HV + 8 * jg)) = pack8(xr);
             }
             // R <- diag(e^{b_last}) R + diag(e^m) Qt^T dO
 #pragma unroll
-            for (int qd = 0; qd < DV / 32; ++qd) {
+            for (int qd = 0; qd < HV / 32; ++qd) {
                 float v[32];
-                tmem_ld32(tmem + lb + K::COL_DR + 32 * qd, v);
+                tmem_ld32_split<HV>(tmem + lb + K::COL_DR + 32 * qd, v);
                 tmem_ld_wait();
 #pragma unroll
                 for (int e = 0; e < 32; ++e) R[32 * qd + e] = fmaf(gmv, R[32 * qd + e], emv * v[e]);
@@ -567,17 +563,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             tc_fence_after();
             // dV -> dv = beta dvhat, dbeta = v dvhat (row s = r)
             {
-                const bool st = row && c * C + r < T;
+                const bool st = c * C + r < T;
                 const size_t o = ((size_t)bh * T + (size_t)c * C + r) * DV;
 #pragma unroll
-                for (int qd = 0; qd < DV / 32; ++qd) {
+                for (int qd = 0; qd < HV / 32; ++qd) {
                     float v[32];
-                    tmem_ld32(tmem + lb + K::COL_DV + 32 * qd, v);
+                    tmem_ld32_split<HV>(tmem + lb + K::COL_DV + 32 * qd, v);
                     tmem_ld_wait();
                     if (st) {
 #pragma unroll
                         for (int h4 = 0; h4 < 4; ++h4) {
-                            const int jg = qd * 4 + h4;
+                            const int jg = (hf * HV + 32 * qd) / 8 + h4;
                             float v8[8], b8[8], ov[8], ob[8];
                             unpack8(*reinterpret_cast<const uint4*>(sm.raw + K::OFF_V + off_raw(r, jg)), v8);
                             unpack8(*reinterpret_cast<const uint4*>(sm.raw + K::OFF_B + off_raw(r, jg)), b8);
@@ -596,17 +592,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             if (it > 0 && !mbar_wait(&sm.post_done, (it - 1) & 1, fail, kWaitLimit)) break;
 #pragma unroll
             for (int which = 0; which < 2; ++which) {
-                float v[64];
-                const uint32_t col = which == 0 ? K::COL_DQ : K::COL_DK;
-                tmem_ld32(tmem + lb + col, v);
-                tmem_ld32(tmem + lb + col + 32, v + 32);
+                float v[32];
+                tmem_ld32_split<32>(tmem + lb + (which == 0 ? K::COL_DQ : K::COL_DK), v);
                 tmem_ld_wait();
-                if (row) {
-                    float4* dst = reinterpret_cast<float4*>(which == 0 ? &sm.u.st.dqs[r][0] : &sm.u.st.dks[r][0]);
+                float4* dst = reinterpret_cast<float4*>(which == 0 ? &sm.u.st.dqs[r][32 * hf] : &sm.u.st.dks[r][32 * hf]);
 #pragma unroll
-                    for (int e4 = 0; e4 < 16; ++e4)
-                        dst[e4] = make_float4(v[4 * e4], v[4 * e4 + 1], v[4 * e4 + 2], v[4 * e4 + 3]);
-                }
+                for (int e4 = 0; e4 < 8; ++e4)
+                    dst[e4] = make_float4(v[4 * e4], v[4 * e4 + 1], v[4 * e4 + 2], v[4 * e4 + 3]);
             }
             tc_fence_before();
             __syncwarp();
@@ -615,10 +607,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 mbar_arrive(&sm.tm2_free);
             }
         }
-        if (!*fail && row && p.dS0) {
-            float4* dst = reinterpret_cast<float4*>(p.dS0 + ((size_t)bh * DK + r) * DV);
+        if (!*fail && p.dS0) {
+            float4* dst = reinterpret_cast<float4*>(p.dS0 + ((size_t)bh * DK + r) * DV + hf * HV);
 #pragma unroll
-            for (int j4 = 0; j4 < DV / 4; ++j4)
+            for (int j4 = 0; j4 < HV / 4; ++j4)
                 dst[j4] = make_float4(R[4 * j4], R[4 * j4 + 1], R[4 * j4 + 2], R[4 * j4 + 3]);
         }
     }
