@@ -214,10 +214,18 @@ def time_steps(fn, K, W, flush=None, barrier=None):
 
 
 # ------------------------------------------------------------ workloads
+def fwd_workspace(rdm, x, dev):
+    """Scratch that lets the forward cut sequences into segments (allocated
+    once, outside the timed region); False when the forward needs none."""
+    n = rdm.rdm_ddts_fwd_workspace_size(*(x[k] for k in SEQ))
+    return torch.empty(n, dtype=torch.uint8, device=dev) if n else False
+
+
 def run_headline(rdm, w, K, W, dev, flush, barrier, pk, rank):
     x = draw_workload(w, device=dev, seed=w.seed + 1000 * rank)
     o = torch.empty(w.B, w.H, w.T, w.dv, dtype=torch.bfloat16, device=dev)
-    fn = lambda: rdm.rdm_ddts_fwd(*(x[n] for n in SEQ), x["S0"], o)
+    wsf = fwd_workspace(rdm, x, dev)
+    fn = lambda: rdm.rdm_ddts_fwd(*(x[n] for n in SEQ), x["S0"], o, workspace=wsf)
     with ClockSampler(dev) as clk:
         times = time_steps(fn, K, W, flush, barrier)
     status = rdm.rdm_ddts_sync_status()
@@ -231,7 +239,7 @@ def run_headline(rdm, w, K, W, dev, flush, barrier, pk, rank):
     def e2e_step():
         for n in SEQ:
             dx[n].copy_(hx[n], non_blocking=True)
-        rdm.rdm_ddts_fwd(*(dx[n] for n in SEQ), None, o)
+        rdm.rdm_ddts_fwd(*(dx[n] for n in SEQ), None, o, workspace=wsf)
         ho.copy_(o, non_blocking=True)
 
     e2e_times = time_steps(e2e_step, max(3, min(K, 10)), 2, None, barrier)
@@ -247,14 +255,16 @@ def run_extras(rdm, dev, pk, K):
     x = draw_workload(w, device=dev)
     o = torch.empty(w.B, w.H, w.T, w.dv, dtype=torch.bfloat16, device=dev)
     ST = torch.empty(w.B, w.H, w.dk, w.dv, device=dev)
-    t = time_steps(lambda: rdm.rdm_ddts_fwd(*(x[n] for n in SEQ), x["S0"], o, ST), max(3, K // 2), 2)
+    wsf = fwd_workspace(rdm, x, dev)
+    t = time_steps(lambda: rdm.rdm_ddts_fwd(*(x[n] for n in SEQ), x["S0"], o, ST, workspace=wsf),
+                   max(3, K // 2), 2)
     ms = statistics.mean(t)
     out["long_context_fwd"] = {
         "workload": w.name, "value": w.B * w.T / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
         "gpu_launches_per_step": 1,
         "roofline": roofline(fwd_bytes(w, True), chunk_flops_fwd(w), ms, pk,
                              ncu_traffic("tc_fwd_kernel", ["tc_fwd.cu"], 2))}
-    del x, o, ST
+    del x, o, ST, wsf
     # training forward + backward (forward saves chunk states for the backward)
     w = WORKLOADS[3]
     x = draw_workload(w, device=dev)
@@ -266,7 +276,8 @@ def run_extras(rdm, dev, pk, K):
     grads["dS0"] = torch.empty_like(x["S0"])
     ws_n = rdm.rdm_ddts_bwd_workspace_size(*(x[n] for n in SEQ), x["S0"], x["dO"], None, saved)
     ws = torch.empty(max(ws_n, 1), dtype=torch.uint8, device=dev)
-    fwd = lambda: rdm.rdm_ddts_fwd(*(x[n] for n in SEQ), x["S0"], o, None, saved)
+    wsf = fwd_workspace(rdm, x, dev)
+    fwd = lambda: rdm.rdm_ddts_fwd(*(x[n] for n in SEQ), x["S0"], o, None, saved, workspace=wsf)
     bwd = lambda: rdm.rdm_ddts_bwd(*(x[n] for n in SEQ), x["S0"], x["dO"], None, saved,
                                    grads=grads, workspace=ws)
     Kb = max(3, K // 4)
@@ -286,7 +297,7 @@ def run_extras(rdm, dev, pk, K):
                                  ncu_traffic("tc_bwd_kernel", ["tc_bwd.cu"], 3)),
         "roofline_step": roofline(fb + bwd_bytes(w), chunk_flops_fwd(w) + chunk_flops_bwd(w),
                                   msf + msb, pk, None)}
-    del x, o, saved, grads, ws
+    del x, o, saved, grads, ws, wsf
     # batched decode, 1024 steps captured in one CUDA graph
     w = WORKLOADS[4]
     steps = w.T

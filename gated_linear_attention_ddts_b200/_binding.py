@@ -27,7 +27,8 @@ class FwdArgs(ctypes.Structure):
     _fields_ = [("B", _I), ("H", _I), ("T", _I), ("dk", _I), ("dv", _I), ("chunk", _I),
                 ("dtype", _I), ("impl", _I),
                 ("q", _VP), ("k", _VP), ("v", _VP), ("g", _VP), ("tau", _VP), ("beta", _VP),
-                ("S0", _VP), ("o", _VP), ("ST", _VP), ("saved_states", _VP)]
+                ("S0", _VP), ("o", _VP), ("ST", _VP), ("saved_states", _VP),
+                ("workspace", _VP), ("workspace_bytes", ctypes.c_size_t)]
 
 
 class BwdArgs(ctypes.Structure):
@@ -48,7 +49,7 @@ class RdmError(RuntimeError):
 
 _lib = None
 
-EXPORTS = ["rdm_ddts_fwd", "rdm_ddts_saved_states_size", "rdm_ddts_bwd",
+EXPORTS = ["rdm_ddts_fwd", "rdm_ddts_fwd_workspace_size", "rdm_ddts_saved_states_size", "rdm_ddts_bwd",
            "rdm_ddts_bwd_workspace_size", "rdm_ddts_bwd_noalloc", "rdm_ddts_decode_step", "rdm_ddts_sync_status",
            "rdm_status_string", "rdm_ddts_version"]
 
@@ -63,6 +64,8 @@ def load():
         lib = ctypes.CDLL(LIB_PATH)
         lib.rdm_ddts_fwd.argtypes = [ctypes.POINTER(FwdArgs), _VP]
         lib.rdm_ddts_fwd.restype = _I
+        lib.rdm_ddts_fwd_workspace_size.argtypes = [ctypes.POINTER(FwdArgs)]
+        lib.rdm_ddts_fwd_workspace_size.restype = ctypes.c_size_t
         lib.rdm_ddts_saved_states_size.argtypes = [_I] * 6
         lib.rdm_ddts_saved_states_size.restype = ctypes.c_size_t
         lib.rdm_ddts_bwd.argtypes = [ctypes.POINTER(BwdArgs), _VP]
@@ -120,19 +123,42 @@ def rdm_ddts_saved_states_size(B, H, T, dk, dv, chunk=0) -> int:
     return int(load().rdm_ddts_saved_states_size(B, H, T, dk, dv, chunk))
 
 
+def _fwd_args(q, k, v, g, tau, beta, S0, o, ST, saved_states, ws, ws_bytes, chunk, impl):
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    return FwdArgs(B, H, T, dk, dv, chunk, _dtype_code(q), IMPL[impl],
+                   _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(tau), _ptr(beta), _ptr(S0), _ptr(o),
+                   _ptr(ST), _ptr(saved_states), _ptr(ws), ws_bytes)
+
+
+def rdm_ddts_fwd_workspace_size(q, k, v, g, tau, beta, *, chunk=0, impl="auto") -> int:
+    a = _fwd_args(q, k, v, g, tau, beta, None, None, None, None, None, 0, chunk, impl)
+    n = load().rdm_ddts_fwd_workspace_size(ctypes.byref(a))
+    if n == ctypes.c_size_t(-1).value:
+        raise RdmError(RDM_ERR_INVALID_ARG, "rdm_ddts_fwd_workspace_size")
+    return int(n)
+
+
 def rdm_ddts_fwd(q, k, v, g, tau, beta, S0=None, o=None, ST=None, saved_states=None, *,
-                 chunk=0, impl="auto", return_state=False, stream=None):
+                 workspace=None, chunk=0, impl="auto", return_state=False, stream=None):
     """Forward over [B,H,T,D] sequences.  Allocates o (and S_T when
-    return_state) with torch if not given.  Returns (o, S_T or None)."""
+    return_state) with torch if not given, and the sequence-segment workspace
+    when none is passed (workspace=False runs without one).  Returns
+    (o, S_T or None)."""
     B, H, T, dk = q.shape
     dv = v.shape[-1]
     if o is None:
         o = torch.empty(B, H, T, dv, dtype=q.dtype, device=q.device)
     if ST is None and return_state:
         ST = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device)
-    a = FwdArgs(B, H, T, dk, dv, chunk, _dtype_code(q), IMPL[impl],
-                _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(tau), _ptr(beta), _ptr(S0), _ptr(o),
-                _ptr(ST), _ptr(saved_states))
+    if workspace is None:
+        need = rdm_ddts_fwd_workspace_size(q, k, v, g, tau, beta, chunk=chunk, impl=impl)
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device) if need else None
+    elif workspace is False:
+        workspace = None
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    a = _fwd_args(q, k, v, g, tau, beta, S0, o, ST, saved_states, workspace, ws_bytes, chunk,
+                  impl)
     _check(load().rdm_ddts_fwd(ctypes.byref(a), _stream(stream)), "rdm_ddts_fwd")
     return o, ST
 

@@ -75,6 +75,18 @@ bool use_tc_bwd(const BwdParams& p, rdm_impl impl) {
     return tc_bwd_supported(p);
 }
 
+SeqParams fwd_params(const rdm_fwd_args* a) {
+    SeqParams p;
+    memset(&p, 0, sizeof(p));
+    p.B = a->B; p.H = a->H; p.T = a->T; p.dk = a->dk; p.dv = a->dv;
+    p.chunk = eff_chunk(a->chunk);
+    p.bf16 = a->dtype == RDM_BF16;
+    p.q = a->q; p.k = a->k; p.v = a->v; p.g = a->g; p.tau = a->tau; p.beta = a->beta;
+    p.S0 = a->S0; p.o = a->o; p.ST = a->ST; p.saved = a->saved_states;
+    p.ws = a->workspace; p.ws_bytes = a->workspace ? a->workspace_bytes : 0;
+    return p;
+}
+
 BwdParams bwd_params(const rdm_bwd_args* a) {
     BwdParams p;
     memset(&p, 0, sizeof(p));
@@ -108,7 +120,8 @@ rdm_status rdm_ddts_fwd(const rdm_fwd_args* a, rdm_stream_t stream) {
     rdm_status st = check_sizes(a->B, a->H, a->T, a->dk, a->dv, a->chunk, a->dtype, a->impl);
     if (st != RDM_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (!opt_aligned(a->S0) || !opt_aligned(a->ST) || !opt_aligned(a->saved_states))
+    if (!opt_aligned(a->S0) || !opt_aligned(a->ST) || !opt_aligned(a->saved_states) ||
+        !opt_aligned(a->workspace))
         return RDM_ERR_INVALID_ARG;
     if (a->T == 0) {
         if (a->impl == RDM_IMPL_TC && a->dtype != RDM_BF16) return RDM_ERR_UNSUPPORTED;
@@ -117,18 +130,21 @@ rdm_status rdm_ddts_fwd(const rdm_fwd_args* a, rdm_stream_t stream) {
     const void* in[] = {a->q, a->k, a->v, a->g, a->tau, a->beta, a->o};
     for (const void* p : in)
         if (!p || !aligned(p)) return RDM_ERR_INVALID_ARG;
-    SeqParams p;
-    memset(&p, 0, sizeof(p));
-    p.B = a->B; p.H = a->H; p.T = a->T; p.dk = a->dk; p.dv = a->dv;
-    p.chunk = eff_chunk(a->chunk);
-    p.bf16 = a->dtype == RDM_BF16;
-    p.q = a->q; p.k = a->k; p.v = a->v; p.g = a->g; p.tau = a->tau; p.beta = a->beta;
-    p.S0 = a->S0; p.o = a->o; p.ST = a->ST; p.saved = a->saved_states;
+    SeqParams p = fwd_params(a);
     p.err = status_word();
     if (!p.err) return RDM_ERR_CUDA;
     const bool tc = use_tc_fwd(p, a->impl);
     if (a->impl == RDM_IMPL_TC && !tc) return RDM_ERR_UNSUPPORTED;
     return from_cuda(tc ? launch_tc_fwd(p, s) : launch_simt_fwd(p, s));
+}
+
+size_t rdm_ddts_fwd_workspace_size(const rdm_fwd_args* a) {
+    if (!a) return (size_t)-1;
+    if (check_sizes(a->B, a->H, a->T, a->dk, a->dv, a->chunk, a->dtype, a->impl) != RDM_OK)
+        return (size_t)-1;
+    if (a->T == 0) return 0;
+    SeqParams p = fwd_params(a);
+    return use_tc_fwd(p, a->impl) ? tc_fwd_workspace(p) : 0;
 }
 
 size_t rdm_ddts_bwd_workspace_size(const rdm_bwd_args* a) {
@@ -210,6 +226,6 @@ const char* rdm_status_string(rdm_status s) {
     return "unknown status";
 }
 
-int rdm_ddts_version(void) { return 100; }
+int rdm_ddts_version(void) { return 200; }
 
 }  // extern "C"

@@ -14,6 +14,8 @@ struct SeqParams {
     void* o;
     float* ST;
     float* saved;        // [B,H,NC,dk,dv] chunk-start states, or null
+    void* ws;            // scratch for sequence segments, or null
+    size_t ws_bytes;
     unsigned* err;       // device status word
 };
 
@@ -52,6 +54,7 @@ cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s);
 
 // tensor-core (tcgen05) chunked path
 bool tc_fwd_supported(const SeqParams& p);
+size_t tc_fwd_workspace(const SeqParams& p);  // bytes that enable sequence segments
 cudaError_t launch_tc_fwd(const SeqParams& p, cudaStream_t s);
 bool tc_bwd_supported(const BwdParams& p);
 size_t tc_bwd_workspace(const BwdParams& p);

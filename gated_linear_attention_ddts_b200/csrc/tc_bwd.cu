@@ -680,7 +680,7 @@ cudaError_t launch_tc_bwd(const BwdParams& p, cudaStream_t s) {
     cudaError_t e;
     if (!saved) {
         // recompute the chunk-start states with the forward kernel
-        SeqParams f;
+        SeqParams f{};  // no workspace: one CTA per sequence
         f.B = p.B; f.H = p.H; f.T = p.T; f.dk = p.dk; f.dv = p.dv; f.chunk = p.chunk; f.bf16 = 1;
         f.q = p.q; f.k = p.k; f.v = p.v; f.g = p.g; f.tau = p.tau; f.beta = p.beta; f.S0 = p.S0;
         f.o = ws + w.states;

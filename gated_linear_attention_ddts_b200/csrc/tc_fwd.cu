@@ -16,15 +16,30 @@
 // chunk whose span is larger is processed as windows of 16 tokens, or of 1
 // token, each window being one pass of the same pipeline (exact for any decay).
 //
-// One CTA owns one (b,h) and a 64-wide slice of d_v.  Warp roles:
-//   warps 0-3  epilogue: A -> masked bf16 operand, state (fp32 registers),
-//              S_hat operand, o store (TMEM lanes = rows)
-//   warps 4-7  gates: TMA tiles -> log-decay scan, Qt, Kt, Vh operands (bf16)
-//   warp  8    TMA producer (q, k, g, tau, v, beta tiles, 128B-swizzled)
-//   warp  9    TMEM allocator and single-thread tcgen05.mma issuer
+// Sequence segments.  When the (b,h) x d_v-slice units do not fill the GPU,
+// each unit's chunks are cut into P contiguous segments, one CTA each.  The
+// state map of a segment is affine, S_out = diag(D) S_in + S_loc, with D the
+// product of its decays and S_loc its state from a zero start.  A segment
+// first runs the state recurrence alone from zero (no Qt, A or o) and
+// publishes (S_loc, log2 D) through global memory; it then folds the maps of
+// all earlier segments onto S_0 to obtain its true entry state and runs the
+// full forward over its chunks.  The last segment skips the first pass.  All
+// CTAs of such a launch are resident together (cooperative launch), and every
+// cross-CTA wait is bounded.
+//
+// One CTA owns one (b,h), a d_v slice of DVT columns and a segment.  Roles:
+//   warps 0-7   epilogue: A -> masked bf16 operand, state (fp32 registers),
+//               S_hat operand, o store (TMEM lanes = rows; the two warps of a
+//               sub-partition take different columns)
+//   warps 8-15  gates: TMA tiles -> log-decay scan, Qt, Kt, Vh operands (bf16)
+//   warp  16    TMA producer (q, k, g, tau, v, beta tiles, 128B-swizzled)
+//   warp  17    TMEM allocator and single-thread tcgen05.mma issuer
 // All hand-offs are mbarriers with bounded waits (a timeout sets the device
 // status word and the CTA exits cleanly).
 #include <cuda.h>
+
+#include <atomic>
+#include <chrono>
 
 #include "launch.h"
 #include "rdm_common.cuh"
@@ -34,11 +49,15 @@ namespace rdm {
 namespace {
 using namespace tc;
 
-constexpr int C = 64;                        // tokens per chunk (tile rows)
+constexpr int C = 64;          // tokens per chunk (tile rows)
+constexpr int kEpiWarps = 8;   // two per SM sub-partition
 constexpr int kGateWarps = 8;  // two per SM sub-partition
-constexpr int kThreads = 32 * (4 + kGateWarps + 2);
-constexpr int kEpiWarp0 = 0, kGateWarp0 = 4, kProdWarp = 4 + kGateWarps, kMmaWarp = 5 + kGateWarps;
-constexpr int kBarGate = 3;  // all gate warps
+constexpr int kThreads = 32 * (kEpiWarps + kGateWarps + 2);
+constexpr int kEpiWarp0 = 0, kGateWarp0 = kEpiWarps, kProdWarp = kEpiWarps + kGateWarps,
+              kMmaWarp = kProdWarp + 1;
+constexpr int kBarGate = 3;        // all gate warps
+constexpr int kBarEpi = 4;         // all epilogue warps
+constexpr int kMinSegChunks = 4;   // shortest segment worth a CTA of its own
 
 template <int DK, int DVT>
 struct Cfg {
@@ -54,6 +73,9 @@ struct Cfg {
     static constexpr int TMEM_COLS = (64 + 3 * DVT) <= 256 ? 256 : 512;
 };
 
+// info[] of an operand slot
+enum { kInfoChunk, kInfoW0, kInfoW1, kInfoLast, kInfoPhase, kInfoP1Last, kInfoN };
+
 template <int DK, int DVT>
 struct alignas(1024) FwdSmem {
     using K = Cfg<DK, DVT>;
@@ -64,7 +86,7 @@ struct alignas(1024) FwdSmem {
     uint8_t abf[C * C * 2];
     uint8_t shat[DK * DVT * 2];
     float em[K::NB][DK], cf[K::NB][DK], gm[K::NB][DK];
-    int info[K::NB][4];  // chunk, w0, w1, last
+    int info[K::NB][kInfoN];
     uint64_t raw_full[K::NS], raw_empty[K::NS], ops_full[K::NB], ops_empty[K::NB];
     uint64_t mma1_done, as_free, abf_full, mmao_done[2], o_free[2];
     int need16[2], need1[2];
@@ -72,9 +94,21 @@ struct alignas(1024) FwdSmem {
     int fail;
 };
 
+// Segment exchange area (global): per (segment < P-1, unit) the local state
+// [DK][DVT] and log2 of the decay product per channel; per (segment, unit) a
+// flag that holds `epoch` once those are written.
+struct SegArgs {
+    int P;
+    unsigned epoch;
+    float* st;
+    float* ld;
+    unsigned* flag;
+};
+
 struct FwdKernelArgs {
     CUtensorMap mq, mk, mg, mt, mv, mb;
     SeqParams p;
+    SegArgs seg;
 };
 
 template <int DK, int DVT>
@@ -87,10 +121,21 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
     FwdSmem<DK, DVT>& sm = *reinterpret_cast<FwdSmem<DK, DVT>*>(
         smem_dyn + ((1024u - (smem_u32(smem_dyn) & 1023u)) & 1023u));
     const SeqParams& p = A.p;
+    const SegArgs& sg = A.seg;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int NJ = p.dv / DVT;
-    const int bh = blockIdx.x / NJ, j0 = (blockIdx.x % NJ) * DVT;
+    const int units = p.B * p.H * NJ;
+    const int unit = blockIdx.x % units, seg = blockIdx.x / units;
+    const int bh = unit / NJ, j0 = (unit % NJ) * DVT;
     const int T = p.T, NC = (T + C - 1) / C;
+    const int P = sg.P;
+    const int c0 = (int)((long long)seg * NC / P), c1 = (int)((long long)(seg + 1) * NC / P);
+    const int nseg = c1 - c0;
+    const bool has_p1 = seg < P - 1;        // runs the state-only first pass
+    const int nL = (has_p1 ? 2 : 1) * nseg;  // chunk passes
+    // pass li: phase 1 (state only) for the first nseg passes when has_p1, else phase 2
+    auto pass_chunk = [&](int li) { return c0 + (li < nseg ? li : li - nseg); };
+    auto pass_p2 = [&](int li) { return !has_p1 || li >= nseg; };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
@@ -99,15 +144,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
         }
         for (int b = 0; b < NB; ++b) {
             mbar_init(&sm.ops_full[b], kGateWarps);
-            mbar_init(&sm.ops_empty[b], 1 + 4);
+            mbar_init(&sm.ops_empty[b], 1 + kEpiWarps);
         }
         mbar_init(&sm.mma1_done, 1);
-        mbar_init(&sm.as_free, 4);
-        mbar_init(&sm.abf_full, 4);
+        mbar_init(&sm.as_free, kEpiWarps);
+        mbar_init(&sm.abf_full, kEpiWarps);
         mbar_init(&sm.mmao_done[0], 1);
         mbar_init(&sm.mmao_done[1], 1);
-        mbar_init(&sm.o_free[0], 4);
-        mbar_init(&sm.o_free[1], 4);
+        mbar_init(&sm.o_free[0], kEpiWarps);
+        mbar_init(&sm.o_free[1], kEpiWarps);
         sm.need16[0] = sm.need16[1] = sm.need1[0] = sm.need1[1] = 0;
         sm.fail = 0;
         fence_mbar_init();
@@ -130,14 +175,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             int issued = 0;
-            for (int c = 0; c < NC; ++c) {
-                const int st = c % NS;
-                if (c >= NS && !mbar_wait(&sm.raw_empty[st], ((c / NS) - 1) & 1, fail, kWaitLimit))
+            for (int li = 0; li < nL; ++li) {
+                const int st = li % NS, c = pass_chunk(li);
+                const bool p2 = pass_p2(li);
+                if (li >= NS && !mbar_wait(&sm.raw_empty[st], ((li / NS) - 1) & 1, fail, kWaitLimit))
                     break;
-                mbar_expect_tx(&sm.raw_full[st], K::RAW);
+                // the state-only pass does not read q
+                mbar_expect_tx(&sm.raw_full[st], K::RAW - (p2 ? 0 : KB * kBox));
                 uint8_t* raw = sm.raw[st];
                 for (int kb = 0; kb < KB; ++kb) {
-                    tma_load_3d(raw + (0 * KB + kb) * kBox, &A.mq, &sm.raw_full[st], 64 * kb, c * C, bh);
+                    if (p2)
+                        tma_load_3d(raw + (0 * KB + kb) * kBox, &A.mq, &sm.raw_full[st], 64 * kb, c * C, bh);
                     tma_load_3d(raw + (1 * KB + kb) * kBox, &A.mk, &sm.raw_full[st], 64 * kb, c * C, bh);
                     tma_load_3d(raw + (2 * KB + kb) * kBox, &A.mg, &sm.raw_full[st], 64 * kb, c * C, bh);
                     tma_load_3d(raw + (3 * KB + kb) * kBox, &A.mt, &sm.raw_full[st], 64 * kb, c * C, bh);
@@ -149,8 +197,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                 ++issued;
             }
             // never leave the CTA with copies in flight
-            for (int c = issued - NS < 0 ? 0 : issued - NS; c < issued; ++c)
-                drain_wait(&sm.raw_full[c % NS], (c / NS) & 1);
+            for (int li = issued - NS < 0 ? 0 : issued - NS; li < issued; ++li)
+                drain_wait(&sm.raw_full[li % NS], (li / NS) & 1);
         }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
@@ -159,47 +207,53 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             constexpr uint32_t id1 = idesc_bf16(64, 64, 0, 0);    // A  = Qt Kt^T
             constexpr uint32_t idS = idesc_bf16(DK, DVT, 1, 1);   // dS = Kt^T Vh
             constexpr uint32_t idO = idesc_bf16(64, DVT, 0, 1);   // O  = A Vh + Qt S_hat
-            int item = 0, n1 = 0, nO = 0;
+            int item = 0, n1 = 0, io = 0;  // io counts the items that produce o
             while (true) {
                 const int ob = item % NB;
                 if (!mbar_wait(&sm.ops_full[ob], (item / NB) & 1, fail, kWaitLimit)) break;
-                const int last = sm.info[ob][3];
+                const int last = sm.info[ob][kInfoLast];
+                const bool p2 = sm.info[ob][kInfoPhase] == 2;
                 if (item > 0 && !mbar_wait(&sm.as_free, (item - 1) & 1, fail, kWaitLimit)) break;
                 tc_fence_after();
-                const uint32_t q = smem_u32(sm.qt[ob]), k = smem_u32(sm.kt[ob]);
-                const uint32_t v = smem_u32(sm.vh[ob]);
+                const uint32_t q = smem_u32(sm.qt[ob]) >> 4, k = smem_u32(sm.kt[ob]) >> 4;
+                const uint32_t v = smem_u32(sm.vh[ob]) >> 4;
+                if (p2) {
 #pragma unroll
-                for (int ks = 0; ks < DK / 16; ++ks)
-                    mma_bf16(tA, sdesc(q + ks * 2 * kQK, kQK, 128), sdesc(k + ks * 2 * kQK, kQK, 128),
-                             id1, ks > 0);
+                    for (int ks = 0; ks < DK / 16; ++ks)
+                        mma_bf16_w(tA, q + sd_lo(ks * 2 * kQK, kQK), sd_hi(128),
+                                   k + sd_lo(ks * 2 * kQK, kQK), sd_hi(128), id1, ks > 0);
+                }
 #pragma unroll
                 for (int ks = 0; ks < C / 16; ++ks)
-                    mma_bf16(tS, sdesc(k + ks * 256, 128, kQK), sdesc(v + ks * 256, 128, 1024), idS,
-                             ks > 0);
+                    mma_bf16_w(tS, k + sd_lo(ks * 256, 128), sd_hi(kQK), v + sd_lo(ks * 256, 128),
+                               sd_hi(1024), idS, ks > 0);
                 mma_commit(&sm.mma1_done);
                 ++n1;
-                if (!mbar_wait(&sm.abf_full, item & 1, fail, kWaitLimit)) break;
-                const int obuf = item & 1;
-                if (item >= 2 && !mbar_wait(&sm.o_free[obuf], ((item >> 1) - 1) & 1, fail, kWaitLimit)) break;
-                tc_fence_after();
-                const uint32_t a = smem_u32(sm.abf), sh = smem_u32(sm.shat);
+                if (p2) {
+                    if (!mbar_wait(&sm.abf_full, io & 1, fail, kWaitLimit)) break;
+                    const int obuf = io & 1;
+                    if (io >= 2 && !mbar_wait(&sm.o_free[obuf], ((io >> 1) - 1) & 1, fail, kWaitLimit))
+                        break;
+                    tc_fence_after();
+                    const uint32_t a = smem_u32(sm.abf) >> 4, sh = smem_u32(sm.shat) >> 4;
 #pragma unroll
-                for (int ks = 0; ks < C / 16; ++ks)
-                    mma_bf16(tO + obuf * DVT, sdesc(a + ks * 2048, 1024, 128),
-                             sdesc(v + ks * 256, 128, 1024), idO, ks > 0);
+                    for (int ks = 0; ks < C / 16; ++ks)
+                        mma_bf16_w(tO + obuf * DVT, a + sd_lo(ks * 2048, 1024), sd_hi(128),
+                                   v + sd_lo(ks * 256, 128), sd_hi(1024), idO, ks > 0);
 #pragma unroll
-                for (int ks = 0; ks < DK / 16; ++ks)
-                    mma_bf16(tO + obuf * DVT, sdesc(q + ks * 2 * kQK, kQK, 128),
-                             sdesc(sh + ks * 256, 128, DK * 16), idO, 1);
-                mma_commit(&sm.mmao_done[obuf]);
+                    for (int ks = 0; ks < DK / 16; ++ks)
+                        mma_bf16_w(tO + obuf * DVT, q + sd_lo(ks * 2 * kQK, kQK), sd_hi(128),
+                                   sh + sd_lo(ks * 256, 128), sd_hi(DK * 16), idO, 1);
+                    mma_commit(&sm.mmao_done[obuf]);
+                    ++io;
+                }
                 mma_commit(&sm.ops_empty[ob]);
-                ++nO;
                 if (last) break;
                 ++item;
             }
             // let issued MMAs finish before TMEM is released
             if (n1 > 0) drain_wait(&sm.mma1_done, (n1 - 1) & 1);
-            if (nO > 0) drain_wait(&sm.mmao_done[(nO - 1) & 1], ((nO - 1) >> 1) & 1);
+            if (io > 0) drain_wait(&sm.mmao_done[(io - 1) & 1], ((io - 1) >> 1) & 1);
         }
         __syncwarp();
     } else if (warp >= kGateWarp0) {
@@ -213,14 +267,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
         constexpr int G = K::G, GW = G / kGateWarps, NSW = 32 / GW, SEGT = C / NSW;
         constexpr int VG = DVT / 8, TPG = 32 * kGateWarps / VG, VIT = C / TPG;
         const int gw = warp - kGateWarp0, gt = gw * 32 + lane;
-        const int cgl = lane % GW, seg = lane / GW;
+        const int cgl = lane % GW, seg_l = lane / GW;
         const int cg = gw * GW + cgl;
-        const int tb = seg * SEGT;  // first token of my segment
+        const int tb = seg_l * SEGT;  // first token of my segment
         const uint32_t full = 0xffffffffu;
         int item = 0;
-        for (int c = 0; c < NC; ++c) {
-            const int st = c % NS;
-            if (!mbar_wait(&sm.raw_full[st], (c / NS) & 1, fail, kWaitLimit)) break;
+        for (int li = 0; li < nL; ++li) {
+            const int st = li % NS, c = pass_chunk(li);
+            const bool p2 = pass_p2(li);
+            if (!mbar_wait(&sm.raw_full[st], (li / NS) & 1, fail, kWaitLimit)) break;
             const uint8_t* raw = sm.raw[st];
             const int nval = min(C, T - c * C);
             float b[SEGT][8], bf[8], bl[8];
@@ -272,16 +327,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
 #pragma unroll
                 for (int e = 0; e < 8; ++e) span = fmaxf(span, bf[e] - bl[e]);
                 if (tb >= nval) span = 0.0f;
-                if (__any_sync(full, !(span <= kSpanMax)) && lane == 0) *flag = c + 1;
+                if (__any_sync(full, !(span <= kSpanMax)) && lane == 0) *flag = li + 1;
                 named_bar(kBarGate, 32 * kGateWarps);
-                return *flag == c + 1;
+                return *flag == li + 1;
             };
             int W = C;
             scan(C);
-            if (too_wide(&sm.need16[c & 1])) {
+            if (too_wide(&sm.need16[li & 1])) {
                 W = 16;
                 scan(16);
-                if (too_wide(&sm.need1[c & 1])) {
+                if (too_wide(&sm.need1[li & 1])) {
                     W = 1;
                     scan(1);
                 }
@@ -302,10 +357,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             };
             auto publish = [&](int ob, int w0, int w1) {
                 if (gt == 0) {
-                    sm.info[ob][0] = c;
-                    sm.info[ob][1] = w0;
-                    sm.info[ob][2] = w1;
-                    sm.info[ob][3] = (c == NC - 1) && (w1 == nval);
+                    const bool end = (c == c1 - 1) && (w1 == nval);
+                    sm.info[ob][kInfoChunk] = c;
+                    sm.info[ob][kInfoW0] = w0;
+                    sm.info[ob][kInfoW1] = w1;
+                    sm.info[ob][kInfoLast] = p2 && end;
+                    sm.info[ob][kInfoPhase] = p2 ? 2 : 1;
+                    sm.info[ob][kInfoP1Last] = !p2 && end;
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
@@ -323,19 +381,29 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
 #pragma unroll
                 for (int u = 0; u < SEGT; ++u) {
                     const int t = tb + u;
-                    float q8[8], k8[8], g8[8], t8[8], oq[8], ok[8];
-                    unpack8(*reinterpret_cast<const uint4*>(raw + 0 * KB * kBox + off_raw(t, cg)), q8);
+                    float k8[8], g8[8], t8[8], ok[8];
                     unpack8(*reinterpret_cast<const uint4*>(raw + 1 * KB * kBox + off_raw(t, cg)), k8);
                     unpack8(*reinterpret_cast<const uint4*>(raw + 2 * KB * kBox + off_raw(t, cg)), g8);
                     unpack8(*reinterpret_cast<const uint4*>(raw + 3 * KB * kBox + off_raw(t, cg)), t8);
+                    if (p2) {
+                        float q8[8], oq[8];
+                        unpack8(*reinterpret_cast<const uint4*>(raw + 0 * KB * kBox + off_raw(t, cg)), q8);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const float d = fmaf(b[u][e], kLog2e, -mL[e]);
-                        const float lah = t8[e] == 0.0f ? 0.0f : t8[e] * lg2_fast(g8[e]);
-                        oq[e] = q8[e] * ex2_fast(d);
-                        ok[e] = k8[e] * ex2_fast(lah - d);
+                        for (int e = 0; e < 8; ++e) {
+                            const float d = fmaf(b[u][e], kLog2e, -mL[e]);
+                            const float lah = t8[e] == 0.0f ? 0.0f : t8[e] * lg2_fast(g8[e]);
+                            oq[e] = q8[e] * ex2_fast(d);
+                            ok[e] = k8[e] * ex2_fast(lah - d);
+                        }
+                        *reinterpret_cast<uint4*>(sm.qt[ob] + off_qk(t, cg * 8)) = pack8(oq);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const float d = fmaf(b[u][e], kLog2e, -mL[e]);
+                            const float lah = t8[e] == 0.0f ? 0.0f : t8[e] * lg2_fast(g8[e]);
+                            ok[e] = k8[e] * ex2_fast(lah - d);
+                        }
                     }
-                    *reinterpret_cast<uint4*>(sm.qt[ob] + off_qk(t, cg * 8)) = pack8(oq);
                     *reinterpret_cast<uint4*>(sm.kt[ob] + off_qk(t, cg * 8)) = pack8(ok);
                 }
                 if (tb == 0) {
@@ -375,7 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                             const float m = W == 1 ? b[u][e] : 0.5f * (bf[e] + bl[e]);
                             const float d = (b[u][e] - m) * kLog2e;
                             const float lah = t8[e] == 0.0f ? 0.0f : t8[e] * lg2_fast(g8[e]);
-                            oq[e] = in ? q8[e] * ex2_fast(d) : 0.0f;
+                            oq[e] = (in && p2) ? q8[e] * ex2_fast(d) : 0.0f;
                             ok[e] = in ? k8[e] * ex2_fast(lah - d) : 0.0f;
                             if (t == w0) {
                                 sm.em[ob][cg * 8 + e] = ex2_fast(m * kLog2e);
@@ -398,33 +466,96 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        const int ew = warp - kEpiWarp0;
-        const bool rowA = lane < 16;                      // valid rows of A and O (M = 64)
-        const int tA = 16 * ew + lane;
-        const bool rowS = (DK == 128) || lane < 16;        // valid state rows (M = DK)
-        const int iS = (DK == 128) ? 32 * ew + lane : 16 * ew + lane;
-        const uint32_t lb = (uint32_t)(32 * ew) << 16;
-        float S[DVT];
+        // A and O are M = 64 accumulators (TMEM lanes 0-15 of each sub-partition):
+        // the split load gives row tA to two threads, lane >> 4 (hf) picking the
+        // half of the columns, and the two warps of a sub-partition (eh) take
+        // different quarters.  The state is M = DK: split the same way for
+        // DK = 64; one row per thread (all 32 lanes), half the columns per warp,
+        // for DK = 128.
+        constexpr bool kSplitS = DK == 64;
+        constexpr int SC = kSplitS ? DVT / 4 : DVT / 2;  // state columns per thread
+        constexpr int OC = DVT / 4;                      // o columns per thread
+        const int ew = warp - kEpiWarp0, sub = ew & 3, eh = ew >> 2;
+        const int hf = lane >> 4;
+        const int tA = 16 * sub + (lane & 15);
+        const int iS = kSplitS ? tA : 32 * sub + lane;
+        const int oc0 = hf * (DVT / 2) + eh * OC;  // first o column of this thread
+        const int sc0 = kSplitS ? oc0 : eh * SC;   // first state column of this thread
+        const uint32_t lb = (uint32_t)(32 * sub) << 16;
+        // SC / OC columns of this thread from a DVT-wide accumulator at `col`
+        auto ld_cols = [&](uint32_t col, float* v, bool state) {
+            if (state && !kSplitS) {
+                if constexpr (SC == 32) tmem_ld32(tmem + lb + col + eh * SC, v);
+                else tmem_ld16(tmem + lb + col + eh * SC, v);
+            } else {
+                if constexpr (OC == 32) tmem_ld32_split<DVT / 2>(tmem + lb + col + eh * OC, v);
+                else tmem_ld16_split<DVT / 2>(tmem + lb + col + eh * OC, v);
+            }
+            tmem_ld_wait();
+        };
+        float S[SC];
+        auto load_s0 = [&]() {
 #pragma unroll
-        for (int j = 0; j < DVT; ++j)
-            S[j] = (rowS && p.S0) ? p.S0[((size_t)bh * DK + iS) * p.dv + j0 + j] : 0.0f;
-        // o rows [w0, w1) of chunk c from the O buffer of item `it`
-        auto store_o = [&](int it, int c, int w0, int w1) -> bool {
-            const int obuf = it & 1;
-            if (!mbar_wait(&sm.mmao_done[obuf], (it >> 1) & 1, fail, kWaitLimit)) return false;
+            for (int j = 0; j < SC; ++j)
+                S[j] = p.S0 ? p.S0[((size_t)bh * DK + iS) * p.dv + j0 + sc0 + j] : 0.0f;
+        };
+        // entry state of this segment: S_0 carried through the maps of all
+        // earlier segments, S <- diag(D_s) S + S_loc_s
+        auto fold_earlier = [&]() -> bool {
+            if (threadIdx.x == 0) {
+                const long long t0 = clock64();
+                for (int s = 0; s < seg && !*fail; ++s)
+                    while (ld_acquire_gpu(&sg.flag[s * units + unit]) != sg.epoch)
+                        if (clock64() - t0 > kWaitLimit) {
+                            *fail = 1;
+                            break;
+                        }
+            }
+            named_bar(kBarEpi, 32 * kEpiWarps);
+            if (*fail) return false;
+            load_s0();
+            for (int s = 0; s < seg; ++s) {
+                const size_t u = (size_t)s * units + unit;
+                const float d = ex2_fast(__ldcg(&sg.ld[u * DK + iS]));
+                const float4* src = reinterpret_cast<const float4*>(sg.st + (u * DK + iS) * DVT + sc0);
+#pragma unroll
+                for (int j4 = 0; j4 < SC / 4; ++j4) {
+                    const float4 x = __ldcg(src + j4);
+                    S[4 * j4] = fmaf(d, S[4 * j4], x.x);
+                    S[4 * j4 + 1] = fmaf(d, S[4 * j4 + 1], x.y);
+                    S[4 * j4 + 2] = fmaf(d, S[4 * j4 + 2], x.z);
+                    S[4 * j4 + 3] = fmaf(d, S[4 * j4 + 3], x.w);
+                }
+            }
+            return true;
+        };
+        // publish this segment's map (S_loc in S, log2 D in ld2)
+        auto publish_segment = [&](float ld2) {
+            const size_t u = (size_t)seg * units + unit;
+            float4* dst = reinterpret_cast<float4*>(sg.st + (u * DK + iS) * DVT + sc0);
+#pragma unroll
+            for (int j4 = 0; j4 < SC / 4; ++j4)
+                dst[j4] = make_float4(S[4 * j4], S[4 * j4 + 1], S[4 * j4 + 2], S[4 * j4 + 3]);
+            if (sc0 == 0) sg.ld[u * DK + iS] = ld2;
+            __threadfence();
+            named_bar(kBarEpi, 32 * kEpiWarps);
+            if (threadIdx.x == 0) st_release_gpu(&sg.flag[u], sg.epoch);
+        };
+        // o rows [w0, w1) of chunk c from the O buffer of o-item `io`
+        auto store_o = [&](int io, int c, int w0, int w1) -> bool {
+            const int obuf = io & 1;
+            if (!mbar_wait(&sm.mmao_done[obuf], (io >> 1) & 1, fail, kWaitLimit)) return false;
             tc_fence_after();
-            const bool st_row = rowA && tA >= w0 && tA < w1;
+            const bool st_row = tA >= w0 && tA < w1;
             __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.o) +
-                                  ((size_t)bh * T + (size_t)c * C + tA) * p.dv + j0;
-#pragma unroll
-            for (int qd = 0; qd < DVT / 32; ++qd) {
-                float v[32];
-                tmem_ld32(tmem + lb + K::COL_O + obuf * DVT + 32 * qd, v);
-                tmem_ld_wait();
+                                  ((size_t)bh * T + (size_t)c * C + tA) * p.dv + j0 + oc0;
+            {
+                float v[OC];
+                ld_cols(K::COL_O + obuf * DVT, v, false);
                 if (st_row) {
 #pragma unroll
-                    for (int sg = 0; sg < 4; ++sg)
-                        reinterpret_cast<uint4*>(orow)[4 * qd + sg] = pack8(v + 8 * sg);
+                    for (int s8 = 0; s8 < OC / 8; ++s8)
+                        reinterpret_cast<uint4*>(orow)[s8] = pack8(v + 8 * s8);
                 }
             }
             tc_fence_before();
@@ -432,61 +563,69 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             if (lane == 0) mbar_arrive(&sm.o_free[obuf]);
             return true;
         };
-        int item = 0, pc = 0, pw0 = 0, pw1 = 0;
-        while (true) {
+        bool ok_run = true;
+        if (P == 1) {
+            load_s0();
+        } else if (has_p1) {
+#pragma unroll
+            for (int j = 0; j < SC; ++j) S[j] = 0.0f;
+        } else {
+            ok_run = fold_earlier();
+        }
+        float ld2 = 0.0f;  // log2 of this segment's decay product (first pass)
+        int item = 0, io = 0, pc = 0, pw0 = 0, pw1 = 0;
+        while (ok_run) {
             const int ob = item % NB;
             if (!mbar_wait(&sm.ops_full[ob], (item / NB) & 1, fail, kWaitLimit)) break;
-            const int c = sm.info[ob][0], w0 = sm.info[ob][1], w1 = sm.info[ob][2];
-            const int last = sm.info[ob][3];
+            const int c = sm.info[ob][kInfoChunk], w0 = sm.info[ob][kInfoW0], w1 = sm.info[ob][kInfoW1];
+            const int last = sm.info[ob][kInfoLast], p1last = sm.info[ob][kInfoP1Last];
+            const bool p2 = sm.info[ob][kInfoPhase] == 2;
             if (!mbar_wait(&sm.mma1_done, item & 1, fail, kWaitLimit)) break;
             tc_fence_after();
-            // A -> causal mask -> bf16 operand (row t = tA, columns s)
-#pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                float v[32];
-                tmem_ld32(tmem + lb + K::COL_A + 32 * hf, v);
-                tmem_ld_wait();
-                if (rowA) {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) v[e] = (32 * hf + e <= tA) ? v[e] : 0.0f;
-#pragma unroll
-                    for (int sg = 0; sg < 4; ++sg)
-                        *reinterpret_cast<uint4*>(sm.abf + off_rowmajor64(tA, 32 * hf + 8 * sg)) =
-                            pack8(v + 8 * sg);
-                }
-            }
-            // S_hat = diag(exp(m)) S_prev, and the chunk-start state if requested
-            if (rowS) {
-                const float em = sm.em[ob][iS];
-#pragma unroll
-                for (int jg = 0; jg < DVT / 8; ++jg) {
-                    float x[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) x[e] = S[jg * 8 + e] * em;
-                    *reinterpret_cast<uint4*>(sm.shat + off_shat<DK>(iS, jg * 8)) = pack8(x);
-                }
-                if (p.saved && w0 == 0) {
-                    float4* dst = reinterpret_cast<float4*>(
-                        p.saved + (((size_t)bh * NC + c) * DK + iS) * p.dv + j0);
-#pragma unroll
-                    for (int j4 = 0; j4 < DVT / 4; ++j4)
-                        dst[j4] = make_float4(S[4 * j4], S[4 * j4 + 1], S[4 * j4 + 2], S[4 * j4 + 3]);
-                }
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.abf_full);
-            // state update S = diag(gamma) S + diag(cfac) (Kt^T Vh)
-            {
-                const float gmv = rowS ? sm.gm[ob][iS] : 0.0f, cfv = rowS ? sm.cf[ob][iS] : 0.0f;
-#pragma unroll
-                for (int qd = 0; qd < DVT / 32; ++qd) {
-                    float v[32];
-                    tmem_ld32(tmem + lb + K::COL_S + 32 * qd, v);
+            if (p2) {
+                // A -> causal mask -> bf16 operand (row t = tA, columns s = a0 + e)
+                {
+                    const int a0 = 32 * hf + 16 * eh;
+                    float v[16];
+                    tmem_ld16_split<32>(tmem + lb + K::COL_A + 16 * eh, v);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) S[32 * qd + e] = fmaf(gmv, S[32 * qd + e], cfv * v[e]);
+                    for (int e = 0; e < 16; ++e) v[e] = (a0 + e <= tA) ? v[e] : 0.0f;
+#pragma unroll
+                    for (int s8 = 0; s8 < 2; ++s8)
+                        *reinterpret_cast<uint4*>(sm.abf + off_rowmajor64(tA, a0 + 8 * s8)) =
+                            pack8(v + 8 * s8);
                 }
+                // S_hat = diag(exp(m)) S_prev, and the chunk-start state if requested
+                {
+                    const float em = sm.em[ob][iS];
+#pragma unroll
+                    for (int jg = 0; jg < SC / 8; ++jg) {
+                        float x[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) x[e] = S[jg * 8 + e] * em;
+                        *reinterpret_cast<uint4*>(sm.shat + off_shat<DK>(iS, sc0 + jg * 8)) = pack8(x);
+                    }
+                    if (p.saved && w0 == 0) {
+                        float4* dst = reinterpret_cast<float4*>(
+                            p.saved + (((size_t)bh * NC + c) * DK + iS) * p.dv + j0 + sc0);
+#pragma unroll
+                        for (int j4 = 0; j4 < SC / 4; ++j4)
+                            dst[j4] = make_float4(S[4 * j4], S[4 * j4 + 1], S[4 * j4 + 2], S[4 * j4 + 3]);
+                    }
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.abf_full);
+            }
+            // state update S = diag(gamma) S + diag(cfac) (Kt^T Vh)
+            {
+                const float gmv = sm.gm[ob][iS], cfv = sm.cf[ob][iS];
+                if (!p2) ld2 += lg2_fast(gmv);
+                float v[SC];
+                ld_cols(K::COL_S, v, true);
+#pragma unroll
+                for (int e = 0; e < SC; ++e) S[e] = fmaf(gmv, S[e], cfv * v[e]);
             }
             tc_fence_before();
             __syncwarp();
@@ -495,22 +634,28 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             // once the tensor core is done with it too
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.ops_empty[ob]);
-            // o of the previous item (its MMA finished while this item's A and state
-            // were processed), then of this one if it is the last
-            if (item > 0 && !store_o(item - 1, pc, pw0, pw1)) break;
-            if (last) {
-                store_o(item, c, w0, w1);
-                break;
+            if (p2) {
+                // o of the previous o-item (its MMA finished while this item's A and
+                // state were processed), then of this one if it is the last
+                if (io > 0 && !store_o(io - 1, pc, pw0, pw1)) break;
+                if (last) {
+                    store_o(io, c, w0, w1);
+                    break;
+                }
+                pc = c;
+                pw0 = w0;
+                pw1 = w1;
+                ++io;
+            } else if (p1last) {
+                publish_segment(ld2);
+                if (!fold_earlier()) break;
             }
-            pc = c;
-            pw0 = w0;
-            pw1 = w1;
             ++item;
         }
-        if (!*fail && rowS && p.ST) {
-            float4* dst = reinterpret_cast<float4*>(p.ST + ((size_t)bh * DK + iS) * p.dv + j0);
+        if (!*fail && p.ST && seg == P - 1) {
+            float4* dst = reinterpret_cast<float4*>(p.ST + ((size_t)bh * DK + iS) * p.dv + j0 + sc0);
 #pragma unroll
-            for (int j4 = 0; j4 < DVT / 4; ++j4)
+            for (int j4 = 0; j4 < SC / 4; ++j4)
                 dst[j4] = make_float4(S[4 * j4], S[4 * j4 + 1], S[4 * j4 + 2], S[4 * j4 + 3]);
         }
     }
@@ -524,8 +669,82 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
     if (threadIdx.x == 0 && sm.fail) atomicOr(p.err, kErrTimeout);
 }
 
+// ------------------------------------------------------------------ host side
+
+int sm_count() {
+    static int cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 1;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+            n = 1;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+struct SegPlan {
+    int DVT, P;
+    size_t st_bytes, ld_bytes, flag_bytes, total;
+};
+
+SegPlan make_plan(const SeqParams& p, int DVT, int P) {
+    const long long units = (long long)p.B * p.H * (p.dv / DVT);
+    SegPlan s;
+    s.DVT = DVT;
+    s.P = P;
+    s.st_bytes = align256((size_t)(P - 1) * units * p.dk * DVT * 4);
+    s.ld_bytes = align256((size_t)(P - 1) * units * p.dk * 4);
+    s.flag_bytes = align256((size_t)P * units * 4);
+    s.total = P > 1 ? s.st_bytes + s.ld_bytes + s.flag_bytes : 0;
+    return s;
+}
+
+// Slice width and segment count.  Per CTA, a chunk costs about 1 time unit
+// with 64 d_v columns and 1.6 with 128 (the gate work is shared by the
+// columns), and a segmented CTA spends about 0.6 more per chunk on its
+// state-only pass.  Segments: as many as fill the SMs with one CTA each, none
+// shorter than kMinSegChunks chunks.  Take the cheaper of the two widths
+// (128 only exists for d_k = 64, d_v = 128); `allow_seg` false forces P = 1.
+SegPlan choose_plan(const SeqParams& p, bool allow_seg) {
+    const int NC = (p.T + C - 1) / C;
+    const int nsm = sm_count();
+    SegPlan best{};
+    double best_cost = 0.0;
+    for (int DVT : {64, 128}) {
+        if (DVT == 128 && !(p.dk == 64 && p.dv == 128)) continue;
+        if (p.dv % DVT) continue;
+        const long long units = (long long)p.B * p.H * (p.dv / DVT);
+        long long P = 1;
+        if (allow_seg && units < nsm) P = nsm / units;
+        if (P > NC / kMinSegChunks) P = NC / kMinSegChunks;
+        if (P < 1) P = 1;
+        const long long waves = (units * P + nsm - 1) / nsm;
+        const double per_chunk = (DVT == 128 ? 1.6 : 1.0) * (P > 1 ? 1.6 : 1.0);
+        const double cost = (double)waves * ((NC + P - 1) / P) * per_chunk;
+        if (best.P == 0 || cost < best_cost) {
+            best = make_plan(p, DVT, (int)P);
+            best_cost = cost;
+        }
+    }
+    return best;
+}
+
+// Tag of one launch for the segment flags: distinct for every launch of the
+// process, and seeded from the clock so that it is unlikely to equal what a
+// reused workspace still holds.
+unsigned next_epoch() {
+    static std::atomic<unsigned> counter{
+        (unsigned)std::chrono::steady_clock::now().time_since_epoch().count() | 1u};
+    const unsigned e = counter.fetch_add(1u) + 1u;
+    return e == 0 ? 1u : e;
+}
+
 template <int DK, int DVT>
-cudaError_t launch_cfg(const SeqParams& p, cudaStream_t s) {
+cudaError_t launch_cfg(const SeqParams& p, SegPlan plan, cudaStream_t s) {
     FwdKernelArgs a;
     a.p = p;
     const uint64_t BH = (uint64_t)p.B * p.H;
@@ -540,9 +759,29 @@ cudaError_t launch_cfg(const SeqParams& p, cudaStream_t s) {
     auto kern = tc_fwd_kernel<DK, DVT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const int grid = (int)(BH * (p.dv / DVT));
-    kern<<<grid, kThreads, smem, s>>>(a);
-    return cudaGetLastError();
+    const unsigned units = (unsigned)(BH * (p.dv / DVT));
+    uint8_t* ws = static_cast<uint8_t*>(p.ws);
+    a.seg.P = plan.P;
+    a.seg.epoch = next_epoch();
+    a.seg.st = plan.P > 1 ? reinterpret_cast<float*>(ws) : nullptr;
+    a.seg.ld = plan.P > 1 ? reinterpret_cast<float*>(ws + plan.st_bytes) : nullptr;
+    a.seg.flag = plan.P > 1 ? reinterpret_cast<unsigned*>(ws + plan.st_bytes + plan.ld_bytes) : nullptr;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(units * (unsigned)plan.P);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeCooperative;  // segments wait on one another
+    at[0].val.cooperative = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = plan.P > 1 ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+cudaError_t launch_plan(const SeqParams& p, const SegPlan& plan, cudaStream_t s) {
+    if (p.dk == 128) return launch_cfg<128, 64>(p, plan, s);
+    return plan.DVT == 128 ? launch_cfg<64, 128>(p, plan, s) : launch_cfg<64, 64>(p, plan, s);
 }
 
 }  // namespace
@@ -552,10 +791,21 @@ bool tc_fwd_supported(const SeqParams& p) {
            (p.dv == 64 || p.dv == 128);
 }
 
+size_t tc_fwd_workspace(const SeqParams& p) {
+    if (!tc_fwd_supported(p)) return 0;
+    return choose_plan(p, true).total;
+}
+
 cudaError_t launch_tc_fwd(const SeqParams& p, cudaStream_t s) {
     if (!tc_fwd_supported(p)) return cudaErrorNotSupported;
-    if (p.dk == 64) return launch_cfg<64, 64>(p, s);
-    return launch_cfg<128, 64>(p, s);
+    SegPlan plan = choose_plan(p, true);
+    if (plan.P > 1 && (p.ws == nullptr || p.ws_bytes < plan.total)) plan = choose_plan(p, false);
+    cudaError_t e = launch_plan(p, plan, s);
+    if (e == cudaErrorCooperativeLaunchTooLarge && plan.P > 1) {
+        (void)cudaGetLastError();  // the CTAs do not all fit at once: run unsegmented
+        e = launch_plan(p, choose_plan(p, false), s);
+    }
+    return e;
 }
 
 }  // namespace rdm

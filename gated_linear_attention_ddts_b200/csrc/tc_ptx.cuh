@@ -137,6 +137,26 @@ __device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b
         ::"r"(tmem_d), "l"(a), "l"(b), "r"(idesc), "r"(accumulate) : "memory");
 }
 
+// The same descriptor as two 32-bit words, for issue loops: with base = the
+// operand's shared address >> 4 computed once, the low word of the tile at byte
+// offset `off` is base + sd_lo(off, lbo) (one integer add; addresses stay below
+// 256 KB so the 14-bit field never carries) and the high word is a constant.
+__host__ __device__ constexpr uint32_t sd_lo(uint32_t off, uint32_t lbo) {
+    return (off >> 4) + ((lbo >> 4) << 16);
+}
+__host__ __device__ constexpr uint32_t sd_hi(uint32_t sbo) { return (sbo >> 4) | (1u << 14); }
+
+__device__ __forceinline__ void mma_bf16_w(uint32_t tmem_d, uint32_t a_lo, uint32_t a_hi,
+                                           uint32_t b_lo, uint32_t b_hi, uint32_t idesc,
+                                           uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n .reg .b64 da, db;\n setp.ne.b32 p, %6, 0;\n"
+        " mov.b64 da, {%1, %2};\n mov.b64 db, {%3, %4};\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %5, p;\n}\n"
+        ::"r"(tmem_d), "r"(a_lo), "r"(a_hi), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Arrive (once) on a CTA-local mbarrier when all previously issued MMAs of
 // this thread have completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
@@ -163,6 +183,20 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
 // the warp's sub-partition) read twice: threads 0-15 get lane (taddr.lane + i),
 // columns taddr.col .. +31; threads 16-31 get lane (taddr.lane + i - 16),
 // columns taddr.col + kSplit .. +31.  All 32 threads of the warp carry data.
+// tmem_ld16_split is the same with 16 columns per thread.
+template <int kSplit>
+__device__ __forceinline__ void tmem_ld16_split(uint32_t taddr, float* v) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x32bx2.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16], %17;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr), "n"(kSplit));
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
 template <int kSplit>
 __device__ __forceinline__ void tmem_ld32_split(uint32_t taddr, float* v) {
     uint32_t r[32];
@@ -228,6 +262,16 @@ __device__ __forceinline__ void named_bar(int id, int count) {
 
 __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
+}
+
+// ------------------------------------------------- flags between CTAs (global)
+__device__ __forceinline__ void st_release_gpu(unsigned* p, unsigned v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
 }
 
 // --------------------------------------------------------------- cluster / DSMEM

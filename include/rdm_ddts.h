@@ -82,6 +82,13 @@ typedef enum { RDM_IMPL_AUTO = 0, RDM_IMPL_SIMT = 1, RDM_IMPL_TC = 2 } rdm_impl;
  *                  in force before each chunk (S_0 for chunk 0); NULL = skip.
  *                  rdm_ddts_bwd can reuse it instead of recomputing.
  *   chunk        : tokens per chunk; 0 selects 64.  Allowed: 64.
+ *   workspace    : optional device scratch of workspace_bytes.  With at least
+ *                  rdm_ddts_fwd_workspace_size() bytes the tensor-core path
+ *                  may cut each sequence into segments processed by separate
+ *                  CTAs (when B*H alone does not fill the GPU); with less, or
+ *                  NULL, it runs each sequence in one CTA.  Results agree up
+ *                  to rounding either way.  Contents on entry are ignored; two
+ *                  calls whose kernels may overlap must not share it.
  */
 typedef struct {
     int B, H, T, dk, dv;
@@ -93,9 +100,16 @@ typedef struct {
     void *o;
     float *ST;
     float *saved_states;
+    void *workspace;
+    size_t workspace_bytes;
 } rdm_fwd_args;
 
 rdm_status rdm_ddts_fwd(const rdm_fwd_args *args, rdm_stream_t stream);
+
+/* Scratch bytes that let rdm_ddts_fwd segment sequences for `args` (0 when it
+ * would not; depends on sizes, dtype, impl and the device's SM count);
+ * (size_t)-1 on invalid sizes. */
+size_t rdm_ddts_fwd_workspace_size(const rdm_fwd_args *args);
 
 /* Bytes of `saved_states` that rdm_ddts_fwd writes for these sizes
  * (B*H*ceil(T/chunk)*d_k*d_v*4); 0 on invalid sizes. */

@@ -1,7 +1,7 @@
 """GPU parity of the tensor-core (tcgen05) chunked forward against the fp64
 oracle, through the C ABI: ragged tails, initial/final states, saved chunk
-states, wide-decay windows, the special cases g = 0 and tau = 0, and the
-full-size workloads (sampled heads)."""
+states, wide-decay windows, the special cases g = 0 and tau = 0, sequences cut
+into segments (one CTA each), and the full-size workloads (sampled heads)."""
 import numpy as np
 import pytest
 import torch
@@ -16,7 +16,7 @@ TOL = 2e-2
 SEQ = ("q", "k", "v", "g", "tau", "beta")
 
 
-def run_tc(x, want_saved=False, impl="tc"):
+def run_tc(x, want_saved=False, impl="tc", workspace=None):
     d = {n: (t.cuda() if t is not None else None) for n, t in x.items()}
     B, H, T, dk = d["q"].shape
     dv = d["v"].shape[-1]
@@ -25,7 +25,7 @@ def run_tc(x, want_saved=False, impl="tc"):
         saved = torch.full((rdm.rdm_ddts_saved_states_size(B, H, T, dk, dv, 64) // 4,),
                            float("nan"), device="cuda")
     o, ST = rdm.rdm_ddts_fwd(*(d[n] for n in SEQ), d.get("S0"), saved_states=saved, impl=impl,
-                             return_state=True)
+                             return_state=True, workspace=workspace)
     torch.cuda.synchronize()
     assert rdm.rdm_ddts_sync_status() == rdm.RDM_OK
     return o, ST, saved
@@ -94,6 +94,77 @@ def test_tc_split_invariance(cuda_ok):
     ob, Sb, _ = run_tc(dict(b, S0=Sa.cpu()))
     assert_close(torch.cat([oa, ob], 2), o, TOL, "split o")
     assert_close(Sb, ST, TOL, "split S_T")
+
+
+def segments_used(x):
+    d = {n: x[n].cuda() for n in SEQ}
+    return rdm.rdm_ddts_fwd_workspace_size(*(d[n] for n in SEQ), impl="tc") > 0
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 64), (64, 128), (128, 64), (128, 128)])
+@pytest.mark.parametrize("T", [64 * 8, 64 * 13 + 37])
+def test_tc_forward_segmented(cuda_ok, dk, dv, T):
+    """Two heads leave most SMs idle, so each sequence is cut into segments that
+    separate CTAs run; their state maps are folded across CTAs.  Output, final
+    state and saved chunk states against the oracle, and against one CTA per
+    sequence (no workspace)."""
+    x = draw_sequence(1, 2, T, dk, dv, torch.bfloat16, seed=3000 + T + dk + dv, s0_std=0.1)
+    assert segments_used(x)
+    o, ST, saved = run_tc(x, want_saved=True)
+    o_ref, S_ref = oracle.fwd(*(x[n] for n in SEQ), x["S0"])
+    assert_close(o, o_ref, TOL, "o")
+    assert_close(ST, S_ref, TOL, "S_T")
+    nc = (T + 63) // 64
+    sv = saved.view(1, 2, nc, dk, dv)
+    for c in sorted({1, nc // 3, nc // 2, (2 * nc) // 3, nc - 1}):
+        ref = oracle.fwd(*(x[n][:, :, :64 * c] for n in SEQ), x["S0"])[1]
+        assert_close(sv[:, :, c], ref, TOL, f"saved state {c}")
+    o1, S1, _ = run_tc(x, workspace=False)
+    assert_close(o, o1.float().cpu().numpy(), TOL, "o segmented vs one CTA")
+    assert_close(ST, S1.cpu().numpy(), TOL, "S_T segmented vs one CTA")
+
+
+@pytest.mark.parametrize("scale", [3.0, 40.0])
+def test_tc_segmented_wide_decay(cuda_ok, scale):
+    """Narrow windows inside segments; decay products across segments that
+    underflow to zero for the short-memory channels."""
+    x = draw_sequence(1, 1, 64 * 9 + 5, 64, 128, torch.bfloat16, seed=41, s0_std=0.1)
+    x["g"] = (x["g"].float() * scale).to(torch.bfloat16)
+    x["g"][:, :, :, :8] = (x["g"][:, :, :, :8].float() / scale / 10).to(torch.bfloat16)
+    assert segments_used(x)
+    o, ST, _ = run_tc(x)
+    o_ref, S_ref = oracle.fwd(*(x[n] for n in SEQ), x["S0"])
+    assert_close(o, o_ref, TOL, "o")
+    assert_close(ST, S_ref, TOL, "S_T")
+
+
+@pytest.mark.parametrize("B,H,T", [(1, 40, 64 * 12 + 9), (4, 25, 130)])
+def test_tc_forward_wide_slices(cuda_ok, B, H, T):
+    """Head counts for which one CTA takes all 128 value columns of a head:
+    40 heads (segmented three ways on a 148-SM part) and 100 heads (one
+    segment, one wave)."""
+    x = draw_sequence(B, H, T, 64, 128, torch.bfloat16, seed=50 + B * H, s0_std=0.1)
+    o, ST, _ = run_tc(x)
+    o_ref, S_ref = oracle.fwd(*(x[n] for n in SEQ), x["S0"])
+    assert_close(o, o_ref, TOL, "o")
+    assert_close(ST, S_ref, TOL, "S_T")
+
+
+def test_tc_segmented_repeat_calls(cuda_ok):
+    """The same workspace serves back-to-back calls (flags tagged per launch)."""
+    x = draw_sequence(1, 2, 64 * 12, 64, 128, torch.bfloat16, seed=43, s0_std=0.1)
+    d = {n: x[n].cuda() for n in SEQ}
+    ws = torch.empty(rdm.rdm_ddts_fwd_workspace_size(*(d[n] for n in SEQ)), dtype=torch.uint8,
+                     device="cuda")
+    S0 = x["S0"].cuda()
+    outs = [rdm.rdm_ddts_fwd(*(d[n] for n in SEQ), S0, workspace=ws, return_state=True)
+            for _ in range(3)]
+    torch.cuda.synchronize()
+    assert rdm.rdm_ddts_sync_status() == rdm.RDM_OK
+    o_ref, S_ref = oracle.fwd(*(x[n] for n in SEQ), x["S0"])
+    for o, ST in outs:
+        assert_close(o, o_ref, TOL, "o")
+        assert_close(ST, S_ref, TOL, "S_T")
 
 
 def sampled_check(w, heads, device_inputs=True):
