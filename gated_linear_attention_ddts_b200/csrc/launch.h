@@ -70,4 +70,11 @@ namespace rdm {
 // driver refuses the map.
 bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t n0, uint64_t n1,
                        uint64_t n2, uint32_t b0, uint32_t b1);
+
+// SM count of the current device (cached).
+int sm_count();
+// Tag of one launch for flags that CTAs of a sequence-segmented kernel set for
+// one another: distinct for every launch of the process, seeded from the clock
+// so that it is unlikely to equal what a reused workspace still holds.
+unsigned next_launch_tag();
 }  // namespace rdm

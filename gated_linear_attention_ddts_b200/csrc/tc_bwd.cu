@@ -28,6 +28,18 @@
 // A chunk whose log-decay span exceeds the range one reference can hold flags
 // its head; those heads are recomputed afterwards by the exact CUDA-core
 // backward (launched behind this kernel, it skips unflagged heads).
+//
+// Sequence segments (when the heads alone do not fill the GPU): each head's
+// chunks are cut into P contiguous segments, one CTA each.  R maps affinely
+// across a segment, R_start = diag(D) R_end + R_loc, so every segment but the
+// first first runs the R recurrence alone from zero at its end (Qt and dO
+// only) and publishes (R_loc, log2 D); a segment then folds the maps of all
+// later segments onto dS_T to obtain its R_end.  The decay-gradient carry
+// into a segment, the suffix sum of (q dq - khat dkhat) over all later tokens
+// plus rowsum(dS_T o S_T), equals rowsum(R_end o S_end) with S_end the state
+// at the segment end (rescaling row i of q by e^eps and of khat and S_0 by
+// e^-eps leaves o unchanged and scales S_T by e^-eps).  All CTAs of such a
+// launch are resident together (cooperative launch); waits are bounded.
 #include <cuda.h>
 
 #include "launch.h"
@@ -43,6 +55,7 @@ constexpr int DK = 64;
 constexpr int kGateWarps = 8;  // one 8-channel group each
 constexpr int kThreads = 32 * (4 + kGateWarps + 2);
 constexpr int kEpiWarp0 = 0, kGateWarp0 = 4, kProdWarp = 4 + kGateWarps, kMmaWarp = 5 + kGateWarps;
+constexpr int kBarEpi = 3;  // the four epilogue warps
 constexpr int kStg = 68;     // row stride (floats) of the dQ / dK staging tiles
 
 template <int DV>
@@ -85,10 +98,22 @@ struct alignas(1024) BwdSmem {
     int fail;
 };
 
+// Segment exchange area (global): per (segment > 0, head) R_loc [DK][DV] and
+// log2 of the decay product per channel; per (segment, head) a flag holding
+// `tag` once those are written.
+struct BwdSeg {
+    int P;
+    unsigned tag;
+    float* st;
+    float* ld;
+    unsigned* flag;
+};
+
 struct BwdKernelArgs {
     CUtensorMap mq, mk, mg, mt, mv, mb, mdo;
     BwdParams p;
     int* flags;
+    BwdSeg seg;
 };
 
 // [row][col] tile with 8-row groups 128 B apart and 8-column groups 1024 B
@@ -106,9 +131,19 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
     BwdSmem<DV>& sm = *reinterpret_cast<BwdSmem<DV>*>(
         smem_dyn + ((1024u - (smem_u32(smem_dyn) & 1023u)) & 1023u));
     const BwdParams& p = A.p;
+    const BwdSeg& sg = A.seg;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int bh = blockIdx.x;
+    const int BH = p.B * p.H;
+    const int bh = blockIdx.x % BH, seg = blockIdx.x / BH;
     const int T = p.T, NC = (T + C - 1) / C;
+    const int P = sg.P;
+    const int cs0 = (int)((long long)seg * NC / P), cs1 = (int)((long long)(seg + 1) * NC / P);
+    const int nseg = cs1 - cs0;
+    const bool has_p1 = seg > 0;             // runs the R-only first pass
+    const bool last_seg = seg == P - 1;      // its R_end is dS_T
+    const int nL = (has_p1 ? 2 : 1) * nseg;  // chunk passes, each over [cs0, cs1) last chunk first
+    auto pass_chunk = [&](int li) { return cs1 - 1 - (li < nseg ? li : li - nseg); };
+    auto pass_p2 = [&](int li) { return !has_p1 || li >= nseg; };
 
     if (threadIdx.x == 0) {
         mbar_init(&sm.raw_full, 1);
@@ -148,17 +183,21 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             int issued = 0;
-            for (int it = 0; it < NC; ++it) {
-                const int c = NC - 1 - it;
-                if (it > 0 && !mbar_wait(&sm.raw_empty, (it - 1) & 1, fail, kWaitLimit)) break;
-                mbar_expect_tx(&sm.raw_full, K::RAW);
+            for (int li = 0; li < nL; ++li) {
+                const int c = pass_chunk(li);
+                const bool p2 = pass_p2(li);
+                if (li > 0 && !mbar_wait(&sm.raw_empty, (li - 1) & 1, fail, kWaitLimit)) break;
+                // the R-only pass reads q, g, tau and dO
+                mbar_expect_tx(&sm.raw_full, p2 ? K::RAW : (3 + VB) * kBox);
                 tma_load_3d(sm.raw + 0 * kBox, &A.mq, &sm.raw_full, 0, c * C, bh);
-                tma_load_3d(sm.raw + 1 * kBox, &A.mk, &sm.raw_full, 0, c * C, bh);
+                if (p2) tma_load_3d(sm.raw + 1 * kBox, &A.mk, &sm.raw_full, 0, c * C, bh);
                 tma_load_3d(sm.raw + 2 * kBox, &A.mg, &sm.raw_full, 0, c * C, bh);
                 tma_load_3d(sm.raw + 3 * kBox, &A.mt, &sm.raw_full, 0, c * C, bh);
                 for (int vb = 0; vb < VB; ++vb) {
-                    tma_load_3d(sm.raw + K::OFF_V + vb * kBox, &A.mv, &sm.raw_full, 64 * vb, c * C, bh);
-                    tma_load_3d(sm.raw + K::OFF_B + vb * kBox, &A.mb, &sm.raw_full, 64 * vb, c * C, bh);
+                    if (p2) {
+                        tma_load_3d(sm.raw + K::OFF_V + vb * kBox, &A.mv, &sm.raw_full, 64 * vb, c * C, bh);
+                        tma_load_3d(sm.raw + K::OFF_B + vb * kBox, &A.mb, &sm.raw_full, 64 * vb, c * C, bh);
+                    }
                     tma_load_3d(sm.raw + K::OFF_DO + vb * kBox, &A.mdo, &sm.raw_full, 64 * vb, c * C, bh);
                 }
                 ++issued;
@@ -181,10 +220,23 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             constexpr uint32_t id_v1 = idesc_bf16(64, DV, 1, 1);   // A^T dO
             constexpr uint32_t id_v2 = idesc_bf16(64, DV, 0, 1);   // Kt R_hat
             int n1 = 0, n2 = 0;
-            for (int it = 0; it < NC; ++it) {
-                if (!mbar_wait(&sm.ops_full, it & 1, fail, kWaitLimit)) break;
-                if (it > 0 && !mbar_wait(&sm.tm1_free, (it - 1) & 1, fail, kWaitLimit)) break;
+            for (int li = 0; li < nL; ++li) {
+                const bool p2 = pass_p2(li);
+                const int i2 = n2;  // index among full passes
+                if (!mbar_wait(&sm.ops_full, li & 1, fail, kWaitLimit)) break;
+                if (li > 0 && !mbar_wait(&sm.tm1_free, (li - 1) & 1, fail, kWaitLimit)) break;
                 tc_fence_after();
+                if (!p2) {
+                    // R-only pass: dR = Qt^T dO
+#pragma unroll
+                    for (int ks = 0; ks < C / 16; ++ks)
+                        mma_bf16(tmem + K::COL_DR, sdesc(q + ks * 256, 128, kQK),
+                                 sdesc(d + ks * 256, 128, 1024), id_r, ks > 0);
+                    mma_commit(&sm.g1_done);
+                    mma_commit(&sm.ops_empty);
+                    ++n1;
+                    continue;
+                }
 #pragma unroll
                 for (int ks = 0; ks < DK / 16; ++ks)
                     mma_bf16(tmem + K::COL_A, sdesc(q + ks * 2 * kQK, kQK, 128),
@@ -197,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 for (int ks = 0; ks < C / 16; ++ks)
                     mma_bf16(tmem + K::COL_DR, sdesc(q + ks * 256, 128, kQK),
                              sdesc(d + ks * 256, 128, 1024), id_r, ks > 0);
-                if (it == 0 && p.dST) {
+                if (i2 == 0 && last_seg && p.dST) {
                     // Kt^T Vh of the last chunk, for S_T (only the final-state gradient needs it)
 #pragma unroll
                     for (int ks = 0; ks < C / 16; ++ks)
@@ -206,9 +258,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 }
                 mma_commit(&sm.g1_done);
                 ++n1;
-                if (!mbar_wait(&sm.g2_ready, it & 1, fail, kWaitLimit)) break;
-                if (!mbar_wait(&sm.shat_full, it & 1, fail, kWaitLimit)) break;
-                if (it > 0 && !mbar_wait(&sm.tm2_free, (it - 1) & 1, fail, kWaitLimit)) break;
+                if (!mbar_wait(&sm.g2_ready, i2 & 1, fail, kWaitLimit)) break;
+                if (!mbar_wait(&sm.shat_full, i2 & 1, fail, kWaitLimit)) break;
+                if (i2 > 0 && !mbar_wait(&sm.tm2_free, (i2 - 1) & 1, fail, kWaitLimit)) break;
                 tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < C / 16; ++ks)
@@ -263,9 +315,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
         const int tb = seg * SEGT;
         const uint32_t full = 0xffffffffu;
         const uint8_t* raw = sm.raw;
-        for (int it = 0; it < NC; ++it) {
-            const int c = NC - 1 - it;
-            if (!mbar_wait(&sm.raw_full, it & 1, fail, kWaitLimit)) break;
+        int i2 = 0;  // full passes done
+        for (int li = 0; li < nL; ++li) {
+            const int c = pass_chunk(li);
+            const bool p2 = pass_p2(li);
+            if (!mbar_wait(&sm.raw_full, li & 1, fail, kWaitLimit)) break;
             const int nval = min(C, T - c * C);
             // ---- pre: running log-decay, reference, operands
             float b[SEGT][8], mL[8], blL[8];
@@ -308,7 +362,45 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 // too wide for one reference: the exact path recomputes this head
                 if (__any_sync(full, !(span <= kSpanMax)) && lane == 0) A.flags[bh] = 1;
             }
-            if (it > 0 && !mbar_wait(&sm.ops_empty, (it - 1) & 1, fail, kWaitLimit)) break;
+            // operand slot free: tensor core done with it (ops_empty) and the epilogue
+            // done with the constants (tm1_free; it consumes em / cf / gm in its
+            // first stage)
+            if (li > 0 && (!mbar_wait(&sm.ops_empty, (li - 1) & 1, fail, kWaitLimit) ||
+                           !mbar_wait(&sm.tm1_free, (li - 1) & 1, fail, kWaitLimit)))
+                break;
+            if (!p2) {
+                // R-only pass: Qt (bf16), the constants and dO
+#pragma unroll
+                for (int u = 0; u < SEGT; ++u) {
+                    const int t = tb + u;
+                    float q8[8], oq[8];
+                    unpack8(*reinterpret_cast<const uint4*>(raw + 0 * kBox + off_raw(t, cg)), q8);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) oq[e] = q8[e] * ex2_fast(fmaf(b[u][e], kLog2e, -mL[e]));
+                    *reinterpret_cast<uint4*>(sm.qt + off_qk(t, cg * 8)) = pack8(oq);
+                }
+                if (tb == 0) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        sm.em[cg * 8 + e] = ex2_fast(mL[e]);
+                        sm.gm[cg * 8 + e] = ex2_fast(blL[e]);
+                    }
+                }
+#pragma unroll
+                for (int iv = 0; iv < VIT; ++iv) {
+                    const int jg = gt / TPG, t = (gt % TPG) + TPG * iv;
+                    *reinterpret_cast<uint4*>(sm.dot + off_rc(t, jg * 8)) =
+                        *reinterpret_cast<const uint4*>(raw + K::OFF_DO + off_raw(t, jg));
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&sm.ops_full);
+                    mbar_arrive(&sm.raw_empty);
+                }
+                if (*fail) break;
+                continue;
+            }
 #pragma unroll
             for (int u = 0; u < SEGT; ++u) {
                 const int t = tb + u;
@@ -384,7 +476,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             if (lane == 0) mbar_arrive(&sm.shat_full);
 
             // ---- post: final gate gradients once dQ, dK of this chunk are staged
-            if (!mbar_wait(&sm.post_ready, it & 1, fail, kWaitLimit)) break;
+            if (!mbar_wait(&sm.post_ready, i2 & 1, fail, kWaitLimit)) break;
             float dG[SEGT][8], dkh[SEGT][8];
 #pragma unroll
             for (int u = 0; u < SEGT; ++u) {
@@ -432,7 +524,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                     const float y = __shfl_down_sync(full, x, d);
                     if (lane + d < 32) x += y;
                 }
-                const float off = (x - tot) + sm.carry[cg * 8 + e] + (it == 0 ? sm.fin[cg * 8 + e] : 0.0f);
+                const float off = (x - tot) + sm.carry[cg * 8 + e] +
+                                  (i2 == 0 && last_seg ? sm.fin[cg * 8 + e] : 0.0f);
 #pragma unroll
                 for (int u = 0; u < SEGT; ++u) dG[u][e] += off;
             }
@@ -472,6 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 mbar_arrive(&sm.post_done);
                 mbar_arrive(&sm.raw_empty);
             }
+            ++i2;
             if (*fail) break;
         }
     } else {
@@ -485,13 +579,100 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
         const int r = 16 * ew + (lane & 15);
         const uint32_t lb = (uint32_t)(32 * ew) << 16;
         float R[HV];  // R[r][hf*HV .. hf*HV + HV)
+        auto load_dst = [&]() {
 #pragma unroll
-        for (int j = 0; j < HV; ++j) R[j] = p.dST ? p.dST[((size_t)bh * DK + r) * DV + hf * HV + j] : 0.0f;
-        for (int it = 0; it < NC; ++it) {
-            const int c = NC - 1 - it;
-            if (!mbar_wait(&sm.ops_full, it & 1, fail, kWaitLimit)) break;
-            if (!mbar_wait(&sm.g1_done, it & 1, fail, kWaitLimit)) break;
+            for (int j = 0; j < HV; ++j)
+                R[j] = p.dST ? p.dST[((size_t)bh * DK + r) * DV + hf * HV + j] : 0.0f;
+        };
+        // R at the end of this segment: dS_T carried through the maps of all later
+        // segments, R <- diag(D_s) R + R_loc_s; then the decay-gradient carry into
+        // the segment, rowsum(R o S) with S the saved state at the segment end
+        auto fold_later = [&]() -> bool {
+            if (threadIdx.x == 0) {
+                const long long t0 = clock64();
+                for (int s2 = P - 1; s2 > seg && !*fail; --s2)
+                    while (ld_acquire_gpu(&sg.flag[s2 * BH + bh]) != sg.tag)
+                        if (clock64() - t0 > kWaitLimit) {
+                            *fail = 1;
+                            break;
+                        }
+            }
+            named_bar(kBarEpi, 128);
+            if (*fail) return false;
+            load_dst();
+            for (int s2 = P - 1; s2 > seg; --s2) {
+                const size_t u = (size_t)s2 * BH + bh;
+                const float d = ex2_fast(__ldcg(&sg.ld[u * DK + r]));
+                const float4* src = reinterpret_cast<const float4*>(sg.st + (u * DK + r) * DV + hf * HV);
+#pragma unroll
+                for (int j4 = 0; j4 < HV / 4; ++j4) {
+                    const float4 x = __ldcg(src + j4);
+                    R[4 * j4] = fmaf(d, R[4 * j4], x.x);
+                    R[4 * j4 + 1] = fmaf(d, R[4 * j4 + 1], x.y);
+                    R[4 * j4 + 2] = fmaf(d, R[4 * j4 + 2], x.z);
+                    R[4 * j4 + 3] = fmaf(d, R[4 * j4 + 3], x.w);
+                }
+            }
+            if (!last_seg) {
+                const float* Se = p.saved + (((size_t)bh * NC + cs1) * DK + r) * DV + hf * HV;
+                float f = 0.0f;
+#pragma unroll
+                for (int j = 0; j < HV; ++j) f = fmaf(R[j], Se[j], f);
+                f += __shfl_xor_sync(0xffffffffu, f, 16);
+                if (hf == 0) sm.carry[r] = f;
+            }
+            return true;
+        };
+        // publish this segment's map (R_loc in R, log2 D in ld2)
+        auto publish_segment = [&](float ld2) {
+            const size_t u = (size_t)seg * BH + bh;
+            float4* dst = reinterpret_cast<float4*>(sg.st + (u * DK + r) * DV + hf * HV);
+#pragma unroll
+            for (int j4 = 0; j4 < HV / 4; ++j4)
+                dst[j4] = make_float4(R[4 * j4], R[4 * j4 + 1], R[4 * j4 + 2], R[4 * j4 + 3]);
+            if (hf == 0) sg.ld[u * DK + r] = ld2;
+            __threadfence();
+            named_bar(kBarEpi, 128);
+            if (threadIdx.x == 0) st_release_gpu(&sg.flag[u], sg.tag);
+        };
+        bool ok_run = true;
+        if (P == 1) {
+            load_dst();
+        } else if (has_p1) {
+#pragma unroll
+            for (int j = 0; j < HV; ++j) R[j] = 0.0f;
+        } else {
+            ok_run = fold_later();
+        }
+        float ld2 = 0.0f;  // log2 of this segment's decay product (R-only pass)
+        int i2 = 0;        // full passes done
+        for (int li = 0; ok_run && li < nL; ++li) {
+            const int c = pass_chunk(li);
+            const bool p2 = pass_p2(li);
+            if (!mbar_wait(&sm.ops_full, li & 1, fail, kWaitLimit)) break;
+            if (!mbar_wait(&sm.g1_done, li & 1, fail, kWaitLimit)) break;
             tc_fence_after();
+            if (!p2) {
+                // R-only pass: R <- diag(e^{b_last}) R + diag(e^m) Qt^T dO
+                const float emv = sm.em[r], gmv = sm.gm[r];
+                ld2 += lg2_fast(gmv);
+#pragma unroll
+                for (int qd = 0; qd < HV / 32; ++qd) {
+                    float v[32];
+                    tmem_ld32_split<HV>(tmem + lb + K::COL_DR + 32 * qd, v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) R[32 * qd + e] = fmaf(gmv, R[32 * qd + e], emv * v[e]);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.tm1_free);
+                if (li == nseg - 1) {
+                    publish_segment(ld2);
+                    if (!fold_later()) break;
+                }
+                continue;
+            }
             // A and B -> causal mask -> bf16 operands (row t = r, columns s = 32 hf + e)
 #pragma unroll
             for (int which = 0; which < 2; ++which) {
@@ -517,7 +698,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                     *reinterpret_cast<uint4*>(dst + off_rc(r, 32 * hf + 8 * sg)) = pack8(v + 8 * sg);
             }
             const float emv = sm.em[r], cfv = sm.cf[r], gmv = sm.gm[r];
-            if (it == 0 && p.dST) {
+            if (i2 == 0 && last_seg && p.dST) {
                 // final-state term rowsum(dS_T o S_T) with S_T = diag(gm) S_prev + diag(cf) Kt^T Vh
                 const float* Sprev = p.saved + (((size_t)bh * NC + c) * DK + r) * DV + hf * HV;
                 float f = 0.0f;
@@ -559,7 +740,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 mbar_arrive(&sm.g2_ready);
                 mbar_arrive(&sm.tm1_free);
             }
-            if (!mbar_wait(&sm.g2_done, it & 1, fail, kWaitLimit)) break;
+            if (!mbar_wait(&sm.g2_done, i2 & 1, fail, kWaitLimit)) break;
             tc_fence_after();
             // dV -> dv = beta dvhat, dbeta = v dvhat (row s = r)
             {
@@ -589,7 +770,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 }
             }
             // dQ, dK -> fp32 staging for the gate warps
-            if (it > 0 && !mbar_wait(&sm.post_done, (it - 1) & 1, fail, kWaitLimit)) break;
+            if (i2 > 0 && !mbar_wait(&sm.post_done, (i2 - 1) & 1, fail, kWaitLimit)) break;
 #pragma unroll
             for (int which = 0; which < 2; ++which) {
                 float v[32];
@@ -606,8 +787,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 mbar_arrive(&sm.post_ready);
                 mbar_arrive(&sm.tm2_free);
             }
+            ++i2;
         }
-        if (!*fail && p.dS0) {
+        if (!*fail && p.dS0 && seg == 0) {
             float4* dst = reinterpret_cast<float4*>(p.dS0 + ((size_t)bh * DK + r) * DV + hf * HV);
 #pragma unroll
             for (int j4 = 0; j4 < HV / 4; ++j4)
@@ -626,23 +808,43 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
+constexpr int kMinSegChunks = 4;  // shortest segment worth a CTA of its own
+
+// Segments per head: as many as fill the SMs with one CTA each, none shorter
+// than kMinSegChunks chunks.
+int bwd_segments(const BwdParams& p) {
+    const long long BH = (long long)p.B * p.H;
+    const int NC = (p.T + C - 1) / C;
+    const int nsm = sm_count();
+    long long P = BH < nsm ? nsm / BH : 1;
+    if (P > NC / kMinSegChunks) P = NC / kMinSegChunks;
+    return P < 1 ? 1 : (int)P;
+}
+
 struct WsLayout {
-    size_t states, oscr, flags, simt, total;
+    int P;
+    size_t states, oscr, flags, simt, seg_st, seg_ld, seg_flag, total;
 };
 
 WsLayout ws_layout(const BwdParams& p) {
     WsLayout w;
     const size_t bh = (size_t)p.B * p.H, nc = (size_t)(p.T + C - 1) / C;
+    w.P = bwd_segments(p);
     w.states = p.saved ? 0 : align256(bh * nc * p.dk * p.dv * 4);
     w.oscr = p.saved ? 0 : align256(bh * (size_t)p.T * p.dv * 2);
     w.flags = align256(bh * 4);
     w.simt = align256(simt_bwd_workspace(p));
-    w.total = w.states + w.oscr + w.flags + w.simt;
+    // segment exchange, indexed by segment (slot 0 unused)
+    w.seg_st = w.P > 1 ? align256((size_t)w.P * bh * p.dk * p.dv * 4) : 0;
+    w.seg_ld = w.P > 1 ? align256((size_t)w.P * bh * p.dk * 4) : 0;
+    w.seg_flag = w.P > 1 ? align256((size_t)w.P * bh * 4) : 0;
+    w.total = w.states + w.oscr + w.flags + w.simt + w.seg_st + w.seg_ld + w.seg_flag;
     return w;
 }
 
 template <int DV>
-cudaError_t launch_dv(const BwdParams& p, const float* saved, int* flags, cudaStream_t s) {
+cudaError_t launch_dv(const BwdParams& p, const float* saved, int* flags, const WsLayout& w,
+                      cudaStream_t s) {
     BwdKernelArgs a;
     a.p = p;
     a.p.saved = saved;
@@ -660,8 +862,27 @@ cudaError_t launch_dv(const BwdParams& p, const float* saved, int* flags, cudaSt
     auto kern = tc_bwd_kernel<DV>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    kern<<<(int)BH, kThreads, smem, s>>>(a);
-    return cudaGetLastError();
+    char* seg = static_cast<char*>(p.ws) + w.states + w.oscr + w.flags + w.simt;
+    for (int P = w.P;; P = 1) {
+        a.seg.P = P;
+        a.seg.tag = next_launch_tag();
+        a.seg.st = P > 1 ? reinterpret_cast<float*>(seg) : nullptr;
+        a.seg.ld = P > 1 ? reinterpret_cast<float*>(seg + w.seg_st) : nullptr;
+        a.seg.flag = P > 1 ? reinterpret_cast<unsigned*>(seg + w.seg_st + w.seg_ld) : nullptr;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(BH * P));
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = s;
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeCooperative;  // segments wait on one another
+        at[0].val.cooperative = 1;
+        cfg.attrs = at;
+        cfg.numAttrs = P > 1 ? 1 : 0;
+        e = cudaLaunchKernelEx(&cfg, kern, a);
+        if (e != cudaErrorCooperativeLaunchTooLarge || P == 1) return e;
+        (void)cudaGetLastError();  // the CTAs do not all fit at once: run unsegmented
+    }
 }
 
 }  // namespace
@@ -692,7 +913,7 @@ cudaError_t launch_tc_bwd(const BwdParams& p, cudaStream_t s) {
     }
     int* flags = reinterpret_cast<int*>(ws + w.states + w.oscr);
     if ((e = cudaMemsetAsync(flags, 0, (size_t)p.B * p.H * 4, s)) != cudaSuccess) return e;
-    e = p.dv == 64 ? launch_dv<64>(p, saved, flags, s) : launch_dv<128>(p, saved, flags, s);
+    e = p.dv == 64 ? launch_dv<64>(p, saved, flags, w, s) : launch_dv<128>(p, saved, flags, w, s);
     if (e != cudaSuccess) return e;
     // heads whose decay span needs narrower windows: exact CUDA-core backward
     BwdParams q = p;

@@ -38,9 +38,6 @@
 // status word and the CTA exits cleanly).
 #include <cuda.h>
 
-#include <atomic>
-#include <chrono>
-
 #include "launch.h"
 #include "rdm_common.cuh"
 #include "tc_common.cuh"
@@ -671,19 +668,6 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
 
 // ------------------------------------------------------------------ host side
 
-int sm_count() {
-    static int cache[64];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 1;
-    if (cache[dev] == 0) {
-        int n = 0;
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
-            n = 1;
-        cache[dev] = n;
-    }
-    return cache[dev];
-}
-
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
 struct SegPlan {
@@ -733,16 +717,6 @@ SegPlan choose_plan(const SeqParams& p, bool allow_seg) {
     return best;
 }
 
-// Tag of one launch for the segment flags: distinct for every launch of the
-// process, and seeded from the clock so that it is unlikely to equal what a
-// reused workspace still holds.
-unsigned next_epoch() {
-    static std::atomic<unsigned> counter{
-        (unsigned)std::chrono::steady_clock::now().time_since_epoch().count() | 1u};
-    const unsigned e = counter.fetch_add(1u) + 1u;
-    return e == 0 ? 1u : e;
-}
-
 template <int DK, int DVT>
 cudaError_t launch_cfg(const SeqParams& p, SegPlan plan, cudaStream_t s) {
     FwdKernelArgs a;
@@ -762,7 +736,7 @@ cudaError_t launch_cfg(const SeqParams& p, SegPlan plan, cudaStream_t s) {
     const unsigned units = (unsigned)(BH * (p.dv / DVT));
     uint8_t* ws = static_cast<uint8_t*>(p.ws);
     a.seg.P = plan.P;
-    a.seg.epoch = next_epoch();
+    a.seg.epoch = next_launch_tag();
     a.seg.st = plan.P > 1 ? reinterpret_cast<float*>(ws) : nullptr;
     a.seg.ld = plan.P > 1 ? reinterpret_cast<float*>(ws + plan.st_bytes) : nullptr;
     a.seg.flag = plan.P > 1 ? reinterpret_cast<unsigned*>(ws + plan.st_bytes + plan.ld_bytes) : nullptr;

@@ -1,8 +1,12 @@
 // tmap.cu -- host construction of TMA tensor maps through the driver entry
-// point (no link-time dependency on libcuda).
+// point (no link-time dependency on libcuda), and the small host helpers the
+// sequence-segmented launches share (SM count, launch tags).
 #include <cudaTypedefs.h>
 
 #include "launch.h"
+
+#include <atomic>
+#include <chrono>
 
 namespace rdm {
 namespace {
@@ -35,6 +39,26 @@ bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t n0, uint64_t
                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+int sm_count() {
+    static int cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 1;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+            n = 1;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+unsigned next_launch_tag() {
+    static std::atomic<unsigned> counter{
+        (unsigned)std::chrono::steady_clock::now().time_since_epoch().count() | 1u};
+    const unsigned e = counter.fetch_add(1u) + 1u;
+    return e == 0 ? 1u : e;
 }
 
 }  // namespace rdm

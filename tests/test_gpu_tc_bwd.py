@@ -1,8 +1,8 @@
 """GPU parity of the tensor-core chunked backward against the fp64 oracle,
 through the C ABI: every gradient (q, k, v, g, tau, beta_hat, S_0), with and
 without an upstream dS_T, with saved or recomputed chunk states, ragged tails,
-wide-decay heads (exact re-run path) and the full training workload (sampled
-heads)."""
+wide-decay heads (exact re-run path), sequences cut into segments (one CTA
+each) and the full training workload (sampled heads)."""
 import pytest
 import torch
 
@@ -55,6 +55,34 @@ def test_tc_backward_matches_simt(cuda_ok):
     b = gpu_bwd(x, impl="simt", use_saved=False)
     for n in GR:
         assert_close(a[n], b[n], TOL, f"tc vs simt {n}")
+
+
+@pytest.mark.parametrize("dv", [64, 128])
+@pytest.mark.parametrize("T", [64 * 8, 64 * 13 + 21])
+def test_tc_backward_segmented(cuda_ok, dv, T):
+    """Two heads leave most SMs idle: each sequence is cut into segments whose R
+    maps and decay-gradient carries are folded across CTAs.  Every gradient
+    against the oracle, with and without dS_T, and against the exact path."""
+    x = draw_sequence(1, 2, T, 64, dv, torch.bfloat16, seed=4000 + T + dv, s0_std=0.1,
+                      with_dO=True)
+    dST = 0.1 * torch.randn(1, 2, 64, dv, generator=torch.Generator().manual_seed(T + 1))
+    g1 = gpu_bwd(x, dST)
+    check(x, dST, g1, "segmented, dST given")
+    check(x, None, gpu_bwd(x, None, use_saved=False), "segmented, no dST, states recomputed")
+    g2 = gpu_bwd(x, dST, impl="simt", use_saved=False)
+    for n in GR:
+        assert_close(g1[n], g2[n], TOL, f"segmented vs exact {n}")
+
+
+def test_tc_backward_segmented_wide_decay(cuda_ok):
+    """A head with a too-wide chunk in one segment only: the whole head is re-run
+    exactly, the other head keeps the segmented result."""
+    x = draw_sequence(1, 2, 64 * 10 + 3, 64, 128, torch.bfloat16, seed=17, s0_std=0.1,
+                      with_dO=True)
+    x["g"] = x["g"].float()
+    x["g"][:, 1, 64 * 7:64 * 8] *= 40.0
+    x["g"] = x["g"].clamp(min=0.05).to(torch.bfloat16)
+    check(x, None, gpu_bwd(x), "segmented, one wide chunk")
 
 
 @pytest.mark.parametrize("scale", [3.0, 40.0])
