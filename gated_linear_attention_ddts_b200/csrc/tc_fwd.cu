@@ -275,7 +275,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             if (!mbar_wait(&sm.raw_full[st], (li / NS) & 1, fail, kWaitLimit)) break;
             const uint8_t* raw = sm.raw[st];
             const int nval = min(C, T - c * C);
-            float b[SEGT][8], bf[8], bl[8];
+            // log2(alpha_hat) of my tokens is kept from the scan for the operand pass
+            // when registers allow (d_k = 64); otherwise that pass re-reads g and tau
+            constexpr bool kKeepLah = SEGT <= 2;
+            float b[SEGT][8], bf[8], bl[8], lah2[kKeepLah ? SEGT : 1][8];
             // window-relative inclusive running sum of log(alpha) over my tokens, and
             // b at the first / last valid token of my window (W in {64, 16})
             auto scan = [&](int W) {
@@ -288,6 +291,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                     for (int e = 0; e < 8; ++e) {
                         const float la = (tb + u < nval) ? log_alpha(g8[e], t8[e]) : 0.0f;
                         b[u][e] = (u == 0 || W == 1) ? la : b[u - 1][e] + la;
+                        if constexpr (kKeepLah)
+                            lah2[u][e] = t8[e] == 0.0f ? 0.0f : t8[e] * lg2_fast(g8[e]);
                     }
                 }
                 if (W == 1) return;
@@ -378,27 +383,33 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
 #pragma unroll
                 for (int u = 0; u < SEGT; ++u) {
                     const int t = tb + u;
-                    float k8[8], g8[8], t8[8], ok[8];
+                    float k8[8], lah[8], ok[8];
                     unpack8(*reinterpret_cast<const uint4*>(raw + 1 * KB * kBox + off_raw(t, cg)), k8);
-                    unpack8(*reinterpret_cast<const uint4*>(raw + 2 * KB * kBox + off_raw(t, cg)), g8);
-                    unpack8(*reinterpret_cast<const uint4*>(raw + 3 * KB * kBox + off_raw(t, cg)), t8);
+                    if constexpr (kKeepLah) {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) lah[e] = lah2[u][e];
+                    } else {
+                        float g8[8], t8[8];
+                        unpack8(*reinterpret_cast<const uint4*>(raw + 2 * KB * kBox + off_raw(t, cg)), g8);
+                        unpack8(*reinterpret_cast<const uint4*>(raw + 3 * KB * kBox + off_raw(t, cg)), t8);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) lah[e] = t8[e] == 0.0f ? 0.0f : t8[e] * lg2_fast(g8[e]);
+                    }
                     if (p2) {
                         float q8[8], oq[8];
                         unpack8(*reinterpret_cast<const uint4*>(raw + 0 * KB * kBox + off_raw(t, cg)), q8);
 #pragma unroll
                         for (int e = 0; e < 8; ++e) {
                             const float d = fmaf(b[u][e], kLog2e, -mL[e]);
-                            const float lah = t8[e] == 0.0f ? 0.0f : t8[e] * lg2_fast(g8[e]);
                             oq[e] = q8[e] * ex2_fast(d);
-                            ok[e] = k8[e] * ex2_fast(lah - d);
+                            ok[e] = k8[e] * ex2_fast(lah[e] - d);
                         }
                         *reinterpret_cast<uint4*>(sm.qt[ob] + off_qk(t, cg * 8)) = pack8(oq);
                     } else {
 #pragma unroll
                         for (int e = 0; e < 8; ++e) {
                             const float d = fmaf(b[u][e], kLog2e, -mL[e]);
-                            const float lah = t8[e] == 0.0f ? 0.0f : t8[e] * lg2_fast(g8[e]);
-                            ok[e] = k8[e] * ex2_fast(lah - d);
+                            ok[e] = k8[e] * ex2_fast(lah[e] - d);
                         }
                     }
                     *reinterpret_cast<uint4*>(sm.kt[ob] + off_qk(t, cg * 8)) = pack8(ok);
