@@ -62,7 +62,8 @@ struct Cfg {
     static constexpr int NB = 2;                   // operand buffers
     static constexpr int KB = DK / 64;             // boxes per key-side tile
     static constexpr int VB = DVT / 64;            // boxes per value-side tile
-    static constexpr int RAW = (4 * KB + 2 * VB) * kBox;
+    static constexpr int RAWK = 4 * KB * kBox;  // q, k, g, tau (NS stages)
+    static constexpr int RAWV = 2 * VB * kBox;  // v, beta (one stage, released early)
     static constexpr int G = DK / 8;               // 8-channel groups
     // A | dS | O (double-buffered: the epilogue reads O of one chunk while the
     // tensor core writes the next)
@@ -76,7 +77,9 @@ enum { kInfoChunk, kInfoW0, kInfoW1, kInfoLast, kInfoPhase, kInfoP1Last, kInfoN 
 template <int DK, int DVT>
 struct alignas(1024) FwdSmem {
     using K = Cfg<DK, DVT>;
-    uint8_t raw[K::NS][K::RAW];
+    uint8_t raw[K::NS][K::RAWK];
+    uint8_t rawv[K::RAWV];
+    uint8_t ostage[C * DVT * 2];  // o tile for the TMA store, 128B-swizzled boxes
     uint8_t qt[K::NB][K::G * kQK];
     uint8_t kt[K::NB][K::G * kQK];
     uint8_t vh[K::NB][C * DVT * 2];
@@ -84,7 +87,7 @@ struct alignas(1024) FwdSmem {
     uint8_t shat[DK * DVT * 2];
     float em[K::NB][DK], cf[K::NB][DK], gm[K::NB][DK];
     int info[K::NB][kInfoN];
-    uint64_t raw_full[K::NS], raw_empty[K::NS], ops_full[K::NB], ops_empty[K::NB];
+    uint64_t raw_full[K::NS], raw_empty[K::NS], v_full, v_empty, ops_full[K::NB], ops_empty[K::NB];
     uint64_t mma1_done, as_free, abf_full, mmao_done[2], o_free[2];
     int need16[2], need1[2];
     uint32_t tmem_base;
@@ -103,7 +106,7 @@ struct SegArgs {
 };
 
 struct FwdKernelArgs {
-    CUtensorMap mq, mk, mg, mt, mv, mb;
+    CUtensorMap mq, mk, mg, mt, mv, mb, mo;
     SeqParams p;
     SegArgs seg;
 };
@@ -139,6 +142,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             mbar_init(&sm.raw_full[s], 1);
             mbar_init(&sm.raw_empty[s], kGateWarps);
         }
+        mbar_init(&sm.v_full, 1);
+        mbar_init(&sm.v_empty, kGateWarps);
         for (int b = 0; b < NB; ++b) {
             mbar_init(&sm.ops_full[b], kGateWarps);
             mbar_init(&sm.ops_empty[b], 1 + kEpiWarps);
@@ -160,7 +165,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
     }
     if (warp == kProdWarp && lane == 0) {
         prefetch_tmap(&A.mq); prefetch_tmap(&A.mk); prefetch_tmap(&A.mg);
-        prefetch_tmap(&A.mt); prefetch_tmap(&A.mv); prefetch_tmap(&A.mb);
+        prefetch_tmap(&A.mt); prefetch_tmap(&A.mv); prefetch_tmap(&A.mb); prefetch_tmap(&A.mo);
     }
     tc_fence_before();
     __syncthreads();
@@ -171,14 +176,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
     if (warp == kProdWarp) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            int issued = 0;
+            int issued = 0, issued_v = 0;
             for (int li = 0; li < nL; ++li) {
                 const int st = li % NS, c = pass_chunk(li);
                 const bool p2 = pass_p2(li);
                 if (li >= NS && !mbar_wait(&sm.raw_empty[st], ((li / NS) - 1) & 1, fail, kWaitLimit))
                     break;
                 // the state-only pass does not read q
-                mbar_expect_tx(&sm.raw_full[st], K::RAW - (p2 ? 0 : KB * kBox));
+                mbar_expect_tx(&sm.raw_full[st], K::RAWK - (p2 ? 0 : KB * kBox));
                 uint8_t* raw = sm.raw[st];
                 for (int kb = 0; kb < KB; ++kb) {
                     if (p2)
@@ -187,15 +192,19 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                     tma_load_3d(raw + (2 * KB + kb) * kBox, &A.mg, &sm.raw_full[st], 64 * kb, c * C, bh);
                     tma_load_3d(raw + (3 * KB + kb) * kBox, &A.mt, &sm.raw_full[st], 64 * kb, c * C, bh);
                 }
-                for (int vb = 0; vb < VB; ++vb) {
-                    tma_load_3d(raw + (4 * KB + vb) * kBox, &A.mv, &sm.raw_full[st], j0 + 64 * vb, c * C, bh);
-                    tma_load_3d(raw + (4 * KB + VB + vb) * kBox, &A.mb, &sm.raw_full[st], j0 + 64 * vb, c * C, bh);
-                }
                 ++issued;
+                if (li >= 1 && !mbar_wait(&sm.v_empty, (li - 1) & 1, fail, kWaitLimit)) break;
+                mbar_expect_tx(&sm.v_full, K::RAWV);
+                for (int vb = 0; vb < VB; ++vb) {
+                    tma_load_3d(sm.rawv + vb * kBox, &A.mv, &sm.v_full, j0 + 64 * vb, c * C, bh);
+                    tma_load_3d(sm.rawv + (VB + vb) * kBox, &A.mb, &sm.v_full, j0 + 64 * vb, c * C, bh);
+                }
+                ++issued_v;
             }
             // never leave the CTA with copies in flight
             for (int li = issued - NS < 0 ? 0 : issued - NS; li < issued; ++li)
                 drain_wait(&sm.raw_full[li % NS], (li / NS) & 1);
+            if (issued_v > 0) drain_wait(&sm.v_full, (issued_v - 1) & 1);
         }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
@@ -344,14 +353,19 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                 }
             }
             // Vh = beta_hat * v for the rows of [w0, w1), zero elsewhere
+            bool have_v = false;
             auto write_vh = [&](int ob, int w0, int w1) {
+                if (!have_v) {
+                    have_v = mbar_wait(&sm.v_full, li & 1, fail, kWaitLimit);
+                    if (!have_v) return;
+                }
 #pragma unroll
                 for (int it = 0; it < VIT; ++it) {
                     const int jg = gt / TPG, t = (gt % TPG) + TPG * it;
                     const bool in = t >= w0 && t < w1;
                     float v8[8], b8[8], o8[8];
-                    unpack8(*reinterpret_cast<const uint4*>(raw + 4 * KB * kBox + off_raw(t, jg)), v8);
-                    unpack8(*reinterpret_cast<const uint4*>(raw + (4 * KB + VB) * kBox + off_raw(t, jg)), b8);
+                    unpack8(*reinterpret_cast<const uint4*>(sm.rawv + off_raw(t, jg)), v8);
+                    unpack8(*reinterpret_cast<const uint4*>(sm.rawv + VB * kBox + off_raw(t, jg)), b8);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) o8[e] = in ? v8[e] * b8[e] : 0.0f;
                     *reinterpret_cast<uint4*>(sm.vh[ob] + off_vh(t, jg * 8)) = pack8(o8);
@@ -469,7 +483,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                 if (!ok_loop) break;
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.raw_empty[st]);
+            if (lane == 0) {
+                mbar_arrive(&sm.raw_empty[st]);
+                mbar_arrive(&sm.v_empty);
+            }
             if (*fail) break;
         }
     } else {
@@ -549,26 +566,41 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             named_bar(kBarEpi, 32 * kEpiWarps);
             if (threadIdx.x == 0) st_release_gpu(&sg.flag[u], sg.epoch);
         };
-        // o rows [w0, w1) of chunk c from the O buffer of o-item `io`
+        // o rows [w0, w1) of chunk c from the O buffer of o-item `io`.  A whole
+        // chunk goes out through the staging tile and one TMA store (rows past T
+        // are clipped by the TMA unit); a window writes its rows directly.
         auto store_o = [&](int io, int c, int w0, int w1) -> bool {
             const int obuf = io & 1;
             if (!mbar_wait(&sm.mmao_done[obuf], (io >> 1) & 1, fail, kWaitLimit)) return false;
             tc_fence_after();
-            const bool st_row = tA >= w0 && tA < w1;
-            __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.o) +
-                                  ((size_t)bh * T + (size_t)c * C + tA) * p.dv + j0 + oc0;
-            {
-                float v[OC];
-                ld_cols(K::COL_O + obuf * DVT, v, false);
-                if (st_row) {
-#pragma unroll
-                    for (int s8 = 0; s8 < OC / 8; ++s8)
-                        reinterpret_cast<uint4*>(orow)[s8] = pack8(v + 8 * s8);
-                }
-            }
+            float v[OC];
+            ld_cols(K::COL_O + obuf * DVT, v, false);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.o_free[obuf]);
+            const bool whole = w0 == 0 && w1 == min(C, T - c * C);
+            if (whole) {
+                // the previous store has read the staging tile
+                if (threadIdx.x == 0) bulk_wait_read_all();
+                named_bar(kBarEpi, 32 * kEpiWarps);
+#pragma unroll
+                for (int s8 = 0; s8 < OC / 8; ++s8)
+                    *reinterpret_cast<uint4*>(sm.ostage + off_raw(tA, (oc0 >> 3) + s8)) = pack8(v + 8 * s8);
+                fence_proxy_async_smem();
+                named_bar(kBarEpi, 32 * kEpiWarps);
+                if (threadIdx.x == 0) {
+#pragma unroll
+                    for (int vb = 0; vb < VB; ++vb)
+                        tma_store_3d(&A.mo, sm.ostage + vb * kBox, j0 + 64 * vb, c * C, bh);
+                    bulk_commit();
+                }
+            } else if (tA >= w0 && tA < w1) {
+                __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.o) +
+                                      ((size_t)bh * T + (size_t)c * C + tA) * p.dv + j0 + oc0;
+#pragma unroll
+                for (int s8 = 0; s8 < OC / 8; ++s8)
+                    reinterpret_cast<uint4*>(orow)[s8] = pack8(v + 8 * s8);
+            }
             return true;
         };
         bool ok_run = true;
@@ -660,6 +692,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             }
             ++item;
         }
+        if (threadIdx.x == 0) bulk_wait_all();  // the o stores have landed
         if (!*fail && p.ST && seg == P - 1) {
             float4* dst = reinterpret_cast<float4*>(p.ST + ((size_t)bh * DK + iS) * p.dv + j0 + sc0);
 #pragma unroll
@@ -738,7 +771,8 @@ cudaError_t launch_cfg(const SeqParams& p, SegPlan plan, cudaStream_t s) {
         !make_tmap_bf16_3d(&a.mg, p.g, p.dk, p.T, BH, 64, 64) ||
         !make_tmap_bf16_3d(&a.mt, p.tau, p.dk, p.T, BH, 64, 64) ||
         !make_tmap_bf16_3d(&a.mv, p.v, p.dv, p.T, BH, 64, 64) ||
-        !make_tmap_bf16_3d(&a.mb, p.beta, p.dv, p.T, BH, 64, 64))
+        !make_tmap_bf16_3d(&a.mb, p.beta, p.dv, p.T, BH, 64, 64) ||
+        !make_tmap_bf16_3d(&a.mo, p.o, p.dv, p.T, BH, 64, 64))
         return cudaErrorInvalidValue;
     const size_t smem = sizeof(FwdSmem<DK, DVT>) + 1024;
     auto kern = tc_fwd_kernel<DK, DVT>;
