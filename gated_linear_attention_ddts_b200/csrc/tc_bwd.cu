@@ -56,7 +56,11 @@ constexpr int kGateWarps = 8;  // one 8-channel group each
 constexpr int kThreads = 32 * (4 + kGateWarps + 2);
 constexpr int kEpiWarp0 = 0, kGateWarp0 = 4, kProdWarp = 4 + kGateWarps, kMmaWarp = 5 + kGateWarps;
 constexpr int kBarEpi = 3;  // the four epilogue warps
-constexpr int kStg = 68;     // row stride (floats) of the dQ / dK staging tiles
+constexpr int kStg = 68;
+// row stride (floats) of the chunk-start state copied into shared memory: a
+// 16-byte skew per row keeps the S_hat conversion free of bank conflicts
+template <int DV>
+constexpr int kSpStride = DV + 4;     // row stride (floats) of the dQ / dK staging tiles
 
 template <int DV>
 struct BCfg {
@@ -77,9 +81,12 @@ struct alignas(1024) BwdSmem {
     uint8_t ktl[8 * kQK];      // pair products of dQ and dK reach ~16 mantissa bits
     uint8_t vh[C * DV * 2];    // [s][j], column groups 1024 B apart
     uint8_t dot[C * DV * 2];   // [t][j]
-    // A, B, S_hat and R_hat operands of the second MMA group; once that group
-    // has completed, the same bytes hold the fp32 dQ / dK staging tiles
+    // A, B and R_hat operands of the second MMA group; once that group has
+    // completed, the same bytes hold the fp32 dQ / dK staging tiles; before the
+    // first stage of the epilogue writes A, they hold the chunk-start state
+    // S_prev (fp32) that the gate warps turn into S_hat
     union {
+        float sprev[DK * kSpStride<DV>];
         struct {
             uint8_t abf[C * C * 2];       // [t][s]
             uint8_t bmb[C * C * 2];       // [t][s]
@@ -92,8 +99,8 @@ struct alignas(1024) BwdSmem {
     uint8_t shat[DK * DV * 2];  // [i][j], e^m S_prev (written by the gate warps)
     float em[DK], cf[DK], gm[DK], fin[DK], carry[DK];
     float bdiag[C];  // B_tt = vhat_t . dO_t (the diagonal kept out of the dQ / dK MMAs)
-    uint64_t raw_full, raw_empty, ops_full, shat_full, ops_empty, g1_done, g2_ready, tm1_free,
-        g2_done, tm2_free, post_ready, post_done;
+    uint64_t raw_full, raw_empty, sp_full, ops_full, shat_full, ops_empty, g1_done, g2_ready,
+        tm1_free, g2_done, tm2_free, post_ready, post_done;
     uint32_t tmem_base;
     int fail;
 };
@@ -148,6 +155,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
     if (threadIdx.x == 0) {
         mbar_init(&sm.raw_full, 1);
         mbar_init(&sm.raw_empty, kGateWarps);
+        mbar_init(&sm.sp_full, 1);
         mbar_init(&sm.ops_full, kGateWarps);
         mbar_init(&sm.shat_full, kGateWarps);
         mbar_init(&sm.ops_empty, 1);
@@ -182,7 +190,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
     if (warp == kProdWarp) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            int issued = 0;
+            int issued = 0, issued_sp = 0;
             for (int li = 0; li < nL; ++li) {
                 const int c = pass_chunk(li);
                 const bool p2 = pass_p2(li);
@@ -201,8 +209,18 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                     tma_load_3d(sm.raw + K::OFF_DO + vb * kBox, &A.mdo, &sm.raw_full, 64 * vb, c * C, bh);
                 }
                 ++issued;
+                if (p2) {
+                    // chunk-start state, row by row into the skewed layout (the union
+                    // is free: the previous full pass has finished its last stage)
+                    const float* Sp = p.saved + ((size_t)bh * NC + c) * DK * DV;
+                    mbar_expect_tx(&sm.sp_full, DK * DV * 4);
+                    for (int i = 0; i < DK; ++i)
+                        bulk_load(sm.u.sprev + i * kSpStride<DV>, Sp + (size_t)i * DV, DV * 4, &sm.sp_full);
+                    ++issued_sp;
+                }
             }
             if (issued > 0) drain_wait(&sm.raw_full, (issued - 1) & 1);
+            if (issued_sp > 0) drain_wait(&sm.sp_full, (issued_sp - 1) & 1);
         }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
@@ -455,10 +473,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             if (lane == 0) mbar_arrive(&sm.ops_full);
             // S_hat = diag(e^m) S_prev for this warp's rows (channels), while the
             // first MMA group runs
+            if (!mbar_wait(&sm.sp_full, i2 & 1, fail, kWaitLimit)) break;
 #pragma unroll
             for (int gi = 0; gi < GW; ++gi) {
                 const int i = (gw * GW + gi) * 8 + (lane >> 2);
-                const float* Sp = p.saved + (((size_t)bh * NC + c) * DK + i) * DV;
+                const float* Sp = sm.u.sprev + i * kSpStride<DV>;
                 constexpr int CPT = DV / 4;  // 8 rows x DV columns over 32 lanes
                 const int c0 = (lane & 3) * CPT;
                 const float emr = sm.em[i];
@@ -673,6 +692,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 }
                 continue;
             }
+            // the gate warps have read S_prev out of the union (and staged S_hat)
+            if (!mbar_wait(&sm.shat_full, i2 & 1, fail, kWaitLimit)) break;
             // A and B -> causal mask -> bf16 operands (row t = r, columns s = 32 hf + e)
 #pragma unroll
             for (int which = 0; which < 2; ++which) {

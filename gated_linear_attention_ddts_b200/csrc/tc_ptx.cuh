@@ -310,6 +310,13 @@ __device__ __forceinline__ uint32_t map_to_rank(const void* p, uint32_t rank) {
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
     return r;
 }
+// Bulk copy global -> shared (this CTA), completion counted as transaction
+// bytes on `bar`.  Both addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
+}
 // Bulk copy shared::cta (this CTA) -> shared::cluster (another CTA), completion
 // counted as transaction bytes on the destination CTA's mbarrier.
 __device__ __forceinline__ void bulk_copy_to_rank(uint32_t dst_cluster_addr, const void* src,
