@@ -347,6 +347,21 @@ def cpu_oracle_rate(w, min_seconds=10.0, max_seconds=30.0, heads=None):
 
 
 # ------------------------------------------------------------------ main
+def max_over_ranks(values, dist=None, device="cpu"):
+    """Element-wise maximum of `values` over all ranks of the process group
+    (the values themselves without one)."""
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def weak_scaling_value(tokens_per_rank, world, ms_per_step):
+    """Whole-job tokens/s: every rank processes its own batch in the step time
+    of the slowest rank."""
+    return tokens_per_rank * world / (ms_per_step / 1e3)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -410,15 +425,10 @@ def main():
     flush = lambda: flush_buf.zero_()
 
     times, clocks, e2e_times, h2d, d2h = run_headline(rdm, w, K, W, dev, flush, barrier, pk, rank)
-    total = torch.tensor([sum(times)], device=dev, dtype=torch.float64)
-    e2e_total = torch.tensor([sum(e2e_times) / len(e2e_times)], device=dev, dtype=torch.float64)
-    if dist:
-        dist.all_reduce(total, op=dist.ReduceOp.MAX)
-        dist.all_reduce(e2e_total, op=dist.ReduceOp.MAX)
-    ms = total.item() / K
+    total, e2e_ms = max_over_ranks([sum(times), sum(e2e_times) / len(e2e_times)], dist, dev)
+    ms = total / K
     tokens = w.B * w.T * world
-    value = tokens / (ms / 1e3)
-    e2e_ms = e2e_total.item()
+    value = weak_scaling_value(w.B * w.T, world, ms)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": W, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -428,7 +438,8 @@ def main():
         "roofline": roofline(fwd_bytes(w, False), chunk_flops_fwd(w), ms, pk,
                              ncu_traffic("tc_fwd_kernel", ["tc_fwd.cu"], 1)),
         "clocks": clocks,
-        "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
+        "e2e": {"value": weak_scaling_value(w.B * w.T, world, e2e_ms), "unit": "tokens/s",
+                "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": K,
     }
