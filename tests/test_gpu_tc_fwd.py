@@ -84,6 +84,31 @@ def test_tc_g_zero_and_tau_zero(cuda_ok):
     assert_close(ST, S[:, :, -1], TOL, "tau=0 S_T")
 
 
+@pytest.mark.parametrize("dk,dv", [(64, 128), (16, 32)])
+def test_chunk_size_invariance(cuda_ok, dk, dv):
+    """The result does not depend on the chunk size asked for: every allowed
+    value against the default (the tensor-core path takes chunks of 64, cut
+    into windows of 16 or 1 token when the decay needs it; other sizes run the
+    exact path) and against the oracle.  Wide decay forces the windows."""
+    x = draw_sequence(1, 2, 300, dk, dv, torch.bfloat16, seed=61, s0_std=0.1)
+    x["g"] = (x["g"].float() * 6.0).to(torch.bfloat16)
+    d = {n: x[n].cuda() for n in SEQ}
+    S0 = x["S0"].cuda()
+    ref = None
+    o_ref, S_ref = oracle.fwd(*(x[n] for n in SEQ), x["S0"])
+    for chunk in (64, 16, 32, 128):
+        o, ST = rdm.rdm_ddts_fwd(*(d[n] for n in SEQ), S0, chunk=chunk, return_state=True)
+        torch.cuda.synchronize()
+        assert rdm.rdm_ddts_sync_status() == rdm.RDM_OK
+        assert_close(o, o_ref, TOL, f"o chunk {chunk}")
+        assert_close(ST, S_ref, TOL, f"S_T chunk {chunk}")
+        if ref is None:
+            ref = (o.float().cpu().numpy(), ST.cpu().numpy())
+        else:
+            assert_close(o, ref[0], TOL, f"o chunk {chunk} vs 64")
+            assert_close(ST, ref[1], TOL, f"S_T chunk {chunk} vs 64")
+
+
 def test_tc_split_invariance(cuda_ok):
     """fwd(T1) then fwd(T2, S_0 = S_T1) equals fwd(T1 + T2) on the GPU."""
     x = draw_sequence(2, 3, 320, 64, 128, torch.bfloat16, seed=21, s0_std=0.1)
