@@ -13,6 +13,13 @@ bullet and Q2 on the fixed-size recurrent state):
     alpha_t = exp(-g_t * tau_t),  alpha_hat_t = g_t ** tau_t
     S_t = diag(alpha_t) S_{t-1} + (alpha_hat_t * k_t)(beta_hat_t * v_t)^T
     o_t = S_t^T q_t
+
+With ``preact=True`` the gate inputs are taken before their activations (the
+same page names a selection gate g_t, a temperature gate tau_t and a low-rank
+beta_hat_t without printing the activations; the reading used here is
+g = softplus(.), which keeps g >= 0, and tau = sigmoid(.), beta_hat =
+sigmoid(.)): they are activated element-wise in fp64 around the same token
+loop, and the backward applies the chain rule to the three gradients.
 """
 from __future__ import annotations
 
@@ -81,10 +88,29 @@ def _p(a):
     return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
 
 
-def fwd(q, k, v, g, tau, beta, S0=None, nthreads=None, lib=None):
+def softplus(x):
+    """log(1 + exp(x)) in float64."""
+    return np.logaddexp(0.0, x)
+
+
+def sigmoid(x):
+    """1 / (1 + exp(-x)) in float64 (each branch evaluated where it cannot overflow)."""
+    e = np.exp(-np.abs(x))
+    return np.where(x >= 0, 1.0 / (1.0 + e), e / (1.0 + e))
+
+
+def activate(g_pre, tau_pre, beta_pre):
+    """Gate activations: g = softplus, tau = sigmoid, beta_hat = sigmoid."""
+    return softplus(g_pre), sigmoid(tau_pre), sigmoid(beta_pre)
+
+
+def fwd(q, k, v, g, tau, beta, S0=None, nthreads=None, lib=None, preact=False):
     """Token-by-token forward.  q,k,g,tau [B,H,T,dk]; v,beta [B,H,T,dv];
-    S0 [B,H,dk,dv] or None (zeros).  Returns (o [B,H,T,dv], S_T [B,H,dk,dv])."""
+    S0 [B,H,dk,dv] or None (zeros).  Returns (o [B,H,T,dv], S_T [B,H,dk,dv]).
+    preact: g, tau, beta are pre-activations (see the module docstring)."""
     q, k, v, g, tau, beta, S0 = map(_f64, (q, k, v, g, tau, beta, S0))
+    if preact:
+        g, tau, beta = activate(g, tau, beta)
     B, H, T, dk = q.shape
     dv = v.shape[-1]
     o = np.zeros((B, H, T, dv))
@@ -96,9 +122,19 @@ def fwd(q, k, v, g, tau, beta, S0=None, nthreads=None, lib=None):
     return o, ST
 
 
-def bwd(q, k, v, g, tau, beta, S0, dO, dST=None, nthreads=None, lib=None):
-    """Reverse mode of the token loop.  Returns dict dq, dk, dv, dg, dtau, dbeta, dS0."""
+def bwd(q, k, v, g, tau, beta, S0, dO, dST=None, nthreads=None, lib=None, preact=False):
+    """Reverse mode of the token loop.  Returns dict dq, dk, dv, dg, dtau, dbeta, dS0.
+    preact: g, tau, beta are pre-activations and dg, dtau, dbeta are the gradients
+    with respect to them (d softplus = sigmoid, d sigmoid = s (1 - s))."""
     q, k, v, g, tau, beta, S0, dO, dST = map(_f64, (q, k, v, g, tau, beta, S0, dO, dST))
+    if preact:
+        g_pre = g
+        g, tau, beta = activate(g, tau, beta)
+        out = bwd(q, k, v, g, tau, beta, S0, dO, dST, nthreads=nthreads, lib=lib)
+        out["dg"] *= sigmoid(g_pre)
+        out["dtau"] *= tau * (1.0 - tau)
+        out["dbeta"] *= beta * (1.0 - beta)
+        return out
     B, H, T, dk = q.shape
     dv = v.shape[-1]
     out = {n: np.zeros(q.shape) for n in ("dq", "dk", "dg", "dtau")}

@@ -240,7 +240,73 @@ def check_bwd_autograd(lib=None, seed=8):
         close(gr[gn], ref[n], 1e-11, f"autograd {gn}")
 
 
+# ------------------------------------------------- gate pre-activations (fused mode)
+def check_preact_matches_torch_activations(lib=None, seed=9):
+    """preact=True equals the plain recurrence on inputs activated by torch's own
+    softplus / sigmoid (a library routine, independent of the oracle)."""
+    import torch
+    rng = np.random.default_rng(seed)
+    x = rand_inputs(rng, 2, 2, 13, 3, 4)
+    pre = dict(g=rng.normal(-1.0, 1.5, x["g"].shape), tau=rng.normal(0.0, 2.0, x["tau"].shape),
+               beta=rng.normal(0.0, 2.0, x["beta"].shape))
+    pre["g"][0, 0, 0, 0], pre["tau"][0, 0, 0, 0] = 40.0, -40.0   # far tails of both activations
+    t = {n: torch.from_numpy(pre[n]) for n in pre}
+    act = dict(g=torch.nn.functional.softplus(t["g"]).numpy(), tau=torch.sigmoid(t["tau"]).numpy(),
+               beta=torch.sigmoid(t["beta"]).numpy())
+    o1, S1 = oracle.fwd(x["q"], x["k"], x["v"], pre["g"], pre["tau"], pre["beta"], x["S0"],
+                        lib=lib, preact=True)
+    o2, S2 = oracle.fwd(x["q"], x["k"], x["v"], act["g"], act["tau"], act["beta"], x["S0"], lib=lib)
+    close(o1, o2, 1e-12, "preact o")
+    close(S1, S2, 1e-12, "preact S_T")
+
+
+def check_preact_special_values(lib=None):
+    """softplus(0) = ln 2 and sigmoid(0) = 1/2 exactly: zero pre-activations give
+    g = ln 2, tau = beta_hat = 1/2 everywhere."""
+    rng = np.random.default_rng(10)
+    x = rand_inputs(rng, 1, 1, 5, 2, 3)
+    z = lambda a: np.zeros_like(a)
+    o1, S1 = oracle.fwd(x["q"], x["k"], x["v"], z(x["g"]), z(x["tau"]), z(x["beta"]), x["S0"],
+                        lib=lib, preact=True)
+    f = lambda a, c: np.full_like(a, c)
+    o2, S2 = oracle.fwd(x["q"], x["k"], x["v"], f(x["g"], math.log(2.0)), f(x["tau"], 0.5),
+                        f(x["beta"], 0.5), x["S0"], lib=lib)
+    close(o1, o2, 1e-14, "zero pre-activations o")
+    close(S1, S2, 1e-14, "zero pre-activations S_T")
+
+
+def check_preact_bwd_finite_differences(lib=None, seed=11):
+    """Gradients with respect to the pre-activations: central differences."""
+    rng = np.random.default_rng(seed)
+    x = rand_inputs(rng, 1, 1, 6, 3, 2)
+    pre = dict(g=rng.normal(-0.5, 1.0, x["g"].shape), tau=rng.normal(0.0, 1.0, x["tau"].shape),
+               beta=rng.normal(0.0, 1.0, x["beta"].shape))
+    dO = rng.standard_normal(x["v"].shape)
+    dST = rng.standard_normal(x["S0"].shape)
+
+    def loss(p):
+        o, ST = oracle.fwd(x["q"], x["k"], x["v"], p["g"], p["tau"], p["beta"], x["S0"], lib=lib,
+                           preact=True)
+        return float(np.sum(o * dO) + np.sum(ST * dST))
+
+    gr = oracle.bwd(x["q"], x["k"], x["v"], pre["g"], pre["tau"], pre["beta"], x["S0"], dO, dST,
+                    lib=lib, preact=True)
+    h = 1e-6
+    for n, gn in (("g", "dg"), ("tau", "dtau"), ("beta", "dbeta")):
+        num = np.zeros_like(pre[n])
+        for idx in np.ndindex(pre[n].shape):
+            pp = {m: pre[m].copy() for m in pre}
+            pm = {m: pre[m].copy() for m in pre}
+            pp[n][idx] += h
+            pm[n][idx] -= h
+            num[idx] = (loss(pp) - loss(pm)) / (2 * h)
+        close(gr[gn], num, 2e-7, f"preact {gn} finite differences")
+
+
+PREACT_PINS = [check_preact_matches_torch_activations, check_preact_special_values,
+               check_preact_bwd_finite_differences]
+
 FORWARD_PINS = [check_worked_example, check_T1_closed_form, check_g_zero, check_tau_zero,
                 check_quadratic, check_linearity, check_split_and_decode]
 BACKWARD_PINS = [check_bwd_finite_differences, check_bwd_autograd]
-ALL_PINS = FORWARD_PINS + BACKWARD_PINS
+ALL_PINS = FORWARD_PINS + BACKWARD_PINS + PREACT_PINS
