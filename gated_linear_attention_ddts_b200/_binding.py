@@ -18,6 +18,9 @@ RDM_OK, RDM_ERR_INVALID_ARG, RDM_ERR_UNSUPPORTED, RDM_ERR_CUDA, RDM_ERR_TIMEOUT,
     RDM_ERR_WORKSPACE = range(6)
 RDM_F32, RDM_BF16 = 0, 1
 IMPL = {"auto": 0, "simt": 1, "tc": 2, 0: 0, 1: 1, 2: 2}
+# what g, tau, beta hold: the gates, or their pre-activations (softplus, sigmoid,
+# sigmoid applied inside; gradients then refer to the pre-activations)
+GATES = {"activated": 0, "preact": 1, 0: 0, 1: 1}
 
 _VP = ctypes.c_void_p
 _I = ctypes.c_int
@@ -28,7 +31,7 @@ class FwdArgs(ctypes.Structure):
                 ("dtype", _I), ("impl", _I),
                 ("q", _VP), ("k", _VP), ("v", _VP), ("g", _VP), ("tau", _VP), ("beta", _VP),
                 ("S0", _VP), ("o", _VP), ("ST", _VP), ("saved_states", _VP),
-                ("workspace", _VP), ("workspace_bytes", ctypes.c_size_t)]
+                ("workspace", _VP), ("workspace_bytes", ctypes.c_size_t), ("gate_inputs", _I)]
 
 
 class BwdArgs(ctypes.Structure):
@@ -38,7 +41,7 @@ class BwdArgs(ctypes.Structure):
                 ("S0", _VP), ("grad_o", _VP), ("grad_ST", _VP), ("saved_states", _VP),
                 ("grad_q", _VP), ("grad_k", _VP), ("grad_v", _VP), ("grad_g", _VP),
                 ("grad_tau", _VP), ("grad_beta", _VP), ("grad_S0", _VP),
-                ("workspace", _VP), ("workspace_bytes", ctypes.c_size_t)]
+                ("workspace", _VP), ("workspace_bytes", ctypes.c_size_t), ("gate_inputs", _I)]
 
 
 class RdmError(RuntimeError):
@@ -123,16 +126,18 @@ def rdm_ddts_saved_states_size(B, H, T, dk, dv, chunk=0) -> int:
     return int(load().rdm_ddts_saved_states_size(B, H, T, dk, dv, chunk))
 
 
-def _fwd_args(q, k, v, g, tau, beta, S0, o, ST, saved_states, ws, ws_bytes, chunk, impl):
+def _fwd_args(q, k, v, g, tau, beta, S0, o, ST, saved_states, ws, ws_bytes, chunk, impl,
+              gates="activated"):
     B, H, T, dk = q.shape
     dv = v.shape[-1]
     return FwdArgs(B, H, T, dk, dv, chunk, _dtype_code(q), IMPL[impl],
                    _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(tau), _ptr(beta), _ptr(S0), _ptr(o),
-                   _ptr(ST), _ptr(saved_states), _ptr(ws), ws_bytes)
+                   _ptr(ST), _ptr(saved_states), _ptr(ws), ws_bytes, GATES[gates])
 
 
-def rdm_ddts_fwd_workspace_size(q, k, v, g, tau, beta, *, chunk=0, impl="auto") -> int:
-    a = _fwd_args(q, k, v, g, tau, beta, None, None, None, None, None, 0, chunk, impl)
+def rdm_ddts_fwd_workspace_size(q, k, v, g, tau, beta, *, chunk=0, impl="auto",
+                                gates="activated") -> int:
+    a = _fwd_args(q, k, v, g, tau, beta, None, None, None, None, None, 0, chunk, impl, gates)
     n = load().rdm_ddts_fwd_workspace_size(ctypes.byref(a))
     if n == ctypes.c_size_t(-1).value:
         raise RdmError(RDM_ERR_INVALID_ARG, "rdm_ddts_fwd_workspace_size")
@@ -140,7 +145,8 @@ def rdm_ddts_fwd_workspace_size(q, k, v, g, tau, beta, *, chunk=0, impl="auto") 
 
 
 def rdm_ddts_fwd(q, k, v, g, tau, beta, S0=None, o=None, ST=None, saved_states=None, *,
-                 workspace=None, chunk=0, impl="auto", return_state=False, stream=None):
+                 workspace=None, chunk=0, impl="auto", return_state=False, stream=None,
+                 gates="activated"):
     """Forward over [B,H,T,D] sequences.  Allocates o (and S_T when
     return_state) with torch if not given, and the sequence-segment workspace
     when none is passed (workspace=False runs without one).  Returns
@@ -152,19 +158,20 @@ def rdm_ddts_fwd(q, k, v, g, tau, beta, S0=None, o=None, ST=None, saved_states=N
     if ST is None and return_state:
         ST = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device)
     if workspace is None:
-        need = rdm_ddts_fwd_workspace_size(q, k, v, g, tau, beta, chunk=chunk, impl=impl)
+        need = rdm_ddts_fwd_workspace_size(q, k, v, g, tau, beta, chunk=chunk, impl=impl,
+                                           gates=gates)
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device) if need else None
     elif workspace is False:
         workspace = None
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     a = _fwd_args(q, k, v, g, tau, beta, S0, o, ST, saved_states, workspace, ws_bytes, chunk,
-                  impl)
+                  impl, gates)
     _check(load().rdm_ddts_fwd(ctypes.byref(a), _stream(stream)), "rdm_ddts_fwd")
     return o, ST
 
 
 def _bwd_args(q, k, v, g, tau, beta, S0, grad_o, grad_ST, saved_states, grads, ws, ws_bytes,
-              chunk, impl):
+              chunk, impl, gates="activated"):
     B, H, T, dk = q.shape
     dv = v.shape[-1]
     return BwdArgs(B, H, T, dk, dv, chunk, _dtype_code(q), IMPL[impl],
@@ -172,13 +179,14 @@ def _bwd_args(q, k, v, g, tau, beta, S0, grad_o, grad_ST, saved_states, grads, w
                    _ptr(grad_o), _ptr(grad_ST), _ptr(saved_states),
                    *(_ptr(grads.get(n)) for n in ("dq", "dk", "dv", "dg", "dtau", "dbeta",
                                                     "dS0")),
-                   _ptr(ws), ws_bytes)
+                   _ptr(ws), ws_bytes, GATES[gates])
 
 
 def rdm_ddts_bwd_workspace_size(q, k, v, g, tau, beta, S0=None, grad_o=None, grad_ST=None,
-                                saved_states=None, *, chunk=0, impl="auto") -> int:
+                                saved_states=None, *, chunk=0, impl="auto",
+                                gates="activated") -> int:
     a = _bwd_args(q, k, v, g, tau, beta, S0, grad_o, grad_ST, saved_states, {}, None, 0,
-                  chunk, impl)
+                  chunk, impl, gates)
     n = load().rdm_ddts_bwd_workspace_size(ctypes.byref(a))
     if n == ctypes.c_size_t(-1).value:
         raise RdmError(RDM_ERR_INVALID_ARG, "rdm_ddts_bwd_workspace_size")
@@ -186,7 +194,8 @@ def rdm_ddts_bwd_workspace_size(q, k, v, g, tau, beta, S0=None, grad_o=None, gra
 
 
 def rdm_ddts_bwd(q, k, v, g, tau, beta, S0, grad_o, grad_ST=None, saved_states=None, *,
-                 grads=None, workspace=None, chunk=0, impl="auto", want_dS0=True, stream=None):
+                 grads=None, workspace=None, chunk=0, impl="auto", want_dS0=True, stream=None,
+                 gates="activated"):
     """Backward.  `grads` may hold preallocated dq, dk, dv, dg, dtau, dbeta, dS0;
     missing ones are allocated with torch, as is the workspace.  Returns the dict."""
     B, H, T, dk = q.shape
@@ -199,16 +208,16 @@ def rdm_ddts_bwd(q, k, v, g, tau, beta, S0, grad_o, grad_ST=None, saved_states=N
         grads["dS0"] = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device)
     if workspace is None:
         need = rdm_ddts_bwd_workspace_size(q, k, v, g, tau, beta, S0, grad_o, grad_ST,
-                                           saved_states, chunk=chunk, impl=impl)
+                                           saved_states, chunk=chunk, impl=impl, gates=gates)
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
     a = _bwd_args(q, k, v, g, tau, beta, S0, grad_o, grad_ST, saved_states, grads, workspace,
-                  workspace.numel() * workspace.element_size(), chunk, impl)
+                  workspace.numel() * workspace.element_size(), chunk, impl, gates)
     _check(load().rdm_ddts_bwd(ctypes.byref(a), _stream(stream)), "rdm_ddts_bwd")
     return grads
 
 
 def rdm_ddts_bwd_noalloc(q, k, v, g, tau, beta, S0, grad_o, grad_ST=None, *, grads=None,
-                         chunk=0, want_dS0=True, stream=None):
+                         chunk=0, want_dS0=True, stream=None, gates="activated"):
     """Backward through the library's own fixed scratch (no workspace
     argument).  Gradient tensors are allocated with torch if not given;
     returns the dict of gradients."""
@@ -220,7 +229,8 @@ def rdm_ddts_bwd_noalloc(q, k, v, g, tau, beta, S0, grad_o, grad_ST=None, *, gra
             grads[n] = torch.empty_like(ref)
     if want_dS0 and grads.get("dS0") is None:
         grads["dS0"] = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device)
-    a = _bwd_args(q, k, v, g, tau, beta, S0, grad_o, grad_ST, None, grads, None, 0, chunk, "simt")
+    a = _bwd_args(q, k, v, g, tau, beta, S0, grad_o, grad_ST, None, grads, None, 0, chunk, "simt",
+                  gates)
     _check(load().rdm_ddts_bwd_noalloc(ctypes.byref(a), _stream(stream)), "rdm_ddts_bwd_noalloc")
     return grads
 

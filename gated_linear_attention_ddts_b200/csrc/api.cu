@@ -55,6 +55,8 @@ rdm_status check_sizes(int B, int H, int T, int dk, int dv, int chunk, rdm_dtype
 
 int eff_chunk(int chunk) { return chunk == 0 ? 64 : chunk; }
 
+bool gates_ok(rdm_gate_inputs g) { return g == RDM_GATES_ACTIVATED || g == RDM_GATES_PREACT; }
+
 // T == 0: no tokens; S_T = S_0 (or zero), no saved states.
 rdm_status empty_sequence(int B, int H, int dk, int dv, const float* S0, float* ST,
                           cudaStream_t s) {
@@ -84,6 +86,7 @@ SeqParams fwd_params(const rdm_fwd_args* a) {
     p.q = a->q; p.k = a->k; p.v = a->v; p.g = a->g; p.tau = a->tau; p.beta = a->beta;
     p.S0 = a->S0; p.o = a->o; p.ST = a->ST; p.saved = a->saved_states;
     p.ws = a->workspace; p.ws_bytes = a->workspace ? a->workspace_bytes : 0;
+    p.preact = a->gate_inputs == RDM_GATES_PREACT;
     return p;
 }
 
@@ -98,6 +101,7 @@ BwdParams bwd_params(const rdm_bwd_args* a) {
     p.dq = a->grad_q; p.dk_ = a->grad_k; p.dv_ = a->grad_v; p.dg = a->grad_g;
     p.dtau = a->grad_tau; p.dbeta = a->grad_beta; p.dS0 = a->grad_S0;
     p.ws = a->workspace; p.ws_bytes = a->workspace_bytes;
+    p.preact = a->gate_inputs == RDM_GATES_PREACT;
     return p;
 }
 
@@ -119,6 +123,7 @@ rdm_status rdm_ddts_fwd(const rdm_fwd_args* a, rdm_stream_t stream) {
     if (!a) return RDM_ERR_INVALID_ARG;
     rdm_status st = check_sizes(a->B, a->H, a->T, a->dk, a->dv, a->chunk, a->dtype, a->impl);
     if (st != RDM_OK) return st;
+    if (!gates_ok(a->gate_inputs)) return RDM_ERR_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (!opt_aligned(a->S0) || !opt_aligned(a->ST) || !opt_aligned(a->saved_states) ||
         !opt_aligned(a->workspace))
@@ -140,7 +145,8 @@ rdm_status rdm_ddts_fwd(const rdm_fwd_args* a, rdm_stream_t stream) {
 
 size_t rdm_ddts_fwd_workspace_size(const rdm_fwd_args* a) {
     if (!a) return (size_t)-1;
-    if (check_sizes(a->B, a->H, a->T, a->dk, a->dv, a->chunk, a->dtype, a->impl) != RDM_OK)
+    if (check_sizes(a->B, a->H, a->T, a->dk, a->dv, a->chunk, a->dtype, a->impl) != RDM_OK ||
+        !gates_ok(a->gate_inputs))
         return (size_t)-1;
     if (a->T == 0) return 0;
     SeqParams p = fwd_params(a);
@@ -149,7 +155,8 @@ size_t rdm_ddts_fwd_workspace_size(const rdm_fwd_args* a) {
 
 size_t rdm_ddts_bwd_workspace_size(const rdm_bwd_args* a) {
     if (!a) return (size_t)-1;
-    if (check_sizes(a->B, a->H, a->T, a->dk, a->dv, a->chunk, a->dtype, a->impl) != RDM_OK)
+    if (check_sizes(a->B, a->H, a->T, a->dk, a->dv, a->chunk, a->dtype, a->impl) != RDM_OK ||
+        !gates_ok(a->gate_inputs))
         return (size_t)-1;
     if (a->T == 0) return 0;
     BwdParams p = bwd_params(a);
@@ -161,6 +168,7 @@ rdm_status rdm_ddts_bwd(const rdm_bwd_args* a, rdm_stream_t stream) {
     if (!a) return RDM_ERR_INVALID_ARG;
     rdm_status st = check_sizes(a->B, a->H, a->T, a->dk, a->dv, a->chunk, a->dtype, a->impl);
     if (st != RDM_OK) return st;
+    if (!gates_ok(a->gate_inputs)) return RDM_ERR_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (!opt_aligned(a->S0) || !opt_aligned(a->grad_ST) || !opt_aligned(a->grad_S0) ||
         !opt_aligned(a->saved_states) || !opt_aligned(a->workspace))
@@ -226,6 +234,6 @@ const char* rdm_status_string(rdm_status s) {
     return "unknown status";
 }
 
-int rdm_ddts_version(void) { return 200; }
+int rdm_ddts_version(void) { return 300; }
 
 }  // extern "C"

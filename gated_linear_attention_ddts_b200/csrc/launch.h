@@ -8,7 +8,8 @@ namespace rdm {
 
 struct SeqParams {
     int B, H, T, dk, dv, chunk;
-    int bf16;  // element type of sequence tensors: 1 = bf16, 0 = float32
+    int bf16;    // element type of sequence tensors: 1 = bf16, 0 = float32
+    int preact;  // g, tau, beta are pre-activations (softplus, sigmoid, sigmoid applied inside)
     const void *q, *k, *v, *g, *tau, *beta;
     const float* S0;
     void* o;
@@ -22,6 +23,7 @@ struct SeqParams {
 struct BwdParams {
     int B, H, T, dk, dv, chunk;
     int bf16;
+    int preact;  // as SeqParams::preact; grad_g, grad_tau, grad_beta then refer to the pre-activations
     const void *q, *k, *v, *g, *tau, *beta;
     const float* S0;
     const void* dO;

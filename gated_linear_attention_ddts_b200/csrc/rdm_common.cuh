@@ -49,6 +49,39 @@ __device__ __forceinline__ float lg2_fast(float x) {
     return y;
 }
 
+// Gate activations for callers that pass the gates before their activations
+// (Rodimus*, digest.lyk-ai.com summary, "Method": a selection gate g_t, a
+// temperature gate tau_t and a low-rank beta_hat_t; the activations are not
+// printed, the reading taken is g = softplus(x) = log(1 + e^x), which keeps
+// g >= 0, and tau = beta_hat = sigmoid(x) = 1 / (1 + e^-x)).
+// Library-accurate versions for the float32 path:
+__device__ __forceinline__ float softplus_acc(float x) {
+    return fmaxf(x, 0.0f) + log1pf(expf(-fabsf(x)));
+}
+__device__ __forceinline__ float sigmoid_acc(float x) { return 1.0f / (1.0f + expf(-x)); }
+// MUFU versions for the bf16 tensor-core path (log1p(y) = y (1 - y/2) to
+// ~y^3/3 when y < 1e-3, else log2(1 + y) ln 2; 1 / (1 + inf) = 0 for x -> -inf):
+__device__ __forceinline__ float softplus_fast(float x) {
+    const float y = ex2_fast(-fabsf(x) * kLog2e);
+    const float l = y < 1e-3f ? y * (1.0f - 0.5f * y) : lg2_fast(1.0f + y) * kLn2;
+    return fmaxf(x, 0.0f) + l;
+}
+__device__ __forceinline__ float sigmoid_fast(float x) {
+    return __frcp_rn(1.0f + ex2_fast(-x * kLog2e));
+}
+// g, tau of eight channels in place
+__device__ __forceinline__ void activate_gates8(float* g8, float* t8) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        g8[e] = softplus_fast(g8[e]);
+        t8[e] = sigmoid_fast(t8[e]);
+    }
+}
+__device__ __forceinline__ void activate_beta8(float* b8) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) b8[e] = sigmoid_fast(b8[e]);
+}
+
 // Device status word bits (set with atomicOr by kernels, read by the host).
 constexpr unsigned kErrTimeout = 1u;
 

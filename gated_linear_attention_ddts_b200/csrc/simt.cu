@@ -51,7 +51,11 @@ __global__ void __launch_bounds__(128) simt_fwd_kernel(SeqParams p) {
         for (int idx = threadIdx.x; idx < nt * DK; idx += blockDim.x) {
             const int tt = idx / DK, i = idx % DK;
             const size_t off = (size_t)(t0 + tt) * DK + i;
-            const float gg = ldf(g + off), ta = ldf(tau + off);
+            float gg = ldf(g + off), ta = ldf(tau + off);
+            if (p.preact) {
+                gg = softplus_acc(gg);
+                ta = sigmoid_acc(ta);
+            }
             s_al[tt][i] = alpha(gg, ta);
             s_kh[tt][i] = alpha_hat(gg, ta) * ldf(k + off);
             s_q[tt][i] = ldf(q + off);
@@ -64,7 +68,8 @@ __global__ void __launch_bounds__(128) simt_fwd_kernel(SeqParams p) {
 #pragma unroll
                 for (int i = 0; i < DK; ++i) dst[(size_t)i * dv] = s[i];
             }
-            const float vh = ldf(beta + (size_t)t * dv + j) * ldf(v + (size_t)t * dv + j);
+            const float bb = ldf(beta + (size_t)t * dv + j);
+            const float vh = (p.preact ? sigmoid_acc(bb) : bb) * ldf(v + (size_t)t * dv + j);
             float acc = 0.0f;
 #pragma unroll
             for (int i = 0; i < DK; ++i) {
@@ -111,13 +116,18 @@ __global__ void __launch_bounds__(128) simt_bwd_fsweep(BwdParams p, float* qdq, 
         for (int idx = threadIdx.x; idx < nt * DV; idx += blockDim.x) {
             const int tt = idx / DV, j = idx % DV;
             const size_t off = (size_t)(t0 + tt) * DV + j;
-            s_vh[tt][j] = ldf(beta + off) * ldf(v + off);
+            const float bb = ldf(beta + off);
+            s_vh[tt][j] = (p.preact ? sigmoid_acc(bb) : bb) * ldf(v + off);
             s_do[tt][j] = ldf(dO + off);
         }
         __syncthreads();
         for (int tt = 0; tt < nt; ++tt) {
             const size_t off = (size_t)(t0 + tt) * dk + i;
-            const float gg = ldf(g + off), ta = ldf(tau + off);
+            float gg = ldf(g + off), ta = ldf(tau + off);
+            if (p.preact) {
+                gg = softplus_acc(gg);
+                ta = sigmoid_acc(ta);
+            }
             const float al = alpha(gg, ta), kh = alpha_hat(gg, ta) * ldf(k + off);
             float acc = 0.0f;
 #pragma unroll
@@ -179,13 +189,19 @@ __global__ void __launch_bounds__(128) simt_bwd_rsweep(BwdParams p, const float*
         for (int idx = threadIdx.x; idx < nt * DV; idx += blockDim.x) {
             const int tt = idx / DV, j = idx % DV;
             const size_t off = (size_t)(t0 + tt) * DV + j;
-            s_vh[tt][j] = ldf(beta + off) * ldf(v + off);
+            const float bb = ldf(beta + off);
+            s_vh[tt][j] = (p.preact ? sigmoid_acc(bb) : bb) * ldf(v + off);
             s_do[tt][j] = ldf(dO + off);
         }
         __syncthreads();
         for (int tt = nt - 1; tt >= 0; --tt) {
             const size_t off = (size_t)(t0 + tt) * dk + i;
-            const float gg = ldf(g + off), ta = ldf(tau + off), kk = ldf(k + off);
+            const float g_in = ldf(g + off), t_in = ldf(tau + off), kk = ldf(k + off);
+            const float gg = p.preact ? softplus_acc(g_in) : g_in;
+            const float ta = p.preact ? sigmoid_acc(t_in) : t_in;
+            // chain factors to the pre-activations: softplus' = sigmoid, sigmoid' = s (1 - s)
+            const float cg = p.preact ? sigmoid_acc(g_in) : 1.0f;
+            const float ct = p.preact ? ta * (1.0f - ta) : 1.0f;
             const float qi = act ? ldf(q + off) : 0.0f;
             const float al = alpha(gg, ta), ah = alpha_hat(gg, ta);
             const float kh = act ? ah * kk : 0.0f;
@@ -212,8 +228,8 @@ __global__ void __launch_bounds__(128) simt_bwd_rsweep(BwdParams p, const float*
             const float dah_dtau = ah == 0.0f ? 0.0f : ah * logf(gg);
             if (act) {
                 stf(dk_ + off, ah * dkh);
-                stf(dg + off, -ta * da + dah_dg * dah);
-                stf(dtau + off, -gg * da + dah_dtau * dah);
+                stf(dg + off, cg * (-ta * da + dah_dg * dah));
+                stf(dtau + off, ct * (-gg * da + dah_dtau * dah));
             }
             a_next = al;
             __syncthreads();
@@ -221,8 +237,10 @@ __global__ void __launch_bounds__(128) simt_bwd_rsweep(BwdParams p, const float*
                 float dvh = 0.0f;
                 for (int w = 0; w < nwarps; ++w) dvh += s_red[w][j];
                 const size_t ov = (size_t)(t0 + tt) * DV + j;
-                stf(dv_ + ov, ldf(beta + ov) * dvh);
-                stf(dbeta + ov, ldf(v + ov) * dvh);
+                const float b_in = ldf(beta + ov);
+                const float bb = p.preact ? sigmoid_acc(b_in) : b_in;
+                stf(dv_ + ov, bb * dvh);
+                stf(dbeta + ov, (p.preact ? bb * (1.0f - bb) : 1.0f) * ldf(v + ov) * dvh);
             }
             __syncthreads();
         }

@@ -130,7 +130,8 @@ __device__ __forceinline__ uint32_t off_rc(int r, int c) {
     return (uint32_t)((r >> 3) * 128 + (c >> 3) * 1024 + (r & 7) * 16 + (c & 7) * 2);
 }
 
-template <int DV>
+// PRE: g, tau, beta arrive before their activations (gradients with respect to those)
+template <int DV, bool PRE>
 __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_constant__ BwdKernelArgs A) {
     using K = BCfg<DV>;
     constexpr int VB = K::VB;
@@ -346,6 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 float g8[8], t8[8];
                 unpack8(*reinterpret_cast<const uint4*>(raw + 2 * kBox + off_raw(tb + u, cg)), g8);
                 unpack8(*reinterpret_cast<const uint4*>(raw + 3 * kBox + off_raw(tb + u, cg)), t8);
+                if constexpr (PRE) activate_gates8(g8, t8);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const float la = (tb + u < nval) ? log_alpha(g8[e], t8[e]) : 0.0f;
@@ -427,6 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 unpack8(*reinterpret_cast<const uint4*>(raw + 1 * kBox + off_raw(t, cg)), k8);
                 unpack8(*reinterpret_cast<const uint4*>(raw + 2 * kBox + off_raw(t, cg)), g8);
                 unpack8(*reinterpret_cast<const uint4*>(raw + 3 * kBox + off_raw(t, cg)), t8);
+                if constexpr (PRE) activate_gates8(g8, t8);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const float dd = fmaf(b[u][e], kLog2e, -mL[e]);
@@ -462,6 +465,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 float v8[8], b8[8], o8[8];
                 unpack8(*reinterpret_cast<const uint4*>(raw + K::OFF_V + off_raw(t, jg)), v8);
                 unpack8(*reinterpret_cast<const uint4*>(raw + K::OFF_B + off_raw(t, jg)), b8);
+                if constexpr (PRE) activate_beta8(b8);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) o8[e] = v8[e] * b8[e];
                 *reinterpret_cast<uint4*>(sm.vh + off_rc(t, jg * 8)) = pack8(o8);
@@ -505,6 +509,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 unpack8(*reinterpret_cast<const uint4*>(raw + 1 * kBox + off_raw(t, cg)), k8);
                 unpack8(*reinterpret_cast<const uint4*>(raw + 2 * kBox + off_raw(t, cg)), g8);
                 unpack8(*reinterpret_cast<const uint4*>(raw + 3 * kBox + off_raw(t, cg)), t8);
+                if constexpr (PRE) activate_gates8(g8, t8);
                 const float4* dq4 = reinterpret_cast<const float4*>(&sm.u.st.dqs[t][cg * 8]);
                 const float4* dk4 = reinterpret_cast<const float4*>(&sm.u.st.dks[t][cg * 8]);
                 const float4 qa = dq4[0], qb = dq4[1], ka = dk4[0], kb4 = dk4[1];
@@ -555,6 +560,19 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 unpack8(*reinterpret_cast<const uint4*>(raw + 1 * kBox + off_raw(t, cg)), k8);
                 unpack8(*reinterpret_cast<const uint4*>(raw + 2 * kBox + off_raw(t, cg)), g8);
                 unpack8(*reinterpret_cast<const uint4*>(raw + 3 * kBox + off_raw(t, cg)), t8);
+                // chain factors to the pre-activations: softplus' = sigmoid, sigmoid' = s (1 - s)
+                float cgf[8], ctf[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    cgf[e] = 1.0f;
+                    ctf[e] = 1.0f;
+                    if constexpr (PRE) {
+                        cgf[e] = sigmoid_fast(g8[e]);
+                        g8[e] = softplus_fast(g8[e]);
+                        t8[e] = sigmoid_fast(t8[e]);
+                        ctf[e] = t8[e] * (1.0f - t8[e]);
+                    }
+                }
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const float gg = g8[e], ta = t8[e];
@@ -564,8 +582,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                     const float dah_dg = ta == 0.0f ? 0.0f : ta * ex2_fast((ta - 1.0f) * l2g);
                     const float dah_dt = ah == 0.0f ? 0.0f : ah * l2g * kLn2;
                     odk[e] = ah * dkh[u][e];
-                    odg[e] = -ta * dG[u][e] + dah_dg * dah;
-                    odt[e] = -gg * dG[u][e] + dah_dt * dah;
+                    odg[e] = cgf[e] * (-ta * dG[u][e] + dah_dg * dah);
+                    odt[e] = ctf[e] * (-gg * dG[u][e] + dah_dt * dah);
                 }
                 if (c * C + t < T) {
                     const size_t o = ((size_t)bh * T + (size_t)c * C + t) * DK + cg * 8;
@@ -779,10 +797,19 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                             float v8[8], b8[8], ov[8], ob[8];
                             unpack8(*reinterpret_cast<const uint4*>(sm.raw + K::OFF_V + off_raw(r, jg)), v8);
                             unpack8(*reinterpret_cast<const uint4*>(sm.raw + K::OFF_B + off_raw(r, jg)), b8);
+                            float cb[8];  // chain factor to the pre-activation of beta_hat
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                cb[e] = 1.0f;
+                                if constexpr (PRE) {
+                                    b8[e] = sigmoid_fast(b8[e]);
+                                    cb[e] = b8[e] * (1.0f - b8[e]);
+                                }
+                            }
 #pragma unroll
                             for (int e = 0; e < 8; ++e) {
                                 ov[e] = b8[e] * v[8 * h4 + e];
-                                ob[e] = v8[e] * v[8 * h4 + e];
+                                ob[e] = cb[e] * v8[e] * v[8 * h4 + e];
                             }
                             *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dv_) + o + 8 * jg) = pack8(ov);
                             *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dbeta) + o + 8 * jg) = pack8(ob);
@@ -863,7 +890,7 @@ WsLayout ws_layout(const BwdParams& p) {
     return w;
 }
 
-template <int DV>
+template <int DV, bool PRE>
 cudaError_t launch_dv(const BwdParams& p, const float* saved, int* flags, const WsLayout& w,
                       cudaStream_t s) {
     BwdKernelArgs a;
@@ -880,7 +907,7 @@ cudaError_t launch_dv(const BwdParams& p, const float* saved, int* flags, const 
         !make_tmap_bf16_3d(&a.mdo, p.dO, DV, p.T, BH, 64, 64))
         return cudaErrorInvalidValue;
     const size_t smem = sizeof(BwdSmem<DV>) + 1024;
-    auto kern = tc_bwd_kernel<DV>;
+    auto kern = tc_bwd_kernel<DV, PRE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     char* seg = static_cast<char*>(p.ws) + w.states + w.oscr + w.flags + w.simt;
@@ -934,7 +961,10 @@ cudaError_t launch_tc_bwd(const BwdParams& p, cudaStream_t s) {
     }
     int* flags = reinterpret_cast<int*>(ws + w.states + w.oscr);
     if ((e = cudaMemsetAsync(flags, 0, (size_t)p.B * p.H * 4, s)) != cudaSuccess) return e;
-    e = p.dv == 64 ? launch_dv<64>(p, saved, flags, w, s) : launch_dv<128>(p, saved, flags, w, s);
+    if (p.preact)
+        e = p.dv == 64 ? launch_dv<64, true>(p, saved, flags, w, s) : launch_dv<128, true>(p, saved, flags, w, s);
+    else
+        e = p.dv == 64 ? launch_dv<64, false>(p, saved, flags, w, s) : launch_dv<128, false>(p, saved, flags, w, s);
     if (e != cudaSuccess) return e;
     // heads whose decay span needs narrower windows: exact CUDA-core backward
     BwdParams q = p;

@@ -111,7 +111,8 @@ struct FwdKernelArgs {
     SegArgs seg;
 };
 
-template <int DK, int DVT>
+// PRE: g, tau, beta arrive before their activations
+template <int DK, int DVT, bool PRE>
 __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_constant__ FwdKernelArgs A) {
     using K = Cfg<DK, DVT>;
     constexpr int NS = K::NS, NB = K::NB, KB = K::KB, VB = K::VB;
@@ -296,6 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                     float g8[8], t8[8];
                     unpack8(*reinterpret_cast<const uint4*>(raw + 2 * KB * kBox + off_raw(tb + u, cg)), g8);
                     unpack8(*reinterpret_cast<const uint4*>(raw + 3 * KB * kBox + off_raw(tb + u, cg)), t8);
+                    if constexpr (PRE) activate_gates8(g8, t8);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const float la = (tb + u < nval) ? log_alpha(g8[e], t8[e]) : 0.0f;
@@ -366,6 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                     float v8[8], b8[8], o8[8];
                     unpack8(*reinterpret_cast<const uint4*>(sm.rawv + off_raw(t, jg)), v8);
                     unpack8(*reinterpret_cast<const uint4*>(sm.rawv + VB * kBox + off_raw(t, jg)), b8);
+                    if constexpr (PRE) activate_beta8(b8);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) o8[e] = in ? v8[e] * b8[e] : 0.0f;
                     *reinterpret_cast<uint4*>(sm.vh[ob] + off_vh(t, jg * 8)) = pack8(o8);
@@ -406,6 +409,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                         float g8[8], t8[8];
                         unpack8(*reinterpret_cast<const uint4*>(raw + 2 * KB * kBox + off_raw(t, cg)), g8);
                         unpack8(*reinterpret_cast<const uint4*>(raw + 3 * KB * kBox + off_raw(t, cg)), t8);
+                        if constexpr (PRE) activate_gates8(g8, t8);
 #pragma unroll
                         for (int e = 0; e < 8; ++e) lah[e] = t8[e] == 0.0f ? 0.0f : t8[e] * lg2_fast(g8[e]);
                     }
@@ -458,6 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                         unpack8(*reinterpret_cast<const uint4*>(raw + 1 * KB * kBox + off_raw(t, cg)), k8);
                         unpack8(*reinterpret_cast<const uint4*>(raw + 2 * KB * kBox + off_raw(t, cg)), g8);
                         unpack8(*reinterpret_cast<const uint4*>(raw + 3 * KB * kBox + off_raw(t, cg)), t8);
+                        if constexpr (PRE) activate_gates8(g8, t8);
 #pragma unroll
                         for (int e = 0; e < 8; ++e) {
                             // reference m = midpoint of the window's b range, blast = b at its end
@@ -761,7 +766,7 @@ SegPlan choose_plan(const SeqParams& p, bool allow_seg) {
     return best;
 }
 
-template <int DK, int DVT>
+template <int DK, int DVT, bool PRE>
 cudaError_t launch_cfg(const SeqParams& p, SegPlan plan, cudaStream_t s) {
     FwdKernelArgs a;
     a.p = p;
@@ -775,7 +780,7 @@ cudaError_t launch_cfg(const SeqParams& p, SegPlan plan, cudaStream_t s) {
         !make_tmap_bf16_3d(&a.mo, p.o, p.dv, p.T, BH, 64, 64))
         return cudaErrorInvalidValue;
     const size_t smem = sizeof(FwdSmem<DK, DVT>) + 1024;
-    auto kern = tc_fwd_kernel<DK, DVT>;
+    auto kern = tc_fwd_kernel<DK, DVT, PRE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const unsigned units = (unsigned)(BH * (p.dv / DVT));
@@ -798,9 +803,14 @@ cudaError_t launch_cfg(const SeqParams& p, SegPlan plan, cudaStream_t s) {
     return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
+template <bool PRE>
+cudaError_t launch_plan_t(const SeqParams& p, const SegPlan& plan, cudaStream_t s) {
+    if (p.dk == 128) return launch_cfg<128, 64, PRE>(p, plan, s);
+    return plan.DVT == 128 ? launch_cfg<64, 128, PRE>(p, plan, s) : launch_cfg<64, 64, PRE>(p, plan, s);
+}
+
 cudaError_t launch_plan(const SeqParams& p, const SegPlan& plan, cudaStream_t s) {
-    if (p.dk == 128) return launch_cfg<128, 64>(p, plan, s);
-    return plan.DVT == 128 ? launch_cfg<64, 128>(p, plan, s) : launch_cfg<64, 64>(p, plan, s);
+    return p.preact ? launch_plan_t<true>(p, plan, s) : launch_plan_t<false>(p, plan, s);
 }
 
 }  // namespace

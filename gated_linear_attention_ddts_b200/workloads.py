@@ -64,20 +64,27 @@ def _gen(device, seed):
 
 
 def draw_sequence(B, H, T, dk, dv, dtype=torch.bfloat16, seed=BASE_SEED, mu_g=-1.0,
-                  s0_std=0.0, with_dO=False, device="cpu"):
+                  s0_std=0.0, with_dO=False, device="cpu", preact=False):
     """Inputs for one forward (and backward) call, layout [B,H,T,D].
 
     Returns a dict with q, k, g, tau [B,H,T,dk], v, beta [B,H,T,dv] in `dtype`,
     optionally dO [B,H,T,dv] in `dtype`, and S0 [B,H,dk,dv] float32 (None when
-    s0_std == 0)."""
+    s0_std == 0).  With preact, g, tau and beta are the normal draws before
+    their softplus / sigmoid (same random numbers as without)."""
     gen = _gen(device, seed)
     f32 = dict(dtype=torch.float32, device=device, generator=gen)
     q = torch.randn(B, H, T, dk, **f32) / math.sqrt(dk)
     k = torch.randn(B, H, T, dk, **f32) / math.sqrt(dk)
     v = torch.randn(B, H, T, dv, **f32)
-    g = torch.nn.functional.softplus(torch.randn(B, H, T, dk, **f32) + mu_g)
-    tau = torch.sigmoid(torch.randn(B, H, T, dk, **f32))
-    beta = torch.sigmoid(torch.randn(B, H, T, dv, **f32))
+    g_pre = torch.randn(B, H, T, dk, **f32) + mu_g
+    tau_pre = torch.randn(B, H, T, dk, **f32)
+    beta_pre = torch.randn(B, H, T, dv, **f32)
+    if preact:
+        g, tau, beta = g_pre, tau_pre, beta_pre
+    else:
+        g = torch.nn.functional.softplus(g_pre)
+        tau = torch.sigmoid(tau_pre)
+        beta = torch.sigmoid(beta_pre)
     out = dict(q=q, k=k, v=v, g=g, tau=tau, beta=beta)
     out = {n: t.to(dtype).contiguous() for n, t in out.items()}
     if with_dO:

@@ -70,6 +70,15 @@ typedef enum { RDM_F32 = 0, RDM_BF16 = 1 } rdm_dtype;
  * not apply. */
 typedef enum { RDM_IMPL_AUTO = 0, RDM_IMPL_SIMT = 1, RDM_IMPL_TC = 2 } rdm_impl;
 
+/* What the g, tau and beta pointers of rdm_fwd_args / rdm_bwd_args hold.
+ * ACTIVATED: the gates themselves (g >= 0, tau >= 0, beta_hat).  PREACT: the
+ * gates before their activations; the kernels apply g = softplus(x) =
+ * log(1 + e^x), tau = sigmoid(x), beta_hat = sigmoid(x) on the fly (the page
+ * names a selection gate, a temperature gate and a low-rank beta_hat without
+ * printing the activations; these are the reading this library takes), and the
+ * backward returns the gradients with respect to the pre-activations. */
+typedef enum { RDM_GATES_ACTIVATED = 0, RDM_GATES_PREACT = 1 } rdm_gate_inputs;
+
 /* ------------------------------------------------------------------ forward
  * Chunkwise-parallel forward over whole sequences (the training / prefill
  * form named in the rebuttal's answer to Q2).
@@ -82,6 +91,7 @@ typedef enum { RDM_IMPL_AUTO = 0, RDM_IMPL_SIMT = 1, RDM_IMPL_TC = 2 } rdm_impl;
  *                  in force before each chunk (S_0 for chunk 0); NULL = skip.
  *                  rdm_ddts_bwd can reuse it instead of recomputing.
  *   chunk        : tokens per chunk; 0 selects 64.  Allowed: 64.
+ *   gate_inputs  : RDM_GATES_ACTIVATED (default, 0) or RDM_GATES_PREACT.
  *   workspace    : optional device scratch of workspace_bytes.  With at least
  *                  rdm_ddts_fwd_workspace_size() bytes the tensor-core path
  *                  may cut each sequence into segments processed by separate
@@ -102,6 +112,7 @@ typedef struct {
     float *saved_states;
     void *workspace;
     size_t workspace_bytes;
+    rdm_gate_inputs gate_inputs;
 } rdm_fwd_args;
 
 rdm_status rdm_ddts_fwd(const rdm_fwd_args *args, rdm_stream_t stream);
@@ -128,6 +139,8 @@ size_t rdm_ddts_saved_states_size(int B, int H, int T, int dk, int dv, int chunk
  *   grad_q, grad_k, grad_g, grad_tau : [B,H,T,d_k] dtype, written
  *   grad_v, grad_beta                : [B,H,T,d_v] dtype, written
  *   grad_S0      : [B,H,d_k,d_v] float32, written; NULL = skip
+ *   gate_inputs  : as for rdm_ddts_fwd; with RDM_GATES_PREACT, grad_g, grad_tau
+ *                  and grad_beta are with respect to the pre-activations.
  *   workspace    : device scratch of at least rdm_ddts_bwd_workspace_size()
  *                  bytes (may be NULL when that size is 0); contents on entry
  *                  are ignored and on exit are unspecified.
@@ -148,6 +161,7 @@ typedef struct {
     float *grad_S0;
     void *workspace;
     size_t workspace_bytes;
+    rdm_gate_inputs gate_inputs;
 } rdm_bwd_args;
 
 rdm_status rdm_ddts_bwd(const rdm_bwd_args *args, rdm_stream_t stream);

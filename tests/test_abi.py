@@ -66,7 +66,7 @@ def _fwd_args(**kw):
     (dict(B=0), 1), (dict(H=-1), 1), (dict(T=-1), 1), (dict(dk=0), 1),
     (dict(dk=48), 2), (dict(dv=256), 2), (dict(chunk=48), 2), (dict(chunk=-2), 1),
     (dict(dtype=7), 1), (dict(impl=9), 1), (dict(q=None), 1), (dict(o=None), 1),
-    (dict(k=(1 << 20) + 8), 1), (dict(S0=(1 << 20) + 4), 1),
+    (dict(k=(1 << 20) + 8), 1), (dict(S0=(1 << 20) + 4), 1), (dict(gate_inputs=7), 1),
 ])
 def test_fwd_validation(lib, kw, status):
     a = _fwd_args(**kw)
