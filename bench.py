@@ -265,6 +265,22 @@ def run_extras(rdm, dev, pk, K):
         "roofline": roofline(fwd_bytes(w, True), chunk_flops_fwd(w), ms, pk,
                              ncu_traffic("tc_fwd_kernel", ["tc_fwd.cu"], 2))}
     del x, o, ST, wsf
+    # headline forward with the gate activations fused (inputs are the
+    # pre-activations; same bytes)
+    w = WORKLOADS[1]
+    x = draw_workload(w, device=dev, preact=True)
+    o = torch.empty(w.B, w.H, w.T, w.dv, dtype=torch.bfloat16, device=dev)
+    n = rdm.rdm_ddts_fwd_workspace_size(*(x[k] for k in SEQ), gates="preact")
+    wsf = torch.empty(n, dtype=torch.uint8, device=dev) if n else False
+    fl = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    t = time_steps(lambda: rdm.rdm_ddts_fwd(*(x[k] for k in SEQ), x["S0"], o, workspace=wsf,
+                                            gates="preact"), max(3, K // 2), 3, lambda: fl.zero_())
+    ms = statistics.mean(t)
+    out["fused_gates_fwd"] = {
+        "workload": w.name + ", gates passed before softplus/sigmoid", "value": w.B * w.T / (ms / 1e3),
+        "unit": "tokens/s", "ms_per_step": ms, "gpu_launches_per_step": 1,
+        "roofline": roofline(fwd_bytes(w, False), chunk_flops_fwd(w), ms, pk, None)}
+    del x, o, wsf, fl
     # training forward + backward (forward saves chunk states for the backward)
     w = WORKLOADS[3]
     x = draw_workload(w, device=dev)
