@@ -72,7 +72,7 @@ struct Cfg {
 };
 
 // info[] of an operand slot
-enum { kInfoChunk, kInfoW0, kInfoW1, kInfoLast, kInfoPhase, kInfoP1Last, kInfoN };
+enum { kInfoChunk, kInfoW0, kInfoW1, kInfoLast, kInfoPhase, kInfoP1Last, kInfoPass, kInfoN };
 
 template <int DK, int DVT>
 struct alignas(1024) FwdSmem {
@@ -88,7 +88,7 @@ struct alignas(1024) FwdSmem {
     float em[K::NB][DK], cf[K::NB][DK], gm[K::NB][DK];
     int info[K::NB][kInfoN];
     uint64_t raw_full[K::NS], raw_empty[K::NS], v_full, v_empty, ops_full[K::NB], ops_empty[K::NB];
-    uint64_t mma1_done, as_free, abf_full, mmao_done[2], o_free[2];
+    uint64_t mma1_done, as_free, abf_full, mmao_done[2], o_free[2], vh_full[K::NB];
     int need16[2], need1[2];
     uint32_t tmem_base;
     int fail;
@@ -116,6 +116,11 @@ template <int DK, int DVT, bool PRE>
 __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_constant__ FwdKernelArgs A) {
     using K = Cfg<DK, DVT>;
     constexpr int NS = K::NS, NB = K::NB, KB = K::KB, VB = K::VB;
+    // Who builds Vh = beta_hat * v: the epilogue warps when d_k = 128 (the gate
+    // warps then carry twice the key-side work and are the slower role, which
+    // also hides the v / beta load behind them); the gate warps otherwise, where
+    // moving it would put that load on the epilogue's path to the first MMA group.
+    auto vh_by_epi = [&](bool) { return DK == 128; };
     // align by pointer arithmetic on the __shared__ array so that every access
     // below stays a shared-memory access (an integer round trip would make it generic)
     extern __shared__ __align__(1024) uint8_t smem_dyn[];
@@ -156,6 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
         mbar_init(&sm.mmao_done[1], 1);
         mbar_init(&sm.o_free[0], kEpiWarps);
         mbar_init(&sm.o_free[1], kEpiWarps);
+        for (int b = 0; b < NB; ++b) mbar_init(&sm.vh_full[b], kEpiWarps);
         sm.need16[0] = sm.need16[1] = sm.need1[0] = sm.need1[1] = 0;
         sm.fail = 0;
         fence_mbar_init();
@@ -220,6 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                 if (!mbar_wait(&sm.ops_full[ob], (item / NB) & 1, fail, kWaitLimit)) break;
                 const int last = sm.info[ob][kInfoLast];
                 const bool p2 = sm.info[ob][kInfoPhase] == 2;
+                if (vh_by_epi(p2) && !mbar_wait(&sm.vh_full[ob], (item / NB) & 1, fail, kWaitLimit)) break;
                 if (item > 0 && !mbar_wait(&sm.as_free, (item - 1) & 1, fail, kWaitLimit)) break;
                 tc_fence_after();
                 const uint32_t q = smem_u32(sm.qt[ob]) >> 4, k = smem_u32(sm.kt[ob]) >> 4;
@@ -357,6 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             // Vh = beta_hat * v for the rows of [w0, w1), zero elsewhere
             bool have_v = false;
             auto write_vh = [&](int ob, int w0, int w1) {
+                if (vh_by_epi(p2)) return;
                 if (!have_v) {
                     have_v = mbar_wait(&sm.v_full, li & 1, fail, kWaitLimit);
                     if (!have_v) return;
@@ -383,6 +391,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                     sm.info[ob][kInfoLast] = p2 && end;
                     sm.info[ob][kInfoPhase] = p2 ? 2 : 1;
                     sm.info[ob][kInfoP1Last] = !p2 && end;
+                    sm.info[ob][kInfoPass] = li;
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
@@ -490,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(&sm.raw_empty[st]);
-                mbar_arrive(&sm.v_empty);
+                if (!vh_by_epi(p2)) mbar_arrive(&sm.v_empty);
             }
             if (*fail) break;
         }
@@ -625,6 +634,34 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             const int c = sm.info[ob][kInfoChunk], w0 = sm.info[ob][kInfoW0], w1 = sm.info[ob][kInfoW1];
             const int last = sm.info[ob][kInfoLast], p1last = sm.info[ob][kInfoP1Last];
             const bool p2 = sm.info[ob][kInfoPhase] == 2;
+            if (vh_by_epi(p2)) {
+                // Vh = beta_hat * v for the rows of [w0, w1), zero elsewhere; the slot is
+                // free once the tensor core has finished the item NB back
+                const int li = sm.info[ob][kInfoPass];
+                const int nval = min(C, T - c * C);
+                if (!mbar_wait(&sm.v_full, li & 1, fail, kWaitLimit)) break;
+                if (item >= NB && !mbar_wait(&sm.ops_empty[ob], ((item / NB) - 1) & 1, fail, kWaitLimit))
+                    break;
+                const int et = threadIdx.x - 32 * kEpiWarp0;
+#pragma unroll
+                for (int it = 0; it < (C * DVT / 8) / (32 * kEpiWarps); ++it) {
+                    const int idx = et + 32 * kEpiWarps * it, jg = idx / C, t = idx % C;
+                    const bool in = t >= w0 && t < w1;
+                    float v8[8], b8[8], o8[8];
+                    unpack8(*reinterpret_cast<const uint4*>(sm.rawv + off_raw(t, jg)), v8);
+                    unpack8(*reinterpret_cast<const uint4*>(sm.rawv + VB * kBox + off_raw(t, jg)), b8);
+                    if constexpr (PRE) activate_beta8(b8);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) o8[e] = in ? v8[e] * b8[e] : 0.0f;
+                    *reinterpret_cast<uint4*>(sm.vh[ob] + off_vh(t, jg * 8)) = pack8(o8);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&sm.vh_full[ob]);
+                    if (w1 == nval) mbar_arrive(&sm.v_empty);  // last window of the chunk
+                }
+            }
             if (!mbar_wait(&sm.mma1_done, item & 1, fail, kWaitLimit)) break;
             tc_fence_after();
             if (p2) {
