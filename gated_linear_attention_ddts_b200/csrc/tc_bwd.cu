@@ -55,7 +55,8 @@ constexpr int DK = 64;
 constexpr int kGateWarps = 8;  // one 8-channel group each
 constexpr int kThreads = 32 * (4 + kGateWarps + 2);
 constexpr int kEpiWarp0 = 0, kGateWarp0 = 4, kProdWarp = 4 + kGateWarps, kMmaWarp = 5 + kGateWarps;
-constexpr int kBarEpi = 3;  // the four epilogue warps
+constexpr int kBarEpi = 3;   // the four epilogue warps
+constexpr int kBarGate = 4;  // the gate warps
 constexpr int kStg = 68;
 // row stride (floats) of the chunk-start state copied into shared memory: a
 // 16-byte skew per row keeps the S_hat conversion free of bank conflicts
@@ -85,8 +86,9 @@ struct alignas(1024) BwdSmem {
     // completed, the same bytes hold the fp32 dQ / dK staging tiles; before the
     // first stage of the epilogue writes A, they hold the chunk-start state
     // S_prev (fp32) that the gate warps turn into S_hat
-    union {
+    union alignas(1024) {
         float sprev[DK * kSpStride<DV>];
+        uint8_t ost[2 * C * DV * 2];  // dv | dbeta tiles for the TMA stores (128B-swizzled)
         struct {
             uint8_t abf[C * C * 2];       // [t][s]
             uint8_t bmb[C * C * 2];       // [t][s]
@@ -118,6 +120,7 @@ struct BwdSeg {
 
 struct BwdKernelArgs {
     CUtensorMap mq, mk, mg, mt, mv, mb, mdo;
+    CUtensorMap mdq, mdk, mdg, mdt, mdv, mdb;  // gradient outputs (TMA stores)
     BwdParams p;
     int* flags;
     BwdSeg seg;
@@ -500,6 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
 
             // ---- post: final gate gradients once dQ, dK of this chunk are staged
             if (!mbar_wait(&sm.post_ready, i2 & 1, fail, kWaitLimit)) break;
+            uint8_t* gst = sm.qt;  // 4 x 8 KB over qt | kt | qtl | ktl
             float dG[SEGT][8], dkh[SEGT][8];
 #pragma unroll
             for (int u = 0; u < SEGT; ++u) {
@@ -527,11 +531,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                     dqo[e] = dq_off + kh * bd;
                     dkh[u][e] = dk_off + q8[e] * bd;
                 }
-                if (c * C + t < T) {
-                    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.dq) +
-                                         ((size_t)bh * T + (size_t)c * C + t) * DK + cg * 8;
-                    *reinterpret_cast<uint4*>(dst) = pack8(dqo);
-                }
+                // staged in the (now idle) Qt / Kt operand buffers, stored by TMA below
+                *reinterpret_cast<uint4*>(gst + 0 * kBox + off_raw(t, cg)) = pack8(dqo);
             }
             // d log(alpha) = suffix sum of dG: in the segment, over later segments of
             // this warp (= later tokens of the chunk), over later chunks (carry)
@@ -585,13 +586,23 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                     odg[e] = cgf[e] * (-ta * dG[u][e] + dah_dg * dah);
                     odt[e] = ctf[e] * (-gg * dG[u][e] + dah_dt * dah);
                 }
-                if (c * C + t < T) {
-                    const size_t o = ((size_t)bh * T + (size_t)c * C + t) * DK + cg * 8;
-                    *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dk_) + o) = pack8(odk);
-                    *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dg) + o) = pack8(odg);
-                    *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dtau) + o) = pack8(odt);
-                }
+                *reinterpret_cast<uint4*>(gst + 1 * kBox + off_raw(t, cg)) = pack8(odk);
+                *reinterpret_cast<uint4*>(gst + 2 * kBox + off_raw(t, cg)) = pack8(odg);
+                *reinterpret_cast<uint4*>(gst + 3 * kBox + off_raw(t, cg)) = pack8(odt);
             }
+            // dq, dk, dg, dtau of the chunk: one TMA store each (rows past T are
+            // clipped); the staging bytes are read before the next operand stage
+            fence_proxy_async_smem();
+            named_bar(kBarGate, 32 * kGateWarps);
+            if (gt == 0) {
+                tma_store_3d(&A.mdq, gst + 0 * kBox, 0, c * C, bh);
+                tma_store_3d(&A.mdk, gst + 1 * kBox, 0, c * C, bh);
+                tma_store_3d(&A.mdg, gst + 2 * kBox, 0, c * C, bh);
+                tma_store_3d(&A.mdt, gst + 3 * kBox, 0, c * C, bh);
+                bulk_commit();
+                bulk_wait_read_all();
+            }
+            named_bar(kBarGate, 32 * kGateWarps);
             __syncwarp();  // every lane has read the old carry
             if (tb == 0) {
 #pragma unroll
@@ -781,44 +792,54 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             }
             if (!mbar_wait(&sm.g2_done, i2 & 1, fail, kWaitLimit)) break;
             tc_fence_after();
-            // dV -> dv = beta dvhat, dbeta = v dvhat (row s = r)
+            // dV -> dv = beta dvhat, dbeta = v dvhat (row s = r), staged in the union
+            // (its A / B / R_hat operands are consumed; the previous chunk's gate
+            // stage has read its dQ / dK staging) and written by TMA stores
+            if (i2 > 0 && !mbar_wait(&sm.post_done, (i2 - 1) & 1, fail, kWaitLimit)) break;
             {
-                const bool st = c * C + r < T;
-                const size_t o = ((size_t)bh * T + (size_t)c * C + r) * DV;
 #pragma unroll
                 for (int qd = 0; qd < HV / 32; ++qd) {
                     float v[32];
                     tmem_ld32_split<HV>(tmem + lb + K::COL_DV + 32 * qd, v);
                     tmem_ld_wait();
-                    if (st) {
 #pragma unroll
-                        for (int h4 = 0; h4 < 4; ++h4) {
-                            const int jg = (hf * HV + 32 * qd) / 8 + h4;
-                            float v8[8], b8[8], ov[8], ob[8];
-                            unpack8(*reinterpret_cast<const uint4*>(sm.raw + K::OFF_V + off_raw(r, jg)), v8);
-                            unpack8(*reinterpret_cast<const uint4*>(sm.raw + K::OFF_B + off_raw(r, jg)), b8);
-                            float cb[8];  // chain factor to the pre-activation of beta_hat
+                    for (int h4 = 0; h4 < 4; ++h4) {
+                        const int jg = (hf * HV + 32 * qd) / 8 + h4;
+                        float v8[8], b8[8], ov[8], ob[8];
+                        unpack8(*reinterpret_cast<const uint4*>(sm.raw + K::OFF_V + off_raw(r, jg)), v8);
+                        unpack8(*reinterpret_cast<const uint4*>(sm.raw + K::OFF_B + off_raw(r, jg)), b8);
+                        float cb[8];  // chain factor to the pre-activation of beta_hat
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) {
-                                cb[e] = 1.0f;
-                                if constexpr (PRE) {
-                                    b8[e] = sigmoid_fast(b8[e]);
-                                    cb[e] = b8[e] * (1.0f - b8[e]);
-                                }
+                        for (int e = 0; e < 8; ++e) {
+                            cb[e] = 1.0f;
+                            if constexpr (PRE) {
+                                b8[e] = sigmoid_fast(b8[e]);
+                                cb[e] = b8[e] * (1.0f - b8[e]);
                             }
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) {
-                                ov[e] = b8[e] * v[8 * h4 + e];
-                                ob[e] = cb[e] * v8[e] * v[8 * h4 + e];
-                            }
-                            *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dv_) + o + 8 * jg) = pack8(ov);
-                            *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dbeta) + o + 8 * jg) = pack8(ob);
                         }
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            ov[e] = b8[e] * v[8 * h4 + e];
+                            ob[e] = cb[e] * v8[e] * v[8 * h4 + e];
+                        }
+                        *reinterpret_cast<uint4*>(sm.u.ost + off_raw(r, jg)) = pack8(ov);
+                        *reinterpret_cast<uint4*>(sm.u.ost + VB * kBox + off_raw(r, jg)) = pack8(ob);
                     }
                 }
+                fence_proxy_async_smem();
+                named_bar(kBarEpi, 128);
+                if (threadIdx.x == 0) {
+#pragma unroll
+                    for (int vb = 0; vb < VB; ++vb) {
+                        tma_store_3d(&A.mdv, sm.u.ost + vb * kBox, 64 * vb, c * C, bh);
+                        tma_store_3d(&A.mdb, sm.u.ost + (VB + vb) * kBox, 64 * vb, c * C, bh);
+                    }
+                    bulk_commit();
+                    bulk_wait_read_all();  // the union takes the dQ / dK staging next
+                }
+                named_bar(kBarEpi, 128);
             }
             // dQ, dK -> fp32 staging for the gate warps
-            if (i2 > 0 && !mbar_wait(&sm.post_done, (i2 - 1) & 1, fail, kWaitLimit)) break;
 #pragma unroll
             for (int which = 0; which < 2; ++which) {
                 float v[32];
@@ -845,6 +866,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
         }
     }
 
+    // the gradient stores (issued by thread 0 and by the first gate thread) have landed
+    if (threadIdx.x == 0 || threadIdx.x == 32 * kGateWarp0) bulk_wait_all();
     tc_fence_before();
     __syncthreads();
     if (warp == kMmaWarp) {
@@ -904,7 +927,13 @@ cudaError_t launch_dv(const BwdParams& p, const float* saved, int* flags, const 
         !make_tmap_bf16_3d(&a.mt, p.tau, DK, p.T, BH, 64, 64) ||
         !make_tmap_bf16_3d(&a.mv, p.v, DV, p.T, BH, 64, 64) ||
         !make_tmap_bf16_3d(&a.mb, p.beta, DV, p.T, BH, 64, 64) ||
-        !make_tmap_bf16_3d(&a.mdo, p.dO, DV, p.T, BH, 64, 64))
+        !make_tmap_bf16_3d(&a.mdo, p.dO, DV, p.T, BH, 64, 64) ||
+        !make_tmap_bf16_3d(&a.mdq, p.dq, DK, p.T, BH, 64, 64) ||
+        !make_tmap_bf16_3d(&a.mdk, p.dk_, DK, p.T, BH, 64, 64) ||
+        !make_tmap_bf16_3d(&a.mdg, p.dg, DK, p.T, BH, 64, 64) ||
+        !make_tmap_bf16_3d(&a.mdt, p.dtau, DK, p.T, BH, 64, 64) ||
+        !make_tmap_bf16_3d(&a.mdv, p.dv_, DV, p.T, BH, 64, 64) ||
+        !make_tmap_bf16_3d(&a.mdb, p.dbeta, DV, p.T, BH, 64, 64))
         return cudaErrorInvalidValue;
     const size_t smem = sizeof(BwdSmem<DV>) + 1024;
     auto kern = tc_bwd_kernel<DV, PRE>;
