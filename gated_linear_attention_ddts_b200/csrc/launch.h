@@ -73,6 +73,11 @@ namespace rdm {
 bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t n0, uint64_t n1,
                        uint64_t n2, uint32_t b0, uint32_t b1);
 
+// 2-D float32 tensor [n1][n0] (n0 innermost, dense) as a TMA map with box
+// {b0, b1} and 128-byte swizzle (b0 * 4 must be 128).
+bool make_tmap_f32_2d(CUtensorMap* map, const void* base, uint64_t n0, uint64_t n1, uint32_t b0,
+                      uint32_t b1);
+
 // SM count of the current device (cached).
 int sm_count();
 // Tag of one launch for flags that CTAs of a sequence-segmented kernel set for

@@ -69,6 +69,7 @@ struct Cfg {
     // tensor core writes the next)
     static constexpr int COL_A = 0, COL_S = 64, COL_O = 64 + DVT;
     static constexpr int TMEM_COLS = (64 + 3 * DVT) <= 256 ? 256 : 512;
+    static constexpr bool STAGE_SAVED = DK == 64 && DVT == 64;
 };
 
 // info[] of an operand slot
@@ -80,6 +81,9 @@ struct alignas(1024) FwdSmem {
     uint8_t raw[K::NS][K::RAWK];
     uint8_t rawv[K::RAWV];
     uint8_t ostage[C * DVT * 2];  // o tile for the TMA store, 128B-swizzled boxes
+    // chunk-start state [DK][DVT] fp32 for the TMA store of the saved states
+    // (32-column 128B-swizzled boxes; where shared memory allows)
+    uint8_t sstage[K::STAGE_SAVED ? DK * DVT * 4 : 16];
     uint8_t qt[K::NB][K::G * kQK];
     uint8_t kt[K::NB][K::G * kQK];
     uint8_t vh[K::NB][C * DVT * 2];
@@ -107,6 +111,7 @@ struct SegArgs {
 
 struct FwdKernelArgs {
     CUtensorMap mq, mk, mg, mt, mv, mb, mo;
+    CUtensorMap msv;  // saved states as [rows = B*H*NC*DK][dv] fp32 (when staged)
     SeqParams p;
     SegArgs seg;
 };
@@ -120,7 +125,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
     // warps then carry twice the key-side work and are the slower role, which
     // also hides the v / beta load behind them); the gate warps otherwise, where
     // moving it would put that load on the epilogue's path to the first MMA group.
-    auto vh_by_epi = [&](bool) { return DK == 128; };
+    constexpr bool kVhEpi = DK == 128;
     // align by pointer arithmetic on the __shared__ array so that every access
     // below stays a shared-memory access (an integer round trip would make it generic)
     extern __shared__ __align__(1024) uint8_t smem_dyn[];
@@ -226,7 +231,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                 if (!mbar_wait(&sm.ops_full[ob], (item / NB) & 1, fail, kWaitLimit)) break;
                 const int last = sm.info[ob][kInfoLast];
                 const bool p2 = sm.info[ob][kInfoPhase] == 2;
-                if (vh_by_epi(p2) && !mbar_wait(&sm.vh_full[ob], (item / NB) & 1, fail, kWaitLimit)) break;
+                if constexpr (kVhEpi)
+                    if (!mbar_wait(&sm.vh_full[ob], (item / NB) & 1, fail, kWaitLimit)) break;
                 if (item > 0 && !mbar_wait(&sm.as_free, (item - 1) & 1, fail, kWaitLimit)) break;
                 tc_fence_after();
                 const uint32_t q = smem_u32(sm.qt[ob]) >> 4, k = smem_u32(sm.kt[ob]) >> 4;
@@ -364,7 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             // Vh = beta_hat * v for the rows of [w0, w1), zero elsewhere
             bool have_v = false;
             auto write_vh = [&](int ob, int w0, int w1) {
-                if (vh_by_epi(p2)) return;
+                if constexpr (kVhEpi) return;
                 if (!have_v) {
                     have_v = mbar_wait(&sm.v_full, li & 1, fail, kWaitLimit);
                     if (!have_v) return;
@@ -391,7 +397,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                     sm.info[ob][kInfoLast] = p2 && end;
                     sm.info[ob][kInfoPhase] = p2 ? 2 : 1;
                     sm.info[ob][kInfoP1Last] = !p2 && end;
-                    sm.info[ob][kInfoPass] = li;
+                    if constexpr (kVhEpi) sm.info[ob][kInfoPass] = li;
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
@@ -499,7 +505,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(&sm.raw_empty[st]);
-                if (!vh_by_epi(p2)) mbar_arrive(&sm.v_empty);
+                if constexpr (!kVhEpi) mbar_arrive(&sm.v_empty);
             }
             if (*fail) break;
         }
@@ -634,7 +640,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             const int c = sm.info[ob][kInfoChunk], w0 = sm.info[ob][kInfoW0], w1 = sm.info[ob][kInfoW1];
             const int last = sm.info[ob][kInfoLast], p1last = sm.info[ob][kInfoP1Last];
             const bool p2 = sm.info[ob][kInfoPhase] == 2;
-            if (vh_by_epi(p2)) {
+            if constexpr (kVhEpi) {
                 // Vh = beta_hat * v for the rows of [w0, w1), zero elsewhere; the slot is
                 // free once the tensor core has finished the item NB back
                 const int li = sm.info[ob][kInfoPass];
@@ -688,17 +694,43 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                         for (int e = 0; e < 8; ++e) x[e] = S[jg * 8 + e] * em;
                         *reinterpret_cast<uint4*>(sm.shat + off_shat<DK>(iS, sc0 + jg * 8)) = pack8(x);
                     }
-                    if (p.saved && w0 == 0) {
-                        float4* dst = reinterpret_cast<float4*>(
-                            p.saved + (((size_t)bh * NC + c) * DK + iS) * p.dv + j0 + sc0);
+                    if constexpr (!K::STAGE_SAVED) {
+                        if (p.saved && w0 == 0) {
+                            float4* dst = reinterpret_cast<float4*>(
+                                p.saved + (((size_t)bh * NC + c) * DK + iS) * p.dv + j0 + sc0);
 #pragma unroll
-                        for (int j4 = 0; j4 < SC / 4; ++j4)
-                            dst[j4] = make_float4(S[4 * j4], S[4 * j4 + 1], S[4 * j4 + 2], S[4 * j4 + 3]);
+                            for (int j4 = 0; j4 < SC / 4; ++j4)
+                                dst[j4] = make_float4(S[4 * j4], S[4 * j4 + 1], S[4 * j4 + 2], S[4 * j4 + 3]);
+                        }
                     }
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm.abf_full);
+                if constexpr (K::STAGE_SAVED) {
+                    // the chunk-start state (S still holds it until the update below)
+                    if (p.saved && w0 == 0) {
+                        if (threadIdx.x == 0) bulk_wait_read_all();  // previous store has read sstage
+                        named_bar(kBarEpi, 32 * kEpiWarps);
+#pragma unroll
+                        for (int j4 = 0; j4 < SC / 4; ++j4) {
+                            const int col = sc0 + 4 * j4;  // 32-column boxes, 16-byte chunks
+                            const uint32_t off = (uint32_t)(col >> 5) * (DK * 128) + iS * 128 +
+                                                 ((((col & 31) >> 2) ^ (iS & 7)) << 4);
+                            *reinterpret_cast<float4*>(sm.sstage + off) =
+                                make_float4(S[4 * j4], S[4 * j4 + 1], S[4 * j4 + 2], S[4 * j4 + 3]);
+                        }
+                        fence_proxy_async_smem();
+                        named_bar(kBarEpi, 32 * kEpiWarps);
+                        if (threadIdx.x == 0) {
+#pragma unroll
+                            for (int bx = 0; bx < DVT / 32; ++bx)
+                                tma_store_2d(&A.msv, sm.sstage + bx * (DK * 128), j0 + 32 * bx,
+                                             (int)(((size_t)bh * NC + c) * DK));
+                            bulk_commit();
+                        }
+                    }
+                }
             }
             // state update S = diag(gamma) S + diag(cfac) (Kt^T Vh)
             {
@@ -815,6 +847,9 @@ cudaError_t launch_cfg(const SeqParams& p, SegPlan plan, cudaStream_t s) {
         !make_tmap_bf16_3d(&a.mv, p.v, p.dv, p.T, BH, 64, 64) ||
         !make_tmap_bf16_3d(&a.mb, p.beta, p.dv, p.T, BH, 64, 64) ||
         !make_tmap_bf16_3d(&a.mo, p.o, p.dv, p.T, BH, 64, 64))
+        return cudaErrorInvalidValue;
+    if (Cfg<DK, DVT>::STAGE_SAVED && p.saved &&
+        !make_tmap_f32_2d(&a.msv, p.saved, p.dv, BH * (uint64_t)((p.T + C - 1) / C) * DK, 32, DK))
         return cudaErrorInvalidValue;
     const size_t smem = sizeof(FwdSmem<DK, DVT>) + 1024;
     auto kern = tc_fwd_kernel<DK, DVT, PRE>;

@@ -41,6 +41,20 @@ bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t n0, uint64_t
     return r == CUDA_SUCCESS;
 }
 
+bool make_tmap_f32_2d(CUtensorMap* map, const void* base, uint64_t n0, uint64_t n1, uint32_t b0,
+                      uint32_t b1) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {n0, n1};
+    cuuint64_t strides[1] = {n0 * 4};
+    cuuint32_t box[2] = {b0, b1};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 int sm_count() {
     static int cache[64];
     int dev = 0;
