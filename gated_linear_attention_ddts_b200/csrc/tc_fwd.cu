@@ -20,12 +20,15 @@
 // each unit's chunks are cut into P contiguous segments, one CTA each.  The
 // state map of a segment is affine, S_out = diag(D) S_in + S_loc, with D the
 // product of its decays and S_loc its state from a zero start.  A segment
-// first runs the state recurrence alone from zero (no Qt, A or o) and
-// publishes (S_loc, log2 D) through global memory; it then folds the maps of
-// all earlier segments onto S_0 to obtain its true entry state and runs the
-// full forward over its chunks.  The last segment skips the first pass.  All
-// CTAs of such a launch are resident together (cooperative launch), and every
-// cross-CTA wait is bounded.
+// first computes S_loc alone (no Qt, A or o): with G_s the running sum of
+// log(alpha) over the segment, S_loc = sum_s (k_s alpha_hat_s exp(G_end - G_s))
+// (beta_hat_s v_s)^T, every factor <= 1, so the products of all its chunks
+// accumulate into one tensor-memory sum (chunks taken last to first, which
+// gives G_end - G_s as a running sum).  It publishes (S_loc, log2 D) through
+// global memory, folds the maps of all earlier segments onto S_0 to obtain its
+// true entry state and runs the full forward over its chunks.  The last
+// segment skips the first pass.  All CTAs of such a launch are resident
+// together (cooperative launch), and every cross-CTA wait is bounded.
 //
 // One CTA owns one (b,h), a d_v slice of DVT columns and a segment.  Roles:
 //   warps 0-7   epilogue: A -> masked bf16 operand, state (fp32 registers),
@@ -37,6 +40,8 @@
 // All hand-offs are mbarriers with bounded waits (a timeout sets the device
 // status word and the CTA exits cleanly).
 #include <cuda.h>
+
+#include <type_traits>
 
 #include "launch.h"
 #include "rdm_common.cuh"
@@ -55,6 +60,7 @@ constexpr int kEpiWarp0 = 0, kGateWarp0 = kEpiWarps, kProdWarp = kEpiWarps + kGa
 constexpr int kBarGate = 3;        // all gate warps
 constexpr int kBarEpi = 4;         // all epilogue warps
 constexpr int kMinSegChunks = 4;   // shortest segment worth a CTA of its own
+constexpr int kAhead = 2;          // L2 prefetch distance of the producer, in passes
 
 template <int DK, int DVT>
 struct Cfg {
@@ -144,8 +150,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
     const int nseg = c1 - c0;
     const bool has_p1 = seg < P - 1;        // runs the state-only first pass
     const int nL = (has_p1 ? 2 : 1) * nseg;  // chunk passes
-    // pass li: phase 1 (state only) for the first nseg passes when has_p1, else phase 2
-    auto pass_chunk = [&](int li) { return c0 + (li < nseg ? li : li - nseg); };
+    // pass li: phase 1 (state only, chunks last to first) for the first nseg
+    // passes when has_p1, else phase 2 (chunks in order)
+    auto pass_chunk = [&](int li) {
+        return !has_p1 ? c0 + li : li < nseg ? c1 - 1 - li : c0 + li - nseg;
+    };
     auto pass_p2 = [&](int li) { return !has_p1 || li >= nseg; };
 
     if (threadIdx.x == 0) {
@@ -205,6 +214,21 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                     tma_load_3d(raw + (3 * KB + kb) * kBox, &A.mt, &sm.raw_full[st], 64 * kb, c * C, bh);
                 }
                 ++issued;
+                // the tiles of the pass kAhead further on, into L2
+                if (li + kAhead < nL) {
+                    const int ca = pass_chunk(li + kAhead);
+                    const bool qa = pass_p2(li + kAhead);
+                    for (int kb = 0; kb < KB; ++kb) {
+                        if (qa) tma_prefetch_3d(&A.mq, 64 * kb, ca * C, bh);
+                        tma_prefetch_3d(&A.mk, 64 * kb, ca * C, bh);
+                        tma_prefetch_3d(&A.mg, 64 * kb, ca * C, bh);
+                        tma_prefetch_3d(&A.mt, 64 * kb, ca * C, bh);
+                    }
+                    for (int vb = 0; vb < VB; ++vb) {
+                        tma_prefetch_3d(&A.mv, j0 + 64 * vb, ca * C, bh);
+                        tma_prefetch_3d(&A.mb, j0 + 64 * vb, ca * C, bh);
+                    }
+                }
                 if (li >= 1 && !mbar_wait(&sm.v_empty, (li - 1) & 1, fail, kWaitLimit)) break;
                 mbar_expect_tx(&sm.v_full, K::RAWV);
                 for (int vb = 0; vb < VB; ++vb) {
@@ -225,15 +249,22 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             constexpr uint32_t id1 = idesc_bf16(64, 64, 0, 0);    // A  = Qt Kt^T
             constexpr uint32_t idS = idesc_bf16(DK, DVT, 1, 1);   // dS = Kt^T Vh
             constexpr uint32_t idO = idesc_bf16(64, DVT, 0, 1);   // O  = A Vh + Qt S_hat
-            int item = 0, n1 = 0, io = 0;  // io counts the items that produce o
+            // io counts the items that produce o, nas the waits for the epilogue to
+            // release A and dS (before every item of the full pass but the first item
+            // of the launch; the state-only pass accumulates into dS unreleased)
+            int item = 0, n1 = 0, io = 0, nas = 0;
             while (true) {
                 const int ob = item % NB;
                 if (!mbar_wait(&sm.ops_full[ob], (item / NB) & 1, fail, kWaitLimit)) break;
                 const int last = sm.info[ob][kInfoLast];
                 const bool p2 = sm.info[ob][kInfoPhase] == 2;
+                const bool p1last = sm.info[ob][kInfoP1Last];
                 if constexpr (kVhEpi)
                     if (!mbar_wait(&sm.vh_full[ob], (item / NB) & 1, fail, kWaitLimit)) break;
-                if (item > 0 && !mbar_wait(&sm.as_free, (item - 1) & 1, fail, kWaitLimit)) break;
+                if (p2 && item > 0) {
+                    if (!mbar_wait(&sm.as_free, nas & 1, fail, kWaitLimit)) break;
+                    ++nas;
+                }
                 tc_fence_after();
                 const uint32_t q = smem_u32(sm.qt[ob]) >> 4, k = smem_u32(sm.kt[ob]) >> 4;
                 const uint32_t v = smem_u32(sm.vh[ob]) >> 4;
@@ -246,9 +277,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
 #pragma unroll
                 for (int ks = 0; ks < C / 16; ++ks)
                     mma_bf16_w(tS, k + sd_lo(ks * 256, 128), sd_hi(kQK), v + sd_lo(ks * 256, 128),
-                               sd_hi(1024), idS, ks > 0);
-                mma_commit(&sm.mma1_done);
-                ++n1;
+                               sd_hi(1024), idS, ks > 0 || (!p2 && item > 0));
+                if (p2 || p1last) {
+                    mma_commit(&sm.mma1_done);
+                    ++n1;
+                }
                 if (p2) {
                     if (!mbar_wait(&sm.abf_full, io & 1, fail, kWaitLimit)) break;
                     const int obuf = io & 1;
@@ -292,10 +325,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
         const int tb = seg_l * SEGT;  // first token of my segment
         const uint32_t full = 0xffffffffu;
         int item = 0;
-        for (int li = 0; li < nL; ++li) {
+        float gt2[8];  // state-only pass: log2 decay of the chunks after the current one
+#pragma unroll
+        for (int e = 0; e < 8; ++e) gt2[e] = 0.0f;
+        // one pass over a chunk; kP2 selects the full pass at compile time (so the
+        // state-only pass's registers are free in the other); false stops the role
+        auto pass = [&](int li, auto kP2) -> bool {
             const int st = li % NS, c = pass_chunk(li);
-            const bool p2 = pass_p2(li);
-            if (!mbar_wait(&sm.raw_full[st], (li / NS) & 1, fail, kWaitLimit)) break;
+            constexpr bool p2 = decltype(kP2)::value;
+            if (!mbar_wait(&sm.raw_full[st], (li / NS) & 1, fail, kWaitLimit)) return false;
             const uint8_t* raw = sm.raw[st];
             const int nval = min(C, T - c * C);
             // log2(alpha_hat) of my tokens is kept from the scan for the operand pass
@@ -357,16 +395,6 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                 named_bar(kBarGate, 32 * kGateWarps);
                 return *flag == li + 1;
             };
-            int W = C;
-            scan(C);
-            if (too_wide(&sm.need16[li & 1])) {
-                W = 16;
-                scan(16);
-                if (too_wide(&sm.need1[li & 1])) {
-                    W = 1;
-                    scan(1);
-                }
-            }
             // Vh = beta_hat * v for the rows of [w0, w1), zero elsewhere
             bool have_v = false;
             auto write_vh = [&](int ob, int w0, int w1) {
@@ -390,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             };
             auto publish = [&](int ob, int w0, int w1) {
                 if (gt == 0) {
-                    const bool end = (c == c1 - 1) && (w1 == nval);
+                    const bool end = p2 ? (c == c1 - 1) && (w1 == nval) : li == nseg - 1;
                     sm.info[ob][kInfoChunk] = c;
                     sm.info[ob][kInfoW0] = w0;
                     sm.info[ob][kInfoW1] = w1;
@@ -403,15 +431,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm.ops_full[ob]);
             };
-            if (W == C) {
-                // ---- one window = the whole chunk (rows past T hold zeros from the
-                // TMA fill, so every row can be computed unmasked)
+            if constexpr (!p2) {
+                // ---- state-only pass (chunks last to first, all of them whole):
+                // Kt = k alpha_hat exp(G_end - G_s), G_end - G_s = gt2 (the decay of
+                // the later chunks, log2) + b_last - b_s; every factor <= 1
+                scan(C);
                 const int ob = item % NB;
                 if (item >= NB && !mbar_wait(&sm.ops_empty[ob], ((item / NB) - 1) & 1, fail, kWaitLimit))
-                    break;
-                float mL[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) mL[e] = 0.5f * (bf[e] + bl[e]) * kLog2e;
+                    return false;
 #pragma unroll
                 for (int u = 0; u < SEGT; ++u) {
                     const int t = tb + u;
@@ -428,7 +455,57 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
 #pragma unroll
                         for (int e = 0; e < 8; ++e) lah[e] = t8[e] == 0.0f ? 0.0f : t8[e] * lg2_fast(g8[e]);
                     }
-                    if (p2) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        ok[e] = k8[e] * ex2_fast(lah[e] + fmaf(bl[e] - b[u][e], kLog2e, gt2[e]));
+                    *reinterpret_cast<uint4*>(sm.kt[ob] + off_qk(t, cg * 8)) = pack8(ok);
+                }
+#pragma unroll
+                for (int e = 0; e < 8; ++e) gt2[e] = fmaf(bl[e], kLog2e, gt2[e]);
+                // log2 of the segment's decay product, for the epilogue
+                if (tb == 0 && li == nseg - 1) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) sm.gm[ob][cg * 8 + e] = gt2[e];
+                }
+                write_vh(ob, 0, C);
+                publish(ob, 0, C);
+                ++item;
+            } else {
+                int W = C;
+                scan(C);
+                if (too_wide(&sm.need16[li & 1])) {
+                    W = 16;
+                    scan(16);
+                    if (too_wide(&sm.need1[li & 1])) {
+                        W = 1;
+                        scan(1);
+                    }
+                }
+                if (W == C) {
+                    // ---- one window = the whole chunk (rows past T hold zeros from the
+                    // TMA fill, so every row can be computed unmasked)
+                    const int ob = item % NB;
+                    if (item >= NB && !mbar_wait(&sm.ops_empty[ob], ((item / NB) - 1) & 1, fail, kWaitLimit))
+                        return false;
+                    float mL[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) mL[e] = 0.5f * (bf[e] + bl[e]) * kLog2e;
+#pragma unroll
+                    for (int u = 0; u < SEGT; ++u) {
+                        const int t = tb + u;
+                        float k8[8], lah[8], ok[8];
+                        unpack8(*reinterpret_cast<const uint4*>(raw + 1 * KB * kBox + off_raw(t, cg)), k8);
+                        if constexpr (kKeepLah) {
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) lah[e] = lah2[u][e];
+                        } else {
+                            float g8[8], t8[8];
+                            unpack8(*reinterpret_cast<const uint4*>(raw + 2 * KB * kBox + off_raw(t, cg)), g8);
+                            unpack8(*reinterpret_cast<const uint4*>(raw + 3 * KB * kBox + off_raw(t, cg)), t8);
+                            if constexpr (PRE) activate_gates8(g8, t8);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) lah[e] = t8[e] == 0.0f ? 0.0f : t8[e] * lg2_fast(g8[e]);
+                        }
                         float q8[8], oq[8];
                         unpack8(*reinterpret_cast<const uint4*>(raw + 0 * KB * kBox + off_raw(t, cg)), q8);
 #pragma unroll
@@ -438,77 +515,76 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                             ok[e] = k8[e] * ex2_fast(lah[e] - d);
                         }
                         *reinterpret_cast<uint4*>(sm.qt[ob] + off_qk(t, cg * 8)) = pack8(oq);
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const float d = fmaf(b[u][e], kLog2e, -mL[e]);
-                            ok[e] = k8[e] * ex2_fast(lah[e] - d);
-                        }
-                    }
-                    *reinterpret_cast<uint4*>(sm.kt[ob] + off_qk(t, cg * 8)) = pack8(ok);
-                }
-                if (tb == 0) {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        sm.em[ob][cg * 8 + e] = ex2_fast(mL[e]);
-                        sm.cf[ob][cg * 8 + e] = ex2_fast(bl[e] * kLog2e - mL[e]);
-                        sm.gm[ob][cg * 8 + e] = ex2_fast(bl[e] * kLog2e);
-                    }
-                }
-                write_vh(ob, 0, C);
-                publish(ob, 0, nval);
-                ++item;
-            } else {
-                bool ok_loop = true;
-                for (int w0 = 0; w0 < nval; w0 += W) {
-                    const int w1 = min(w0 + W, nval);
-                    const int ob = item % NB;
-                    if (item >= NB &&
-                        !mbar_wait(&sm.ops_empty[ob], ((item / NB) - 1) & 1, fail, kWaitLimit)) {
-                        ok_loop = false;
-                        break;
-                    }
-#pragma unroll 1
-                    for (int u = 0; u < SEGT; ++u) {
-                        const int t = tb + u;
-                        const bool in = t >= w0 && t < w1;
-                        float q8[8], k8[8], g8[8], t8[8], oq[8], ok[8];
-                        unpack8(*reinterpret_cast<const uint4*>(raw + 0 * KB * kBox + off_raw(t, cg)), q8);
-                        unpack8(*reinterpret_cast<const uint4*>(raw + 1 * KB * kBox + off_raw(t, cg)), k8);
-                        unpack8(*reinterpret_cast<const uint4*>(raw + 2 * KB * kBox + off_raw(t, cg)), g8);
-                        unpack8(*reinterpret_cast<const uint4*>(raw + 3 * KB * kBox + off_raw(t, cg)), t8);
-                        if constexpr (PRE) activate_gates8(g8, t8);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            // reference m = midpoint of the window's b range, blast = b at its end
-                            const float blast = W == 1 ? b[u][e] : bl[e];
-                            const float m = W == 1 ? b[u][e] : 0.5f * (bf[e] + bl[e]);
-                            const float d = (b[u][e] - m) * kLog2e;
-                            const float lah = t8[e] == 0.0f ? 0.0f : t8[e] * lg2_fast(g8[e]);
-                            oq[e] = (in && p2) ? q8[e] * ex2_fast(d) : 0.0f;
-                            ok[e] = in ? k8[e] * ex2_fast(lah - d) : 0.0f;
-                            if (t == w0) {
-                                sm.em[ob][cg * 8 + e] = ex2_fast(m * kLog2e);
-                                sm.cf[ob][cg * 8 + e] = ex2_fast((blast - m) * kLog2e);
-                                sm.gm[ob][cg * 8 + e] = ex2_fast(blast * kLog2e);
-                            }
-                        }
-                        *reinterpret_cast<uint4*>(sm.qt[ob] + off_qk(t, cg * 8)) = pack8(oq);
                         *reinterpret_cast<uint4*>(sm.kt[ob] + off_qk(t, cg * 8)) = pack8(ok);
                     }
-                    write_vh(ob, w0, w1);
-                    publish(ob, w0, w1);
+                    if (tb == 0) {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            sm.em[ob][cg * 8 + e] = ex2_fast(mL[e]);
+                            sm.cf[ob][cg * 8 + e] = ex2_fast(bl[e] * kLog2e - mL[e]);
+                            sm.gm[ob][cg * 8 + e] = ex2_fast(bl[e] * kLog2e);
+                        }
+                    }
+                    write_vh(ob, 0, C);
+                    publish(ob, 0, nval);
                     ++item;
+                } else {
+                    bool ok_loop = true;
+                    for (int w0 = 0; w0 < nval; w0 += W) {
+                        const int w1 = min(w0 + W, nval);
+                        const int ob = item % NB;
+                        if (item >= NB &&
+                            !mbar_wait(&sm.ops_empty[ob], ((item / NB) - 1) & 1, fail, kWaitLimit)) {
+                            ok_loop = false;
+                            break;
+                        }
+#pragma unroll 1
+                        for (int u = 0; u < SEGT; ++u) {
+                            const int t = tb + u;
+                            const bool in = t >= w0 && t < w1;
+                            float q8[8], k8[8], g8[8], t8[8], oq[8], ok[8];
+                            unpack8(*reinterpret_cast<const uint4*>(raw + 0 * KB * kBox + off_raw(t, cg)), q8);
+                            unpack8(*reinterpret_cast<const uint4*>(raw + 1 * KB * kBox + off_raw(t, cg)), k8);
+                            unpack8(*reinterpret_cast<const uint4*>(raw + 2 * KB * kBox + off_raw(t, cg)), g8);
+                            unpack8(*reinterpret_cast<const uint4*>(raw + 3 * KB * kBox + off_raw(t, cg)), t8);
+                            if constexpr (PRE) activate_gates8(g8, t8);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                // reference m = midpoint of the window's b range, blast = b at its end
+                                const float blast = W == 1 ? b[u][e] : bl[e];
+                                const float m = W == 1 ? b[u][e] : 0.5f * (bf[e] + bl[e]);
+                                const float d = (b[u][e] - m) * kLog2e;
+                                const float lah = t8[e] == 0.0f ? 0.0f : t8[e] * lg2_fast(g8[e]);
+                                oq[e] = in ? q8[e] * ex2_fast(d) : 0.0f;
+                                ok[e] = in ? k8[e] * ex2_fast(lah - d) : 0.0f;
+                                if (t == w0) {
+                                    sm.em[ob][cg * 8 + e] = ex2_fast(m * kLog2e);
+                                    sm.cf[ob][cg * 8 + e] = ex2_fast((blast - m) * kLog2e);
+                                    sm.gm[ob][cg * 8 + e] = ex2_fast(blast * kLog2e);
+                                }
+                            }
+                            *reinterpret_cast<uint4*>(sm.qt[ob] + off_qk(t, cg * 8)) = pack8(oq);
+                            *reinterpret_cast<uint4*>(sm.kt[ob] + off_qk(t, cg * 8)) = pack8(ok);
+                        }
+                        write_vh(ob, w0, w1);
+                        publish(ob, w0, w1);
+                        ++item;
+                    }
+                    if (!ok_loop) return false;
                 }
-                if (!ok_loop) break;
             }
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(&sm.raw_empty[st]);
                 if constexpr (!kVhEpi) mbar_arrive(&sm.v_empty);
             }
-            if (*fail) break;
-        }
+            return !*fail;
+        };
+        int li = 0;
+        bool run = true;
+        if (has_p1)
+            for (; run && li < nseg; ++li) run = pass(li, std::false_type{});
+        for (; run && li < nL; ++li) run = pass(li, std::true_type{});
     } else {
         // ------------------------------------------------------------ epilogue
         // A and O are M = 64 accumulators (TMEM lanes 0-15 of each sub-partition):
@@ -632,8 +708,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
         } else {
             ok_run = fold_earlier();
         }
-        float ld2 = 0.0f;  // log2 of this segment's decay product (first pass)
-        int item = 0, io = 0, pc = 0, pw0 = 0, pw1 = 0;
+        int item = 0, io = 0, nm1 = 0, pc = 0, pw0 = 0, pw1 = 0;
         while (ok_run) {
             const int ob = item % NB;
             if (!mbar_wait(&sm.ops_full[ob], (item / NB) & 1, fail, kWaitLimit)) break;
@@ -668,9 +743,34 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                     if (w1 == nval) mbar_arrive(&sm.v_empty);  // last window of the chunk
                 }
             }
-            if (!mbar_wait(&sm.mma1_done, item & 1, fail, kWaitLimit)) break;
+            if (!p2) {
+                // state-only pass: nothing to read until its last item, after which dS
+                // holds S_loc and the slot holds log2 D
+                if (p1last) {
+                    const float ld2 = sm.gm[ob][iS];
+                    if (!mbar_wait(&sm.mma1_done, nm1 & 1, fail, kWaitLimit)) break;
+                    ++nm1;
+                    tc_fence_after();
+                    ld_cols(K::COL_S, S, true);
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) {
+                        mbar_arrive(&sm.as_free);
+                        mbar_arrive(&sm.ops_empty[ob]);
+                    }
+                    publish_segment(ld2);
+                    if (!fold_earlier()) break;
+                } else {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sm.ops_empty[ob]);
+                }
+                ++item;
+                continue;
+            }
+            if (!mbar_wait(&sm.mma1_done, nm1 & 1, fail, kWaitLimit)) break;
+            ++nm1;
             tc_fence_after();
-            if (p2) {
+            {
                 // A -> causal mask -> bf16 operand (row t = tA, columns s = a0 + e)
                 {
                     const int a0 = 32 * hf + 16 * eh;
@@ -735,7 +835,6 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             // state update S = diag(gamma) S + diag(cfac) (Kt^T Vh)
             {
                 const float gmv = sm.gm[ob][iS], cfv = sm.cf[ob][iS];
-                if (!p2) ld2 += lg2_fast(gmv);
                 float v[SC];
                 ld_cols(K::COL_S, v, true);
 #pragma unroll
@@ -748,22 +847,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             // once the tensor core is done with it too
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.ops_empty[ob]);
-            if (p2) {
-                // o of the previous o-item (its MMA finished while this item's A and
-                // state were processed), then of this one if it is the last
-                if (io > 0 && !store_o(io - 1, pc, pw0, pw1)) break;
-                if (last) {
-                    store_o(io, c, w0, w1);
-                    break;
-                }
-                pc = c;
-                pw0 = w0;
-                pw1 = w1;
-                ++io;
-            } else if (p1last) {
-                publish_segment(ld2);
-                if (!fold_earlier()) break;
+            // o of the previous o-item (its MMA finished while this item's A and
+            // state were processed), then of this one if it is the last
+            if (io > 0 && !store_o(io - 1, pc, pw0, pw1)) break;
+            if (last) {
+                store_o(io, c, w0, w1);
+                break;
             }
+            pc = c;
+            pw0 = w0;
+            pw1 = w1;
+            ++io;
             ++item;
         }
         if (threadIdx.x == 0) bulk_wait_all();  // the o stores have landed

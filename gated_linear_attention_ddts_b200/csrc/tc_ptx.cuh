@@ -255,6 +255,14 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const void* tmap, uint64_
         : "memory");
 }
 
+// TMA L2 prefetch of one tile (no shared-memory destination, no completion to
+// wait for): brings a later tile toward the SM while earlier ones are in use.
+__device__ __forceinline__ void tma_prefetch_3d(const void* tmap, int c0, int c1, int c2) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];"
+                 ::"l"(tmap), "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
+}
+
 // TMA tile store shared -> global (bulk-group completion).  Rows or columns
 // of the box that fall outside the tensor are not written.
 __device__ __forceinline__ void tma_store_3d(const void* tmap, const void* src, int c0, int c1,
