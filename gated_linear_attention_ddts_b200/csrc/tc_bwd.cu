@@ -32,9 +32,12 @@
 // Sequence segments (when the heads alone do not fill the GPU): each head's
 // chunks are cut into P contiguous segments, one CTA each.  R maps affinely
 // across a segment, R_start = diag(D) R_end + R_loc, so every segment but the
-// first first runs the R recurrence alone from zero at its end (Qt and dO
-// only) and publishes (R_loc, log2 D); a segment then folds the maps of all
-// later segments onto dS_T to obtain its R_end.  The decay-gradient carry
+// first first computes R_loc alone (q, g, tau and dO only) and publishes
+// (R_loc, log2 D); a segment then folds the maps of all later segments onto
+// dS_T to obtain its R_end.  With G_t the running sum of log(alpha) from the
+// segment start, R_loc = sum_t (q_t exp(G_t)) dO_t^T, every factor <= 1: the
+// products of all its chunks accumulate into one tensor-memory sum (chunks
+// taken first to last, which gives G_t as a running sum).  The decay-gradient carry
 // into a segment, the suffix sum of (q dq - khat dkhat) over all later tokens
 // plus rowsum(dS_T o S_T), equals rowsum(R_end o S_end) with S_end the state
 // at the segment end (rescaling row i of q by e^eps and of khat and S_0 by
@@ -102,7 +105,7 @@ struct alignas(1024) BwdSmem {
     float em[DK], cf[DK], gm[DK], fin[DK], carry[DK];
     float bdiag[C];  // B_tt = vhat_t . dO_t (the diagonal kept out of the dQ / dK MMAs)
     uint64_t raw_full, raw_empty, sp_full, ops_full, shat_full, ops_empty, g1_done, g2_ready,
-        tm1_free, g2_done, tm2_free, post_ready, post_done;
+        tm1_free, g2_done, tm2_free, post_ready, post_done, p1_done;
     uint32_t tmem_base;
     int fail;
 };
@@ -152,8 +155,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
     const int nseg = cs1 - cs0;
     const bool has_p1 = seg > 0;             // runs the R-only first pass
     const bool last_seg = seg == P - 1;      // its R_end is dS_T
-    const int nL = (has_p1 ? 2 : 1) * nseg;  // chunk passes, each over [cs0, cs1) last chunk first
-    auto pass_chunk = [&](int li) { return cs1 - 1 - (li < nseg ? li : li - nseg); };
+    // chunk passes: the R-only pass over [cs0, cs1) first chunk first, then the
+    // full pass last chunk first
+    const int nL = (has_p1 ? 2 : 1) * nseg;
+    auto pass_chunk = [&](int li) {
+        return !has_p1 ? cs1 - 1 - li : li < nseg ? cs0 + li : cs1 - 1 - (li - nseg);
+    };
     auto pass_p2 = [&](int li) { return !has_p1 || li >= nseg; };
 
     if (threadIdx.x == 0) {
@@ -170,6 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
         mbar_init(&sm.tm2_free, 4);
         mbar_init(&sm.post_ready, 4);
         mbar_init(&sm.post_done, kGateWarps);
+        mbar_init(&sm.p1_done, kGateWarps);
         sm.fail = 0;
         fence_mbar_init();
     }
@@ -246,17 +254,22 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 const bool p2 = pass_p2(li);
                 const int i2 = n2;  // index among full passes
                 if (!mbar_wait(&sm.ops_full, li & 1, fail, kWaitLimit)) break;
-                if (li > 0 && !mbar_wait(&sm.tm1_free, (li - 1) & 1, fail, kWaitLimit)) break;
+                // group-1 accumulators released by the epilogue: after the R-only
+                // pass, and after each full pass (tm1_free completes once for each)
+                const int ntf = i2 + (has_p1 ? 1 : 0);
+                if (p2 && ntf > 0 && !mbar_wait(&sm.tm1_free, (ntf - 1) & 1, fail, kWaitLimit)) break;
                 tc_fence_after();
                 if (!p2) {
-                    // R-only pass: dR = Qt^T dO
+                    // R-only pass: R_loc += Qt^T dO over all its chunks
 #pragma unroll
                     for (int ks = 0; ks < C / 16; ++ks)
                         mma_bf16(tmem + K::COL_DR, sdesc(q + ks * 256, 128, kQK),
-                                 sdesc(d + ks * 256, 128, 1024), id_r, ks > 0);
-                    mma_commit(&sm.g1_done);
+                                 sdesc(d + ks * 256, 128, 1024), id_r, ks > 0 || li > 0);
+                    if (li == nseg - 1) {
+                        mma_commit(&sm.g1_done);
+                        ++n1;
+                    }
                     mma_commit(&sm.ops_empty);
-                    ++n1;
                     continue;
                 }
 #pragma unroll
@@ -338,6 +351,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
         const uint32_t full = 0xffffffffu;
         const uint8_t* raw = sm.raw;
         int i2 = 0;  // full passes done
+        float gh2[8];  // R-only pass: log2 decay from the segment start to this chunk
+#pragma unroll
+        for (int e = 0; e < 8; ++e) gh2[e] = 0.0f;
         for (int li = 0; li < nL; ++li) {
             const int c = pass_chunk(li);
             const bool p2 = pass_p2(li);
@@ -383,31 +399,37 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                     span = fmaxf(span, bf - bl);
                 }
                 // too wide for one reference: the exact path recomputes this head
-                if (__any_sync(full, !(span <= kSpanMax)) && lane == 0) A.flags[bh] = 1;
+                // (the R-only pass needs no reference)
+                if (p2 && __any_sync(full, !(span <= kSpanMax)) && lane == 0) A.flags[bh] = 1;
             }
-            // operand slot free: tensor core done with it (ops_empty) and the epilogue
-            // done with the constants (tm1_free; it consumes em / cf / gm in its
+            // operand slot free: tensor core done with it (ops_empty) and, for a full
+            // pass, the epilogue done with the constants (tm1_free, once after the
+            // R-only pass and once per full pass; it consumes em / cf / gm in its
             // first stage)
-            if (li > 0 && (!mbar_wait(&sm.ops_empty, (li - 1) & 1, fail, kWaitLimit) ||
-                           !mbar_wait(&sm.tm1_free, (li - 1) & 1, fail, kWaitLimit)))
-                break;
+            if (li > 0 && !mbar_wait(&sm.ops_empty, (li - 1) & 1, fail, kWaitLimit)) break;
+            if (p2) {
+                const int ntf = i2 + (has_p1 ? 1 : 0);
+                if (ntf > 0 && !mbar_wait(&sm.tm1_free, (ntf - 1) & 1, fail, kWaitLimit)) break;
+            }
             if (!p2) {
-                // R-only pass: Qt (bf16), the constants and dO
+                // R-only pass: Qt = q exp(G_t) relative to the segment start (gh2 the
+                // decay of the earlier chunks, log2; every factor <= 1), and dO
 #pragma unroll
                 for (int u = 0; u < SEGT; ++u) {
                     const int t = tb + u;
                     float q8[8], oq[8];
                     unpack8(*reinterpret_cast<const uint4*>(raw + 0 * kBox + off_raw(t, cg)), q8);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) oq[e] = q8[e] * ex2_fast(fmaf(b[u][e], kLog2e, -mL[e]));
+                    for (int e = 0; e < 8; ++e) oq[e] = q8[e] * ex2_fast(fmaf(b[u][e], kLog2e, gh2[e]));
                     *reinterpret_cast<uint4*>(sm.qt + off_qk(t, cg * 8)) = pack8(oq);
                 }
-                if (tb == 0) {
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        sm.em[cg * 8 + e] = ex2_fast(mL[e]);
-                        sm.gm[cg * 8 + e] = ex2_fast(blL[e]);
-                    }
+                for (int e = 0; e < 8; ++e) gh2[e] += blL[e];
+                const bool p1last = li == nseg - 1;
+                // log2 of the segment's decay product, for the epilogue
+                if (p1last && tb == 0) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) sm.gm[cg * 8 + e] = gh2[e];
                 }
 #pragma unroll
                 for (int iv = 0; iv < VIT; ++iv) {
@@ -420,6 +442,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 if (lane == 0) {
                     mbar_arrive(&sm.ops_full);
                     mbar_arrive(&sm.raw_empty);
+                    if (p1last) mbar_arrive(&sm.p1_done);
                 }
                 if (*fail) break;
                 continue;
@@ -692,35 +715,32 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
         } else {
             ok_run = fold_later();
         }
-        float ld2 = 0.0f;  // log2 of this segment's decay product (R-only pass)
-        int i2 = 0;        // full passes done
-        for (int li = 0; ok_run && li < nL; ++li) {
-            const int c = pass_chunk(li);
-            const bool p2 = pass_p2(li);
-            if (!mbar_wait(&sm.ops_full, li & 1, fail, kWaitLimit)) break;
-            if (!mbar_wait(&sm.g1_done, li & 1, fail, kWaitLimit)) break;
-            tc_fence_after();
-            if (!p2) {
-                // R-only pass: R <- diag(e^{b_last}) R + diag(e^m) Qt^T dO
-                const float emv = sm.em[r], gmv = sm.gm[r];
-                ld2 += lg2_fast(gmv);
+        int i2 = 0;  // full passes done
+        if (ok_run && has_p1) {
+            // R-only pass: R_loc is the accumulated group-1 sum once its last
+            // chunk's products are done; log2 D comes from the gate warps
+            ok_run = mbar_wait(&sm.p1_done, 0, fail, kWaitLimit) &&
+                     mbar_wait(&sm.g1_done, 0, fail, kWaitLimit);
+            if (ok_run) {
+                tc_fence_after();
+                const float ld2 = sm.gm[r];
 #pragma unroll
                 for (int qd = 0; qd < HV / 32; ++qd) {
-                    float v[32];
-                    tmem_ld32_split<HV>(tmem + lb + K::COL_DR + 32 * qd, v);
+                    tmem_ld32_split<HV>(tmem + lb + K::COL_DR + 32 * qd, R + 32 * qd);
                     tmem_ld_wait();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) R[32 * qd + e] = fmaf(gmv, R[32 * qd + e], emv * v[e]);
                 }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm.tm1_free);
-                if (li == nseg - 1) {
-                    publish_segment(ld2);
-                    if (!fold_later()) break;
-                }
-                continue;
+                publish_segment(ld2);
+                ok_run = fold_later();
             }
+        }
+        for (int li = has_p1 ? nseg : 0; ok_run && li < nL; ++li) {
+            const int c = pass_chunk(li);
+            if (!mbar_wait(&sm.ops_full, li & 1, fail, kWaitLimit)) break;
+            if (!mbar_wait(&sm.g1_done, (i2 + (has_p1 ? 1 : 0)) & 1, fail, kWaitLimit)) break;
+            tc_fence_after();
             // the gate warps have read S_prev out of the union (and staged S_hat)
             if (!mbar_wait(&sm.shat_full, i2 & 1, fail, kWaitLimit)) break;
             // A and B -> causal mask -> bf16 operands (row t = r, columns s = 32 hf + e)
