@@ -221,6 +221,23 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                     tma_load_3d(sm.raw + K::OFF_DO + vb * kBox, &A.mdo, &sm.raw_full, 64 * vb, c * C, bh);
                 }
                 ++issued;
+                // the next pass's tiles (and chunk-start state) into L2 while this one runs
+                if (li + 1 < nL) {
+                    const int cn = pass_chunk(li + 1);
+                    const bool pn = pass_p2(li + 1);
+                    tma_prefetch_3d(&A.mq, 0, cn * C, bh);
+                    if (pn) tma_prefetch_3d(&A.mk, 0, cn * C, bh);
+                    tma_prefetch_3d(&A.mg, 0, cn * C, bh);
+                    tma_prefetch_3d(&A.mt, 0, cn * C, bh);
+                    for (int vb = 0; vb < VB; ++vb) {
+                        if (pn) {
+                            tma_prefetch_3d(&A.mv, 64 * vb, cn * C, bh);
+                            tma_prefetch_3d(&A.mb, 64 * vb, cn * C, bh);
+                        }
+                        tma_prefetch_3d(&A.mdo, 64 * vb, cn * C, bh);
+                    }
+                    if (pn) bulk_prefetch_l2(p.saved + ((size_t)bh * NC + cn) * DK * DV, DK * DV * 4);
+                }
                 if (p2) {
                     // chunk-start state, row by row into the skewed layout (the union
                     // is free: the previous full pass has finished its last stage)

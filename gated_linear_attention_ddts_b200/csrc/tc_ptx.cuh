@@ -263,6 +263,11 @@ __device__ __forceinline__ void tma_prefetch_3d(const void* tmap, int c0, int c1
                  : "memory");
 }
 
+// L2 prefetch of a contiguous global range (16-byte aligned, size a multiple of 16).
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // TMA tile store shared -> global (bulk-group completion).  Rows or columns
 // of the box that fall outside the tensor are not written.
 __device__ __forceinline__ void tma_store_3d(const void* tmap, const void* src, int c0, int c1,
