@@ -93,6 +93,14 @@ def chunk_flops_bwd(w, C=64):
     return w.B * w.H * w.T * ((C + 1) * (3 * w.dk + 2 * w.dv) + 10 * w.dk * w.dv)
 
 
+# sources (kernel file and the device headers it includes) that a stored ncu
+# traffic figure is keyed to: the figure is reported only while they are unchanged
+_DEV_HDR = ["tc_ptx.cuh", "tc_common.cuh", "rdm_common.cuh", "launch.h"]
+FWD_SRC = ["tc_fwd.cu"] + _DEV_HDR
+BWD_SRC = ["tc_bwd.cu"] + _DEV_HDR
+DECODE_SRC = ["decode.cu", "rdm_common.cuh", "launch.h"]
+
+
 def src_sha(*names):
     h = hashlib.sha256()
     for n in names:
@@ -263,7 +271,7 @@ def run_extras(rdm, dev, pk, K):
         "workload": w.name, "value": w.B * w.T / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
         "gpu_launches_per_step": 1,
         "roofline": roofline(fwd_bytes(w, True), chunk_flops_fwd(w), ms, pk,
-                             ncu_traffic("tc_fwd_kernel", ["tc_fwd.cu"], 2))}
+                             ncu_traffic("tc_fwd_kernel", FWD_SRC, 2))}
     del x, o, ST, wsf
     # headline forward with the gate activations fused (inputs are the
     # pre-activations; same bytes)
@@ -308,9 +316,9 @@ def run_extras(rdm, dev, pk, K):
         # once for heads the tensor-core kernel handled)
         "gpu_launches_per_step": 4,
         "roofline_fwd": roofline(fb, chunk_flops_fwd(w), msf, pk,
-                                 ncu_traffic("tc_fwd_kernel", ["tc_fwd.cu"], 3)),
+                                 ncu_traffic("tc_fwd_kernel", FWD_SRC, 3)),
         "roofline_bwd": roofline(bwd_bytes(w), chunk_flops_bwd(w), msb, pk,
-                                 ncu_traffic("tc_bwd_kernel", ["tc_bwd.cu"], 3)),
+                                 ncu_traffic("tc_bwd_kernel", BWD_SRC, 3)),
         "roofline_step": roofline(fb + bwd_bytes(w), chunk_flops_fwd(w) + chunk_flops_bwd(w),
                                   msf + msb, pk, None)}
     del x, o, saved, grads, ws, wsf
@@ -337,7 +345,7 @@ def run_extras(rdm, dev, pk, K):
         "workload": w.name, "value": w.B * steps / (ms / 1e3), "unit": "tokens/s",
         "ms_per_step": per, "ms_per_graph": ms, "gpu_launches_per_step": 1,
         "roofline": roofline(decode_bytes(w), 2 * w.B * w.H * w.dk * w.dv * 3, per, pk,
-                             ncu_traffic("decode_kernel", ["decode.cu"], 4), timed_alone=False)}
+                             ncu_traffic("decode_kernel", DECODE_SRC, 4), timed_alone=False)}
     del g, xd, S, od
     return out
 
@@ -452,7 +460,7 @@ def main():
         "gated_linear_attention_ddts_b200/workloads.py)", "config": cfg,
         "token_heads_per_s": value * w.H,
         "roofline": roofline(fwd_bytes(w, False), chunk_flops_fwd(w), ms, pk,
-                             ncu_traffic("tc_fwd_kernel", ["tc_fwd.cu"], 1)),
+                             ncu_traffic("tc_fwd_kernel", FWD_SRC, 1)),
         "clocks": clocks,
         "e2e": {"value": weak_scaling_value(w.B * w.T, world, e2e_ms), "unit": "tokens/s",
                 "ms_per_step": e2e_ms,
