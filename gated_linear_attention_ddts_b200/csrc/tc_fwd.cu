@@ -24,10 +24,13 @@
 // log(alpha) over the segment, S_loc = sum_s (k_s alpha_hat_s exp(G_end - G_s))
 // (beta_hat_s v_s)^T, every factor <= 1, so the products of all its chunks
 // accumulate into one tensor-memory sum (chunks taken last to first, which
-// gives G_end - G_s as a running sum).  It publishes (S_loc, log2 D) through
-// global memory, folds the maps of all earlier segments onto S_0 to obtain its
-// true entry state and runs the full forward over its chunks.  The last
-// segment skips the first pass.  All CTAs of such a launch are resident
+// gives G_end - G_s as a running sum).  The chunks before the last segment are
+// the ones whose maps are needed; that state-only work is shared equally by all
+// P CTAs (range j by segment j's CTA, cut in two where a segment boundary falls
+// inside it), so every CTA starts its full pass after (P-1)/P of a segment.
+// Each piece's (S_loc, log2 D) goes through global memory; a CTA folds the
+// pieces before its segment onto S_0 to obtain its true entry state and runs
+// the full forward over its chunks.  All CTAs of such a launch are resident
 // together (cooperative launch), and every cross-CTA wait is bounded.
 //
 // One CTA owns one (b,h), a d_v slice of DVT columns and a segment.  Roles:
@@ -60,6 +63,7 @@ constexpr int kEpiWarp0 = 0, kGateWarp0 = kEpiWarps, kProdWarp = kEpiWarps + kGa
 constexpr int kBarGate = 3;        // all gate warps
 constexpr int kBarEpi = 4;         // all epilogue warps
 constexpr int kMinSegChunks = 4;   // shortest segment worth a CTA of its own
+constexpr int kMaxSeg = 160;       // most segments per sequence
 constexpr int kAhead = 2;          // L2 prefetch distance of the producer, in passes
 
 template <int DK, int DVT>
@@ -100,13 +104,53 @@ struct alignas(1024) FwdSmem {
     uint64_t raw_full[K::NS], raw_empty[K::NS], v_full, v_empty, ops_full[K::NB], ops_empty[K::NB];
     uint64_t mma1_done, as_free, abf_full, mmao_done[2], o_free[2], vh_full[K::NB];
     int need16[2], need1[2];
+    uint8_t before[2 * kMaxSeg];  // state-only pieces that precede this CTA's segment
     uint32_t tmem_base;
     int fail;
 };
 
-// Segment exchange area (global): per (segment < P-1, unit) the local state
-// [DK][DVT] and log2 of the decay product per channel; per (segment, unit) a
-// flag that holds `epoch` once those are written.
+// Segment s covers chunks [seg_start(s), seg_start(s+1)).
+__host__ __device__ inline int seg_start(int s, int NC, int P) {
+    const unsigned long long x = (unsigned long long)s * (unsigned)NC;
+    return x <= 0xffffffffull ? (int)((unsigned)x / (unsigned)P) : (int)(x / (unsigned)P);
+}
+// State-only range [a0, a1) of segment j's CTA: the P-th part j of the chunks
+// before the last segment.  `mid` is the segment boundary strictly inside it
+// (a1 when none); the pieces are [a0, mid) (slot 2j) and [mid, a1) (slot 2j+1).
+struct P1Range {
+    int a0, a1, mid;
+};
+// (kept out of line: the integer divisions stay out of the role loops' code)
+__host__ __device__ __noinline__ P1Range p1_range(int j, int NC, int P) {
+    const int n1 = seg_start(P - 1, NC, P);
+    P1Range r;
+    r.a0 = seg_start(j, n1, P);
+    r.a1 = seg_start(j + 1, n1, P);
+    r.mid = r.a1;
+    for (int s = P - 1; s >= 1; --s) {
+        const int cs = seg_start(s, NC, P);
+        if (cs > r.a0 && cs < r.a1) r.mid = cs;
+    }
+    return r;
+}
+// true when no state-only range holds two segment boundaries (each range is
+// then at most two pieces)
+bool p1_ranges_ok(int NC, int P) {
+    for (int j = 0; j < P; ++j) {
+        const P1Range r = p1_range(j, NC, P);
+        int inside = 0;
+        for (int s = 1; s < P; ++s) {
+            const int cs = seg_start(s, NC, P);
+            inside += cs > r.a0 && cs < r.a1;
+        }
+        if (inside > 1 || r.a1 <= r.a0) return false;
+    }
+    return true;
+}
+
+// Segment exchange area (global): per (piece slot < 2P, unit) the local state
+// [DK][DVT] and log2 of the decay product per channel, and a flag that holds
+// `epoch` once those are written.
 struct SegArgs {
     int P;
     unsigned epoch;
@@ -146,16 +190,20 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
     const int bh = unit / NJ, j0 = (unit % NJ) * DVT;
     const int T = p.T, NC = (T + C - 1) / C;
     const int P = sg.P;
-    const int c0 = (int)((long long)seg * NC / P), c1 = (int)((long long)(seg + 1) * NC / P);
+    const int c0 = seg_start(seg, NC, P), c1 = seg_start(seg + 1, NC, P);
     const int nseg = c1 - c0;
-    const bool has_p1 = seg < P - 1;        // runs the state-only first pass
-    const int nL = (has_p1 ? 2 : 1) * nseg;  // chunk passes
-    // pass li: phase 1 (state only, chunks last to first) for the first nseg
-    // passes when has_p1, else phase 2 (chunks in order)
-    auto pass_chunk = [&](int li) {
-        return !has_p1 ? c0 + li : li < nseg ? c1 - 1 - li : c0 + li - nseg;
-    };
-    auto pass_p2 = [&](int li) { return !has_p1 || li >= nseg; };
+    // state-only range of this CTA (none when P == 1)
+    const P1Range g1 = P > 1 ? p1_range(seg, NC, P) : P1Range{0, 0, 0};
+    const int nP1 = g1.a1 - g1.a0;
+    const bool has_p1 = nP1 > 0, split1 = g1.mid < g1.a1;
+    const int nL = nP1 + nseg;  // chunk passes
+    // pass li: phase 1 (state only, chunks a1-1 down to a0) for the first nP1
+    // passes, then phase 2 (the segment's chunks in order)
+    auto pass_chunk = [&](int li) { return li < nP1 ? g1.a1 - 1 - li : c0 + li - nP1; };
+    auto pass_p2 = [&](int li) { return li >= nP1; };
+    // state-only chunks that open / close a piece (in processing order)
+    auto piece_open = [&](int c) { return c == g1.a1 - 1 || (split1 && c == g1.mid - 1); };
+    auto piece_close = [&](int c) { return c == g1.a0 || (split1 && c == g1.mid); };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
@@ -250,8 +298,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             constexpr uint32_t idS = idesc_bf16(DK, DVT, 1, 1);   // dS = Kt^T Vh
             constexpr uint32_t idO = idesc_bf16(64, DVT, 0, 1);   // O  = A Vh + Qt S_hat
             // io counts the items that produce o, nas the waits for the epilogue to
-            // release A and dS (before every item of the full pass but the first item
-            // of the launch; the state-only pass accumulates into dS unreleased)
+            // release A and dS (before every item that starts dS from zero, but the
+            // first item of the launch; a state-only piece accumulates into dS)
             int item = 0, n1 = 0, io = 0, nas = 0;
             while (true) {
                 const int ob = item % NB;
@@ -259,9 +307,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                 const int last = sm.info[ob][kInfoLast];
                 const bool p2 = sm.info[ob][kInfoPhase] == 2;
                 const bool p1last = sm.info[ob][kInfoP1Last];
+                const bool fresh = p2 || piece_open(sm.info[ob][kInfoChunk]);
                 if constexpr (kVhEpi)
                     if (!mbar_wait(&sm.vh_full[ob], (item / NB) & 1, fail, kWaitLimit)) break;
-                if (p2 && item > 0) {
+                if (fresh && item > 0) {
                     if (!mbar_wait(&sm.as_free, nas & 1, fail, kWaitLimit)) break;
                     ++nas;
                 }
@@ -277,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
 #pragma unroll
                 for (int ks = 0; ks < C / 16; ++ks)
                     mma_bf16_w(tS, k + sd_lo(ks * 256, 128), sd_hi(kQK), v + sd_lo(ks * 256, 128),
-                               sd_hi(1024), idS, ks > 0 || (!p2 && item > 0));
+                               sd_hi(1024), idS, ks > 0 || !fresh);
                 if (p2 || p1last) {
                     mma_commit(&sm.mma1_done);
                     ++n1;
@@ -418,7 +467,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             };
             auto publish = [&](int ob, int w0, int w1) {
                 if (gt == 0) {
-                    const bool end = p2 ? (c == c1 - 1) && (w1 == nval) : li == nseg - 1;
+                    const bool end = p2 ? (c == c1 - 1) && (w1 == nval) : piece_close(c);
                     sm.info[ob][kInfoChunk] = c;
                     sm.info[ob][kInfoW0] = w0;
                     sm.info[ob][kInfoW1] = w1;
@@ -433,8 +482,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             };
             if constexpr (!p2) {
                 // ---- state-only pass (chunks last to first, all of them whole):
-                // Kt = k alpha_hat exp(G_end - G_s), G_end - G_s = gt2 (the decay of
-                // the later chunks, log2) + b_last - b_s; every factor <= 1
+                // Kt = k alpha_hat exp(G_end - G_s) with G_end the end of the piece,
+                // G_end - G_s = gt2 (the decay of the piece's later chunks, log2) +
+                // b_last - b_s; every factor <= 1
+                if (piece_open(c)) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) gt2[e] = 0.0f;
+                }
                 scan(C);
                 const int ob = item % NB;
                 if (item >= NB && !mbar_wait(&sm.ops_empty[ob], ((item / NB) - 1) & 1, fail, kWaitLimit))
@@ -462,8 +516,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                 }
 #pragma unroll
                 for (int e = 0; e < 8; ++e) gt2[e] = fmaf(bl[e], kLog2e, gt2[e]);
-                // log2 of the segment's decay product, for the epilogue
-                if (tb == 0 && li == nseg - 1) {
+                // log2 of the piece's decay product, for the epilogue
+                if (tb == 0 && piece_close(c)) {
 #pragma unroll
                     for (int e = 0; e < 8; ++e) sm.gm[ob][cg * 8 + e] = gt2[e];
                 }
@@ -582,8 +636,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
         };
         int li = 0;
         bool run = true;
-        if (has_p1)
-            for (; run && li < nseg; ++li) run = pass(li, std::false_type{});
+        for (; run && li < nP1; ++li) run = pass(li, std::false_type{});
         for (; run && li < nL; ++li) run = pass(li, std::true_type{});
     } else {
         // ------------------------------------------------------------ epilogue
@@ -620,23 +673,35 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             for (int j = 0; j < SC; ++j)
                 S[j] = p.S0 ? p.S0[((size_t)bh * DK + iS) * p.dv + j0 + sc0 + j] : 0.0f;
         };
-        // entry state of this segment: S_0 carried through the maps of all
-        // earlier segments, S <- diag(D_s) S + S_loc_s
+        // entry state of this segment: S_0 carried through the maps of all the
+        // state-only pieces before it, in chunk order, S <- diag(D) S + S_loc
         auto fold_earlier = [&]() -> bool {
+            // which pieces: slot 2j + h is [a0, mid) or [mid, a1) of range j; one
+            // slot per thread (the range arithmetic divides 64-bit integers)
+            const int et = threadIdx.x - 32 * kEpiWarp0;
+            for (int slot = et; slot < 2 * P; slot += 32 * kEpiWarps) {
+                const P1Range r = p1_range(slot >> 1, NC, P);
+                const int lo = (slot & 1) ? r.mid : r.a0, hi = (slot & 1) ? r.a1 : r.mid;
+                sm.before[slot] = lo < hi && hi <= c0;
+            }
+            named_bar(kBarEpi, 32 * kEpiWarps);
             if (threadIdx.x == 0) {
                 const long long t0 = clock64();
-                for (int s = 0; s < seg && !*fail; ++s)
-                    while (ld_acquire_gpu(&sg.flag[s * units + unit]) != sg.epoch)
+                for (int slot = 0; slot < 2 * P && !*fail; ++slot) {
+                    if (!sm.before[slot]) continue;
+                    while (ld_acquire_gpu(&sg.flag[slot * units + unit]) != sg.epoch)
                         if (clock64() - t0 > kWaitLimit) {
                             *fail = 1;
                             break;
                         }
+                }
             }
             named_bar(kBarEpi, 32 * kEpiWarps);
             if (*fail) return false;
             load_s0();
-            for (int s = 0; s < seg; ++s) {
-                const size_t u = (size_t)s * units + unit;
+            for (int slot = 0; slot < 2 * P; ++slot) {
+                if (!sm.before[slot]) continue;
+                const size_t u = (size_t)slot * units + unit;
                 const float d = ex2_fast(__ldcg(&sg.ld[u * DK + iS]));
                 const float4* src = reinterpret_cast<const float4*>(sg.st + (u * DK + iS) * DVT + sc0);
 #pragma unroll
@@ -650,9 +715,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             }
             return true;
         };
-        // publish this segment's map (S_loc in S, log2 D in ld2)
-        auto publish_segment = [&](float ld2) {
-            const size_t u = (size_t)seg * units + unit;
+        // publish the map of a state-only piece (S_loc in S, log2 D in ld2)
+        auto publish_piece = [&](int slot, float ld2) {
+            const size_t u = (size_t)slot * units + unit;
             float4* dst = reinterpret_cast<float4*>(sg.st + (u * DK + iS) * DVT + sc0);
 #pragma unroll
             for (int j4 = 0; j4 < SC / 4; ++j4)
@@ -702,10 +767,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
         bool ok_run = true;
         if (P == 1) {
             load_s0();
-        } else if (has_p1) {
-#pragma unroll
-            for (int j = 0; j < SC; ++j) S[j] = 0.0f;
-        } else {
+        } else if (!has_p1) {
             ok_run = fold_earlier();
         }
         int item = 0, io = 0, nm1 = 0, pc = 0, pw0 = 0, pw1 = 0;
@@ -744,8 +806,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                 }
             }
             if (!p2) {
-                // state-only pass: nothing to read until its last item, after which dS
-                // holds S_loc and the slot holds log2 D
+                // state-only pass: nothing to read until the last chunk of a piece,
+                // after which dS holds its S_loc and the slot its log2 D; after the
+                // CTA's last piece (chunk a0), the entry state of its segment
                 if (p1last) {
                     const float ld2 = sm.gm[ob][iS];
                     if (!mbar_wait(&sm.mma1_done, nm1 & 1, fail, kWaitLimit)) break;
@@ -758,8 +821,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                         mbar_arrive(&sm.as_free);
                         mbar_arrive(&sm.ops_empty[ob]);
                     }
-                    publish_segment(ld2);
-                    if (!fold_earlier()) break;
+                    publish_piece(2 * seg + ((split1 && c == g1.mid) ? 1 : 0), ld2);
+                    if (c == g1.a0 && !fold_earlier()) break;
                 } else {
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&sm.ops_empty[ob]);
@@ -892,19 +955,21 @@ SegPlan make_plan(const SeqParams& p, int DVT, int P) {
     SegPlan s;
     s.DVT = DVT;
     s.P = P;
-    s.st_bytes = align256((size_t)(P - 1) * units * p.dk * DVT * 4);
-    s.ld_bytes = align256((size_t)(P - 1) * units * p.dk * 4);
-    s.flag_bytes = align256((size_t)P * units * 4);
+    // two piece slots per segment
+    s.st_bytes = align256((size_t)2 * P * units * p.dk * DVT * 4);
+    s.ld_bytes = align256((size_t)2 * P * units * p.dk * 4);
+    s.flag_bytes = align256((size_t)2 * P * units * 4);
     s.total = P > 1 ? s.st_bytes + s.ld_bytes + s.flag_bytes : 0;
     return s;
 }
 
 // Slice width and segment count.  Per CTA, a chunk costs about 1 time unit
 // with 64 d_v columns and 1.6 with 128 (the gate work is shared by the
-// columns), and a segmented CTA spends about 0.6 more per chunk on its
-// state-only pass.  Segments: as many as fill the SMs with one CTA each, none
-// shorter than kMinSegChunks chunks.  Take the cheaper of the two widths
-// (128 only exists for d_k = 64, d_v = 128); `allow_seg` false forces P = 1.
+// columns), and a segmented CTA spends about 0.6 more per chunk on its share
+// of the state-only work.  Segments: as many as fill the SMs with one CTA
+// each, none shorter than kMinSegChunks chunks, and no state-only range cut
+// twice.  Take the cheaper of the two widths (128 only exists for d_k = 64,
+// d_v = 128); `allow_seg` false forces P = 1.
 SegPlan choose_plan(const SeqParams& p, bool allow_seg) {
     const int NC = (p.T + C - 1) / C;
     const int nsm = sm_count();
@@ -917,6 +982,8 @@ SegPlan choose_plan(const SeqParams& p, bool allow_seg) {
         long long P = 1;
         if (allow_seg && units < nsm) P = nsm / units;
         if (P > NC / kMinSegChunks) P = NC / kMinSegChunks;
+        if (P > kMaxSeg) P = kMaxSeg;
+        while (P > 1 && !p1_ranges_ok(NC, (int)P)) --P;
         if (P < 1) P = 1;
         const long long waves = (units * P + nsm - 1) / nsm;
         const double per_chunk = (DVT == 128 ? 1.6 : 1.0) * (P > 1 ? 1.6 : 1.0);

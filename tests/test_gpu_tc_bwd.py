@@ -85,6 +85,16 @@ def test_tc_backward_segmented_wide_decay(cuda_ok):
     check(x, None, gpu_bwd(x), "segmented, one wide chunk")
 
 
+def test_tc_backward_segmented_no_decay(cuda_ok):
+    """R-only passes over a later half with tau = 0 (alpha = 1: plain sums of
+    q dO^T over whole segments) and g = 0 on no channel (dg needs g > 0)."""
+    x = draw_sequence(1, 2, 64 * 12 + 7, 64, 128, torch.bfloat16, seed=59, s0_std=0.1,
+                      with_dO=True)
+    x["tau"][:, :, 64 * 6:] = 0
+    dST = 0.1 * torch.randn(1, 2, 64, 128, generator=torch.Generator().manual_seed(59))
+    check(x, dST, gpu_bwd(x, dST), "segmented, no decay in the later half")
+
+
 @pytest.mark.parametrize("scale", [3.0, 40.0])
 def test_tc_backward_wide_decay(cuda_ok, scale):
     """Heads whose chunk decay span exceeds one reference are re-run exactly."""

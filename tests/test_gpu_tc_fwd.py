@@ -163,6 +163,26 @@ def test_tc_segmented_wide_decay(cuda_ok, scale):
     assert_close(ST, S_ref, TOL, "S_T")
 
 
+@pytest.mark.parametrize("dk,dv", [(64, 128), (128, 64)])
+def test_tc_segmented_special_gates(cuda_ok, dk, dv):
+    """State-only passes that sum outer products with no decay at all (tau = 0:
+    alpha = alpha_hat = 1) over half of the sequence, and channels with g = 0
+    (alpha = 1; alpha_hat = 0 where tau > 0, 1 where tau = 0)."""
+    x = draw_sequence(1, 2, 64 * 12 + 7, dk, dv, torch.bfloat16, seed=53 + dk, s0_std=0.1)
+    x["tau"][:, :, :64 * 6] = 0
+    x["g"][:, :, :, :8] = 0
+    assert segments_used(x)
+    o, ST, saved = run_tc(x, want_saved=True)
+    o_ref, S_ref = oracle.fwd(*(x[n] for n in SEQ), x["S0"])
+    assert_close(o, o_ref, TOL, "o")
+    assert_close(ST, S_ref, TOL, "S_T")
+    nc = (64 * 12 + 7 + 63) // 64
+    sv = saved.view(1, 2, nc, dk, dv)
+    for c in (3, 6, 9):
+        ref = oracle.fwd(*(x[n][:, :, :64 * c] for n in SEQ), x["S0"])[1]
+        assert_close(sv[:, :, c], ref, TOL, f"saved state {c}")
+
+
 @pytest.mark.parametrize("B,H,T", [(1, 40, 64 * 12 + 9), (4, 25, 130)])
 def test_tc_forward_wide_slices(cuda_ok, B, H, T):
     """Head counts for which one CTA takes all 128 value columns of a head:
