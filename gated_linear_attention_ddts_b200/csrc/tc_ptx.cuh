@@ -1,7 +1,7 @@
 // tc_ptx.cuh -- thin inline-PTX wrappers for the sm_100a features the chunked
 // kernels use: mbarriers (with bounded waits), TMEM allocation, tcgen05.mma
 // (kind::f16, bf16 operands, f32 accumulation in TMEM), tcgen05.commit /
-// tcgen05.ld, TMA tensor loads, cluster barriers and distributed shared memory.
+// tcgen05.ld, TMA tensor loads and stores, bulk copies and L2 prefetches.
 //
 // Operand layouts in shared memory are the "no swizzle" canonical UMMA layouts
 // built from 8x8 core matrices (8 rows of 16 bytes, 128 contiguous bytes):
@@ -31,12 +31,6 @@ __device__ __forceinline__ void fence_mbar_init() {
 
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
-// arrive on a barrier of another CTA of the cluster (address from mapa)
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar_addr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];"
-                 ::"r"(cluster_bar_addr) : "memory");
 }
 
 __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
@@ -223,16 +217,6 @@ __device__ __forceinline__ void tmem_ld_wait() {
 }
 
 // ----------------------------------------------------------------------- TMA
-// 2-D tiled tensor load (no multicast) into shared memory, completion counted
-// on a CTA-local mbarrier.  c0 is the innermost coordinate (elements).
-__device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, uint64_t* bar, int c0,
-                                            int c1) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4}], [%2];"
-        ::"r"(smem_u32(dst)), "l"(tmap), "r"(smem_u32(bar)), "r"(c0), "r"(c1) : "memory");
-}
-
 // 3-D tiled tensor load (no multicast): coordinates innermost first.
 __device__ __forceinline__ void tma_load_3d(void* dst, const void* tmap, uint64_t* bar, int c0,
                                             int c1, int c2) {
@@ -300,37 +284,12 @@ __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
     return v;
 }
 
-// --------------------------------------------------------------- cluster / DSMEM
-__device__ __forceinline__ uint32_t cluster_rank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-__device__ __forceinline__ void cluster_sync() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n"
-                 "barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-// shared::cluster address of `p` (a shared::cta pointer of this CTA) in CTA `rank`
-__device__ __forceinline__ uint32_t map_to_rank(const void* p, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
-    return r;
-}
 // Bulk copy global -> shared (this CTA), completion counted as transaction
 // bytes on `bar`.  Both addresses 16-byte aligned, bytes a multiple of 16.
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
     asm volatile(
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
         ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
-}
-// Bulk copy shared::cta (this CTA) -> shared::cluster (another CTA), completion
-// counted as transaction bytes on the destination CTA's mbarrier.
-__device__ __forceinline__ void bulk_copy_to_rank(uint32_t dst_cluster_addr, const void* src,
-                                                  uint32_t bytes, uint32_t bar_cluster_addr) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-        ::"r"(dst_cluster_addr), "r"(smem_u32(src)), "r"(bytes), "r"(bar_cluster_addr)
-        : "memory");
 }
 
 }  // namespace tc
