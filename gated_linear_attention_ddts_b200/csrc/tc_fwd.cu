@@ -388,7 +388,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             // log2(alpha_hat) of my tokens is kept from the scan for the operand pass
             // when registers allow (d_k = 64); otherwise that pass re-reads g and tau
             constexpr bool kKeepLah = SEGT <= 2;
-            float b[SEGT][8], bf[8], bl[8], lah2[kKeepLah ? SEGT : 1][8];
+            float b[SEGT][8], bf[8], bl[8];
+            [[maybe_unused]] float lah2[kKeepLah ? SEGT : 1][8];
             // window-relative inclusive running sum of log(alpha) over my tokens, and
             // b at the first / last valid token of my window (W in {64, 16})
             auto scan = [&](int W) {
