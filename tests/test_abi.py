@@ -73,6 +73,36 @@ def test_fwd_validation(lib, kw, status):
     assert lib.rdm_ddts_fwd(ctypes.byref(a), None) == status
 
 
+def _bwd_args(**kw):
+    from gated_linear_attention_ddts_b200._binding import BwdArgs
+    fake = 1 << 20
+    base = dict(B=1, H=1, T=8, dk=64, dv=64, chunk=0, dtype=1, impl=0, q=fake, k=fake, v=fake,
+                g=fake, tau=fake, beta=fake, S0=None, grad_o=fake, grad_ST=None,
+                saved_states=None, grad_q=fake, grad_k=fake, grad_v=fake, grad_g=fake,
+                grad_tau=fake, grad_beta=fake, grad_S0=None, workspace=None, workspace_bytes=0,
+                gate_inputs=0)
+    base.update(kw)
+    return BwdArgs(**base)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(B=0), 1), (dict(T=-3), 1), (dict(dk=48), 2), (dict(dv=256), 2), (dict(dtype=5), 1),
+    (dict(impl=9), 1), (dict(gate_inputs=2), 1), (dict(grad_o=None), 1), (dict(q=None), 1),
+    (dict(grad_q=(1 << 20) + 8), 1), (dict(grad_beta=None), 1), (dict(S0=(1 << 20) + 4), 1),
+    (dict(saved_states=(1 << 20) + 4), 1), (dict(workspace=(1 << 20) + 2), 1),
+])
+def test_bwd_validation(lib, kw, status):
+    """Host-side checks of the backward reject before touching the device."""
+    a = _bwd_args(**kw)
+    assert lib.rdm_ddts_bwd(ctypes.byref(a), None) == status
+
+
+def test_workspace_size_of_invalid_sizes(lib):
+    size_max = ctypes.c_size_t(-1).value
+    assert lib.rdm_ddts_fwd_workspace_size(ctypes.byref(_fwd_args(B=0))) == size_max
+    assert lib.rdm_ddts_bwd_workspace_size(ctypes.byref(_bwd_args(dk=-1))) == size_max
+
+
 def test_decode_validation(lib):
     fake = 1 << 20
     args = [fake] * 6 + [fake, fake]
