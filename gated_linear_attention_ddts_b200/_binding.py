@@ -54,7 +54,7 @@ _lib = None
 
 EXPORTS = ["rdm_ddts_fwd", "rdm_ddts_fwd_workspace_size", "rdm_ddts_saved_states_size", "rdm_ddts_bwd",
            "rdm_ddts_bwd_workspace_size", "rdm_ddts_bwd_noalloc", "rdm_ddts_decode_step", "rdm_ddts_sync_status",
-           "rdm_status_string", "rdm_ddts_version"]
+           "rdm_status_string", "rdm_ddts_set_test_hooks", "rdm_ddts_version"]
 
 
 def load():
@@ -83,6 +83,8 @@ def load():
         lib.rdm_ddts_sync_status.restype = _I
         lib.rdm_status_string.argtypes = [_I]
         lib.rdm_status_string.restype = ctypes.c_char_p
+        lib.rdm_ddts_set_test_hooks.argtypes = [ctypes.c_longlong, _I]
+        lib.rdm_ddts_set_test_hooks.restype = _I
         lib.rdm_ddts_version.argtypes = []
         lib.rdm_ddts_version.restype = _I
         _lib = lib
@@ -255,6 +257,13 @@ def rdm_ddts_sync_status(stream=None) -> int:
 
 def rdm_status_string(status: int) -> str:
     return status_string(status)
+
+
+def rdm_ddts_set_test_hooks(wait_limit_cycles: int = 0, withhold_segment_flags: int = 0) -> None:
+    """Test hooks of the bounded on-device waits (see include/rdm_ddts.h);
+    (0, 0) restores the defaults."""
+    _check(load().rdm_ddts_set_test_hooks(int(wait_limit_cycles), int(withhold_segment_flags)),
+           "rdm_ddts_set_test_hooks")
 
 
 def rdm_ddts_version() -> int:

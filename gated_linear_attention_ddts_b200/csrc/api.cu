@@ -4,6 +4,8 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "../../include/rdm_ddts.h"
 #include "launch.h"
 #include "rdm_common.cuh"
@@ -28,6 +30,16 @@ unsigned* status_word() {
         g_status_ptr[dev] = static_cast<unsigned*>(ptr);
     }
     return g_status_ptr[dev];
+}
+
+// Test hooks (rdm_ddts_set_test_hooks): a shorter bound for on-device waits and
+// segment flags that are never published; 0 = off.
+std::atomic<long long> g_hook_wait_limit{0};
+std::atomic<int> g_hook_withhold{0};
+
+long long wait_limit() {
+    const long long w = g_hook_wait_limit.load(std::memory_order_relaxed);
+    return w > 0 ? w : kDefaultWaitLimit;
 }
 
 bool dim_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
@@ -87,6 +99,8 @@ SeqParams fwd_params(const rdm_fwd_args* a) {
     p.S0 = a->S0; p.o = a->o; p.ST = a->ST; p.saved = a->saved_states;
     p.ws = a->workspace; p.ws_bytes = a->workspace ? a->workspace_bytes : 0;
     p.preact = a->gate_inputs == RDM_GATES_PREACT;
+    p.wait_limit = wait_limit();
+    p.withhold_flags = g_hook_withhold.load(std::memory_order_relaxed);
     return p;
 }
 
@@ -102,6 +116,8 @@ BwdParams bwd_params(const rdm_bwd_args* a) {
     p.dtau = a->grad_tau; p.dbeta = a->grad_beta; p.dS0 = a->grad_S0;
     p.ws = a->workspace; p.ws_bytes = a->workspace_bytes;
     p.preact = a->gate_inputs == RDM_GATES_PREACT;
+    p.wait_limit = wait_limit();
+    p.withhold_flags = g_hook_withhold.load(std::memory_order_relaxed);
     return p;
 }
 
@@ -234,6 +250,14 @@ const char* rdm_status_string(rdm_status s) {
     return "unknown status";
 }
 
-int rdm_ddts_version(void) { return 300; }
+rdm_status rdm_ddts_set_test_hooks(long long wait_limit_cycles, int withhold_segment_flags) {
+    if (wait_limit_cycles < 0 || (withhold_segment_flags != 0 && withhold_segment_flags != 1))
+        return RDM_ERR_INVALID_ARG;
+    g_hook_wait_limit.store(wait_limit_cycles, std::memory_order_relaxed);
+    g_hook_withhold.store(withhold_segment_flags, std::memory_order_relaxed);
+    return RDM_OK;
+}
+
+int rdm_ddts_version(void) { return 400; }
 
 }  // extern "C"

@@ -10,8 +10,11 @@
 // synchronise the whole device -- can still run the backward.
 //
 // The array is kNoAllocScratchBytes (16 MiB) per device and lives as long as
-// the library is loaded.  Its device address is looked up once per device, on
-// the first call made with that device current.
+// the library is loaded.  CUDA loads the library's module on a device lazily,
+// so the first call there allocates the array and may synchronise; callers
+// make one call at start-up.  The device address is looked up on every call
+// (cheap once the module is loaded): nothing cached can go stale across a
+// cudaDeviceReset, and no host state is shared between threads.
 #include <string.h>
 
 #include "../../include/rdm_ddts.h"
@@ -21,23 +24,16 @@ namespace rdm {
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = 16u << 20;
-constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-void* g_scratch_addr[kMaxDevices];  // device address of g_noalloc_scratch, per device
-
 // Host code must not hand the symbol itself to a kernel: on the host it names a
-// shadow variable, not device memory.  Look up the real address per device.
+// shadow variable, not device memory.  Look up the real address on the current
+// device.
 rdm_status scratch_for_current_device(void** out) {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return RDM_ERR_CUDA;
-    if (!g_scratch_addr[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return RDM_ERR_CUDA;
-        g_scratch_addr[dev] = p;
-    }
-    *out = g_scratch_addr[dev];
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return RDM_ERR_CUDA;
+    *out = p;
     return RDM_OK;
 }
 

@@ -6,6 +6,10 @@
 
 namespace rdm {
 
+// Default bound of every on-device wait (mbarrier phases, role barriers, flags
+// set by other CTAs): about one second of SM clock cycles.
+constexpr long long kDefaultWaitLimit = 2000000000LL;
+
 struct SeqParams {
     int B, H, T, dk, dv, chunk;
     int bf16;    // element type of sequence tensors: 1 = bf16, 0 = float32
@@ -18,6 +22,8 @@ struct SeqParams {
     void* ws;            // scratch for sequence segments, or null
     size_t ws_bytes;
     unsigned* err;       // device status word
+    long long wait_limit;  // SM clock cycles a bounded wait may take before it gives up
+    int withhold_flags;    // test hook: segment CTAs never publish their flags
 };
 
 struct BwdParams {
@@ -34,6 +40,8 @@ struct BwdParams {
     void* ws;            // scratch
     size_t ws_bytes;
     unsigned* err;
+    long long wait_limit;  // as SeqParams
+    int withhold_flags;
 };
 
 struct DecodeParams {

@@ -58,8 +58,8 @@ constexpr int DK = 64;
 constexpr int kGateWarps = 8;  // one 8-channel group each
 constexpr int kThreads = 32 * (4 + kGateWarps + 2);
 constexpr int kEpiWarp0 = 0, kGateWarp0 = 4, kProdWarp = 4 + kGateWarps, kMmaWarp = 5 + kGateWarps;
-constexpr int kBarEpi = 3;   // the four epilogue warps
-constexpr int kBarGate = 4;  // the gate warps
+constexpr int kBarEpi = 3;   // named barrier of the four epilogue warps
+constexpr int kBarGate = 4;  // named barrier of the gate warps
 constexpr int kStg = 68;
 // row stride (floats) of the chunk-start state copied into shared memory: a
 // 16-byte skew per row keeps the S_hat conversion free of bank conflicts
@@ -108,6 +108,7 @@ struct alignas(1024) BwdSmem {
         tm1_free, g2_done, tm2_free, post_ready, post_done, p1_done;
     uint32_t tmem_base;
     int fail;
+    int epi_fail;  // the epilogue's own exit decision (written before a role barrier)
 };
 
 // Segment exchange area (global): per (segment > 0, head) R_loc [DK][DV] and
@@ -145,6 +146,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
     BwdSmem<DV>& sm = *reinterpret_cast<BwdSmem<DV>*>(
         smem_dyn + ((1024u - (smem_u32(smem_dyn) & 1023u)) & 1023u));
     const BwdParams& p = A.p;
+    const long long WL = p.wait_limit > 0 ? p.wait_limit : kDefaultWaitLimit;  // bound of every wait
     const BwdSeg& sg = A.seg;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int BH = p.B * p.H;
@@ -178,6 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
         mbar_init(&sm.post_ready, 4);
         mbar_init(&sm.post_done, kGateWarps);
         mbar_init(&sm.p1_done, kGateWarps);
+        sm.epi_fail = 0;
         sm.fail = 0;
         fence_mbar_init();
     }
@@ -206,7 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             for (int li = 0; li < nL; ++li) {
                 const int c = pass_chunk(li);
                 const bool p2 = pass_p2(li);
-                if (li > 0 && !mbar_wait(&sm.raw_empty, (li - 1) & 1, fail, kWaitLimit)) break;
+                if (li > 0 && !mbar_wait(&sm.raw_empty, (li - 1) & 1, fail, WL)) break;
                 // the R-only pass reads q, g, tau and dO
                 mbar_expect_tx(&sm.raw_full, p2 ? K::RAW : (3 + VB) * kBox);
                 tma_load_3d(sm.raw + 0 * kBox, &A.mq, &sm.raw_full, 0, c * C, bh);
@@ -270,11 +273,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             for (int li = 0; li < nL; ++li) {
                 const bool p2 = pass_p2(li);
                 const int i2 = n2;  // index among full passes
-                if (!mbar_wait(&sm.ops_full, li & 1, fail, kWaitLimit)) break;
+                if (!mbar_wait(&sm.ops_full, li & 1, fail, WL)) break;
                 // group-1 accumulators released by the epilogue: after the R-only
                 // pass, and after each full pass (tm1_free completes once for each)
                 const int ntf = i2 + (has_p1 ? 1 : 0);
-                if (p2 && ntf > 0 && !mbar_wait(&sm.tm1_free, (ntf - 1) & 1, fail, kWaitLimit)) break;
+                if (p2 && ntf > 0 && !mbar_wait(&sm.tm1_free, (ntf - 1) & 1, fail, WL)) break;
                 tc_fence_after();
                 if (!p2) {
                     // R-only pass: R_loc += Qt^T dO over all its chunks
@@ -310,9 +313,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 }
                 mma_commit(&sm.g1_done);
                 ++n1;
-                if (!mbar_wait(&sm.g2_ready, i2 & 1, fail, kWaitLimit)) break;
-                if (!mbar_wait(&sm.shat_full, i2 & 1, fail, kWaitLimit)) break;
-                if (i2 > 0 && !mbar_wait(&sm.tm2_free, (i2 - 1) & 1, fail, kWaitLimit)) break;
+                if (!mbar_wait(&sm.g2_ready, i2 & 1, fail, WL)) break;
+                if (!mbar_wait(&sm.shat_full, i2 & 1, fail, WL)) break;
+                if (i2 > 0 && !mbar_wait(&sm.tm2_free, (i2 - 1) & 1, fail, WL)) break;
                 tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < C / 16; ++ks)
@@ -374,7 +377,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
         for (int li = 0; li < nL; ++li) {
             const int c = pass_chunk(li);
             const bool p2 = pass_p2(li);
-            if (!mbar_wait(&sm.raw_full, li & 1, fail, kWaitLimit)) break;
+            if (!mbar_wait_own(&sm.raw_full, li & 1, fail, WL)) break;
             const int nval = min(C, T - c * C);
             // ---- pre: running log-decay, reference, operands
             float b[SEGT][8], mL[8], blL[8];
@@ -423,10 +426,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             // pass, the epilogue done with the constants (tm1_free, once after the
             // R-only pass and once per full pass; it consumes em / cf / gm in its
             // first stage)
-            if (li > 0 && !mbar_wait(&sm.ops_empty, (li - 1) & 1, fail, kWaitLimit)) break;
+            if (li > 0 && !mbar_wait_own(&sm.ops_empty, (li - 1) & 1, fail, WL)) break;
             if (p2) {
                 const int ntf = i2 + (has_p1 ? 1 : 0);
-                if (ntf > 0 && !mbar_wait(&sm.tm1_free, (ntf - 1) & 1, fail, kWaitLimit)) break;
+                if (ntf > 0 && !mbar_wait_own(&sm.tm1_free, (ntf - 1) & 1, fail, WL)) break;
             }
             if (!p2) {
                 // R-only pass: Qt = q exp(G_t) relative to the segment start (gh2 the
@@ -461,7 +464,6 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                     mbar_arrive(&sm.raw_empty);
                     if (p1last) mbar_arrive(&sm.p1_done);
                 }
-                if (*fail) break;
                 continue;
             }
 #pragma unroll
@@ -520,7 +522,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             if (lane == 0) mbar_arrive(&sm.ops_full);
             // S_hat = diag(e^m) S_prev for this warp's rows (channels), while the
             // first MMA group runs
-            if (!mbar_wait(&sm.sp_full, i2 & 1, fail, kWaitLimit)) break;
+            if (!mbar_wait_own(&sm.sp_full, i2 & 1, fail, WL)) break;
 #pragma unroll
             for (int gi = 0; gi < GW; ++gi) {
                 const int i = (gw * GW + gi) * 8 + (lane >> 2);
@@ -542,7 +544,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             if (lane == 0) mbar_arrive(&sm.shat_full);
 
             // ---- post: final gate gradients once dQ, dK of this chunk are staged
-            if (!mbar_wait(&sm.post_ready, i2 & 1, fail, kWaitLimit)) break;
+            if (!mbar_wait_own(&sm.post_ready, i2 & 1, fail, WL)) break;
             uint8_t* gst = sm.qt;  // 4 x 8 KB over qt | kt | qtl | ktl
             float dG[SEGT][8], dkh[SEGT][8];
 #pragma unroll
@@ -654,7 +656,6 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 mbar_arrive(&sm.raw_empty);
             }
             ++i2;
-            if (*fail) break;
         }
     } else {
         // ------------------------------------------------------------ epilogue
@@ -680,13 +681,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 const long long t0 = clock64();
                 for (int s2 = P - 1; s2 > seg && !*fail; --s2)
                     while (ld_acquire_gpu(&sg.flag[s2 * BH + bh]) != sg.tag)
-                        if (clock64() - t0 > kWaitLimit) {
+                        if (clock64() - t0 > WL) {
                             *fail = 1;
+                            sm.epi_fail = 1;
                             break;
                         }
             }
             named_bar(kBarEpi, 128);
-            if (*fail) return false;
+            if (sm.epi_fail) return false;  // written by thread 0 before the barrier
             load_dst();
             for (int s2 = P - 1; s2 > seg; --s2) {
                 const size_t u = (size_t)s2 * BH + bh;
@@ -712,7 +714,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             return true;
         };
         // publish this segment's map (R_loc in R, log2 D in ld2)
-        auto publish_segment = [&](float ld2) {
+        auto publish_segment = [&](float ld2) -> bool {
             const size_t u = (size_t)seg * BH + bh;
             float4* dst = reinterpret_cast<float4*>(sg.st + (u * DK + r) * DV + hf * HV);
 #pragma unroll
@@ -721,7 +723,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             if (hf == 0) sg.ld[u * DK + r] = ld2;
             __threadfence();
             named_bar(kBarEpi, 128);
-            if (threadIdx.x == 0) st_release_gpu(&sg.flag[u], sg.tag);
+            if (threadIdx.x == 0 && !p.withhold_flags) st_release_gpu(&sg.flag[u], sg.tag);
+            return true;
         };
         bool ok_run = true;
         if (P == 1) {
@@ -736,8 +739,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
         if (ok_run && has_p1) {
             // R-only pass: R_loc is the accumulated group-1 sum once its last
             // chunk's products are done; log2 D comes from the gate warps
-            ok_run = mbar_wait(&sm.p1_done, 0, fail, kWaitLimit) &&
-                     mbar_wait(&sm.g1_done, 0, fail, kWaitLimit);
+            ok_run = mbar_wait_own(&sm.p1_done, 0, fail, WL) &&
+                     mbar_wait_own(&sm.g1_done, 0, fail, WL);
             if (ok_run) {
                 tc_fence_after();
                 const float ld2 = sm.gm[r];
@@ -749,17 +752,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm.tm1_free);
-                publish_segment(ld2);
-                ok_run = fold_later();
+                ok_run = publish_segment(ld2) && fold_later();
             }
         }
         for (int li = has_p1 ? nseg : 0; ok_run && li < nL; ++li) {
             const int c = pass_chunk(li);
-            if (!mbar_wait(&sm.ops_full, li & 1, fail, kWaitLimit)) break;
-            if (!mbar_wait(&sm.g1_done, (i2 + (has_p1 ? 1 : 0)) & 1, fail, kWaitLimit)) break;
+            if (!mbar_wait_own(&sm.ops_full, li & 1, fail, WL)) break;
+            if (!mbar_wait_own(&sm.g1_done, (i2 + (has_p1 ? 1 : 0)) & 1, fail, WL)) break;
             tc_fence_after();
             // the gate warps have read S_prev out of the union (and staged S_hat)
-            if (!mbar_wait(&sm.shat_full, i2 & 1, fail, kWaitLimit)) break;
+            if (!mbar_wait_own(&sm.shat_full, i2 & 1, fail, WL)) break;
             // A and B -> causal mask -> bf16 operands (row t = r, columns s = 32 hf + e)
 #pragma unroll
             for (int which = 0; which < 2; ++which) {
@@ -827,12 +829,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 mbar_arrive(&sm.g2_ready);
                 mbar_arrive(&sm.tm1_free);
             }
-            if (!mbar_wait(&sm.g2_done, i2 & 1, fail, kWaitLimit)) break;
+            if (!mbar_wait_own(&sm.g2_done, i2 & 1, fail, WL)) break;
             tc_fence_after();
             // dV -> dv = beta dvhat, dbeta = v dvhat (row s = r), staged in the union
             // (its A / B / R_hat operands are consumed; the previous chunk's gate
             // stage has read its dQ / dK staging) and written by TMA stores
-            if (i2 > 0 && !mbar_wait(&sm.post_done, (i2 - 1) & 1, fail, kWaitLimit)) break;
+            if (i2 > 0 && !mbar_wait_own(&sm.post_done, (i2 - 1) & 1, fail, WL)) break;
             {
 #pragma unroll
                 for (int qd = 0; qd < HV / 32; ++qd) {
@@ -1022,6 +1024,9 @@ cudaError_t launch_tc_bwd(const BwdParams& p, cudaStream_t s) {
         f.ST = nullptr;
         f.saved = reinterpret_cast<float*>(ws);
         f.err = p.err;
+        f.preact = p.preact;
+        f.wait_limit = p.wait_limit;
+        f.withhold_flags = p.withhold_flags;
         if ((e = launch_tc_fwd(f, s)) != cudaSuccess) return e;
         saved = f.saved;
     }

@@ -60,12 +60,25 @@ __device__ __forceinline__ uint4 pack8(const float* f) {
     return u;
 }
 
+// Element-wise product of two bf16 pairs, rounded once to bf16 (the product of
+// two bf16 values is exact in fp32, so this equals widening both, multiplying
+// in fp32 and rounding the result: one instruction instead of seven).
+__device__ __forceinline__ uint32_t bmul2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint4 bmul8(uint4 a, uint4 b) {
+    return make_uint4(bmul2(a.x, b.x), bmul2(a.y, b.y), bmul2(a.z, b.z), bmul2(a.w, b.w));
+}
+
 __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
     const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity))
         if (clock64() - t0 > kWaitLimit) return false;
     return true;
 }
+
 
 
 }  // namespace tc

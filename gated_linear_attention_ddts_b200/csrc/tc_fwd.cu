@@ -60,8 +60,8 @@ constexpr int kGateWarps = 8;  // two per SM sub-partition
 constexpr int kThreads = 32 * (kEpiWarps + kGateWarps + 2);
 constexpr int kEpiWarp0 = 0, kGateWarp0 = kEpiWarps, kProdWarp = kEpiWarps + kGateWarps,
               kMmaWarp = kProdWarp + 1;
-constexpr int kBarGate = 3;        // all gate warps
-constexpr int kBarEpi = 4;         // all epilogue warps
+constexpr int kBarGate = 3;        // named barrier of the gate warps
+constexpr int kBarEpi = 4;         // named barrier of the epilogue warps
 constexpr int kMinSegChunks = 4;   // shortest segment worth a CTA of its own
 constexpr int kMaxSeg = 160;       // most segments per sequence
 constexpr int kAhead = 2;          // L2 prefetch distance of the producer, in passes
@@ -104,6 +104,7 @@ struct alignas(1024) FwdSmem {
     uint64_t raw_full[K::NS], raw_empty[K::NS], v_full, v_empty, ops_full[K::NB], ops_empty[K::NB];
     uint64_t mma1_done, as_free, abf_full, mmao_done[2], o_free[2], vh_full[K::NB];
     int need16[2], need1[2];
+    int epi_fail;  // the epilogue's own exit decision (written before a role barrier)
     uint8_t before[2 * kMaxSeg];  // state-only pieces that precede this CTA's segment
     uint32_t tmem_base;
     int fail;
@@ -183,12 +184,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
         smem_dyn + ((1024u - (smem_u32(smem_dyn) & 1023u)) & 1023u));
     const SeqParams& p = A.p;
     const SegArgs& sg = A.seg;
+    const long long WL = p.wait_limit > 0 ? p.wait_limit : kDefaultWaitLimit;  // bound of every wait
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int NJ = p.dv / DVT;
     const int units = p.B * p.H * NJ;
     const int unit = blockIdx.x % units, seg = blockIdx.x / units;
     const int bh = unit / NJ, j0 = (unit % NJ) * DVT;
     const int T = p.T, NC = (T + C - 1) / C;
+    const int NCS = (T + p.chunk - 1) / p.chunk;  // saved chunk-start states per sequence
     const int P = sg.P;
     const int c0 = seg_start(seg, NC, P), c1 = seg_start(seg + 1, NC, P);
     const int nseg = c1 - c0;
@@ -224,6 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
         mbar_init(&sm.o_free[0], kEpiWarps);
         mbar_init(&sm.o_free[1], kEpiWarps);
         for (int b = 0; b < NB; ++b) mbar_init(&sm.vh_full[b], kEpiWarps);
+        sm.epi_fail = 0;
         sm.need16[0] = sm.need16[1] = sm.need1[0] = sm.need1[1] = 0;
         sm.fail = 0;
         fence_mbar_init();
@@ -249,7 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             for (int li = 0; li < nL; ++li) {
                 const int st = li % NS, c = pass_chunk(li);
                 const bool p2 = pass_p2(li);
-                if (li >= NS && !mbar_wait(&sm.raw_empty[st], ((li / NS) - 1) & 1, fail, kWaitLimit))
+                if (li >= NS && !mbar_wait(&sm.raw_empty[st], ((li / NS) - 1) & 1, fail, WL))
                     break;
                 // the state-only pass does not read q
                 mbar_expect_tx(&sm.raw_full[st], K::RAWK - (p2 ? 0 : KB * kBox));
@@ -277,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                         tma_prefetch_3d(&A.mb, j0 + 64 * vb, ca * C, bh);
                     }
                 }
-                if (li >= 1 && !mbar_wait(&sm.v_empty, (li - 1) & 1, fail, kWaitLimit)) break;
+                if (li >= 1 && !mbar_wait(&sm.v_empty, (li - 1) & 1, fail, WL)) break;
                 mbar_expect_tx(&sm.v_full, K::RAWV);
                 for (int vb = 0; vb < VB; ++vb) {
                     tma_load_3d(sm.rawv + vb * kBox, &A.mv, &sm.v_full, j0 + 64 * vb, c * C, bh);
@@ -303,15 +307,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             int item = 0, n1 = 0, io = 0, nas = 0;
             while (true) {
                 const int ob = item % NB;
-                if (!mbar_wait(&sm.ops_full[ob], (item / NB) & 1, fail, kWaitLimit)) break;
+                if (!mbar_wait(&sm.ops_full[ob], (item / NB) & 1, fail, WL)) break;
                 const int last = sm.info[ob][kInfoLast];
                 const bool p2 = sm.info[ob][kInfoPhase] == 2;
                 const bool p1last = sm.info[ob][kInfoP1Last];
                 const bool fresh = p2 || piece_open(sm.info[ob][kInfoChunk]);
                 if constexpr (kVhEpi)
-                    if (!mbar_wait(&sm.vh_full[ob], (item / NB) & 1, fail, kWaitLimit)) break;
+                    if (!mbar_wait(&sm.vh_full[ob], (item / NB) & 1, fail, WL)) break;
                 if (fresh && item > 0) {
-                    if (!mbar_wait(&sm.as_free, nas & 1, fail, kWaitLimit)) break;
+                    if (!mbar_wait(&sm.as_free, nas & 1, fail, WL)) break;
                     ++nas;
                 }
                 tc_fence_after();
@@ -332,9 +336,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                     ++n1;
                 }
                 if (p2) {
-                    if (!mbar_wait(&sm.abf_full, io & 1, fail, kWaitLimit)) break;
+                    if (!mbar_wait(&sm.abf_full, io & 1, fail, WL)) break;
                     const int obuf = io & 1;
-                    if (io >= 2 && !mbar_wait(&sm.o_free[obuf], ((io >> 1) - 1) & 1, fail, kWaitLimit))
+                    if (io >= 2 && !mbar_wait(&sm.o_free[obuf], ((io >> 1) - 1) & 1, fail, WL))
                         break;
                     tc_fence_after();
                     const uint32_t a = smem_u32(sm.abf) >> 4, sh = smem_u32(sm.shat) >> 4;
@@ -373,6 +377,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
         const int cg = gw * GW + cgl;
         const int tb = seg_l * SEGT;  // first token of my segment
         const uint32_t full = 0xffffffffu;
+        const int W0 = p.chunk;  // window width asked for: 64, 32 or 16 tokens
         int item = 0;
         float gt2[8];  // state-only pass: log2 decay of the chunks after the current one
 #pragma unroll
@@ -382,7 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
         auto pass = [&](int li, auto kP2) -> bool {
             const int st = li % NS, c = pass_chunk(li);
             constexpr bool p2 = decltype(kP2)::value;
-            if (!mbar_wait(&sm.raw_full[st], (li / NS) & 1, fail, kWaitLimit)) return false;
+            if (!mbar_wait_own(&sm.raw_full[st], (li / NS) & 1, fail, WL)) return false;
             const uint8_t* raw = sm.raw[st];
             const int nval = min(C, T - c * C);
             // log2(alpha_hat) of my tokens is kept from the scan for the operand pass
@@ -408,8 +413,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                     }
                 }
                 if (W == 1) return;
-                const int WL = W / SEGT * GW;        // lanes per window
-                const int l0 = lane & ~(WL - 1);     // first lane of my window
+                const int WLN = W / SEGT * GW;       // lanes per window
+                const int l0 = lane & ~(WLN - 1);    // first lane of my window
                 const int tw0 = (l0 / GW) * SEGT;    // first token of my window
                 const int tl = min(tw0 + W, nval) - 1;  // last valid token of my window
                 const int lsrc = cgl + GW * (max(tl, tw0) / SEGT);
@@ -421,7 +426,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
 #pragma unroll
                     for (int d = GW; d < 32; d <<= 1) {
                         const float y = __shfl_up_sync(full, x, d);
-                        if ((lane & (WL - 1)) >= d) x += y;
+                        if ((lane & (WLN - 1)) >= d) x += y;
                     }
                     const float excl = x - tot;
                     float mine = 0.0f;
@@ -450,20 +455,28 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             auto write_vh = [&](int ob, int w0, int w1) {
                 if constexpr (kVhEpi) return;
                 if (!have_v) {
-                    have_v = mbar_wait(&sm.v_full, li & 1, fail, kWaitLimit);
+                    have_v = mbar_wait_own(&sm.v_full, li & 1, fail, WL);
                     if (!have_v) return;
                 }
 #pragma unroll
                 for (int it = 0; it < VIT; ++it) {
                     const int jg = gt / TPG, t = (gt % TPG) + TPG * it;
                     const bool in = t >= w0 && t < w1;
-                    float v8[8], b8[8], o8[8];
-                    unpack8(*reinterpret_cast<const uint4*>(sm.rawv + off_raw(t, jg)), v8);
-                    unpack8(*reinterpret_cast<const uint4*>(sm.rawv + VB * kBox + off_raw(t, jg)), b8);
-                    if constexpr (PRE) activate_beta8(b8);
+                    const uint4 v8 = *reinterpret_cast<const uint4*>(sm.rawv + off_raw(t, jg));
+                    const uint4 b8 = *reinterpret_cast<const uint4*>(sm.rawv + VB * kBox + off_raw(t, jg));
+                    uint4 o8 = make_uint4(0u, 0u, 0u, 0u);
+                    if constexpr (PRE) {
+                        float vf[8], bf8[8], of[8];
+                        unpack8(v8, vf);
+                        unpack8(b8, bf8);
+                        activate_beta8(bf8);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) o8[e] = in ? v8[e] * b8[e] : 0.0f;
-                    *reinterpret_cast<uint4*>(sm.vh[ob] + off_vh(t, jg * 8)) = pack8(o8);
+                        for (int e = 0; e < 8; ++e) of[e] = vf[e] * bf8[e];
+                        if (in) o8 = pack8(of);
+                    } else {
+                        if (in) o8 = bmul8(v8, b8);
+                    }
+                    *reinterpret_cast<uint4*>(sm.vh[ob] + off_vh(t, jg * 8)) = o8;
                 }
             };
             auto publish = [&](int ob, int w0, int w1) {
@@ -492,7 +505,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                 }
                 scan(C);
                 const int ob = item % NB;
-                if (item >= NB && !mbar_wait(&sm.ops_empty[ob], ((item / NB) - 1) & 1, fail, kWaitLimit))
+                if (item >= NB && !mbar_wait_own(&sm.ops_empty[ob], ((item / NB) - 1) & 1, fail, WL))
                     return false;
 #pragma unroll
                 for (int u = 0; u < SEGT; ++u) {
@@ -523,24 +536,30 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                     for (int e = 0; e < 8; ++e) sm.gm[ob][cg * 8 + e] = gt2[e];
                 }
                 write_vh(ob, 0, C);
+                if (!kVhEpi && !have_v) return false;
                 publish(ob, 0, C);
                 ++item;
             } else {
-                int W = C;
-                scan(C);
-                if (too_wide(&sm.need16[li & 1])) {
+                // window width: the chunk size asked for (64, 32 or 16 tokens),
+                // narrowed to 16 and then to single tokens while some window
+                // spans more log-decay than one reference holds
+                int W = W0;
+                scan(W);
+                bool wide = too_wide(&sm.need16[li & 1]);
+                if (wide && W > 16) {
                     W = 16;
                     scan(16);
-                    if (too_wide(&sm.need1[li & 1])) {
-                        W = 1;
-                        scan(1);
-                    }
+                    wide = too_wide(&sm.need1[li & 1]);
+                }
+                if (wide) {
+                    W = 1;
+                    scan(1);
                 }
                 if (W == C) {
                     // ---- one window = the whole chunk (rows past T hold zeros from the
                     // TMA fill, so every row can be computed unmasked)
                     const int ob = item % NB;
-                    if (item >= NB && !mbar_wait(&sm.ops_empty[ob], ((item / NB) - 1) & 1, fail, kWaitLimit))
+                    if (item >= NB && !mbar_wait_own(&sm.ops_empty[ob], ((item / NB) - 1) & 1, fail, WL))
                         return false;
                     float mL[8];
 #pragma unroll
@@ -581,6 +600,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                         }
                     }
                     write_vh(ob, 0, C);
+                    if (!kVhEpi && !have_v) return false;
                     publish(ob, 0, nval);
                     ++item;
                 } else {
@@ -589,7 +609,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                         const int w1 = min(w0 + W, nval);
                         const int ob = item % NB;
                         if (item >= NB &&
-                            !mbar_wait(&sm.ops_empty[ob], ((item / NB) - 1) & 1, fail, kWaitLimit)) {
+                            !mbar_wait_own(&sm.ops_empty[ob], ((item / NB) - 1) & 1, fail, WL)) {
                             ok_loop = false;
                             break;
                         }
@@ -622,6 +642,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                             *reinterpret_cast<uint4*>(sm.kt[ob] + off_qk(t, cg * 8)) = pack8(ok);
                         }
                         write_vh(ob, w0, w1);
+                        if (!kVhEpi && !have_v) {
+                            ok_loop = false;
+                            break;
+                        }
                         publish(ob, w0, w1);
                         ++item;
                     }
@@ -633,7 +657,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                 mbar_arrive(&sm.raw_empty[st]);
                 if constexpr (!kVhEpi) mbar_arrive(&sm.v_empty);
             }
-            return !*fail;
+            return true;
         };
         int li = 0;
         bool run = true;
@@ -669,6 +693,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             tmem_ld_wait();
         };
         float S[SC];
+        auto epi_sync = [&]() { named_bar(kBarEpi, 32 * kEpiWarps); };
         auto load_s0 = [&]() {
 #pragma unroll
             for (int j = 0; j < SC; ++j)
@@ -685,20 +710,21 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                 const int lo = (slot & 1) ? r.mid : r.a0, hi = (slot & 1) ? r.a1 : r.mid;
                 sm.before[slot] = lo < hi && hi <= c0;
             }
-            named_bar(kBarEpi, 32 * kEpiWarps);
+            epi_sync();
             if (threadIdx.x == 0) {
                 const long long t0 = clock64();
                 for (int slot = 0; slot < 2 * P && !*fail; ++slot) {
                     if (!sm.before[slot]) continue;
                     while (ld_acquire_gpu(&sg.flag[slot * units + unit]) != sg.epoch)
-                        if (clock64() - t0 > kWaitLimit) {
+                        if (clock64() - t0 > WL) {
                             *fail = 1;
+                            sm.epi_fail = 1;
                             break;
                         }
                 }
             }
-            named_bar(kBarEpi, 32 * kEpiWarps);
-            if (*fail) return false;
+            epi_sync();
+            if (sm.epi_fail) return false;  // written by thread 0 before the barrier
             load_s0();
             for (int slot = 0; slot < 2 * P; ++slot) {
                 if (!sm.before[slot]) continue;
@@ -717,7 +743,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             return true;
         };
         // publish the map of a state-only piece (S_loc in S, log2 D in ld2)
-        auto publish_piece = [&](int slot, float ld2) {
+        auto publish_piece = [&](int slot, float ld2) -> bool {
             const size_t u = (size_t)slot * units + unit;
             float4* dst = reinterpret_cast<float4*>(sg.st + (u * DK + iS) * DVT + sc0);
 #pragma unroll
@@ -725,15 +751,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                 dst[j4] = make_float4(S[4 * j4], S[4 * j4 + 1], S[4 * j4 + 2], S[4 * j4 + 3]);
             if (sc0 == 0) sg.ld[u * DK + iS] = ld2;
             __threadfence();
-            named_bar(kBarEpi, 32 * kEpiWarps);
-            if (threadIdx.x == 0) st_release_gpu(&sg.flag[u], sg.epoch);
+            epi_sync();
+            if (threadIdx.x == 0 && !p.withhold_flags) st_release_gpu(&sg.flag[u], sg.epoch);
+            return true;
         };
         // o rows [w0, w1) of chunk c from the O buffer of o-item `io`.  A whole
         // chunk goes out through the staging tile and one TMA store (rows past T
         // are clipped by the TMA unit); a window writes its rows directly.
         auto store_o = [&](int io, int c, int w0, int w1) -> bool {
             const int obuf = io & 1;
-            if (!mbar_wait(&sm.mmao_done[obuf], (io >> 1) & 1, fail, kWaitLimit)) return false;
+            if (!mbar_wait_own(&sm.mmao_done[obuf], (io >> 1) & 1, fail, WL)) return false;
             tc_fence_after();
             float v[OC];
             ld_cols(K::COL_O + obuf * DVT, v, false);
@@ -744,12 +771,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             if (whole) {
                 // the previous store has read the staging tile
                 if (threadIdx.x == 0) bulk_wait_read_all();
-                named_bar(kBarEpi, 32 * kEpiWarps);
+                epi_sync();
 #pragma unroll
                 for (int s8 = 0; s8 < OC / 8; ++s8)
                     *reinterpret_cast<uint4*>(sm.ostage + off_raw(tA, (oc0 >> 3) + s8)) = pack8(v + 8 * s8);
                 fence_proxy_async_smem();
-                named_bar(kBarEpi, 32 * kEpiWarps);
+                epi_sync();
                 if (threadIdx.x == 0) {
 #pragma unroll
                     for (int vb = 0; vb < VB; ++vb)
@@ -774,7 +801,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
         int item = 0, io = 0, nm1 = 0, pc = 0, pw0 = 0, pw1 = 0;
         while (ok_run) {
             const int ob = item % NB;
-            if (!mbar_wait(&sm.ops_full[ob], (item / NB) & 1, fail, kWaitLimit)) break;
+            if (!mbar_wait_own(&sm.ops_full[ob], (item / NB) & 1, fail, WL)) break;
             const int c = sm.info[ob][kInfoChunk], w0 = sm.info[ob][kInfoW0], w1 = sm.info[ob][kInfoW1];
             const int last = sm.info[ob][kInfoLast], p1last = sm.info[ob][kInfoP1Last];
             const bool p2 = sm.info[ob][kInfoPhase] == 2;
@@ -783,21 +810,29 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                 // free once the tensor core has finished the item NB back
                 const int li = sm.info[ob][kInfoPass];
                 const int nval = min(C, T - c * C);
-                if (!mbar_wait(&sm.v_full, li & 1, fail, kWaitLimit)) break;
-                if (item >= NB && !mbar_wait(&sm.ops_empty[ob], ((item / NB) - 1) & 1, fail, kWaitLimit))
+                if (!mbar_wait_own(&sm.v_full, li & 1, fail, WL)) break;
+                if (item >= NB && !mbar_wait_own(&sm.ops_empty[ob], ((item / NB) - 1) & 1, fail, WL))
                     break;
                 const int et = threadIdx.x - 32 * kEpiWarp0;
 #pragma unroll
                 for (int it = 0; it < (C * DVT / 8) / (32 * kEpiWarps); ++it) {
                     const int idx = et + 32 * kEpiWarps * it, jg = idx / C, t = idx % C;
                     const bool in = t >= w0 && t < w1;
-                    float v8[8], b8[8], o8[8];
-                    unpack8(*reinterpret_cast<const uint4*>(sm.rawv + off_raw(t, jg)), v8);
-                    unpack8(*reinterpret_cast<const uint4*>(sm.rawv + VB * kBox + off_raw(t, jg)), b8);
-                    if constexpr (PRE) activate_beta8(b8);
+                    const uint4 v8 = *reinterpret_cast<const uint4*>(sm.rawv + off_raw(t, jg));
+                    const uint4 b8 = *reinterpret_cast<const uint4*>(sm.rawv + VB * kBox + off_raw(t, jg));
+                    uint4 o8 = make_uint4(0u, 0u, 0u, 0u);
+                    if constexpr (PRE) {
+                        float vf[8], bf8[8], of[8];
+                        unpack8(v8, vf);
+                        unpack8(b8, bf8);
+                        activate_beta8(bf8);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) o8[e] = in ? v8[e] * b8[e] : 0.0f;
-                    *reinterpret_cast<uint4*>(sm.vh[ob] + off_vh(t, jg * 8)) = pack8(o8);
+                        for (int e = 0; e < 8; ++e) of[e] = vf[e] * bf8[e];
+                        if (in) o8 = pack8(of);
+                    } else {
+                        if (in) o8 = bmul8(v8, b8);
+                    }
+                    *reinterpret_cast<uint4*>(sm.vh[ob] + off_vh(t, jg * 8)) = o8;
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
@@ -812,7 +847,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                 // CTA's last piece (chunk a0), the entry state of its segment
                 if (p1last) {
                     const float ld2 = sm.gm[ob][iS];
-                    if (!mbar_wait(&sm.mma1_done, nm1 & 1, fail, kWaitLimit)) break;
+                    if (!mbar_wait_own(&sm.mma1_done, nm1 & 1, fail, WL)) break;
                     ++nm1;
                     tc_fence_after();
                     ld_cols(K::COL_S, S, true);
@@ -822,7 +857,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                         mbar_arrive(&sm.as_free);
                         mbar_arrive(&sm.ops_empty[ob]);
                     }
-                    publish_piece(2 * seg + ((split1 && c == g1.mid) ? 1 : 0), ld2);
+                    if (!publish_piece(2 * seg + ((split1 && c == g1.mid) ? 1 : 0), ld2)) break;
                     if (c == g1.a0 && !fold_earlier()) break;
                 } else {
                     __syncwarp();
@@ -831,9 +866,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                 ++item;
                 continue;
             }
-            if (!mbar_wait(&sm.mma1_done, nm1 & 1, fail, kWaitLimit)) break;
+            if (!mbar_wait_own(&sm.mma1_done, nm1 & 1, fail, WL)) break;
             ++nm1;
             tc_fence_after();
+            // saved states: the state in force before every chunk of the size asked
+            // for, i.e. before window starts that are multiples of it
+            const bool save_here = p.saved != nullptr && (w0 % p.chunk) == 0;
+            const int cs = (c * C + w0) / p.chunk;
             {
                 // A -> causal mask -> bf16 operand (row t = tA, columns s = a0 + e)
                 {
@@ -859,9 +898,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                         *reinterpret_cast<uint4*>(sm.shat + off_shat<DK>(iS, sc0 + jg * 8)) = pack8(x);
                     }
                     if constexpr (!K::STAGE_SAVED) {
-                        if (p.saved && w0 == 0) {
+                        if (save_here) {
                             float4* dst = reinterpret_cast<float4*>(
-                                p.saved + (((size_t)bh * NC + c) * DK + iS) * p.dv + j0 + sc0);
+                                p.saved + (((size_t)bh * NCS + cs) * DK + iS) * p.dv + j0 + sc0);
 #pragma unroll
                             for (int j4 = 0; j4 < SC / 4; ++j4)
                                 dst[j4] = make_float4(S[4 * j4], S[4 * j4 + 1], S[4 * j4 + 2], S[4 * j4 + 3]);
@@ -873,9 +912,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                 if (lane == 0) mbar_arrive(&sm.abf_full);
                 if constexpr (K::STAGE_SAVED) {
                     // the chunk-start state (S still holds it until the update below)
-                    if (p.saved && w0 == 0) {
+                    if (save_here) {
                         if (threadIdx.x == 0) bulk_wait_read_all();  // previous store has read sstage
-                        named_bar(kBarEpi, 32 * kEpiWarps);
+                        epi_sync();
 #pragma unroll
                         for (int j4 = 0; j4 < SC / 4; ++j4) {
                             const int col = sc0 + 4 * j4;  // 32-column boxes, 16-byte chunks
@@ -885,12 +924,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                                 make_float4(S[4 * j4], S[4 * j4 + 1], S[4 * j4 + 2], S[4 * j4 + 3]);
                         }
                         fence_proxy_async_smem();
-                        named_bar(kBarEpi, 32 * kEpiWarps);
+                        epi_sync();
                         if (threadIdx.x == 0) {
 #pragma unroll
                             for (int bx = 0; bx < DVT / 32; ++bx)
                                 tma_store_2d(&A.msv, sm.sstage + bx * (DK * 128), j0 + 32 * bx,
-                                             (int)(((size_t)bh * NC + c) * DK));
+                                             (int)(((size_t)bh * NCS + cs) * DK));
                             bulk_commit();
                         }
                     }
@@ -1011,7 +1050,8 @@ cudaError_t launch_cfg(const SeqParams& p, SegPlan plan, cudaStream_t s) {
         !make_tmap_bf16_3d(&a.mo, p.o, p.dv, p.T, BH, 64, 64))
         return cudaErrorInvalidValue;
     if (Cfg<DK, DVT>::STAGE_SAVED && p.saved &&
-        !make_tmap_f32_2d(&a.msv, p.saved, p.dv, BH * (uint64_t)((p.T + C - 1) / C) * DK, 32, DK))
+        !make_tmap_f32_2d(&a.msv, p.saved, p.dv, BH * (uint64_t)((p.T + p.chunk - 1) / p.chunk) * DK,
+                          32, DK))
         return cudaErrorInvalidValue;
     const size_t smem = sizeof(FwdSmem<DK, DVT>) + 1024;
     auto kern = tc_fwd_kernel<DK, DVT, PRE>;
@@ -1050,7 +1090,8 @@ cudaError_t launch_plan(const SeqParams& p, const SegPlan& plan, cudaStream_t s)
 }  // namespace
 
 bool tc_fwd_supported(const SeqParams& p) {
-    return p.bf16 && p.chunk == C && p.T >= 1 && (p.dk == 64 || p.dk == 128) &&
+    return p.bf16 && (p.chunk == 16 || p.chunk == 32 || p.chunk == C) && p.T >= 1 &&
+           (p.dk == 64 || p.dk == 128) &&
            (p.dv == 64 || p.dv == 128);
 }
 

@@ -69,6 +69,26 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     }
 }
 
+// Bounded wait for the warps of a role that meet at named barriers (bar.sync).
+// It gives up only on its own clock and never looks at the shared failure flag:
+// the warps of one role wait for the same phases in the same order, and a
+// phase either completes for all of them or for none, so they all pass or all
+// run out together and no warp is left waiting at a role barrier that another
+// warp has skipped by leaving early.  On running out it raises *fail (for the
+// other roles and the status word) and returns false.
+__device__ __forceinline__ bool mbar_wait_own(uint64_t* bar, uint32_t parity, volatile int* fail,
+                                              long long limit) {
+    const long long t0 = clock64();
+    while (true) {
+        if (mbar_try_wait(bar, parity))
+            return true;
+        if (clock64() - t0 > limit) {
+            *fail = 1;
+            return false;
+        }
+    }
+}
+
 // Make generic-proxy writes to shared memory visible to the async proxy
 // (tensor core / TMA reads) -- issued by the writing threads before the
 // barrier that hands the data over.

@@ -90,7 +90,15 @@ typedef enum { RDM_GATES_ACTIVATED = 0, RDM_GATES_PREACT = 1 } rdm_gate_inputs;
  *   saved_states : [B,H,ceil(T/chunk),d_k,d_v] float32, written with the state
  *                  in force before each chunk (S_0 for chunk 0); NULL = skip.
  *                  rdm_ddts_bwd can reuse it instead of recomputing.
- *   chunk        : tokens per chunk; 0 selects 64.  Allowed: 64.
+ *   chunk        : tokens per chunk (the block over which the intra-chunk
+ *                  quadratic form is evaluated and between whose ends the state
+ *                  is passed); 0 selects 64.  Allowed: 16, 32, 64, 128.  The
+ *                  tensor-core path evaluates chunks of 16, 32 or 64 tokens
+ *                  (narrowing any chunk to 16 tokens, then to single tokens,
+ *                  where its log-decay span is too wide for one fp32
+ *                  reference); chunk 128 runs the exact token-serial path.
+ *                  Results agree across chunk sizes up to rounding.
+ *                  saved_states then holds one state per chunk of this size.
  *   gate_inputs  : RDM_GATES_ACTIVATED (default, 0) or RDM_GATES_PREACT.
  *   workspace    : optional device scratch of workspace_bytes.  With at least
  *                  rdm_ddts_fwd_workspace_size() bytes the tensor-core path
@@ -180,8 +188,13 @@ size_t rdm_ddts_bwd_workspace_size(const rdm_bwd_args *args);
  * path (args->impl, args->workspace and args->workspace_bytes are ignored).
  * The scratch comes from one 16 MiB array inside the library, allocated on
  * every device that loads it and held until the process exits.
- *   - The first call on a device, with that device current, looks up the
- *     array's device address; make that first call before any stream capture.
+ *   - The first call on a device, with that device current, loads the
+ *     library's module there if that has not happened yet (CUDA loads modules
+ *     lazily), which allocates the 16 MiB and may synchronise the device, and
+ *     looks up the array's device address.  Make one call at start-up, before
+ *     relying on the no-allocation guarantee and before any stream capture.
+ *     The address is looked up again on every call (it is cheap once the
+ *     module is loaded), so it stays right across cudaDeviceReset.
  *   - Problems needing more scratch than 16 MiB (B*H*T*d_k*4 + B*H*d_k*4
  *     bytes) return RDM_ERR_WORKSPACE and launch nothing.
  *   - All calls share the one array and it keeps whatever the last call left;
@@ -215,6 +228,22 @@ rdm_status rdm_ddts_sync_status(rdm_stream_t stream);
 
 /* Static, NUL-terminated description of a status code. */
 const char *rdm_status_string(rdm_status status);
+
+/* ----------------------------------------------------------------- testing
+ * Test hooks for the failure path of the bounded on-device waits; not for
+ * production use.  They apply to every later call in the process (all host
+ * threads) until reset with (0, 0).
+ *   wait_limit_cycles      : SM clock cycles after which a bounded wait gives
+ *                            up (0 = the default, about one second).
+ *   withhold_segment_flags : 1 = CTAs of a sequence-segmented tensor-core
+ *                            launch never publish the flag that tells later
+ *                            segments their input is ready, so those segments'
+ *                            waits run out: the kernel then stops, sets the
+ *                            device status word and returns, and
+ *                            rdm_ddts_sync_status reports RDM_ERR_TIMEOUT.
+ *                            Outputs of such a call are unspecified.
+ * Returns RDM_ERR_INVALID_ARG for a negative limit or a flag other than 0/1. */
+rdm_status rdm_ddts_set_test_hooks(long long wait_limit_cycles, int withhold_segment_flags);
 
 /* Library ABI version (major*10000 + minor*100 + patch). */
 int rdm_ddts_version(void);

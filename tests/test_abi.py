@@ -117,3 +117,11 @@ def test_decode_validation(lib):
 def test_sizes(lib):
     assert lib.rdm_ddts_saved_states_size(2, 3, 130, 64, 128, 64) == 2 * 3 * 3 * 64 * 128 * 4
     assert lib.rdm_ddts_saved_states_size(2, 3, 130, 64, 100, 64) == 0
+
+
+def test_test_hooks_validation(lib):
+    from gated_linear_attention_ddts_b200._binding import RDM_ERR_INVALID_ARG, RDM_OK
+    assert lib.rdm_ddts_set_test_hooks(-1, 0) == RDM_ERR_INVALID_ARG
+    assert lib.rdm_ddts_set_test_hooks(0, 2) == RDM_ERR_INVALID_ARG
+    assert lib.rdm_ddts_set_test_hooks(1000, 1) == RDM_OK
+    assert lib.rdm_ddts_set_test_hooks(0, 0) == RDM_OK

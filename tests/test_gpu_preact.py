@@ -77,6 +77,22 @@ def test_preact_backward_tc(cuda_ok, dv, T):
         assert_close(gr[n], ref[n], 2e-2, f"preact {n}")
 
 
+@pytest.mark.parametrize("T", [100, 64 * 9 + 3])
+def test_preact_backward_tc_states_recomputed(cuda_ok, T):
+    """No saved states passed: the backward recomputes them with a forward
+    launch of its own, which has to activate the gates too."""
+    x = draw_sequence(1, 2, T, 64, 128, torch.bfloat16, seed=710 + T, s0_std=0.1,
+                      with_dO=True, preact=True)
+    d = dev(x)
+    gr = rdm.rdm_ddts_bwd(*(d[n] for n in SEQ), d["S0"], d["dO"], None, None, impl="tc",
+                          gates="preact")
+    torch.cuda.synchronize()
+    assert rdm.rdm_ddts_sync_status() == rdm.RDM_OK
+    ref = oracle.bwd(*(x[n] for n in SEQ), x["S0"], x["dO"], preact=True)
+    for n in GR:
+        assert_close(gr[n], ref[n], 2e-2, f"preact, states recomputed: {n}")
+
+
 def test_preact_backward_simt_fp32(cuda_ok):
     x = draw_sequence(1, 2, 90, 16, 32, torch.float32, seed=93, s0_std=0.1, with_dO=True,
                       preact=True)

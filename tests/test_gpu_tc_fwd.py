@@ -84,29 +84,58 @@ def test_tc_g_zero_and_tau_zero(cuda_ok):
     assert_close(ST, S[:, :, -1], TOL, "tau=0 S_T")
 
 
-@pytest.mark.parametrize("dk,dv", [(64, 128), (16, 32)])
-def test_chunk_size_invariance(cuda_ok, dk, dv):
-    """The result does not depend on the chunk size asked for: every allowed
-    value against the default (the tensor-core path takes chunks of 64, cut
-    into windows of 16 or 1 token when the decay needs it; other sizes run the
-    exact path) and against the oracle.  Wide decay forces the windows."""
-    x = draw_sequence(1, 2, 300, dk, dv, torch.bfloat16, seed=61, s0_std=0.1)
-    x["g"] = (x["g"].float() * 6.0).to(torch.bfloat16)
+@pytest.mark.parametrize("dk,dv", [(64, 128), (128, 64), (64, 64)])
+@pytest.mark.parametrize("scale", [1.0, 6.0])
+def test_chunk_size_invariance(cuda_ok, dk, dv, scale):
+    """The chunked tensor-core kernel evaluated with chunks of 16, 32 and 64
+    tokens (impl="tc": every one of them runs on the tensor cores) gives the same
+    output, final state and saved chunk-start states up to rounding, against
+    the oracle and against chunk 64.  Chunk 128 runs the exact path and joins
+    the comparison.  scale 6 widens the decay so that some chunks are narrowed
+    to 16-token or single-token windows inside the kernel as well.  (Chunkwise
+    form: paperhub.cn OpenReview rebuttal, "Efficient Parallelization".)"""
+    B, H, T = 1, 2, 300
+    x = draw_sequence(B, H, T, dk, dv, torch.bfloat16, seed=61 + dk + dv, s0_std=0.1)
+    x["g"] = (x["g"].float() * scale).to(torch.bfloat16)
     d = {n: x[n].cuda() for n in SEQ}
     S0 = x["S0"].cuda()
-    ref = None
     o_ref, S_ref = oracle.fwd(*(x[n] for n in SEQ), x["S0"])
-    for chunk in (64, 16, 32, 128):
-        o, ST = rdm.rdm_ddts_fwd(*(d[n] for n in SEQ), S0, chunk=chunk, return_state=True)
+    ref = None
+    for chunk in (64, 32, 16, 128):
+        impl = "tc" if chunk <= 64 else "auto"
+        saved = torch.full((rdm.rdm_ddts_saved_states_size(B, H, T, dk, dv, chunk) // 4,),
+                           float("nan"), device="cuda")
+        o, ST = rdm.rdm_ddts_fwd(*(d[n] for n in SEQ), S0, saved_states=saved, chunk=chunk,
+                                 impl=impl, return_state=True)
         torch.cuda.synchronize()
         assert rdm.rdm_ddts_sync_status() == rdm.RDM_OK
         assert_close(o, o_ref, TOL, f"o chunk {chunk}")
         assert_close(ST, S_ref, TOL, f"S_T chunk {chunk}")
+        nc = (T + chunk - 1) // chunk
+        sv = saved.view(B, H, nc, dk, dv)
+        for c in sorted({1, nc // 2, nc - 1}):
+            sref = oracle.fwd(*(x[n][:, :, :chunk * c] for n in SEQ), x["S0"])[1]
+            assert_close(sv[:, :, c], sref, TOL, f"saved state {c} of chunk {chunk}")
         if ref is None:
             ref = (o.float().cpu().numpy(), ST.cpu().numpy())
         else:
             assert_close(o, ref[0], TOL, f"o chunk {chunk} vs 64")
             assert_close(ST, ref[1], TOL, f"S_T chunk {chunk} vs 64")
+
+
+@pytest.mark.parametrize("chunk", [16, 32])
+def test_chunk_size_segmented(cuda_ok, chunk):
+    """Small chunks inside sequence segments (state-only passes, folded maps)."""
+    x = draw_sequence(1, 2, 64 * 11 + 21, 64, 128, torch.bfloat16, seed=71 + chunk, s0_std=0.1)
+    assert segments_used(x)
+    d = {n: x[n].cuda() for n in SEQ}
+    o, ST = rdm.rdm_ddts_fwd(*(d[n] for n in SEQ), x["S0"].cuda(), chunk=chunk, impl="tc",
+                             return_state=True)
+    torch.cuda.synchronize()
+    assert rdm.rdm_ddts_sync_status() == rdm.RDM_OK
+    o_ref, S_ref = oracle.fwd(*(x[n] for n in SEQ), x["S0"])
+    assert_close(o, o_ref, TOL, f"o chunk {chunk}")
+    assert_close(ST, S_ref, TOL, f"S_T chunk {chunk}")
 
 
 def test_tc_split_invariance(cuda_ok):
@@ -221,8 +250,8 @@ def sampled_check(w, heads, device_inputs=True):
         xs = {n: x[n][b:b + 1, h:h + 1].cpu() for n in SEQ}
         s0 = x["S0"][b:b + 1, h:h + 1].cpu() if x["S0"] is not None else None
         o_ref, S_ref = oracle.fwd(*(xs[n] for n in SEQ), s0)
-        assert_close(o[b:b + 1, h:h + 1], o_ref, TOL, f"o head ({b},{h})")
-        assert_close(ST[b:b + 1, h:h + 1], S_ref, TOL, f"S_T head ({b},{h})")
+        assert_close(o[b:b + 1, h:h + 1], o_ref, TOL, f"workload {w.name[:12]} o head ({b},{h})")
+        assert_close(ST[b:b + 1, h:h + 1], S_ref, TOL, f"workload {w.name[:12]} S_T head ({b},{h})")
 
 
 def test_workload1_full_size_sampled(cuda_ok):
