@@ -31,7 +31,8 @@ class FwdArgs(ctypes.Structure):
                 ("dtype", _I), ("impl", _I),
                 ("q", _VP), ("k", _VP), ("v", _VP), ("g", _VP), ("tau", _VP), ("beta", _VP),
                 ("S0", _VP), ("o", _VP), ("ST", _VP), ("saved_states", _VP),
-                ("workspace", _VP), ("workspace_bytes", ctypes.c_size_t), ("gate_inputs", _I)]
+                ("workspace", _VP), ("workspace_bytes", ctypes.c_size_t), ("gate_inputs", _I),
+                ("feedthrough", _VP)]
 
 
 class BwdArgs(ctypes.Structure):
@@ -41,7 +42,14 @@ class BwdArgs(ctypes.Structure):
                 ("S0", _VP), ("grad_o", _VP), ("grad_ST", _VP), ("saved_states", _VP),
                 ("grad_q", _VP), ("grad_k", _VP), ("grad_v", _VP), ("grad_g", _VP),
                 ("grad_tau", _VP), ("grad_beta", _VP), ("grad_S0", _VP),
-                ("workspace", _VP), ("workspace_bytes", ctypes.c_size_t), ("gate_inputs", _I)]
+                ("workspace", _VP), ("workspace_bytes", ctypes.c_size_t), ("gate_inputs", _I),
+                ("feedthrough", _VP), ("grad_feedthrough", _VP)]
+
+
+class DecodeArgs(ctypes.Structure):
+    _fields_ = [("B", _I), ("H", _I), ("dk", _I), ("dv", _I), ("dtype", _I),
+                ("q", _VP), ("k", _VP), ("v", _VP), ("g", _VP), ("tau", _VP), ("beta", _VP),
+                ("S", _VP), ("o", _VP), ("feedthrough", _VP)]
 
 
 class RdmError(RuntimeError):
@@ -53,7 +61,8 @@ class RdmError(RuntimeError):
 _lib = None
 
 EXPORTS = ["rdm_ddts_fwd", "rdm_ddts_fwd_workspace_size", "rdm_ddts_saved_states_size", "rdm_ddts_bwd",
-           "rdm_ddts_bwd_workspace_size", "rdm_ddts_bwd_noalloc", "rdm_ddts_decode_step", "rdm_ddts_sync_status",
+           "rdm_ddts_bwd_workspace_size", "rdm_ddts_bwd_noalloc", "rdm_ddts_decode_step", "rdm_ddts_decode",
+           "rdm_ddts_sync_status",
            "rdm_status_string", "rdm_ddts_set_test_hooks", "rdm_ddts_version"]
 
 
@@ -79,6 +88,8 @@ def load():
         lib.rdm_ddts_bwd_noalloc.restype = _I
         lib.rdm_ddts_decode_step.argtypes = [_I] * 5 + [_VP] * 9
         lib.rdm_ddts_decode_step.restype = _I
+        lib.rdm_ddts_decode.argtypes = [ctypes.POINTER(DecodeArgs), _VP]
+        lib.rdm_ddts_decode.restype = _I
         lib.rdm_ddts_sync_status.argtypes = [_VP]
         lib.rdm_ddts_sync_status.restype = _I
         lib.rdm_status_string.argtypes = [_I]
@@ -129,12 +140,13 @@ def rdm_ddts_saved_states_size(B, H, T, dk, dv, chunk=0) -> int:
 
 
 def _fwd_args(q, k, v, g, tau, beta, S0, o, ST, saved_states, ws, ws_bytes, chunk, impl,
-              gates="activated"):
+              gates="activated", feedthrough=None):
     B, H, T, dk = q.shape
     dv = v.shape[-1]
     return FwdArgs(B, H, T, dk, dv, chunk, _dtype_code(q), IMPL[impl],
                    _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(tau), _ptr(beta), _ptr(S0), _ptr(o),
-                   _ptr(ST), _ptr(saved_states), _ptr(ws), ws_bytes, GATES[gates])
+                   _ptr(ST), _ptr(saved_states), _ptr(ws), ws_bytes, GATES[gates],
+                   _ptr(feedthrough))
 
 
 def rdm_ddts_fwd_workspace_size(q, k, v, g, tau, beta, *, chunk=0, impl="auto",
@@ -148,11 +160,11 @@ def rdm_ddts_fwd_workspace_size(q, k, v, g, tau, beta, *, chunk=0, impl="auto",
 
 def rdm_ddts_fwd(q, k, v, g, tau, beta, S0=None, o=None, ST=None, saved_states=None, *,
                  workspace=None, chunk=0, impl="auto", return_state=False, stream=None,
-                 gates="activated"):
+                 gates="activated", feedthrough=None):
     """Forward over [B,H,T,D] sequences.  Allocates o (and S_T when
     return_state) with torch if not given, and the sequence-segment workspace
-    when none is passed (workspace=False runs without one).  Returns
-    (o, S_T or None)."""
+    when none is passed (workspace=False runs without one).  feedthrough: [H,dv]
+    float32 weights d, o_t += d * v_t.  Returns (o, S_T or None)."""
     B, H, T, dk = q.shape
     dv = v.shape[-1]
     if o is None:
@@ -167,13 +179,13 @@ def rdm_ddts_fwd(q, k, v, g, tau, beta, S0=None, o=None, ST=None, saved_states=N
         workspace = None
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     a = _fwd_args(q, k, v, g, tau, beta, S0, o, ST, saved_states, workspace, ws_bytes, chunk,
-                  impl, gates)
+                  impl, gates, feedthrough)
     _check(load().rdm_ddts_fwd(ctypes.byref(a), _stream(stream)), "rdm_ddts_fwd")
     return o, ST
 
 
 def _bwd_args(q, k, v, g, tau, beta, S0, grad_o, grad_ST, saved_states, grads, ws, ws_bytes,
-              chunk, impl, gates="activated"):
+              chunk, impl, gates="activated", feedthrough=None):
     B, H, T, dk = q.shape
     dv = v.shape[-1]
     return BwdArgs(B, H, T, dk, dv, chunk, _dtype_code(q), IMPL[impl],
@@ -181,7 +193,7 @@ def _bwd_args(q, k, v, g, tau, beta, S0, grad_o, grad_ST, saved_states, grads, w
                    _ptr(grad_o), _ptr(grad_ST), _ptr(saved_states),
                    *(_ptr(grads.get(n)) for n in ("dq", "dk", "dv", "dg", "dtau", "dbeta",
                                                     "dS0")),
-                   _ptr(ws), ws_bytes, GATES[gates])
+                   _ptr(ws), ws_bytes, GATES[gates], _ptr(feedthrough), _ptr(grads.get("dfeed")))
 
 
 def rdm_ddts_bwd_workspace_size(q, k, v, g, tau, beta, S0=None, grad_o=None, grad_ST=None,
@@ -197,9 +209,10 @@ def rdm_ddts_bwd_workspace_size(q, k, v, g, tau, beta, S0=None, grad_o=None, gra
 
 def rdm_ddts_bwd(q, k, v, g, tau, beta, S0, grad_o, grad_ST=None, saved_states=None, *,
                  grads=None, workspace=None, chunk=0, impl="auto", want_dS0=True, stream=None,
-                 gates="activated"):
-    """Backward.  `grads` may hold preallocated dq, dk, dv, dg, dtau, dbeta, dS0;
-    missing ones are allocated with torch, as is the workspace.  Returns the dict."""
+                 gates="activated", feedthrough=None):
+    """Backward.  `grads` may hold preallocated dq, dk, dv, dg, dtau, dbeta, dS0
+    (and dfeed when feedthrough is given); missing ones are allocated with
+    torch, as is the workspace.  Returns the dict."""
     B, H, T, dk = q.shape
     dv = v.shape[-1]
     grads = dict(grads or {})
@@ -208,12 +221,14 @@ def rdm_ddts_bwd(q, k, v, g, tau, beta, S0, grad_o, grad_ST=None, saved_states=N
             grads[n] = torch.empty_like(ref)
     if want_dS0 and grads.get("dS0") is None:
         grads["dS0"] = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device)
+    if feedthrough is not None and grads.get("dfeed") is None:
+        grads["dfeed"] = torch.empty(H, dv, dtype=torch.float32, device=q.device)
     if workspace is None:
         need = rdm_ddts_bwd_workspace_size(q, k, v, g, tau, beta, S0, grad_o, grad_ST,
                                            saved_states, chunk=chunk, impl=impl, gates=gates)
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
     a = _bwd_args(q, k, v, g, tau, beta, S0, grad_o, grad_ST, saved_states, grads, workspace,
-                  workspace.numel() * workspace.element_size(), chunk, impl, gates)
+                  workspace.numel() * workspace.element_size(), chunk, impl, gates, feedthrough)
     _check(load().rdm_ddts_bwd(ctypes.byref(a), _stream(stream)), "rdm_ddts_bwd")
     return grads
 
@@ -248,6 +263,19 @@ def rdm_ddts_decode_step(q, k, v, g, tau, beta, S, o=None, *, stream=None):
                                      _ptr(g), _ptr(tau), _ptr(beta), _ptr(S), _ptr(o),
                                      _stream(stream))
     _check(st, "rdm_ddts_decode_step")
+    return o
+
+
+def rdm_ddts_decode(q, k, v, g, tau, beta, S, o=None, *, feedthrough=None, stream=None):
+    """rdm_ddts_decode_step with the feedthrough: o = S^T q + d * v when
+    feedthrough ([H,dv] float32) is given."""
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    if o is None:
+        o = torch.empty(B, H, dv, dtype=q.dtype, device=q.device)
+    a = DecodeArgs(B, H, dk, dv, _dtype_code(q), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(tau),
+                   _ptr(beta), _ptr(S), _ptr(o), _ptr(feedthrough))
+    _check(load().rdm_ddts_decode(ctypes.byref(a), _stream(stream)), "rdm_ddts_decode")
     return o
 
 

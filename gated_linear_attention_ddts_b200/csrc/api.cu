@@ -101,6 +101,7 @@ SeqParams fwd_params(const rdm_fwd_args* a) {
     p.preact = a->gate_inputs == RDM_GATES_PREACT;
     p.wait_limit = wait_limit();
     p.withhold_flags = g_hook_withhold.load(std::memory_order_relaxed);
+    p.dfeed = a->feedthrough;
     return p;
 }
 
@@ -118,6 +119,8 @@ BwdParams bwd_params(const rdm_bwd_args* a) {
     p.preact = a->gate_inputs == RDM_GATES_PREACT;
     p.wait_limit = wait_limit();
     p.withhold_flags = g_hook_withhold.load(std::memory_order_relaxed);
+    p.dfeed = a->feedthrough;
+    p.grad_dfeed = a->grad_feedthrough;
     return p;
 }
 
@@ -142,7 +145,7 @@ rdm_status rdm_ddts_fwd(const rdm_fwd_args* a, rdm_stream_t stream) {
     if (!gates_ok(a->gate_inputs)) return RDM_ERR_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (!opt_aligned(a->S0) || !opt_aligned(a->ST) || !opt_aligned(a->saved_states) ||
-        !opt_aligned(a->workspace))
+        !opt_aligned(a->workspace) || !opt_aligned(a->feedthrough))
         return RDM_ERR_INVALID_ARG;
     if (a->T == 0) {
         if (a->impl == RDM_IMPL_TC && a->dtype != RDM_BF16) return RDM_ERR_UNSUPPORTED;
@@ -187,11 +190,16 @@ rdm_status rdm_ddts_bwd(const rdm_bwd_args* a, rdm_stream_t stream) {
     if (!gates_ok(a->gate_inputs)) return RDM_ERR_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (!opt_aligned(a->S0) || !opt_aligned(a->grad_ST) || !opt_aligned(a->grad_S0) ||
-        !opt_aligned(a->saved_states) || !opt_aligned(a->workspace))
+        !opt_aligned(a->saved_states) || !opt_aligned(a->workspace) ||
+        !opt_aligned(a->feedthrough) || !opt_aligned(a->grad_feedthrough))
         return RDM_ERR_INVALID_ARG;
+    if (a->grad_feedthrough && !a->feedthrough) return RDM_ERR_INVALID_ARG;
     if (a->T == 0) {
         if (a->impl == RDM_IMPL_TC && a->dtype != RDM_BF16) return RDM_ERR_UNSUPPORTED;
-        // no tokens: dS_0 = dS_T
+        // no tokens: dS_0 = dS_T, and the feedthrough gradient is zero
+        if (a->grad_feedthrough &&
+            cudaMemsetAsync(a->grad_feedthrough, 0, (size_t)a->H * a->dv * 4, s) != cudaSuccess)
+            return RDM_ERR_CUDA;
         return empty_sequence(a->B, a->H, a->dk, a->dv, a->grad_ST, a->grad_S0, s);
     }
     const void* in[] = {a->q, a->k, a->v, a->g, a->tau, a->beta, a->grad_o, a->grad_q,
@@ -205,21 +213,34 @@ rdm_status rdm_ddts_bwd(const rdm_bwd_args* a, rdm_stream_t stream) {
     if (a->impl == RDM_IMPL_TC && !tc) return RDM_ERR_UNSUPPORTED;
     const size_t need = tc ? tc_bwd_workspace(p) : simt_bwd_workspace(p);
     if (need > 0 && (!a->workspace || a->workspace_bytes < need)) return RDM_ERR_WORKSPACE;
-    return from_cuda(tc ? launch_tc_bwd(p, s) : launch_simt_bwd(p, s));
+    cudaError_t e = tc ? launch_tc_bwd(p, s) : launch_simt_bwd(p, s);
+    if (e == cudaSuccess && p.grad_dfeed) e = launch_feed_grad(p, s);
+    return from_cuda(e);
+}
+
+rdm_status rdm_ddts_decode(const rdm_decode_args* a, rdm_stream_t stream) {
+    if (!a) return RDM_ERR_INVALID_ARG;
+    rdm_status st = check_sizes(a->B, a->H, 1, a->dk, a->dv, 0, a->dtype, RDM_IMPL_AUTO);
+    if (st != RDM_OK) return st;
+    const void* in[] = {a->q, a->k, a->v, a->g, a->tau, a->beta, a->S, a->o};
+    for (const void* p : in)
+        if (!p || !aligned(p)) return RDM_ERR_INVALID_ARG;
+    if (!opt_aligned(a->feedthrough)) return RDM_ERR_INVALID_ARG;
+    DecodeParams p;
+    p.B = a->B; p.H = a->H; p.dk = a->dk; p.dv = a->dv; p.bf16 = a->dtype == RDM_BF16;
+    p.q = a->q; p.k = a->k; p.v = a->v; p.g = a->g; p.tau = a->tau; p.beta = a->beta;
+    p.S = a->S; p.o = a->o; p.dfeed = a->feedthrough;
+    return from_cuda(launch_decode(p, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 rdm_status rdm_ddts_decode_step(int B, int H, int dk, int dv, rdm_dtype dtype, const void* q,
                                 const void* k, const void* v, const void* g, const void* tau,
                                 const void* beta, float* S, void* o, rdm_stream_t stream) {
-    rdm_status st = check_sizes(B, H, 1, dk, dv, 0, dtype, RDM_IMPL_AUTO);
-    if (st != RDM_OK) return st;
-    const void* in[] = {q, k, v, g, tau, beta, S, o};
-    for (const void* p : in)
-        if (!p || !aligned(p)) return RDM_ERR_INVALID_ARG;
-    DecodeParams p;
-    p.B = B; p.H = H; p.dk = dk; p.dv = dv; p.bf16 = dtype == RDM_BF16;
-    p.q = q; p.k = k; p.v = v; p.g = g; p.tau = tau; p.beta = beta; p.S = S; p.o = o;
-    return from_cuda(launch_decode(p, reinterpret_cast<cudaStream_t>(stream)));
+    rdm_decode_args a;
+    a.B = B; a.H = H; a.dk = dk; a.dv = dv; a.dtype = dtype;
+    a.q = q; a.k = k; a.v = v; a.g = g; a.tau = tau; a.beta = beta; a.S = S; a.o = o;
+    a.feedthrough = nullptr;
+    return rdm_ddts_decode(&a, stream);
 }
 
 rdm_status rdm_ddts_sync_status(rdm_stream_t stream) {
@@ -258,6 +279,6 @@ rdm_status rdm_ddts_set_test_hooks(long long wait_limit_cycles, int withhold_seg
     return RDM_OK;
 }
 
-int rdm_ddts_version(void) { return 400; }
+int rdm_ddts_version(void) { return 500; }
 
 }  // extern "C"

@@ -76,6 +76,13 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(DecodeParams p) {
     __syncthreads();
     if (rs == 0) {
         float4 o4 = s_red[0][cq];
+        if (p.dfeed) {  // feedthrough o += d (.) v
+            const float* d = p.dfeed + (size_t)(bh % p.H) * DV + 4 * cq;
+            o4.x = fmaf(d[0], ldf(v + 4 * cq + 0), o4.x);
+            o4.y = fmaf(d[1], ldf(v + 4 * cq + 1), o4.y);
+            o4.z = fmaf(d[2], ldf(v + 4 * cq + 2), o4.z);
+            o4.w = fmaf(d[3], ldf(v + 4 * cq + 3), o4.w);
+        }
 #pragma unroll
         for (int r = 1; r < RS; ++r) {
             const float4 x = s_red[r][cq];

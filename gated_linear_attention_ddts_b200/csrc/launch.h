@@ -24,6 +24,7 @@ struct SeqParams {
     unsigned* err;       // device status word
     long long wait_limit;  // SM clock cycles a bounded wait may take before it gives up
     int withhold_flags;    // test hook: segment CTAs never publish their flags
+    const float* dfeed;    // feedthrough weights [H][dv]: o_t += d (.) v_t; null = none
 };
 
 struct BwdParams {
@@ -42,6 +43,8 @@ struct BwdParams {
     unsigned* err;
     long long wait_limit;  // as SeqParams
     int withhold_flags;
+    const float* dfeed;    // feedthrough weights [H][dv], or null
+    float* grad_dfeed;     // dL/d(feedthrough) [H][dv], written when non-null
 };
 
 struct DecodeParams {
@@ -50,6 +53,7 @@ struct DecodeParams {
     const void *q, *k, *v, *g, *tau, *beta;
     float* S;
     void* o;
+    const float* dfeed;  // feedthrough weights [H][dv], or null
 };
 
 // exact token-serial CUDA-core path (any supported shape, float32 or bf16)
@@ -61,6 +65,10 @@ cudaError_t launch_simt_bwd_flagged(const BwdParams& p, const int* flags, cudaSt
 
 // decode step
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s);
+
+// gradient of the feedthrough weights: grad_d[h][j] = sum_{b,t} dO[b,h,t,j] v[b,h,t,j]
+// (zeroes grad_d, then accumulates; float32 atomics)
+cudaError_t launch_feed_grad(const BwdParams& p, cudaStream_t s);
 
 // tensor-core (tcgen05) chunked path
 bool tc_fwd_supported(const SeqParams& p);

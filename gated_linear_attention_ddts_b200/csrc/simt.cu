@@ -69,8 +69,10 @@ __global__ void __launch_bounds__(128) simt_fwd_kernel(SeqParams p) {
                 for (int i = 0; i < DK; ++i) dst[(size_t)i * dv] = s[i];
             }
             const float bb = ldf(beta + (size_t)t * dv + j);
-            const float vh = (p.preact ? sigmoid_acc(bb) : bb) * ldf(v + (size_t)t * dv + j);
-            float acc = 0.0f;
+            const float vt = ldf(v + (size_t)t * dv + j);
+            const float vh = (p.preact ? sigmoid_acc(bb) : bb) * vt;
+            // feedthrough o_t += d (.) v_t
+            float acc = p.dfeed ? p.dfeed[(size_t)(bh % p.H) * dv + j] * vt : 0.0f;
 #pragma unroll
             for (int i = 0; i < DK; ++i) {
                 s[i] = fmaf(s_al[tt][i], s[i], s_kh[tt][i] * vh);
@@ -239,7 +241,8 @@ __global__ void __launch_bounds__(128) simt_bwd_rsweep(BwdParams p, const float*
                 const size_t ov = (size_t)(t0 + tt) * DV + j;
                 const float b_in = ldf(beta + ov);
                 const float bb = p.preact ? sigmoid_acc(b_in) : b_in;
-                stf(dv_ + ov, bb * dvh);
+                const float df = p.dfeed ? p.dfeed[(size_t)(bh % p.H) * DV + j] * ldf(dO + ov) : 0.0f;
+                stf(dv_ + ov, fmaf(bb, dvh, df));
                 stf(dbeta + ov, (p.preact ? bb * (1.0f - bb) : 1.0f) * ldf(v + ov) * dvh);
             }
             __syncthreads();

@@ -673,6 +673,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             for (int j = 0; j < HV; ++j)
                 R[j] = p.dST ? p.dST[((size_t)bh * DK + r) * DV + hf * HV + j] : 0.0f;
         };
+        // A segment's map in the workspace is kept in the epilogue's register
+        // order (float4 k of thread et at k * 128 + et), so that every warp
+        // instruction reads or writes 512 contiguous bytes.
+        auto seg_map_ptr = [&](size_t u) {
+            return reinterpret_cast<float4*>(sg.st) + u * (DK * DV / 4) + (threadIdx.x - 32 * kEpiWarp0);
+        };
         // R at the end of this segment: dS_T carried through the maps of all later
         // segments, R <- diag(D_s) R + R_loc_s; then the decay-gradient carry into
         // the segment, rowsum(R o S) with S the saved state at the segment end
@@ -693,10 +699,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             for (int s2 = P - 1; s2 > seg; --s2) {
                 const size_t u = (size_t)s2 * BH + bh;
                 const float d = ex2_fast(__ldcg(&sg.ld[u * DK + r]));
-                const float4* src = reinterpret_cast<const float4*>(sg.st + (u * DK + r) * DV + hf * HV);
+                const float4* src = seg_map_ptr(u);
 #pragma unroll
                 for (int j4 = 0; j4 < HV / 4; ++j4) {
-                    const float4 x = __ldcg(src + j4);
+                    const float4 x = __ldcg(src + j4 * 128);
                     R[4 * j4] = fmaf(d, R[4 * j4], x.x);
                     R[4 * j4 + 1] = fmaf(d, R[4 * j4 + 1], x.y);
                     R[4 * j4 + 2] = fmaf(d, R[4 * j4 + 2], x.z);
@@ -716,10 +722,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
         // publish this segment's map (R_loc in R, log2 D in ld2)
         auto publish_segment = [&](float ld2) -> bool {
             const size_t u = (size_t)seg * BH + bh;
-            float4* dst = reinterpret_cast<float4*>(sg.st + (u * DK + r) * DV + hf * HV);
+            float4* dst = seg_map_ptr(u);
 #pragma unroll
             for (int j4 = 0; j4 < HV / 4; ++j4)
-                dst[j4] = make_float4(R[4 * j4], R[4 * j4 + 1], R[4 * j4 + 2], R[4 * j4 + 3]);
+                dst[j4 * 128] = make_float4(R[4 * j4], R[4 * j4 + 1], R[4 * j4 + 2], R[4 * j4 + 3]);
             if (hf == 0) sg.ld[u * DK + r] = ld2;
             __threadfence();
             named_bar(kBarEpi, 128);
@@ -860,6 +866,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                         for (int e = 0; e < 8; ++e) {
                             ov[e] = b8[e] * v[8 * h4 + e];
                             ob[e] = cb[e] * v8[e] * v[8 * h4 + e];
+                        }
+                        if (p.dfeed != nullptr) {  // feedthrough: dv_t += d (.) dO_t
+                            float do8[8];
+                            unpack8(*reinterpret_cast<const uint4*>(sm.raw + K::OFF_DO + off_raw(r, jg)), do8);
+                            const float4* dr = reinterpret_cast<const float4*>(p.dfeed + (size_t)(bh % p.H) * DV + 8 * jg);
+                            const float4 d0 = __ldg(dr), d1 = __ldg(dr + 1);
+                            const float dd[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) ov[e] = fmaf(dd[e], do8[e], ov[e]);
                         }
                         *reinterpret_cast<uint4*>(sm.u.ost + off_raw(r, jg)) = pack8(ov);
                         *reinterpret_cast<uint4*>(sm.u.ost + VB * kBox + off_raw(r, jg)) = pack8(ob);

@@ -105,6 +105,8 @@ struct alignas(1024) FwdSmem {
     uint64_t mma1_done, as_free, abf_full, mmao_done[2], o_free[2], vh_full[K::NB];
     int need16[2], need1[2];
     int epi_fail;  // the epilogue's own exit decision (written before a role barrier)
+    int nbefore;                   // state-only pieces before this CTA's segment
+    uint16_t blist[2 * kMaxSeg];   // their slots, in chunk order
     uint8_t before[2 * kMaxSeg];  // state-only pieces that precede this CTA's segment
     uint32_t tmem_base;
     int fail;
@@ -167,16 +169,19 @@ struct FwdKernelArgs {
     SegArgs seg;
 };
 
-// PRE: g, tau, beta arrive before their activations
-template <int DK, int DVT, bool PRE>
+// PRE: g, tau, beta arrive before their activations; FEED: o_t += d (.) v_t
+template <int DK, int DVT, bool PRE, bool FEED>
 __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_constant__ FwdKernelArgs A) {
     using K = Cfg<DK, DVT>;
     constexpr int NS = K::NS, NB = K::NB, KB = K::KB, VB = K::VB;
     // Who builds Vh = beta_hat * v: the epilogue warps when d_k = 128 (the gate
     // warps then carry twice the key-side work and are the slower role, which
-    // also hides the v / beta load behind them); the gate warps otherwise, where
-    // moving it would put that load on the epilogue's path to the first MMA group.
-    constexpr bool kVhEpi = DK == 128;
+    // also hides the v / beta load behind them) and when the gates arrive before
+    // their activations (the gate warps then also evaluate softplus and sigmoid
+    // on the key side; measured 124 -> 116 us on the 130M-scale layer); the gate
+    // warps otherwise, where moving it would put that load on the epilogue's
+    // path to the first MMA group.
+    constexpr bool kVhEpi = DK == 128 || PRE;
     // align by pointer arithmetic on the __shared__ array so that every access
     // below stays a shared-memory access (an integer round trip would make it generic)
     extern __shared__ __align__(1024) uint8_t smem_dyn[];
@@ -701,9 +706,18 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
         };
         // entry state of this segment: S_0 carried through the maps of all the
         // state-only pieces before it, in chunk order, S <- diag(D) S + S_loc
-        auto fold_earlier = [&]() -> bool {
-            // which pieces: slot 2j + h is [a0, mid) or [mid, a1) of range j; one
-            // slot per thread (the range arithmetic divides 64-bit integers)
+        // A piece's state in the workspace is kept in the epilogue's register
+        // order: float4 k of thread et at index k * 256 + et, so that each warp
+        // instruction reads or writes 512 contiguous bytes (the rows of the
+        // state are 512 bytes apart in the threads' own layout).
+        auto piece_ptr = [&](size_t u) {
+            return reinterpret_cast<float4*>(sg.st) + u * (DK * DVT / 4) + (threadIdx.x - 32 * kEpiWarp0);
+        };
+        // which state-only pieces precede this segment (slot 2j + h is [a0, mid)
+        // or [mid, a1) of range j), in chunk order: worked out at the start,
+        // while the first tiles are still in flight (one slot per thread; the
+        // range arithmetic divides 64-bit integers)
+        auto plan_fold = [&]() {
             const int et = threadIdx.x - 32 * kEpiWarp0;
             for (int slot = et; slot < 2 * P; slot += 32 * kEpiWarps) {
                 const P1Range r = p1_range(slot >> 1, NC, P);
@@ -712,10 +726,28 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             }
             epi_sync();
             if (threadIdx.x == 0) {
+                int nb = 0;
+                for (int slot = 0; slot < 2 * P; ++slot)
+                    if (sm.before[slot]) sm.blist[nb++] = (uint16_t)slot;
+                sm.nbefore = nb;
+            }
+            epi_sync();
+        };
+        // entry state of this segment: S_0 carried through the maps of the pieces
+        // before it, S <- diag(D_p) S + S_loc_p in chunk order, evaluated as
+        //   S = (prod_p D_p) S_0 + sum_p (prod_{p' after p} D_p') S_loc_p
+        // (same products, every piece's loads in flight together)
+        auto fold_earlier = [&]() -> bool {
+            const int nb = sm.nbefore;
+            if (nb == 0) {
+                load_s0();
+                return true;
+            }
+            if (threadIdx.x == 0) {
                 const long long t0 = clock64();
-                for (int slot = 0; slot < 2 * P && !*fail; ++slot) {
-                    if (!sm.before[slot]) continue;
-                    while (ld_acquire_gpu(&sg.flag[slot * units + unit]) != sg.epoch)
+                for (int i = 0; i < nb && !sm.epi_fail; ++i) {
+                    const unsigned* fl = &sg.flag[sm.blist[i] * units + unit];
+                    while (ld_acquire_gpu(fl) != sg.epoch)
                         if (clock64() - t0 > WL) {
                             *fail = 1;
                             sm.epi_fail = 1;
@@ -725,34 +757,47 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             }
             epi_sync();
             if (sm.epi_fail) return false;  // written by thread 0 before the barrier
-            load_s0();
-            for (int slot = 0; slot < 2 * P; ++slot) {
-                if (!sm.before[slot]) continue;
-                const size_t u = (size_t)slot * units + unit;
-                const float d = ex2_fast(__ldcg(&sg.ld[u * DK + iS]));
-                const float4* src = reinterpret_cast<const float4*>(sg.st + (u * DK + iS) * DVT + sc0);
+#pragma unroll
+            for (int j = 0; j < SC; ++j) S[j] = 0.0f;
+            float lsum = 0.0f;  // log2 of the decay of the pieces after the current one
+#pragma unroll 1
+            for (int i = nb - 1; i >= 0; --i) {
+                const size_t u = (size_t)sm.blist[i] * units + unit;
+                const float4* src = piece_ptr(u);
+                const float sc = ex2_fast(lsum);
+                lsum += __ldcg(&sg.ld[u * DK + iS]);
 #pragma unroll
                 for (int j4 = 0; j4 < SC / 4; ++j4) {
-                    const float4 x = __ldcg(src + j4);
-                    S[4 * j4] = fmaf(d, S[4 * j4], x.x);
-                    S[4 * j4 + 1] = fmaf(d, S[4 * j4 + 1], x.y);
-                    S[4 * j4 + 2] = fmaf(d, S[4 * j4 + 2], x.z);
-                    S[4 * j4 + 3] = fmaf(d, S[4 * j4 + 3], x.w);
+                    const float4 x = __ldcg(src + j4 * 32 * kEpiWarps);
+                    S[4 * j4] = fmaf(sc, x.x, S[4 * j4]);
+                    S[4 * j4 + 1] = fmaf(sc, x.y, S[4 * j4 + 1]);
+                    S[4 * j4 + 2] = fmaf(sc, x.z, S[4 * j4 + 2]);
+                    S[4 * j4 + 3] = fmaf(sc, x.w, S[4 * j4 + 3]);
                 }
+            }
+            if (p.S0) {
+                const float d0 = ex2_fast(lsum);
+                const float* s0 = p.S0 + ((size_t)bh * DK + iS) * p.dv + j0 + sc0;
+#pragma unroll
+                for (int j = 0; j < SC; ++j) S[j] = fmaf(d0, s0[j], S[j]);
             }
             return true;
         };
         // publish the map of a state-only piece (S_loc in S, log2 D in ld2)
         auto publish_piece = [&](int slot, float ld2) -> bool {
             const size_t u = (size_t)slot * units + unit;
-            float4* dst = reinterpret_cast<float4*>(sg.st + (u * DK + iS) * DVT + sc0);
+            float4* dst = piece_ptr(u);
 #pragma unroll
             for (int j4 = 0; j4 < SC / 4; ++j4)
-                dst[j4] = make_float4(S[4 * j4], S[4 * j4 + 1], S[4 * j4 + 2], S[4 * j4 + 3]);
+                dst[j4 * 32 * kEpiWarps] = make_float4(S[4 * j4], S[4 * j4 + 1], S[4 * j4 + 2], S[4 * j4 + 3]);
             if (sc0 == 0) sg.ld[u * DK + iS] = ld2;
-            __threadfence();
+            // every row is written (CTA barrier); one fence at GPU scope then makes
+            // all of them visible before the flag is
             epi_sync();
-            if (threadIdx.x == 0 && !p.withhold_flags) st_release_gpu(&sg.flag[u], sg.epoch);
+            if (threadIdx.x == 0 && !p.withhold_flags) {
+                __threadfence();
+                st_release_gpu(&sg.flag[u], sg.epoch);
+            }
             return true;
         };
         // o rows [w0, w1) of chunk c from the O buffer of o-item `io`.  A whole
@@ -767,6 +812,22 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.o_free[obuf]);
+            // feedthrough o_t += d (.) v_t (row tA, this thread's columns); v of
+            // this chunk has left shared memory, its rows come back from L2
+            if (FEED && c * C + tA < T) {
+                const uint4* vr = reinterpret_cast<const uint4*>(
+                    static_cast<const __nv_bfloat16*>(p.v) + ((size_t)bh * T + (size_t)c * C + tA) * p.dv + j0 + oc0);
+                const float4* dr = reinterpret_cast<const float4*>(p.dfeed + (size_t)(bh % p.H) * p.dv + j0 + oc0);
+#pragma unroll
+                for (int s8 = 0; s8 < OC / 8; ++s8) {
+                    float x[8];
+                    unpack8(__ldg(vr + s8), x);
+                    const float4 d0 = __ldg(dr + 2 * s8), d1 = __ldg(dr + 2 * s8 + 1);
+                    const float dd[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) v[8 * s8 + e] = fmaf(dd[e], x[e], v[8 * s8 + e]);
+                }
+            }
             const bool whole = w0 == 0 && w1 == min(C, T - c * C);
             if (whole) {
                 // the previous store has read the staging tile
@@ -795,8 +856,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
         bool ok_run = true;
         if (P == 1) {
             load_s0();
-        } else if (!has_p1) {
-            ok_run = fold_earlier();
+        } else {
+            plan_fold();
+            if (!has_p1) ok_run = fold_earlier();
         }
         int item = 0, io = 0, nm1 = 0, pc = 0, pw0 = 0, pw1 = 0;
         while (ok_run) {
@@ -1036,7 +1098,7 @@ SegPlan choose_plan(const SeqParams& p, bool allow_seg) {
     return best;
 }
 
-template <int DK, int DVT, bool PRE>
+template <int DK, int DVT, bool PRE, bool FEED>
 cudaError_t launch_cfg(const SeqParams& p, SegPlan plan, cudaStream_t s) {
     FwdKernelArgs a;
     a.p = p;
@@ -1054,7 +1116,7 @@ cudaError_t launch_cfg(const SeqParams& p, SegPlan plan, cudaStream_t s) {
                           32, DK))
         return cudaErrorInvalidValue;
     const size_t smem = sizeof(FwdSmem<DK, DVT>) + 1024;
-    auto kern = tc_fwd_kernel<DK, DVT, PRE>;
+    auto kern = tc_fwd_kernel<DK, DVT, PRE, FEED>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const unsigned units = (unsigned)(BH * (p.dv / DVT));
@@ -1077,14 +1139,17 @@ cudaError_t launch_cfg(const SeqParams& p, SegPlan plan, cudaStream_t s) {
     return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
-template <bool PRE>
+template <bool PRE, bool FEED>
 cudaError_t launch_plan_t(const SeqParams& p, const SegPlan& plan, cudaStream_t s) {
-    if (p.dk == 128) return launch_cfg<128, 64, PRE>(p, plan, s);
-    return plan.DVT == 128 ? launch_cfg<64, 128, PRE>(p, plan, s) : launch_cfg<64, 64, PRE>(p, plan, s);
+    if (p.dk == 128) return launch_cfg<128, 64, PRE, FEED>(p, plan, s);
+    return plan.DVT == 128 ? launch_cfg<64, 128, PRE, FEED>(p, plan, s)
+                           : launch_cfg<64, 64, PRE, FEED>(p, plan, s);
 }
 
 cudaError_t launch_plan(const SeqParams& p, const SegPlan& plan, cudaStream_t s) {
-    return p.preact ? launch_plan_t<true>(p, plan, s) : launch_plan_t<false>(p, plan, s);
+    if (p.dfeed)
+        return p.preact ? launch_plan_t<true, true>(p, plan, s) : launch_plan_t<false, true>(p, plan, s);
+    return p.preact ? launch_plan_t<true, false>(p, plan, s) : launch_plan_t<false, false>(p, plan, s);
 }
 
 }  // namespace

@@ -107,6 +107,15 @@ typedef enum { RDM_GATES_ACTIVATED = 0, RDM_GATES_PREACT = 1 } rdm_gate_inputs;
  *                  NULL, it runs each sequence in one CTA.  Results agree up
  *                  to rounding either way.  Contents on entry are ignored; two
  *                  calls whose kernels may overlap must not share it.
+ *   feedthrough  : [H,d_v] float32 weights d, or NULL for none.  With d the
+ *                  output is o_t = S_t^T q_t + d (.) v_t: the feedthrough d_t
+ *                  of the paper's Eq. (11), which the rebuttal's answer to Q6
+ *                  (paperhub.cn OpenReview page) names the SSM feedthrough, as
+ *                  in Mamba and Mamba2 (a learned per-channel skip from the SSM
+ *                  input, here v_t, to the output).  The pages print neither
+ *                  its shape nor its input; this library takes one weight per
+ *                  head and value channel, constant over time, applied to v_t
+ *                  (not to beta_hat * v_t).  Added in the store stage of o.
  */
 typedef struct {
     int B, H, T, dk, dv;
@@ -121,6 +130,7 @@ typedef struct {
     void *workspace;
     size_t workspace_bytes;
     rdm_gate_inputs gate_inputs;
+    const float *feedthrough;
 } rdm_fwd_args;
 
 rdm_status rdm_ddts_fwd(const rdm_fwd_args *args, rdm_stream_t stream);
@@ -152,6 +162,13 @@ size_t rdm_ddts_saved_states_size(int B, int H, int T, int dk, int dv, int chunk
  *   workspace    : device scratch of at least rdm_ddts_bwd_workspace_size()
  *                  bytes (may be NULL when that size is 0); contents on entry
  *                  are ignored and on exit are unspecified.
+ *   feedthrough  : the forward's feedthrough weights [H,d_v] float32, or NULL
+ *                  (then grad_v has no feedthrough term and grad_feedthrough
+ *                  is not written).  grad_v then includes d (.) grad_o.
+ *   grad_feedthrough : [H,d_v] float32, written with sum over b and t of
+ *                  grad_o (.) v when non-NULL (requires feedthrough non-NULL;
+ *                  accumulated with float32 atomics, so the summation order
+ *                  may differ between calls).
  * Gradients with respect to g are undefined where g = 0 (g^(tau-1) is
  * unbounded there); d/dtau uses alpha_hat * ln g = 0 where alpha_hat = 0.
  */
@@ -170,6 +187,8 @@ typedef struct {
     void *workspace;
     size_t workspace_bytes;
     rdm_gate_inputs gate_inputs;
+    const float *feedthrough;
+    float *grad_feedthrough;
 } rdm_bwd_args;
 
 rdm_status rdm_ddts_bwd(const rdm_bwd_args *args, rdm_stream_t stream);
@@ -218,6 +237,20 @@ rdm_status rdm_ddts_decode_step(int B, int H, int dk, int dv, rdm_dtype dtype,
                                 const void *q, const void *k, const void *v,
                                 const void *g, const void *tau, const void *beta,
                                 float *S, void *o, rdm_stream_t stream);
+
+/* The same decode step with the arguments in a struct and the feedthrough:
+ * o = S^T q + d (.) v when feedthrough ([H,d_v] float32) is non-NULL.
+ * rdm_ddts_decode_step is this call with feedthrough = NULL. */
+typedef struct {
+    int B, H, dk, dv;
+    rdm_dtype dtype;
+    const void *q, *k, *v, *g, *tau, *beta;
+    float *S;
+    void *o;
+    const float *feedthrough;
+} rdm_decode_args;
+
+rdm_status rdm_ddts_decode(const rdm_decode_args *args, rdm_stream_t stream);
 
 /* ------------------------------------------------------------------ status */
 

@@ -50,9 +50,9 @@ def load_library(path: str):
     lib = ctypes.CDLL(path)
     P = ctypes.POINTER(ctypes.c_double)
     I = ctypes.c_int
-    lib.rdm_oracle_fwd.argtypes = [I] * 5 + [P] * 9 + [I]
-    lib.rdm_oracle_bwd.argtypes = [I] * 5 + [P] * 16 + [I]
-    lib.rdm_oracle_decode_step.argtypes = [I] * 4 + [P] * 8 + [I]
+    lib.rdm_oracle_fwd.argtypes = [I] * 5 + [P] * 10 + [I]
+    lib.rdm_oracle_bwd.argtypes = [I] * 5 + [P] * 18 + [I]
+    lib.rdm_oracle_decode_step.argtypes = [I] * 4 + [P] * 9 + [I]
     for f in (lib.rdm_oracle_fwd, lib.rdm_oracle_bwd, lib.rdm_oracle_decode_step):
         f.restype = I
     return lib
@@ -104,11 +104,14 @@ def activate(g_pre, tau_pre, beta_pre):
     return softplus(g_pre), sigmoid(tau_pre), sigmoid(beta_pre)
 
 
-def fwd(q, k, v, g, tau, beta, S0=None, nthreads=None, lib=None, preact=False):
+def fwd(q, k, v, g, tau, beta, S0=None, nthreads=None, lib=None, preact=False, d=None):
     """Token-by-token forward.  q,k,g,tau [B,H,T,dk]; v,beta [B,H,T,dv];
     S0 [B,H,dk,dv] or None (zeros).  Returns (o [B,H,T,dv], S_T [B,H,dk,dv]).
-    preact: g, tau, beta are pre-activations (see the module docstring)."""
-    q, k, v, g, tau, beta, S0 = map(_f64, (q, k, v, g, tau, beta, S0))
+    preact: g, tau, beta are pre-activations (see the module docstring).
+    d: feedthrough weights [H,dv] or None; o_t += d (.) v_t (the feedthrough of
+    Eq. (11), paperhub.cn rebuttal answer to Q6; reading: one weight per head
+    and value channel, applied to v_t)."""
+    q, k, v, g, tau, beta, S0, d = map(_f64, (q, k, v, g, tau, beta, S0, d))
     if preact:
         g, tau, beta = activate(g, tau, beta)
     B, H, T, dk = q.shape
@@ -116,21 +119,22 @@ def fwd(q, k, v, g, tau, beta, S0=None, nthreads=None, lib=None, preact=False):
     o = np.zeros((B, H, T, dv))
     ST = np.zeros((B, H, dk, dv))
     rc = _load(lib).rdm_oracle_fwd(B, H, T, dk, dv, _p(q), _p(k), _p(v), _p(g), _p(tau), _p(beta),
-                                _p(S0), _p(o), _p(ST), nthreads or default_threads())
+                                _p(S0), _p(d), _p(o), _p(ST), nthreads or default_threads())
     if rc != 0:
         raise RuntimeError("rdm_oracle_fwd failed")
     return o, ST
 
 
-def bwd(q, k, v, g, tau, beta, S0, dO, dST=None, nthreads=None, lib=None, preact=False):
-    """Reverse mode of the token loop.  Returns dict dq, dk, dv, dg, dtau, dbeta, dS0.
+def bwd(q, k, v, g, tau, beta, S0, dO, dST=None, nthreads=None, lib=None, preact=False, d=None):
+    """Reverse mode of the token loop.  Returns dict dq, dk, dv, dg, dtau, dbeta, dS0
+    (and dd [H,dv], the feedthrough gradient summed over the batch, when d is given).
     preact: g, tau, beta are pre-activations and dg, dtau, dbeta are the gradients
     with respect to them (d softplus = sigmoid, d sigmoid = s (1 - s))."""
-    q, k, v, g, tau, beta, S0, dO, dST = map(_f64, (q, k, v, g, tau, beta, S0, dO, dST))
+    q, k, v, g, tau, beta, S0, dO, dST, d = map(_f64, (q, k, v, g, tau, beta, S0, dO, dST, d))
     if preact:
         g_pre = g
         g, tau, beta = activate(g, tau, beta)
-        out = bwd(q, k, v, g, tau, beta, S0, dO, dST, nthreads=nthreads, lib=lib)
+        out = bwd(q, k, v, g, tau, beta, S0, dO, dST, nthreads=nthreads, lib=lib, d=d)
         out["dg"] *= sigmoid(g_pre)
         out["dtau"] *= tau * (1.0 - tau)
         out["dbeta"] *= beta * (1.0 - beta)
@@ -140,26 +144,29 @@ def bwd(q, k, v, g, tau, beta, S0, dO, dST=None, nthreads=None, lib=None, preact
     out = {n: np.zeros(q.shape) for n in ("dq", "dk", "dg", "dtau")}
     out.update({n: np.zeros(v.shape) for n in ("dv", "dbeta")})
     out["dS0"] = np.zeros((B, H, dk, dv))
+    dd_pair = np.zeros((B, H, dv)) if d is not None else None
     rc = _load(lib).rdm_oracle_bwd(B, H, T, dk, dv, _p(q), _p(k), _p(v), _p(g), _p(tau), _p(beta),
-                                _p(S0), _p(dO), _p(dST), _p(out["dq"]), _p(out["dk"]),
+                                _p(S0), _p(dO), _p(dST), _p(d), _p(out["dq"]), _p(out["dk"]),
                                 _p(out["dv"]), _p(out["dg"]), _p(out["dtau"]), _p(out["dbeta"]),
-                                _p(out["dS0"]), nthreads or default_threads())
+                                _p(out["dS0"]), _p(dd_pair), nthreads or default_threads())
     if rc != 0:
         raise RuntimeError("rdm_oracle_bwd failed")
+    if d is not None:
+        out["dd"] = dd_pair.sum(axis=0)
     return out
 
 
-def decode_step(q, k, v, g, tau, beta, S, nthreads=None, lib=None):
+def decode_step(q, k, v, g, tau, beta, S, nthreads=None, lib=None, d=None):
     """One token per (b,h).  q,k,g,tau [B,H,dk]; v,beta [B,H,dv]; S [B,H,dk,dv]
-    float64 numpy, updated in place.  Returns o [B,H,dv]."""
+    float64 numpy, updated in place; d feedthrough [H,dv] or None.  Returns o [B,H,dv]."""
     if not (isinstance(S, np.ndarray) and S.dtype == np.float64 and S.flags.c_contiguous):
         raise TypeError("S must be a C-contiguous float64 numpy array (updated in place)")
-    q, k, v, g, tau, beta = map(_f64, (q, k, v, g, tau, beta))
+    q, k, v, g, tau, beta, d = map(_f64, (q, k, v, g, tau, beta, d))
     B, H, dk = q.shape
     dv = v.shape[-1]
     o = np.zeros((B, H, dv))
     rc = _load(lib).rdm_oracle_decode_step(B, H, dk, dv, _p(q), _p(k), _p(v), _p(g), _p(tau),
-                                        _p(beta), _p(S), _p(o), nthreads or default_threads())
+                                        _p(beta), _p(d), _p(S), _p(o), nthreads or default_threads())
     if rc != 0:
         raise RuntimeError("rdm_oracle_decode_step failed")
     return o

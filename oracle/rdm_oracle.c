@@ -20,6 +20,12 @@
  *     the state is a fixed d_k x d_v matrix carried across tokens (paperhub.cn
  *     rebuttal Q2 and Q5-3, Table 4 "State size n x m").
  *
+ * Feedthrough (optional): o_t += d (.) v_t with d one weight per head and value
+ *   channel, d[h][j]: the feedthrough d_t of the paper's Eq. (11), which the
+ *   paperhub.cn OpenReview rebuttal (answer to Q6) names the SSM feedthrough
+ *   as used in Mamba and Mamba2, a learned skip from the SSM input (here v_t)
+ *   to the output.  Its shape and input are not printed; this is the reading.
+ *
  * Backward: reverse-mode differentiation of exactly that loop, step by step
  * (no chunking, no cumulative-sum identities).  States S_{t-1} needed by the
  * reverse step are recomputed from checkpoints taken every CKPT tokens.
@@ -46,6 +52,8 @@ typedef struct {
     const double *q, *k, *v, *g, *tau, *beta, *S0, *dO, *dST;
     double *o, *ST;
     double *dq, *dk_, *dv_, *dg, *dtau, *dbeta, *dS0;
+    const double *dfeed;    /* feedthrough weights [H][dv], or NULL */
+    double *ddfeed;         /* per-(b,h) feedthrough gradient [B*H][dv], or NULL */
     int next;               /* next (b,h) pair to take */
     int failed;
     pthread_mutex_t lock;
@@ -75,6 +83,12 @@ static void step_token(int dk, int dv, const double *q, const double *k, const d
     }
 }
 
+/* Feedthrough of one token: o += d (.) v. */
+static void add_feedthrough(int dv, const double *d, const double *v, double *o)
+{
+    for (int j = 0; j < dv; ++j) o[j] += d[j] * v[j];
+}
+
 static int take_pair(job_t *J)
 {
     pthread_mutex_lock(&J->lock);
@@ -98,6 +112,8 @@ static void *fwd_worker(void *arg)
             size_t ok = sk + (size_t)t * dk, ov = sv + (size_t)t * dv;
             step_token(dk, dv, J->q + ok, J->k + ok, J->v + ov, J->g + ok, J->tau + ok,
                        J->beta + ov, S, J->o ? J->o + ov : NULL);
+            if (J->o && J->dfeed) add_feedthrough(dv, J->dfeed + (size_t)(p % J->H) * dv,
+                                                  J->v + ov, J->o + ov);
         }
         if (J->ST) memcpy(J->ST + ss, S, sizeof(double) * dk * dv);
     }
@@ -133,7 +149,7 @@ static int dims_ok(int B, int H, int T, int dk, int dv)
 int rdm_oracle_fwd(int B, int H, int T, int dk, int dv,
                    const double *q, const double *k, const double *v,
                    const double *g, const double *tau, const double *beta,
-                   const double *S0, double *o, double *ST, int nthreads)
+                   const double *S0, const double *dfeed, double *o, double *ST, int nthreads)
 {
     if (!dims_ok(B, H, T, dk, dv)) return -1;
     if (T > 0 && (!q || !k || !v || !g || !tau || !beta)) return -1;
@@ -141,7 +157,7 @@ int rdm_oracle_fwd(int B, int H, int T, int dk, int dv,
     memset(&J, 0, sizeof(J));
     J.B = B; J.H = H; J.T = T; J.dk = dk; J.dv = dv;
     J.q = q; J.k = k; J.v = v; J.g = g; J.tau = tau; J.beta = beta; J.S0 = S0;
-    J.o = o; J.ST = ST;
+    J.o = o; J.ST = ST; J.dfeed = dfeed;
     return run_pool(&J, fwd_worker, nthreads);
 }
 
@@ -154,6 +170,8 @@ static void *decode_worker(void *arg)
         size_t ok = (size_t)p * dk, ov = (size_t)p * dv;
         step_token(dk, dv, J->q + ok, J->k + ok, J->v + ov, J->g + ok, J->tau + ok,
                    J->beta + ov, J->ST + (size_t)p * dk * dv, J->o ? J->o + ov : NULL);
+        if (J->o && J->dfeed) add_feedthrough(dv, J->dfeed + (size_t)(p % J->H) * dv,
+                                              J->v + ov, J->o + ov);
     }
     return NULL;
 }
@@ -163,14 +181,14 @@ static void *decode_worker(void *arg)
 int rdm_oracle_decode_step(int B, int H, int dk, int dv,
                            const double *q, const double *k, const double *v,
                            const double *g, const double *tau, const double *beta,
-                           double *S, double *o, int nthreads)
+                           const double *dfeed, double *S, double *o, int nthreads)
 {
     if (!dims_ok(B, H, 1, dk, dv) || !S || !q || !k || !v || !g || !tau || !beta) return -1;
     job_t J;
     memset(&J, 0, sizeof(J));
     J.B = B; J.H = H; J.T = 1; J.dk = dk; J.dv = dv;
     J.q = q; J.k = k; J.v = v; J.g = g; J.tau = tau; J.beta = beta;
-    J.ST = S; J.o = o;
+    J.ST = S; J.o = o; J.dfeed = dfeed;
     return run_pool(&J, decode_worker, nthreads);
 }
 
@@ -271,6 +289,14 @@ static void *bwd_worker(void *arg)
                     J->dv_[ov + j] = beta[j] * dvh[j];
                     J->dbeta[ov + j] = v[j] * dvh[j];
                 }
+                /* feedthrough o_t += d (.) v_t */
+                if (J->dfeed) {
+                    const double *d = J->dfeed + (size_t)(p % J->H) * dv;
+                    for (int j = 0; j < dv; ++j) {
+                        J->dv_[ov + j] += d[j] * dO[j];
+                        if (J->ddfeed) J->ddfeed[(size_t)p * dv + j] += dO[j] * v[j];
+                    }
+                }
             }
         }
         if (J->dS0) memcpy(J->dS0 + ss, dS, sizeof(double) * SS);
@@ -285,8 +311,9 @@ int rdm_oracle_bwd(int B, int H, int T, int dk, int dv,
                    const double *q, const double *k, const double *v,
                    const double *g, const double *tau, const double *beta,
                    const double *S0, const double *dO, const double *dST,
+                   const double *dfeed,
                    double *dq, double *dk_, double *dv_, double *dg, double *dtau,
-                   double *dbeta, double *dS0, int nthreads)
+                   double *dbeta, double *dS0, double *ddfeed, int nthreads)
 {
     if (!dims_ok(B, H, T, dk, dv)) return -1;
     if (T > 0 && (!q || !k || !v || !g || !tau || !beta || !dO || !dq || !dk_ || !dv_ ||
@@ -298,5 +325,6 @@ int rdm_oracle_bwd(int B, int H, int T, int dk, int dv,
     J.q = q; J.k = k; J.v = v; J.g = g; J.tau = tau; J.beta = beta; J.S0 = S0;
     J.dO = dO; J.dST = dST;
     J.dq = dq; J.dk_ = dk_; J.dv_ = dv_; J.dg = dg; J.dtau = dtau; J.dbeta = dbeta; J.dS0 = dS0;
+    J.dfeed = dfeed; J.ddfeed = ddfeed;
     return run_pool(&J, bwd_worker, nthreads);
 }

@@ -306,7 +306,90 @@ def check_preact_bwd_finite_differences(lib=None, seed=11):
 PREACT_PINS = [check_preact_matches_torch_activations, check_preact_special_values,
                check_preact_bwd_finite_differences]
 
+
+# ------------------------------------------ feedthrough o_t += d (.) v_t (Eq. (11)'s d_t)
+def check_feedthrough_dead_state(lib=None, seed=12):
+    """k = 0 and S_0 = 0 keep the state at zero, so o_t = d (.) v_t exactly (per
+    head: d is [H, d_v], broadcast over batch and time)."""
+    rng = np.random.default_rng(seed)
+    x = rand_inputs(rng, 2, 3, 7, 4, 5)
+    x["k"][:] = 0.0
+    x["S0"][:] = 0.0
+    d = rng.standard_normal((3, 5))
+    o, ST = oracle.fwd(**x, d=d, lib=lib)
+    close(o, d[None, :, None, :] * x["v"], 0.0, "dead state: o = d v")
+    close(ST, np.zeros_like(ST), 0.0, "dead state: S_T")
+
+
+def check_feedthrough_linearity(lib=None, seed=13):
+    """o(d) - o(0) = d (.) v_t and S_T does not depend on d; the decode step
+    agrees with the forward token by token."""
+    rng = np.random.default_rng(seed)
+    x = rand_inputs(rng, 2, 2, 9, 3, 4)
+    d = rng.standard_normal((2, 4))
+    o1, S1 = oracle.fwd(**x, d=d, lib=lib)
+    o0, S0 = oracle.fwd(**x, lib=lib)
+    close(o1 - o0, d[None, :, None, :] * x["v"], 1e-13, "o(d) - o(0)")
+    close(S1, S0, 0.0, "S_T independent of d")
+    S = np.ascontiguousarray(x["S0"].copy())
+    seq = ("q", "k", "v", "g", "tau", "beta")
+    for t in range(x["q"].shape[2]):
+        ot = oracle.decode_step(*(x[n][:, :, t] for n in seq), S, d=d, lib=lib)
+        close(ot, o1[:, :, t], 1e-13, f"decode with d, step {t}")
+
+
+def check_feedthrough_bwd(lib=None, seed=14):
+    """Reverse mode with the feedthrough: central differences of L = <o, dO> +
+    <S_T, dS_T> for v and for d itself (d summed over the batch), and
+    torch.autograd through the naive loop."""
+    import torch
+    rng = np.random.default_rng(seed)
+    B, H, T, dk, dv = 2, 2, 5, 3, 2
+    x = rand_inputs(rng, B, H, T, dk, dv, g_lo=0.1, g_hi=2.0)
+    d = rng.standard_normal((H, dv))
+    dO = rng.standard_normal((B, H, T, dv))
+    dST = rng.standard_normal((B, H, dk, dv))
+    gr = oracle.bwd(**x, dO=dO, dST=dST, d=d, lib=lib)
+
+    def loss(xx, dd):
+        o, ST = oracle.fwd(**xx, d=dd, lib=lib)
+        return float(np.sum(o * dO) + np.sum(ST * dST))
+
+    h = 1e-6
+    num_d = np.zeros_like(d)
+    for idx in np.ndindex(d.shape):
+        dp, dm = d.copy(), d.copy()
+        dp[idx] += h
+        dm[idx] -= h
+        num_d[idx] = (loss(x, dp) - loss(x, dm)) / (2 * h)
+    close(gr["dd"], num_d, 2e-7, "finite differences dd")
+    num_v = np.zeros_like(x["v"])
+    for idx in np.ndindex(x["v"].shape):
+        xp = {m: a.copy() for m, a in x.items()}
+        xp["v"][idx] += h
+        lp = loss(xp, d)
+        xp["v"][idx] -= 2 * h
+        num_v[idx] = (lp - loss(xp, d)) / (2 * h)
+    close(gr["dv"], num_v, 2e-7, "finite differences dv with feedthrough")
+    t = {n: torch.tensor(a, dtype=torch.float64, requires_grad=True) for n, a in x.items()}
+    td = torch.tensor(d, dtype=torch.float64, requires_grad=True)
+    S = t["S0"]
+    outs = []
+    for s in range(T):
+        al = torch.exp(-t["g"][:, :, s] * t["tau"][:, :, s])
+        kh = torch.pow(t["g"][:, :, s], t["tau"][:, :, s]) * t["k"][:, :, s]
+        S = al[..., :, None] * S + kh[..., :, None] * (t["beta"][:, :, s] * t["v"][:, :, s])[..., None, :]
+        outs.append((S * t["q"][:, :, s][..., :, None]).sum(-2) + td[None] * t["v"][:, :, s])
+    L = (torch.stack(outs, 2) * torch.tensor(dO)).sum() + (S * torch.tensor(dST)).sum()
+    L.backward()
+    close(gr["dd"], td.grad.numpy(), 1e-11, "autograd dd")
+    for n, gn in dict(q="dq", k="dk", v="dv", g="dg", tau="dtau", beta="dbeta", S0="dS0").items():
+        close(gr[gn], t[n].grad.numpy(), 1e-11, f"autograd with feedthrough {gn}")
+
+
+FEED_PINS = [check_feedthrough_dead_state, check_feedthrough_linearity, check_feedthrough_bwd]
+
 FORWARD_PINS = [check_worked_example, check_T1_closed_form, check_g_zero, check_tau_zero,
                 check_quadratic, check_linearity, check_split_and_decode]
 BACKWARD_PINS = [check_bwd_finite_differences, check_bwd_autograd]
-ALL_PINS = FORWARD_PINS + BACKWARD_PINS + PREACT_PINS
+ALL_PINS = FORWARD_PINS + BACKWARD_PINS + PREACT_PINS + FEED_PINS

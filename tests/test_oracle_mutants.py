@@ -45,6 +45,16 @@ MUTANTS = [
      "J->dv_[ov + j] = v[j] * dvh[j];", P.BACKWARD_PINS),
     ("bwd upstream dS_T ignored", "if (J->dST) memcpy(dS, J->dST + ss, sizeof(double) * SS);",
      "if (0) memcpy(dS, J->dST + ss, sizeof(double) * SS);", P.BACKWARD_PINS),
+    ("feedthrough on the gated input", "for (int j = 0; j < dv; ++j) o[j] += d[j] * v[j];",
+     "for (int j = 0; j < dv; ++j) o[j] += d[j] * v[j] * 0.5;", P.FEED_PINS),
+    ("feedthrough weight of another head",
+     "J->dfeed + (size_t)(p % J->H) * dv,\n                                                  J->v + ov",
+     "J->dfeed + (size_t)((p + 1) % J->H) * dv,\n                                                  J->v + ov",
+     P.FEED_PINS),
+    ("bwd feedthrough dv dropped", "J->dv_[ov + j] += d[j] * dO[j];", "J->dv_[ov + j] += 0.0;",
+     P.FEED_PINS),
+    ("bwd feedthrough dd with vhat", "J->ddfeed[(size_t)p * dv + j] += dO[j] * v[j];",
+     "J->ddfeed[(size_t)p * dv + j] += dO[j] * v[j] * beta[j];", P.FEED_PINS),
 ]
 
 
