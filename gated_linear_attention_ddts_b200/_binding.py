@@ -52,6 +52,17 @@ class DecodeArgs(ctypes.Structure):
                 ("S", _VP), ("o", _VP), ("feedthrough", _VP)]
 
 
+class ConvArgs(ctypes.Structure):
+    _fields_ = [("B", _I), ("H", _I), ("T", _I), ("D", _I), ("W", _I), ("dtype", _I), ("silu", _I),
+                ("x", _VP), ("weight", _VP), ("bias", _VP), ("state_in", _VP), ("y", _VP),
+                ("state_out", _VP)]
+
+
+class ConvBwdArgs(ctypes.Structure):
+    _fields_ = [("fwd", ConvArgs), ("grad_y", _VP), ("grad_state_out", _VP), ("grad_x", _VP),
+                ("grad_weight", _VP), ("grad_bias", _VP), ("grad_state_in", _VP)]
+
+
 class RdmError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
@@ -63,7 +74,8 @@ _lib = None
 EXPORTS = ["rdm_ddts_fwd", "rdm_ddts_fwd_workspace_size", "rdm_ddts_saved_states_size", "rdm_ddts_bwd",
            "rdm_ddts_bwd_workspace_size", "rdm_ddts_bwd_noalloc", "rdm_ddts_decode_step", "rdm_ddts_decode",
            "rdm_ddts_sync_status",
-           "rdm_status_string", "rdm_ddts_set_test_hooks", "rdm_ddts_version"]
+           "rdm_status_string", "rdm_ddts_set_test_hooks", "rdm_ddts_version", "rdm_shortconv_fwd",
+           "rdm_shortconv_bwd"]
 
 
 def load():
@@ -94,6 +106,10 @@ def load():
         lib.rdm_ddts_sync_status.restype = _I
         lib.rdm_status_string.argtypes = [_I]
         lib.rdm_status_string.restype = ctypes.c_char_p
+        lib.rdm_shortconv_fwd.argtypes = [ctypes.POINTER(ConvArgs), _VP]
+        lib.rdm_shortconv_fwd.restype = _I
+        lib.rdm_shortconv_bwd.argtypes = [ctypes.POINTER(ConvBwdArgs), _VP]
+        lib.rdm_shortconv_bwd.restype = _I
         lib.rdm_ddts_set_test_hooks.argtypes = [ctypes.c_longlong, _I]
         lib.rdm_ddts_set_test_hooks.restype = _I
         lib.rdm_ddts_version.argtypes = []
@@ -277,6 +293,43 @@ def rdm_ddts_decode(q, k, v, g, tau, beta, S, o=None, *, feedthrough=None, strea
                    _ptr(beta), _ptr(S), _ptr(o), _ptr(feedthrough))
     _check(load().rdm_ddts_decode(ctypes.byref(a), _stream(stream)), "rdm_ddts_decode")
     return o
+
+
+def _conv_args(x, weight, bias, state_in, y, state_out, silu):
+    B, H, T, D = x.shape
+    return ConvArgs(B, H, T, D, weight.shape[-1], _dtype_code(x), int(bool(silu)), _ptr(x),
+                    _ptr(weight), _ptr(bias), _ptr(state_in), _ptr(y), _ptr(state_out))
+
+
+def rdm_shortconv_fwd(x, weight, bias=None, state_in=None, *, silu=False, y=None,
+                      return_state=False, stream=None):
+    """Causal depthwise short convolution along the tokens: x [B,H,T,D], weight
+    [H,D,W] float32, bias [H,D] float32, state_in [B,H,W-1,D] (the previous
+    W-1 inputs).  Returns (y, state_out or None)."""
+    B, H, T, D = x.shape
+    W = weight.shape[-1]
+    if y is None:
+        y = torch.empty_like(x)
+    state_out = torch.empty(B, H, W - 1, D, dtype=x.dtype, device=x.device) if return_state else None
+    a = _conv_args(x, weight, bias, state_in, y, state_out, silu)
+    _check(load().rdm_shortconv_fwd(ctypes.byref(a), _stream(stream)), "rdm_shortconv_fwd")
+    return y, state_out
+
+
+def rdm_shortconv_bwd(x, weight, bias, state_in, grad_y, grad_state_out=None, *, silu=False,
+                      stream=None):
+    """Reverse mode of rdm_shortconv_fwd.  Returns dict dx, dw, dbias (None
+    without bias) and dxs (None without state_in)."""
+    B, H, T, D = x.shape
+    W = weight.shape[-1]
+    out = dict(dx=torch.empty_like(x), dw=torch.empty_like(weight),
+               dbias=torch.empty_like(bias) if bias is not None else None,
+               dxs=torch.empty_like(state_in) if state_in is not None else None)
+    a = ConvBwdArgs(_conv_args(x, weight, bias, state_in, None, None, silu), _ptr(grad_y),
+                    _ptr(grad_state_out), _ptr(out["dx"]), _ptr(out["dw"]), _ptr(out["dbias"]),
+                    _ptr(out["dxs"]))
+    _check(load().rdm_shortconv_bwd(ctypes.byref(a), _stream(stream)), "rdm_shortconv_bwd")
+    return out
 
 
 def rdm_ddts_sync_status(stream=None) -> int:

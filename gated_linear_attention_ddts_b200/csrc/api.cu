@@ -243,6 +243,58 @@ rdm_status rdm_ddts_decode_step(int B, int H, int dk, int dv, rdm_dtype dtype, c
     return rdm_ddts_decode(&a, stream);
 }
 
+static rdm_status conv_check(const rdm_shortconv_args* a) {
+    if (!a || a->B < 1 || a->H < 1 || a->T < 0 || a->W < 1) return RDM_ERR_INVALID_ARG;
+    if (a->dtype != RDM_F32 && a->dtype != RDM_BF16) return RDM_ERR_INVALID_ARG;
+    if (!(a->D == 16 || a->D == 32 || a->D == 64 || a->D == 128) || a->W > 4) return RDM_ERR_UNSUPPORTED;
+    if ((double)a->B * a->H * (double)(a->T > 0 ? a->T : 1) * a->D > 4.0e18 || (double)a->B * a->H > 2.0e9)
+        return RDM_ERR_INVALID_ARG;
+    if (!a->weight || !aligned(a->weight) || !opt_aligned(a->bias) || !opt_aligned(a->state_in))
+        return RDM_ERR_INVALID_ARG;
+    if (a->T > 0 && (!a->x || !aligned(a->x))) return RDM_ERR_INVALID_ARG;
+    return RDM_OK;
+}
+
+static ConvParams conv_params(const rdm_shortconv_args* a) {
+    ConvParams p;
+    memset(&p, 0, sizeof(p));
+    p.B = a->B; p.H = a->H; p.T = a->T; p.D = a->D; p.W = a->W;
+    p.bf16 = a->dtype == RDM_BF16;
+    p.silu = a->silu != 0;
+    p.x = a->x; p.w = a->weight; p.bias = a->bias; p.xs = a->state_in;
+    p.y = a->y; p.xs_out = a->W > 1 ? a->state_out : nullptr;
+    return p;
+}
+
+rdm_status rdm_shortconv_fwd(const rdm_shortconv_args* a, rdm_stream_t stream) {
+    rdm_status st = conv_check(a);
+    if (st != RDM_OK) return st;
+    if (a->T > 0 && (!a->y || !aligned(a->y))) return RDM_ERR_INVALID_ARG;
+    if (!opt_aligned(a->state_out)) return RDM_ERR_INVALID_ARG;
+    return from_cuda(launch_conv_fwd(conv_params(a), reinterpret_cast<cudaStream_t>(stream)));
+}
+
+rdm_status rdm_shortconv_bwd(const rdm_shortconv_bwd_args* a, rdm_stream_t stream) {
+    if (!a) return RDM_ERR_INVALID_ARG;
+    rdm_status st = conv_check(&a->fwd);
+    if (st != RDM_OK) return st;
+    if (!a->grad_weight || !aligned(a->grad_weight) || !opt_aligned(a->grad_bias) ||
+        !opt_aligned(a->grad_state_in) || !opt_aligned(a->grad_state_out))
+        return RDM_ERR_INVALID_ARG;
+    if (a->fwd.T > 0 && (!a->grad_y || !aligned(a->grad_y) || !a->grad_x || !aligned(a->grad_x)))
+        return RDM_ERR_INVALID_ARG;
+    ConvParams p = conv_params(&a->fwd);
+    p.y = nullptr;
+    p.xs_out = nullptr;
+    p.dy = a->grad_y;
+    p.dxs_out = a->fwd.W > 1 ? a->grad_state_out : nullptr;
+    p.dx = a->grad_x;
+    p.dw = a->grad_weight;
+    p.dbias = a->fwd.bias ? a->grad_bias : nullptr;
+    p.dxs = (a->fwd.state_in && a->fwd.W > 1) ? a->grad_state_in : nullptr;
+    return from_cuda(launch_conv_bwd(p, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 rdm_status rdm_ddts_sync_status(rdm_stream_t stream) {
     cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return RDM_ERR_CUDA;
@@ -279,6 +331,6 @@ rdm_status rdm_ddts_set_test_hooks(long long wait_limit_cycles, int withhold_seg
     return RDM_OK;
 }
 
-int rdm_ddts_version(void) { return 500; }
+int rdm_ddts_version(void) { return 600; }
 
 }  // extern "C"

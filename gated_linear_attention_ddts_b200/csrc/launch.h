@@ -66,6 +66,27 @@ cudaError_t launch_simt_bwd_flagged(const BwdParams& p, const int* flags, cudaSt
 // decode step
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s);
 
+// ShortConv: causal depthwise convolution along the tokens (shortconv.cu)
+struct ConvParams {
+    int B, H, T, D, W;
+    int bf16;   // element type of x, y, states and their gradients
+    int silu;   // y = z * sigmoid(z) instead of y = z
+    const void* x;       // [B,H,T,D]
+    const float* w;      // [H,D,W]
+    const float* bias;   // [H,D] or null
+    const void* xs;      // carried-in state [B,H,W-1,D] or null (zeros)
+    void* y;             // [B,H,T,D]
+    void* xs_out;        // carried-out state [B,H,W-1,D] or null
+    const void* dy;      // backward: dL/dy
+    const void* dxs_out; // dL/d(carried-out state) or null
+    void* dx;            // dL/dx
+    float* dw;           // dL/dw [H,D,W]
+    float* dbias;        // dL/dbias [H,D] or null
+    void* dxs;           // dL/d(carried-in state) or null
+};
+cudaError_t launch_conv_fwd(const ConvParams& p, cudaStream_t s);
+cudaError_t launch_conv_bwd(const ConvParams& p, cudaStream_t s);
+
 // gradient of the feedthrough weights: grad_d[h][j] = sum_{b,t} dO[b,h,t,j] v[b,h,t,j]
 // (zeroes grad_d, then accumulates; float32 atomics)
 cudaError_t launch_feed_grad(const BwdParams& p, cudaStream_t s);

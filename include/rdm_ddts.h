@@ -252,6 +252,62 @@ typedef struct {
 
 rdm_status rdm_ddts_decode(const rdm_decode_args *args, rdm_stream_t stream);
 
+/* -------------------------------------------------------------- ShortConv
+ * The short convolution of the Rodimus block (Rodimus* digest.lyk-ai.com
+ * summary, "Method", third Rodimus bullet: ShortConv next to the GLU for local
+ * context aggregation).  The pages print neither its width, its activation nor
+ * where it sits; this library takes a causal depthwise convolution along the
+ * tokens with one filter of width W <= 4 per (head, channel), an optional bias
+ * and an optional SiLU, on sequences in the layout of the recurrence's inputs:
+ *
+ *   z[b,h,t,c] = bias[h,c] + sum_{i=0}^{W-1} w[h,c,i] * x[b,h,t-i,c]
+ *   y = z   or   y = z * sigmoid(z)  (silu = 1)
+ *
+ * x at t - i < 0 comes from the carried-in state (the W-1 inputs before the
+ * sequence, oldest first), or is zero without one; the state after the
+ * sequence (its last W-1 inputs) can be written out, so sequences can be cut
+ * into pieces and decoded token by token with T = 1.
+ *
+ *   x, y        : [B,H,T,D] dtype        D in {16, 32, 64, 128}; W in {1,2,3,4}
+ *   weight      : [H,D,W] float32        bias : [H,D] float32 or NULL
+ *   state_in    : [B,H,W-1,D] dtype or NULL (zeros)
+ *   state_out   : [B,H,W-1,D] dtype or NULL (not written); must not alias x,
+ *                 y or state_in
+ * All pointers are device pointers, 16-byte aligned; nothing is allocated.
+ */
+typedef struct {
+    int B, H, T, D, W;
+    rdm_dtype dtype;
+    int silu;
+    const void *x;
+    const float *weight;
+    const float *bias;
+    const void *state_in;
+    void *y;
+    void *state_out;
+} rdm_shortconv_args;
+
+rdm_status rdm_shortconv_fwd(const rdm_shortconv_args *args, rdm_stream_t stream);
+
+/* Reverse mode of rdm_shortconv_fwd for dL/dy = grad_y and dL/d(state_out) =
+ * grad_state_out (NULL = zero).  Writes grad_x [B,H,T,D] dtype, grad_weight
+ * [H,D,W] float32, grad_bias [H,D] float32 (when bias and grad_bias are
+ * non-NULL) and grad_state_in [B,H,W-1,D] dtype (when state_in and
+ * grad_state_in are non-NULL).  The weight and bias gradients are sums over
+ * batch and tokens accumulated with float32 atomics (summation order may vary
+ * between calls). */
+typedef struct {
+    rdm_shortconv_args fwd;      /* the forward's arguments (y, state_out unused) */
+    const void *grad_y;
+    const void *grad_state_out;
+    void *grad_x;
+    float *grad_weight;
+    float *grad_bias;
+    void *grad_state_in;
+} rdm_shortconv_bwd_args;
+
+rdm_status rdm_shortconv_bwd(const rdm_shortconv_bwd_args *args, rdm_stream_t stream);
+
 /* ------------------------------------------------------------------ status */
 
 /* Synchronises `stream`, then reports (and clears) the device status word of

@@ -53,7 +53,10 @@ def load_library(path: str):
     lib.rdm_oracle_fwd.argtypes = [I] * 5 + [P] * 10 + [I]
     lib.rdm_oracle_bwd.argtypes = [I] * 5 + [P] * 18 + [I]
     lib.rdm_oracle_decode_step.argtypes = [I] * 4 + [P] * 9 + [I]
-    for f in (lib.rdm_oracle_fwd, lib.rdm_oracle_bwd, lib.rdm_oracle_decode_step):
+    lib.rdm_oracle_shortconv_fwd.argtypes = [I] * 5 + [P] * 4 + [I] + [P] * 2
+    lib.rdm_oracle_shortconv_bwd.argtypes = [I] * 5 + [P] * 4 + [I] + [P] * 6
+    for f in (lib.rdm_oracle_fwd, lib.rdm_oracle_bwd, lib.rdm_oracle_decode_step,
+              lib.rdm_oracle_shortconv_fwd, lib.rdm_oracle_shortconv_bwd):
         f.restype = I
     return lib
 
@@ -170,3 +173,40 @@ def decode_step(q, k, v, g, tau, beta, S, nthreads=None, lib=None, d=None):
     if rc != 0:
         raise RuntimeError("rdm_oracle_decode_step failed")
     return o
+
+
+def shortconv_fwd(x, w, bias=None, xs=None, silu=False, lib=None):
+    """Causal depthwise short convolution along the tokens (the ShortConv of the
+    Rodimus block; digest.lyk-ai.com summary, "Method"; width, activation and
+    carried state are this library's reading):
+        z[b,h,t,c] = bias[h,c] + sum_i w[h,c,i] x[b,h,t-i,c],   y = z or z*sigmoid(z)
+    x [B,H,T,D]; w [H,D,W]; bias [H,D] or None; xs [B,H,W-1,D] the previous W-1
+    inputs (oldest first) or None for zeros.  Returns (y [B,H,T,D], state after
+    the sequence [B,H,W-1,D])."""
+    x, w, bias, xs = map(_f64, (x, w, bias, xs))
+    B, H, T, D = x.shape
+    W = w.shape[-1]
+    y = np.zeros((B, H, T, D))
+    xs_out = np.zeros((B, H, W - 1, D))
+    rc = _load(lib).rdm_oracle_shortconv_fwd(B, H, T, D, W, _p(x), _p(w), _p(bias), _p(xs),
+                                             int(bool(silu)), _p(y), _p(xs_out))
+    if rc != 0:
+        raise RuntimeError("rdm_oracle_shortconv_fwd failed")
+    return y, xs_out
+
+
+def shortconv_bwd(x, w, bias, xs, dy, dxs_out=None, silu=False, lib=None):
+    """Reverse mode of shortconv_fwd.  Returns dict dx, dw, dbias (None without
+    bias) and dxs (None without a carried-in state)."""
+    x, w, bias, xs, dy, dxs_out = map(_f64, (x, w, bias, xs, dy, dxs_out))
+    B, H, T, D = x.shape
+    W = w.shape[-1]
+    out = dict(dx=np.zeros((B, H, T, D)), dw=np.zeros((H, D, W)),
+               dbias=np.zeros((H, D)) if bias is not None else None,
+               dxs=np.zeros((B, H, W - 1, D)) if xs is not None else None)
+    rc = _load(lib).rdm_oracle_shortconv_bwd(B, H, T, D, W, _p(x), _p(w), _p(bias), _p(xs),
+                                             int(bool(silu)), _p(dy), _p(dxs_out), _p(out["dx"]),
+                                             _p(out["dw"]), _p(out["dbias"]), _p(out["dxs"]))
+    if rc != 0:
+        raise RuntimeError("rdm_oracle_shortconv_bwd failed")
+    return out

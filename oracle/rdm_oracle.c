@@ -328,3 +328,98 @@ int rdm_oracle_bwd(int B, int H, int T, int dk, int dv,
     J.dfeed = dfeed; J.ddfeed = ddfeed;
     return run_pool(&J, bwd_worker, nthreads);
 }
+
+/* ------------------------------------------------------------- short conv
+ * ShortConv of the Rodimus block (digest.lyk-ai.com summary, "Method", third
+ * Rodimus bullet: a short convolution for local context next to the GLU).  The
+ * pages print neither its width, placement nor activation; the reading taken
+ * is a causal depthwise convolution along the tokens, one filter of width W per
+ * (head, channel):
+ *     z[b,h,t,c] = bias[h,c] + sum_{i=0}^{W-1} w[h,c,i] * x[b,h,t-i,c]
+ *     y = z, or y = z * sigmoid(z) (SiLU) when silu != 0
+ * with x at t - i < 0 taken from the carried-in state xs[b,h,W-1+(t-i),c] (the
+ * previous W-1 tokens, oldest first; zeros when xs is NULL).  The state after
+ * the sequence (its last W-1 inputs, including carried-in ones when T < W-1)
+ * is written to xs_out when non-NULL.  Layouts: x, y [B,H,T,D]; w [H,D,W];
+ * bias [H,D] or NULL; xs, xs_out [B,H,W-1,D]. */
+static double conv_input(const double *x, const double *xs, int T, int D, int W, int t, int c)
+{
+    if (t >= 0) return t < T ? x[(size_t)t * D + c] : 0.0;
+    int s = W - 1 + t;            /* position in the carried-in state */
+    return (xs && s >= 0) ? xs[(size_t)s * D + c] : 0.0;
+}
+
+int rdm_oracle_shortconv_fwd(int B, int H, int T, int D, int W, const double *x,
+                             const double *w, const double *bias, const double *xs,
+                             int silu, double *y, double *xs_out)
+{
+    if (B < 0 || H < 0 || T < 0 || D < 1 || W < 1 || !w) return -1;
+    for (int p = 0; p < B * H; ++p) {
+        const int h = p % H;
+        const double *xp = x + (size_t)p * T * D;
+        const double *sp = xs ? xs + (size_t)p * (W - 1) * D : NULL;
+        for (int t = 0; t < T; ++t)
+            for (int c = 0; c < D; ++c) {
+                double z = bias ? bias[(size_t)h * D + c] : 0.0;
+                for (int i = 0; i < W; ++i)
+                    z += w[((size_t)h * D + c) * W + i] * conv_input(xp, sp, T, D, W, t - i, c);
+                y[((size_t)p * T + t) * D + c] = silu ? z / (1.0 + exp(-z)) : z;
+            }
+        if (xs_out)
+            for (int s = 0; s < W - 1; ++s)
+                for (int c = 0; c < D; ++c)
+                    xs_out[((size_t)p * (W - 1) + s) * D + c] =
+                        conv_input(xp, sp, T, D, W, T - (W - 1) + s, c);
+    }
+    return 0;
+}
+
+/* Reverse mode of rdm_oracle_shortconv_fwd for the loss with dL/dy = dy (and
+ * dL/dxs_out = dxs_out when non-NULL): dx [B,H,T,D], dw [H,D,W], dbias [H,D]
+ * (NULL = skip), dxs [B,H,W-1,D] (NULL = skip).  Written by direct
+ * differentiation of the loops above: z is recomputed per output. */
+int rdm_oracle_shortconv_bwd(int B, int H, int T, int D, int W, const double *x,
+                             const double *w, const double *bias, const double *xs, int silu,
+                             const double *dy, const double *dxs_out, double *dx, double *dw,
+                             double *dbias, double *dxs)
+{
+    if (B < 0 || H < 0 || T < 0 || D < 1 || W < 1 || !w || !dx || !dw) return -1;
+    memset(dx, 0, sizeof(double) * (size_t)B * H * T * D);
+    memset(dw, 0, sizeof(double) * (size_t)H * D * W);
+    if (dbias) memset(dbias, 0, sizeof(double) * (size_t)H * D);
+    if (dxs) memset(dxs, 0, sizeof(double) * (size_t)B * H * (W - 1) * D);
+    for (int p = 0; p < B * H; ++p) {
+        const int h = p % H;
+        const double *xp = x + (size_t)p * T * D;
+        const double *sp = xs ? xs + (size_t)p * (W - 1) * D : NULL;
+        /* the carried-out state is a copy of inputs: route its gradient back */
+        if (dxs_out)
+            for (int s = 0; s < W - 1; ++s)
+                for (int c = 0; c < D; ++c) {
+                    const double gsv = dxs_out[((size_t)p * (W - 1) + s) * D + c];
+                    const int t = T - (W - 1) + s;
+                    if (t >= 0) dx[((size_t)p * T + t) * D + c] += gsv;
+                    else if (dxs && W - 1 + t >= 0) dxs[((size_t)p * (W - 1) + W - 1 + t) * D + c] += gsv;
+                }
+        for (int t = 0; t < T; ++t)
+            for (int c = 0; c < D; ++c) {
+                double z = bias ? bias[(size_t)h * D + c] : 0.0;
+                for (int i = 0; i < W; ++i)
+                    z += w[((size_t)h * D + c) * W + i] * conv_input(xp, sp, T, D, W, t - i, c);
+                double gz = dy[((size_t)p * T + t) * D + c];
+                if (silu) {
+                    const double s = 1.0 / (1.0 + exp(-z));
+                    gz *= s * (1.0 + z * (1.0 - s));
+                }
+                if (dbias) dbias[(size_t)h * D + c] += gz;
+                for (int i = 0; i < W; ++i) {
+                    const int ti = t - i;
+                    dw[((size_t)h * D + c) * W + i] += gz * conv_input(xp, sp, T, D, W, ti, c);
+                    const double gx = gz * w[((size_t)h * D + c) * W + i];
+                    if (ti >= 0) dx[((size_t)p * T + ti) * D + c] += gx;
+                    else if (dxs && W - 1 + ti >= 0) dxs[((size_t)p * (W - 1) + W - 1 + ti) * D + c] += gx;
+                }
+            }
+    }
+    return 0;
+}

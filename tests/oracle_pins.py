@@ -389,7 +389,107 @@ def check_feedthrough_bwd(lib=None, seed=14):
 
 FEED_PINS = [check_feedthrough_dead_state, check_feedthrough_linearity, check_feedthrough_bwd]
 
+
+# ------------------------------------------------ ShortConv (causal depthwise convolution)
+def conv_inputs(rng, B=2, H=3, T=11, D=5, W=4):
+    return dict(x=rng.standard_normal((B, H, T, D)), w=rng.standard_normal((H, D, W)),
+                bias=rng.standard_normal((H, D)), xs=rng.standard_normal((B, H, W - 1, D)))
+
+
+def check_conv_width_one(lib=None, seed=20):
+    """W = 1: y = w (.) x + bias, element-wise; the carried state is empty."""
+    rng = np.random.default_rng(seed)
+    c = conv_inputs(rng, W=1)
+    y, xs_out = oracle.shortconv_fwd(c["x"], c["w"], c["bias"], None, lib=lib)
+    close(y, c["w"][None, :, None, :, 0] * c["x"] + c["bias"][None, :, None, :], 1e-14, "W=1")
+    assert xs_out.shape == (2, 3, 0, 5)
+
+
+def check_conv_numpy_convolve(lib=None, seed=21):
+    """Every channel of every head equals numpy.convolve (full mode, first T
+    outputs) of that channel's sequence with its filter (zero carried state)."""
+    rng = np.random.default_rng(seed)
+    for W in (2, 3, 4):
+        c = conv_inputs(rng, W=W)
+        y, _ = oracle.shortconv_fwd(c["x"], c["w"], None, None, lib=lib)
+        ref = np.zeros_like(y)
+        B, H, T, D = y.shape
+        for b, h, ch in np.ndindex(B, H, D):
+            ref[b, h, :, ch] = np.convolve(c["x"][b, h, :, ch], c["w"][h, ch])[:T]
+        close(y, ref, 1e-13, f"numpy.convolve W={W}")
+
+
+def check_conv_impulse_and_state(lib=None, seed=22):
+    """An impulse at token t0 returns the filter at t0..t0+W-1 (causality: nothing
+    before t0); a sequence cut in two with the state carried across equals the
+    whole sequence, outputs and final state."""
+    rng = np.random.default_rng(seed)
+    c = conv_inputs(rng, T=12, W=4)
+    x = np.zeros_like(c["x"])
+    x[:, :, 5, :] = 1.0
+    y, _ = oracle.shortconv_fwd(x, c["w"], None, None, lib=lib)
+    assert np.all(y[:, :, :5] == 0.0) and np.all(y[:, :, 9:] == 0.0)
+    close(y[:, :, 5:9], np.broadcast_to(np.moveaxis(c["w"], -1, 1)[None], y[:, :, 5:9].shape),
+          0.0, "impulse response")
+    for silu in (False, True):
+        yw, sw = oracle.shortconv_fwd(c["x"], c["w"], c["bias"], c["xs"], silu=silu, lib=lib)
+        for cut in (1, 2, 7):
+            y1, s1 = oracle.shortconv_fwd(c["x"][:, :, :cut], c["w"], c["bias"], c["xs"], silu=silu,
+                                          lib=lib)
+            y2, s2 = oracle.shortconv_fwd(c["x"][:, :, cut:], c["w"], c["bias"], s1, silu=silu, lib=lib)
+            close(np.concatenate([y1, y2], 2), yw, 1e-13, f"cut at {cut}")
+            close(s2, sw, 0.0, f"state after cut at {cut}")
+        close(sw, c["x"][:, :, -3:], 0.0, "final state = last W-1 inputs")
+
+
+def check_conv_silu_and_grads(lib=None, seed=23):
+    """SiLU output equals torch's silu of the linear output; the reverse mode
+    equals torch.autograd through torch's grouped conv1d (left padding W-1 with
+    the carried state, flipped filters) and central differences."""
+    import torch
+    rng = np.random.default_rng(seed)
+    c = conv_inputs(rng, B=2, H=2, T=6, D=3, W=3)
+    ylin, _ = oracle.shortconv_fwd(c["x"], c["w"], c["bias"], c["xs"], lib=lib)
+    ysil, _ = oracle.shortconv_fwd(c["x"], c["w"], c["bias"], c["xs"], silu=True, lib=lib)
+    close(ysil, torch.nn.functional.silu(torch.from_numpy(ylin)).numpy(), 1e-14, "silu")
+    dy = rng.standard_normal(ylin.shape)
+    dso = rng.standard_normal(c["xs"].shape)
+    for silu in (False, True):
+        gr = oracle.shortconv_bwd(c["x"], c["w"], c["bias"], c["xs"], dy, dso, silu=silu, lib=lib)
+        t = {n: torch.tensor(a, dtype=torch.float64, requires_grad=True) for n, a in c.items()}
+        B, H, T, D = c["x"].shape
+        W = c["w"].shape[-1]
+        seq = torch.cat([t["xs"], t["x"]], 2)                           # [B,H,W-1+T,D]
+        inp = seq.permute(0, 1, 3, 2).reshape(B, H * D, W - 1 + T)
+        wt = torch.flip(t["w"], [-1]).reshape(H * D, 1, W)
+        z = torch.nn.functional.conv1d(inp, wt, t["bias"].reshape(H * D), groups=H * D)
+        z = z.reshape(B, H, D, T).permute(0, 1, 3, 2)
+        yt = torch.nn.functional.silu(z) if silu else z
+        st = seq[:, :, T:]                                               # last W-1 inputs
+        L = (yt * torch.tensor(dy)).sum() + (st * torch.tensor(dso)).sum()
+        L.backward()
+        for n, gn in (("x", "dx"), ("w", "dw"), ("bias", "dbias"), ("xs", "dxs")):
+            close(gr[gn], t[n].grad.numpy(), 1e-12, f"conv autograd {gn} silu={silu}")
+    # central differences on one weight and one state entry (silu on)
+    gr = oracle.shortconv_bwd(c["x"], c["w"], c["bias"], c["xs"], dy, dso, silu=True, lib=lib)
+
+    def loss(cc):
+        y, s = oracle.shortconv_fwd(cc["x"], cc["w"], cc["bias"], cc["xs"], silu=True, lib=lib)
+        return float(np.sum(y * dy) + np.sum(s * dso))
+
+    h = 1e-6
+    for n, idx, gn in (("w", (1, 2, 0), "dw"), ("xs", (0, 1, 1, 2), "dxs"), ("x", (1, 0, 5, 1), "dx")):
+        cp = {m: a.copy() for m, a in c.items()}
+        cm = {m: a.copy() for m, a in c.items()}
+        cp[n][idx] += h
+        cm[n][idx] -= h
+        close(gr[gn][idx], (loss(cp) - loss(cm)) / (2 * h), 1e-7, f"conv finite difference {gn}")
+
+
+CONV_PINS = [check_conv_width_one, check_conv_numpy_convolve, check_conv_impulse_and_state,
+             check_conv_silu_and_grads]
+
 FORWARD_PINS = [check_worked_example, check_T1_closed_form, check_g_zero, check_tau_zero,
                 check_quadratic, check_linearity, check_split_and_decode]
 BACKWARD_PINS = [check_bwd_finite_differences, check_bwd_autograd]
-ALL_PINS = FORWARD_PINS + BACKWARD_PINS + PREACT_PINS + FEED_PINS
+ALL_PINS = FORWARD_PINS + BACKWARD_PINS + PREACT_PINS + FEED_PINS + CONV_PINS

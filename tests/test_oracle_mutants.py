@@ -55,6 +55,14 @@ MUTANTS = [
      P.FEED_PINS),
     ("bwd feedthrough dd with vhat", "J->ddfeed[(size_t)p * dv + j] += dO[j] * v[j];",
      "J->ddfeed[(size_t)p * dv + j] += dO[j] * v[j] * beta[j];", P.FEED_PINS),
+    ("conv filter flipped",
+     "z += w[((size_t)h * D + c) * W + i] * conv_input(xp, sp, T, D, W, t - i, c);\n                y[",
+     "z += w[((size_t)h * D + c) * W + (W - 1 - i)] * conv_input(xp, sp, T, D, W, t - i, c);\n                y[",
+     P.CONV_PINS),
+    ("conv state newest first", "int s = W - 1 + t;", "int s = -1 - t;", P.CONV_PINS),
+    ("conv silu derivative", "gz *= s * (1.0 + z * (1.0 - s));", "gz *= s;", P.CONV_PINS),
+    ("conv weight grad off by one", "dw[((size_t)h * D + c) * W + i] += gz * conv_input(xp, sp, T, D, W, ti, c);",
+     "dw[((size_t)h * D + c) * W + i] += gz * conv_input(xp, sp, T, D, W, ti - 1, c);", P.CONV_PINS),
 ]
 
 
