@@ -108,19 +108,25 @@ def src_sha(*names):
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel, source_files, workload):
-    """DRAM bytes per launch from the committed ncu summary, or None when the
-    kernel source changed since that capture."""
-    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+def ncu_counters(kernel, source_files, workload):
+    """Counters of one ncu capture of `kernel` on `workload` from the committed
+    summary (profiles/ncu_counters.json), or None when the kernel's source
+    changed since that capture: DRAM bytes per launch, the tensor-pipe
+    utilisation and the DRAM throughput ncu reported."""
+    p = os.path.join(ROOT, "profiles", "ncu_counters.json")
     if not os.path.exists(p):
         return None
     d = json.load(open(p)).get(f"{kernel}@{workload}")
     if not d or d.get("src_sha") != src_sha(*source_files):
         return None
-    return d.get("dram_bytes_per_launch")
+    return d
 
 
-def roofline(bytes_, flops, ms, pk, traffic, timed_alone=True):
+def roofline(bytes_, flops, ms, pk, counters, timed_alone=True):
+    """Roofline object of one kernel: achieved = algorithmic bytes (or flops) per
+    launch / measured time.  `counters` (ncu_counters) adds the DRAM traffic of
+    a launch and the captured kernel's tensor-pipe and DRAM utilisation."""
+    traffic = counters.get("dram_bytes_per_launch") if counters else None
     t = ms / 1e3
     ach_gbs = bytes_ / t / 1e9
     ach_tf = flops / t / 1e12
@@ -128,12 +134,18 @@ def roofline(bytes_, flops, ms, pk, traffic, timed_alone=True):
     t_hbm = bytes_ / (pk["hbm_gbs"] * 1e9)
     t_tc = flops / (tf_peak * 1e12)
     if t_hbm >= t_tc:
-        return {"bound": "hbm", "achieved": round(ach_gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": round(ach_gbs / pk["hbm_gbs"], 4), "traffic": traffic,
-                "algorithmic_bytes": int(bytes_), "peak_source": pk["source"]}
-    return {"bound": "tensor", "achieved": round(ach_tf, 2), "peak": tf_peak, "unit": "TFLOP/s",
-            "frac": round(ach_tf / tf_peak, 4), "traffic": traffic, "algorithmic_flops": int(flops),
-            "peak_source": pk["source"]}
+        out = {"bound": "hbm", "achieved": round(ach_gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+               "frac": round(ach_gbs / pk["hbm_gbs"], 4), "traffic": traffic,
+               "algorithmic_bytes": int(bytes_), "peak_source": pk["source"]}
+    else:
+        out = {"bound": "tensor", "achieved": round(ach_tf, 2), "peak": tf_peak, "unit": "TFLOP/s",
+               "frac": round(ach_tf / tf_peak, 4), "traffic": traffic,
+               "algorithmic_flops": int(flops), "peak_source": pk["source"]}
+    if counters:
+        out["ncu"] = {k: counters[k] for k in ("tensor_pipe_pct", "dram_throughput_pct",
+                                               "dram_gbs", "issue_active_pct", "duration_us")
+                      if k in counters}
+    return out
 
 
 class ClockSampler:
@@ -271,7 +283,7 @@ def run_extras(rdm, dev, pk, K):
         "workload": w.name, "value": w.B * w.T / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
         "gpu_launches_per_step": 1,
         "roofline": roofline(fwd_bytes(w, True), chunk_flops_fwd(w), ms, pk,
-                             ncu_traffic("tc_fwd_kernel", FWD_SRC, 2))}
+                             ncu_counters("tc_fwd_kernel", FWD_SRC, 2))}
     del x, o, ST, wsf
     # headline forward with the gate activations fused (inputs are the
     # pre-activations; same bytes)
@@ -287,7 +299,8 @@ def run_extras(rdm, dev, pk, K):
     out["fused_gates_fwd"] = {
         "workload": w.name + ", gates passed before softplus/sigmoid", "value": w.B * w.T / (ms / 1e3),
         "unit": "tokens/s", "ms_per_step": ms, "gpu_launches_per_step": 1,
-        "roofline": roofline(fwd_bytes(w, False), chunk_flops_fwd(w), ms, pk, None)}
+        "roofline": roofline(fwd_bytes(w, False), chunk_flops_fwd(w), ms, pk,
+                             ncu_counters("tc_fwd_kernel", FWD_SRC, "1pre"))}
     del x, o, wsf, fl
     # training forward + backward (forward saves chunk states for the backward)
     w = WORKLOADS[3]
@@ -316,12 +329,66 @@ def run_extras(rdm, dev, pk, K):
         # once for heads the tensor-core kernel handled)
         "gpu_launches_per_step": 4,
         "roofline_fwd": roofline(fb, chunk_flops_fwd(w), msf, pk,
-                                 ncu_traffic("tc_fwd_kernel", FWD_SRC, 3)),
+                                 ncu_counters("tc_fwd_kernel", FWD_SRC, 3)),
         "roofline_bwd": roofline(bwd_bytes(w), chunk_flops_bwd(w), msb, pk,
-                                 ncu_traffic("tc_bwd_kernel", BWD_SRC, 3)),
+                                 ncu_counters("tc_bwd_kernel", BWD_SRC, 3)),
         "roofline_step": roofline(fb + bwd_bytes(w), chunk_flops_fwd(w) + chunk_flops_bwd(w),
                                   msf + msb, pk, None)}
     del x, o, saved, grads, ws, wsf
+    # headline forward with the feedthrough o_t += d (.) v_t (same algorithmic
+    # bytes plus d; v is re-read from L2 in the store stage)
+    w = WORKLOADS[1]
+    x = draw_workload(w, device=dev)
+    o = torch.empty(w.B, w.H, w.T, w.dv, dtype=torch.bfloat16, device=dev)
+    dfe = torch.randn(w.H, w.dv, device=dev, generator=torch.Generator(device=dev).manual_seed(3))
+    wsf = fwd_workspace(rdm, x, dev)
+    fl = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    t = time_steps(lambda: rdm.rdm_ddts_fwd(*(x[k] for k in SEQ), x["S0"], o, workspace=wsf,
+                                            feedthrough=dfe), max(3, K // 2), 3, lambda: fl.zero_())
+    ms = statistics.mean(t)
+    out["feedthrough_fwd"] = {
+        "workload": w.name + ", feedthrough o += d * v", "value": w.B * w.T / (ms / 1e3),
+        "unit": "tokens/s", "ms_per_step": ms, "gpu_launches_per_step": 1,
+        "roofline": roofline(fwd_bytes(w, False) + w.H * w.dv * 4, chunk_flops_fwd(w), ms, pk, None)}
+    del x, o, wsf, dfe
+    # ShortConv (width 4, SiLU) forward + backward on the q, k and v tensors of
+    # the same layer (D = 64, 64, 128)
+    gen = torch.Generator(device=dev).manual_seed(4)
+    convs = []
+    for D in (w.dk, w.dk, w.dv):
+        xc = torch.randn(w.B, w.H, w.T, D, device=dev, generator=gen).to(torch.bfloat16)
+        wc = torch.randn(w.H, D, 4, device=dev, generator=gen) / 4
+        bc = torch.randn(w.H, D, device=dev, generator=gen) * 0.1
+        gy = torch.randn(w.B, w.H, w.T, D, device=dev, generator=gen).to(torch.bfloat16)
+        outs = dict(dx=torch.empty_like(xc), dw=torch.empty_like(wc), dbias=torch.empty_like(bc))
+        convs.append((xc, wc, bc, gy, torch.empty_like(xc), outs))
+
+    def conv_step():
+        for xc, wc, bc, gy, yc, outs in convs:
+            rdm.rdm_shortconv_fwd(xc, wc, bc, None, silu=True, y=yc)
+            rdm.rdm_shortconv_bwd(xc, wc, bc, None, gy, None, silu=True, out=outs)
+
+    # six short kernels per step: replayed as one CUDA graph so that the step
+    # is timed on the device, not through the Python binding's per-call overhead
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        conv_step()
+        gconv = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gconv, stream=side):
+            conv_step()
+    torch.cuda.current_stream().wait_stream(side)
+    t = time_steps(lambda: gconv.replay(), max(3, K // 2), 3, lambda: fl.zero_())
+    ms = statistics.mean(t)
+    cb = w.B * w.H * w.T * 2 * (w.dk + w.dk + w.dv) * (2 + 3)   # fwd: x, y; bwd: x, dy, dx
+    out["shortconv_fwd_bwd"] = {
+        "workload": "ShortConv width 4 + SiLU, fwd+bwd over q, k, v of " + w.name,
+        "value": w.B * w.T / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
+        # per tensor: forward kernel, backward kernel (the weight gradients are zeroed
+        # by memset, not counted)
+        "gpu_launches_per_step": 6, "cuda_graph": True,
+        "roofline": roofline(cb, 0, ms, pk, None)}
+    del gconv, convs, fl
     # batched decode, 1024 steps captured in one CUDA graph
     w = WORKLOADS[4]
     steps = w.T
@@ -345,7 +412,7 @@ def run_extras(rdm, dev, pk, K):
         "workload": w.name, "value": w.B * steps / (ms / 1e3), "unit": "tokens/s",
         "ms_per_step": per, "ms_per_graph": ms, "gpu_launches_per_step": 1,
         "roofline": roofline(decode_bytes(w), 2 * w.B * w.H * w.dk * w.dv * 3, per, pk,
-                             ncu_traffic("decode_kernel", DECODE_SRC, 4), timed_alone=False)}
+                             ncu_counters("decode_kernel", DECODE_SRC, 4), timed_alone=False)}
     del g, xd, S, od
     return out
 
@@ -460,7 +527,7 @@ def main():
         "gated_linear_attention_ddts_b200/workloads.py)", "config": cfg,
         "token_heads_per_s": value * w.H,
         "roofline": roofline(fwd_bytes(w, False), chunk_flops_fwd(w), ms, pk,
-                             ncu_traffic("tc_fwd_kernel", FWD_SRC, 1)),
+                             ncu_counters("tc_fwd_kernel", FWD_SRC, 1)),
         "clocks": clocks,
         "e2e": {"value": weak_scaling_value(w.B * w.T, world, e2e_ms), "unit": "tokens/s",
                 "ms_per_step": e2e_ms,

@@ -317,14 +317,19 @@ def rdm_shortconv_fwd(x, weight, bias=None, state_in=None, *, silu=False, y=None
 
 
 def rdm_shortconv_bwd(x, weight, bias, state_in, grad_y, grad_state_out=None, *, silu=False,
-                      stream=None):
+                      out=None, stream=None):
     """Reverse mode of rdm_shortconv_fwd.  Returns dict dx, dw, dbias (None
-    without bias) and dxs (None without state_in)."""
-    B, H, T, D = x.shape
-    W = weight.shape[-1]
-    out = dict(dx=torch.empty_like(x), dw=torch.empty_like(weight),
-               dbias=torch.empty_like(bias) if bias is not None else None,
-               dxs=torch.empty_like(state_in) if state_in is not None else None)
+    without bias) and dxs (None without state_in); `out` may hold them
+    preallocated."""
+    out = dict(out or {})
+    if out.get("dx") is None:
+        out["dx"] = torch.empty_like(x)
+    if out.get("dw") is None:
+        out["dw"] = torch.empty_like(weight)
+    if out.get("dbias") is None:
+        out["dbias"] = torch.empty_like(bias) if bias is not None else None
+    if out.get("dxs") is None:
+        out["dxs"] = torch.empty_like(state_in) if state_in is not None else None
     a = ConvBwdArgs(_conv_args(x, weight, bias, state_in, None, None, silu), _ptr(grad_y),
                     _ptr(grad_state_out), _ptr(out["dx"]), _ptr(out["dw"]), _ptr(out["dbias"]),
                     _ptr(out["dxs"]))

@@ -83,6 +83,7 @@ struct ConvParams {
     float* dw;           // dL/dw [H,D,W]
     float* dbias;        // dL/dbias [H,D] or null
     void* dxs;           // dL/d(carried-in state) or null
+    int conv_groups;     // backward: token groups per block (set by the launcher)
 };
 cudaError_t launch_conv_fwd(const ConvParams& p, cudaStream_t s);
 cudaError_t launch_conv_bwd(const ConvParams& p, cudaStream_t s);

@@ -10,11 +10,15 @@
 // HBM-bound streaming: one thread owns 16 bytes of channels (8 bf16 or 4
 // float32) over a run of kRun consecutive tokens and keeps the last W inputs
 // of its channels in registers, so every input row is read once per run (plus
-// a W-1 row halo that the neighbouring run has just pulled into L2) and every
-// output row written once; a warp's loads and stores cover whole 16-byte
-// column groups of consecutive rows.  The backward walks the same runs with a
+// a W-1 row halo that the neighbouring run of the same block has just pulled
+// into L1) and every output row written once; a warp's loads and stores cover
+// whole 16-byte column groups of consecutive rows.  Runs are short and fully
+// unrolled so that each thread has all of its loads in flight at once (with
+// 16-token runs walked one load at a time the kernels ran at 7% of HBM).  The backward walks the same runs with a
 // look-ahead window of W values of dL/dz, and reduces the weight and bias
 // gradients in shared memory before one float32 atomic per value and block.
+#include <algorithm>
+
 #include "launch.h"
 #include "rdm_common.cuh"
 
@@ -22,19 +26,22 @@ namespace rdm {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kRun = 16;  // tokens per thread
+constexpr int kRun = 4;  // tokens per thread (loops fully unrolled: every load in flight at once)
 
 template <typename T>
 struct Vec {
     static constexpr int N = 16 / sizeof(T);  // channels per 16-byte group
 };
 
+// inputs are read through the read-only path (x, dy and the states are never
+// written by these kernels; the API requires outputs not to alias inputs), so
+// the loads of a run can be issued ahead of its stores
 __device__ __forceinline__ void load_vec(const float* p, float* f) {
-    const float4 u = *reinterpret_cast<const float4*>(p);
+    const float4 u = __ldg(reinterpret_cast<const float4*>(p));
     f[0] = u.x; f[1] = u.y; f[2] = u.z; f[3] = u.w;
 }
 __device__ __forceinline__ void load_vec(const __nv_bfloat16* p, float* f) {
-    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
@@ -93,7 +100,10 @@ __global__ void __launch_bounds__(kThreads) conv_fwd_kernel(ConvParams p) {
 #pragma unroll
     for (int k = 0; k < W - 1; ++k) input_row<T>(p, bh, t0 - (W - 1) + k, c0, win[k]);
     T* y = static_cast<T*>(p.y) + (size_t)bh * p.T * p.D + c0;
-    for (int t = t0; t < t1; ++t) {
+#pragma unroll
+    for (int k = 0; k < kRun; ++k) {
+        const int t = t0 + k;
+        if (t >= t1) break;
         input_row<T>(p, bh, t, c0, win[W - 1]);
         float z[N];
 #pragma unroll
@@ -158,10 +168,9 @@ __global__ void __launch_bounds__(kThreads) conv_bwd_kernel(ConvParams p) {
     const int CG = p.D / N, R = kThreads / CG;
     const int bh = blockIdx.x, h = bh % p.H;
     const int cg = threadIdx.x % CG, run = threadIdx.x / CG, c0 = cg * N;
-    const int t0 = (blockIdx.y * R + run) * kRun, t1 = min(t0 + kRun, p.T);
-    __shared__ float s_acc[128 * 5];  // CG * (W + 1) * N = D (W + 1) <= 128 * 5 floats
-    for (int i = threadIdx.x; i < CG * (W + 1) * N; i += kThreads) s_acc[i] = 0.0f;
-    __syncthreads();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    // per-warp partial sums of the weight and bias gradients: [warp][cg][W+1][N]
+    __shared__ float s_red[kThreads / 32][128 * 5];  // CG (W + 1) N = D (W + 1) <= 640
     float wv[W][N], bv[N], aw[W][N], ab[N];
 #pragma unroll
     for (int e = 0; e < N; ++e) {
@@ -173,14 +182,22 @@ __global__ void __launch_bounds__(kThreads) conv_bwd_kernel(ConvParams p) {
         bv[e] = p.bias ? p.bias[(size_t)h * p.D + c0 + e] : 0.0f;
         ab[e] = 0.0f;
     }
-    if (t0 < p.T) {
+    T* dx = static_cast<T*>(p.dx) + (size_t)bh * p.T * p.D + c0;
+    const int tout0 = p.T - (p.W - 1);  // first token copied into the carried-out state
+    // the block's tile of tokens is a whole number of R x kRun groups; every
+    // thread walks its run in each group (the weight gradients accumulate in
+    // registers across the groups)
+    for (int t0 = (blockIdx.y * p.conv_groups * R + run) * kRun; t0 < min(p.T, (blockIdx.y + 1) * p.conv_groups * R * kRun);
+         t0 += R * kRun) {
+        const int t1 = min(t0 + kRun, p.T);
         // dzw[k] = dz[t + k] for the output t = the oldest token of the window
         float dzw[W][N];
 #pragma unroll
         for (int k = 0; k < W - 1; ++k) dz_row<T, W>(p, bh, t0 + k, c0, wv, bv, dzw[k]);
-        T* dx = static_cast<T*>(p.dx) + (size_t)bh * p.T * p.D + c0;
-        const int tout0 = p.T - (p.W - 1);  // first token copied into the carried-out state
-        for (int t = t0; t < t1; ++t) {
+#pragma unroll
+        for (int k = 0; k < kRun; ++k) {
+            const int t = t0 + k;
+            if (t >= t1) break;
             dz_row<T, W>(p, bh, t + W - 1, c0, wv, bv, dzw[W - 1]);
             float xw[W][N];  // x[t - i]
 #pragma unroll
@@ -191,7 +208,7 @@ __global__ void __launch_bounds__(kThreads) conv_bwd_kernel(ConvParams p) {
                 float a = 0.0f;
 #pragma unroll
                 for (int i = 0; i < W; ++i) {
-                    a = fmaf(wv[i][e], dzw[i][e], a);        // dx[t] = sum_i w_i dz[t + i]
+                    a = fmaf(wv[i][e], dzw[i][e], a);                // dx[t] = sum_i w_i dz[t + i]
                     aw[i][e] = fmaf(dzw[0][e], xw[i][e], aw[i][e]);  // dw_i += dz[t] x[t - i]
                 }
                 ab[e] += dzw[0][e];
@@ -205,26 +222,35 @@ __global__ void __launch_bounds__(kThreads) conv_bwd_kernel(ConvParams p) {
             }
             store_vec(dx + (size_t)t * p.D, g);
 #pragma unroll
-            for (int k = 0; k < W - 1; ++k)
+            for (int kk = 0; kk < W - 1; ++kk)
 #pragma unroll
-                for (int e = 0; e < N; ++e) dzw[k][e] = dzw[k + 1][e];
+                for (int e = 0; e < N; ++e) dzw[kk][e] = dzw[kk + 1][e];
         }
     }
-    // weight and bias gradients: shared-memory sums over the runs, then global
+    // weight and bias gradients: sum the lanes of a warp that hold the same
+    // channels (lanes cg, cg + CG, ...), one slot per warp in shared memory, a
+    // sum over the warps, then one float32 atomic per value and block
 #pragma unroll
     for (int e = 0; e < N; ++e) {
 #pragma unroll
-        for (int i = 0; i < W; ++i) atomicAdd(&s_acc[(cg * (W + 1) + i) * N + e], aw[i][e]);
-        atomicAdd(&s_acc[(cg * (W + 1) + W) * N + e], ab[e]);
+        for (int i = 0; i <= W; ++i) {
+            float x = i < W ? aw[i][e] : ab[e];
+            for (int off = CG; off < 32; off <<= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+            if (lane < CG) s_red[warp][(cg * (W + 1) + i) * N + e] = x;
+        }
     }
     __syncthreads();
-    (void)R;
+    // CG divides 32, so every warp holds every channel group
     for (int idx = threadIdx.x; idx < CG * (W + 1) * N; idx += kThreads) {
-        const int e = idx % N, i = (idx / N) % (W + 1), g = idx / (N * (W + 1));
-        const int c = g * N + e;
-        if (i < W) atomicAdd(p.dw + ((size_t)h * p.D + c) * W + i, s_acc[idx]);
-        else if (p.dbias) atomicAdd(p.dbias + (size_t)h * p.D + c, s_acc[idx]);
+        const int e = idx % N, i = (idx / N) % (W + 1), gi = idx / (N * (W + 1));
+        float a = 0.0f;
+#pragma unroll
+        for (int w2 = 0; w2 < kThreads / 32; ++w2) a += s_red[w2][idx];
+        const int c = gi * N + e;
+        if (i < W) atomicAdd(p.dw + ((size_t)h * p.D + c) * W + i, a);
+        else if (p.dbias) atomicAdd(p.dbias + (size_t)h * p.D + c, a);
     }
+    (void)R;
 }
 
 // gradient of the carried-in state: dxs[s] = sum_i w_i dz[s-(W-1)+i] over tokens
@@ -283,9 +309,16 @@ cudaError_t bwd_tw(const ConvParams& p, cudaStream_t s) {
     cudaError_t e = cudaMemsetAsync(p.dw, 0, (size_t)p.H * p.D * W * sizeof(float), s);
     if (e == cudaSuccess && p.dbias) e = cudaMemsetAsync(p.dbias, 0, (size_t)p.H * p.D * sizeof(float), s);
     if (e != cudaSuccess) return e;
+    // tiles of `groups` R x kRun token groups: about four blocks per SM in all,
+    // so each block sums the weight gradients over several groups before its
+    // atomics
     const int R = kThreads / (p.D / Vec<T>::N);
-    const dim3 grid(p.B * p.H, (p.T + R * kRun - 1) / (R * kRun));
-    if (p.T > 0) conv_bwd_kernel<T, W><<<grid, kThreads, 0, s>>>(p);
+    const int ngroups = (p.T + R * kRun - 1) / (R * kRun);
+    const int want_tiles = std::max(1, (4 * sm_count() + p.B * p.H - 1) / (p.B * p.H));
+    ConvParams q = p;
+    q.conv_groups = std::max(1, (ngroups + want_tiles - 1) / want_tiles);
+    const dim3 grid(p.B * p.H, (ngroups + q.conv_groups - 1) / q.conv_groups);
+    if (p.T > 0) conv_bwd_kernel<T, W><<<grid, kThreads, 0, s>>>(q);
     if constexpr (W > 1) {
         if (p.dxs) {
             const size_t n = (size_t)p.B * p.H * (W - 1) * (p.D / Vec<T>::N);

@@ -5,7 +5,7 @@
 // (alpha = exp(-g*tau), khat = g^tau * k, vhat = beta_hat * v; Rodimus*,
 // digest.lyk-ai.com summary, "Method") organised by chunks of 64 tokens, last
 // chunk first.  With b_t the inclusive running sum of log(alpha) in the chunk,
-// m the per-channel reference of the forward (midpoint of the b range),
+// m the per-channel reference of the forward (half the chunk's total, b_last / 2),
 // Qt = q e^{b-m}, Kt = khat e^{m-b}, S_prev the state before the chunk (saved by
 // the forward) and R = dL/dS at the end of the chunk (flowing backwards):
 //
@@ -412,11 +412,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                         b[u][e] += x - tot;
                         if (u == usrc) mine = b[u][e];
                     }
-                    const float bf = __shfl_sync(full, b[0][e], cgl);
+                    // reference m = half the chunk's total log decay: b runs over
+                    // [b_last, 0], so every factor stays inside exp(+-|b_last|/2)
                     const float bl = __shfl_sync(full, mine, lsrc);
-                    mL[e] = 0.5f * (bf + bl) * kLog2e;
+                    mL[e] = 0.5f * bl * kLog2e;
                     blL[e] = bl * kLog2e;
-                    span = fmaxf(span, bf - bl);
+                    span = fmaxf(span, -bl);
                 }
                 // too wide for one reference: the exact path recomputes this head
                 // (the R-only pass needs no reference)

@@ -4,17 +4,20 @@
 // answer to Q2 and "Efficient Parallelization": selection only along d_k makes
 // the chunkwise form possible).  Per (b,h) and chunk of C = 64 tokens, with
 // b_t the inclusive running sum of log(alpha) = -g*tau inside the window and
-// m a per-channel reference (the midpoint of the window's b range):
+// m a per-channel reference (half the window's total, m = b_last / 2):
 //
 //   Qt = q * exp(b_t - m)              Kt = k * alpha_hat * exp(m - b_s)
 //   A  = mask_{s<=t}(Qt Kt^T)          Vh = beta_hat * v
 //   o  = A Vh + Qt (diag(exp(m)) S_prev)                 (intra + inter chunk)
 //   S  = diag(exp(b_last)) S_prev + diag(exp(b_last - m)) Kt^T Vh
 //
-// Every factor stays inside exp(+-span/2) with span = b_first - b_last of the
-// window, so products are exact in fp32 range whenever span <= kSpanMax.  A
-// chunk whose span is larger is processed as windows of 16 tokens, or of 1
-// token, each window being one pass of the same pipeline (exact for any decay).
+// b_t runs over [b_last, 0] (every log decay is <= 0), so every factor stays
+// inside exp(+-|b_last|/2), and products are exact in fp32 range whenever
+// |b_last| <= kSpanMax.  A chunk with a larger total is processed as windows of
+// 16 tokens, or of 1 token, each window being one pass of the same pipeline
+// (exact for any decay).  (The midpoint of the b range is a slightly tighter
+// reference but needs b at the window's first token, one more shuffle per
+// channel: measured 10% slower on the d_k = 128 long-context forward.)
 //
 // Sequence segments.  When the (b,h) x d_v-slice units do not fill the GPU,
 // each unit's chunks are cut into P contiguous segments, one CTA each.  The
@@ -398,10 +401,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             // log2(alpha_hat) of my tokens is kept from the scan for the operand pass
             // when registers allow (d_k = 64); otherwise that pass re-reads g and tau
             constexpr bool kKeepLah = SEGT <= 2;
-            float b[SEGT][8], bf[8], bl[8];
+            float b[SEGT][8], bl[8];
             [[maybe_unused]] float lah2[kKeepLah ? SEGT : 1][8];
             // window-relative inclusive running sum of log(alpha) over my tokens, and
-            // b at the first / last valid token of my window (W in {64, 16})
+            // b at the last valid token of my window (W in {64, 32, 16})
             auto scan = [&](int W) {
 #pragma unroll
                 for (int u = 0; u < SEGT; ++u) {
@@ -440,7 +443,6 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                         b[u][e] += excl;
                         if (u == usrc) mine = b[u][e];
                     }
-                    bf[e] = __shfl_sync(full, b[0][e], l0 + cgl);
                     bl[e] = __shfl_sync(full, mine, lsrc);
                 }
             };
@@ -449,7 +451,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             auto too_wide = [&](int* flag) {
                 float span = 0.0f;
 #pragma unroll
-                for (int e = 0; e < 8; ++e) span = fmaxf(span, bf[e] - bl[e]);
+                for (int e = 0; e < 8; ++e) span = fmaxf(span, -bl[e]);
                 if (tb >= nval) span = 0.0f;
                 if (__any_sync(full, !(span <= kSpanMax)) && lane == 0) *flag = li + 1;
                 named_bar(kBarGate, 32 * kGateWarps);
@@ -568,7 +570,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                         return false;
                     float mL[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) mL[e] = 0.5f * (bf[e] + bl[e]) * kLog2e;
+                    for (int e = 0; e < 8; ++e) mL[e] = 0.5f * bl[e] * kLog2e;
 #pragma unroll
                     for (int u = 0; u < SEGT; ++u) {
                         const int t = tb + u;
@@ -630,9 +632,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                             if constexpr (PRE) activate_gates8(g8, t8);
 #pragma unroll
                             for (int e = 0; e < 8; ++e) {
-                                // reference m = midpoint of the window's b range, blast = b at its end
+                                // reference m = half the window's total log decay, blast = b at its end
                                 const float blast = W == 1 ? b[u][e] : bl[e];
-                                const float m = W == 1 ? b[u][e] : 0.5f * (bf[e] + bl[e]);
+                                const float m = W == 1 ? b[u][e] : 0.5f * bl[e];
                                 const float d = (b[u][e] - m) * kLog2e;
                                 const float lah = t8[e] == 0.0f ? 0.0f : t8[e] * lg2_fast(g8[e]);
                                 oq[e] = in ? q8[e] * ex2_fast(d) : 0.0f;

@@ -271,8 +271,10 @@ rdm_status rdm_ddts_decode(const rdm_decode_args *args, rdm_stream_t stream);
  *   x, y        : [B,H,T,D] dtype        D in {16, 32, 64, 128}; W in {1,2,3,4}
  *   weight      : [H,D,W] float32        bias : [H,D] float32 or NULL
  *   state_in    : [B,H,W-1,D] dtype or NULL (zeros)
- *   state_out   : [B,H,W-1,D] dtype or NULL (not written); must not alias x,
- *                 y or state_in
+ *   state_out   : [B,H,W-1,D] dtype or NULL (not written)
+ * Outputs must not alias inputs (y, state_out vs x, state_in; in the backward
+ * grad_x, grad_state_in vs x, state_in, grad_y, grad_state_out): the kernels
+ * read their inputs through the read-only path.
  * All pointers are device pointers, 16-byte aligned; nothing is allocated.
  */
 typedef struct {
