@@ -55,8 +55,12 @@ def load_library(path: str):
     lib.rdm_oracle_decode_step.argtypes = [I] * 4 + [P] * 9 + [I]
     lib.rdm_oracle_shortconv_fwd.argtypes = [I] * 5 + [P] * 4 + [I] + [P] * 2
     lib.rdm_oracle_shortconv_bwd.argtypes = [I] * 5 + [P] * 4 + [I] + [P] * 6
+    D = ctypes.c_double
+    lib.rdm_oracle_ska_fwd.argtypes = [I] * 6 + [D] + [P] * 4
+    lib.rdm_oracle_ska_decode.argtypes = [I] * 5 + [D, ctypes.POINTER(ctypes.c_longlong)] + [P] * 6
     for f in (lib.rdm_oracle_fwd, lib.rdm_oracle_bwd, lib.rdm_oracle_decode_step,
-              lib.rdm_oracle_shortconv_fwd, lib.rdm_oracle_shortconv_bwd):
+              lib.rdm_oracle_shortconv_fwd, lib.rdm_oracle_shortconv_bwd,
+              lib.rdm_oracle_ska_fwd, lib.rdm_oracle_ska_decode):
         f.restype = I
     return lib
 
@@ -210,3 +214,41 @@ def shortconv_bwd(x, w, bias, xs, dy, dxs_out=None, silu=False, lib=None):
     if rc != 0:
         raise RuntimeError("rdm_oracle_shortconv_bwd failed")
     return out
+
+
+def ska_fwd(q, k, v, window, scale=None, lib=None):
+    """Sliding-window shared-key attention (SW-SKA of Rodimus+; digest.lyk-ai.com
+    summary, "Method"; paperhub.cn rebuttal, Q1): token t of head h attends to
+    tokens max(0, t-window+1)..t through the one key row per token that all heads
+    share, scores scaled by ``scale`` (default 1/sqrt(d_k)), softmax over the
+    window.  q [B,H,T,dk], k [B,T,dk], v [B,H,T,dv] -> o [B,H,T,dv] float64."""
+    q, k, v = map(_f64, (q, k, v))
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    sc = 1.0 / np.sqrt(dk) if scale is None else float(scale)
+    o = np.zeros((B, H, T, dv))
+    if _load(lib).rdm_oracle_ska_fwd(B, H, T, dk, dv, int(window), sc, _p(q), _p(k), _p(v),
+                                     _p(o)) != 0:
+        raise RuntimeError("rdm_oracle_ska_fwd failed")
+    return o
+
+
+def ska_decode(q, k, v, k_cache, v_cache, pos, window, scale=None, lib=None):
+    """One SW-SKA decode step against ring caches of ``window`` slots (position p
+    lives in slot p mod window).  q [B,H,dk], k [B,dk], v [B,H,dv], k_cache
+    [B,window,dk], v_cache [B,H,window,dv], pos [B] the tokens seen before this
+    one.  Returns (o [B,H,dv], new k_cache, new v_cache), all float64."""
+    q, k, v, kc, vc = map(_f64, (q, k, v, k_cache, v_cache))
+    kc, vc = kc.copy(), vc.copy()
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    sc = 1.0 / np.sqrt(dk) if scale is None else float(scale)
+    ps = np.ascontiguousarray(np.asarray(pos.cpu() if hasattr(pos, "cpu") else pos,
+                                         dtype=np.int64))
+    o = np.zeros((B, H, dv))
+    rc = _load(lib).rdm_oracle_ska_decode(
+        B, H, dk, dv, int(window), sc, ps.ctypes.data_as(ctypes.POINTER(ctypes.c_longlong)),
+        _p(q), _p(k), _p(v), _p(kc), _p(vc), _p(o))
+    if rc != 0:
+        raise RuntimeError("rdm_oracle_ska_decode failed")
+    return o, kc, vc

@@ -423,3 +423,95 @@ int rdm_oracle_shortconv_bwd(int B, int H, int T, int D, int W, const double *x,
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------ SW-SKA
+ * Sliding-window shared-key attention of Rodimus+ (digest.lyk-ai.com summary,
+ * "Method", Rodimus+ bullets: attention over a sliding window for local context,
+ * with one key shared by all heads to shrink the KV cache; paperhub.cn
+ * OpenReview rebuttal, answer to Q1: multi-head query and value projections
+ * and a multi-query key projection).  The pages print neither the window nor
+ * the score scale; the reading taken is, per batch b, head h and token t,
+ *     s_u = scale * q[b,h,t] . k[b,u]        for u = max(0, t-w+1) .. t
+ *     o[b,h,t] = sum_u softmax(s)_u v[b,h,u]
+ * with one key row per token shared by every head.  Layouts: q [B,H,T,dk],
+ * k [B,T,dk], v [B,H,T,dv], o [B,H,T,dv].  The softmax subtracts the largest
+ * score first, which leaves the exact value unchanged. */
+static void ska_attend(int n, int dk, int dv, double scale, const double *q,
+                       const double *const *krow, const double *const *vrow, double *p,
+                       double *o)
+{
+    double mx = -INFINITY, sum = 0.0;
+    for (int u = 0; u < n; ++u) {
+        double a = 0.0;
+        for (int i = 0; i < dk; ++i) a += q[i] * krow[u][i];
+        p[u] = scale * a;
+        if (p[u] > mx) mx = p[u];
+    }
+    for (int u = 0; u < n; ++u) {
+        p[u] = exp(p[u] - mx);
+        sum += p[u];
+    }
+    for (int j = 0; j < dv; ++j) o[j] = 0.0;
+    for (int u = 0; u < n; ++u)
+        for (int j = 0; j < dv; ++j) o[j] += (p[u] / sum) * vrow[u][j];
+}
+
+int rdm_oracle_ska_fwd(int B, int H, int T, int dk, int dv, int w, double scale,
+                       const double *q, const double *k, const double *v, double *o)
+{
+    if (B < 0 || H < 0 || T < 0 || dk < 1 || dv < 1 || w < 1) return -1;
+    double *p = (double *)malloc(sizeof(double) * (size_t)w);
+    const double **kr = (const double **)malloc(sizeof(double *) * (size_t)w);
+    const double **vr = (const double **)malloc(sizeof(double *) * (size_t)w);
+    if (!p || !kr || !vr) { free(p); free(kr); free(vr); return -1; }
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < H; ++h) {
+            const size_t bh = (size_t)b * H + h;
+            for (int t = 0; t < T; ++t) {
+                const int u0 = t - w + 1 > 0 ? t - w + 1 : 0;
+                for (int u = u0; u <= t; ++u) {
+                    kr[u - u0] = k + ((size_t)b * T + u) * dk;
+                    vr[u - u0] = v + (bh * T + u) * dv;
+                }
+                ska_attend(t - u0 + 1, dk, dv, scale, q + (bh * T + t) * dk, kr, vr, p,
+                           o + (bh * T + t) * dv);
+            }
+        }
+    free(p); free(kr); free(vr);
+    return 0;
+}
+
+/* One decode step against a ring KV cache of w slots: token position pos[b]
+ * (the number of tokens seen before this one) goes to slot pos[b] mod w, so the
+ * cache holds positions max(0, pos-w+1) .. pos after the write.  Layouts:
+ * q [B,H,dk], k [B,dk], v [B,H,dv], kc [B,w,dk], vc [B,H,w,dv], o [B,H,dv].
+ * The cached positions are visited oldest first. */
+int rdm_oracle_ska_decode(int B, int H, int dk, int dv, int w, double scale,
+                          const long long *pos, const double *q, const double *k,
+                          const double *v, double *kc, double *vc, double *o)
+{
+    if (B < 0 || H < 0 || dk < 1 || dv < 1 || w < 1) return -1;
+    double *p = (double *)malloc(sizeof(double) * (size_t)w);
+    const double **kr = (const double **)malloc(sizeof(double *) * (size_t)w);
+    const double **vr = (const double **)malloc(sizeof(double *) * (size_t)w);
+    if (!p || !kr || !vr) { free(p); free(kr); free(vr); return -1; }
+    for (int b = 0; b < B; ++b) {
+        if (pos[b] < 0) { free(p); free(kr); free(vr); return -1; }
+        const long long t = pos[b], u0 = t - w + 1 > 0 ? t - w + 1 : 0;
+        const int slot = (int)(t % w);
+        for (int i = 0; i < dk; ++i) kc[((size_t)b * w + slot) * dk + i] = k[(size_t)b * dk + i];
+        for (int h = 0; h < H; ++h)
+            for (int j = 0; j < dv; ++j)
+                vc[(((size_t)b * H + h) * w + slot) * dv + j] = v[((size_t)b * H + h) * dv + j];
+        for (int h = 0; h < H; ++h) {
+            for (long long u = u0; u <= t; ++u) {
+                kr[u - u0] = kc + ((size_t)b * w + (size_t)(u % w)) * dk;
+                vr[u - u0] = vc + (((size_t)b * H + h) * w + (size_t)(u % w)) * dv;
+            }
+            ska_attend((int)(t - u0 + 1), dk, dv, scale, q + ((size_t)b * H + h) * dk, kr, vr,
+                       p, o + ((size_t)b * H + h) * dv);
+        }
+    }
+    free(p); free(kr); free(vr);
+    return 0;
+}

@@ -489,7 +489,117 @@ def check_conv_silu_and_grads(lib=None, seed=23):
 CONV_PINS = [check_conv_width_one, check_conv_numpy_convolve, check_conv_impulse_and_state,
              check_conv_silu_and_grads]
 
+# ------------------------------------------------------------------ SW-SKA pins
+def ska_inputs(rng, B=2, H=3, T=13, dk=4, dv=5):
+    return dict(q=rng.standard_normal((B, H, T, dk)), k=rng.standard_normal((B, T, dk)),
+                v=rng.standard_normal((B, H, T, dv)))
+
+
+def check_ska_hand_example(lib=None):
+    """Worked by hand: d_k = d_v = 1, scale 1, window 2, q = 1, k = (0, ln 3, 0),
+    v = (1, 2, 5).  Token 0 sees only itself: 1.  Token 1 weighs e^0 : e^{ln 3}
+    = 1 : 3, so (1 + 3*2)/4 = 7/4.  Token 2 sees tokens 1, 2 with weights 3 : 1,
+    so (3*2 + 5)/4 = 11/4."""
+    q = np.ones((1, 1, 3, 1))
+    k = np.array([0.0, math.log(3.0), 0.0]).reshape(1, 3, 1)
+    v = np.array([1.0, 2.0, 5.0]).reshape(1, 1, 3, 1)
+    o = oracle.ska_fwd(q, k, v, 2, scale=1.0, lib=lib)
+    close(o[0, 0, :, 0], [1.0, 1.75, 2.75], 1e-15, "SW-SKA hand example")
+
+
+def check_ska_window_one_and_uniform(lib=None, seed=30):
+    """Window 1 returns v itself; with q = 0 every score is 0, so each token
+    returns the plain mean of v over its window: a moving average, taken here
+    from numpy prefix sums."""
+    rng = np.random.default_rng(seed)
+    x = ska_inputs(rng)
+    close(oracle.ska_fwd(x["q"], x["k"], x["v"], 1, lib=lib), x["v"], 1e-15, "window 1")
+    T = x["v"].shape[2]
+    for w in (2, 5, 40):
+        o = oracle.ska_fwd(np.zeros_like(x["q"]), x["k"], x["v"], w, lib=lib)
+        c = np.concatenate([np.zeros_like(x["v"][:, :, :1]), np.cumsum(x["v"], 2)], 2)
+        lo = np.maximum(np.arange(T) - w + 1, 0)
+        n = (np.arange(T) - lo + 1)[None, None, :, None]
+        close(o, (c[:, :, 1:] - c[:, :, lo]) / n, 1e-13, f"moving average window {w}")
+
+
+def check_ska_matches_torch_sdpa(lib=None, seed=31):
+    """Against torch's scaled_dot_product_attention in fp64 (its own softmax and
+    1/sqrt(d_k) default scale), the shared key row repeated for every head: causal
+    when the window covers the sequence, else with a boolean band mask that keeps
+    keys t-w+1..t; plus an explicit scale."""
+    import torch
+    F = torch.nn.functional
+    rng = np.random.default_rng(seed)
+    x = ska_inputs(rng, T=17, dk=6, dv=3)
+    q, v = torch.from_numpy(x["q"]), torch.from_numpy(x["v"])
+    k = torch.from_numpy(x["k"])[:, None].expand(-1, q.shape[1], -1, -1)
+    T = q.shape[2]
+    close(oracle.ska_fwd(x["q"], x["k"], x["v"], T, lib=lib),
+          F.scaled_dot_product_attention(q, k, v, is_causal=True).numpy(), 1e-13, "full causal")
+    ti = torch.arange(T)
+    for w in (2, 3, 8):
+        band = (ti[None, :] <= ti[:, None]) & (ti[None, :] > ti[:, None] - w)
+        close(oracle.ska_fwd(x["q"], x["k"], x["v"], w, lib=lib),
+              F.scaled_dot_product_attention(q, k, v, attn_mask=band).numpy(), 1e-13,
+              f"band window {w}")
+        close(oracle.ska_fwd(x["q"], x["k"], x["v"], w, scale=0.3, lib=lib),
+              F.scaled_dot_product_attention(q, k, v, attn_mask=band, scale=0.3).numpy(), 1e-13,
+              f"band window {w} scale 0.3")
+
+
+def check_ska_invariants(lib=None, seed=32):
+    """Adding one vector c to every key shifts each token's scores by the same
+    q.c, which softmax ignores; permuting the heads of q and v permutes the
+    output's heads (the key is shared, nothing else couples heads)."""
+    rng = np.random.default_rng(seed)
+    x = ska_inputs(rng)
+    o = oracle.ska_fwd(x["q"], x["k"], x["v"], 4, lib=lib)
+    c = rng.standard_normal(x["k"].shape[-1])
+    close(oracle.ska_fwd(x["q"], x["k"] + c, x["v"], 4, lib=lib), o, 1e-12, "key shift")
+    perm = [2, 0, 1]
+    close(oracle.ska_fwd(x["q"][:, perm], x["k"], x["v"][:, perm], 4, lib=lib), o[:, perm], 0.0,
+          "head permutation")
+
+
+def check_ska_decode_matches_forward(lib=None, seed=33):
+    """Token-by-token decode against ring caches (position p in slot p mod w),
+    from empty caches and past several wrap-arounds, reproduces the forward at
+    every token; after the last step the caches hold the last w keys and values
+    at their slots.  Sequences of one batch at different positions decode in
+    one call."""
+    rng = np.random.default_rng(seed)
+    x = ska_inputs(rng, T=19)
+    B, H, T, dk = x["q"].shape
+    dv = x["v"].shape[-1]
+    for w in (1, 4, 7, 30):
+        o = oracle.ska_fwd(x["q"], x["k"], x["v"], w, lib=lib)
+        kc, vc = np.zeros((B, w, dk)), np.zeros((B, H, w, dv))
+        for t in range(T):
+            od, kc, vc = oracle.ska_decode(x["q"][:, :, t], x["k"][:, t], x["v"][:, :, t], kc, vc,
+                                           np.full(B, t), w, lib=lib)
+            close(od, o[:, :, t], 1e-13, f"decode window {w} token {t}")
+        for p in range(max(0, T - w), T):
+            close(kc[:, p % w], x["k"][:, p], 0.0, f"k cache slot of position {p}")
+            close(vc[:, :, p % w], x["v"][:, :, p], 0.0, f"v cache slot of position {p}")
+    # ragged positions: batch 0 at its token 3, batch 1 at its token 11
+    w = 5
+    o = oracle.ska_fwd(x["q"], x["k"], x["v"], w, lib=lib)
+    kc, vc = np.zeros((B, w, dk)), np.zeros((B, H, w, dv))
+    for b, t in ((0, 3), (1, 11)):
+        for p in range(max(0, t - w + 1), t):
+            kc[b, p % w], vc[b, :, p % w] = x["k"][b, p], x["v"][b, :, p]
+    sel = (np.array([0, 1]), np.array([3, 11]))
+    od, _, _ = oracle.ska_decode(x["q"][sel[0], :, sel[1]], x["k"][sel], x["v"][sel[0], :, sel[1]],
+                                 kc, vc, np.array([3, 11]), w, lib=lib)
+    close(od[0], o[0, :, 3], 1e-13, "ragged batch 0")
+    close(od[1], o[1, :, 11], 1e-13, "ragged batch 1")
+
+
+SKA_PINS = [check_ska_hand_example, check_ska_window_one_and_uniform, check_ska_matches_torch_sdpa,
+            check_ska_invariants, check_ska_decode_matches_forward]
+
 FORWARD_PINS = [check_worked_example, check_T1_closed_form, check_g_zero, check_tau_zero,
                 check_quadratic, check_linearity, check_split_and_decode]
 BACKWARD_PINS = [check_bwd_finite_differences, check_bwd_autograd]
-ALL_PINS = FORWARD_PINS + BACKWARD_PINS + PREACT_PINS + FEED_PINS + CONV_PINS
+ALL_PINS = FORWARD_PINS + BACKWARD_PINS + PREACT_PINS + FEED_PINS + CONV_PINS + SKA_PINS

@@ -63,6 +63,20 @@ MUTANTS = [
     ("conv silu derivative", "gz *= s * (1.0 + z * (1.0 - s));", "gz *= s;", P.CONV_PINS),
     ("conv weight grad off by one", "dw[((size_t)h * D + c) * W + i] += gz * conv_input(xp, sp, T, D, W, ti, c);",
      "dw[((size_t)h * D + c) * W + i] += gz * conv_input(xp, sp, T, D, W, ti - 1, c);", P.CONV_PINS),
+    ("ska window one too wide", "const int u0 = t - w + 1 > 0 ? t - w + 1 : 0;",
+     "const int u0 = t - w > 0 ? t - w : 0;", P.SKA_PINS),
+    ("ska scale dropped", "p[u] = scale * a;", "p[u] = a;", P.SKA_PINS),
+    ("ska unnormalised", "o[j] += (p[u] / sum) * vrow[u][j];", "o[j] += p[u] * vrow[u][j];",
+     P.SKA_PINS),
+    ("ska value of the next head", "vr[u - u0] = v + (bh * T + u) * dv;",
+     "vr[u - u0] = v + (((bh + 1) % ((size_t)B * H)) * T + u) * dv;", P.SKA_PINS),
+    ("ska key of the next token", "kr[u - u0] = k + ((size_t)b * T + u) * dk;",
+     "kr[u - u0] = k + ((size_t)b * T + (u + 1 < T ? u + 1 : u)) * dk;", P.SKA_PINS),
+    ("ska decode slot shifted", "const int slot = (int)(t % w);",
+     "const int slot = (int)((t + 1) % w);", P.SKA_PINS),
+    ("ska decode window one too narrow",
+     "const long long t = pos[b], u0 = t - w + 1 > 0 ? t - w + 1 : 0;",
+     "const long long t = pos[b], u0 = t - w + 2 > 0 ? t - w + 2 : 0;", P.SKA_PINS),
 ]
 
 
