@@ -37,8 +37,8 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from gated_linear_attention_ddts_b200.workloads import (WORKLOADS, draw_decode,  # noqa: E402
-                                                        draw_workload)
+from gated_linear_attention_ddts_b200.workloads import (SKA_DEC, SKA_FWD, WORKLOADS,  # noqa: E402
+                                                        draw_decode, draw_workload)
 
 SEQ = ("q", "k", "v", "g", "tau", "beta")
 METRIC = "DDTS recurrence tokens/s (fwd, fwd+bwd, decode) on 1 B200; % of roofline"
@@ -99,6 +99,7 @@ _DEV_HDR = ["tc_ptx.cuh", "tc_common.cuh", "rdm_common.cuh", "launch.h"]
 FWD_SRC = ["tc_fwd.cu"] + _DEV_HDR
 BWD_SRC = ["tc_bwd.cu"] + _DEV_HDR
 DECODE_SRC = ["decode.cu", "rdm_common.cuh", "launch.h"]
+SKA_SRC = ["ska.cu", "ska_launch.h"] + _DEV_HDR
 
 
 def src_sha(*names):
@@ -389,6 +390,7 @@ def run_extras(rdm, dev, pk, K):
         "gpu_launches_per_step": 6, "cuda_graph": True,
         "roofline": roofline(cb, 0, ms, pk, None)}
     del gconv, convs, fl
+    out.update(run_ska(rdm, dev, pk, K))
     # batched decode, 1024 steps captured in one CUDA graph
     w = WORKLOADS[4]
     steps = w.T
@@ -414,6 +416,69 @@ def run_extras(rdm, dev, pk, K):
         "roofline": roofline(decode_bytes(w), 2 * w.B * w.H * w.dk * w.dv * 3, per, pk,
                              ncu_counters("decode_kernel", DECODE_SRC, 4), timed_alone=False)}
     del g, xd, S, od
+    return out
+
+
+def ska_keys(T, window):
+    """Query-key pairs inside the sliding window: sum_t min(t + 1, window)."""
+    n = min(T, window)
+    return n * (n + 1) // 2 + (T - n) * window
+
+
+def run_ska(rdm, dev, pk, K):
+    """Sliding-window shared-key attention of the Rodimus+ block: the forward
+    on a 130M-scale layer and batched decode against ring KV caches."""
+    out = {}
+    B, H, T, d, win = SKA_FWD
+    gen = torch.Generator(device=dev).manual_seed(5)
+    q = torch.randn(B, H, T, d, device=dev, generator=gen).to(torch.bfloat16)
+    k = torch.randn(B, T, d, device=dev, generator=gen).to(torch.bfloat16)
+    v = torch.randn(B, H, T, d, device=dev, generator=gen).to(torch.bfloat16)
+    o = torch.empty_like(v)
+    fl = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    t = time_steps(lambda: rdm.rdm_ska_fwd(q, k, v, win, o=o), max(3, K // 2), 3, lambda: fl.zero_())
+    ms = statistics.mean(t)
+    pairs = B * H * ska_keys(T, win)
+    out["ska_fwd"] = {
+        "workload": f"SW-SKA forward B{B} H{H} T{T} d_k=d_v={d} window {win} (one shared key head)",
+        "value": B * T / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
+        "gpu_launches_per_step": 1,
+        "roofline": roofline(2 * (B * H * T * 3 * d + B * T * d), 2 * pairs * 2 * d, ms, pk,
+                             ncu_counters("ska_fwd_kernel", SKA_SRC, "ska1")),
+        "exp2_per_step": pairs}
+    del q, k, v, o
+    # decode: rings full (positions from 1000 on), STEPS tokens per CUDA graph
+    B, H, d, win, steps = SKA_DEC
+    kc = torch.randn(B, win, d, device=dev, generator=gen).to(torch.bfloat16)
+    vc = torch.randn(B, H, win, d, device=dev, generator=gen).to(torch.bfloat16)
+    xq = torch.randn(steps, B, H, d, device=dev, generator=gen).to(torch.bfloat16)
+    xk = torch.randn(steps, B, d, device=dev, generator=gen).to(torch.bfloat16)
+    xv = torch.randn(steps, B, H, d, device=dev, generator=gen).to(torch.bfloat16)
+    od = torch.empty(steps, B, H, d, dtype=torch.bfloat16, device=dev)
+    pos = torch.full((B,), 1000, dtype=torch.int32, device=dev)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        rdm.rdm_ska_decode(xq[0], xk[0], xv[0], kc, vc, pos, o=od[0])
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            for s_ in range(steps):
+                rdm.rdm_ska_decode(xq[s_], xk[s_], xv[s_], kc, vc, pos, o=od[s_])
+    torch.cuda.current_stream().wait_stream(side)
+    t = time_steps(lambda: g.replay(), 5, 2)
+    ms = statistics.mean(t)
+    per = ms / steps
+    # per step: every cached key row once, every cached value row once, q, k, v
+    # in, o out, the new key and value rows written
+    by = 2 * (B * win * d + B * H * win * d + B * H * d * 3 + B * d * 2 + B * H * d)
+    out["ska_decode"] = {
+        "workload": f"SW-SKA decode B{B} H{H} d_k=d_v={d} window {win}, full rings, "
+                    f"{steps} steps per CUDA graph",
+        "value": B * steps / (ms / 1e3), "unit": "tokens/s", "ms_per_step": per,
+        "ms_per_graph": ms, "gpu_launches_per_step": 2, "cuda_graph": True,
+        "roofline": roofline(by, 2 * B * H * win * 2 * d, per, pk,
+                             ncu_counters("ska_decode_kernel", SKA_SRC, "ska4"), timed_alone=False)}
+    del g, kc, vc, xq, xk, xv, od
     return out
 
 

@@ -63,6 +63,18 @@ class ConvBwdArgs(ctypes.Structure):
                 ("grad_weight", _VP), ("grad_bias", _VP), ("grad_state_in", _VP)]
 
 
+class SkaFwdArgs(ctypes.Structure):
+    _fields_ = [("B", _I), ("H", _I), ("T", _I), ("dk", _I), ("dv", _I), ("window", _I),
+                ("scale", ctypes.c_float), ("dtype", _I), ("q", _VP), ("k", _VP), ("v", _VP),
+                ("o", _VP), ("k_cache", _VP), ("v_cache", _VP), ("pos", _VP)]
+
+
+class SkaDecodeArgs(ctypes.Structure):
+    _fields_ = [("B", _I), ("H", _I), ("dk", _I), ("dv", _I), ("window", _I),
+                ("scale", ctypes.c_float), ("dtype", _I), ("q", _VP), ("k", _VP), ("v", _VP),
+                ("k_cache", _VP), ("v_cache", _VP), ("pos", _VP), ("advance_pos", _I), ("o", _VP)]
+
+
 class RdmError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
@@ -75,7 +87,7 @@ EXPORTS = ["rdm_ddts_fwd", "rdm_ddts_fwd_workspace_size", "rdm_ddts_saved_states
            "rdm_ddts_bwd_workspace_size", "rdm_ddts_bwd_noalloc", "rdm_ddts_decode_step", "rdm_ddts_decode",
            "rdm_ddts_sync_status",
            "rdm_status_string", "rdm_ddts_set_test_hooks", "rdm_ddts_version", "rdm_shortconv_fwd",
-           "rdm_shortconv_bwd"]
+           "rdm_shortconv_bwd", "rdm_ska_fwd", "rdm_ska_decode"]
 
 
 def load():
@@ -110,6 +122,10 @@ def load():
         lib.rdm_shortconv_fwd.restype = _I
         lib.rdm_shortconv_bwd.argtypes = [ctypes.POINTER(ConvBwdArgs), _VP]
         lib.rdm_shortconv_bwd.restype = _I
+        lib.rdm_ska_fwd.argtypes = [ctypes.POINTER(SkaFwdArgs), _VP]
+        lib.rdm_ska_fwd.restype = _I
+        lib.rdm_ska_decode.argtypes = [ctypes.POINTER(SkaDecodeArgs), _VP]
+        lib.rdm_ska_decode.restype = _I
         lib.rdm_ddts_set_test_hooks.argtypes = [ctypes.c_longlong, _I]
         lib.rdm_ddts_set_test_hooks.restype = _I
         lib.rdm_ddts_version.argtypes = []
@@ -335,6 +351,42 @@ def rdm_shortconv_bwd(x, weight, bias, state_in, grad_y, grad_state_out=None, *,
                     _ptr(out["dxs"]))
     _check(load().rdm_shortconv_bwd(ctypes.byref(a), _stream(stream)), "rdm_shortconv_bwd")
     return out
+
+
+def rdm_ska_fwd(q, k, v, window, *, scale=0.0, o=None, k_cache=None, v_cache=None, pos=None,
+                stream=None):
+    """Sliding-window shared-key attention: q [B,H,T,dk], k [B,T,dk] (one key
+    row per token, shared by the heads), v [B,H,T,dv], all bf16; token t
+    attends to tokens t-window+1..t.  scale 0 means 1/sqrt(dk).  With k_cache
+    [B,window,dk] / v_cache [B,H,window,dv] / pos [B] int32 given, the last
+    min(T, window) keys and values are written to slot (position mod window)
+    and pos is set to T.  Returns o [B,H,T,dv]."""
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    if o is None:
+        o = torch.empty(B, H, T, dv, dtype=q.dtype, device=q.device)
+    a = SkaFwdArgs(B, H, T, dk, dv, int(window), float(scale), _dtype_code(q), _ptr(q), _ptr(k),
+                   _ptr(v), _ptr(o), _ptr(k_cache), _ptr(v_cache), _ptr(pos))
+    _check(load().rdm_ska_fwd(ctypes.byref(a), _stream(stream)), "rdm_ska_fwd")
+    return o
+
+
+def rdm_ska_decode(q, k, v, k_cache, v_cache, pos, *, scale=0.0, advance_pos=True, o=None,
+                   stream=None):
+    """One SW-SKA decode step against ring caches: q [B,H,dk], k [B,dk], v
+    [B,H,dv] bf16; k_cache [B,window,dk], v_cache [B,H,window,dv] updated in
+    place; pos [B] int32 tokens seen before this one (incremented when
+    advance_pos).  Returns o [B,H,dv]."""
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    window = k_cache.shape[1]
+    if o is None:
+        o = torch.empty(B, H, dv, dtype=q.dtype, device=q.device)
+    a = SkaDecodeArgs(B, H, dk, dv, int(window), float(scale), _dtype_code(q), _ptr(q), _ptr(k),
+                      _ptr(v), _ptr(k_cache), _ptr(v_cache), _ptr(pos), int(bool(advance_pos)),
+                      _ptr(o))
+    _check(load().rdm_ska_decode(ctypes.byref(a), _stream(stream)), "rdm_ska_decode")
+    return o
 
 
 def rdm_ddts_sync_status(stream=None) -> int:

@@ -9,6 +9,7 @@
 #include "../../include/rdm_ddts.h"
 #include "launch.h"
 #include "rdm_common.cuh"
+#include "ska_launch.h"
 
 namespace rdm {
 
@@ -295,6 +296,62 @@ rdm_status rdm_shortconv_bwd(const rdm_shortconv_bwd_args* a, rdm_stream_t strea
     return from_cuda(launch_conv_bwd(p, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+static bool ska_dim_ok(int d) { return d == 64 || d == 128; }
+
+static float ska_scale(float scale, int dk) {
+    return scale == 0.0f ? 1.0f / sqrtf((float)dk) : scale;
+}
+
+rdm_status rdm_ska_fwd(const rdm_ska_fwd_args* a, rdm_stream_t stream) {
+    if (!a || a->B < 1 || a->H < 1 || a->T < 0 || a->window < 1) return RDM_ERR_INVALID_ARG;
+    if (!(a->scale >= 0.0f) || isinf(a->scale)) return RDM_ERR_INVALID_ARG;
+    if (a->dtype != RDM_BF16) return a->dtype == RDM_F32 ? RDM_ERR_UNSUPPORTED : RDM_ERR_INVALID_ARG;
+    if (!ska_dim_ok(a->dk) || !ska_dim_ok(a->dv)) return RDM_ERR_UNSUPPORTED;
+    if ((double)a->B * a->H * ((a->T + 127) / 128) > 2.0e9 || a->T > (1 << 30))
+        return RDM_ERR_INVALID_ARG;
+    if (a->T > 0 && (!a->q || !a->k || !a->v || !a->o)) return RDM_ERR_INVALID_ARG;
+    if (!opt_aligned(a->q) || !opt_aligned(a->k) || !opt_aligned(a->v) || !opt_aligned(a->o) ||
+        !opt_aligned(a->k_cache) || !opt_aligned(a->v_cache) ||
+        (reinterpret_cast<uintptr_t>(a->pos) & 3u) != 0)
+        return RDM_ERR_INVALID_ARG;
+    if (a->T > 0 && ((a->k_cache && !a->k) || (a->v_cache && !a->v))) return RDM_ERR_INVALID_ARG;
+    unsigned* err = status_word();
+    if (!err) return RDM_ERR_CUDA;
+    SkaParams p;
+    memset(&p, 0, sizeof(p));
+    p.B = a->B; p.H = a->H; p.T = a->T; p.dk = a->dk; p.dv = a->dv; p.window = a->window;
+    p.scale = ska_scale(a->scale, a->dk);
+    p.q = a->q; p.k = a->k; p.v = a->v; p.o = a->o;
+    p.k_cache = a->T > 0 ? a->k_cache : nullptr;
+    p.v_cache = a->T > 0 ? a->v_cache : nullptr;
+    p.pos = a->pos;
+    p.err = err;
+    p.wait_limit = wait_limit();
+    return from_cuda(launch_ska_fwd(p, static_cast<cudaStream_t>(stream)));
+}
+
+rdm_status rdm_ska_decode(const rdm_ska_decode_args* a, rdm_stream_t stream) {
+    if (!a || a->B < 1 || a->H < 1 || a->window < 1 || a->window > 32768) return RDM_ERR_INVALID_ARG;
+    if (!(a->scale >= 0.0f) || isinf(a->scale)) return RDM_ERR_INVALID_ARG;
+    if (a->dtype != RDM_BF16) return a->dtype == RDM_F32 ? RDM_ERR_UNSUPPORTED : RDM_ERR_INVALID_ARG;
+    if (!ska_dim_ok(a->dk) || !ska_dim_ok(a->dv)) return RDM_ERR_UNSUPPORTED;
+    if ((double)a->B * a->H > 2.0e9) return RDM_ERR_INVALID_ARG;
+    if (!a->q || !a->k || !a->v || !a->k_cache || !a->v_cache || !a->pos || !a->o)
+        return RDM_ERR_INVALID_ARG;
+    if (!aligned(a->q) || !aligned(a->k) || !aligned(a->v) || !aligned(a->k_cache) ||
+        !aligned(a->v_cache) || !aligned(a->o) || (reinterpret_cast<uintptr_t>(a->pos) & 3u) != 0)
+        return RDM_ERR_INVALID_ARG;
+    SkaDecodeParams p;
+    memset(&p, 0, sizeof(p));
+    p.B = a->B; p.H = a->H; p.dk = a->dk; p.dv = a->dv; p.window = a->window;
+    p.scale = ska_scale(a->scale, a->dk);
+    p.q = a->q; p.k = a->k; p.v = a->v; p.k_cache = a->k_cache; p.v_cache = a->v_cache;
+    p.pos = a->pos; p.advance = a->advance_pos != 0; p.o = a->o;
+    p.err = status_word();
+    if (!p.err) return RDM_ERR_CUDA;
+    return from_cuda(launch_ska_decode(p, static_cast<cudaStream_t>(stream)));
+}
+
 rdm_status rdm_ddts_sync_status(rdm_stream_t stream) {
     cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return RDM_ERR_CUDA;
@@ -307,6 +364,7 @@ rdm_status rdm_ddts_sync_status(rdm_stream_t stream) {
         if (cudaMemcpy(w, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
             return RDM_ERR_CUDA;
         if (h & kErrTimeout) return RDM_ERR_TIMEOUT;
+        if (h & kErrBadValue) return RDM_ERR_INVALID_ARG;
     }
     return RDM_OK;
 }
@@ -331,6 +389,6 @@ rdm_status rdm_ddts_set_test_hooks(long long wait_limit_cycles, int withhold_seg
     return RDM_OK;
 }
 
-int rdm_ddts_version(void) { return 600; }
+int rdm_ddts_version(void) { return 700; }
 
 }  // extern "C"

@@ -1,0 +1,529 @@
+// ska.cu -- sliding-window shared-key attention (SW-SKA), the attention half of
+// the Rodimus+ block ("Rodimus*: Breaking the Accuracy-Efficiency Trade-Off with
+// Efficient Attentions"; digest.lyk-ai.com summary, "Method", Rodimus+ bullets:
+// a sliding window for local context, one key shared by every head so the KV
+// cache shrinks; paperhub.cn OpenReview rebuttal, answer to Q1: multi-head
+// query and value projections, a multi-query key projection).  Per batch b,
+// head h, token t:
+//
+//   s_u = scale * q[b,h,t] . k[b,u]   for u = max(0, t-w+1) .. t
+//   o[b,h,t] = sum_u softmax(s)_u v[b,h,u]
+//
+// Forward (tensor cores, bf16 in, fp32 accumulation): one CTA per (b, h, tile
+// of 128 queries).  TMA brings the query tile once and the key and value tiles
+// of the window through a two-stage ring (128-byte swizzle, used by the MMA as
+// is); tcgen05 computes S = Q K^T into TMEM, four softmax warps (one query row
+// per thread) mask the window, keep the running row maximum and sum, write
+// P = 2^(S*c - m) as bf16 into shared memory, and tcgen05 computes P V into a
+// second TMEM buffer, which the same threads fold into registers with the
+// rescale exp2(m_old - m_new).  Issue order S_n, PV_{n-1} lets the softmax of
+// tile n overlap the P V product of tile n-1.
+//
+// Decode: one CTA per (b, h) against ring caches (position p in slot p mod w):
+// the new key and value are written to their slot and used from the inputs,
+// scores go through shared memory, then a coalesced sweep over the value rows.
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "launch.h"
+#include "rdm_common.cuh"
+#include "ska_launch.h"
+#include "tc_common.cuh"
+
+namespace rdm {
+
+using namespace tc;
+
+namespace {
+
+constexpr int kQRows = 128;          // queries per CTA (MMA M)
+constexpr int kSoftWarps = 4;        // one query row per thread
+constexpr int kProdWarp = 4, kMmaWarp = 5;
+constexpr int kSkaThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+
+// 128-byte-swizzle shared-memory descriptor (sm_100 layout type 2): K-major
+// tiles of 64-element (128-byte) rows in 8-row, 1024-byte atoms, or MN-major
+// tiles whose 64-element rows run along M/N.
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    return sdesc(saddr, lbo, sbo) | (2ull << 61);
+}
+
+template <int DK, int DV>
+struct SkaCfg {
+    static constexpr int NK = DV == 128 ? 64 : 128;  // keys per tile (MMA N of S, K of P V)
+    static constexpr int Q_BYTES = kQRows * DK * 2;
+    static constexpr int K_BYTES = NK * DK * 2;
+    static constexpr int V_BYTES = NK * DV * 2;
+    static constexpr int P_BYTES = kQRows * NK * 2;
+    static_assert(2 * NK + 2 * DV <= (int)kTmemCols, "TMEM budget");
+};
+
+template <int DK, int DV>
+struct SkaSmem {
+    using K = SkaCfg<DK, DV>;
+    alignas(1024) uint8_t q[K::Q_BYTES];
+    alignas(1024) uint8_t k[2][K::K_BYTES];
+    alignas(1024) uint8_t v[2][K::V_BYTES];
+    alignas(1024) uint8_t p[2][K::P_BYTES];  // no-swizzle K-major (8x8 core matrices)
+    uint64_t q_full, k_full[2], v_full[2], kv_empty[2];
+    uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2], o_full[2], o_empty[2], mma_done;
+    uint32_t tmem_base;
+    int fail;
+};
+
+struct SkaKernelArgs {
+    SkaParams p;
+    CUtensorMap mq, mk, mv;
+};
+
+// Warp-uniform bounded wait: every lane waits, then the warp agrees; a lane
+// that saw the failure flag makes the whole warp give up together (the tcgen05
+// loads that follow are warp-collective).
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* fail,
+                                          long long limit) {
+    const bool ok = mbar_wait(bar, parity, fail, limit);
+    return __all_sync(0xffffffffu, ok);
+}
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(kSkaThreads, 1) ska_fwd_kernel(const __grid_constant__ SkaKernelArgs A) {
+    using K = SkaCfg<DK, DV>;
+    constexpr int NK = K::NK;
+    extern __shared__ __align__(1024) uint8_t smem_dyn[];
+    SkaSmem<DK, DV>& sm = *reinterpret_cast<SkaSmem<DK, DV>*>(
+        smem_dyn + ((1024u - (smem_u32(smem_dyn) & 1023u)) & 1023u));
+    const SkaParams& p = A.p;
+    const long long WL = p.wait_limit > 0 ? p.wait_limit : kDefaultWaitLimit;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int T = p.T, NQ = (T + kQRows - 1) / kQRows;
+    // heads of one (b, query tile) are adjacent in launch order: they read the
+    // same shared key tiles, which then come from L2
+    const int h = blockIdx.x % p.H;
+    const int qt = (blockIdx.x / p.H) % NQ;
+    const int b = blockIdx.x / (p.H * NQ);
+    const int bh = b * p.H + h;
+    const int t0 = qt * kQRows;
+    const int lo0 = t0 - p.window + 1;  // first key any row of the tile can see
+    const int j_lo = (lo0 > 0 ? lo0 : 0) / NK;
+    const int j_hi = min(t0 + kQRows - 1, T - 1) / NK;
+    const int NT = j_hi - j_lo + 1;  // key tiles
+
+    if (threadIdx.x == 0) {
+        mbar_init(&sm.q_full, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&sm.k_full[s], 1);
+            mbar_init(&sm.v_full[s], 1);
+            mbar_init(&sm.kv_empty[s], 1);
+            mbar_init(&sm.s_full[s], 1);
+            mbar_init(&sm.s_empty[s], kSoftWarps);
+            mbar_init(&sm.p_full[s], kSoftWarps);
+            mbar_init(&sm.p_empty[s], 1);
+            mbar_init(&sm.o_full[s], 1);
+            mbar_init(&sm.o_empty[s], kSoftWarps);
+        }
+        mbar_init(&sm.mma_done, 1);
+        sm.fail = 0;
+        fence_mbar_init();
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc(&sm.tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    if (warp == kProdWarp && lane == 0) {
+        prefetch_tmap(&A.mq); prefetch_tmap(&A.mk); prefetch_tmap(&A.mv);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    const uint32_t tS = tmem, tO = tmem + 2 * NK;  // S buffers, then P V buffers
+    volatile int* fail = &sm.fail;
+
+    if (warp == kProdWarp) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            mbar_expect_tx(&sm.q_full, K::Q_BYTES);
+#pragma unroll
+            for (int x = 0; x < DK / 64; ++x)
+                tma_load_3d(sm.q + x * kQRows * 128, &A.mq, &sm.q_full, 64 * x, t0, bh);
+            int last[2] = {-1, -1};
+            for (int n = 0; n < NT; ++n) {
+                const int st = n & 1;
+                if (!mbar_wait(&sm.kv_empty[st], ((n >> 1) & 1) ^ 1, fail, WL)) break;
+                const int kb = (j_lo + n) * NK;
+                mbar_expect_tx(&sm.k_full[st], K::K_BYTES);
+#pragma unroll
+                for (int x = 0; x < DK / 64; ++x)
+                    tma_load_3d(sm.k[st] + x * NK * 128, &A.mk, &sm.k_full[st], 64 * x, kb, b);
+                mbar_expect_tx(&sm.v_full[st], K::V_BYTES);
+#pragma unroll
+                for (int x = 0; x < DV / 64; ++x)
+                    tma_load_3d(sm.v[st] + x * NK * 128, &A.mv, &sm.v_full[st], 64 * x, kb, bh);
+                last[st] = n;
+            }
+            // no copy may land after the CTA has gone: wait (bounded, on our own
+            // clock) for the last ones issued into each stage and for the query
+            mbar_wait_own(&sm.q_full, 0, fail, WL);
+            for (int st = 0; st < 2; ++st)
+                if (last[st] >= 0) {
+                    mbar_wait_own(&sm.k_full[st], (last[st] >> 1) & 1, fail, WL);
+                    mbar_wait_own(&sm.v_full[st], (last[st] >> 1) & 1, fail, WL);
+                }
+        }
+        __syncwarp();
+    } else if (warp == kMmaWarp) {
+        // ----------------------------------------------------------------- MMA
+        if (lane == 0) {
+            constexpr uint32_t idS = idesc_bf16(kQRows, NK, 0, 0);  // S = Q K^T
+            constexpr uint32_t idO = idesc_bf16(kQRows, DV, 0, 1);  // O = P V (V MN-major)
+            const uint32_t qa = smem_u32(sm.q);
+            auto pv = [&](int m) -> bool {
+                const int st = m & 1;
+                const uint32_t ph = (m >> 1) & 1;
+                if (!mbar_wait(&sm.p_full[st], ph, fail, WL)) return false;
+                if (!mbar_wait(&sm.o_empty[st], ph ^ 1, fail, WL)) return false;
+                if (!mbar_wait(&sm.v_full[st], ph, fail, WL)) return false;
+                tc_fence_after();
+                const uint32_t pa = smem_u32(sm.p[st]), va = smem_u32(sm.v[st]);
+#pragma unroll
+                for (int ks = 0; ks < NK / 16; ++ks)
+                    mma_bf16(tO + st * DV, sdesc(pa + ks * 256, 128, NK * 16),
+                             sdesc_sw128(va + ks * 2048, NK * 128, 1024), idO, ks > 0);
+                mma_commit(&sm.o_full[st]);
+                mma_commit(&sm.kv_empty[st]);
+                mma_commit(&sm.p_empty[st]);
+                return true;
+            };
+            bool ok = mbar_wait(&sm.q_full, 0, fail, WL);
+            for (int n = 0; ok && n < NT; ++n) {
+                const int st = n & 1;
+                const uint32_t ph = (n >> 1) & 1;
+                if (!mbar_wait(&sm.k_full[st], ph, fail, WL) ||
+                    !mbar_wait(&sm.s_empty[st], ph ^ 1, fail, WL)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t ka = smem_u32(sm.k[st]);
+#pragma unroll
+                for (int ks = 0; ks < DK / 16; ++ks) {
+                    const int x = ks / 4, off = (ks % 4) * 32;
+                    mma_bf16(tS + st * NK, sdesc_sw128(qa + x * kQRows * 128 + off, 16, 1024),
+                             sdesc_sw128(ka + x * NK * 128 + off, 16, 1024), idS, ks > 0);
+                }
+                mma_commit(&sm.s_full[st]);
+                if (n > 0) ok = pv(n - 1);
+            }
+            if (ok && NT > 0) pv(NT - 1);
+            // every MMA issued has finished before TMEM is released
+            mma_commit(&sm.mma_done);
+            mbar_wait_own(&sm.mma_done, 0, fail, WL);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------- softmax
+        const int r = warp * 32 + lane;  // query row = TMEM lane
+        const int t = t0 + r;
+        const int lo = t - p.window + 1, hi = min(t, T - 1);
+        const float c = p.scale * kLog2e;
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        float o[DV];
+#pragma unroll
+        for (int j = 0; j < DV; ++j) o[j] = 0.0f;
+        float m_run = -INFINITY, l = 0.0f, corr_pending = 1.0f;
+        auto fold = [&](int i, float cr) -> bool {
+            const int st = i & 1;
+            if (!warp_wait(&sm.o_full[st], (i >> 1) & 1, fail, WL)) return false;
+            tc_fence_after();
+            float x[DV];
+#pragma unroll
+            for (int q32 = 0; q32 < DV / 32; ++q32)
+                tmem_ld32(tO + st * DV + lane_off + q32 * 32, x + q32 * 32);
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.o_empty[st]);
+#pragma unroll
+            for (int j = 0; j < DV; ++j) o[j] = fmaf(o[j], cr, x[j]);
+            return true;
+        };
+        bool ok = true;
+        for (int n = 0; n < NT; ++n) {
+            const int st = n & 1;
+            const uint32_t ph = (n >> 1) & 1;
+            if (!warp_wait(&sm.s_full[st], ph, fail, WL)) { ok = false; break; }
+            tc_fence_after();
+            float s[NK];
+#pragma unroll
+            for (int q32 = 0; q32 < NK / 32; ++q32)
+                tmem_ld32(tS + st * NK + lane_off + q32 * 32, s + q32 * 32);
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.s_empty[st]);
+            const int kb = (j_lo + n) * NK;
+            if (kb < lo || kb + NK - 1 > hi) {
+#pragma unroll
+                for (int i = 0; i < NK; ++i)
+                    if (kb + i < lo || kb + i > hi) s[i] = -INFINITY;
+            }
+            float mx = s[0];
+#pragma unroll
+            for (int i = 1; i < NK; ++i) mx = fmaxf(mx, s[i]);
+            const float m_new = fmaxf(m_run, mx * c);
+            const float m_use = m_new == -INFINITY ? 0.0f : m_new;
+            const float corr = ex2_fast(m_run - m_use);
+            float sum = 0.0f;
+#pragma unroll
+            for (int i = 0; i < NK; ++i) {
+                s[i] = ex2_fast(fmaf(s[i], c, -m_use));
+                sum += s[i];
+            }
+            l = fmaf(l, corr, sum);
+            m_run = m_new;
+            if (!warp_wait(&sm.p_empty[st], ph ^ 1, fail, WL)) { ok = false; break; }
+            // P row r, keys 8*kc .. 8*kc+7 -> core matrix (r/8, kc): byte
+            // (r/8)*(NK*16) + kc*128 + (r%8)*16
+            uint8_t* prow = sm.p[st] + (r >> 3) * (NK * 16) + (r & 7) * 16;
+#pragma unroll
+            for (int kc = 0; kc < NK / 8; ++kc)
+                *reinterpret_cast<uint4*>(prow + kc * 128) = pack8(s + 8 * kc);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.p_full[st]);
+            if (n > 0 && !fold(n - 1, corr_pending)) { ok = false; break; }
+            corr_pending = corr;
+        }
+        if (ok && NT > 0) ok = fold(NT - 1, corr_pending);
+        if (ok && t < T) {
+            const float inv = l > 0.0f ? 1.0f / l : 0.0f;
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) +
+                                                  ((size_t)bh * T + t) * DV);
+#pragma unroll
+            for (int j8 = 0; j8 < DV / 8; ++j8) {
+                float y[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) y[e] = o[8 * j8 + e] * inv;
+                dst[j8] = pack8(y);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+    if (threadIdx.x == 0 && sm.fail) atomicOr(p.err, kErrTimeout);
+}
+
+// Ring-cache fill after a forward over positions 0..T-1: the last min(T, w)
+// keys and values go to slot (position mod w); pos[b] = T.  One thread per
+// 16-byte piece of a row.
+__global__ void ska_cache_fill_kernel(const SkaParams p) {
+    const int n = min(p.T, p.window);
+    const int kp = p.dk / 8, vp = p.dv / 8;  // 16-byte pieces per row
+    const long long nk = p.k_cache ? (long long)p.B * n * kp : 0;
+    const long long nv = p.v_cache ? (long long)p.B * p.H * n * vp : 0;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < nk + nv;
+         i += (long long)gridDim.x * blockDim.x) {
+        if (i < nk) {
+            const int x = (int)(i % kp);
+            const long long row = i / kp;
+            const int b = (int)(row / n), u = (int)(row % n);
+            const int pos = p.T - n + u, slot = pos % p.window;
+            const uint4* src = reinterpret_cast<const uint4*>(p.k) + ((size_t)b * p.T + pos) * kp + x;
+            reinterpret_cast<uint4*>(p.k_cache)[((size_t)b * p.window + slot) * kp + x] = __ldg(src);
+        } else {
+            const long long j = i - nk;
+            const int x = (int)(j % vp);
+            const long long row = j / vp;
+            const long long bh = row / n;
+            const int u = (int)(row % n);
+            const int pos = p.T - n + u, slot = pos % p.window;
+            const uint4* src = reinterpret_cast<const uint4*>(p.v) + ((size_t)bh * p.T + pos) * vp + x;
+            reinterpret_cast<uint4*>(p.v_cache)[((size_t)bh * p.window + slot) * vp + x] = __ldg(src);
+        }
+    }
+    if (p.pos && blockIdx.x == 0)
+        for (int b = threadIdx.x; b < p.B; b += blockDim.x) p.pos[b] = p.T;
+}
+
+// ------------------------------------------------------------------ decode
+constexpr int kDecThreads = 256;
+
+__device__ __forceinline__ float block_reduce(float x, float* red, bool is_max) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float y = __shfl_xor_sync(0xffffffffu, x, o);
+        x = is_max ? fmaxf(x, y) : x + y;
+    }
+    __syncthreads();  // red may still be read from the previous reduction
+    if (lane == 0) red[warp] = x;
+    __syncthreads();
+    x = red[0];
+#pragma unroll
+    for (int w = 1; w < kDecThreads / 32; ++w) x = is_max ? fmaxf(x, red[w]) : x + red[w];
+    return x;
+}
+
+// One CTA per (b, h).  Valid slots are 0..n-1 with n = min(pos+1, w) (before
+// the ring is full, slot = position); the current token's slot takes the new
+// key and value from the inputs, and this CTA writes them into the caches (the
+// key by head 0 only; no other CTA reads that slot from the cache).
+template <int DK, int DV>
+__global__ void __launch_bounds__(kDecThreads) ska_decode_kernel(const SkaDecodeParams p) {
+    extern __shared__ float dsm[];
+    float* sc = dsm;                       // [w] scores, then weights
+    float* part = dsm + p.window;          // [16][DV] partial outputs
+    __shared__ float qs[DK];
+    __shared__ float red[kDecThreads / 32];
+    const int bh = blockIdx.x, b = bh / p.H, h = bh % p.H;
+    const int pos = p.pos[b];
+    if (pos < 0) {  // the whole CTA leaves; nothing is read or written
+        if (threadIdx.x == 0) atomicOr(p.err, kErrBadValue);
+        return;
+    }
+    const int w = p.window, n = min(pos + 1, w), cur = pos % w;
+    const __nv_bfloat16* kin = static_cast<const __nv_bfloat16*>(p.k) + (size_t)b * DK;
+    const __nv_bfloat16* vin = static_cast<const __nv_bfloat16*>(p.v) + (size_t)bh * DV;
+    const __nv_bfloat16* kc = static_cast<const __nv_bfloat16*>(p.k_cache) + (size_t)b * w * DK;
+    const __nv_bfloat16* vc = static_cast<const __nv_bfloat16*>(p.v_cache) + (size_t)bh * w * DV;
+    const float c = p.scale * kLog2e;
+    for (int i = threadIdx.x; i < DK; i += kDecThreads)
+        qs[i] = __bfloat162float(static_cast<const __nv_bfloat16*>(p.q)[(size_t)bh * DK + i]) * c;
+    // write the new token into its slot
+    if (h == 0)
+        for (int i = threadIdx.x; i < DK / 8; i += kDecThreads)
+            reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.k_cache) +
+                                     ((size_t)b * w + cur) * DK)[i] = reinterpret_cast<const uint4*>(kin)[i];
+    for (int i = threadIdx.x; i < DV / 8; i += kDecThreads)
+        reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.v_cache) +
+                                 ((size_t)bh * w + cur) * DV)[i] = reinterpret_cast<const uint4*>(vin)[i];
+    __syncthreads();
+    // scores (log2 units): one slot per thread, the key row read in 16-byte pieces
+    float mx = -INFINITY;
+    for (int u = threadIdx.x; u < n; u += kDecThreads) {
+        const uint4* kr = reinterpret_cast<const uint4*>(u == cur ? kin : kc + (size_t)u * DK);
+        float a = 0.0f;
+#pragma unroll
+        for (int x = 0; x < DK / 8; ++x) {
+            float f[8];
+            unpack8(__ldg(kr + x), f);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) a = fmaf(qs[8 * x + e], f[e], a);
+        }
+        sc[u] = a;
+        mx = fmaxf(mx, a);
+    }
+    mx = block_reduce(mx, red, true);
+    float sum = 0.0f;
+    for (int u = threadIdx.x; u < n; u += kDecThreads) {
+        const float e = ex2_fast(sc[u] - mx);
+        sc[u] = e;
+        sum += e;
+    }
+    sum = block_reduce(sum, red, false);  // its first barrier also publishes sc
+    // weighted sum of value rows: thread = (slot lane g, 8-column piece x)
+    constexpr int XP = DV / 8, G = kDecThreads / XP;
+    const int x = threadIdx.x % XP, g = threadIdx.x / XP;
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+    const uint4* vbase = reinterpret_cast<const uint4*>(vc);
+#pragma unroll 4
+    for (int u = g; u < n; u += G) {
+        const uint4 wv = u == cur ? reinterpret_cast<const uint4*>(vin)[x] : __ldg(vbase + (size_t)u * XP + x);
+        float f[8];
+        unpack8(wv, f);
+        const float pu = sc[u];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = fmaf(pu, f[e], acc[e]);
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) part[g * DV + 8 * x + e] = acc[e];
+    __syncthreads();
+    const float inv = 1.0f / sum;
+    for (int j = threadIdx.x; j < DV; j += kDecThreads) {
+        float a = 0.0f;
+        for (int gg = 0; gg < G; ++gg) a += part[gg * DV + j];
+        static_cast<__nv_bfloat16*>(p.o)[(size_t)bh * DV + j] = __float2bfloat16_rn(a * inv);
+    }
+}
+
+__global__ void ska_advance_kernel(int* pos, int B) {
+    const int b = blockIdx.x * blockDim.x + threadIdx.x;
+    if (b < B) pos[b] += 1;
+}
+
+template <int DK, int DV>
+cudaError_t launch_fwd_cfg(const SkaParams& p, cudaStream_t s) {
+    using Kc = SkaCfg<DK, DV>;
+    SkaKernelArgs a;
+    a.p = p;
+    const uint64_t BH = (uint64_t)p.B * p.H;
+    if (!make_tmap_bf16_3d(&a.mq, p.q, DK, p.T, BH, 64, kQRows) ||
+        !make_tmap_bf16_3d(&a.mk, p.k, DK, p.T, p.B, 64, Kc::NK) ||
+        !make_tmap_bf16_3d(&a.mv, p.v, DV, p.T, BH, 64, Kc::NK))
+        return cudaErrorInvalidValue;
+    const size_t smem = sizeof(SkaSmem<DK, DV>) + 1024;
+    auto kern = ska_fwd_kernel<DK, DV>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = (unsigned)(BH * ((p.T + kQRows - 1) / kQRows));
+    kern<<<grid, kSkaThreads, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
+template <int DK, int DV>
+cudaError_t launch_dec_cfg(const SkaDecodeParams& p, cudaStream_t s) {
+    constexpr int G = kDecThreads / (DV / 8);
+    const size_t smem = ((size_t)p.window + (size_t)G * DV) * 4;
+    auto kern = ska_decode_kernel<DK, DV>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<(unsigned)(p.B * p.H), kDecThreads, smem, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t ska_decode_smem(int window, int dv) {
+    return ((size_t)window + (size_t)(kDecThreads / (dv / 8)) * dv) * 4;
+}
+
+cudaError_t launch_ska_fwd(const SkaParams& p, cudaStream_t s) {
+    cudaError_t e = cudaSuccess;
+    if (p.T > 0) {
+        if (p.dk == 64)
+            e = p.dv == 64 ? launch_fwd_cfg<64, 64>(p, s) : launch_fwd_cfg<64, 128>(p, s);
+        else
+            e = p.dv == 64 ? launch_fwd_cfg<128, 64>(p, s) : launch_fwd_cfg<128, 128>(p, s);
+        if (e != cudaSuccess) return e;
+    }
+    if (p.k_cache || p.v_cache || p.pos) {
+        const long long n = p.T < p.window ? p.T : p.window;
+        const long long work = (long long)p.B * n * (p.dk / 8 + (long long)p.H * (p.dv / 8));
+        const long long blocks = (work + 255) / 256;
+        const unsigned grid = (unsigned)(blocks < 1 ? 1 : blocks > 4 * 148 * 8 ? 4 * 148 * 8 : blocks);
+        ska_cache_fill_kernel<<<grid, 256, 0, s>>>(p);
+        e = cudaGetLastError();
+    }
+    return e;
+}
+
+cudaError_t launch_ska_decode(const SkaDecodeParams& p, cudaStream_t s) {
+    cudaError_t e;
+    if (p.dk == 64)
+        e = p.dv == 64 ? launch_dec_cfg<64, 64>(p, s) : launch_dec_cfg<64, 128>(p, s);
+    else
+        e = p.dv == 64 ? launch_dec_cfg<128, 64>(p, s) : launch_dec_cfg<128, 128>(p, s);
+    if (e != cudaSuccess || !p.advance) return e;
+    ska_advance_kernel<<<(p.B + 255) / 256, 256, 0, s>>>(p.pos, p.B);
+    return cudaGetLastError();
+}
+
+}  // namespace rdm

@@ -114,3 +114,13 @@ def draw_decode(B, H, dk, dv, steps, dtype=torch.bfloat16, seed=BASE_SEED + 4, m
     beta = torch.sigmoid(torch.randn(steps, B, H, dv, **f32))
     out = dict(q=q, k=k, v=v, g=g, tau=tau, beta=beta)
     return {n: t.to(dtype).contiguous() for n, t in out.items()}
+
+
+# Sliding-window shared-key attention (the attention half of the Rodimus+ block;
+# the pages give neither its window nor its head sizes): a forward on a
+# 130M-scale layer, d_model 768 as 12 heads of 64 with one shared key head,
+# window 512 -- (B, H, T, d, window) -- and batched decode at the 1.6B scale,
+# d_model 2048 as 16 heads of 128, against full ring caches of 512 slots --
+# (B, H, d, window, steps per timed graph).  q, k, v ~ N(0, 1) in bf16.
+SKA_FWD = (8, 12, 2048, 64, 512)
+SKA_DEC = (256, 16, 128, 512, 64)

@@ -34,8 +34,8 @@
  *   - Domain: g >= 0, tau >= 0.  Values are not checked on the device;
  *     out-of-domain values give NaN as the formulas do.  0^0 = 1, 0^tau = 0.
  *   - Host-side validation failures return a status and launch nothing.
- *     Kernel-side failures (a bounded wait that ran out) set a device status
- *     word that rdm_ddts_sync_status reports.
+ *     Kernel-side failures (a bounded wait that ran out, a decode position
+ *     out of range) set a device status word that rdm_ddts_sync_status reports.
  *   - Supported sizes: d_k, d_v in {16, 32, 64, 128}; any T >= 0; B*H >= 1.
  *     The tensor-core path covers bf16 with d_k in {64, 128} and d_v in
  *     {64, 128} (d_v a multiple of the per-CTA tile); every other supported
@@ -309,6 +309,69 @@ typedef struct {
 } rdm_shortconv_bwd_args;
 
 rdm_status rdm_shortconv_bwd(const rdm_shortconv_bwd_args *args, rdm_stream_t stream);
+
+/* ------------------------------------------------------------------ SW-SKA
+ * Sliding-window shared-key attention, the attention half of the Rodimus+
+ * block (Rodimus* digest.lyk-ai.com summary, "Method", Rodimus+ bullets: a
+ * sliding window for local context and one key shared by all heads to shrink
+ * the KV cache; paperhub.cn OpenReview rebuttal, answer to Q1: multi-head query
+ * and value projections, a multi-query key projection).  The pages print
+ * neither the window nor the score scale; this library takes, per batch b,
+ * head h and token t,
+ *
+ *   s_u = scale * q[b,h,t] . k[b,u]      for u = max(0, t-window+1) .. t
+ *   o[b,h,t] = sum_u softmax(s)_u v[b,h,u]
+ *
+ * with one key row per token shared by every head, scale = 1/sqrt(d_k) when
+ * 0 is passed.
+ *
+ *   q : [B,H,T,d_k] bf16     k : [B,T,d_k] bf16     v, o : [B,H,T,d_v] bf16
+ *   d_k, d_v in {64, 128}; window >= 1; T >= 0; dtype must be RDM_BF16.
+ * Arithmetic: bf16 tensor-core products with float32 accumulation; the
+ * softmax weights enter the second product rounded to bf16.
+ *
+ * Decode keeps a ring KV cache of `window` slots: the token at position p
+ * (counted from 0 at the start of the sequence) lives in slot p mod window.
+ *   k_cache : [B,window,d_k] bf16     v_cache : [B,H,window,d_v] bf16
+ *   pos     : [B] int32, tokens of each sequence seen before this step
+ * The forward fills the caches from a prompt when k_cache / v_cache are given
+ * (the last min(T, window) keys and values at their slots) and sets pos[b] = T
+ * when pos is given.  A decode step writes the new key and value into slot
+ * pos[b] mod window, attends to positions max(0, pos-window+1) .. pos, and adds
+ * one to pos[b] when advance_pos != 0.  Sequences of one batch may be at
+ * different positions.  Decode takes window <= 32768.  A negative pos[b]
+ * leaves that sequence untouched and makes rdm_ddts_sync_status return
+ * RDM_ERR_INVALID_ARG.
+ * All pointers are device pointers, 16-byte aligned (pos: 4-byte aligned);
+ * outputs must not alias inputs; nothing is allocated.
+ */
+typedef struct {
+    int B, H, T, dk, dv, window;
+    float scale;                 /* > 0, or 0 for 1/sqrt(d_k) */
+    rdm_dtype dtype;
+    const void *q, *k, *v;
+    void *o;
+    void *k_cache;               /* NULL = not filled */
+    void *v_cache;               /* NULL = not filled */
+    int *pos;                    /* NULL = not written */
+} rdm_ska_fwd_args;
+
+rdm_status rdm_ska_fwd(const rdm_ska_fwd_args *args, rdm_stream_t stream);
+
+typedef struct {
+    int B, H, dk, dv, window;
+    float scale;                 /* > 0, or 0 for 1/sqrt(d_k) */
+    rdm_dtype dtype;
+    const void *q;               /* [B,H,d_k] */
+    const void *k;               /* [B,d_k] */
+    const void *v;               /* [B,H,d_v] */
+    void *k_cache, *v_cache;     /* updated in place */
+    int *pos;                    /* [B] int32 */
+    int advance_pos;             /* != 0: pos[b] += 1 after the step */
+    void *o;                     /* [B,H,d_v] */
+} rdm_ska_decode_args;
+
+rdm_status rdm_ska_decode(const rdm_ska_decode_args *args, rdm_stream_t stream);
 
 /* ------------------------------------------------------------------ status */
 

@@ -125,3 +125,38 @@ def test_test_hooks_validation(lib):
     assert lib.rdm_ddts_set_test_hooks(0, 2) == RDM_ERR_INVALID_ARG
     assert lib.rdm_ddts_set_test_hooks(1000, 1) == RDM_OK
     assert lib.rdm_ddts_set_test_hooks(0, 0) == RDM_OK
+
+
+def _ska_fwd(**kw):
+    from gated_linear_attention_ddts_b200._binding import SkaFwdArgs
+    fake = 1 << 20
+    base = dict(B=1, H=2, T=8, dk=64, dv=64, window=4, scale=0.0, dtype=1, q=fake, k=fake, v=fake,
+                o=fake, k_cache=None, v_cache=None, pos=None)
+    base.update(kw)
+    return SkaFwdArgs(**base)
+
+
+def _ska_dec(**kw):
+    from gated_linear_attention_ddts_b200._binding import SkaDecodeArgs
+    fake = 1 << 20
+    base = dict(B=1, H=2, dk=64, dv=64, window=4, scale=0.0, dtype=1, q=fake, k=fake, v=fake,
+                k_cache=fake, v_cache=fake, pos=fake, advance_pos=1, o=fake)
+    base.update(kw)
+    return SkaDecodeArgs(**base)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(window=0), 1), (dict(B=0), 1), (dict(T=-1), 1), (dict(scale=-1.0), 1),
+    (dict(scale=float("nan")), 1), (dict(scale=float("inf")), 1), (dict(dtype=0), 2),
+    (dict(dtype=5), 1), (dict(dk=32), 2), (dict(dv=16), 2), (dict(q=(1 << 20) + 8), 1),
+    (dict(o=None), 1), (dict(k_cache=(1 << 20) + 2), 1), (dict(pos=(1 << 20) + 2), 1)])
+def test_ska_fwd_validation(lib, kw, status):
+    assert lib.rdm_ska_fwd(ctypes.byref(_ska_fwd(**kw)), None) == status
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(window=0), 1), (dict(window=32769), 1), (dict(H=0), 1), (dict(scale=-2.0), 1),
+    (dict(dtype=0), 2), (dict(dk=16), 2), (dict(k_cache=None), 1), (dict(pos=None), 1),
+    (dict(v=(1 << 20) + 2), 1), (dict(o=None), 1)])
+def test_ska_decode_validation(lib, kw, status):
+    assert lib.rdm_ska_decode(ctypes.byref(_ska_dec(**kw)), None) == status
