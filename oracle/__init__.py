@@ -163,6 +163,37 @@ def bwd(q, k, v, g, tau, beta, S0, dO, dST=None, nthreads=None, lib=None, preact
     return out
 
 
+def lowrank_beta_pre(u, w_up):
+    """beta_hat's pre-activation from its low-rank factorisation (Rodimus*,
+    digest.lyk-ai.com summary, "Method": beta_hat is built from low-rank
+    matrices to cut parameters and filter input noise).  The reading: the
+    token's input projected down to rank r, u [B,T,r] (one row per token, shared
+    by the heads), times an up-projection w_up [H,r,dv] gives the
+    pre-activation [B,H,T,dv]; beta_hat = sigmoid of it."""
+    return np.einsum("btr,hrj->bhtj", _f64(u), _f64(w_up))
+
+
+def fwd_lowrank(q, k, v, g_pre, tau_pre, u, w_up, S0=None, nthreads=None, lib=None, d=None):
+    """Forward with every gate passed before its activation and beta_hat's
+    pre-activation given by its low-rank factors u [B,T,r], w_up [H,r,dv]."""
+    return fwd(q, k, v, g_pre, tau_pre, lowrank_beta_pre(u, w_up), S0, nthreads=nthreads, lib=lib,
+               preact=True, d=d)
+
+
+def bwd_lowrank(q, k, v, g_pre, tau_pre, u, w_up, S0, dO, dST=None, nthreads=None, lib=None, d=None):
+    """Reverse mode of fwd_lowrank: the gradient with respect to beta_hat's
+    pre-activation, db [B,H,T,dv], is contracted into du[b,t,:] = sum_h
+    w_up[h] db[b,h,t,:] and dw_up[h] = sum_{b,t} u[b,t,:]^T db[b,h,t,:]; the
+    dict has du and dw_up in place of dbeta."""
+    u, w_up = _f64(u), _f64(w_up)
+    out = bwd(q, k, v, g_pre, tau_pre, lowrank_beta_pre(u, w_up), S0, dO, dST, nthreads=nthreads,
+              lib=lib, preact=True, d=d)
+    db = out.pop("dbeta")
+    out["du"] = np.einsum("bhtj,hrj->btr", db, w_up)
+    out["dw_up"] = np.einsum("btr,bhtj->hrj", u, db)
+    return out
+
+
 def decode_step(q, k, v, g, tau, beta, S, nthreads=None, lib=None, d=None):
     """One token per (b,h).  q,k,g,tau [B,H,dk]; v,beta [B,H,dv]; S [B,H,dk,dv]
     float64 numpy, updated in place; d feedthrough [H,dv] or None.  Returns o [B,H,dv]."""

@@ -489,6 +489,67 @@ def check_conv_silu_and_grads(lib=None, seed=23):
 CONV_PINS = [check_conv_width_one, check_conv_numpy_convolve, check_conv_impulse_and_state,
              check_conv_silu_and_grads]
 
+# ------------------------------------------------------- low-rank beta_hat pins
+def lowrank_inputs(rng, B=2, H=3, T=7, dk=4, dv=6, r=5):
+    x = rand_inputs(rng, B, H, T, dk, dv)
+    x["g"] = rng.standard_normal(x["g"].shape) - 1.0   # pre-activations
+    x["tau"] = rng.standard_normal(x["tau"].shape)
+    u = rng.standard_normal((B, T, r))
+    w_up = rng.standard_normal((H, r, dv)) / np.sqrt(r)
+    return x, u, w_up
+
+
+def check_lowrank_rank_one_outer_product(lib=None, seed=40):
+    """Rank 1: u[b,t,0] = a[b,t] and w_up[h,0,j] = c[h,j] give the
+    pre-activation a[b,t] c[h,j] (an outer product, formed here with
+    numpy.multiply.outer); the forward equals the full-rank pre-activation
+    forward on it.  All axis lengths differ, so a swapped index changes shapes
+    or values."""
+    rng = np.random.default_rng(seed)
+    x, _, _ = lowrank_inputs(rng)
+    B, H, T, _ = x["q"].shape
+    dv = x["v"].shape[-1]
+    a = rng.standard_normal((B, T))
+    c = rng.standard_normal((H, dv))
+    pre = np.moveaxis(np.multiply.outer(a, c), 2, 1)            # [B,H,T,dv]
+    o_lr, S_lr = oracle.fwd_lowrank(x["q"], x["k"], x["v"], x["g"], x["tau"], a[..., None],
+                                    c[:, None, :], x["S0"], lib=lib)
+    o_fr, S_fr = oracle.fwd(x["q"], x["k"], x["v"], x["g"], x["tau"], pre, x["S0"], lib=lib,
+                            preact=True)
+    close(o_lr, o_fr, 1e-13, "rank-1 low-rank o")
+    close(S_lr, S_fr, 1e-13, "rank-1 low-rank S_T")
+
+
+def check_lowrank_finite_differences(lib=None, seed=41):
+    """du and dw_up against central differences of the forward's loss
+    sum(o * dO) + sum(S_T * dS_T)."""
+    rng = np.random.default_rng(seed)
+    x, u, w_up = lowrank_inputs(rng, T=5)
+    dO = rng.standard_normal(x["v"].shape)
+    dST = rng.standard_normal(x["S0"].shape)
+    gr = oracle.bwd_lowrank(x["q"], x["k"], x["v"], x["g"], x["tau"], u, w_up, x["S0"], dO, dST,
+                            lib=lib)
+
+    def loss(uu, ww):
+        o, ST = oracle.fwd_lowrank(x["q"], x["k"], x["v"], x["g"], x["tau"], uu, ww, x["S0"], lib=lib)
+        return float(np.sum(o * dO) + np.sum(ST * dST))
+
+    h = 1e-6
+    for idx in ((0, 0, 0), (1, 4, 3), (0, 2, 4)):
+        up, um = u.copy(), u.copy()
+        up[idx] += h
+        um[idx] -= h
+        close(gr["du"][idx], (loss(up, w_up) - loss(um, w_up)) / (2 * h), 1e-7, f"du {idx}")
+    for idx in ((0, 0, 0), (2, 4, 5), (1, 3, 2)):
+        wp, wm = w_up.copy(), w_up.copy()
+        wp[idx] += h
+        wm[idx] -= h
+        close(gr["dw_up"][idx], (loss(u, wp) - loss(u, wm)) / (2 * h), 1e-7, f"dw_up {idx}")
+
+
+LOWRANK_PINS = [check_lowrank_rank_one_outer_product, check_lowrank_finite_differences]
+
+
 # ------------------------------------------------------------------ SW-SKA pins
 def ska_inputs(rng, B=2, H=3, T=13, dk=4, dv=5):
     return dict(q=rng.standard_normal((B, H, T, dk)), k=rng.standard_normal((B, T, dk)),
@@ -602,4 +663,5 @@ SKA_PINS = [check_ska_hand_example, check_ska_window_one_and_uniform, check_ska_
 FORWARD_PINS = [check_worked_example, check_T1_closed_form, check_g_zero, check_tau_zero,
                 check_quadratic, check_linearity, check_split_and_decode]
 BACKWARD_PINS = [check_bwd_finite_differences, check_bwd_autograd]
-ALL_PINS = FORWARD_PINS + BACKWARD_PINS + PREACT_PINS + FEED_PINS + CONV_PINS + SKA_PINS
+ALL_PINS = (FORWARD_PINS + BACKWARD_PINS + PREACT_PINS + FEED_PINS + CONV_PINS + SKA_PINS +
+            LOWRANK_PINS)

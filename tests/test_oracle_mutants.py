@@ -4,6 +4,8 @@ one pin fails.  A pin set that let a mutant through would not pin the oracle."""
 import os
 import subprocess
 
+import numpy as np
+
 import pytest
 
 import oracle
@@ -97,3 +99,47 @@ def test_pins_catch_mutant(tmp_path, name, orig, slip, pins):
         except (AssertionError, RuntimeError, FloatingPointError, ValueError):
             caught.append(check.__name__)
     assert caught, f"mutant '{name}' passed every pin"
+
+
+# Slips in the oracle's Python-level low-rank beta_hat step (the C source is
+# untouched): each replaces one function for the duration of the check.
+def _lr_heads_reversed(u, w_up):
+    return np.einsum("btr,hrj->bhtj", oracle._f64(u), oracle._f64(w_up)[::-1])
+
+
+def _lr_bwd_one_head(q, k, v, g_pre, tau_pre, u, w_up, S0, dO, dST=None, nthreads=None, lib=None,
+                     d=None):
+    out = oracle.bwd(q, k, v, g_pre, tau_pre, oracle.lowrank_beta_pre(u, w_up), S0, dO, dST,
+                     lib=lib, preact=True)
+    db = out.pop("dbeta")
+    w = oracle._f64(w_up)
+    out["du"] = np.einsum("btj,rj->btr", db[:, 0], w[0]) * w.shape[0]
+    out["dw_up"] = np.einsum("btr,bhtj->hrj", oracle._f64(u), db)
+    return out
+
+
+def _lr_bwd_no_sigmoid_grad(q, k, v, g_pre, tau_pre, u, w_up, S0, dO, dST=None, nthreads=None,
+                            lib=None, d=None):
+    pre = oracle.lowrank_beta_pre(u, w_up)
+    out = oracle.bwd(q, k, v, g_pre, tau_pre, pre, S0, dO, dST, lib=lib, preact=True)
+    s = oracle.sigmoid(pre)
+    db = out.pop("dbeta") / (s * (1.0 - s))
+    out["du"] = np.einsum("bhtj,hrj->btr", db, oracle._f64(w_up))
+    out["dw_up"] = np.einsum("btr,bhtj->hrj", oracle._f64(u), db)
+    return out
+
+
+LOWRANK_SLIPS = [("lowrank_beta_pre", _lr_heads_reversed), ("bwd_lowrank", _lr_bwd_one_head),
+                 ("bwd_lowrank", _lr_bwd_no_sigmoid_grad)]
+
+
+@pytest.mark.parametrize("name,slip", LOWRANK_SLIPS, ids=[f.__name__ for _, f in LOWRANK_SLIPS])
+def test_lowrank_pins_catch_python_slip(monkeypatch, name, slip):
+    monkeypatch.setattr(oracle, name, slip)
+    caught = []
+    for check in P.LOWRANK_PINS:
+        try:
+            check()
+        except (AssertionError, ValueError):
+            caught.append(check.__name__)
+    assert caught, f"no low-rank pin caught the slip {slip.__name__}"
