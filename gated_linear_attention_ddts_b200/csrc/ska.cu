@@ -37,10 +37,13 @@ using namespace tc;
 namespace {
 
 constexpr int kQRows = 128;          // queries per CTA (MMA M)
-constexpr int kSoftWarps = 4;        // one query row per thread
-constexpr int kProdWarp = 4, kMmaWarp = 5;
-constexpr int kSkaThreads = 192;
-constexpr uint32_t kTmemCols = 512;
+// eight softmax warps: warps w and w + 4 share the TMEM lane quarter w % 4
+// (query rows 32 (w % 4) ..), each taking half of the key columns of S and
+// half of the output columns, so that two warps per scheduler interleave
+constexpr int kSoftWarps = 8;
+constexpr int kProdWarp = 8, kMmaWarp = 9;
+constexpr int kSkaThreads = 320;
+constexpr int kStages = 3;  // key and value tiles in flight
 
 // 128-byte-swizzle shared-memory descriptor (sm_100 layout type 2): K-major
 // tiles of 64-element (128-byte) rows in 8-row, 1024-byte atoms, or MN-major
@@ -51,23 +54,27 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
 
 template <int DK, int DV>
 struct SkaCfg {
-    static constexpr int NK = DV == 128 ? 64 : 128;  // keys per tile (MMA N of S, K of P V)
+    static constexpr int NK = 64;  // keys per tile (MMA N of S, K of P V)
     static constexpr int Q_BYTES = kQRows * DK * 2;
     static constexpr int K_BYTES = NK * DK * 2;
     static constexpr int V_BYTES = NK * DV * 2;
     static constexpr int P_BYTES = kQRows * NK * 2;
-    static_assert(2 * NK + 2 * DV <= (int)kTmemCols, "TMEM budget");
+    // S and P V double-buffered; 256 columns let two CTAs share an SM
+    static constexpr uint32_t TMEM_COLS = 2 * NK + 2 * DV <= 256 ? 256 : 512;
+    static constexpr int CTAS_PER_SM = TMEM_COLS == 256 && DK == 64 ? 2 : 1;
 };
 
 template <int DK, int DV>
 struct SkaSmem {
     using K = SkaCfg<DK, DV>;
     alignas(1024) uint8_t q[K::Q_BYTES];
-    alignas(1024) uint8_t k[2][K::K_BYTES];
-    alignas(1024) uint8_t v[2][K::V_BYTES];
+    alignas(1024) uint8_t k[kStages][K::K_BYTES];
+    alignas(1024) uint8_t v[kStages][K::V_BYTES];
     alignas(1024) uint8_t p[2][K::P_BYTES];  // no-swizzle K-major (8x8 core matrices)
-    uint64_t q_full, k_full[2], v_full[2], kv_empty[2];
+    uint64_t q_full, k_full[kStages], v_full[kStages], k_empty[kStages], v_empty[kStages];
     uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2], o_full[2], o_empty[2], mma_done;
+    float red_max[2][2][kQRows];  // [tile parity][column half][row]: partial row maxima
+    float red_sum[2][kQRows];     // [column half][row]: partial row sums at the end
     uint32_t tmem_base;
     int fail;
 };
@@ -77,17 +84,21 @@ struct SkaKernelArgs {
     CUtensorMap mq, mk, mv;
 };
 
-// Warp-uniform bounded wait: every lane waits, then the warp agrees; a lane
-// that saw the failure flag makes the whole warp give up together (the tcgen05
-// loads that follow are warp-collective).
+// Warp-uniform bounded wait of the softmax warps: every lane waits on its own
+// clock (never on the shared failure flag, which another role may raise at any
+// moment), then the warp agrees.  Both warps of a pair wait for the same phases
+// in the same order, so they pass or run out together and never leave one
+// another alone at their pair barrier; the tcgen05 loads that follow are
+// warp-collective.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* fail,
                                           long long limit) {
-    const bool ok = mbar_wait(bar, parity, fail, limit);
+    const bool ok = mbar_wait_own(bar, parity, fail, limit);
     return __all_sync(0xffffffffu, ok);
 }
 
 template <int DK, int DV>
-__global__ void __launch_bounds__(kSkaThreads, 1) ska_fwd_kernel(const __grid_constant__ SkaKernelArgs A) {
+__global__ void __launch_bounds__(kSkaThreads, SkaCfg<DK, DV>::CTAS_PER_SM)
+    ska_fwd_kernel(const __grid_constant__ SkaKernelArgs A) {
     using K = SkaCfg<DK, DV>;
     constexpr int NK = K::NK;
     extern __shared__ __align__(1024) uint8_t smem_dyn[];
@@ -111,10 +122,13 @@ __global__ void __launch_bounds__(kSkaThreads, 1) ska_fwd_kernel(const __grid_co
 
     if (threadIdx.x == 0) {
         mbar_init(&sm.q_full, 1);
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < kStages; ++s) {
             mbar_init(&sm.k_full[s], 1);
             mbar_init(&sm.v_full[s], 1);
-            mbar_init(&sm.kv_empty[s], 1);
+            mbar_init(&sm.k_empty[s], 1);
+            mbar_init(&sm.v_empty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
             mbar_init(&sm.s_full[s], 1);
             mbar_init(&sm.s_empty[s], kSoftWarps);
             mbar_init(&sm.p_full[s], kSoftWarps);
@@ -127,7 +141,7 @@ __global__ void __launch_bounds__(kSkaThreads, 1) ska_fwd_kernel(const __grid_co
         fence_mbar_init();
     }
     if (warp == kMmaWarp) {
-        tmem_alloc(&sm.tmem_base, kTmemCols);
+        tmem_alloc(&sm.tmem_base, K::TMEM_COLS);
         tmem_relinquish();
     }
     if (warp == kProdWarp && lane == 0) {
@@ -147,29 +161,32 @@ __global__ void __launch_bounds__(kSkaThreads, 1) ska_fwd_kernel(const __grid_co
 #pragma unroll
             for (int x = 0; x < DK / 64; ++x)
                 tma_load_3d(sm.q + x * kQRows * 128, &A.mq, &sm.q_full, 64 * x, t0, bh);
-            int last[2] = {-1, -1};
+            int nk = 0, nv = 0;  // key / value tiles issued
             for (int n = 0; n < NT; ++n) {
-                const int st = n & 1;
-                if (!mbar_wait(&sm.kv_empty[st], ((n >> 1) & 1) ^ 1, fail, WL)) break;
+                const int st = n % kStages;
+                const uint32_t ph = ((n / kStages) & 1) ^ 1;
                 const int kb = (j_lo + n) * NK;
+                // the key stage frees after Q K^T, the value stage after P V
+                if (!mbar_wait(&sm.k_empty[st], ph, fail, WL)) break;
                 mbar_expect_tx(&sm.k_full[st], K::K_BYTES);
 #pragma unroll
                 for (int x = 0; x < DK / 64; ++x)
                     tma_load_3d(sm.k[st] + x * NK * 128, &A.mk, &sm.k_full[st], 64 * x, kb, b);
+                ++nk;
+                if (!mbar_wait(&sm.v_empty[st], ph, fail, WL)) break;
                 mbar_expect_tx(&sm.v_full[st], K::V_BYTES);
 #pragma unroll
                 for (int x = 0; x < DV / 64; ++x)
                     tma_load_3d(sm.v[st] + x * NK * 128, &A.mv, &sm.v_full[st], 64 * x, kb, bh);
-                last[st] = n;
+                ++nv;
             }
             // no copy may land after the CTA has gone: wait (bounded, on our own
             // clock) for the last ones issued into each stage and for the query
             mbar_wait_own(&sm.q_full, 0, fail, WL);
-            for (int st = 0; st < 2; ++st)
-                if (last[st] >= 0) {
-                    mbar_wait_own(&sm.k_full[st], (last[st] >> 1) & 1, fail, WL);
-                    mbar_wait_own(&sm.v_full[st], (last[st] >> 1) & 1, fail, WL);
-                }
+            for (int n = nk - kStages > 0 ? nk - kStages : 0; n < nk; ++n)
+                mbar_wait_own(&sm.k_full[n % kStages], (n / kStages) & 1, fail, WL);
+            for (int n = nv - kStages > 0 ? nv - kStages : 0; n < nv; ++n)
+                mbar_wait_own(&sm.v_full[n % kStages], (n / kStages) & 1, fail, WL);
         }
         __syncwarp();
     } else if (warp == kMmaWarp) {
@@ -179,33 +196,33 @@ __global__ void __launch_bounds__(kSkaThreads, 1) ska_fwd_kernel(const __grid_co
             constexpr uint32_t idO = idesc_bf16(kQRows, DV, 0, 1);  // O = P V (V MN-major)
             const uint32_t qa = smem_u32(sm.q);
             auto pv = [&](int m) -> bool {
-                const int st = m & 1;
+                const int st = m & 1, vs = m % kStages;
                 const uint32_t ph = (m >> 1) & 1;
                 if (!mbar_wait(&sm.p_full[st], ph, fail, WL)) return false;
                 if (!mbar_wait(&sm.o_empty[st], ph ^ 1, fail, WL)) return false;
-                if (!mbar_wait(&sm.v_full[st], ph, fail, WL)) return false;
+                if (!mbar_wait(&sm.v_full[vs], (m / kStages) & 1, fail, WL)) return false;
                 tc_fence_after();
-                const uint32_t pa = smem_u32(sm.p[st]), va = smem_u32(sm.v[st]);
+                const uint32_t pa = smem_u32(sm.p[st]), va = smem_u32(sm.v[vs]);
 #pragma unroll
                 for (int ks = 0; ks < NK / 16; ++ks)
                     mma_bf16(tO + st * DV, sdesc(pa + ks * 256, 128, NK * 16),
                              sdesc_sw128(va + ks * 2048, NK * 128, 1024), idO, ks > 0);
                 mma_commit(&sm.o_full[st]);
-                mma_commit(&sm.kv_empty[st]);
+                mma_commit(&sm.v_empty[vs]);
                 mma_commit(&sm.p_empty[st]);
                 return true;
             };
             bool ok = mbar_wait(&sm.q_full, 0, fail, WL);
             for (int n = 0; ok && n < NT; ++n) {
-                const int st = n & 1;
+                const int st = n & 1, ks_ = n % kStages;
                 const uint32_t ph = (n >> 1) & 1;
-                if (!mbar_wait(&sm.k_full[st], ph, fail, WL) ||
+                if (!mbar_wait(&sm.k_full[ks_], (n / kStages) & 1, fail, WL) ||
                     !mbar_wait(&sm.s_empty[st], ph ^ 1, fail, WL)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t ka = smem_u32(sm.k[st]);
+                const uint32_t ka = smem_u32(sm.k[ks_]);
 #pragma unroll
                 for (int ks = 0; ks < DK / 16; ++ks) {
                     const int x = ks / 4, off = (ks % 4) * 32;
@@ -213,6 +230,7 @@ __global__ void __launch_bounds__(kSkaThreads, 1) ska_fwd_kernel(const __grid_co
                              sdesc_sw128(ka + x * NK * 128 + off, 16, 1024), idS, ks > 0);
                 }
                 mma_commit(&sm.s_full[st]);
+                mma_commit(&sm.k_empty[ks_]);
                 if (n > 0) ok = pv(n - 1);
             }
             if (ok && NT > 0) pv(NT - 1);
@@ -223,72 +241,81 @@ __global__ void __launch_bounds__(kSkaThreads, 1) ska_fwd_kernel(const __grid_co
         __syncwarp();
     } else {
         // ------------------------------------------------------------- softmax
-        const int r = warp * 32 + lane;  // query row = TMEM lane
+        constexpr int NH = NK / 2, DH = DV / 2;  // key / output columns of this warp
+        const int quarter = warp & 3, half = warp >> 2;
+        const int r = quarter * 32 + lane;  // query row = TMEM lane
         const int t = t0 + r;
         const int lo = t - p.window + 1, hi = min(t, T - 1);
         const float c = p.scale * kLog2e;
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-        float o[DV];
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        const int bar_pair = 1 + quarter;  // named barrier of warps quarter, quarter + 4
+        float o[DH];
 #pragma unroll
-        for (int j = 0; j < DV; ++j) o[j] = 0.0f;
+        for (int j = 0; j < DH; ++j) o[j] = 0.0f;
         float m_run = -INFINITY, l = 0.0f, corr_pending = 1.0f;
         auto fold = [&](int i, float cr) -> bool {
             const int st = i & 1;
             if (!warp_wait(&sm.o_full[st], (i >> 1) & 1, fail, WL)) return false;
             tc_fence_after();
-            float x[DV];
+            float x[DH];
 #pragma unroll
-            for (int q32 = 0; q32 < DV / 32; ++q32)
-                tmem_ld32(tO + st * DV + lane_off + q32 * 32, x + q32 * 32);
+            for (int q32 = 0; q32 < DH / 32; ++q32)
+                tmem_ld32(tO + st * DV + half * DH + lane_off + q32 * 32, x + q32 * 32);
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.o_empty[st]);
 #pragma unroll
-            for (int j = 0; j < DV; ++j) o[j] = fmaf(o[j], cr, x[j]);
+            for (int j = 0; j < DH; ++j) o[j] = fmaf(o[j], cr, x[j]);
             return true;
         };
         bool ok = true;
         for (int n = 0; n < NT; ++n) {
             const int st = n & 1;
             const uint32_t ph = (n >> 1) & 1;
+            // the pair's warps meet at bar_pair below: both reach it or, after a
+            // failed wait, neither does (the waits are warp-uniform and both warps
+            // of a pair wait for the same phases)
             if (!warp_wait(&sm.s_full[st], ph, fail, WL)) { ok = false; break; }
             tc_fence_after();
-            float s[NK];
+            float s_[NH];
 #pragma unroll
-            for (int q32 = 0; q32 < NK / 32; ++q32)
-                tmem_ld32(tS + st * NK + lane_off + q32 * 32, s + q32 * 32);
+            for (int q32 = 0; q32 < NH / 32; ++q32)
+                tmem_ld32(tS + st * NK + half * NH + lane_off + q32 * 32, s_ + q32 * 32);
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.s_empty[st]);
-            const int kb = (j_lo + n) * NK;
-            if (kb < lo || kb + NK - 1 > hi) {
+            const int kb = (j_lo + n) * NK + half * NH;
+            if (kb < lo || kb + NH - 1 > hi) {
 #pragma unroll
-                for (int i = 0; i < NK; ++i)
-                    if (kb + i < lo || kb + i > hi) s[i] = -INFINITY;
+                for (int i = 0; i < NH; ++i)
+                    if (kb + i < lo || kb + i > hi) s_[i] = -INFINITY;
             }
-            float mx = s[0];
+            float m4[4] = {s_[0], s_[1], s_[2], s_[3]};
 #pragma unroll
-            for (int i = 1; i < NK; ++i) mx = fmaxf(mx, s[i]);
+            for (int i = 4; i < NH; ++i) m4[i & 3] = fmaxf(m4[i & 3], s_[i]);
+            sm.red_max[st][half][r] = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+            named_bar(bar_pair, 64);
+            const float mx = fmaxf(sm.red_max[st][0][r], sm.red_max[st][1][r]);
             const float m_new = fmaxf(m_run, mx * c);
             const float m_use = m_new == -INFINITY ? 0.0f : m_new;
             const float corr = ex2_fast(m_run - m_use);
-            float sum = 0.0f;
+            float l4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-            for (int i = 0; i < NK; ++i) {
-                s[i] = ex2_fast(fmaf(s[i], c, -m_use));
-                sum += s[i];
+            for (int i = 0; i < NH; ++i) {
+                s_[i] = ex2_fast(fmaf(s_[i], c, -m_use));
+                l4[i & 3] += s_[i];
             }
-            l = fmaf(l, corr, sum);
+            l = fmaf(l, corr, (l4[0] + l4[1]) + (l4[2] + l4[3]));
             m_run = m_new;
             if (!warp_wait(&sm.p_empty[st], ph ^ 1, fail, WL)) { ok = false; break; }
             // P row r, keys 8*kc .. 8*kc+7 -> core matrix (r/8, kc): byte
             // (r/8)*(NK*16) + kc*128 + (r%8)*16
-            uint8_t* prow = sm.p[st] + (r >> 3) * (NK * 16) + (r & 7) * 16;
+            uint8_t* prow = sm.p[st] + (r >> 3) * (NK * 16) + (r & 7) * 16 + half * (NH / 8) * 128;
 #pragma unroll
-            for (int kc = 0; kc < NK / 8; ++kc)
-                *reinterpret_cast<uint4*>(prow + kc * 128) = pack8(s + 8 * kc);
+            for (int kc = 0; kc < NH / 8; ++kc)
+                *reinterpret_cast<uint4*>(prow + kc * 128) = pack8(s_ + 8 * kc);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.p_full[st]);
@@ -296,12 +323,18 @@ __global__ void __launch_bounds__(kSkaThreads, 1) ska_fwd_kernel(const __grid_co
             corr_pending = corr;
         }
         if (ok && NT > 0) ok = fold(NT - 1, corr_pending);
+        // row sum over both halves; the pair meets once more only when both got here
+        if (ok) {
+            sm.red_sum[half][r] = l;
+            named_bar(bar_pair, 64);
+            l = sm.red_sum[0][r] + sm.red_sum[1][r];
+        }
         if (ok && t < T) {
             const float inv = l > 0.0f ? 1.0f / l : 0.0f;
             uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) +
-                                                  ((size_t)bh * T + t) * DV);
+                                                  ((size_t)bh * T + t) * DV + half * DH);
 #pragma unroll
-            for (int j8 = 0; j8 < DV / 8; ++j8) {
+            for (int j8 = 0; j8 < DH / 8; ++j8) {
                 float y[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) y[e] = o[8 * j8 + e] * inv;
@@ -314,7 +347,7 @@ __global__ void __launch_bounds__(kSkaThreads, 1) ska_fwd_kernel(const __grid_co
     __syncthreads();
     if (warp == kMmaWarp) {
         tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
+        tmem_dealloc(tmem, K::TMEM_COLS);
     }
     if (threadIdx.x == 0 && sm.fail) atomicOr(p.err, kErrTimeout);
 }
