@@ -38,7 +38,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from gated_linear_attention_ddts_b200.workloads import (SKA_DEC, SKA_FWD, WORKLOADS,  # noqa: E402
-                                                        draw_decode, draw_workload)
+                                                        draw_decode, draw_lowrank, draw_workload)
 
 SEQ = ("q", "k", "v", "g", "tau", "beta")
 METRIC = "DDTS recurrence tokens/s (fwd, fwd+bwd, decode) on 1 B200; % of roofline"
@@ -302,7 +302,21 @@ def run_extras(rdm, dev, pk, K):
         "unit": "tokens/s", "ms_per_step": ms, "gpu_launches_per_step": 1,
         "roofline": roofline(fwd_bytes(w, False), chunk_flops_fwd(w), ms, pk,
                              ncu_counters("tc_fwd_kernel", FWD_SRC, "1pre"))}
-    del x, o, wsf, fl
+    # the same with a rank-16 beta_hat built on chip from u [B,T,16] and w_up
+    # [H,16,dv]: beta's pre-activation is no longer read
+    u, wu = draw_lowrank(w.B, w.H, w.T, w.dv, 16, seed=w.seed + 40, device=dev)
+    t = time_steps(lambda: rdm.rdm_ddts_fwd(*(x[k] for k in SEQ[:5]), None, x["S0"], o, workspace=wsf,
+                                            gates="preact", beta_lowrank=(u, wu)),
+                   max(3, K // 2), 3, lambda: fl.zero_())
+    ms = statistics.mean(t)
+    lr_bytes = fwd_bytes(w, False) - w.B * w.H * w.T * w.dv * 2 + u.numel() * 2 + wu.numel() * 4
+    out["lowrank_beta_fwd"] = {
+        "workload": w.name + ", gates passed before their activations, rank-16 beta_hat",
+        "value": w.B * w.T / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
+        "gpu_launches_per_step": 1,
+        "roofline": roofline(lr_bytes, chunk_flops_fwd(w) + 2 * w.B * w.H * w.T * 16 * w.dv, ms, pk,
+                             ncu_counters("tc_fwd_kernel", FWD_SRC, "1lr"))}
+    del x, o, wsf, fl, u, wu
     # training forward + backward (forward saves chunk states for the backward)
     w = WORKLOADS[3]
     x = draw_workload(w, device=dev)

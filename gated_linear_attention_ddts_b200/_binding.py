@@ -32,7 +32,7 @@ class FwdArgs(ctypes.Structure):
                 ("q", _VP), ("k", _VP), ("v", _VP), ("g", _VP), ("tau", _VP), ("beta", _VP),
                 ("S0", _VP), ("o", _VP), ("ST", _VP), ("saved_states", _VP),
                 ("workspace", _VP), ("workspace_bytes", ctypes.c_size_t), ("gate_inputs", _I),
-                ("feedthrough", _VP)]
+                ("feedthrough", _VP), ("beta_rank", _I), ("beta_u", _VP), ("beta_w", _VP)]
 
 
 class BwdArgs(ctypes.Structure):
@@ -43,7 +43,8 @@ class BwdArgs(ctypes.Structure):
                 ("grad_q", _VP), ("grad_k", _VP), ("grad_v", _VP), ("grad_g", _VP),
                 ("grad_tau", _VP), ("grad_beta", _VP), ("grad_S0", _VP),
                 ("workspace", _VP), ("workspace_bytes", ctypes.c_size_t), ("gate_inputs", _I),
-                ("feedthrough", _VP), ("grad_feedthrough", _VP)]
+                ("feedthrough", _VP), ("grad_feedthrough", _VP), ("beta_rank", _I),
+                ("beta_u", _VP), ("beta_w", _VP), ("grad_beta_u", _VP), ("grad_beta_w", _VP)]
 
 
 class DecodeArgs(ctypes.Structure):
@@ -171,19 +172,29 @@ def rdm_ddts_saved_states_size(B, H, T, dk, dv, chunk=0) -> int:
     return int(load().rdm_ddts_saved_states_size(B, H, T, dk, dv, chunk))
 
 
+def _lowrank(beta_lowrank):
+    """(rank, u, w) of a low-rank beta_hat given as (u [B,T,r], w_up [H,r,dv])."""
+    if beta_lowrank is None:
+        return 0, None, None
+    u, w = beta_lowrank
+    return int(u.shape[-1]), u, w
+
+
 def _fwd_args(q, k, v, g, tau, beta, S0, o, ST, saved_states, ws, ws_bytes, chunk, impl,
-              gates="activated", feedthrough=None):
+              gates="activated", feedthrough=None, beta_lowrank=None):
     B, H, T, dk = q.shape
     dv = v.shape[-1]
+    r, u, w = _lowrank(beta_lowrank)
     return FwdArgs(B, H, T, dk, dv, chunk, _dtype_code(q), IMPL[impl],
                    _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(tau), _ptr(beta), _ptr(S0), _ptr(o),
                    _ptr(ST), _ptr(saved_states), _ptr(ws), ws_bytes, GATES[gates],
-                   _ptr(feedthrough))
+                   _ptr(feedthrough), r, _ptr(u), _ptr(w))
 
 
 def rdm_ddts_fwd_workspace_size(q, k, v, g, tau, beta, *, chunk=0, impl="auto",
-                                gates="activated") -> int:
-    a = _fwd_args(q, k, v, g, tau, beta, None, None, None, None, None, 0, chunk, impl, gates)
+                                gates="activated", beta_lowrank=None) -> int:
+    a = _fwd_args(q, k, v, g, tau, beta, None, None, None, None, None, 0, chunk, impl, gates,
+                  None, beta_lowrank)
     n = load().rdm_ddts_fwd_workspace_size(ctypes.byref(a))
     if n == ctypes.c_size_t(-1).value:
         raise RdmError(RDM_ERR_INVALID_ARG, "rdm_ddts_fwd_workspace_size")
@@ -192,11 +203,13 @@ def rdm_ddts_fwd_workspace_size(q, k, v, g, tau, beta, *, chunk=0, impl="auto",
 
 def rdm_ddts_fwd(q, k, v, g, tau, beta, S0=None, o=None, ST=None, saved_states=None, *,
                  workspace=None, chunk=0, impl="auto", return_state=False, stream=None,
-                 gates="activated", feedthrough=None):
+                 gates="activated", feedthrough=None, beta_lowrank=None):
     """Forward over [B,H,T,D] sequences.  Allocates o (and S_T when
     return_state) with torch if not given, and the sequence-segment workspace
     when none is passed (workspace=False runs without one).  feedthrough: [H,dv]
-    float32 weights d, o_t += d * v_t.  Returns (o, S_T or None)."""
+    float32 weights d, o_t += d * v_t.  beta_lowrank: (u [B,T,r], w_up [H,r,dv]
+    float32) for beta_hat = sigmoid(u . w_up) (gates="preact"; beta unused, may
+    be None).  Returns (o, S_T or None)."""
     B, H, T, dk = q.shape
     dv = v.shape[-1]
     if o is None:
@@ -205,34 +218,47 @@ def rdm_ddts_fwd(q, k, v, g, tau, beta, S0=None, o=None, ST=None, saved_states=N
         ST = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device)
     if workspace is None:
         need = rdm_ddts_fwd_workspace_size(q, k, v, g, tau, beta, chunk=chunk, impl=impl,
-                                           gates=gates)
+                                           gates=gates, beta_lowrank=beta_lowrank)
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device) if need else None
     elif workspace is False:
         workspace = None
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     a = _fwd_args(q, k, v, g, tau, beta, S0, o, ST, saved_states, workspace, ws_bytes, chunk,
-                  impl, gates, feedthrough)
+                  impl, gates, feedthrough, beta_lowrank)
     _check(load().rdm_ddts_fwd(ctypes.byref(a), _stream(stream)), "rdm_ddts_fwd")
     return o, ST
 
 
 def _bwd_args(q, k, v, g, tau, beta, S0, grad_o, grad_ST, saved_states, grads, ws, ws_bytes,
-              chunk, impl, gates="activated", feedthrough=None):
+              chunk, impl, gates="activated", feedthrough=None, beta_lowrank=None):
     B, H, T, dk = q.shape
     dv = v.shape[-1]
+    r, u, w = _lowrank(beta_lowrank)
     return BwdArgs(B, H, T, dk, dv, chunk, _dtype_code(q), IMPL[impl],
                    _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(tau), _ptr(beta), _ptr(S0),
                    _ptr(grad_o), _ptr(grad_ST), _ptr(saved_states),
                    *(_ptr(grads.get(n)) for n in ("dq", "dk", "dv", "dg", "dtau", "dbeta",
                                                     "dS0")),
-                   _ptr(ws), ws_bytes, GATES[gates], _ptr(feedthrough), _ptr(grads.get("dfeed")))
+                   _ptr(ws), ws_bytes, GATES[gates], _ptr(feedthrough), _ptr(grads.get("dfeed")),
+                   r, _ptr(u), _ptr(w), _ptr(grads.get("du")), _ptr(grads.get("dw_up")))
+
+
+def _alloc_grads(grads, q, k, v, g, tau, beta, beta_lowrank):
+    refs = [("dq", q), ("dk", k), ("dg", g), ("dtau", tau), ("dv", v)]
+    if beta_lowrank is None:
+        refs.append(("dbeta", beta))
+    else:
+        refs += [("du", beta_lowrank[0]), ("dw_up", beta_lowrank[1])]
+    for n, ref in refs:
+        if grads.get(n) is None:
+            grads[n] = torch.empty_like(ref)
 
 
 def rdm_ddts_bwd_workspace_size(q, k, v, g, tau, beta, S0=None, grad_o=None, grad_ST=None,
                                 saved_states=None, *, chunk=0, impl="auto",
-                                gates="activated") -> int:
+                                gates="activated", beta_lowrank=None) -> int:
     a = _bwd_args(q, k, v, g, tau, beta, S0, grad_o, grad_ST, saved_states, {}, None, 0,
-                  chunk, impl, gates)
+                  chunk, impl, gates, None, beta_lowrank)
     n = load().rdm_ddts_bwd_workspace_size(ctypes.byref(a))
     if n == ctypes.c_size_t(-1).value:
         raise RdmError(RDM_ERR_INVALID_ARG, "rdm_ddts_bwd_workspace_size")
@@ -241,45 +267,44 @@ def rdm_ddts_bwd_workspace_size(q, k, v, g, tau, beta, S0=None, grad_o=None, gra
 
 def rdm_ddts_bwd(q, k, v, g, tau, beta, S0, grad_o, grad_ST=None, saved_states=None, *,
                  grads=None, workspace=None, chunk=0, impl="auto", want_dS0=True, stream=None,
-                 gates="activated", feedthrough=None):
+                 gates="activated", feedthrough=None, beta_lowrank=None):
     """Backward.  `grads` may hold preallocated dq, dk, dv, dg, dtau, dbeta, dS0
-    (and dfeed when feedthrough is given); missing ones are allocated with
-    torch, as is the workspace.  Returns the dict."""
+    (and dfeed when feedthrough is given; du and dw_up in place of dbeta with
+    beta_lowrank); missing ones are allocated with torch, as is the workspace.
+    Returns the dict."""
     B, H, T, dk = q.shape
     dv = v.shape[-1]
     grads = dict(grads or {})
-    for n, ref in (("dq", q), ("dk", k), ("dg", g), ("dtau", tau), ("dv", v), ("dbeta", beta)):
-        if grads.get(n) is None:
-            grads[n] = torch.empty_like(ref)
+    _alloc_grads(grads, q, k, v, g, tau, beta, beta_lowrank)
     if want_dS0 and grads.get("dS0") is None:
         grads["dS0"] = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device)
     if feedthrough is not None and grads.get("dfeed") is None:
         grads["dfeed"] = torch.empty(H, dv, dtype=torch.float32, device=q.device)
     if workspace is None:
         need = rdm_ddts_bwd_workspace_size(q, k, v, g, tau, beta, S0, grad_o, grad_ST,
-                                           saved_states, chunk=chunk, impl=impl, gates=gates)
+                                           saved_states, chunk=chunk, impl=impl, gates=gates,
+                                           beta_lowrank=beta_lowrank)
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
     a = _bwd_args(q, k, v, g, tau, beta, S0, grad_o, grad_ST, saved_states, grads, workspace,
-                  workspace.numel() * workspace.element_size(), chunk, impl, gates, feedthrough)
+                  workspace.numel() * workspace.element_size(), chunk, impl, gates, feedthrough,
+                  beta_lowrank)
     _check(load().rdm_ddts_bwd(ctypes.byref(a), _stream(stream)), "rdm_ddts_bwd")
     return grads
 
 
 def rdm_ddts_bwd_noalloc(q, k, v, g, tau, beta, S0, grad_o, grad_ST=None, *, grads=None,
-                         chunk=0, want_dS0=True, stream=None, gates="activated"):
+                         chunk=0, want_dS0=True, stream=None, gates="activated", beta_lowrank=None):
     """Backward through the library's own fixed scratch (no workspace
     argument).  Gradient tensors are allocated with torch if not given;
     returns the dict of gradients."""
     B, H, T, dk = q.shape
     dv = v.shape[-1]
     grads = dict(grads or {})
-    for n, ref in (("dq", q), ("dk", k), ("dg", g), ("dtau", tau), ("dv", v), ("dbeta", beta)):
-        if grads.get(n) is None:
-            grads[n] = torch.empty_like(ref)
+    _alloc_grads(grads, q, k, v, g, tau, beta, beta_lowrank)
     if want_dS0 and grads.get("dS0") is None:
         grads["dS0"] = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device)
     a = _bwd_args(q, k, v, g, tau, beta, S0, grad_o, grad_ST, None, grads, None, 0, chunk, "simt",
-                  gates)
+                  gates, None, beta_lowrank)
     _check(load().rdm_ddts_bwd_noalloc(ctypes.byref(a), _stream(stream)), "rdm_ddts_bwd_noalloc")
     return grads
 

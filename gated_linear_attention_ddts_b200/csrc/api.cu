@@ -103,7 +103,25 @@ SeqParams fwd_params(const rdm_fwd_args* a) {
     p.wait_limit = wait_limit();
     p.withhold_flags = g_hook_withhold.load(std::memory_order_relaxed);
     p.dfeed = a->feedthrough;
+    p.beta_rank = a->beta_rank;
+    p.beta_u = a->beta_u;
+    p.beta_w = a->beta_w;
     return p;
+}
+
+// Low-rank beta_hat arguments (beta_rank > 0): rank 8 or 16, the factors given
+// and aligned, gates passed as pre-activations.
+rdm_status check_lowrank(int rank, const void* u, const float* w, rdm_gate_inputs g) {
+    if (rank == 0) return RDM_OK;
+    if (rank < 0) return RDM_ERR_INVALID_ARG;
+    if (rank != 8 && rank != 16) return RDM_ERR_UNSUPPORTED;
+    if (g != RDM_GATES_PREACT || !u || !w || !aligned(u) || !aligned(w)) return RDM_ERR_INVALID_ARG;
+    return RDM_OK;
+}
+
+size_t lowrank_buffer_bytes(int B, int H, int T, int dv, rdm_dtype dt) {
+    const size_t n = (size_t)B * H * T * dv * (dt == RDM_BF16 ? 2 : 4);
+    return (n + 255) / 256 * 256;
 }
 
 BwdParams bwd_params(const rdm_bwd_args* a) {
@@ -144,29 +162,33 @@ rdm_status rdm_ddts_fwd(const rdm_fwd_args* a, rdm_stream_t stream) {
     rdm_status st = check_sizes(a->B, a->H, a->T, a->dk, a->dv, a->chunk, a->dtype, a->impl);
     if (st != RDM_OK) return st;
     if (!gates_ok(a->gate_inputs)) return RDM_ERR_INVALID_ARG;
+    st = check_lowrank(a->beta_rank, a->beta_u, a->beta_w, a->gate_inputs);
+    if (st != RDM_OK) return st;
+    const bool lr = a->beta_rank > 0;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (!opt_aligned(a->S0) || !opt_aligned(a->ST) || !opt_aligned(a->saved_states) ||
         !opt_aligned(a->workspace) || !opt_aligned(a->feedthrough))
         return RDM_ERR_INVALID_ARG;
     if (a->T == 0) {
-        if (a->impl == RDM_IMPL_TC && a->dtype != RDM_BF16) return RDM_ERR_UNSUPPORTED;
+        if ((a->impl == RDM_IMPL_TC || lr) && a->dtype != RDM_BF16) return RDM_ERR_UNSUPPORTED;
         return empty_sequence(a->B, a->H, a->dk, a->dv, a->S0, a->ST, s);
     }
-    const void* in[] = {a->q, a->k, a->v, a->g, a->tau, a->beta, a->o};
+    const void* in[] = {a->q, a->k, a->v, a->g, a->tau, lr ? a->v : a->beta, a->o};
     for (const void* p : in)
         if (!p || !aligned(p)) return RDM_ERR_INVALID_ARG;
     SeqParams p = fwd_params(a);
     p.err = status_word();
     if (!p.err) return RDM_ERR_CUDA;
     const bool tc = use_tc_fwd(p, a->impl);
-    if (a->impl == RDM_IMPL_TC && !tc) return RDM_ERR_UNSUPPORTED;
+    if ((a->impl == RDM_IMPL_TC || lr) && !tc) return RDM_ERR_UNSUPPORTED;
     return from_cuda(tc ? launch_tc_fwd(p, s) : launch_simt_fwd(p, s));
 }
 
 size_t rdm_ddts_fwd_workspace_size(const rdm_fwd_args* a) {
     if (!a) return (size_t)-1;
     if (check_sizes(a->B, a->H, a->T, a->dk, a->dv, a->chunk, a->dtype, a->impl) != RDM_OK ||
-        !gates_ok(a->gate_inputs))
+        !gates_ok(a->gate_inputs) ||
+        check_lowrank(a->beta_rank, a->beta_u, a->beta_w, a->gate_inputs) == RDM_ERR_INVALID_ARG)
         return (size_t)-1;
     if (a->T == 0) return 0;
     SeqParams p = fwd_params(a);
@@ -178,10 +200,14 @@ size_t rdm_ddts_bwd_workspace_size(const rdm_bwd_args* a) {
     if (check_sizes(a->B, a->H, a->T, a->dk, a->dv, a->chunk, a->dtype, a->impl) != RDM_OK ||
         !gates_ok(a->gate_inputs))
         return (size_t)-1;
+    if (check_lowrank(a->beta_rank, a->beta_u, a->beta_w, a->gate_inputs) == RDM_ERR_INVALID_ARG)
+        return (size_t)-1;
     if (a->T == 0) return 0;
     BwdParams p = bwd_params(a);
-    if (use_tc_bwd(p, a->impl)) return tc_bwd_workspace(p);
-    return simt_bwd_workspace(p);
+    const size_t base = use_tc_bwd(p, a->impl) ? tc_bwd_workspace(p) : simt_bwd_workspace(p);
+    if (a->beta_rank <= 0) return base;
+    // the expanded pre-activation and its gradient follow the kernels' scratch
+    return (base + 255) / 256 * 256 + 2 * lowrank_buffer_bytes(a->B, a->H, a->T, a->dv, a->dtype);
 }
 
 rdm_status rdm_ddts_bwd(const rdm_bwd_args* a, rdm_stream_t stream) {
@@ -189,6 +215,12 @@ rdm_status rdm_ddts_bwd(const rdm_bwd_args* a, rdm_stream_t stream) {
     rdm_status st = check_sizes(a->B, a->H, a->T, a->dk, a->dv, a->chunk, a->dtype, a->impl);
     if (st != RDM_OK) return st;
     if (!gates_ok(a->gate_inputs)) return RDM_ERR_INVALID_ARG;
+    st = check_lowrank(a->beta_rank, a->beta_u, a->beta_w, a->gate_inputs);
+    if (st != RDM_OK) return st;
+    const bool lr = a->beta_rank > 0;
+    if (lr && (!a->grad_beta_u || !a->grad_beta_w || !aligned(a->grad_beta_u) ||
+               !aligned(a->grad_beta_w)))
+        return RDM_ERR_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (!opt_aligned(a->S0) || !opt_aligned(a->grad_ST) || !opt_aligned(a->grad_S0) ||
         !opt_aligned(a->saved_states) || !opt_aligned(a->workspace) ||
@@ -201,10 +233,14 @@ rdm_status rdm_ddts_bwd(const rdm_bwd_args* a, rdm_stream_t stream) {
         if (a->grad_feedthrough &&
             cudaMemsetAsync(a->grad_feedthrough, 0, (size_t)a->H * a->dv * 4, s) != cudaSuccess)
             return RDM_ERR_CUDA;
+        if (lr && cudaMemsetAsync(a->grad_beta_w, 0, (size_t)a->H * a->beta_rank * a->dv * 4, s) !=
+                      cudaSuccess)
+            return RDM_ERR_CUDA;
         return empty_sequence(a->B, a->H, a->dk, a->dv, a->grad_ST, a->grad_S0, s);
     }
-    const void* in[] = {a->q, a->k, a->v, a->g, a->tau, a->beta, a->grad_o, a->grad_q,
-                        a->grad_k, a->grad_v, a->grad_g, a->grad_tau, a->grad_beta};
+    const void* in[] = {a->q, a->k, a->v, a->g, a->tau, lr ? a->v : a->beta, a->grad_o, a->grad_q,
+                        a->grad_k, a->grad_v, a->grad_g, a->grad_tau,
+                        lr ? a->grad_v : a->grad_beta};
     for (const void* p : in)
         if (!p || !aligned(p)) return RDM_ERR_INVALID_ARG;
     BwdParams p = bwd_params(a);
@@ -212,10 +248,28 @@ rdm_status rdm_ddts_bwd(const rdm_bwd_args* a, rdm_stream_t stream) {
     if (!p.err) return RDM_ERR_CUDA;
     const bool tc = use_tc_bwd(p, a->impl);
     if (a->impl == RDM_IMPL_TC && !tc) return RDM_ERR_UNSUPPORTED;
-    const size_t need = tc ? tc_bwd_workspace(p) : simt_bwd_workspace(p);
+    const size_t base = tc ? tc_bwd_workspace(p) : simt_bwd_workspace(p);
+    const size_t lrb = lr ? lowrank_buffer_bytes(a->B, a->H, a->T, a->dv, a->dtype) : 0;
+    const size_t need = lr ? (base + 255) / 256 * 256 + 2 * lrb : base;
     if (need > 0 && (!a->workspace || a->workspace_bytes < need)) return RDM_ERR_WORKSPACE;
+    LowRankParams lp{};
+    if (lr) {
+        // beta_pre = u . w_up into the workspace, its gradient beside it
+        uint8_t* ws = static_cast<uint8_t*>(a->workspace) + (base + 255) / 256 * 256;
+        lp.B = a->B; lp.H = a->H; lp.T = a->T; lp.dv = a->dv; lp.r = a->beta_rank;
+        lp.bf16 = a->dtype == RDM_BF16;
+        lp.u = a->beta_u; lp.w = a->beta_w;
+        lp.beta_pre = ws; lp.dbeta_pre = ws + lrb;
+        lp.du = a->grad_beta_u; lp.dw = a->grad_beta_w;
+        p.beta = lp.beta_pre;
+        p.dbeta = ws + lrb;
+        p.ws_bytes = base;
+        cudaError_t e = launch_lowrank_expand(lp, s);
+        if (e != cudaSuccess) return from_cuda(e);
+    }
     cudaError_t e = tc ? launch_tc_bwd(p, s) : launch_simt_bwd(p, s);
     if (e == cudaSuccess && p.grad_dfeed) e = launch_feed_grad(p, s);
+    if (e == cudaSuccess && lr) e = launch_lowrank_grad(lp, s);
     return from_cuda(e);
 }
 
@@ -264,6 +318,8 @@ static ConvParams conv_params(const rdm_shortconv_args* a) {
     p.silu = a->silu != 0;
     p.x = a->x; p.w = a->weight; p.bias = a->bias; p.xs = a->state_in;
     p.y = a->y; p.xs_out = a->W > 1 ? a->state_out : nullptr;
+    p.err = status_word();
+    p.wait_limit = wait_limit();
     return p;
 }
 
@@ -272,7 +328,9 @@ rdm_status rdm_shortconv_fwd(const rdm_shortconv_args* a, rdm_stream_t stream) {
     if (st != RDM_OK) return st;
     if (a->T > 0 && (!a->y || !aligned(a->y))) return RDM_ERR_INVALID_ARG;
     if (!opt_aligned(a->state_out)) return RDM_ERR_INVALID_ARG;
-    return from_cuda(launch_conv_fwd(conv_params(a), reinterpret_cast<cudaStream_t>(stream)));
+    const ConvParams p = conv_params(a);
+    if (!p.err) return RDM_ERR_CUDA;
+    return from_cuda(launch_conv_fwd(p, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 rdm_status rdm_shortconv_bwd(const rdm_shortconv_bwd_args* a, rdm_stream_t stream) {
@@ -285,6 +343,7 @@ rdm_status rdm_shortconv_bwd(const rdm_shortconv_bwd_args* a, rdm_stream_t strea
     if (a->fwd.T > 0 && (!a->grad_y || !aligned(a->grad_y) || !a->grad_x || !aligned(a->grad_x)))
         return RDM_ERR_INVALID_ARG;
     ConvParams p = conv_params(&a->fwd);
+    if (!p.err) return RDM_ERR_CUDA;
     p.y = nullptr;
     p.xs_out = nullptr;
     p.dy = a->grad_y;

@@ -25,6 +25,11 @@ struct SeqParams {
     long long wait_limit;  // SM clock cycles a bounded wait may take before it gives up
     int withhold_flags;    // test hook: segment CTAs never publish their flags
     const float* dfeed;    // feedthrough weights [H][dv]: o_t += d (.) v_t; null = none
+    // low-rank beta_hat (preact only): pre-activation u[b,t,:] . w_up[h][:, j],
+    // u [B,T,beta_rank] bf16, w_up [H,beta_rank,dv] float32; beta unused.  0 = off
+    int beta_rank;
+    const void* beta_u;
+    const float* beta_w;
 };
 
 struct BwdParams {
@@ -83,7 +88,9 @@ struct ConvParams {
     float* dw;           // dL/dw [H,D,W]
     float* dbias;        // dL/dbias [H,D] or null
     void* dxs;           // dL/d(carried-in state) or null
-    int conv_groups;     // backward: token groups per block (set by the launcher)
+    int tile;            // tokens per block (set by the launcher)
+    unsigned* err;       // device status word (a staging wait that ran out)
+    long long wait_limit;
 };
 cudaError_t launch_conv_fwd(const ConvParams& p, cudaStream_t s);
 cudaError_t launch_conv_bwd(const ConvParams& p, cudaStream_t s);
@@ -91,6 +98,21 @@ cudaError_t launch_conv_bwd(const ConvParams& p, cudaStream_t s);
 // gradient of the feedthrough weights: grad_d[h][j] = sum_{b,t} dO[b,h,t,j] v[b,h,t,j]
 // (zeroes grad_d, then accumulates; float32 atomics)
 cudaError_t launch_feed_grad(const BwdParams& p, cudaStream_t s);
+
+// low-rank beta_hat (lowrank.cu): expansion of the pre-activation for the
+// backward, and the contraction of its gradient
+struct LowRankParams {
+    int B, H, T, dv, r;
+    int bf16;                // element type of u, beta_pre, dbeta_pre, du
+    const void* u;           // [B,T,r]
+    const float* w;          // [H,r,dv]
+    void* beta_pre;          // [B,H,T,dv] written by the expansion
+    const void* dbeta_pre;   // [B,H,T,dv] gradient w.r.t. the pre-activation
+    void* du;                // [B,T,r]
+    float* dw;               // [H,r,dv]
+};
+cudaError_t launch_lowrank_expand(const LowRankParams& p, cudaStream_t s);
+cudaError_t launch_lowrank_grad(const LowRankParams& p, cudaStream_t s);
 
 // tensor-core (tcgen05) chunked path
 bool tc_fwd_supported(const SeqParams& p);
@@ -110,6 +132,11 @@ namespace rdm {
 // driver refuses the map.
 bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t n0, uint64_t n1,
                        uint64_t n2, uint32_t b0, uint32_t b1);
+
+// The same without swizzle (rows of the box land b0 * 2 bytes apart); b0 * 2
+// a multiple of 16.
+bool make_tmap_bf16_3d_plain(CUtensorMap* map, const void* base, uint64_t n0, uint64_t n1,
+                             uint64_t n2, uint32_t b0, uint32_t b1);
 
 // 2-D float32 tensor [n1][n0] (n0 innermost, dense) as a TMA map with box
 // {b0, b1} and 128-byte swizzle (b0 * 4 must be 128).

@@ -77,9 +77,20 @@ __device__ __forceinline__ void activate_gates8(float* g8, float* t8) {
         t8[e] = sigmoid_fast(t8[e]);
     }
 }
+// beta_hat = sigmoid(x) = (1 + tanh(x / 2)) / 2 with the single-instruction
+// tanh (PTX tanh.approx, relative error about 2^-11): beta_hat only scales v,
+// whose bf16 rounding (2^-9) already bounds the path's accuracy, so one MUFU
+// operation per element replaces the exponential and the reciprocal.  (tau
+// keeps sigmoid_fast: its errors compound along the decay products.)
+__device__ __forceinline__ float tanh_fast(float x) {
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float sigmoid_tanh(float x) { return fmaf(0.5f, tanh_fast(0.5f * x), 0.5f); }
 __device__ __forceinline__ void activate_beta8(float* b8) {
 #pragma unroll
-    for (int e = 0; e < 8; ++e) b8[e] = sigmoid_fast(b8[e]);
+    for (int e = 0; e < 8; ++e) b8[e] = sigmoid_tanh(b8[e]);
 }
 
 // Device status word bits (set with atomicOr by kernels, read by the host).

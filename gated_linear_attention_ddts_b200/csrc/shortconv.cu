@@ -7,23 +7,26 @@
 //
 // with x at t-i < 0 read from the carried-in state (the previous W-1 inputs).
 //
-// HBM-bound streaming: one thread owns 16 bytes of channels (8 bf16 or 4
-// float32) over a run of kRun consecutive tokens and keeps the last W inputs
-// of its channels in registers, so every input row is read once per run (plus
-// a W-1 row halo that the neighbouring run of the same block has just pulled
-// into L1) and every output row written once; a warp's loads and stores cover
-// whole 16-byte column groups of consecutive rows.  Runs are short and fully
-// unrolled so that each thread has all of its loads in flight at once (with
-// 16-token runs walked one load at a time the kernels ran at 7% of HBM).  The backward walks the same runs with a
-// look-ahead window of W values of dL/dz, and reduces the weight and bias
-// gradients in shared memory before one float32 atomic per value and block.
+// HBM-bound streaming through shared memory: a block takes a tile of tokens of
+// one (b, h) (8192 elements, 128 tokens at D = 64), whose rows are contiguous
+// in HBM, and has the bulk copy engine bring the tile and its W-1 row halo
+// into shared memory in one transfer (the backward: x and dy, with the halo on
+// both sides); the threads then work out of shared memory, 16 bytes of
+// channels of one token at a time, and store whole rows.  The backward first
+// writes dL/dz of the tile to shared memory (z recomputed from the staged x
+// when the SiLU is on), then forms dx and the weight and bias gradients, which
+// are reduced over the block (shuffles, then shared memory) before one float32
+// atomic per value and block.
 #include <algorithm>
 
 #include "launch.h"
 #include "rdm_common.cuh"
+#include "tc_ptx.cuh"
 
 namespace rdm {
 namespace {
+
+using namespace tc;
 
 constexpr int kThreads = 256;
 constexpr int kRun = 4;  // tokens per thread (loops fully unrolled: every load in flight at once)
@@ -81,43 +84,113 @@ __device__ __forceinline__ float silu_grad(float z) {
     return s * (1.0f + z * (1.0f - s));
 }
 
+// 16 bytes of a staged row (shared memory) as floats
+__device__ __forceinline__ void lds_vec(const float* p, float* f) {
+    const float4 u = *reinterpret_cast<const float4*>(p);
+    f[0] = u.x; f[1] = u.y; f[2] = u.z; f[3] = u.w;
+}
+__device__ __forceinline__ void lds_vec(const __nv_bfloat16* p, float* f) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        f[2 * e] = __uint_as_float(w[e] << 16);
+        f[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+    }
+}
+
+template <typename T>
+__device__ __forceinline__ T zero_val() { return T(0.0f); }
+
+// Stage the rows of tokens [lo, hi) of sequence bh (rows of D elements) into
+// dst: the in-sequence rows [max(lo, 0), min(hi, T)) are handed to the bulk
+// copy engine by thread 0 (the rows of one (b, h) are contiguous in HBM);
+// tokens before the sequence come from the carried-in state (zeros without
+// one, or when `state` is null), tokens past its end are zeros.  Returns the
+// bytes the bulk copy will deliver on `bar`.
 template <typename T, int W>
-__global__ void __launch_bounds__(kThreads) conv_fwd_kernel(ConvParams p) {
+__device__ uint32_t stage_rows(const ConvParams& p, const T* seq, const T* state, int bh, int lo,
+                               int hi, T* dst, uint64_t* bar) {
+    const int a = max(lo, 0), e = min(hi, p.T);
+    const uint32_t bytes = a < e ? (uint32_t)((size_t)(e - a) * p.D * sizeof(T)) : 0u;
+    if (threadIdx.x == 0 && bytes)
+        bulk_load(dst + (size_t)(a - lo) * p.D, seq + ((size_t)bh * p.T + a) * p.D, bytes, bar);
+    for (int i = threadIdx.x; i < (a - lo) * p.D; i += kThreads) {
+        const int s = W - 1 + lo + i / p.D;  // position in the carried-in state
+        dst[i] = (state && s >= 0) ? state[((size_t)bh * (W - 1) + s) * p.D + i % p.D] : zero_val<T>();
+    }
+    for (int i = (e - lo) * p.D + threadIdx.x; i < (hi - lo) * p.D; i += kThreads)
+        dst[i] = zero_val<T>();
+    return bytes;
+}
+
+// Every thread waits (bounded) for the staged rows.  A wait that runs out sets
+// the status word; the thread then waits once more, also bounded, so that no
+// copy lands after the block has left, and the block skips its work.
+__device__ __forceinline__ bool staged(uint64_t* bar, const ConvParams& p) {
+    const long long lim = p.wait_limit > 0 ? p.wait_limit : kDefaultWaitLimit;
+    long long t0 = clock64();
+    while (!mbar_try_wait(bar, 0))
+        if (clock64() - t0 > lim) {
+            atomicOr(p.err, kErrTimeout);
+            t0 = clock64();
+            while (!mbar_try_wait(bar, 0) && clock64() - t0 <= lim) {
+            }
+            return false;
+        }
+    return true;
+}
+
+// Forward: one block per tile of `p.tile` tokens of one (b, h).  The tile's
+// inputs and the W-1 rows before it are staged in shared memory by one bulk
+// copy; then thread (channel group cg, token lane r) produces 16 bytes of
+// channels for tokens t0 + r, t0 + r + R, ... (a warp stores whole rows).
+template <typename T, int W>
+__global__ void __launch_bounds__(kThreads) conv_fwd_kernel(const ConvParams p) {
     constexpr int N = Vec<T>::N;
+    extern __shared__ __align__(128) uint8_t conv_smem[];
+    __shared__ uint64_t bar;
+    T* xs = reinterpret_cast<T*>(conv_smem);  // rows of tokens [t0 - (W-1), t1)
     const int CG = p.D / N, R = kThreads / CG;
-    const int bh = blockIdx.x, h = bh % p.H;
-    const int cg = threadIdx.x % CG, run = threadIdx.x / CG, c0 = cg * N;
-    const int t0 = (blockIdx.y * R + run) * kRun, t1 = min(t0 + kRun, p.T);
-    if (t0 >= p.T) return;  // no barrier in this kernel
+    const int ntile = (p.T + p.tile - 1) / p.tile;
+    const int bh = blockIdx.x / ntile, h = bh % p.H;
+    const int t0 = (blockIdx.x % ntile) * p.tile, t1 = min(t0 + p.tile, p.T);
+    const int lo = t0 - (W - 1);
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    const uint32_t bytes = stage_rows<T, W>(p, static_cast<const T*>(p.x), static_cast<const T*>(p.xs),
+                                            bh, lo, t1, xs, &bar);
+    if (threadIdx.x == 0) mbar_expect_tx(&bar, bytes);
+    const int cg = threadIdx.x % CG, r0 = threadIdx.x / CG, c0 = cg * N;
     float wv[W][N], bv[N];
 #pragma unroll
     for (int e = 0; e < N; ++e) {
 #pragma unroll
-        for (int i = 0; i < W; ++i) wv[i][e] = p.w[((size_t)h * p.D + c0 + e) * W + i];
-        bv[e] = p.bias ? p.bias[(size_t)h * p.D + c0 + e] : 0.0f;
+        for (int i = 0; i < W; ++i) wv[i][e] = __ldg(p.w + ((size_t)h * p.D + c0 + e) * W + i);
+        bv[e] = p.bias ? __ldg(p.bias + (size_t)h * p.D + c0 + e) : 0.0f;
     }
-    float win[W][N];  // win[k] = x[t - (W-1) + k]
-#pragma unroll
-    for (int k = 0; k < W - 1; ++k) input_row<T>(p, bh, t0 - (W - 1) + k, c0, win[k]);
+    __syncthreads();  // the rows the threads filled
+    if (!__syncthreads_and(staged(&bar, p))) return;  // the block leaves together
     T* y = static_cast<T*>(p.y) + (size_t)bh * p.T * p.D + c0;
-#pragma unroll
-    for (int k = 0; k < kRun; ++k) {
-        const int t = t0 + k;
-        if (t >= t1) break;
-        input_row<T>(p, bh, t, c0, win[W - 1]);
+    for (int t = t0 + r0; t < t1; t += R) {
         float z[N];
 #pragma unroll
-        for (int e = 0; e < N; ++e) {
-            float a = bv[e];
+        for (int e = 0; e < N; ++e) z[e] = bv[e];
 #pragma unroll
-            for (int i = 0; i < W; ++i) a = fmaf(wv[i][e], win[W - 1 - i][e], a);
-            z[e] = p.silu ? silu_f(a) : a;
+        for (int i = 0; i < W; ++i) {
+            float xv[N];
+            lds_vec(xs + (size_t)(t - i - lo) * p.D + c0, xv);
+#pragma unroll
+            for (int e = 0; e < N; ++e) z[e] = fmaf(wv[i][e], xv[e], z[e]);
+        }
+        if (p.silu) {
+#pragma unroll
+            for (int e = 0; e < N; ++e) z[e] = silu_f(z[e]);
         }
         store_vec(y + (size_t)t * p.D, z);
-#pragma unroll
-        for (int k = 0; k < W - 1; ++k)
-#pragma unroll
-            for (int e = 0; e < N; ++e) win[k][e] = win[k + 1][e];
     }
 }
 
@@ -162,95 +235,143 @@ __device__ __forceinline__ void dz_row(const ConvParams& p, int bh, int t, int c
     }
 }
 
+// Backward: one block per tile of `p.tile` tokens of one (b, h).  Staged: x of
+// tokens [t0 - (W-1), t1 + W - 1) and dy of [t0, t1 + W - 1) (bulk copies, as
+// in the forward).  Phase 1 writes dL/dz of tokens [t0, t1 + W - 1) (zero past
+// the end) to shared memory as float32; phase 2 gives dx[t] = sum_i w_i dz[t+i]
+// (plus the carried-out state's gradient where it copies x[t]) and accumulates
+// the weight and bias gradients, which are summed over the block and added
+// with one float32 atomic per value.
 template <typename T, int W>
-__global__ void __launch_bounds__(kThreads) conv_bwd_kernel(ConvParams p) {
+__global__ void __launch_bounds__(kThreads) conv_bwd_kernel(const ConvParams p) {
     constexpr int N = Vec<T>::N;
+    extern __shared__ __align__(128) uint8_t conv_smem[];
+    __shared__ uint64_t bar;
+    const int TT = p.tile;
+    const int ntile = (p.T + TT - 1) / TT;
+    const int bh = blockIdx.x / ntile, h = bh % p.H;
+    const int t0 = (blockIdx.x % ntile) * TT, t1 = min(t0 + TT, p.T);
+    const int lo = t0 - (W - 1), hi = t1 + W - 1;   // x rows [lo, hi)
+    const int nz = hi - t0;                          // dz and dy rows [t0, hi)
+    T* xs = reinterpret_cast<T*>(conv_smem);
+    T* dys = xs + (size_t)(TT + 2 * (W - 1)) * p.D;
+    float* dzs = reinterpret_cast<float*>(dys + (size_t)(TT + W - 1) * p.D);
+    float* s_red = dzs + (size_t)(TT + W - 1) * p.D;   // [warps][D (W + 1)]
     const int CG = p.D / N, R = kThreads / CG;
-    const int bh = blockIdx.x, h = bh % p.H;
-    const int cg = threadIdx.x % CG, run = threadIdx.x / CG, c0 = cg * N;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    // per-warp partial sums of the weight and bias gradients: [warp][cg][W+1][N]
-    __shared__ float s_red[kThreads / 32][128 * 5];  // CG (W + 1) N = D (W + 1) <= 640
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    uint32_t bytes = stage_rows<T, W>(p, static_cast<const T*>(p.x), static_cast<const T*>(p.xs), bh,
+                                      lo, hi, xs, &bar);
+    bytes += stage_rows<T, W>(p, static_cast<const T*>(p.dy), nullptr, bh, t0, hi, dys, &bar);
+    if (threadIdx.x == 0) mbar_expect_tx(&bar, bytes);
+    const int cg = threadIdx.x % CG, r0 = threadIdx.x / CG, c0 = cg * N;
     float wv[W][N], bv[N], aw[W][N], ab[N];
 #pragma unroll
     for (int e = 0; e < N; ++e) {
 #pragma unroll
         for (int i = 0; i < W; ++i) {
-            wv[i][e] = p.w[((size_t)h * p.D + c0 + e) * W + i];
+            wv[i][e] = __ldg(p.w + ((size_t)h * p.D + c0 + e) * W + i);
             aw[i][e] = 0.0f;
         }
-        bv[e] = p.bias ? p.bias[(size_t)h * p.D + c0 + e] : 0.0f;
+        bv[e] = p.bias ? __ldg(p.bias + (size_t)h * p.D + c0 + e) : 0.0f;
         ab[e] = 0.0f;
     }
-    T* dx = static_cast<T*>(p.dx) + (size_t)bh * p.T * p.D + c0;
-    const int tout0 = p.T - (p.W - 1);  // first token copied into the carried-out state
-    // the block's tile of tokens is a whole number of R x kRun groups; every
-    // thread walks its run in each group (the weight gradients accumulate in
-    // registers across the groups)
-    for (int t0 = (blockIdx.y * p.conv_groups * R + run) * kRun; t0 < min(p.T, (blockIdx.y + 1) * p.conv_groups * R * kRun);
-         t0 += R * kRun) {
-        const int t1 = min(t0 + kRun, p.T);
-        // dzw[k] = dz[t + k] for the output t = the oldest token of the window
-        float dzw[W][N];
+    __syncthreads();  // the rows the threads filled
+    if (!__syncthreads_and(staged(&bar, p))) return;  // the block leaves together
+    // phase 1: dz = dy, through the SiLU when on (z recomputed from the staged x)
+    for (int u = r0; u < nz; u += R) {
+        const int t = t0 + u;
+        float dz[N];
+        if (t < p.T) {
+            lds_vec(dys + (size_t)u * p.D + c0, dz);
+            if (p.silu) {
+                float z[N];
 #pragma unroll
-        for (int k = 0; k < W - 1; ++k) dz_row<T, W>(p, bh, t0 + k, c0, wv, bv, dzw[k]);
-#pragma unroll
-        for (int k = 0; k < kRun; ++k) {
-            const int t = t0 + k;
-            if (t >= t1) break;
-            dz_row<T, W>(p, bh, t + W - 1, c0, wv, bv, dzw[W - 1]);
-            float xw[W][N];  // x[t - i]
-#pragma unroll
-            for (int i = 0; i < W; ++i) input_row<T>(p, bh, t - i, c0, xw[i]);
-            float g[N];
-#pragma unroll
-            for (int e = 0; e < N; ++e) {
-                float a = 0.0f;
+                for (int e = 0; e < N; ++e) z[e] = bv[e];
 #pragma unroll
                 for (int i = 0; i < W; ++i) {
-                    a = fmaf(wv[i][e], dzw[i][e], a);                // dx[t] = sum_i w_i dz[t + i]
-                    aw[i][e] = fmaf(dzw[0][e], xw[i][e], aw[i][e]);  // dw_i += dz[t] x[t - i]
+                    float xv[N];
+                    lds_vec(xs + (size_t)(t - i - lo) * p.D + c0, xv);
+#pragma unroll
+                    for (int e = 0; e < N; ++e) z[e] = fmaf(wv[i][e], xv[e], z[e]);
                 }
-                ab[e] += dzw[0][e];
-                g[e] = a;
+#pragma unroll
+                for (int e = 0; e < N; ++e) dz[e] *= silu_grad(z[e]);
             }
-            if (p.dxs_out != nullptr && t >= tout0) {  // the carried-out state copies x[t]
-                float go[N];
-                load_vec(static_cast<const T*>(p.dxs_out) + ((size_t)bh * (p.W - 1) + (t - tout0)) * p.D + c0, go);
+        } else {
 #pragma unroll
-                for (int e = 0; e < N; ++e) g[e] += go[e];
-            }
-            store_vec(dx + (size_t)t * p.D, g);
-#pragma unroll
-            for (int kk = 0; kk < W - 1; ++kk)
-#pragma unroll
-                for (int e = 0; e < N; ++e) dzw[kk][e] = dzw[kk + 1][e];
+            for (int e = 0; e < N; ++e) dz[e] = 0.0f;
         }
+        float* row = dzs + (size_t)u * p.D + c0;
+#pragma unroll
+        for (int e = 0; e < N; e += 4) *reinterpret_cast<float4*>(row + e) = make_float4(dz[e], dz[e + 1], dz[e + 2], dz[e + 3]);
     }
-    // weight and bias gradients: sum the lanes of a warp that hold the same
-    // channels (lanes cg, cg + CG, ...), one slot per warp in shared memory, a
-    // sum over the warps, then one float32 atomic per value and block
+    __syncthreads();
+    // phase 2
+    T* dx = static_cast<T*>(p.dx) + (size_t)bh * p.T * p.D + c0;
+    const int tout0 = p.T - (W - 1);  // first token copied into the carried-out state
+    for (int t = t0 + r0; t < t1; t += R) {
+        const int u = t - t0;
+        float dzr[W][N];
+#pragma unroll
+        for (int i = 0; i < W; ++i)
+#pragma unroll
+            for (int e = 0; e < N; e += 4) {
+                const float4 f = *reinterpret_cast<const float4*>(dzs + (size_t)(u + i) * p.D + c0 + e);
+                dzr[i][e] = f.x; dzr[i][e + 1] = f.y; dzr[i][e + 2] = f.z; dzr[i][e + 3] = f.w;
+            }
+        float g[N];
+#pragma unroll
+        for (int e = 0; e < N; ++e) {
+            float a = 0.0f;
+#pragma unroll
+            for (int i = 0; i < W; ++i) a = fmaf(wv[i][e], dzr[i][e], a);
+            g[e] = a;
+            ab[e] += dzr[0][e];
+        }
+#pragma unroll
+        for (int i = 0; i < W; ++i) {
+            float xv[N];
+            lds_vec(xs + (size_t)(t - i - lo) * p.D + c0, xv);
+#pragma unroll
+            for (int e = 0; e < N; ++e) aw[i][e] = fmaf(dzr[0][e], xv[e], aw[i][e]);
+        }
+        if (p.dxs_out != nullptr && t >= tout0) {
+            float go[N];
+            load_vec(static_cast<const T*>(p.dxs_out) + ((size_t)bh * (W - 1) + (t - tout0)) * p.D + c0, go);
+#pragma unroll
+            for (int e = 0; e < N; ++e) g[e] += go[e];
+        }
+        store_vec(dx + (size_t)t * p.D, g);
+    }
+    // weight and bias gradients: the lanes of a warp that hold the same channels
+    // (lanes cg, cg + CG, ...) by shuffles, one slot per warp in shared memory,
+    // a sum over the warps, then one float32 atomic per value and block
+    const int DW1 = p.D * (W + 1);
 #pragma unroll
     for (int e = 0; e < N; ++e) {
 #pragma unroll
         for (int i = 0; i <= W; ++i) {
             float x = i < W ? aw[i][e] : ab[e];
             for (int off = CG; off < 32; off <<= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
-            if (lane < CG) s_red[warp][(cg * (W + 1) + i) * N + e] = x;
+            if (lane < CG) s_red[warp * DW1 + (cg * (W + 1) + i) * N + e] = x;
         }
     }
     __syncthreads();
-    // CG divides 32, so every warp holds every channel group
-    for (int idx = threadIdx.x; idx < CG * (W + 1) * N; idx += kThreads) {
+    // CG divides 32 (D / N <= 32), so every warp holds every channel group
+    for (int idx = threadIdx.x; idx < DW1; idx += kThreads) {
         const int e = idx % N, i = (idx / N) % (W + 1), gi = idx / (N * (W + 1));
         float a = 0.0f;
 #pragma unroll
-        for (int w2 = 0; w2 < kThreads / 32; ++w2) a += s_red[w2][idx];
+        for (int w2 = 0; w2 < kThreads / 32; ++w2) a += s_red[w2 * DW1 + idx];
         const int c = gi * N + e;
         if (i < W) atomicAdd(p.dw + ((size_t)h * p.D + c) * W + i, a);
         else if (p.dbias) atomicAdd(p.dbias + (size_t)h * p.D + c, a);
     }
-    (void)R;
 }
 
 // gradient of the carried-in state: dxs[s] = sum_i w_i dz[s-(W-1)+i] over tokens
@@ -292,11 +413,32 @@ __global__ void conv_state_grad_kernel(ConvParams p) {
     }
 }
 
+// Tokens per block: tiles of 8192 elements (128 tokens at D = 64), at least W.
+int conv_tile(const ConvParams& p) { return std::max(8192 / p.D, 8); }
+
 template <typename T, int W>
-cudaError_t fwd_tw(const ConvParams& p, cudaStream_t s) {
-    const int R = kThreads / (p.D / Vec<T>::N);
-    const dim3 grid(p.B * p.H, (p.T + R * kRun - 1) / (R * kRun));
-    if (p.T > 0) conv_fwd_kernel<T, W><<<grid, kThreads, 0, s>>>(p);
+size_t fwd_smem(const ConvParams& p) {
+    return (size_t)(p.tile + W - 1) * p.D * sizeof(T);
+}
+
+template <typename T, int W>
+size_t bwd_smem(const ConvParams& p) {
+    return (size_t)(p.tile + 2 * (W - 1)) * p.D * sizeof(T) + (size_t)(p.tile + W - 1) * p.D * sizeof(T) +
+           (size_t)(p.tile + W - 1) * p.D * 4 + (size_t)(kThreads / 32) * p.D * (W + 1) * 4;
+}
+
+template <typename T, int W>
+cudaError_t fwd_tw(const ConvParams& p0, cudaStream_t s) {
+    ConvParams p = p0;
+    p.tile = conv_tile(p);
+    if (p.T > 0) {
+        const size_t smem = fwd_smem<T, W>(p);
+        auto kern = conv_fwd_kernel<T, W>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        const unsigned grid = (unsigned)((size_t)p.B * p.H * ((p.T + p.tile - 1) / p.tile));
+        kern<<<grid, kThreads, smem, s>>>(p);
+    }
     if (p.xs_out && W > 1) {
         const size_t n = (size_t)p.B * p.H * (W - 1) * p.D;
         conv_state_kernel<T><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(p);
@@ -305,20 +447,20 @@ cudaError_t fwd_tw(const ConvParams& p, cudaStream_t s) {
 }
 
 template <typename T, int W>
-cudaError_t bwd_tw(const ConvParams& p, cudaStream_t s) {
+cudaError_t bwd_tw(const ConvParams& p0, cudaStream_t s) {
+    ConvParams p = p0;
+    p.tile = conv_tile(p);
     cudaError_t e = cudaMemsetAsync(p.dw, 0, (size_t)p.H * p.D * W * sizeof(float), s);
     if (e == cudaSuccess && p.dbias) e = cudaMemsetAsync(p.dbias, 0, (size_t)p.H * p.D * sizeof(float), s);
     if (e != cudaSuccess) return e;
-    // tiles of `groups` R x kRun token groups: about four blocks per SM in all,
-    // so each block sums the weight gradients over several groups before its
-    // atomics
-    const int R = kThreads / (p.D / Vec<T>::N);
-    const int ngroups = (p.T + R * kRun - 1) / (R * kRun);
-    const int want_tiles = std::max(1, (4 * sm_count() + p.B * p.H - 1) / (p.B * p.H));
-    ConvParams q = p;
-    q.conv_groups = std::max(1, (ngroups + want_tiles - 1) / want_tiles);
-    const dim3 grid(p.B * p.H, (ngroups + q.conv_groups - 1) / q.conv_groups);
-    if (p.T > 0) conv_bwd_kernel<T, W><<<grid, kThreads, 0, s>>>(q);
+    if (p.T > 0) {
+        const size_t smem = bwd_smem<T, W>(p);
+        auto kern = conv_bwd_kernel<T, W>;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        const unsigned grid = (unsigned)((size_t)p.B * p.H * ((p.T + p.tile - 1) / p.tile));
+        kern<<<grid, kThreads, smem, s>>>(p);
+    }
     if constexpr (W > 1) {
         if (p.dxs) {
             const size_t n = (size_t)p.B * p.H * (W - 1) * (p.D / Vec<T>::N);

@@ -10,14 +10,15 @@
 //   o[b,h,t] = sum_u softmax(s)_u v[b,h,u]
 //
 // Forward (tensor cores, bf16 in, fp32 accumulation): one CTA per (b, h, tile
-// of 128 queries).  TMA brings the query tile once and the key and value tiles
-// of the window through a two-stage ring (128-byte swizzle, used by the MMA as
-// is); tcgen05 computes S = Q K^T into TMEM, four softmax warps (one query row
-// per thread) mask the window, keep the running row maximum and sum, write
-// P = 2^(S*c - m) as bf16 into shared memory, and tcgen05 computes P V into a
-// second TMEM buffer, which the same threads fold into registers with the
-// rescale exp2(m_old - m_new).  Issue order S_n, PV_{n-1} lets the softmax of
-// tile n overlap the P V product of tile n-1.
+// of 128 queries), two CTAs per SM where TMEM allows.  TMA brings the query
+// tile once and the 64-key tiles of the window through a three-stage ring
+// (128-byte swizzle, used by the MMA as is); tcgen05 computes S = Q K^T into
+// TMEM, eight softmax warps (two per query row, each with half of the keys and
+// half of the output columns) mask the window, keep the running row maximum and
+// sum, write P = 2^(S*c - m) as bf16 into shared memory, and tcgen05 computes
+// P V into a second TMEM buffer, which the same threads fold into registers
+// with the rescale exp2(m_old - m_new).  Issue order S_n, PV_{n-1} lets the
+// softmax of tile n overlap the P V product of tile n-1.
 //
 // Decode: one CTA per (b, h) against ring caches (position p in slot p mod w):
 // the new key and value are written to their slot and used from the inputs,

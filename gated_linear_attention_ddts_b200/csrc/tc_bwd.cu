@@ -859,7 +859,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                         for (int e = 0; e < 8; ++e) {
                             cb[e] = 1.0f;
                             if constexpr (PRE) {
-                                b8[e] = sigmoid_fast(b8[e]);
+                                b8[e] = sigmoid_tanh(b8[e]);
                                 cb[e] = b8[e] * (1.0f - b8[e]);
                             }
                         }

@@ -68,6 +68,10 @@ constexpr int kBarEpi = 4;         // named barrier of the epilogue warps
 constexpr int kMinSegChunks = 4;   // shortest segment worth a CTA of its own
 constexpr int kMaxSeg = 160;       // most segments per sequence
 constexpr int kAhead = 2;          // L2 prefetch distance of the producer, in passes
+// low-rank beta_hat: the factor u is read as 16 columns (ranks below 16 come
+// zero-filled from TMA, with zero rows of w_up): a 64 x 16 bf16 tile
+constexpr int kLrMax = 16;
+constexpr int kLrTileBytes = 64 * kLrMax * 2;
 
 template <int DK, int DVT>
 struct Cfg {
@@ -167,13 +171,15 @@ struct SegArgs {
 
 struct FwdKernelArgs {
     CUtensorMap mq, mk, mg, mt, mv, mb, mo;
+    CUtensorMap mu;  // low-rank beta_hat factor u [B][T][r] as boxes of 16 columns x 64 tokens
     CUtensorMap msv;  // saved states as [rows = B*H*NC*DK][dv] fp32 (when staged)
     SeqParams p;
     SegArgs seg;
 };
 
-// PRE: g, tau, beta arrive before their activations; FEED: o_t += d (.) v_t
-template <int DK, int DVT, bool PRE, bool FEED>
+// PRE: g, tau, beta arrive before their activations; FEED: o_t += d (.) v_t;
+// LR: beta_hat's pre-activation is u_t . w_up[h] (rank r <= 16), built on chip
+template <int DK, int DVT, bool PRE, bool FEED, bool LR>
 __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_constant__ FwdKernelArgs A) {
     using K = Cfg<DK, DVT>;
     constexpr int NS = K::NS, NB = K::NB, KB = K::KB, VB = K::VB;
@@ -246,7 +252,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
     }
     if (warp == kProdWarp && lane == 0) {
         prefetch_tmap(&A.mq); prefetch_tmap(&A.mk); prefetch_tmap(&A.mg);
-        prefetch_tmap(&A.mt); prefetch_tmap(&A.mv); prefetch_tmap(&A.mb); prefetch_tmap(&A.mo);
+        prefetch_tmap(&A.mt); prefetch_tmap(&A.mv); prefetch_tmap(&A.mo);
+        prefetch_tmap(LR ? &A.mu : &A.mb);
     }
     tc_fence_before();
     __syncthreads();
@@ -286,15 +293,18 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                     }
                     for (int vb = 0; vb < VB; ++vb) {
                         tma_prefetch_3d(&A.mv, j0 + 64 * vb, ca * C, bh);
-                        tma_prefetch_3d(&A.mb, j0 + 64 * vb, ca * C, bh);
+                        if constexpr (!LR) tma_prefetch_3d(&A.mb, j0 + 64 * vb, ca * C, bh);
                     }
                 }
                 if (li >= 1 && !mbar_wait(&sm.v_empty, (li - 1) & 1, fail, WL)) break;
-                mbar_expect_tx(&sm.v_full, K::RAWV);
+                mbar_expect_tx(&sm.v_full, LR ? VB * kBox + kLrTileBytes : K::RAWV);
                 for (int vb = 0; vb < VB; ++vb) {
                     tma_load_3d(sm.rawv + vb * kBox, &A.mv, &sm.v_full, j0 + 64 * vb, c * C, bh);
-                    tma_load_3d(sm.rawv + (VB + vb) * kBox, &A.mb, &sm.v_full, j0 + 64 * vb, c * C, bh);
+                    if constexpr (!LR)
+                        tma_load_3d(sm.rawv + (VB + vb) * kBox, &A.mb, &sm.v_full, j0 + 64 * vb, c * C, bh);
                 }
+                // the u rows of the chunk's tokens into the (otherwise unused) beta space
+                if constexpr (LR) tma_load_3d(sm.rawv + VB * kBox, &A.mu, &sm.v_full, 0, c * C, bh / p.H);
                 ++issued_v;
             }
             // never leave the CTA with copies in flight
@@ -855,6 +865,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             }
             return true;
         };
+        if constexpr (LR) {
+            // w_up[h][:, j0 .. j0 + DVT) as float32 [16][DVT] beside the u tile
+            // (rows r .. 15 zero), staged once for all chunks
+            float* wsm = reinterpret_cast<float*>(sm.rawv + VB * kBox + kLrTileBytes);
+            const int et = threadIdx.x - 32 * kEpiWarp0, hh = bh % p.H;
+            for (int i = et; i < kLrMax * DVT; i += 32 * kEpiWarps) {
+                const int rho = i / DVT, j = i % DVT;
+                wsm[i] = rho < p.beta_rank ? p.beta_w[((size_t)hh * p.beta_rank + rho) * p.dv + j0 + j] : 0.0f;
+            }
+            epi_sync();
+        }
         bool ok_run = true;
         if (P == 1) {
             load_s0();
@@ -878,6 +899,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                 if (item >= NB && !mbar_wait_own(&sm.ops_empty[ob], ((item / NB) - 1) & 1, fail, WL))
                     break;
                 const int et = threadIdx.x - 32 * kEpiWarp0;
+                // LR: this thread's token (the same for every item below) and its
+                // row of the u tile
+                float ur[LR ? kLrMax : 1];
+                if constexpr (LR) {
+                    const uint8_t* urow = sm.rawv + VB * kBox + (et % C) * (kLrMax * 2);
+                    unpack8(*reinterpret_cast<const uint4*>(urow), ur);
+                    unpack8(*reinterpret_cast<const uint4*>(urow + 16), ur + 8);
+                }
 #pragma unroll
                 for (int it = 0; it < (C * DVT / 8) / (32 * kEpiWarps); ++it) {
                     const int idx = et + 32 * kEpiWarps * it, jg = idx / C, t = idx % C;
@@ -888,7 +917,24 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                     if constexpr (PRE) {
                         float vf[8], bf8[8], of[8];
                         unpack8(v8, vf);
-                        unpack8(b8, bf8);
+                        if constexpr (LR) {
+                            // pre-activation u_t . w_up[:, jg*8 + e] (the warp reads
+                            // one w row: a shared-memory broadcast)
+                            const float4* w4 = reinterpret_cast<const float4*>(
+                                sm.rawv + VB * kBox + kLrTileBytes) + jg * 2;
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) bf8[e] = 0.0f;
+#pragma unroll
+                            for (int rho = 0; rho < kLrMax; ++rho) {
+                                const float4 wa = w4[rho * (DVT / 4)], wb = w4[rho * (DVT / 4) + 1];
+                                bf8[0] = fmaf(ur[rho], wa.x, bf8[0]); bf8[1] = fmaf(ur[rho], wa.y, bf8[1]);
+                                bf8[2] = fmaf(ur[rho], wa.z, bf8[2]); bf8[3] = fmaf(ur[rho], wa.w, bf8[3]);
+                                bf8[4] = fmaf(ur[rho], wb.x, bf8[4]); bf8[5] = fmaf(ur[rho], wb.y, bf8[5]);
+                                bf8[6] = fmaf(ur[rho], wb.z, bf8[6]); bf8[7] = fmaf(ur[rho], wb.w, bf8[7]);
+                            }
+                        } else {
+                            unpack8(b8, bf8);
+                        }
                         activate_beta8(bf8);
 #pragma unroll
                         for (int e = 0; e < 8; ++e) of[e] = vf[e] * bf8[e];
@@ -1100,7 +1146,7 @@ SegPlan choose_plan(const SeqParams& p, bool allow_seg) {
     return best;
 }
 
-template <int DK, int DVT, bool PRE, bool FEED>
+template <int DK, int DVT, bool PRE, bool FEED, bool LR>
 cudaError_t launch_cfg(const SeqParams& p, SegPlan plan, cudaStream_t s) {
     FwdKernelArgs a;
     a.p = p;
@@ -1110,15 +1156,17 @@ cudaError_t launch_cfg(const SeqParams& p, SegPlan plan, cudaStream_t s) {
         !make_tmap_bf16_3d(&a.mg, p.g, p.dk, p.T, BH, 64, 64) ||
         !make_tmap_bf16_3d(&a.mt, p.tau, p.dk, p.T, BH, 64, 64) ||
         !make_tmap_bf16_3d(&a.mv, p.v, p.dv, p.T, BH, 64, 64) ||
-        !make_tmap_bf16_3d(&a.mb, p.beta, p.dv, p.T, BH, 64, 64) ||
         !make_tmap_bf16_3d(&a.mo, p.o, p.dv, p.T, BH, 64, 64))
+        return cudaErrorInvalidValue;
+    if (LR ? !make_tmap_bf16_3d_plain(&a.mu, p.beta_u, p.beta_rank, p.T, p.B, kLrMax, 64)
+           : !make_tmap_bf16_3d(&a.mb, p.beta, p.dv, p.T, BH, 64, 64))
         return cudaErrorInvalidValue;
     if (Cfg<DK, DVT>::STAGE_SAVED && p.saved &&
         !make_tmap_f32_2d(&a.msv, p.saved, p.dv, BH * (uint64_t)((p.T + p.chunk - 1) / p.chunk) * DK,
                           32, DK))
         return cudaErrorInvalidValue;
     const size_t smem = sizeof(FwdSmem<DK, DVT>) + 1024;
-    auto kern = tc_fwd_kernel<DK, DVT, PRE, FEED>;
+    auto kern = tc_fwd_kernel<DK, DVT, PRE, FEED, LR>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const unsigned units = (unsigned)(BH * (p.dv / DVT));
@@ -1141,17 +1189,22 @@ cudaError_t launch_cfg(const SeqParams& p, SegPlan plan, cudaStream_t s) {
     return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
-template <bool PRE, bool FEED>
+template <bool PRE, bool FEED, bool LR>
 cudaError_t launch_plan_t(const SeqParams& p, const SegPlan& plan, cudaStream_t s) {
-    if (p.dk == 128) return launch_cfg<128, 64, PRE, FEED>(p, plan, s);
-    return plan.DVT == 128 ? launch_cfg<64, 128, PRE, FEED>(p, plan, s)
-                           : launch_cfg<64, 64, PRE, FEED>(p, plan, s);
+    if (p.dk == 128) return launch_cfg<128, 64, PRE, FEED, LR>(p, plan, s);
+    return plan.DVT == 128 ? launch_cfg<64, 128, PRE, FEED, LR>(p, plan, s)
+                           : launch_cfg<64, 64, PRE, FEED, LR>(p, plan, s);
+}
+
+template <bool FEED>
+cudaError_t launch_plan_f(const SeqParams& p, const SegPlan& plan, cudaStream_t s) {
+    if (p.beta_rank > 0) return launch_plan_t<true, FEED, true>(p, plan, s);  // implies preact
+    return p.preact ? launch_plan_t<true, FEED, false>(p, plan, s)
+                    : launch_plan_t<false, FEED, false>(p, plan, s);
 }
 
 cudaError_t launch_plan(const SeqParams& p, const SegPlan& plan, cudaStream_t s) {
-    if (p.dfeed)
-        return p.preact ? launch_plan_t<true, true>(p, plan, s) : launch_plan_t<false, true>(p, plan, s);
-    return p.preact ? launch_plan_t<true, false>(p, plan, s) : launch_plan_t<false, false>(p, plan, s);
+    return p.dfeed ? launch_plan_f<true>(p, plan, s) : launch_plan_f<false>(p, plan, s);
 }
 
 }  // namespace

@@ -41,6 +41,21 @@ bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t n0, uint64_t
     return r == CUDA_SUCCESS;
 }
 
+bool make_tmap_bf16_3d_plain(CUtensorMap* map, const void* base, uint64_t n0, uint64_t n1,
+                             uint64_t n2, uint32_t b0, uint32_t b1) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {n0, n1, n2};
+    cuuint64_t strides[2] = {n0 * 2, n0 * n1 * 2};
+    cuuint32_t box[3] = {b0, b1, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 bool make_tmap_f32_2d(CUtensorMap* map, const void* base, uint64_t n0, uint64_t n1, uint32_t b0,
                       uint32_t b1) {
     auto fn = encode_fn();

@@ -124,3 +124,13 @@ def draw_decode(B, H, dk, dv, steps, dtype=torch.bfloat16, seed=BASE_SEED + 4, m
 # (B, H, d, window, steps per timed graph).  q, k, v ~ N(0, 1) in bf16.
 SKA_FWD = (8, 12, 2048, 64, 512)
 SKA_DEC = (256, 16, 128, 512, 64)
+
+
+def draw_lowrank(B, H, T, dv, r, dtype=torch.bfloat16, seed=BASE_SEED + 40, device="cpu"):
+    """Factors of a low-rank beta_hat: u [B,T,r] ~ N(0, 1) in `dtype` (one row
+    per token, shared by the heads) and w_up [H,r,dv] ~ N(0, 1/r) float32."""
+    gen = _gen(device, seed)
+    f32 = dict(dtype=torch.float32, device=device, generator=gen)
+    u = torch.randn(B, T, r, **f32).to(dtype).contiguous()
+    w_up = (torch.randn(H, r, dv, **f32) / math.sqrt(r)).contiguous()
+    return u, w_up

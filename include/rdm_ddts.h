@@ -116,6 +116,18 @@ typedef enum { RDM_GATES_ACTIVATED = 0, RDM_GATES_PREACT = 1 } rdm_gate_inputs;
  *                  its shape nor its input; this library takes one weight per
  *                  head and value channel, constant over time, applied to v_t
  *                  (not to beta_hat * v_t).  Added in the store stage of o.
+ *   beta_rank    : 0, or the rank r (8 or 16) of a low-rank beta_hat (Rodimus*
+ *                  digest.lyk-ai.com summary, "Method": beta_hat is built from
+ *                  low-rank matrices to cut parameters and filter input noise).
+ *                  The reading taken: a per-token factor beta_u [B,T,r] dtype,
+ *                  shared by the heads (the token's input projected down to
+ *                  rank r), times an up-projection beta_w [H,r,d_v] float32
+ *                  gives beta_hat's pre-activation,
+ *                    beta_hat[b,h,t,j] = sigmoid(sum_rho beta_u[b,t,rho] beta_w[h,rho,j]),
+ *                  built on chip by the tensor-core kernel (beta is then
+ *                  ignored and may be NULL).  Requires RDM_GATES_PREACT and the
+ *                  tensor-core path (bf16, d_k and d_v in {64, 128}, chunk 16,
+ *                  32 or 64); RDM_ERR_UNSUPPORTED otherwise.
  */
 typedef struct {
     int B, H, T, dk, dv;
@@ -131,6 +143,9 @@ typedef struct {
     size_t workspace_bytes;
     rdm_gate_inputs gate_inputs;
     const float *feedthrough;
+    int beta_rank;
+    const void *beta_u;
+    const float *beta_w;
 } rdm_fwd_args;
 
 rdm_status rdm_ddts_fwd(const rdm_fwd_args *args, rdm_stream_t stream);
@@ -169,6 +184,14 @@ size_t rdm_ddts_saved_states_size(int B, int H, int T, int dk, int dv, int chunk
  *                  grad_o (.) v when non-NULL (requires feedthrough non-NULL;
  *                  accumulated with float32 atomics, so the summation order
  *                  may differ between calls).
+ *   beta_rank, beta_u, beta_w : the forward's low-rank beta_hat (beta_rank 0 =
+ *                  none).  With it grad_beta is not written (may be NULL) and
+ *                  grad_beta_u [B,T,r] dtype and grad_beta_w [H,r,d_v] float32
+ *                  receive the gradients of the factors (grad_beta_w summed with
+ *                  float32 atomics).  The backward expands the pre-activation
+ *                  into the workspace and contracts its gradient afterwards, so
+ *                  rdm_ddts_bwd_workspace_size grows by two [B,H,T,d_v] dtype
+ *                  buffers; both the tensor-core and the exact path take it.
  * Gradients with respect to g are undefined where g = 0 (g^(tau-1) is
  * unbounded there); d/dtau uses alpha_hat * ln g = 0 where alpha_hat = 0.
  */
@@ -189,6 +212,11 @@ typedef struct {
     rdm_gate_inputs gate_inputs;
     const float *feedthrough;
     float *grad_feedthrough;
+    int beta_rank;
+    const void *beta_u;
+    const float *beta_w;
+    void *grad_beta_u;
+    float *grad_beta_w;
 } rdm_bwd_args;
 
 rdm_status rdm_ddts_bwd(const rdm_bwd_args *args, rdm_stream_t stream);

@@ -1,7 +1,7 @@
 #!/usr/bin/env python
 """Small launches of each kernel, the command that profiler captures wrap.
 
-    python profile_kernels.py fwd1|fwd1pre|fwd1feed|fwd2|fwdbwd3|decode4|conv1|ska1|ska4
+    python profile_kernels.py fwd1|fwd1pre|fwd1feed|fwd1lr|fwd2|fwdbwd3|decode4|conv1|ska1|ska4
 
 One workload per call: the mode draws its inputs on the device, runs the
 kernel(s) three times and synchronises.  fwd1 is the 130M-scale layer forward
@@ -10,7 +10,8 @@ their activations, fwd2 the long-context forward (B1 H16 T32768 d_k=d_v=128),
 fwdbwd3 the training forward (saving chunk states) and backward (B4 H16 T4096
 d_k64 d_v128), decode4 four steps of the batched decode (B256 H16 d_k64 d_v128;
 only 4 steps of inputs are drawn instead of 1024, the kernel is the same),
-fwd1feed the 130M-scale layer forward with the feedthrough, conv1 the
+fwd1feed the 130M-scale layer forward with the feedthrough, fwd1lr the same
+layer with the gates passed before their activations and a rank-16 beta_hat, conv1 the
 ShortConv forward and backward (width 4, SiLU) on a q-shaped tensor of that
 layer (B8 H6 T2048 D64), ska1 the sliding-window shared-key attention forward
 (B8 H12 T2048 d_k=d_v=64, window 512) and ska4 its batched decode step against
@@ -25,20 +26,23 @@ sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
 
 import gated_linear_attention_ddts_b200 as rdm  # noqa: E402
 from gated_linear_attention_ddts_b200.workloads import (SKA_DEC, SKA_FWD, WORKLOADS,  # noqa: E402
-                                                        draw_decode, draw_workload)
+                                                        draw_decode, draw_lowrank, draw_workload)
 
 SEQ = ("q", "k", "v", "g", "tau", "beta")
 
 
 def main(mode: str) -> int:
-    if mode in ("fwd1", "fwd1pre", "fwd1feed", "fwd2"):
+    if mode in ("fwd1", "fwd1pre", "fwd1feed", "fwd2", "fwd1lr"):
         w = WORKLOADS[2 if mode == "fwd2" else 1]
-        pre = mode == "fwd1pre"
+        pre = mode in ("fwd1pre", "fwd1lr")
         x = draw_workload(w, device="cuda", preact=pre)
         d = torch.randn(w.H, w.dv, device="cuda") if mode == "fwd1feed" else None
+        lr = draw_lowrank(w.B, w.H, w.T, w.dv, 16, seed=w.seed + 40, device="cuda") \
+            if mode == "fwd1lr" else None
         for _ in range(3):
-            rdm.rdm_ddts_fwd(*(x[n] for n in SEQ), x["S0"], return_state=w.return_state,
-                             gates="preact" if pre else "activated", feedthrough=d)
+            rdm.rdm_ddts_fwd(*(x[n] for n in SEQ[:5]), None if lr else x["beta"], x["S0"],
+                             return_state=w.return_state, gates="preact" if pre else "activated",
+                             feedthrough=d, beta_lowrank=lr)
     elif mode == "conv1":
         w = WORKLOADS[1]
         x = torch.randn(w.B, w.H, w.T, w.dk, device="cuda").to(torch.bfloat16)

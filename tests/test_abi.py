@@ -67,6 +67,11 @@ def _fwd_args(**kw):
     (dict(dk=48), 2), (dict(dv=256), 2), (dict(chunk=48), 2), (dict(chunk=-2), 1),
     (dict(dtype=7), 1), (dict(impl=9), 1), (dict(q=None), 1), (dict(o=None), 1),
     (dict(k=(1 << 20) + 8), 1), (dict(S0=(1 << 20) + 4), 1), (dict(gate_inputs=7), 1),
+    # low-rank beta_hat: rank 8 or 16, pre-activation gates, factors given and aligned
+    (dict(beta_rank=-1), 1), (dict(beta_rank=4, gate_inputs=1, beta_u=1 << 20, beta_w=1 << 20), 2),
+    (dict(beta_rank=16, gate_inputs=0, beta_u=1 << 20, beta_w=1 << 20), 1),
+    (dict(beta_rank=16, gate_inputs=1, beta_u=None, beta_w=1 << 20), 1),
+    (dict(beta_rank=8, gate_inputs=1, beta_u=1 << 20, beta_w=(1 << 20) + 4), 1),
 ])
 def test_fwd_validation(lib, kw, status):
     a = _fwd_args(**kw)
@@ -90,6 +95,10 @@ def _bwd_args(**kw):
     (dict(impl=9), 1), (dict(gate_inputs=2), 1), (dict(grad_o=None), 1), (dict(q=None), 1),
     (dict(grad_q=(1 << 20) + 8), 1), (dict(grad_beta=None), 1), (dict(S0=(1 << 20) + 4), 1),
     (dict(saved_states=(1 << 20) + 4), 1), (dict(workspace=(1 << 20) + 2), 1),
+    (dict(beta_rank=32, gate_inputs=1, beta_u=1 << 20, beta_w=1 << 20), 2),
+    (dict(beta_rank=8, gate_inputs=1, beta_u=1 << 20, beta_w=1 << 20, grad_beta_w=1 << 20), 1),
+    (dict(beta_rank=8, gate_inputs=1, beta_u=1 << 20, beta_w=1 << 20, grad_beta_u=1 << 20,
+          grad_beta_w=(1 << 20) + 8), 1),
 ])
 def test_bwd_validation(lib, kw, status):
     """Host-side checks of the backward reject before touching the device."""
