@@ -7,16 +7,18 @@
 //
 // with x at t-i < 0 read from the carried-in state (the previous W-1 inputs).
 //
-// HBM-bound streaming through shared memory: a block takes a tile of tokens of
-// one (b, h) (8192 elements, 128 tokens at D = 64), whose rows are contiguous
-// in HBM, and has the bulk copy engine bring the tile and its W-1 row halo
-// into shared memory in one transfer (the backward: x and dy, with the halo on
-// both sides); the threads then work out of shared memory, 16 bytes of
-// channels of one token at a time, and store whole rows.  The backward first
-// writes dL/dz of the tile to shared memory (z recomputed from the staged x
-// when the SiLU is on), then forms dx and the weight and bias gradients, which
-// are reduced over the block (shuffles, then shared memory) before one float32
-// atomic per value and block.
+// HBM-bound streaming through shared memory: persistent blocks (two per SM)
+// take tiles of 8192 elements of one (b, h) (128 tokens at D = 64) in turn.
+// The rows of a tile are contiguous in HBM; thread 0 keeps a ring of tiles in
+// flight, each tile and its W-1 row halo arriving by one bulk copy (the
+// backward: x and dy, halos on both sides), so the copy engine streams while
+// the threads work out of shared memory on the tile before.  Forward threads
+// take a run of consecutive tokens of 16 bytes of channels, unpack each staged
+// row once and slide it through a window of the last W rows.  The backward
+// first writes dL/dz of the tile to shared memory (z recomputed from the
+// staged x when the SiLU is on), then forms dx and the weight and bias
+// gradients, reduced over the block (shuffles, then shared memory) before one
+// float32 atomic per value and tile.
 #include <algorithm>
 
 #include "launch.h"
@@ -29,7 +31,6 @@ namespace {
 using namespace tc;
 
 constexpr int kThreads = 256;
-constexpr int kRun = 4;  // tokens per thread (loops fully unrolled: every load in flight at once)
 
 template <typename T>
 struct Vec {
@@ -77,10 +78,12 @@ __device__ __forceinline__ void input_row(const ConvParams& p, int bh, int t, in
     }
 }
 
-__device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)); }
+// SiLU with the fast reciprocal-based division (__fdividef: 2 ulp where the
+// denominator 1 + e^-z is below 2^126, and 0 beyond, where z e^z < 1e-36)
+__device__ __forceinline__ float silu_f(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 // d silu / dz = s (1 + z (1 - s)), s = sigmoid(z)
 __device__ __forceinline__ float silu_grad(float z) {
-    const float s = 1.0f / (1.0f + __expf(-z));
+    const float s = __fdividef(1.0f, 1.0f + __expf(-z));
     return s * (1.0f + z * (1.0f - s));
 }
 
@@ -102,95 +105,153 @@ __device__ __forceinline__ void lds_vec(const __nv_bfloat16* p, float* f) {
 template <typename T>
 __device__ __forceinline__ T zero_val() { return T(0.0f); }
 
-// Stage the rows of tokens [lo, hi) of sequence bh (rows of D elements) into
-// dst: the in-sequence rows [max(lo, 0), min(hi, T)) are handed to the bulk
-// copy engine by thread 0 (the rows of one (b, h) are contiguous in HBM);
-// tokens before the sequence come from the carried-in state (zeros without
-// one, or when `state` is null), tokens past its end are zeros.  Returns the
-// bytes the bulk copy will deliver on `bar`.
-template <typename T, int W>
-__device__ uint32_t stage_rows(const ConvParams& p, const T* seq, const T* state, int bh, int lo,
-                               int hi, T* dst, uint64_t* bar) {
+constexpr int kConvStages = 3;     // tiles in flight per forward block
+constexpr int kConvBwdStages = 2;  // per backward block (two blocks per SM fit)
+
+// A tile: tokens [t0, t1) of sequence bh.
+struct ConvTile {
+    int bh, h, t0, t1;
+};
+__device__ __forceinline__ ConvTile conv_tile_of(const ConvParams& p, int g) {
+    const int ntile = (p.T + p.tile - 1) / p.tile;
+    ConvTile c;
+    c.bh = g / ntile;
+    c.h = c.bh % p.H;
+    c.t0 = (g % ntile) * p.tile;
+    c.t1 = min(c.t0 + p.tile, p.T);
+    return c;
+}
+
+// Thread 0: bulk copy of the in-sequence rows [max(lo, 0), min(hi, T)) of
+// sequence bh into dst, whose row 0 is token lo (the rows of one (b, h) are
+// contiguous in HBM).  Returns the bytes it will deliver on `bar`.
+template <typename T>
+__device__ uint32_t copy_rows(const ConvParams& p, const T* seq, int bh, int lo, int hi, T* dst,
+                              uint64_t* bar) {
     const int a = max(lo, 0), e = min(hi, p.T);
-    const uint32_t bytes = a < e ? (uint32_t)((size_t)(e - a) * p.D * sizeof(T)) : 0u;
-    if (threadIdx.x == 0 && bytes)
-        bulk_load(dst + (size_t)(a - lo) * p.D, seq + ((size_t)bh * p.T + a) * p.D, bytes, bar);
-    for (int i = threadIdx.x; i < (a - lo) * p.D; i += kThreads) {
-        const int s = W - 1 + lo + i / p.D;  // position in the carried-in state
-        dst[i] = (state && s >= 0) ? state[((size_t)bh * (W - 1) + s) * p.D + i % p.D] : zero_val<T>();
-    }
-    for (int i = (e - lo) * p.D + threadIdx.x; i < (hi - lo) * p.D; i += kThreads)
-        dst[i] = zero_val<T>();
+    if (a >= e) return 0u;
+    const uint32_t bytes = (uint32_t)((size_t)(e - a) * p.D * sizeof(T));
+    bulk_load(dst + (size_t)(a - lo) * p.D, seq + ((size_t)bh * p.T + a) * p.D, bytes, bar);
     return bytes;
 }
 
-// Every thread waits (bounded) for the staged rows.  A wait that runs out sets
-// the status word; the thread then waits once more, also bounded, so that no
-// copy lands after the block has left, and the block skips its work.
-__device__ __forceinline__ bool staged(uint64_t* bar, const ConvParams& p) {
-    const long long lim = p.wait_limit > 0 ? p.wait_limit : kDefaultWaitLimit;
-    long long t0 = clock64();
-    while (!mbar_try_wait(bar, 0))
-        if (clock64() - t0 > lim) {
-            atomicOr(p.err, kErrTimeout);
-            t0 = clock64();
-            while (!mbar_try_wait(bar, 0) && clock64() - t0 <= lim) {
-            }
-            return false;
-        }
-    return true;
-}
-
-// Forward: one block per tile of `p.tile` tokens of one (b, h).  The tile's
-// inputs and the W-1 rows before it are staged in shared memory by one bulk
-// copy; then thread (channel group cg, token lane r) produces 16 bytes of
-// channels for tokens t0 + r, t0 + r + R, ... (a warp stores whole rows).
+// The rows of tokens lo .. -1 (lo < 0, the tile at the start of a sequence)
+// from the carried-in state, zeros without one; all threads, then a barrier.
 template <typename T, int W>
-__global__ void __launch_bounds__(kThreads) conv_fwd_kernel(const ConvParams p) {
-    constexpr int N = Vec<T>::N;
-    extern __shared__ __align__(128) uint8_t conv_smem[];
-    __shared__ uint64_t bar;
-    T* xs = reinterpret_cast<T*>(conv_smem);  // rows of tokens [t0 - (W-1), t1)
-    const int CG = p.D / N, R = kThreads / CG;
-    const int ntile = (p.T + p.tile - 1) / p.tile;
-    const int bh = blockIdx.x / ntile, h = bh % p.H;
-    const int t0 = (blockIdx.x % ntile) * p.tile, t1 = min(t0 + p.tile, p.T);
-    const int lo = t0 - (W - 1);
-    if (threadIdx.x == 0) {
-        mbar_init(&bar, 1);
-        fence_mbar_init();
+__device__ void fill_state_rows(const ConvParams& p, int bh, int lo, T* dst) {
+    for (int i = threadIdx.x; i < -lo * p.D; i += kThreads) {
+        const int s = W - 1 + lo + i / p.D;  // position in the carried-in state
+        dst[i] = (p.xs && s >= 0) ? static_cast<const T*>(p.xs)[((size_t)bh * (W - 1) + s) * p.D + i % p.D]
+                                  : zero_val<T>();
     }
     __syncthreads();
-    const uint32_t bytes = stage_rows<T, W>(p, static_cast<const T*>(p.x), static_cast<const T*>(p.xs),
-                                            bh, lo, t1, xs, &bar);
-    if (threadIdx.x == 0) mbar_expect_tx(&bar, bytes);
-    const int cg = threadIdx.x % CG, r0 = threadIdx.x / CG, c0 = cg * N;
-    float wv[W][N], bv[N];
-#pragma unroll
-    for (int e = 0; e < N; ++e) {
-#pragma unroll
-        for (int i = 0; i < W; ++i) wv[i][e] = __ldg(p.w + ((size_t)h * p.D + c0 + e) * W + i);
-        bv[e] = p.bias ? __ldg(p.bias + (size_t)h * p.D + c0 + e) : 0.0f;
+}
+
+// Every thread waits (bounded) for phase `parity` of a stage; the block agrees
+// (a wait that ran out sets the status word and the block leaves together).
+__device__ __forceinline__ bool stage_ready(uint64_t* bar, uint32_t parity, const ConvParams& p) {
+    const long long lim = p.wait_limit > 0 ? p.wait_limit : kDefaultWaitLimit;
+    const long long t0 = clock64();
+    bool ok = true;
+    while (!mbar_try_wait(bar, parity))
+        if (clock64() - t0 > lim) {
+            ok = false;
+            break;
+        }
+    ok = __syncthreads_and(ok);
+    if (!ok && threadIdx.x == 0) atomicOr(p.err, kErrTimeout);
+    return ok;
+}
+
+// Before a block that gave up leaves: thread 0 waits (bounded) for the copies
+// still in flight into its S stages (tiles k .. k + S - 1 that exist).
+template <int S>
+__device__ void drain_stages(uint64_t* full, int k, int g, int total, const ConvParams& p) {
+    if (threadIdx.x != 0) return;
+    const long long lim = p.wait_limit > 0 ? p.wait_limit : kDefaultWaitLimit;
+    for (int j = 0; j < S && g + j * (int)gridDim.x < total; ++j) {
+        const int kk = k + j;
+        const long long t0 = clock64();
+        while (!mbar_try_wait(&full[kk % S], (kk / S) & 1) && clock64() - t0 <= lim) {
+        }
     }
-    __syncthreads();  // the rows the threads filled
-    if (!__syncthreads_and(staged(&bar, p))) return;  // the block leaves together
-    T* y = static_cast<T*>(p.y) + (size_t)bh * p.T * p.D + c0;
-    for (int t = t0 + r0; t < t1; t += R) {
-        float z[N];
+}
+
+// Forward: persistent blocks (two per SM) take tiles of `p.tile` tokens of one
+// (b, h) in turn.  Thread 0 keeps kConvStages tiles in flight: each tile's
+// rows and the W-1 rows before it arrive by one bulk copy into a ring stage;
+// then thread (channel group cg, run of RUN consecutive tokens) unpacks each
+// staged row once, slides it through a window of the last W rows and stores
+// 16 bytes of channels per token.
+template <typename T, int W>
+__global__ void __launch_bounds__(kThreads, 2) conv_fwd_kernel(const ConvParams p) {
+    constexpr int N = Vec<T>::N, RUN = 32 / N;
+    extern __shared__ __align__(128) uint8_t conv_smem[];
+    __shared__ uint64_t full[kConvStages];
+    const int CG = p.D / N;
+    const int total = p.B * p.H * ((p.T + p.tile - 1) / p.tile);
+    const size_t stage = (size_t)(p.tile + W - 1) * p.D;  // elements per ring stage
+    T* ring = reinterpret_cast<T*>(conv_smem);
+    auto issue = [&](int g, int s) {
+        const ConvTile c = conv_tile_of(p, g);
+        mbar_expect_tx(&full[s], (uint32_t)((size_t)(c.t1 - max(c.t0 - (W - 1), 0)) * p.D * sizeof(T)));
+        copy_rows<T>(p, static_cast<const T*>(p.x), c.bh, c.t0 - (W - 1), c.t1, ring + s * stage, &full[s]);
+    };
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kConvStages; ++s) mbar_init(&full[s], 1);
+        fence_mbar_init();
+        for (int s = 0; s < kConvStages; ++s)
+            if (blockIdx.x + s * (int)gridDim.x < total) issue(blockIdx.x + s * gridDim.x, s);
+    }
+    __syncthreads();
+    const int cg = threadIdx.x % CG, run = threadIdx.x / CG, c0 = cg * N;
+    int k = 0;
+    for (int g = blockIdx.x; g < total; g += gridDim.x, ++k) {
+        const int s = k % kConvStages;
+        const ConvTile c = conv_tile_of(p, g);
+        const int lo = c.t0 - (W - 1);
+        float wv[W][N], bv[N];
 #pragma unroll
-        for (int e = 0; e < N; ++e) z[e] = bv[e];
+        for (int e = 0; e < N; ++e) {
 #pragma unroll
-        for (int i = 0; i < W; ++i) {
-            float xv[N];
-            lds_vec(xs + (size_t)(t - i - lo) * p.D + c0, xv);
-#pragma unroll
-            for (int e = 0; e < N; ++e) z[e] = fmaf(wv[i][e], xv[e], z[e]);
+            for (int i = 0; i < W; ++i) wv[i][e] = __ldg(p.w + ((size_t)c.h * p.D + c0 + e) * W + i);
+            bv[e] = p.bias ? __ldg(p.bias + (size_t)c.h * p.D + c0 + e) : 0.0f;
         }
-        if (p.silu) {
-#pragma unroll
-            for (int e = 0; e < N; ++e) z[e] = silu_f(z[e]);
+        if (!stage_ready(&full[s], (k / kConvStages) & 1, p)) {
+            drain_stages<kConvStages>(full, k, g, total, p);
+            return;
         }
-        store_vec(y + (size_t)t * p.D, z);
+        T* xs = ring + s * stage;
+        if (W > 1 && lo < 0) fill_state_rows<T, W>(p, c.bh, lo, xs);
+        const int ta = c.t0 + run * RUN;
+        if (ta < c.t1) {
+            T* y = static_cast<T*>(p.y) + (size_t)c.bh * p.T * p.D + c0;
+            float win[W][N];  // win[j] = x[t - (W-1) + j]
+#pragma unroll
+            for (int j = 0; j < W - 1; ++j) lds_vec(xs + (size_t)(ta - (W - 1) + j - lo) * p.D + c0, win[j]);
+#pragma unroll
+            for (int r = 0; r < RUN; ++r) {
+                const int t = ta + r;
+                if (t >= c.t1) break;
+                lds_vec(xs + (size_t)(t - lo) * p.D + c0, win[W - 1]);
+                float z[N];
+#pragma unroll
+                for (int e = 0; e < N; ++e) {
+                    float a = bv[e];
+#pragma unroll
+                    for (int i = 0; i < W; ++i) a = fmaf(wv[i][e], win[W - 1 - i][e], a);
+                    z[e] = p.silu ? silu_f(a) : a;
+                }
+                store_vec(y + (size_t)t * p.D, z);
+#pragma unroll
+                for (int j = 0; j < W - 1; ++j)
+#pragma unroll
+                    for (int e = 0; e < N; ++e) win[j][e] = win[j + 1][e];
+            }
+        }
+        __syncthreads();  // stage s fully read: refill it with the tile kConvStages ahead
+        const int g2 = g + kConvStages * gridDim.x;
+        if (threadIdx.x == 0 && g2 < total) issue(g2, s);
     }
 }
 
@@ -235,142 +296,162 @@ __device__ __forceinline__ void dz_row(const ConvParams& p, int bh, int t, int c
     }
 }
 
-// Backward: one block per tile of `p.tile` tokens of one (b, h).  Staged: x of
-// tokens [t0 - (W-1), t1 + W - 1) and dy of [t0, t1 + W - 1) (bulk copies, as
-// in the forward).  Phase 1 writes dL/dz of tokens [t0, t1 + W - 1) (zero past
-// the end) to shared memory as float32; phase 2 gives dx[t] = sum_i w_i dz[t+i]
-// (plus the carried-out state's gradient where it copies x[t]) and accumulates
-// the weight and bias gradients, which are summed over the block and added
-// with one float32 atomic per value.
+// Backward: persistent blocks as in the forward.  A ring stage holds x of
+// tokens [t0 - (W-1), t1 + W - 1) and dy of [t0, t1 + W - 1) (two bulk copies
+// on one barrier).  Phase 1 writes dL/dz of tokens [t0, t1 + W - 1) (zero past
+// the end; z recomputed from the staged x for the SiLU) to shared memory as
+// float32; phase 2 gives dx[t] = sum_i w_i dz[t+i] (plus the carried-out
+// state's gradient where it copies x[t]) and the weight and bias partial sums,
+// reduced over the block (shuffles, then shared memory) and added with one
+// float32 atomic per value and tile.
 template <typename T, int W>
-__global__ void __launch_bounds__(kThreads) conv_bwd_kernel(const ConvParams p) {
+__global__ void __launch_bounds__(kThreads, 2) conv_bwd_kernel(const ConvParams p) {
     constexpr int N = Vec<T>::N;
     extern __shared__ __align__(128) uint8_t conv_smem[];
-    __shared__ uint64_t bar;
+    __shared__ uint64_t full[kConvBwdStages];
     const int TT = p.tile;
-    const int ntile = (p.T + TT - 1) / TT;
-    const int bh = blockIdx.x / ntile, h = bh % p.H;
-    const int t0 = (blockIdx.x % ntile) * TT, t1 = min(t0 + TT, p.T);
-    const int lo = t0 - (W - 1), hi = t1 + W - 1;   // x rows [lo, hi)
-    const int nz = hi - t0;                          // dz and dy rows [t0, hi)
-    T* xs = reinterpret_cast<T*>(conv_smem);
-    T* dys = xs + (size_t)(TT + 2 * (W - 1)) * p.D;
-    float* dzs = reinterpret_cast<float*>(dys + (size_t)(TT + W - 1) * p.D);
-    float* s_red = dzs + (size_t)(TT + W - 1) * p.D;   // [warps][D (W + 1)]
+    const int total = p.B * p.H * ((p.T + TT - 1) / TT);
+    const size_t xrows = TT + 2 * (W - 1), yrows = TT + W - 1;
+    const size_t stage = (xrows + yrows) * p.D;  // elements per ring stage
+    T* ring = reinterpret_cast<T*>(conv_smem);
+    float* dzs = reinterpret_cast<float*>(ring + kConvBwdStages * stage);
+    float* s_red = dzs + yrows * p.D;  // [warps][D (W + 1)]
     const int CG = p.D / N, R = kThreads / CG;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    auto issue = [&](int g, int s) {
+        const ConvTile c = conv_tile_of(p, g);
+        const int lo = c.t0 - (W - 1), hi = c.t1 + W - 1;
+        const size_t bx = (size_t)(min(hi, p.T) - max(lo, 0)) * p.D * sizeof(T);
+        const size_t by = (size_t)(min(hi, p.T) - c.t0) * p.D * sizeof(T);
+        mbar_expect_tx(&full[s], (uint32_t)(bx + by));
+        T* st = ring + s * stage;
+        copy_rows<T>(p, static_cast<const T*>(p.x), c.bh, lo, hi, st, &full[s]);
+        copy_rows<T>(p, static_cast<const T*>(p.dy), c.bh, c.t0, hi, st + xrows * p.D, &full[s]);
+    };
     if (threadIdx.x == 0) {
-        mbar_init(&bar, 1);
+        for (int s = 0; s < kConvBwdStages; ++s) mbar_init(&full[s], 1);
         fence_mbar_init();
+        for (int s = 0; s < kConvBwdStages; ++s)
+            if (blockIdx.x + s * (int)gridDim.x < total) issue(blockIdx.x + s * gridDim.x, s);
     }
     __syncthreads();
-    uint32_t bytes = stage_rows<T, W>(p, static_cast<const T*>(p.x), static_cast<const T*>(p.xs), bh,
-                                      lo, hi, xs, &bar);
-    bytes += stage_rows<T, W>(p, static_cast<const T*>(p.dy), nullptr, bh, t0, hi, dys, &bar);
-    if (threadIdx.x == 0) mbar_expect_tx(&bar, bytes);
     const int cg = threadIdx.x % CG, r0 = threadIdx.x / CG, c0 = cg * N;
-    float wv[W][N], bv[N], aw[W][N], ab[N];
-#pragma unroll
-    for (int e = 0; e < N; ++e) {
-#pragma unroll
-        for (int i = 0; i < W; ++i) {
-            wv[i][e] = __ldg(p.w + ((size_t)h * p.D + c0 + e) * W + i);
-            aw[i][e] = 0.0f;
-        }
-        bv[e] = p.bias ? __ldg(p.bias + (size_t)h * p.D + c0 + e) : 0.0f;
-        ab[e] = 0.0f;
-    }
-    __syncthreads();  // the rows the threads filled
-    if (!__syncthreads_and(staged(&bar, p))) return;  // the block leaves together
-    // phase 1: dz = dy, through the SiLU when on (z recomputed from the staged x)
-    for (int u = r0; u < nz; u += R) {
-        const int t = t0 + u;
-        float dz[N];
-        if (t < p.T) {
-            lds_vec(dys + (size_t)u * p.D + c0, dz);
-            if (p.silu) {
-                float z[N];
-#pragma unroll
-                for (int e = 0; e < N; ++e) z[e] = bv[e];
-#pragma unroll
-                for (int i = 0; i < W; ++i) {
-                    float xv[N];
-                    lds_vec(xs + (size_t)(t - i - lo) * p.D + c0, xv);
-#pragma unroll
-                    for (int e = 0; e < N; ++e) z[e] = fmaf(wv[i][e], xv[e], z[e]);
-                }
-#pragma unroll
-                for (int e = 0; e < N; ++e) dz[e] *= silu_grad(z[e]);
-            }
-        } else {
-#pragma unroll
-            for (int e = 0; e < N; ++e) dz[e] = 0.0f;
-        }
-        float* row = dzs + (size_t)u * p.D + c0;
-#pragma unroll
-        for (int e = 0; e < N; e += 4) *reinterpret_cast<float4*>(row + e) = make_float4(dz[e], dz[e + 1], dz[e + 2], dz[e + 3]);
-    }
-    __syncthreads();
-    // phase 2
-    T* dx = static_cast<T*>(p.dx) + (size_t)bh * p.T * p.D + c0;
     const int tout0 = p.T - (W - 1);  // first token copied into the carried-out state
-    for (int t = t0 + r0; t < t1; t += R) {
-        const int u = t - t0;
-        float dzr[W][N];
-#pragma unroll
-        for (int i = 0; i < W; ++i)
-#pragma unroll
-            for (int e = 0; e < N; e += 4) {
-                const float4 f = *reinterpret_cast<const float4*>(dzs + (size_t)(u + i) * p.D + c0 + e);
-                dzr[i][e] = f.x; dzr[i][e + 1] = f.y; dzr[i][e + 2] = f.z; dzr[i][e + 3] = f.w;
-            }
-        float g[N];
+    const int DW1 = p.D * (W + 1);
+    int k = 0;
+    for (int g = blockIdx.x; g < total; g += gridDim.x, ++k) {
+        const int s = k % kConvBwdStages;
+        const ConvTile c = conv_tile_of(p, g);
+        const int lo = c.t0 - (W - 1), nz = c.t1 + W - 1 - c.t0;
+        float wv[W][N], bv[N], aw[W][N], ab[N];
 #pragma unroll
         for (int e = 0; e < N; ++e) {
+#pragma unroll
+            for (int i = 0; i < W; ++i) {
+                wv[i][e] = __ldg(p.w + ((size_t)c.h * p.D + c0 + e) * W + i);
+                aw[i][e] = 0.0f;
+            }
+            bv[e] = p.bias ? __ldg(p.bias + (size_t)c.h * p.D + c0 + e) : 0.0f;
+            ab[e] = 0.0f;
+        }
+        if (!stage_ready(&full[s], (k / kConvBwdStages) & 1, p)) {
+            drain_stages<kConvBwdStages>(full, k, g, total, p);
+            return;
+        }
+        T* xs = ring + s * stage;
+        const T* dys = xs + xrows * p.D;
+        if (W > 1 && lo < 0) fill_state_rows<T, W>(p, c.bh, lo, xs);
+        // phase 1
+        for (int u = r0; u < nz; u += R) {
+            const int t = c.t0 + u;
+            float dz[N];
+            if (t < p.T) {
+                lds_vec(dys + (size_t)u * p.D + c0, dz);
+                if (p.silu) {
+                    float z[N];
+#pragma unroll
+                    for (int e = 0; e < N; ++e) z[e] = bv[e];
+#pragma unroll
+                    for (int i = 0; i < W; ++i) {
+                        float xv[N];
+                        lds_vec(xs + (size_t)(t - i - lo) * p.D + c0, xv);
+#pragma unroll
+                        for (int e = 0; e < N; ++e) z[e] = fmaf(wv[i][e], xv[e], z[e]);
+                    }
+#pragma unroll
+                    for (int e = 0; e < N; ++e) dz[e] *= silu_grad(z[e]);
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < N; ++e) dz[e] = 0.0f;
+            }
+            float* row = dzs + (size_t)u * p.D + c0;
+#pragma unroll
+            for (int e = 0; e < N; e += 4)
+                *reinterpret_cast<float4*>(row + e) = make_float4(dz[e], dz[e + 1], dz[e + 2], dz[e + 3]);
+        }
+        __syncthreads();
+        // phase 2
+        T* dx = static_cast<T*>(p.dx) + (size_t)c.bh * p.T * p.D + c0;
+        for (int t = c.t0 + r0; t < c.t1; t += R) {
+            const int u = t - c.t0;
+            float dzr[W][N];
+#pragma unroll
+            for (int i = 0; i < W; ++i)
+#pragma unroll
+                for (int e = 0; e < N; e += 4) {
+                    const float4 f = *reinterpret_cast<const float4*>(dzs + (size_t)(u + i) * p.D + c0 + e);
+                    dzr[i][e] = f.x; dzr[i][e + 1] = f.y; dzr[i][e + 2] = f.z; dzr[i][e + 3] = f.w;
+                }
+            float gx[N];
+#pragma unroll
+            for (int e = 0; e < N; ++e) {
+                float a = 0.0f;
+#pragma unroll
+                for (int i = 0; i < W; ++i) a = fmaf(wv[i][e], dzr[i][e], a);
+                gx[e] = a;
+                ab[e] += dzr[0][e];
+            }
+#pragma unroll
+            for (int i = 0; i < W; ++i) {
+                float xv[N];
+                lds_vec(xs + (size_t)(t - i - lo) * p.D + c0, xv);
+#pragma unroll
+                for (int e = 0; e < N; ++e) aw[i][e] = fmaf(dzr[0][e], xv[e], aw[i][e]);
+            }
+            if (p.dxs_out != nullptr && t >= tout0) {
+                float go[N];
+                load_vec(static_cast<const T*>(p.dxs_out) + ((size_t)c.bh * (W - 1) + (t - tout0)) * p.D + c0, go);
+#pragma unroll
+                for (int e = 0; e < N; ++e) gx[e] += go[e];
+            }
+            store_vec(dx + (size_t)t * p.D, gx);
+        }
+        // weight and bias gradients of the tile: lanes holding the same channels
+        // (cg, cg + CG, ...) by shuffles, one slot per warp, a sum over the warps
+#pragma unroll
+        for (int e = 0; e < N; ++e) {
+#pragma unroll
+            for (int i = 0; i <= W; ++i) {
+                float x = i < W ? aw[i][e] : ab[e];
+                for (int off = CG; off < 32; off <<= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+                if (lane < CG) s_red[warp * DW1 + (cg * (W + 1) + i) * N + e] = x;
+            }
+        }
+        __syncthreads();  // s_red written; stage s and dz fully read
+        const int g2 = g + kConvBwdStages * gridDim.x;
+        if (threadIdx.x == 0 && g2 < total) issue(g2, s);
+        // CG divides 32 (D / N <= 32), so every warp holds every channel group
+        for (int idx = threadIdx.x; idx < DW1; idx += kThreads) {
+            const int e = idx % N, i = (idx / N) % (W + 1), gi = idx / (N * (W + 1));
             float a = 0.0f;
 #pragma unroll
-            for (int i = 0; i < W; ++i) a = fmaf(wv[i][e], dzr[i][e], a);
-            g[e] = a;
-            ab[e] += dzr[0][e];
+            for (int w2 = 0; w2 < kThreads / 32; ++w2) a += s_red[w2 * DW1 + idx];
+            const int ch = gi * N + e;
+            if (i < W) atomicAdd(p.dw + ((size_t)c.h * p.D + ch) * W + i, a);
+            else if (p.dbias) atomicAdd(p.dbias + (size_t)c.h * p.D + ch, a);
         }
-#pragma unroll
-        for (int i = 0; i < W; ++i) {
-            float xv[N];
-            lds_vec(xs + (size_t)(t - i - lo) * p.D + c0, xv);
-#pragma unroll
-            for (int e = 0; e < N; ++e) aw[i][e] = fmaf(dzr[0][e], xv[e], aw[i][e]);
-        }
-        if (p.dxs_out != nullptr && t >= tout0) {
-            float go[N];
-            load_vec(static_cast<const T*>(p.dxs_out) + ((size_t)bh * (W - 1) + (t - tout0)) * p.D + c0, go);
-#pragma unroll
-            for (int e = 0; e < N; ++e) g[e] += go[e];
-        }
-        store_vec(dx + (size_t)t * p.D, g);
-    }
-    // weight and bias gradients: the lanes of a warp that hold the same channels
-    // (lanes cg, cg + CG, ...) by shuffles, one slot per warp in shared memory,
-    // a sum over the warps, then one float32 atomic per value and block
-    const int DW1 = p.D * (W + 1);
-#pragma unroll
-    for (int e = 0; e < N; ++e) {
-#pragma unroll
-        for (int i = 0; i <= W; ++i) {
-            float x = i < W ? aw[i][e] : ab[e];
-            for (int off = CG; off < 32; off <<= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
-            if (lane < CG) s_red[warp * DW1 + (cg * (W + 1) + i) * N + e] = x;
-        }
-    }
-    __syncthreads();
-    // CG divides 32 (D / N <= 32), so every warp holds every channel group
-    for (int idx = threadIdx.x; idx < DW1; idx += kThreads) {
-        const int e = idx % N, i = (idx / N) % (W + 1), gi = idx / (N * (W + 1));
-        float a = 0.0f;
-#pragma unroll
-        for (int w2 = 0; w2 < kThreads / 32; ++w2) a += s_red[w2 * DW1 + idx];
-        const int c = gi * N + e;
-        if (i < W) atomicAdd(p.dw + ((size_t)h * p.D + c) * W + i, a);
-        else if (p.dbias) atomicAdd(p.dbias + (size_t)h * p.D + c, a);
+        __syncthreads();  // s_red read before the next tile writes it
     }
 }
 
@@ -413,18 +494,26 @@ __global__ void conv_state_grad_kernel(ConvParams p) {
     }
 }
 
-// Tokens per block: tiles of 8192 elements (128 tokens at D = 64), at least W.
+// Tokens per tile: 8192 elements (128 tokens at D = 64).
 int conv_tile(const ConvParams& p) { return std::max(8192 / p.D, 8); }
 
 template <typename T, int W>
 size_t fwd_smem(const ConvParams& p) {
-    return (size_t)(p.tile + W - 1) * p.D * sizeof(T);
+    return (size_t)kConvStages * (p.tile + W - 1) * p.D * sizeof(T);
 }
 
 template <typename T, int W>
 size_t bwd_smem(const ConvParams& p) {
-    return (size_t)(p.tile + 2 * (W - 1)) * p.D * sizeof(T) + (size_t)(p.tile + W - 1) * p.D * sizeof(T) +
-           (size_t)(p.tile + W - 1) * p.D * 4 + (size_t)(kThreads / 32) * p.D * (W + 1) * 4;
+    const size_t stage = (size_t)(2 * p.tile + 3 * (W - 1)) * p.D * sizeof(T);
+    return kConvBwdStages * stage + (size_t)(p.tile + W - 1) * p.D * 4 +
+           (size_t)(kThreads / 32) * p.D * (W + 1) * 4;
+}
+
+// Persistent grid: two blocks per SM, or fewer when there are fewer tiles.
+unsigned conv_grid(const ConvParams& p) {
+    const long long tiles = (long long)p.B * p.H * ((p.T + p.tile - 1) / p.tile);
+    const long long cap = 2LL * sm_count();
+    return (unsigned)(tiles < cap ? tiles : cap);
 }
 
 template <typename T, int W>
@@ -436,8 +525,7 @@ cudaError_t fwd_tw(const ConvParams& p0, cudaStream_t s) {
         auto kern = conv_fwd_kernel<T, W>;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        const unsigned grid = (unsigned)((size_t)p.B * p.H * ((p.T + p.tile - 1) / p.tile));
-        kern<<<grid, kThreads, smem, s>>>(p);
+        kern<<<conv_grid(p), kThreads, smem, s>>>(p);
     }
     if (p.xs_out && W > 1) {
         const size_t n = (size_t)p.B * p.H * (W - 1) * p.D;
@@ -458,8 +546,7 @@ cudaError_t bwd_tw(const ConvParams& p0, cudaStream_t s) {
         auto kern = conv_bwd_kernel<T, W>;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        const unsigned grid = (unsigned)((size_t)p.B * p.H * ((p.T + p.tile - 1) / p.tile));
-        kern<<<grid, kThreads, smem, s>>>(p);
+        kern<<<conv_grid(p), kThreads, smem, s>>>(p);
     }
     if constexpr (W > 1) {
         if (p.dxs) {

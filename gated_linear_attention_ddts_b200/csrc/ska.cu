@@ -11,7 +11,7 @@
 //
 // Forward (tensor cores, bf16 in, fp32 accumulation): one CTA per (b, h, tile
 // of 128 queries), two CTAs per SM where TMEM allows.  TMA brings the query
-// tile once and the 64-key tiles of the window through a three-stage ring
+// tile once and the 64-key tiles of the window through rings of four key and three value stages
 // (128-byte swizzle, used by the MMA as is); tcgen05 computes S = Q K^T into
 // TMEM, eight softmax warps (two per query row, each with half of the keys and
 // half of the output columns) mask the window, keep the running row maximum and
@@ -44,7 +44,6 @@ constexpr int kQRows = 128;          // queries per CTA (MMA M)
 constexpr int kSoftWarps = 8;
 constexpr int kProdWarp = 8, kMmaWarp = 9;
 constexpr int kSkaThreads = 320;
-constexpr int kStages = 3;  // key and value tiles in flight
 
 // 128-byte-swizzle shared-memory descriptor (sm_100 layout type 2): K-major
 // tiles of 64-element (128-byte) rows in 8-row, 1024-byte atoms, or MN-major
@@ -63,17 +62,24 @@ struct SkaCfg {
     // S and P V double-buffered; 256 columns let two CTAs share an SM
     static constexpr uint32_t TMEM_COLS = 2 * NK + 2 * DV <= 256 ? 256 : 512;
     static constexpr int CTAS_PER_SM = TMEM_COLS == 256 && DK == 64 ? 2 : 1;
+    // key and value tiles in flight (a tile takes a few microseconds to land
+    // when every SM streams; keys run further ahead, the MMA waits on them first)
+    static constexpr int KS = 4, VS = 3;
 };
 
 template <int DK, int DV>
 struct SkaSmem {
     using K = SkaCfg<DK, DV>;
     alignas(1024) uint8_t q[K::Q_BYTES];
-    alignas(1024) uint8_t k[kStages][K::K_BYTES];
-    alignas(1024) uint8_t v[kStages][K::V_BYTES];
+    alignas(1024) uint8_t k[K::KS][K::K_BYTES];
+    alignas(1024) uint8_t v[K::VS][K::V_BYTES];
     alignas(1024) uint8_t p[2][K::P_BYTES];  // no-swizzle K-major (8x8 core matrices)
-    uint64_t q_full, k_full[kStages], v_full[kStages], k_empty[kStages], v_empty[kStages];
-    uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2], o_full[2], o_empty[2], mma_done;
+    uint64_t q_full, k_full[K::KS], v_full[K::VS], k_empty[K::KS], v_empty[K::VS];
+    // S, P and O buffers need no "empty" barriers: the MMA thread writes S_n and
+    // O_n only after p_full of tile n-2 (resp. n), on which every softmax warp
+    // arrives after it has read S_{n-2} (resp. folded O_{n-2}), and the softmax
+    // writes P_n only after o_full of tile n-2 (P V of tile n-2 done)
+    uint64_t s_full[2], p_full[2], o_full[2], mma_done;
     float red_max[2][2][kQRows];  // [tile parity][column half][row]: partial row maxima
     float red_sum[2][kQRows];     // [column half][row]: partial row sums at the end
     uint32_t tmem_base;
@@ -84,6 +90,19 @@ struct SkaKernelArgs {
     SkaParams p;
     CUtensorMap mq, mk, mv;
 };
+
+// Non-blocking probe of an mbarrier phase (test_wait returns at once; a
+// try_wait would suspend the thread for a while when the phase is open, which
+// would hold the producer on one ring while the other has a free stage).
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n"
+        " mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+    return ok != 0;
+}
 
 // Warp-uniform bounded wait of the softmax warps: every lane waits on its own
 // clock (never on the shared failure flag, which another role may raise at any
@@ -123,19 +142,18 @@ __global__ void __launch_bounds__(kSkaThreads, SkaCfg<DK, DV>::CTAS_PER_SM)
 
     if (threadIdx.x == 0) {
         mbar_init(&sm.q_full, 1);
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < K::KS; ++s) {
             mbar_init(&sm.k_full[s], 1);
-            mbar_init(&sm.v_full[s], 1);
             mbar_init(&sm.k_empty[s], 1);
+        }
+        for (int s = 0; s < K::VS; ++s) {
+            mbar_init(&sm.v_full[s], 1);
             mbar_init(&sm.v_empty[s], 1);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&sm.s_full[s], 1);
-            mbar_init(&sm.s_empty[s], kSoftWarps);
             mbar_init(&sm.p_full[s], kSoftWarps);
-            mbar_init(&sm.p_empty[s], 1);
             mbar_init(&sm.o_full[s], 1);
-            mbar_init(&sm.o_empty[s], kSoftWarps);
         }
         mbar_init(&sm.mma_done, 1);
         sm.fail = 0;
@@ -162,32 +180,49 @@ __global__ void __launch_bounds__(kSkaThreads, SkaCfg<DK, DV>::CTAS_PER_SM)
 #pragma unroll
             for (int x = 0; x < DK / 64; ++x)
                 tma_load_3d(sm.q + x * kQRows * 128, &A.mq, &sm.q_full, 64 * x, t0, bh);
+            // keys and values refill independently: a key stage frees after
+            // Q K^T, a value stage after P V; whichever ring has a free stage is
+            // served (polled), so key prefetch never waits behind a value slot
             int nk = 0, nv = 0;  // key / value tiles issued
-            for (int n = 0; n < NT; ++n) {
-                const int st = n % kStages;
-                const uint32_t ph = ((n / kStages) & 1) ^ 1;
-                const int kb = (j_lo + n) * NK;
-                // the key stage frees after Q K^T, the value stage after P V
-                if (!mbar_wait(&sm.k_empty[st], ph, fail, WL)) break;
-                mbar_expect_tx(&sm.k_full[st], K::K_BYTES);
+            long long idle0 = clock64();
+            while (nk < NT || nv < NT) {
+                bool moved = false;
+                if (nk < NT && mbar_test(&sm.k_empty[nk % K::KS], ((nk / K::KS) & 1) ^ 1)) {
+                    const int st = nk % K::KS;
+                    mbar_expect_tx(&sm.k_full[st], K::K_BYTES);
 #pragma unroll
-                for (int x = 0; x < DK / 64; ++x)
-                    tma_load_3d(sm.k[st] + x * NK * 128, &A.mk, &sm.k_full[st], 64 * x, kb, b);
-                ++nk;
-                if (!mbar_wait(&sm.v_empty[st], ph, fail, WL)) break;
-                mbar_expect_tx(&sm.v_full[st], K::V_BYTES);
+                    for (int x = 0; x < DK / 64; ++x)
+                        tma_load_3d(sm.k[st] + x * NK * 128, &A.mk, &sm.k_full[st], 64 * x,
+                                    (j_lo + nk) * NK, b);
+                    ++nk;
+                    moved = true;
+                }
+                if (nv < nk && mbar_test(&sm.v_empty[nv % K::VS], ((nv / K::VS) & 1) ^ 1)) {
+                    const int st = nv % K::VS;
+                    mbar_expect_tx(&sm.v_full[st], K::V_BYTES);
 #pragma unroll
-                for (int x = 0; x < DV / 64; ++x)
-                    tma_load_3d(sm.v[st] + x * NK * 128, &A.mv, &sm.v_full[st], 64 * x, kb, bh);
-                ++nv;
+                    for (int x = 0; x < DV / 64; ++x)
+                        tma_load_3d(sm.v[st] + x * NK * 128, &A.mv, &sm.v_full[st], 64 * x,
+                                    (j_lo + nv) * NK, bh);
+                    ++nv;
+                    moved = true;
+                }
+                if (moved) {
+                    idle0 = clock64();
+                } else if (*fail) {
+                    break;
+                } else if (clock64() - idle0 > WL) {
+                    *fail = 1;
+                    break;
+                }
             }
             // no copy may land after the CTA has gone: wait (bounded, on our own
             // clock) for the last ones issued into each stage and for the query
             mbar_wait_own(&sm.q_full, 0, fail, WL);
-            for (int n = nk - kStages > 0 ? nk - kStages : 0; n < nk; ++n)
-                mbar_wait_own(&sm.k_full[n % kStages], (n / kStages) & 1, fail, WL);
-            for (int n = nv - kStages > 0 ? nv - kStages : 0; n < nv; ++n)
-                mbar_wait_own(&sm.v_full[n % kStages], (n / kStages) & 1, fail, WL);
+            for (int n = nk - K::KS > 0 ? nk - K::KS : 0; n < nk; ++n)
+                mbar_wait_own(&sm.k_full[n % K::KS], (n / K::KS) & 1, fail, WL);
+            for (int n = nv - K::VS > 0 ? nv - K::VS : 0; n < nv; ++n)
+                mbar_wait_own(&sm.v_full[n % K::VS], (n / K::VS) & 1, fail, WL);
         }
         __syncwarp();
     } else if (warp == kMmaWarp) {
@@ -197,28 +232,28 @@ __global__ void __launch_bounds__(kSkaThreads, SkaCfg<DK, DV>::CTAS_PER_SM)
             constexpr uint32_t idO = idesc_bf16(kQRows, DV, 0, 1);  // O = P V (V MN-major)
             const uint32_t qa = smem_u32(sm.q);
             auto pv = [&](int m) -> bool {
-                const int st = m & 1, vs = m % kStages;
+                const int st = m & 1, vs = m % K::VS;
                 const uint32_t ph = (m >> 1) & 1;
+                // p_full[m] also means the softmax has read O_{m-2} out of buffer
+                // st (each warp folds tile m-2 before it writes P_m)
                 if (!mbar_wait(&sm.p_full[st], ph, fail, WL)) return false;
-                if (!mbar_wait(&sm.o_empty[st], ph ^ 1, fail, WL)) return false;
-                if (!mbar_wait(&sm.v_full[vs], (m / kStages) & 1, fail, WL)) return false;
+                if (!mbar_wait(&sm.v_full[vs], (m / K::VS) & 1, fail, WL)) return false;
                 tc_fence_after();
                 const uint32_t pa = smem_u32(sm.p[st]), va = smem_u32(sm.v[vs]);
 #pragma unroll
                 for (int ks = 0; ks < NK / 16; ++ks)
                     mma_bf16(tO + st * DV, sdesc(pa + ks * 256, 128, NK * 16),
                              sdesc_sw128(va + ks * 2048, NK * 128, 1024), idO, ks > 0);
-                mma_commit(&sm.o_full[st]);
+                mma_commit(&sm.o_full[st]);  // also frees P buffer st for P_{m+2}
                 mma_commit(&sm.v_empty[vs]);
-                mma_commit(&sm.p_empty[st]);
                 return true;
             };
             bool ok = mbar_wait(&sm.q_full, 0, fail, WL);
             for (int n = 0; ok && n < NT; ++n) {
-                const int st = n & 1, ks_ = n % kStages;
-                const uint32_t ph = (n >> 1) & 1;
-                if (!mbar_wait(&sm.k_full[ks_], (n / kStages) & 1, fail, WL) ||
-                    !mbar_wait(&sm.s_empty[st], ph ^ 1, fail, WL)) {
+                const int st = n & 1, ks_ = n % K::KS;
+                // S buffer st is free: p_full of tile n-2 (waited in pv(n-2) above)
+                // comes after every softmax warp loaded S_{n-2}
+                if (!mbar_wait(&sm.k_full[ks_], (n / K::KS) & 1, fail, WL)) {
                     ok = false;
                     break;
                 }
@@ -263,9 +298,7 @@ __global__ void __launch_bounds__(kSkaThreads, SkaCfg<DK, DV>::CTAS_PER_SM)
             for (int q32 = 0; q32 < DH / 32; ++q32)
                 tmem_ld32(tO + st * DV + half * DH + lane_off + q32 * 32, x + q32 * 32);
             tmem_ld_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.o_empty[st]);
+            tc_fence_before();  // ordered before the next p_full arrival
 #pragma unroll
             for (int j = 0; j < DH; ++j) o[j] = fmaf(o[j], cr, x[j]);
             return true;
@@ -284,9 +317,7 @@ __global__ void __launch_bounds__(kSkaThreads, SkaCfg<DK, DV>::CTAS_PER_SM)
             for (int q32 = 0; q32 < NH / 32; ++q32)
                 tmem_ld32(tS + st * NK + half * NH + lane_off + q32 * 32, s_ + q32 * 32);
             tmem_ld_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.s_empty[st]);
+            tc_fence_before();  // ordered before this tile's p_full arrival
             const int kb = (j_lo + n) * NK + half * NH;
             if (kb < lo || kb + NH - 1 > hi) {
 #pragma unroll
@@ -310,7 +341,7 @@ __global__ void __launch_bounds__(kSkaThreads, SkaCfg<DK, DV>::CTAS_PER_SM)
             }
             l = fmaf(l, corr, (l4[0] + l4[1]) + (l4[2] + l4[3]));
             m_run = m_new;
-            if (!warp_wait(&sm.p_empty[st], ph ^ 1, fail, WL)) { ok = false; break; }
+            // P buffer st is free: o_full of tile n-2 was waited in fold(n-2)
             // P row r, keys 8*kc .. 8*kc+7 -> core matrix (r/8, kc): byte
             // (r/8)*(NK*16) + kc*128 + (r%8)*16
             uint8_t* prow = sm.p[st] + (r >> 3) * (NK * 16) + (r & 7) * 16 + half * (NH / 8) * 128;

@@ -56,6 +56,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // callers then skip the remaining work and exit cleanly.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* fail,
                                           long long limit) {
+    if (mbar_try_wait(bar, parity)) return true;  // the common case: no clock, no flag read
     if (*fail) return false;
     const long long t0 = clock64();
     while (true) {
@@ -78,6 +79,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 // other roles and the status word) and returns false.
 __device__ __forceinline__ bool mbar_wait_own(uint64_t* bar, uint32_t parity, volatile int* fail,
                                               long long limit) {
+    if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
         if (mbar_try_wait(bar, parity))
