@@ -100,6 +100,7 @@ FWD_SRC = ["tc_fwd.cu"] + _DEV_HDR
 BWD_SRC = ["tc_bwd.cu"] + _DEV_HDR
 DECODE_SRC = ["decode.cu", "rdm_common.cuh", "launch.h"]
 SKA_SRC = ["ska.cu", "ska_launch.h"] + _DEV_HDR
+CONV_SRC = ["shortconv.cu"] + _DEV_HDR
 
 
 def src_sha(*names):

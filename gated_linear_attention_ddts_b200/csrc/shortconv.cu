@@ -32,9 +32,11 @@ using namespace tc;
 
 constexpr int kThreads = 256;
 
+// Four channels per thread (8 bytes of bf16, 16 of float32): small register
+// footprints, so four blocks fit an SM and hide the shared-memory latencies.
 template <typename T>
 struct Vec {
-    static constexpr int N = 16 / sizeof(T);  // channels per 16-byte group
+    static constexpr int N = 4;
 };
 
 // inputs are read through the read-only path (x, dy and the states are never
@@ -45,23 +47,19 @@ __device__ __forceinline__ void load_vec(const float* p, float* f) {
     f[0] = u.x; f[1] = u.y; f[2] = u.z; f[3] = u.w;
 }
 __device__ __forceinline__ void load_vec(const __nv_bfloat16* p, float* f) {
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        f[2 * e] = __uint_as_float(w[e] << 16);
-        f[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
-    }
+    const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+    f[0] = __uint_as_float(u.x << 16); f[1] = __uint_as_float(u.x & 0xffff0000u);
+    f[2] = __uint_as_float(u.y << 16); f[3] = __uint_as_float(u.y & 0xffff0000u);
 }
 __device__ __forceinline__ void store_vec(float* p, const float* f) {
     *reinterpret_cast<float4*>(p) = make_float4(f[0], f[1], f[2], f[3]);
 }
 __device__ __forceinline__ void store_vec(__nv_bfloat16* p, const float* f) {
-    uint4 u;
+    uint2 u;
     __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) h[e] = __floats2bfloat162_rn(f[2 * e], f[2 * e + 1]);
-    *reinterpret_cast<uint4*>(p) = u;
+    h[0] = __floats2bfloat162_rn(f[0], f[1]);
+    h[1] = __floats2bfloat162_rn(f[2], f[3]);
+    *reinterpret_cast<uint2*>(p) = u;
 }
 
 // input row t (t < 0: from the carried-in state, zeros without one) of my channels
@@ -93,13 +91,9 @@ __device__ __forceinline__ void lds_vec(const float* p, float* f) {
     f[0] = u.x; f[1] = u.y; f[2] = u.z; f[3] = u.w;
 }
 __device__ __forceinline__ void lds_vec(const __nv_bfloat16* p, float* f) {
-    const uint4 u = *reinterpret_cast<const uint4*>(p);
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        f[2 * e] = __uint_as_float(w[e] << 16);
-        f[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
-    }
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    f[0] = __uint_as_float(u.x << 16); f[1] = __uint_as_float(u.x & 0xffff0000u);
+    f[2] = __uint_as_float(u.y << 16); f[3] = __uint_as_float(u.y & 0xffff0000u);
 }
 
 template <typename T>
@@ -166,10 +160,10 @@ __device__ __forceinline__ bool stage_ready(uint64_t* bar, uint32_t parity, cons
 // Before a block that gave up leaves: thread 0 waits (bounded) for the copies
 // still in flight into its S stages (tiles k .. k + S - 1 that exist).
 template <int S>
-__device__ void drain_stages(uint64_t* full, int k, int g, int total, const ConvParams& p) {
+__device__ void drain_stages(uint64_t* full, int k, int g, int g1, const ConvParams& p) {
     if (threadIdx.x != 0) return;
     const long long lim = p.wait_limit > 0 ? p.wait_limit : kDefaultWaitLimit;
-    for (int j = 0; j < S && g + j * (int)gridDim.x < total; ++j) {
+    for (int j = 0; j < S && g + j < g1; ++j) {
         const int kk = k + j;
         const long long t0 = clock64();
         while (!mbar_try_wait(&full[kk % S], (kk / S) & 1) && clock64() - t0 <= lim) {
@@ -177,19 +171,22 @@ __device__ void drain_stages(uint64_t* full, int k, int g, int total, const Conv
     }
 }
 
-// Forward: persistent blocks (two per SM) take tiles of `p.tile` tokens of one
-// (b, h) in turn.  Thread 0 keeps kConvStages tiles in flight: each tile's
+// Forward: persistent blocks (four per SM) take contiguous runs of tiles of
+// `p.tile` tokens of one (b, h).  Thread 0 keeps kConvStages tiles in flight: each tile's
 // rows and the W-1 rows before it arrive by one bulk copy into a ring stage;
 // then thread (channel group cg, run of RUN consecutive tokens) unpacks each
 // staged row once, slides it through a window of the last W rows and stores
 // 16 bytes of channels per token.
 template <typename T, int W>
-__global__ void __launch_bounds__(kThreads, 2) conv_fwd_kernel(const ConvParams p) {
+__global__ void __launch_bounds__(kThreads, 4) conv_fwd_kernel(const ConvParams p) {
     constexpr int N = Vec<T>::N, RUN = 32 / N;
     extern __shared__ __align__(128) uint8_t conv_smem[];
     __shared__ uint64_t full[kConvStages];
     const int CG = p.D / N;
     const int total = p.B * p.H * ((p.T + p.tile - 1) / p.tile);
+    // a contiguous run of tiles per block (same sequence, mostly the same head)
+    const int per = (total + (int)gridDim.x - 1) / (int)gridDim.x;
+    const int g0 = blockIdx.x * per, g1 = min(total, g0 + per);
     const size_t stage = (size_t)(p.tile + W - 1) * p.D;  // elements per ring stage
     T* ring = reinterpret_cast<T*>(conv_smem);
     auto issue = [&](int g, int s) {
@@ -201,24 +198,28 @@ __global__ void __launch_bounds__(kThreads, 2) conv_fwd_kernel(const ConvParams 
         for (int s = 0; s < kConvStages; ++s) mbar_init(&full[s], 1);
         fence_mbar_init();
         for (int s = 0; s < kConvStages; ++s)
-            if (blockIdx.x + s * (int)gridDim.x < total) issue(blockIdx.x + s * gridDim.x, s);
+            if (g0 + s < g1) issue(g0 + s, s);
     }
     __syncthreads();
     const int cg = threadIdx.x % CG, run = threadIdx.x / CG, c0 = cg * N;
+    float wv[W][N], bv[N];
+    int cur_h = -1;
     int k = 0;
-    for (int g = blockIdx.x; g < total; g += gridDim.x, ++k) {
+    for (int g = g0; g < g1; ++g, ++k) {
         const int s = k % kConvStages;
         const ConvTile c = conv_tile_of(p, g);
         const int lo = c.t0 - (W - 1);
-        float wv[W][N], bv[N];
+        if (c.h != cur_h) {  // consecutive tiles mostly share the head
+            cur_h = c.h;
 #pragma unroll
-        for (int e = 0; e < N; ++e) {
+            for (int e = 0; e < N; ++e) {
 #pragma unroll
-            for (int i = 0; i < W; ++i) wv[i][e] = __ldg(p.w + ((size_t)c.h * p.D + c0 + e) * W + i);
-            bv[e] = p.bias ? __ldg(p.bias + (size_t)c.h * p.D + c0 + e) : 0.0f;
+                for (int i = 0; i < W; ++i) wv[i][e] = __ldg(p.w + ((size_t)c.h * p.D + c0 + e) * W + i);
+                bv[e] = p.bias ? __ldg(p.bias + (size_t)c.h * p.D + c0 + e) : 0.0f;
+            }
         }
         if (!stage_ready(&full[s], (k / kConvStages) & 1, p)) {
-            drain_stages<kConvStages>(full, k, g, total, p);
+            drain_stages<kConvStages>(full, k, g, g1, p);
             return;
         }
         T* xs = ring + s * stage;
@@ -250,8 +251,7 @@ __global__ void __launch_bounds__(kThreads, 2) conv_fwd_kernel(const ConvParams 
             }
         }
         __syncthreads();  // stage s fully read: refill it with the tile kConvStages ahead
-        const int g2 = g + kConvStages * gridDim.x;
-        if (threadIdx.x == 0 && g2 < total) issue(g2, s);
+        if (threadIdx.x == 0 && g + kConvStages < g1) issue(g + kConvStages, s);
     }
 }
 
@@ -296,21 +296,24 @@ __device__ __forceinline__ void dz_row(const ConvParams& p, int bh, int t, int c
     }
 }
 
-// Backward: persistent blocks as in the forward.  A ring stage holds x of
+// Backward: persistent blocks (three per SM) with contiguous runs of tiles of
+// 4096 elements, as in the forward.  A ring stage holds x of
 // tokens [t0 - (W-1), t1 + W - 1) and dy of [t0, t1 + W - 1) (two bulk copies
 // on one barrier).  Phase 1 writes dL/dz of tokens [t0, t1 + W - 1) (zero past
 // the end; z recomputed from the staged x for the SiLU) to shared memory as
 // float32; phase 2 gives dx[t] = sum_i w_i dz[t+i] (plus the carried-out
 // state's gradient where it copies x[t]) and the weight and bias partial sums,
 // reduced over the block (shuffles, then shared memory) and added with one
-// float32 atomic per value and tile.
+// float32 atomic per value for each run of tiles of one head.
 template <typename T, int W>
-__global__ void __launch_bounds__(kThreads, 2) conv_bwd_kernel(const ConvParams p) {
+__global__ void __launch_bounds__(kThreads, 3) conv_bwd_kernel(const ConvParams p) {
     constexpr int N = Vec<T>::N;
     extern __shared__ __align__(128) uint8_t conv_smem[];
     __shared__ uint64_t full[kConvBwdStages];
     const int TT = p.tile;
     const int total = p.B * p.H * ((p.T + TT - 1) / TT);
+    const int per = (total + (int)gridDim.x - 1) / (int)gridDim.x;
+    const int g0 = blockIdx.x * per, g1 = min(total, g0 + per);
     const size_t xrows = TT + 2 * (W - 1), yrows = TT + W - 1;
     const size_t stage = (xrows + yrows) * p.D;  // elements per ring stage
     T* ring = reinterpret_cast<T*>(conv_smem);
@@ -332,30 +335,61 @@ __global__ void __launch_bounds__(kThreads, 2) conv_bwd_kernel(const ConvParams 
         for (int s = 0; s < kConvBwdStages; ++s) mbar_init(&full[s], 1);
         fence_mbar_init();
         for (int s = 0; s < kConvBwdStages; ++s)
-            if (blockIdx.x + s * (int)gridDim.x < total) issue(blockIdx.x + s * gridDim.x, s);
+            if (g0 + s < g1) issue(g0 + s, s);
     }
     __syncthreads();
     const int cg = threadIdx.x % CG, r0 = threadIdx.x / CG, c0 = cg * N;
     const int tout0 = p.T - (W - 1);  // first token copied into the carried-out state
     const int DW1 = p.D * (W + 1);
-    int k = 0;
-    for (int g = blockIdx.x; g < total; g += gridDim.x, ++k) {
-        const int s = k % kConvBwdStages;
-        const ConvTile c = conv_tile_of(p, g);
-        const int lo = c.t0 - (W - 1), nz = c.t1 + W - 1 - c.t0;
-        float wv[W][N], bv[N], aw[W][N], ab[N];
+    float wv[W][N], bv[N], aw[W][N], ab[N];
+    // weight and bias gradients summed over the block's tiles of head h: lanes
+    // holding the same channels (cg, cg + CG, ...) by shuffles, one slot per
+    // warp in shared memory, a sum over the warps, one float32 atomic per value
+    auto flush = [&](int h) {
 #pragma unroll
         for (int e = 0; e < N; ++e) {
 #pragma unroll
-            for (int i = 0; i < W; ++i) {
-                wv[i][e] = __ldg(p.w + ((size_t)c.h * p.D + c0 + e) * W + i);
-                aw[i][e] = 0.0f;
+            for (int i = 0; i <= W; ++i) {
+                float x = i < W ? aw[i][e] : ab[e];
+                for (int off = CG; off < 32; off <<= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+                if (lane < CG) s_red[warp * DW1 + (cg * (W + 1) + i) * N + e] = x;
             }
-            bv[e] = p.bias ? __ldg(p.bias + (size_t)c.h * p.D + c0 + e) : 0.0f;
-            ab[e] = 0.0f;
+        }
+        __syncthreads();
+        // CG divides 32 (D / N <= 32), so every warp holds every channel group
+        for (int idx = threadIdx.x; idx < DW1; idx += kThreads) {
+            const int e = idx % N, i = (idx / N) % (W + 1), gi = idx / (N * (W + 1));
+            float a = 0.0f;
+#pragma unroll
+            for (int w2 = 0; w2 < kThreads / 32; ++w2) a += s_red[w2 * DW1 + idx];
+            const int ch = gi * N + e;
+            if (i < W) atomicAdd(p.dw + ((size_t)h * p.D + ch) * W + i, a);
+            else if (p.dbias) atomicAdd(p.dbias + (size_t)h * p.D + ch, a);
+        }
+        __syncthreads();  // s_red read before it is written again
+    };
+    int cur_h = -1;
+    int k = 0;
+    for (int g = g0; g < g1; ++g, ++k) {
+        const int s = k % kConvBwdStages;
+        const ConvTile c = conv_tile_of(p, g);
+        const int lo = c.t0 - (W - 1), nz = c.t1 + W - 1 - c.t0;
+        if (c.h != cur_h) {  // block-uniform
+            if (cur_h >= 0) flush(cur_h);
+            cur_h = c.h;
+#pragma unroll
+            for (int e = 0; e < N; ++e) {
+#pragma unroll
+                for (int i = 0; i < W; ++i) {
+                    wv[i][e] = __ldg(p.w + ((size_t)c.h * p.D + c0 + e) * W + i);
+                    aw[i][e] = 0.0f;
+                }
+                bv[e] = p.bias ? __ldg(p.bias + (size_t)c.h * p.D + c0 + e) : 0.0f;
+                ab[e] = 0.0f;
+            }
         }
         if (!stage_ready(&full[s], (k / kConvBwdStages) & 1, p)) {
-            drain_stages<kConvBwdStages>(full, k, g, total, p);
+            drain_stages<kConvBwdStages>(full, k, g, g1, p);
             return;
         }
         T* xs = ring + s * stage;
@@ -385,10 +419,7 @@ __global__ void __launch_bounds__(kThreads, 2) conv_bwd_kernel(const ConvParams 
 #pragma unroll
                 for (int e = 0; e < N; ++e) dz[e] = 0.0f;
             }
-            float* row = dzs + (size_t)u * p.D + c0;
-#pragma unroll
-            for (int e = 0; e < N; e += 4)
-                *reinterpret_cast<float4*>(row + e) = make_float4(dz[e], dz[e + 1], dz[e + 2], dz[e + 3]);
+            *reinterpret_cast<float4*>(dzs + (size_t)u * p.D + c0) = make_float4(dz[0], dz[1], dz[2], dz[3]);
         }
         __syncthreads();
         // phase 2
@@ -397,12 +428,10 @@ __global__ void __launch_bounds__(kThreads, 2) conv_bwd_kernel(const ConvParams 
             const int u = t - c.t0;
             float dzr[W][N];
 #pragma unroll
-            for (int i = 0; i < W; ++i)
-#pragma unroll
-                for (int e = 0; e < N; e += 4) {
-                    const float4 f = *reinterpret_cast<const float4*>(dzs + (size_t)(u + i) * p.D + c0 + e);
-                    dzr[i][e] = f.x; dzr[i][e + 1] = f.y; dzr[i][e + 2] = f.z; dzr[i][e + 3] = f.w;
-                }
+            for (int i = 0; i < W; ++i) {
+                const float4 f = *reinterpret_cast<const float4*>(dzs + (size_t)(u + i) * p.D + c0);
+                dzr[i][0] = f.x; dzr[i][1] = f.y; dzr[i][2] = f.z; dzr[i][3] = f.w;
+            }
             float gx[N];
 #pragma unroll
             for (int e = 0; e < N; ++e) {
@@ -427,32 +456,10 @@ __global__ void __launch_bounds__(kThreads, 2) conv_bwd_kernel(const ConvParams 
             }
             store_vec(dx + (size_t)t * p.D, gx);
         }
-        // weight and bias gradients of the tile: lanes holding the same channels
-        // (cg, cg + CG, ...) by shuffles, one slot per warp, a sum over the warps
-#pragma unroll
-        for (int e = 0; e < N; ++e) {
-#pragma unroll
-            for (int i = 0; i <= W; ++i) {
-                float x = i < W ? aw[i][e] : ab[e];
-                for (int off = CG; off < 32; off <<= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
-                if (lane < CG) s_red[warp * DW1 + (cg * (W + 1) + i) * N + e] = x;
-            }
-        }
-        __syncthreads();  // s_red written; stage s and dz fully read
-        const int g2 = g + kConvBwdStages * gridDim.x;
-        if (threadIdx.x == 0 && g2 < total) issue(g2, s);
-        // CG divides 32 (D / N <= 32), so every warp holds every channel group
-        for (int idx = threadIdx.x; idx < DW1; idx += kThreads) {
-            const int e = idx % N, i = (idx / N) % (W + 1), gi = idx / (N * (W + 1));
-            float a = 0.0f;
-#pragma unroll
-            for (int w2 = 0; w2 < kThreads / 32; ++w2) a += s_red[w2 * DW1 + idx];
-            const int ch = gi * N + e;
-            if (i < W) atomicAdd(p.dw + ((size_t)c.h * p.D + ch) * W + i, a);
-            else if (p.dbias) atomicAdd(p.dbias + (size_t)c.h * p.D + ch, a);
-        }
-        __syncthreads();  // s_red read before the next tile writes it
+        __syncthreads();  // stage s and dz fully read: refill the stage
+        if (threadIdx.x == 0 && g + kConvBwdStages < g1) issue(g + kConvBwdStages, s);
     }
+    if (cur_h >= 0) flush(cur_h);
 }
 
 // gradient of the carried-in state: dxs[s] = sum_i w_i dz[s-(W-1)+i] over tokens
@@ -494,8 +501,9 @@ __global__ void conv_state_grad_kernel(ConvParams p) {
     }
 }
 
-// Tokens per tile: 8192 elements (128 tokens at D = 64).
+// Tokens per tile: 8192 elements (128 tokens at D = 64) forward, 4096 backward.
 int conv_tile(const ConvParams& p) { return std::max(8192 / p.D, 8); }
+int conv_tile_bwd(const ConvParams& p) { return std::max(4096 / p.D, 8); }
 
 template <typename T, int W>
 size_t fwd_smem(const ConvParams& p) {
@@ -509,10 +517,10 @@ size_t bwd_smem(const ConvParams& p) {
            (size_t)(kThreads / 32) * p.D * (W + 1) * 4;
 }
 
-// Persistent grid: two blocks per SM, or fewer when there are fewer tiles.
-unsigned conv_grid(const ConvParams& p) {
+// Persistent grid: `per_sm` blocks per SM, or fewer when there are fewer tiles.
+unsigned conv_grid(const ConvParams& p, int per_sm) {
     const long long tiles = (long long)p.B * p.H * ((p.T + p.tile - 1) / p.tile);
-    const long long cap = 2LL * sm_count();
+    const long long cap = (long long)per_sm * sm_count();
     return (unsigned)(tiles < cap ? tiles : cap);
 }
 
@@ -525,7 +533,7 @@ cudaError_t fwd_tw(const ConvParams& p0, cudaStream_t s) {
         auto kern = conv_fwd_kernel<T, W>;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        kern<<<conv_grid(p), kThreads, smem, s>>>(p);
+        kern<<<conv_grid(p, 4), kThreads, smem, s>>>(p);
     }
     if (p.xs_out && W > 1) {
         const size_t n = (size_t)p.B * p.H * (W - 1) * p.D;
@@ -537,7 +545,7 @@ cudaError_t fwd_tw(const ConvParams& p0, cudaStream_t s) {
 template <typename T, int W>
 cudaError_t bwd_tw(const ConvParams& p0, cudaStream_t s) {
     ConvParams p = p0;
-    p.tile = conv_tile(p);
+    p.tile = conv_tile_bwd(p);
     cudaError_t e = cudaMemsetAsync(p.dw, 0, (size_t)p.H * p.D * W * sizeof(float), s);
     if (e == cudaSuccess && p.dbias) e = cudaMemsetAsync(p.dbias, 0, (size_t)p.H * p.D * sizeof(float), s);
     if (e != cudaSuccess) return e;
@@ -546,7 +554,7 @@ cudaError_t bwd_tw(const ConvParams& p0, cudaStream_t s) {
         auto kern = conv_bwd_kernel<T, W>;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        kern<<<conv_grid(p), kThreads, smem, s>>>(p);
+        kern<<<conv_grid(p, 3), kThreads, smem, s>>>(p);
     }
     if constexpr (W > 1) {
         if (p.dxs) {

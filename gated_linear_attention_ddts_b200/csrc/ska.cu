@@ -45,12 +45,10 @@ constexpr int kSoftWarps = 8;
 constexpr int kProdWarp = 8, kMmaWarp = 9;
 constexpr int kSkaThreads = 320;
 
-// 128-byte-swizzle shared-memory descriptor (sm_100 layout type 2): K-major
-// tiles of 64-element (128-byte) rows in 8-row, 1024-byte atoms, or MN-major
-// tiles whose 64-element rows run along M/N.
-__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-    return sdesc(saddr, lbo, sbo) | (2ull << 61);
-}
+// Shared-memory operands: K-major 128-byte-swizzled TMA tiles (Q, K: rows of
+// 64 elements in 8-row, 1024-byte atoms; descriptor layout type 2 of sm_100),
+// MN-major 128-byte-swizzled V tiles (64-element rows along N), and P in the
+// no-swizzle K-major layout of 8x8 core matrices.
 
 template <int DK, int DV>
 struct SkaCfg {
@@ -230,7 +228,18 @@ __global__ void __launch_bounds__(kSkaThreads, SkaCfg<DK, DV>::CTAS_PER_SM)
         if (lane == 0) {
             constexpr uint32_t idS = idesc_bf16(kQRows, NK, 0, 0);  // S = Q K^T
             constexpr uint32_t idO = idesc_bf16(kQRows, DV, 0, 1);  // O = P V (V MN-major)
-            const uint32_t qa = smem_u32(sm.q);
+            // Descriptors as two 32-bit words, built once: the low word is the
+            // start address / 16 plus the leading offset, so the operand of step
+            // ks of stage s is base + a constant (one add per MMA); the high word
+            // (stride offset, sm_100 version bit, layout) is fixed per operand.
+            constexpr uint32_t kSw128 = 2u << 29;
+            const uint32_t q_lo = (smem_u32(sm.q) >> 4) | (1u << 16);
+            const uint32_t k_lo = (smem_u32(sm.k[0]) >> 4) | (1u << 16);
+            const uint32_t p_lo = (smem_u32(sm.p[0]) >> 4) | ((128u >> 4) << 16);
+            const uint32_t v_lo = (smem_u32(sm.v[0]) >> 4) | (((uint32_t)NK * 128 >> 4) << 16);
+            constexpr uint32_t qk_hi = (1024u >> 4) | (1u << 14) | kSw128;
+            constexpr uint32_t p_hi = ((uint32_t)NK * 16 >> 4) | (1u << 14);
+            constexpr uint32_t v_hi = (1024u >> 4) | (1u << 14) | kSw128;
             auto pv = [&](int m) -> bool {
                 const int st = m & 1, vs = m % K::VS;
                 const uint32_t ph = (m >> 1) & 1;
@@ -239,11 +248,11 @@ __global__ void __launch_bounds__(kSkaThreads, SkaCfg<DK, DV>::CTAS_PER_SM)
                 if (!mbar_wait(&sm.p_full[st], ph, fail, WL)) return false;
                 if (!mbar_wait(&sm.v_full[vs], (m / K::VS) & 1, fail, WL)) return false;
                 tc_fence_after();
-                const uint32_t pa = smem_u32(sm.p[st]), va = smem_u32(sm.v[vs]);
+                const uint32_t pa = p_lo + st * (K::P_BYTES >> 4), va = v_lo + vs * (K::V_BYTES >> 4);
 #pragma unroll
                 for (int ks = 0; ks < NK / 16; ++ks)
-                    mma_bf16(tO + st * DV, sdesc(pa + ks * 256, 128, NK * 16),
-                             sdesc_sw128(va + ks * 2048, NK * 128, 1024), idO, ks > 0);
+                    mma_bf16_w(tO + st * DV, pa + ks * (256 >> 4), p_hi, va + ks * (2048 >> 4), v_hi, idO,
+                               ks > 0);
                 mma_commit(&sm.o_full[st]);  // also frees P buffer st for P_{m+2}
                 mma_commit(&sm.v_empty[vs]);
                 return true;
@@ -258,12 +267,12 @@ __global__ void __launch_bounds__(kSkaThreads, SkaCfg<DK, DV>::CTAS_PER_SM)
                     break;
                 }
                 tc_fence_after();
-                const uint32_t ka = smem_u32(sm.k[ks_]);
+                const uint32_t ka = k_lo + ks_ * (K::K_BYTES >> 4);
 #pragma unroll
                 for (int ks = 0; ks < DK / 16; ++ks) {
-                    const int x = ks / 4, off = (ks % 4) * 32;
-                    mma_bf16(tS + st * NK, sdesc_sw128(qa + x * kQRows * 128 + off, 16, 1024),
-                             sdesc_sw128(ka + x * NK * 128 + off, 16, 1024), idS, ks > 0);
+                    const uint32_t off = ((ks / 4) * (kQRows * 128) + (ks % 4) * 32) >> 4;
+                    const uint32_t koff = ((ks / 4) * (NK * 128) + (ks % 4) * 32) >> 4;
+                    mma_bf16_w(tS + st * NK, q_lo + off, qk_hi, ka + koff, qk_hi, idS, ks > 0);
                 }
                 mma_commit(&sm.s_full[st]);
                 mma_commit(&sm.k_empty[ks_]);
@@ -458,6 +467,12 @@ __global__ void __launch_bounds__(kDecThreads) ska_decode_kernel(const SkaDecode
     const __nv_bfloat16* kc = static_cast<const __nv_bfloat16*>(p.k_cache) + (size_t)b * w * DK;
     const __nv_bfloat16* vc = static_cast<const __nv_bfloat16*>(p.v_cache) + (size_t)bh * w * DV;
     const float c = p.scale * kLog2e;
+    // start the value rows (and, once per sequence, the shared key rows) toward
+    // L2 while the scores are formed, so the value sweep reads from L2
+    if (threadIdx.x == 0) {
+        bulk_prefetch_l2(vc, (uint32_t)n * DV * 2);
+        if (h == 0) bulk_prefetch_l2(kc, (uint32_t)n * DK * 2);
+    }
     for (int i = threadIdx.x; i < DK; i += kDecThreads)
         qs[i] = __bfloat162float(static_cast<const __nv_bfloat16*>(p.q)[(size_t)bh * DK + i]) * c;
     // write the new token into its slot
