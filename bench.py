@@ -365,7 +365,8 @@ def run_extras(rdm, dev, pk, K):
     out["feedthrough_fwd"] = {
         "workload": w.name + ", feedthrough o += d * v", "value": w.B * w.T / (ms / 1e3),
         "unit": "tokens/s", "ms_per_step": ms, "gpu_launches_per_step": 1,
-        "roofline": roofline(fwd_bytes(w, False) + w.H * w.dv * 4, chunk_flops_fwd(w), ms, pk, None)}
+        "roofline": roofline(fwd_bytes(w, False) + w.H * w.dv * 4, chunk_flops_fwd(w), ms, pk,
+                             ncu_counters("tc_fwd_kernel", FWD_SRC, "1feed"))}
     del x, o, wsf, dfe
     # ShortConv (width 4, SiLU) forward + backward on the q, k and v tensors of
     # the same layer (D = 64, 64, 128)

@@ -76,12 +76,22 @@ __device__ __forceinline__ void input_row(const ConvParams& p, int bh, int t, in
     }
 }
 
-// SiLU with the fast reciprocal-based division (__fdividef: 2 ulp where the
-// denominator 1 + e^-z is below 2^126, and 0 beyond, where z e^z < 1e-36)
-__device__ __forceinline__ float silu_f(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
-// d silu / dz = s (1 + z (1 - s)), s = sigmoid(z)
-__device__ __forceinline__ float silu_grad(float z) {
-    const float s = __fdividef(1.0f, 1.0f + __expf(-z));
+// SiLU(z) = z sigmoid(z) and d SiLU / dz = s (1 + z (1 - s)), s = sigmoid(z).
+// float32 path: sigmoid through the fast reciprocal-based division
+// (__fdividef: 2 ulp while the denominator 1 + e^-z is below 2^126, and 0
+// beyond, where z e^z < 1e-36).  bf16 path, whose outputs carry 8 significant
+// bits: sigmoid(z) = (1 + tanh(z/2)) / 2 with the single-instruction tanh
+// (relative error about 2^-11), one MUFU operation per element instead of an
+// exponential and a reciprocal.
+template <typename T>
+__device__ __forceinline__ float sigmoid_t(float z) { return __fdividef(1.0f, 1.0f + __expf(-z)); }
+template <>
+__device__ __forceinline__ float sigmoid_t<__nv_bfloat16>(float z) { return sigmoid_tanh(z); }
+template <typename T>
+__device__ __forceinline__ float silu_t(float z) { return z * sigmoid_t<T>(z); }
+template <typename T>
+__device__ __forceinline__ float silu_grad_t(float z) {
+    const float s = sigmoid_t<T>(z);
     return s * (1.0f + z * (1.0f - s));
 }
 
@@ -241,7 +251,7 @@ __global__ void __launch_bounds__(kThreads, 4) conv_fwd_kernel(const ConvParams 
                     float a = bv[e];
 #pragma unroll
                     for (int i = 0; i < W; ++i) a = fmaf(wv[i][e], win[W - 1 - i][e], a);
-                    z[e] = p.silu ? silu_f(a) : a;
+                    z[e] = p.silu ? silu_t<T>(a) : a;
                 }
                 store_vec(y + (size_t)t * p.D, z);
 #pragma unroll
@@ -291,7 +301,7 @@ __device__ __forceinline__ void dz_row(const ConvParams& p, int bh, int t, int c
             float a = bv[e];
 #pragma unroll
             for (int i = 0; i < W; ++i) a = fmaf(wv[i][e], xw[i][e], a);
-            dz[e] *= silu_grad(a);
+            dz[e] *= silu_grad_t<T>(a);
         }
     }
 }
@@ -413,7 +423,7 @@ __global__ void __launch_bounds__(kThreads, 3) conv_bwd_kernel(const ConvParams 
                         for (int e = 0; e < N; ++e) z[e] = fmaf(wv[i][e], xv[e], z[e]);
                     }
 #pragma unroll
-                    for (int e = 0; e < N; ++e) dz[e] *= silu_grad(z[e]);
+                    for (int e = 0; e < N; ++e) dz[e] *= silu_grad_t<T>(z[e]);
                 }
             } else {
 #pragma unroll
