@@ -20,9 +20,11 @@
 // with the rescale exp2(m_old - m_new).  Issue order S_n, PV_{n-1} lets the
 // softmax of tile n overlap the P V product of tile n-1.
 //
-// Decode: one CTA per (b, h) against ring caches (position p in slot p mod w):
-// the new key and value are written to their slot and used from the inputs,
-// scores go through shared memory, then a coalesced sweep over the value rows.
+// Decode: one CTA per (b, group of up to eight heads) against ring caches
+// (position p in slot p mod w): the new key and value are written to their slot
+// and used from the inputs, each cached key row is read once for the group's
+// heads, scores go through shared memory, then a coalesced sweep over the
+// value rows of each head.
 #include <cuda_bf16.h>
 #include <stdint.h>
 
@@ -428,109 +430,148 @@ __global__ void ska_cache_fill_kernel(const SkaParams p) {
 // ------------------------------------------------------------------ decode
 constexpr int kDecThreads = 256;
 
-__device__ __forceinline__ float block_reduce(float x, float* red, bool is_max) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        const float y = __shfl_xor_sync(0xffffffffu, x, o);
-        x = is_max ? fmaxf(x, y) : x + y;
-    }
-    __syncthreads();  // red may still be read from the previous reduction
-    if (lane == 0) red[warp] = x;
-    __syncthreads();
-    x = red[0];
-#pragma unroll
-    for (int w = 1; w < kDecThreads / 32; ++w) x = is_max ? fmaxf(x, red[w]) : x + red[w];
-    return x;
+// dynamic shared memory of a decode CTA: G rows of scores, then the slot
+// lanes' partial outputs
+size_t ska_decode_smem_g(int window, int dv, int G) {
+    return ((size_t)G * window + (size_t)(kDecThreads / (dv / 8)) * dv) * 4;
 }
 
-// One CTA per (b, h).  Valid slots are 0..n-1 with n = min(pos+1, w) (before
-// the ring is full, slot = position); the current token's slot takes the new
-// key and value from the inputs, and this CTA writes them into the caches (the
-// key by head 0 only; no other CTA reads that slot from the cache).
-template <int DK, int DV>
+// G block-wide reductions at once (max or sum of v[g] over the CTA's threads);
+// the results land in out[g] (shared memory) for every thread.  Two barriers:
+// `red` is free again when the next call writes it.
+template <int G>
+__device__ __forceinline__ void block_reduce_g(float* v, float (*red)[kDecThreads / 32], float* out,
+                                               bool is_max) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        float x = v[g];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float y = __shfl_xor_sync(0xffffffffu, x, o);
+            x = is_max ? fmaxf(x, y) : x + y;
+        }
+        if (lane == 0) red[g][warp] = x;
+    }
+    __syncthreads();
+    if (threadIdx.x < G) {
+        float x = red[threadIdx.x][0];
+#pragma unroll
+        for (int w = 1; w < kDecThreads / 32; ++w)
+            x = is_max ? fmaxf(x, red[threadIdx.x][w]) : x + red[threadIdx.x][w];
+        out[threadIdx.x] = x;
+    }
+    __syncthreads();
+}
+
+// One CTA per (b, group of G heads).  Valid slots are 0..n-1, n = min(pos+1, w)
+// (before the ring fills, slot = position); the current token's slot takes
+// the new key and value from the inputs, and this CTA writes them into the
+// caches (the key by the group of head 0 only; no CTA reads that slot from the
+// cache).  Each key row is read once for the G heads of the group.
+template <int DK, int DV, int G>
 __global__ void __launch_bounds__(kDecThreads) ska_decode_kernel(const SkaDecodeParams p) {
     extern __shared__ float dsm[];
-    float* sc = dsm;                       // [w] scores, then weights
-    float* part = dsm + p.window;          // [16][DV] partial outputs
-    __shared__ float qs[DK];
-    __shared__ float red[kDecThreads / 32];
-    const int bh = blockIdx.x, b = bh / p.H, h = bh % p.H;
+    constexpr int XP = DV / 8, LG = kDecThreads / XP;   // value pieces, slot lanes
+    float* sc = dsm;                       // [G][w] scores, then weights
+    float* part = dsm + G * p.window;      // [LG][DV] partial outputs
+    __shared__ float qs[G][DK];
+    __shared__ float red[G][kDecThreads / 32];
+    __shared__ float stat[2][G];           // row maximum, row sum
+    const int ng = p.H / G;
+    const int b = blockIdx.x / ng, h0 = (blockIdx.x % ng) * G;
     const int pos = p.pos[b];
     if (pos < 0) {  // the whole CTA leaves; nothing is read or written
         if (threadIdx.x == 0) atomicOr(p.err, kErrBadValue);
         return;
     }
     const int w = p.window, n = min(pos + 1, w), cur = pos % w;
+    const size_t bh0 = (size_t)b * p.H + h0;
     const __nv_bfloat16* kin = static_cast<const __nv_bfloat16*>(p.k) + (size_t)b * DK;
-    const __nv_bfloat16* vin = static_cast<const __nv_bfloat16*>(p.v) + (size_t)bh * DV;
+    const __nv_bfloat16* vin = static_cast<const __nv_bfloat16*>(p.v) + bh0 * DV;
     const __nv_bfloat16* kc = static_cast<const __nv_bfloat16*>(p.k_cache) + (size_t)b * w * DK;
-    const __nv_bfloat16* vc = static_cast<const __nv_bfloat16*>(p.v_cache) + (size_t)bh * w * DV;
+    const __nv_bfloat16* vc = static_cast<const __nv_bfloat16*>(p.v_cache) + bh0 * w * DV;
     const float c = p.scale * kLog2e;
-    // start the value rows (and, once per sequence, the shared key rows) toward
-    // L2 while the scores are formed, so the value sweep reads from L2
-    if (threadIdx.x == 0) {
-        bulk_prefetch_l2(vc, (uint32_t)n * DV * 2);
-        if (h == 0) bulk_prefetch_l2(kc, (uint32_t)n * DK * 2);
-    }
-    for (int i = threadIdx.x; i < DK; i += kDecThreads)
-        qs[i] = __bfloat162float(static_cast<const __nv_bfloat16*>(p.q)[(size_t)bh * DK + i]) * c;
-    // write the new token into its slot
-    if (h == 0)
+    // start the shared key rows toward L2 once per sequence (the group of head
+    // 0); prefetching the value rows as well measured slower (they evict one
+    // another: the groups' value rows far exceed L2)
+    if (threadIdx.x == 0 && h0 == 0) bulk_prefetch_l2(kc, (uint32_t)n * DK * 2);
+    for (int i = threadIdx.x; i < G * DK; i += kDecThreads)
+        qs[i / DK][i % DK] =
+            __bfloat162float(static_cast<const __nv_bfloat16*>(p.q)[bh0 * DK + i]) * c;
+    if (h0 == 0)
         for (int i = threadIdx.x; i < DK / 8; i += kDecThreads)
-            reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.k_cache) +
-                                     ((size_t)b * w + cur) * DK)[i] = reinterpret_cast<const uint4*>(kin)[i];
-    for (int i = threadIdx.x; i < DV / 8; i += kDecThreads)
-        reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.v_cache) +
-                                 ((size_t)bh * w + cur) * DV)[i] = reinterpret_cast<const uint4*>(vin)[i];
+            reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.k_cache) + ((size_t)b * w + cur) * DK)[i] =
+                reinterpret_cast<const uint4*>(kin)[i];
+    for (int i = threadIdx.x; i < G * (DV / 8); i += kDecThreads) {
+        const int g = i / (DV / 8), x = i % (DV / 8);
+        reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.v_cache) + ((bh0 + g) * w + cur) * DV)[x] =
+            reinterpret_cast<const uint4*>(vin + (size_t)g * DV)[x];
+    }
     __syncthreads();
-    // scores (log2 units): one slot per thread, the key row read in 16-byte pieces
-    float mx = -INFINITY;
+    // scores (log2 units): one slot per thread, its key row read once for G heads
+    float mx[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) mx[g] = -INFINITY;
     for (int u = threadIdx.x; u < n; u += kDecThreads) {
         const uint4* kr = reinterpret_cast<const uint4*>(u == cur ? kin : kc + (size_t)u * DK);
-        float a = 0.0f;
+        float a[G];
 #pragma unroll
+        for (int g = 0; g < G; ++g) a[g] = 0.0f;
+#pragma unroll 4
         for (int x = 0; x < DK / 8; ++x) {
             float f[8];
             unpack8(__ldg(kr + x), f);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) a = fmaf(qs[8 * x + e], f[e], a);
+            for (int g = 0; g < G; ++g)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) a[g] = fmaf(qs[g][8 * x + e], f[e], a[g]);
         }
-        sc[u] = a;
-        mx = fmaxf(mx, a);
-    }
-    mx = block_reduce(mx, red, true);
-    float sum = 0.0f;
-    for (int u = threadIdx.x; u < n; u += kDecThreads) {
-        const float e = ex2_fast(sc[u] - mx);
-        sc[u] = e;
-        sum += e;
-    }
-    sum = block_reduce(sum, red, false);  // its first barrier also publishes sc
-    // weighted sum of value rows: thread = (slot lane g, 8-column piece x)
-    constexpr int XP = DV / 8, G = kDecThreads / XP;
-    const int x = threadIdx.x % XP, g = threadIdx.x / XP;
-    float acc[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
-    const uint4* vbase = reinterpret_cast<const uint4*>(vc);
+        for (int g = 0; g < G; ++g) {
+            sc[g * w + u] = a[g];
+            mx[g] = fmaxf(mx[g], a[g]);
+        }
+    }
+    block_reduce_g<G>(mx, red, stat[0], true);
+    float sum[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) sum[g] = 0.0f;
+    for (int u = threadIdx.x; u < n; u += kDecThreads)
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            const float e = ex2_fast(sc[g * w + u] - stat[0][g]);
+            sc[g * w + u] = e;
+            sum[g] += e;
+        }
+    block_reduce_g<G>(sum, red, stat[1], false);  // its barriers also publish sc
+    // weighted sum of value rows, head by head: thread = (slot lane lg, 8-column piece x)
+    const int x = threadIdx.x % XP, lg = threadIdx.x / XP;
+    for (int g = 0; g < G; ++g) {
+        const uint4* vbase = reinterpret_cast<const uint4*>(vc + (size_t)g * w * DV);
+        const uint4* vnew = reinterpret_cast<const uint4*>(vin + (size_t)g * DV);
+        float acc[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
 #pragma unroll 4
-    for (int u = g; u < n; u += G) {
-        const uint4 wv = u == cur ? reinterpret_cast<const uint4*>(vin)[x] : __ldg(vbase + (size_t)u * XP + x);
-        float f[8];
-        unpack8(wv, f);
-        const float pu = sc[u];
+        for (int u = lg; u < n; u += LG) {
+            const uint4 wv = u == cur ? vnew[x] : __ldg(vbase + (size_t)u * XP + x);
+            float f[8];
+            unpack8(wv, f);
+            const float pu = sc[g * w + u];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = fmaf(pu, f[e], acc[e]);
-    }
+            for (int e = 0; e < 8; ++e) acc[e] = fmaf(pu, f[e], acc[e]);
+        }
 #pragma unroll
-    for (int e = 0; e < 8; ++e) part[g * DV + 8 * x + e] = acc[e];
-    __syncthreads();
-    const float inv = 1.0f / sum;
-    for (int j = threadIdx.x; j < DV; j += kDecThreads) {
-        float a = 0.0f;
-        for (int gg = 0; gg < G; ++gg) a += part[gg * DV + j];
-        static_cast<__nv_bfloat16*>(p.o)[(size_t)bh * DV + j] = __float2bfloat16_rn(a * inv);
+        for (int e = 0; e < 8; ++e) part[lg * DV + 8 * x + e] = acc[e];
+        __syncthreads();
+        const float inv = 1.0f / stat[1][g];
+        for (int j = threadIdx.x; j < DV; j += kDecThreads) {
+            float a = 0.0f;
+            for (int l2 = 0; l2 < LG; ++l2) a += part[l2 * DV + j];
+            static_cast<__nv_bfloat16*>(p.o)[(bh0 + g) * DV + j] = __float2bfloat16_rn(a * inv);
+        }
+        __syncthreads();  // part is rewritten by the next head
     }
 }
 
@@ -558,22 +599,31 @@ cudaError_t launch_fwd_cfg(const SkaParams& p, cudaStream_t s) {
     return cudaGetLastError();
 }
 
-template <int DK, int DV>
-cudaError_t launch_dec_cfg(const SkaDecodeParams& p, cudaStream_t s) {
-    constexpr int G = kDecThreads / (DV / 8);
-    const size_t smem = ((size_t)p.window + (size_t)G * DV) * 4;
-    auto kern = ska_decode_kernel<DK, DV>;
+template <int DK, int DV, int G>
+cudaError_t launch_dec_g(const SkaDecodeParams& p, cudaStream_t s) {
+    const size_t smem = ska_decode_smem_g(p.window, DV, G);
+    auto kern = ska_decode_kernel<DK, DV, G>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    kern<<<(unsigned)(p.B * p.H), kDecThreads, smem, s>>>(p);
+    kern<<<(unsigned)(p.B * (p.H / G)), kDecThreads, smem, s>>>(p);
     return cudaGetLastError();
+}
+
+// Heads per CTA: 8 where they divide H and their scores fit shared memory
+// (each key row is then read once for eight heads; measured on B256 H16
+// d 128 window 512: 216 us per step with one head per CTA, 167 with four, 122
+// with eight, 150 with all sixteen, where 256 CTAs leave SMs idle), else 4, 2, 1.
+template <int DK, int DV>
+cudaError_t launch_dec_cfg(const SkaDecodeParams& p, cudaStream_t s) {
+    constexpr size_t kFit = 200u << 10;
+    if (p.H % 8 == 0 && ska_decode_smem_g(p.window, DV, 8) <= kFit) return launch_dec_g<DK, DV, 8>(p, s);
+    if (p.H % 4 == 0 && ska_decode_smem_g(p.window, DV, 4) <= kFit) return launch_dec_g<DK, DV, 4>(p, s);
+    if (p.H % 2 == 0 && ska_decode_smem_g(p.window, DV, 2) <= kFit) return launch_dec_g<DK, DV, 2>(p, s);
+    return launch_dec_g<DK, DV, 1>(p, s);
 }
 
 }  // namespace
 
-size_t ska_decode_smem(int window, int dv) {
-    return ((size_t)window + (size_t)(kDecThreads / (dv / 8)) * dv) * 4;
-}
 
 cudaError_t launch_ska_fwd(const SkaParams& p, cudaStream_t s) {
     cudaError_t e = cudaSuccess;

@@ -36,6 +36,5 @@ struct SkaDecodeParams {
 };
 cudaError_t launch_ska_fwd(const SkaParams& p, cudaStream_t s);
 cudaError_t launch_ska_decode(const SkaDecodeParams& p, cudaStream_t s);
-size_t ska_decode_smem(int window, int dv);  // dynamic shared memory of one decode CTA
 
 }  // namespace rdm

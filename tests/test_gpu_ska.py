@@ -167,3 +167,25 @@ def test_ska_decode_full_size_sampled(cuda_ok):
         o_ref, _, _ = oracle.ska_decode(q[b:b + 1], k[b:b + 1], v[b:b + 1], kc[b:b + 1],
                                         vc[b:b + 1], pos[b:b + 1].numpy(), w)
         assert_close(od[b:b + 1], o_ref, TOL, f"decode full size b={b}")
+
+
+@pytest.mark.parametrize("H", [1, 2, 4, 6, 8, 16])
+def test_ska_decode_head_groups(cuda_ok, H):
+    """Head counts that select every grouping of heads per CTA (8, 4, 2, 1
+    heads sharing one pass over the key rows), with wrapped rings at different
+    positions per sequence."""
+    B, d, w = 3, 64, 24
+    g = torch.Generator().manual_seed(H)
+    kc = torch.randn(B, w, d, generator=g).to(torch.bfloat16)
+    vc = torch.randn(B, H, w, d, generator=g).to(torch.bfloat16)
+    q = torch.randn(B, H, d, generator=g).to(torch.bfloat16)
+    k = torch.randn(B, d, generator=g).to(torch.bfloat16)
+    v = torch.randn(B, H, d, generator=g).to(torch.bfloat16)
+    pos = torch.tensor([5, 23, 70], dtype=torch.int32)
+    kcd, vcd = kc.cuda(), vc.cuda()
+    od = rdm.rdm_ska_decode(q.cuda(), k.cuda(), v.cuda(), kcd, vcd, pos.cuda()).cpu()
+    assert rdm.rdm_ddts_sync_status() == 0
+    o_ref, kc_ref, vc_ref = oracle.ska_decode(q, k, v, kc, vc, pos.numpy(), w)
+    assert_close(od, o_ref, TOL, f"decode H={H}")
+    assert_close(kcd, kc_ref, 0.0, f"k cache H={H}")
+    assert_close(vcd, vc_ref, 0.0, f"v cache H={H}")
