@@ -189,3 +189,17 @@ def test_ska_decode_head_groups(cuda_ok, H):
     assert_close(od, o_ref, TOL, f"decode H={H}")
     assert_close(kcd, kc_ref, 0.0, f"k cache H={H}")
     assert_close(vcd, vc_ref, 0.0, f"v cache H={H}")
+
+
+@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 128), (128, 64)])
+def test_ska_fwd_persistent_ctas_walk_several_tiles(cuda_ok, dk, dv):
+    """Head sizes with one CTA per SM run persistent CTAs: with more query
+    tiles than SMs (2 x 8 x 12 = 192 tiles of 128 queries), CTAs walk several
+    tiles of different heads; sampled heads against the oracle."""
+    B, H, T, w = 2, 8, 1500, 300
+    q, k, v = ska_inputs(B, H, T, dk, dv, seed=dk + 2 * dv)
+    o = rdm.rdm_ska_fwd(q.cuda(), k.cuda(), v.cuda(), w).cpu()
+    assert rdm.rdm_ddts_sync_status() == 0
+    for b, h in ((0, 0), (1, 5), (1, 7)):
+        ref = oracle.ska_fwd(q[b:b + 1, h:h + 1], k[b:b + 1], v[b:b + 1, h:h + 1], w)
+        assert_close(o[b:b + 1, h:h + 1], ref, TOL, f"persistent dk={dk} dv={dv} b={b} h={h}")
