@@ -320,6 +320,7 @@ static ConvParams conv_params(const rdm_shortconv_args* a) {
     p.y = a->y; p.xs_out = a->W > 1 ? a->state_out : nullptr;
     p.err = status_word();
     p.wait_limit = wait_limit();
+    p.withhold = g_hook_withhold.load(std::memory_order_relaxed);
     return p;
 }
 
@@ -386,6 +387,7 @@ rdm_status rdm_ska_fwd(const rdm_ska_fwd_args* a, rdm_stream_t stream) {
     p.pos = a->pos;
     p.err = err;
     p.wait_limit = wait_limit();
+    p.withhold = g_hook_withhold.load(std::memory_order_relaxed);
     return from_cuda(launch_ska_fwd(p, static_cast<cudaStream_t>(stream)));
 }
 

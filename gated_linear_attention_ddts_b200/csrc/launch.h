@@ -91,6 +91,7 @@ struct ConvParams {
     int tile;            // tokens per block (set by the launcher)
     unsigned* err;       // device status word (a staging wait that ran out)
     long long wait_limit;
+    int withhold;        // test hook: the staging copies are never issued
 };
 cudaError_t launch_conv_fwd(const ConvParams& p, cudaStream_t s);
 cudaError_t launch_conv_bwd(const ConvParams& p, cudaStream_t s);

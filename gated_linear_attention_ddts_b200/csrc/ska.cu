@@ -201,7 +201,7 @@ __global__ void __launch_bounds__(kSkaThreads, SkaCfg<DK, DV>::CTAS_PER_SM)
         if (lane == 0 && nq > 0) {
             int qq = 0;               // query tiles whose Q has been issued
             int qk = 0, jk = 0;       // key stream: query tile, key tile within it
-            int qv = 0, jv = 0;       // value stream
+            int qv = p.withhold ? nq : 0, jv = 0;  // value stream (none under the test hook)
             int nk = 0, nv = 0;       // key / value tiles issued in all
             SkaTile tk = ska_tile<NK>(p, blockIdx.x), tv = tk;
             long long idle0 = clock64();

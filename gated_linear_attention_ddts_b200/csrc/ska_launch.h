@@ -22,6 +22,7 @@ struct SkaParams {
     int* pos;              // [B] set to T after the forward, or null
     unsigned* err;
     long long wait_limit;
+    int withhold;          // test hook: the producer never loads value tiles
 };
 struct SkaDecodeParams {
     int B, H, dk, dv, window;

@@ -419,9 +419,11 @@ const char *rdm_status_string(rdm_status status);
  *                            up (0 = the default, about one second).
  *   withhold_segment_flags : 1 = CTAs of a sequence-segmented tensor-core
  *                            launch never publish the flag that tells later
- *                            segments their input is ready, so those segments'
- *                            waits run out: the kernel then stops, sets the
- *                            device status word and returns, and
+ *                            segments their input is ready, the SW-SKA forward
+ *                            never loads its value tiles and the ShortConv
+ *                            kernels never issue their staging copies, so the
+ *                            waits on them run out: the kernel then stops, sets
+ *                            the device status word and returns, and
  *                            rdm_ddts_sync_status reports RDM_ERR_TIMEOUT.
  *                            Outputs of such a call are unspecified.
  * Returns RDM_ERR_INVALID_ARG for a negative limit or a flag other than 0/1. */
