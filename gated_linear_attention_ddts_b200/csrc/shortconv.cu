@@ -7,18 +7,18 @@
 //
 // with x at t-i < 0 read from the carried-in state (the previous W-1 inputs).
 //
-// HBM-bound streaming through shared memory: persistent blocks (two per SM)
-// take tiles of 8192 elements of one (b, h) (128 tokens at D = 64) in turn.
-// The rows of a tile are contiguous in HBM; thread 0 keeps a ring of tiles in
-// flight, each tile and its W-1 row halo arriving by one bulk copy (the
-// backward: x and dy, halos on both sides), so the copy engine streams while
-// the threads work out of shared memory on the tile before.  Forward threads
-// take a run of consecutive tokens of 16 bytes of channels, unpack each staged
-// row once and slide it through a window of the last W rows.  The backward
-// first writes dL/dz of the tile to shared memory (z recomputed from the
-// staged x when the SiLU is on), then forms dx and the weight and bias
-// gradients, reduced over the block (shuffles, then shared memory) before one
-// float32 atomic per value and tile.
+// HBM-bound streaming through shared memory: persistent blocks take tiles of
+// one (b, h) in turn (forward: 4096 elements, four blocks per SM; backward:
+// 8192, two per SM).  The rows of a tile are contiguous in HBM; thread 0 keeps
+// a ring of tiles in flight, each tile and its W-1 row halo arriving by one
+// bulk copy (the backward: x and dy, halos on both sides), so the copy engine
+// streams while the threads work out of shared memory on the tile before.
+// Every thread takes a run of consecutive tokens of 4 channels and slides the
+// staged rows through windows: the forward through a window of the last W
+// inputs; the backward through one of inputs and one of dL/dz (z recomputed
+// from the inputs when the SiLU is on), forming dx and the weight and bias
+// gradients in a single sweep; those are reduced over the block (shuffles,
+// then shared memory) before one float32 atomic per value and head.
 #include <algorithm>
 
 #include "launch.h"
@@ -106,10 +106,21 @@ __device__ __forceinline__ void lds_vec(const __nv_bfloat16* p, float* f) {
     f[2] = __uint_as_float(u.y << 16); f[3] = __uint_as_float(u.y & 0xffff0000u);
 }
 
+// SiLU of the forward in three operations for bf16: with h = z/2,
+// z sigmoid(z) = h (1 + tanh(h)) = fma(h, tanh(h), h).
+template <typename T>
+__device__ __forceinline__ float silu_fwd(float z) { return silu_t<T>(z); }
+template <>
+__device__ __forceinline__ float silu_fwd<__nv_bfloat16>(float z) {
+    const float h = 0.5f * z;
+    return fmaf(h, tanh_fast(h), h);
+}
+
 template <typename T>
 __device__ __forceinline__ T zero_val() { return T(0.0f); }
 
-constexpr int kConvStages = 3;     // tiles in flight per forward block
+constexpr int kConvStages = 4;     // tiles in flight per forward block
+constexpr int kConvFwdRun = 4;     // consecutive tokens per forward thread
 constexpr int kConvBwdStages = 2;  // per backward block (two blocks per SM fit)
 
 // A tile: tokens [t0, t1) of sequence bh.
@@ -182,14 +193,16 @@ __device__ void drain_stages(uint64_t* full, int k, int g, int g1, const ConvPar
 }
 
 // Forward: persistent blocks (four per SM) take contiguous runs of tiles of
-// `p.tile` tokens of one (b, h).  Thread 0 keeps kConvStages tiles in flight: each tile's
-// rows and the W-1 rows before it arrive by one bulk copy into a ring stage;
-// then thread (channel group cg, run of RUN consecutive tokens) unpacks each
-// staged row once, slides it through a window of the last W rows and stores
-// 16 bytes of channels per token.
-template <typename T, int W>
+// `p.tile` tokens of one (b, h).  Thread 0 keeps kConvStages tiles in flight:
+// each tile's rows and the W-1 rows before it arrive by one bulk copy into a
+// ring stage; then thread (channel group cg, run of kConvFwdRun consecutive
+// tokens) unpacks each staged row once, slides it through a window of the last
+// W rows and stores 16 bytes of channels per token (8 for bf16).  Small tiles
+// (4096 elements) give every block several, so that the first tiles' work
+// overlaps the later tiles' copies.
+template <typename T, int W, bool SILU>
 __global__ void __launch_bounds__(kThreads, 4) conv_fwd_kernel(const ConvParams p) {
-    constexpr int N = Vec<T>::N, RUN = 32 / N;
+    constexpr int N = Vec<T>::N, RUN = kConvFwdRun;
     extern __shared__ __align__(128) uint8_t conv_smem[];
     __shared__ uint64_t full[kConvStages];
     const int CG = p.D / N;
@@ -237,24 +250,26 @@ __global__ void __launch_bounds__(kThreads, 4) conv_fwd_kernel(const ConvParams 
         if (W > 1 && lo < 0) fill_state_rows<T, W>(p, c.bh, lo, xs);
         const int ta = c.t0 + run * RUN;
         if (ta < c.t1) {
-            T* y = static_cast<T*>(p.y) + (size_t)c.bh * p.T * p.D + c0;
+            // staged row of token t at t - lo; my first window row is token ta - (W-1)
+            const T* xr = xs + (size_t)(ta - (W - 1) - lo) * p.D + c0;
+            T* yr = static_cast<T*>(p.y) + ((size_t)c.bh * p.T + ta) * p.D + c0;
+            const int nrun = min(RUN, c.t1 - ta);
             float win[W][N];  // win[j] = x[t - (W-1) + j]
 #pragma unroll
-            for (int j = 0; j < W - 1; ++j) lds_vec(xs + (size_t)(ta - (W - 1) + j - lo) * p.D + c0, win[j]);
+            for (int j = 0; j < W - 1; ++j) lds_vec(xr + (size_t)j * p.D, win[j]);
 #pragma unroll
             for (int r = 0; r < RUN; ++r) {
-                const int t = ta + r;
-                if (t >= c.t1) break;
-                lds_vec(xs + (size_t)(t - lo) * p.D + c0, win[W - 1]);
+                if (r >= nrun) break;
+                lds_vec(xr + (size_t)(r + W - 1) * p.D, win[W - 1]);
                 float z[N];
 #pragma unroll
                 for (int e = 0; e < N; ++e) {
                     float a = bv[e];
 #pragma unroll
                     for (int i = 0; i < W; ++i) a = fmaf(wv[i][e], win[W - 1 - i][e], a);
-                    z[e] = p.silu ? silu_t<T>(a) : a;
+                    z[e] = SILU ? silu_fwd<T>(a) : a;
                 }
-                store_vec(y + (size_t)t * p.D, z);
+                store_vec(yr + (size_t)r * p.D, z);
 #pragma unroll
                 for (int j = 0; j < W - 1; ++j)
 #pragma unroll
@@ -307,18 +322,23 @@ __device__ __forceinline__ void dz_row(const ConvParams& p, int bh, int t, int c
     }
 }
 
-// Backward: persistent blocks (three per SM) with contiguous runs of tiles of
-// 4096 elements, as in the forward.  A ring stage holds x of
-// tokens [t0 - (W-1), t1 + W - 1) and dy of [t0, t1 + W - 1) (two bulk copies
-// on one barrier).  Phase 1 writes dL/dz of tokens [t0, t1 + W - 1) (zero past
-// the end; z recomputed from the staged x for the SiLU) to shared memory as
-// float32; phase 2 gives dx[t] = sum_i w_i dz[t+i] (plus the carried-out
-// state's gradient where it copies x[t]) and the weight and bias partial sums,
-// reduced over the block (shuffles, then shared memory) and added with one
-// float32 atomic per value for each run of tiles of one head.
-template <typename T, int W>
-__global__ void __launch_bounds__(kThreads, 3) conv_bwd_kernel(const ConvParams p) {
-    constexpr int N = Vec<T>::N;
+// Backward: persistent blocks (two per SM) with contiguous runs of tiles of
+// 8192 elements, as in the forward.  A ring stage holds x of tokens
+// [t0 - (W-1), t1 + W - 1) and dy of [t0, t1 + W - 1) (two bulk copies on one
+// barrier).  Thread (channel group cg, run of kConvBwdRun consecutive tokens
+// [ta, tb)) sweeps u over [ta, tb + W - 1) once: x[u] enters a window of the
+// last W inputs, dL/dz[u] (dy through the SiLU, z recomputed from the window;
+// zero past the end) enters a window of the last W of those, and
+//   dx[u - (W-1)] = sum_i w_i dz[u - (W-1) + i]        (once the window is full)
+//   dw_i += x[u - i] dz[u],  dbias += dz[u]             (u inside the run)
+// so every staged row is read once per thread, plus the W-1 rows of halo on
+// each side of its run.  The weight and bias partial sums are reduced over
+// the block (shuffles, then shared memory) and added with one float32 atomic
+// per value for each run of tiles of one head.
+constexpr int kConvBwdRun = 8;
+template <typename T, int W, bool SILU>
+__global__ void __launch_bounds__(kThreads, 2) conv_bwd_kernel(const ConvParams p) {
+    constexpr int N = Vec<T>::N, RUN = kConvBwdRun;
     extern __shared__ __align__(128) uint8_t conv_smem[];
     __shared__ uint64_t full[kConvBwdStages];
     const int TT = p.tile;
@@ -328,9 +348,8 @@ __global__ void __launch_bounds__(kThreads, 3) conv_bwd_kernel(const ConvParams 
     const size_t xrows = TT + 2 * (W - 1), yrows = TT + W - 1;
     const size_t stage = (xrows + yrows) * p.D;  // elements per ring stage
     T* ring = reinterpret_cast<T*>(conv_smem);
-    float* dzs = reinterpret_cast<float*>(ring + kConvBwdStages * stage);
-    float* s_red = dzs + yrows * p.D;  // [warps][D (W + 1)]
-    const int CG = p.D / N, R = kThreads / CG;
+    float* s_red = reinterpret_cast<float*>(ring + kConvBwdStages * stage);  // [warps][D (W + 1)]
+    const int CG = p.D / N;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     auto issue = [&](int g, int s) {
         const ConvTile c = conv_tile_of(p, g);
@@ -385,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, 3) conv_bwd_kernel(const ConvParams 
     for (int g = g0; g < g1; ++g, ++k) {
         const int s = k % kConvBwdStages;
         const ConvTile c = conv_tile_of(p, g);
-        const int lo = c.t0 - (W - 1), nz = c.t1 + W - 1 - c.t0;
+        const int lo = c.t0 - (W - 1);
         if (c.h != cur_h) {  // block-uniform
             if (cur_h >= 0) flush(cur_h);
             cur_h = c.h;
@@ -407,68 +426,79 @@ __global__ void __launch_bounds__(kThreads, 3) conv_bwd_kernel(const ConvParams 
         T* xs = ring + s * stage;
         const T* dys = xs + xrows * p.D;
         if (W > 1 && lo < 0) fill_state_rows<T, W>(p, c.bh, lo, xs);
-        // phase 1
-        for (int u = r0; u < nz; u += R) {
-            const int t = c.t0 + u;
-            float dz[N];
-            if (t < p.T) {
-                lds_vec(dys + (size_t)u * p.D + c0, dz);
-                if (p.silu) {
-                    float z[N];
+        const int ta = c.t0 + r0 * RUN, tb = min(ta + RUN, c.t1);
+        if (ta < c.t1) {
+            // staged rows: x of token u at row u - lo, dy of token u at row u - t0;
+            // rows at or past T are not staged and never enter a result
+            T* dx = static_cast<T*>(p.dx) + (size_t)c.bh * p.T * p.D + c0;
+            float xw[W][N];   // xw[j] = x[u - (W-1) + j] once x[u] is in
+            float dzw[W][N];  // dzw[j] = dz[u - (W-1) + j] once dz[u] is in
 #pragma unroll
-                    for (int e = 0; e < N; ++e) z[e] = bv[e];
+            for (int j = 0; j < W - 1; ++j) lds_vec(xs + (size_t)(ta - (W - 1) + j - lo) * p.D + c0, xw[j]);
 #pragma unroll
-                    for (int i = 0; i < W; ++i) {
-                        float xv[N];
-                        lds_vec(xs + (size_t)(t - i - lo) * p.D + c0, xv);
+            for (int j = 0; j < W; ++j)
 #pragma unroll
-                        for (int e = 0; e < N; ++e) z[e] = fmaf(wv[i][e], xv[e], z[e]);
+                for (int e = 0; e < N; ++e) dzw[j][e] = 0.0f;
+#pragma unroll
+            for (int k2 = 0; k2 < RUN + W - 1; ++k2) {
+                const int u = ta + k2;
+                if (u >= tb + W - 1) break;
+                lds_vec(xs + (size_t)(u - lo) * p.D + c0, xw[W - 1]);
+                float dz[N];
+                if (u < p.T) {
+                    lds_vec(dys + (size_t)(u - c.t0) * p.D + c0, dz);
+                    if constexpr (SILU) {
+#pragma unroll
+                        for (int e = 0; e < N; ++e) {
+                            float z = bv[e];
+#pragma unroll
+                            for (int i = 0; i < W; ++i) z = fmaf(wv[i][e], xw[W - 1 - i][e], z);
+                            dz[e] *= silu_grad_t<T>(z);
+                        }
                     }
+                } else {
 #pragma unroll
-                    for (int e = 0; e < N; ++e) dz[e] *= silu_grad_t<T>(z[e]);
+                    for (int e = 0; e < N; ++e) dz[e] = 0.0f;
                 }
-            } else {
+                if (u < tb) {
 #pragma unroll
-                for (int e = 0; e < N; ++e) dz[e] = 0.0f;
+                    for (int e = 0; e < N; ++e) {
+#pragma unroll
+                        for (int i = 0; i < W; ++i) aw[i][e] = fmaf(xw[W - 1 - i][e], dz[e], aw[i][e]);
+                        ab[e] += dz[e];
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < W - 1; ++j)
+#pragma unroll
+                    for (int e = 0; e < N; ++e) dzw[j][e] = dzw[j + 1][e];
+#pragma unroll
+                for (int e = 0; e < N; ++e) dzw[W - 1][e] = dz[e];
+                if (k2 >= W - 1) {
+                    const int t = u - (W - 1);  // in [ta, tb)
+                    float gx[N];
+#pragma unroll
+                    for (int e = 0; e < N; ++e) {
+                        float a = 0.0f;
+#pragma unroll
+                        for (int i = 0; i < W; ++i) a = fmaf(wv[i][e], dzw[i][e], a);
+                        gx[e] = a;
+                    }
+                    if (p.dxs_out != nullptr && t >= tout0) {
+                        float go[N];
+                        load_vec(static_cast<const T*>(p.dxs_out) + ((size_t)c.bh * (W - 1) + (t - tout0)) * p.D + c0, go);
+#pragma unroll
+                        for (int e = 0; e < N; ++e) gx[e] += go[e];
+                    }
+                    store_vec(dx + (size_t)t * p.D, gx);
+                }
+#pragma unroll
+                for (int j = 0; j < W - 1; ++j)
+#pragma unroll
+                    for (int e = 0; e < N; ++e) xw[j][e] = xw[j + 1][e];
             }
-            *reinterpret_cast<float4*>(dzs + (size_t)u * p.D + c0) = make_float4(dz[0], dz[1], dz[2], dz[3]);
         }
-        __syncthreads();
-        // phase 2
-        T* dx = static_cast<T*>(p.dx) + (size_t)c.bh * p.T * p.D + c0;
-        for (int t = c.t0 + r0; t < c.t1; t += R) {
-            const int u = t - c.t0;
-            float dzr[W][N];
-#pragma unroll
-            for (int i = 0; i < W; ++i) {
-                const float4 f = *reinterpret_cast<const float4*>(dzs + (size_t)(u + i) * p.D + c0);
-                dzr[i][0] = f.x; dzr[i][1] = f.y; dzr[i][2] = f.z; dzr[i][3] = f.w;
-            }
-            float gx[N];
-#pragma unroll
-            for (int e = 0; e < N; ++e) {
-                float a = 0.0f;
-#pragma unroll
-                for (int i = 0; i < W; ++i) a = fmaf(wv[i][e], dzr[i][e], a);
-                gx[e] = a;
-                ab[e] += dzr[0][e];
-            }
-#pragma unroll
-            for (int i = 0; i < W; ++i) {
-                float xv[N];
-                lds_vec(xs + (size_t)(t - i - lo) * p.D + c0, xv);
-#pragma unroll
-                for (int e = 0; e < N; ++e) aw[i][e] = fmaf(dzr[0][e], xv[e], aw[i][e]);
-            }
-            if (p.dxs_out != nullptr && t >= tout0) {
-                float go[N];
-                load_vec(static_cast<const T*>(p.dxs_out) + ((size_t)c.bh * (W - 1) + (t - tout0)) * p.D + c0, go);
-#pragma unroll
-                for (int e = 0; e < N; ++e) gx[e] += go[e];
-            }
-            store_vec(dx + (size_t)t * p.D, gx);
-        }
-        __syncthreads();  // stage s and dz fully read: refill the stage
+        __syncthreads();  // stage s fully read: refill it
         if (threadIdx.x == 0 && g + kConvBwdStages < g1) issue(g + kConvBwdStages, s);
     }
     if (cur_h >= 0) flush(cur_h);
@@ -513,9 +543,10 @@ __global__ void conv_state_grad_kernel(ConvParams p) {
     }
 }
 
-// Tokens per tile: 8192 elements (128 tokens at D = 64) forward, 4096 backward.
-int conv_tile(const ConvParams& p) { return std::max(8192 / p.D, 8); }
-int conv_tile_bwd(const ConvParams& p) { return std::max(4096 / p.D, 8); }
+// Tokens per tile: a run of kConvFwdRun (forward: 4096 elements, 64 tokens at
+// D = 64) or kConvBwdRun (backward: 8192 elements) tokens for every thread.
+int conv_tile(const ConvParams& p) { return kConvFwdRun * kThreads / (p.D / Vec<float>::N); }
+int conv_tile_bwd(const ConvParams& p) { return kConvBwdRun * kThreads / (p.D / Vec<float>::N); }
 
 template <typename T, int W>
 size_t fwd_smem(const ConvParams& p) {
@@ -525,8 +556,7 @@ size_t fwd_smem(const ConvParams& p) {
 template <typename T, int W>
 size_t bwd_smem(const ConvParams& p) {
     const size_t stage = (size_t)(2 * p.tile + 3 * (W - 1)) * p.D * sizeof(T);
-    return kConvBwdStages * stage + (size_t)(p.tile + W - 1) * p.D * 4 +
-           (size_t)(kThreads / 32) * p.D * (W + 1) * 4;
+    return kConvBwdStages * stage + (size_t)(kThreads / 32) * p.D * (W + 1) * 4;
 }
 
 // Persistent grid: `per_sm` blocks per SM, or fewer when there are fewer tiles.
@@ -542,7 +572,7 @@ cudaError_t fwd_tw(const ConvParams& p0, cudaStream_t s) {
     p.tile = conv_tile(p);
     if (p.T > 0) {
         const size_t smem = fwd_smem<T, W>(p);
-        auto kern = conv_fwd_kernel<T, W>;
+        auto kern = p.silu ? conv_fwd_kernel<T, W, true> : conv_fwd_kernel<T, W, false>;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         kern<<<conv_grid(p, 4), kThreads, smem, s>>>(p);
@@ -563,10 +593,10 @@ cudaError_t bwd_tw(const ConvParams& p0, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     if (p.T > 0) {
         const size_t smem = bwd_smem<T, W>(p);
-        auto kern = conv_bwd_kernel<T, W>;
+        auto kern = p.silu ? conv_bwd_kernel<T, W, true> : conv_bwd_kernel<T, W, false>;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        kern<<<conv_grid(p, 3), kThreads, smem, s>>>(p);
+        kern<<<conv_grid(p, 2), kThreads, smem, s>>>(p);
     }
     if constexpr (W > 1) {
         if (p.dxs) {
