@@ -207,9 +207,10 @@ __global__ void __launch_bounds__(kThreads, 4) conv_fwd_kernel(const ConvParams 
     __shared__ uint64_t full[kConvStages];
     const int CG = p.D / N;
     const int total = p.B * p.H * ((p.T + p.tile - 1) / p.tile);
-    // a contiguous run of tiles per block (same sequence, mostly the same head)
-    const int per = (total + (int)gridDim.x - 1) / (int)gridDim.x;
-    const int g0 = blockIdx.x * per, g1 = min(total, g0 + per);
+    // a contiguous run of tiles per block (same sequence, mostly the same head);
+    // the runs of the blocks differ by at most one tile
+    const int g0 = (int)((long long)blockIdx.x * total / gridDim.x);
+    const int g1 = (int)((long long)(blockIdx.x + 1) * total / gridDim.x);
     const size_t stage = (size_t)(p.tile + W - 1) * p.D;  // elements per ring stage
     T* ring = reinterpret_cast<T*>(conv_smem);
     auto issue = [&](int g, int s) {
@@ -343,8 +344,9 @@ __global__ void __launch_bounds__(kThreads, 2) conv_bwd_kernel(const ConvParams 
     __shared__ uint64_t full[kConvBwdStages];
     const int TT = p.tile;
     const int total = p.B * p.H * ((p.T + TT - 1) / TT);
-    const int per = (total + (int)gridDim.x - 1) / (int)gridDim.x;
-    const int g0 = blockIdx.x * per, g1 = min(total, g0 + per);
+    // contiguous runs of tiles that differ by at most one tile between blocks
+    const int g0 = (int)((long long)blockIdx.x * total / gridDim.x);
+    const int g1 = (int)((long long)(blockIdx.x + 1) * total / gridDim.x);
     const size_t xrows = TT + 2 * (W - 1), yrows = TT + W - 1;
     const size_t stage = (xrows + yrows) * p.D;  // elements per ring stage
     T* ring = reinterpret_cast<T*>(conv_smem);
