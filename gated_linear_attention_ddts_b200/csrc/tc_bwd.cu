@@ -633,6 +633,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 *reinterpret_cast<uint4*>(gst + 2 * kBox + off_raw(t, cg)) = pack8(odg);
                 *reinterpret_cast<uint4*>(gst + 3 * kBox + off_raw(t, cg)) = pack8(odt);
             }
+            // this warp's last read of the raw tiles and of the dQ / dK staging (the
+            // epilogue read its raw rows before it handed over the staging): the
+            // producer may load the next chunk while the gradients are stored
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.raw_empty);
             // dq, dk, dg, dtau of the chunk: one TMA store each (rows past T are
             // clipped); the staging bytes are read before the next operand stage
             fence_proxy_async_smem();
@@ -652,10 +657,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 for (int e = 0; e < 8; ++e) sm.carry[cg * 8 + e] = dG[0][e];
             }
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&sm.post_done);
-                mbar_arrive(&sm.raw_empty);
-            }
+            if (lane == 0) mbar_arrive(&sm.post_done);
             ++i2;
         }
     } else {
