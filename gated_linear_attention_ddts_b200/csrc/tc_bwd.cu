@@ -79,19 +79,21 @@ struct BCfg {
 template <int DV>
 struct alignas(1024) BwdSmem {
     uint8_t raw[BCfg<DV>::RAW];
+    // Vh and dO operands (no-swizzle layouts); once the second MMA group has
+    // completed, the same bytes stage dv | dbeta for their TMA stores
+    // (128B-swizzled, hence their 1024-byte aligned place after the raw tiles)
+    uint8_t vh[C * DV * 2];    // [s][j], column groups 1024 B apart
+    uint8_t dot[C * DV * 2];   // [t][j]
     uint8_t qt[8 * kQK];       // [t][i]
     uint8_t kt[8 * kQK];       // [s][i]
     uint8_t qtl[8 * kQK];      // bf16 remainders Qt - bf16(Qt), Kt - bf16(Kt): the
     uint8_t ktl[8 * kQK];      // pair products of dQ and dK reach ~16 mantissa bits
-    uint8_t vh[C * DV * 2];    // [s][j], column groups 1024 B apart
-    uint8_t dot[C * DV * 2];   // [t][j]
     // A, B and R_hat operands of the second MMA group; once that group has
     // completed, the same bytes hold the fp32 dQ / dK staging tiles; before the
     // first stage of the epilogue writes A, they hold the chunk-start state
     // S_prev (fp32) that the gate warps turn into S_hat
     union alignas(1024) {
         float sprev[DK * kSpStride<DV>];
-        uint8_t ost[2 * C * DV * 2];  // dv | dbeta tiles for the TMA stores (128B-swizzled)
         struct {
             uint8_t abf[C * C * 2];       // [t][s]
             uint8_t bmb[C * C * 2];       // [t][s]
@@ -105,7 +107,7 @@ struct alignas(1024) BwdSmem {
     float em[DK], cf[DK], gm[DK], fin[DK], carry[DK];
     float bdiag[C];  // B_tt = vhat_t . dO_t (the diagonal kept out of the dQ / dK MMAs)
     uint64_t raw_full, raw_empty, sp_full, ops_full, shat_full, ops_empty, g1_done, g2_ready,
-        tm1_free, g2_done, tm2_free, post_ready, post_done, p1_done;
+        tm1_free, g2_done, tm2_free, post_ready, post_done, p1_done, vh_free;
     uint32_t tmem_base;
     int fail;
     int epi_fail;  // the epilogue's own exit decision (written before a role barrier)
@@ -129,6 +131,11 @@ struct BwdKernelArgs {
     int* flags;
     BwdSeg seg;
 };
+
+// Arrive `n` times at once on a CTA-local mbarrier.
+__device__ __forceinline__ void mbar_arrive_n(uint64_t* bar, uint32_t n) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(n) : "memory");
+}
 
 // [row][col] tile with 8-row groups 128 B apart and 8-column groups 1024 B
 // apart (64 rows): K-major for (rows = M/N, K = cols), MN-major for (MN = cols,
@@ -167,7 +174,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
 
     if (threadIdx.x == 0) {
         mbar_init(&sm.raw_full, 1);
-        mbar_init(&sm.raw_empty, kGateWarps);
+        mbar_init(&sm.raw_empty, kGateWarps + 4);  // the epilogue reads v, beta, dO too
         mbar_init(&sm.sp_full, 1);
         mbar_init(&sm.ops_full, kGateWarps);
         mbar_init(&sm.shat_full, kGateWarps);
@@ -180,6 +187,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
         mbar_init(&sm.post_ready, 4);
         mbar_init(&sm.post_done, kGateWarps);
         mbar_init(&sm.p1_done, kGateWarps);
+        mbar_init(&sm.vh_free, 1);
         sm.epi_fail = 0;
         sm.fail = 0;
         fence_mbar_init();
@@ -462,7 +470,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 __syncwarp();
                 if (lane == 0) {
                     mbar_arrive(&sm.ops_full);
-                    mbar_arrive(&sm.raw_empty);
+                    // the epilogue reads no raw tile in this pass: warp 0 arrives
+                    // for its four warps as well
+                    if (gw == 0) mbar_arrive_n(&sm.raw_empty, 5);
+                    else mbar_arrive(&sm.raw_empty);
                     if (p1last) mbar_arrive(&sm.p1_done);
                 }
                 continue;
@@ -505,6 +516,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                     sm.gm[cg * 8 + e] = ex2_fast(blL[e]);
                 }
             }
+            // Vh and dO operand buffers: the epilogue's dv / dbeta stores of the
+            // previous chunk have read them
+            if (i2 > 0 && !mbar_wait_own(&sm.vh_free, (i2 - 1) & 1, fail, WL)) break;
 #pragma unroll
             for (int iv = 0; iv < VIT; ++iv) {
                 const int jg = gt / TPG, t = (gt % TPG) + TPG * iv;
@@ -840,12 +854,27 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             }
             if (!mbar_wait_own(&sm.g2_done, i2 & 1, fail, WL)) break;
             tc_fence_after();
-            // dV -> dv = beta dvhat, dbeta = v dvhat (row s = r), staged in the union
-            // (its A / B / R_hat operands are consumed; the previous chunk's gate
-            // stage has read its dQ / dK staging) and written by TMA stores
+            // dQ, dK -> fp32 staging for the gate warps first (the union: the
+            // previous chunk's gate stage has read its staging), so that their final
+            // stage runs beside the dv / dbeta stage below
             if (i2 > 0 && !mbar_wait_own(&sm.post_done, (i2 - 1) & 1, fail, WL)) break;
-            {
 #pragma unroll
+            for (int which = 0; which < 2; ++which) {
+                float v[32];
+                tmem_ld32_split<32>(tmem + lb + (which == 0 ? K::COL_DQ : K::COL_DK), v);
+                tmem_ld_wait();
+                float4* dst = reinterpret_cast<float4*>(which == 0 ? &sm.u.st.dqs[r][32 * hf] : &sm.u.st.dks[r][32 * hf]);
+#pragma unroll
+                for (int e4 = 0; e4 < 8; ++e4)
+                    dst[e4] = make_float4(v[4 * e4], v[4 * e4 + 1], v[4 * e4 + 2], v[4 * e4 + 3]);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.post_ready);
+            // dV -> dv = beta dvhat, dbeta = v dvhat (row s = r), staged in the Vh |
+            // dO operand buffers (idle once the second group has completed) and
+            // written by TMA stores
+            {
+#pragma unroll 1
                 for (int qd = 0; qd < HV / 32; ++qd) {
                     float v[32];
                     tmem_ld32_split<HV>(tmem + lb + K::COL_DV + 32 * qd, v);
@@ -879,39 +908,29 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
 #pragma unroll
                             for (int e = 0; e < 8; ++e) ov[e] = fmaf(dd[e], do8[e], ov[e]);
                         }
-                        *reinterpret_cast<uint4*>(sm.u.ost + off_raw(r, jg)) = pack8(ov);
-                        *reinterpret_cast<uint4*>(sm.u.ost + VB * kBox + off_raw(r, jg)) = pack8(ob);
+                        *reinterpret_cast<uint4*>(sm.vh + off_raw(r, jg)) = pack8(ov);
+                        *reinterpret_cast<uint4*>(sm.dot + off_raw(r, jg)) = pack8(ob);
                     }
+                }
+                // this warp's last read of the raw tiles (v, beta, dO) and of TMEM
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&sm.raw_empty);
+                    mbar_arrive(&sm.tm2_free);
                 }
                 fence_proxy_async_smem();
                 named_bar(kBarEpi, 128);
                 if (threadIdx.x == 0) {
 #pragma unroll
                     for (int vb = 0; vb < VB; ++vb) {
-                        tma_store_3d(&A.mdv, sm.u.ost + vb * kBox, 64 * vb, c * C, bh);
-                        tma_store_3d(&A.mdb, sm.u.ost + (VB + vb) * kBox, 64 * vb, c * C, bh);
+                        tma_store_3d(&A.mdv, sm.vh + vb * kBox, 64 * vb, c * C, bh);
+                        tma_store_3d(&A.mdb, sm.dot + vb * kBox, 64 * vb, c * C, bh);
                     }
                     bulk_commit();
-                    bulk_wait_read_all();  // the union takes the dQ / dK staging next
+                    bulk_wait_read_all();  // the gate warps write the next chunk's operands there
+                    mbar_arrive(&sm.vh_free);
                 }
-                named_bar(kBarEpi, 128);
-            }
-            // dQ, dK -> fp32 staging for the gate warps
-#pragma unroll
-            for (int which = 0; which < 2; ++which) {
-                float v[32];
-                tmem_ld32_split<32>(tmem + lb + (which == 0 ? K::COL_DQ : K::COL_DK), v);
-                tmem_ld_wait();
-                float4* dst = reinterpret_cast<float4*>(which == 0 ? &sm.u.st.dqs[r][32 * hf] : &sm.u.st.dks[r][32 * hf]);
-#pragma unroll
-                for (int e4 = 0; e4 < 8; ++e4)
-                    dst[e4] = make_float4(v[4 * e4], v[4 * e4 + 1], v[4 * e4 + 2], v[4 * e4 + 3]);
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&sm.post_ready);
-                mbar_arrive(&sm.tm2_free);
             }
             ++i2;
         }
