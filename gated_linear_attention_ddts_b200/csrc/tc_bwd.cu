@@ -786,7 +786,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             // the gate warps have read S_prev out of the union (and staged S_hat)
             if (!mbar_wait_own(&sm.shat_full, i2 & 1, fail, WL)) break;
             // A and B -> causal mask -> bf16 operands (row t = r, columns s = 32 hf + e)
-#pragma unroll
+#pragma unroll 1
             for (int which = 0; which < 2; ++which) {
                 float v[32];
                 tmem_ld32_split<32>(tmem + lb + (which == 0 ? K::COL_A : K::COL_B), v);
@@ -858,7 +858,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             // previous chunk's gate stage has read its staging), so that their final
             // stage runs beside the dv / dbeta stage below
             if (i2 > 0 && !mbar_wait_own(&sm.post_done, (i2 - 1) & 1, fail, WL)) break;
-#pragma unroll
+#pragma unroll 1
             for (int which = 0; which < 2; ++which) {
                 float v[32];
                 tmem_ld32_split<32>(tmem + lb + (which == 0 ? K::COL_DQ : K::COL_DK), v);
