@@ -106,7 +106,7 @@ struct alignas(1024) BwdSmem {
     uint8_t shat[DK * DV * 2];  // [i][j], e^m S_prev (written by the gate warps)
     float em[DK], cf[DK], gm[DK], fin[DK], carry[DK];
     float bdiag[C];  // B_tt = vhat_t . dO_t (the diagonal kept out of the dQ / dK MMAs)
-    uint64_t raw_full, raw_empty, sp_full, ops_full, shat_full, ops_empty, g1_done, g2_ready,
+    uint64_t raw_full, rawv_full, raw_empty, sp_full, ops_full, shat_full, ops_empty, g1_done, g2_ready,
         tm1_free, g2_done, tm2_free, post_ready, post_done, p1_done, vh_free;
     uint32_t tmem_base;
     int fail;
@@ -173,7 +173,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
     auto pass_p2 = [&](int li) { return !has_p1 || li >= nseg; };
 
     if (threadIdx.x == 0) {
-        mbar_init(&sm.raw_full, 1);
+        mbar_init(&sm.raw_full, 1);   // q, k, g, tau
+        mbar_init(&sm.rawv_full, 1);  // v, beta, dO
         mbar_init(&sm.raw_empty, kGateWarps + 4);  // the epilogue reads v, beta, dO too
         mbar_init(&sm.sp_full, 1);
         mbar_init(&sm.ops_full, kGateWarps);
@@ -219,17 +220,21 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 const bool p2 = pass_p2(li);
                 if (li > 0 && !mbar_wait(&sm.raw_empty, (li - 1) & 1, fail, WL)) break;
                 // the R-only pass reads q, g, tau and dO
-                mbar_expect_tx(&sm.raw_full, p2 ? K::RAW : (3 + VB) * kBox);
-                tma_load_3d(sm.raw + 0 * kBox, &A.mq, &sm.raw_full, 0, c * C, bh);
-                if (p2) tma_load_3d(sm.raw + 1 * kBox, &A.mk, &sm.raw_full, 0, c * C, bh);
+                // the key side first (the gate warps start with its scan), then the
+                // value side on its own barrier
+                mbar_expect_tx(&sm.raw_full, (p2 ? 4 : 3) * kBox);
                 tma_load_3d(sm.raw + 2 * kBox, &A.mg, &sm.raw_full, 0, c * C, bh);
                 tma_load_3d(sm.raw + 3 * kBox, &A.mt, &sm.raw_full, 0, c * C, bh);
+                tma_load_3d(sm.raw + 0 * kBox, &A.mq, &sm.raw_full, 0, c * C, bh);
+                if (p2) tma_load_3d(sm.raw + 1 * kBox, &A.mk, &sm.raw_full, 0, c * C, bh);
+                // the R-only pass reads dO only
+                mbar_expect_tx(&sm.rawv_full, (p2 ? 3 : 1) * VB * kBox);
                 for (int vb = 0; vb < VB; ++vb) {
                     if (p2) {
-                        tma_load_3d(sm.raw + K::OFF_V + vb * kBox, &A.mv, &sm.raw_full, 64 * vb, c * C, bh);
-                        tma_load_3d(sm.raw + K::OFF_B + vb * kBox, &A.mb, &sm.raw_full, 64 * vb, c * C, bh);
+                        tma_load_3d(sm.raw + K::OFF_V + vb * kBox, &A.mv, &sm.rawv_full, 64 * vb, c * C, bh);
+                        tma_load_3d(sm.raw + K::OFF_B + vb * kBox, &A.mb, &sm.rawv_full, 64 * vb, c * C, bh);
                     }
-                    tma_load_3d(sm.raw + K::OFF_DO + vb * kBox, &A.mdo, &sm.raw_full, 64 * vb, c * C, bh);
+                    tma_load_3d(sm.raw + K::OFF_DO + vb * kBox, &A.mdo, &sm.rawv_full, 64 * vb, c * C, bh);
                 }
                 ++issued;
                 // the next pass's tiles (and chunk-start state) into L2 while this one runs
@@ -259,7 +264,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                     ++issued_sp;
                 }
             }
-            if (issued > 0) drain_wait(&sm.raw_full, (issued - 1) & 1);
+            if (issued > 0) {
+                drain_wait(&sm.raw_full, (issued - 1) & 1);
+                drain_wait(&sm.rawv_full, (issued - 1) & 1);
+            }
             if (issued_sp > 0) drain_wait(&sm.sp_full, (issued_sp - 1) & 1);
         }
     } else if (warp == kMmaWarp) {
@@ -460,6 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
 #pragma unroll
                     for (int e = 0; e < 8; ++e) sm.gm[cg * 8 + e] = gh2[e];
                 }
+                if (!mbar_wait_own(&sm.rawv_full, li & 1, fail, WL)) break;
 #pragma unroll
                 for (int iv = 0; iv < VIT; ++iv) {
                     const int jg = gt / TPG, t = (gt % TPG) + TPG * iv;
@@ -519,6 +528,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             // Vh and dO operand buffers: the epilogue's dv / dbeta stores of the
             // previous chunk have read them
             if (i2 > 0 && !mbar_wait_own(&sm.vh_free, (i2 - 1) & 1, fail, WL)) break;
+            if (!mbar_wait_own(&sm.rawv_full, li & 1, fail, WL)) break;
 #pragma unroll
             for (int iv = 0; iv < VIT; ++iv) {
                 const int jg = gt / TPG, t = (gt % TPG) + TPG * iv;
