@@ -100,7 +100,7 @@ FWD_SRC = ["tc_fwd.cu"] + _DEV_HDR
 BWD_SRC = ["tc_bwd.cu"] + _DEV_HDR
 DECODE_SRC = ["decode.cu", "rdm_common.cuh", "launch.h"]
 SKA_SRC = ["ska.cu", "ska_launch.h"] + _DEV_HDR
-CONV_SRC = ["shortconv.cu"] + _DEV_HDR
+CONV_SRC = ["shortconv.cu", "conv_launch.h"] + _DEV_HDR
 
 
 def src_sha(*names):
@@ -380,13 +380,16 @@ def run_extras(rdm, dev, pk, K):
         outs = dict(dx=torch.empty_like(xc), dw=torch.empty_like(wc), dbias=torch.empty_like(bc))
         convs.append((xc, wc, bc, gy, torch.empty_like(xc), outs))
 
-    def conv_step():
-        for xc, wc, bc, gy, yc, outs in convs:
-            rdm.rdm_shortconv_fwd(xc, wc, bc, None, silu=True, y=yc)
-            rdm.rdm_shortconv_bwd(xc, wc, bc, None, gy, None, silu=True, out=outs)
+    # the three tensors in one batched forward and one batched backward launch
+    fwd_many = [dict(x=xc, weight=wc, bias=bc, y=yc) for xc, wc, bc, gy, yc, outs in convs]
+    bwd_many = [dict(x=xc, weight=wc, bias=bc, grad_y=gy, out=outs) for xc, wc, bc, gy, yc, outs in convs]
 
-    # six short kernels per step: replayed as one CUDA graph so that the step
-    # is timed on the device, not through the Python binding's per-call overhead
+    def conv_step():
+        rdm.rdm_shortconv_fwd_many(fwd_many, silu=True)
+        rdm.rdm_shortconv_bwd_many(bwd_many, silu=True)
+
+    # short kernels: replayed as one CUDA graph so that the step is timed on the
+    # device, not through the Python binding's per-call overhead
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(side):
@@ -401,9 +404,9 @@ def run_extras(rdm, dev, pk, K):
     out["shortconv_fwd_bwd"] = {
         "workload": "ShortConv width 4 + SiLU, fwd+bwd over q, k, v of " + w.name,
         "value": w.B * w.T / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
-        # per tensor: forward kernel, backward kernel (the weight gradients are zeroed
-        # by memset, not counted)
-        "gpu_launches_per_step": 6, "cuda_graph": True,
+        # one batched forward and one batched backward kernel (the weight gradients
+        # are zeroed by memsets, not counted)
+        "gpu_launches_per_step": 2, "cuda_graph": True,
         "roofline": roofline(cb, 0, ms, pk, None)}
     del gconv, convs, fl
     out.update(run_ska(rdm, dev, pk, K))

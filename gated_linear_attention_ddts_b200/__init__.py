@@ -12,12 +12,13 @@ from ._binding import (IMPL, RDM_BF16, RDM_ERR_CUDA, RDM_ERR_INVALID_ARG, RDM_ER
                        rdm_ddts_bwd, rdm_ddts_bwd_noalloc, rdm_ddts_bwd_workspace_size, rdm_ddts_decode, rdm_ddts_decode_step,
                        rdm_ddts_fwd, rdm_ddts_fwd_workspace_size, rdm_ddts_saved_states_size,
                        rdm_ddts_set_test_hooks, rdm_ddts_sync_status,
-                       rdm_ddts_version, rdm_shortconv_bwd, rdm_shortconv_fwd,
-                       rdm_ska_decode, rdm_ska_fwd, rdm_status_string)
+                       rdm_ddts_version, rdm_shortconv_bwd, rdm_shortconv_bwd_many, rdm_shortconv_fwd,
+                       rdm_shortconv_fwd_many, rdm_ska_decode, rdm_ska_fwd, rdm_status_string)
 
 __all__ = ["rdm_ddts_fwd", "rdm_ddts_fwd_workspace_size", "rdm_ddts_bwd", "rdm_ddts_bwd_noalloc", "rdm_ddts_bwd_workspace_size",
            "rdm_ddts_saved_states_size", "rdm_ddts_decode", "rdm_ddts_decode_step", "rdm_ddts_sync_status",
            "rdm_status_string", "rdm_ddts_set_test_hooks", "rdm_ddts_version", "rdm_shortconv_fwd",
-           "rdm_shortconv_bwd", "rdm_ska_fwd", "rdm_ska_decode", "RdmError", "IMPL", "RDM_OK",
+           "rdm_shortconv_bwd", "rdm_shortconv_fwd_many", "rdm_shortconv_bwd_many", "rdm_ska_fwd",
+           "rdm_ska_decode", "RdmError", "IMPL", "RDM_OK",
            "RDM_ERR_INVALID_ARG", "RDM_ERR_UNSUPPORTED", "RDM_ERR_CUDA", "RDM_ERR_TIMEOUT",
            "RDM_ERR_WORKSPACE", "RDM_F32", "RDM_BF16"]

@@ -88,7 +88,8 @@ EXPORTS = ["rdm_ddts_fwd", "rdm_ddts_fwd_workspace_size", "rdm_ddts_saved_states
            "rdm_ddts_bwd_workspace_size", "rdm_ddts_bwd_noalloc", "rdm_ddts_decode_step", "rdm_ddts_decode",
            "rdm_ddts_sync_status",
            "rdm_status_string", "rdm_ddts_set_test_hooks", "rdm_ddts_version", "rdm_shortconv_fwd",
-           "rdm_shortconv_bwd", "rdm_ska_fwd", "rdm_ska_decode"]
+           "rdm_shortconv_bwd", "rdm_shortconv_fwd_many", "rdm_shortconv_bwd_many", "rdm_ska_fwd",
+           "rdm_ska_decode"]
 
 
 def load():
@@ -123,6 +124,10 @@ def load():
         lib.rdm_shortconv_fwd.restype = _I
         lib.rdm_shortconv_bwd.argtypes = [ctypes.POINTER(ConvBwdArgs), _VP]
         lib.rdm_shortconv_bwd.restype = _I
+        lib.rdm_shortconv_fwd_many.argtypes = [ctypes.POINTER(ConvArgs), _I, _VP]
+        lib.rdm_shortconv_fwd_many.restype = _I
+        lib.rdm_shortconv_bwd_many.argtypes = [ctypes.POINTER(ConvBwdArgs), _I, _VP]
+        lib.rdm_shortconv_bwd_many.restype = _I
         lib.rdm_ska_fwd.argtypes = [ctypes.POINTER(SkaFwdArgs), _VP]
         lib.rdm_ska_fwd.restype = _I
         lib.rdm_ska_decode.argtypes = [ctypes.POINTER(SkaDecodeArgs), _VP]
@@ -376,6 +381,54 @@ def rdm_shortconv_bwd(x, weight, bias, state_in, grad_y, grad_state_out=None, *,
                     _ptr(out["dxs"]))
     _check(load().rdm_shortconv_bwd(ctypes.byref(a), _stream(stream)), "rdm_shortconv_bwd")
     return out
+
+
+def rdm_shortconv_fwd_many(problems, *, silu=False, stream=None):
+    """Several independent ShortConv forwards in one launch.  `problems` is a
+    list (at most 4) of dicts with x, weight and optionally bias, state_in, y
+    and return_state, as for rdm_shortconv_fwd (same dtype and W in all).
+    Returns a list of (y, state_out or None)."""
+    outs, args = [], []
+    for pr in problems:
+        x, weight = pr["x"], pr["weight"]
+        B, H, T, D = x.shape
+        W = weight.shape[-1]
+        y = pr.get("y")
+        if y is None:
+            y = torch.empty_like(x)
+        state_out = (torch.empty(B, H, W - 1, D, dtype=x.dtype, device=x.device)
+                     if pr.get("return_state") else None)
+        args.append(_conv_args(x, weight, pr.get("bias"), pr.get("state_in"), y, state_out, silu))
+        outs.append((y, state_out))
+    arr = (ConvArgs * len(args))(*args)
+    _check(load().rdm_shortconv_fwd_many(arr, len(args), _stream(stream)), "rdm_shortconv_fwd_many")
+    return outs
+
+
+def rdm_shortconv_bwd_many(problems, *, silu=False, stream=None):
+    """Several independent ShortConv backwards in one launch.  `problems` is a
+    list (at most 4) of dicts with x, weight, grad_y and optionally bias,
+    state_in, grad_state_out and out, as for rdm_shortconv_bwd.  Returns a list
+    of dicts dx, dw, dbias, dxs."""
+    outs, args = [], []
+    for pr in problems:
+        x, weight, bias, state_in = pr["x"], pr["weight"], pr.get("bias"), pr.get("state_in")
+        out = dict(pr.get("out") or {})
+        if out.get("dx") is None:
+            out["dx"] = torch.empty_like(x)
+        if out.get("dw") is None:
+            out["dw"] = torch.empty_like(weight)
+        if out.get("dbias") is None:
+            out["dbias"] = torch.empty_like(bias) if bias is not None else None
+        if out.get("dxs") is None:
+            out["dxs"] = torch.empty_like(state_in) if state_in is not None else None
+        args.append(ConvBwdArgs(_conv_args(x, weight, bias, state_in, None, None, silu),
+                                _ptr(pr["grad_y"]), _ptr(pr.get("grad_state_out")), _ptr(out["dx"]),
+                                _ptr(out["dw"]), _ptr(out["dbias"]), _ptr(out["dxs"])))
+        outs.append(out)
+    arr = (ConvBwdArgs * len(args))(*args)
+    _check(load().rdm_shortconv_bwd_many(arr, len(args), _stream(stream)), "rdm_shortconv_bwd_many")
+    return outs
 
 
 def rdm_ska_fwd(q, k, v, window, *, scale=0.0, o=None, k_cache=None, v_cache=None, pos=None,

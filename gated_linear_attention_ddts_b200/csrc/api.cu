@@ -7,6 +7,7 @@
 #include <atomic>
 
 #include "../../include/rdm_ddts.h"
+#include "conv_launch.h"
 #include "launch.h"
 #include "rdm_common.cuh"
 #include "ska_launch.h"
@@ -324,18 +325,16 @@ static ConvParams conv_params(const rdm_shortconv_args* a) {
     return p;
 }
 
-rdm_status rdm_shortconv_fwd(const rdm_shortconv_args* a, rdm_stream_t stream) {
+// argument checks of one problem (no CUDA call)
+static rdm_status conv_fwd_check(const rdm_shortconv_args* a) {
     rdm_status st = conv_check(a);
     if (st != RDM_OK) return st;
     if (a->T > 0 && (!a->y || !aligned(a->y))) return RDM_ERR_INVALID_ARG;
     if (!opt_aligned(a->state_out)) return RDM_ERR_INVALID_ARG;
-    const ConvParams p = conv_params(a);
-    if (!p.err) return RDM_ERR_CUDA;
-    return from_cuda(launch_conv_fwd(p, reinterpret_cast<cudaStream_t>(stream)));
+    return RDM_OK;
 }
 
-rdm_status rdm_shortconv_bwd(const rdm_shortconv_bwd_args* a, rdm_stream_t stream) {
-    if (!a) return RDM_ERR_INVALID_ARG;
+static rdm_status conv_bwd_check(const rdm_shortconv_bwd_args* a) {
     rdm_status st = conv_check(&a->fwd);
     if (st != RDM_OK) return st;
     if (!a->grad_weight || !aligned(a->grad_weight) || !opt_aligned(a->grad_bias) ||
@@ -343,17 +342,69 @@ rdm_status rdm_shortconv_bwd(const rdm_shortconv_bwd_args* a, rdm_stream_t strea
         return RDM_ERR_INVALID_ARG;
     if (a->fwd.T > 0 && (!a->grad_y || !aligned(a->grad_y) || !a->grad_x || !aligned(a->grad_x)))
         return RDM_ERR_INVALID_ARG;
-    ConvParams p = conv_params(&a->fwd);
-    if (!p.err) return RDM_ERR_CUDA;
-    p.y = nullptr;
-    p.xs_out = nullptr;
-    p.dy = a->grad_y;
-    p.dxs_out = a->fwd.W > 1 ? a->grad_state_out : nullptr;
-    p.dx = a->grad_x;
-    p.dw = a->grad_weight;
-    p.dbias = a->fwd.bias ? a->grad_bias : nullptr;
-    p.dxs = (a->fwd.state_in && a->fwd.W > 1) ? a->grad_state_in : nullptr;
-    return from_cuda(launch_conv_bwd(p, reinterpret_cast<cudaStream_t>(stream)));
+    return RDM_OK;
+}
+
+static rdm_status conv_bwd_params(const rdm_shortconv_bwd_args* a, ConvParams* p) {
+    *p = conv_params(&a->fwd);
+    if (!p->err) return RDM_ERR_CUDA;
+    p->y = nullptr;
+    p->xs_out = nullptr;
+    p->dy = a->grad_y;
+    p->dxs_out = a->fwd.W > 1 ? a->grad_state_out : nullptr;
+    p->dx = a->grad_x;
+    p->dw = a->grad_weight;
+    p->dbias = a->fwd.bias ? a->grad_bias : nullptr;
+    p->dxs = (a->fwd.state_in && a->fwd.W > 1) ? a->grad_state_in : nullptr;
+    return RDM_OK;
+}
+
+// one launch serves problems of the same element type, width and activation
+static bool conv_same_kind(const rdm_shortconv_args& a, const rdm_shortconv_args& b) {
+    return a.dtype == b.dtype && a.W == b.W && (a.silu != 0) == (b.silu != 0);
+}
+
+rdm_status rdm_shortconv_fwd(const rdm_shortconv_args* a, rdm_stream_t stream) {
+    return rdm_shortconv_fwd_many(a, 1, stream);
+}
+
+rdm_status rdm_shortconv_bwd(const rdm_shortconv_bwd_args* a, rdm_stream_t stream) {
+    return rdm_shortconv_bwd_many(a, 1, stream);
+}
+
+rdm_status rdm_shortconv_fwd_many(const rdm_shortconv_args* a, int n, rdm_stream_t stream) {
+    if (!a || n < 1 || n > kMaxConvBatch) return RDM_ERR_INVALID_ARG;
+    for (int i = 0; i < n; ++i) {
+        if (!conv_same_kind(a[0], a[i])) return RDM_ERR_INVALID_ARG;
+        rdm_status st = conv_fwd_check(&a[i]);
+        if (st != RDM_OK) return st;
+    }
+    ConvParams ps[kMaxConvBatch];
+    for (int i = 0; i < n; ++i) {
+        ps[i] = conv_params(&a[i]);
+        if (!ps[i].err) return RDM_ERR_CUDA;
+    }
+    // problems without sequences have nothing to compute
+    int m = 0;
+    for (int i = 0; i < n; ++i)
+        if (ps[i].B * ps[i].H > 0) ps[m++] = ps[i];
+    if (m == 0) return RDM_OK;
+    return from_cuda(launch_conv_fwd_many(ps, m, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+rdm_status rdm_shortconv_bwd_many(const rdm_shortconv_bwd_args* a, int n, rdm_stream_t stream) {
+    if (!a || n < 1 || n > kMaxConvBatch) return RDM_ERR_INVALID_ARG;
+    for (int i = 0; i < n; ++i) {
+        if (!conv_same_kind(a[0].fwd, a[i].fwd)) return RDM_ERR_INVALID_ARG;
+        rdm_status st = conv_bwd_check(&a[i]);
+        if (st != RDM_OK) return st;
+    }
+    ConvParams ps[kMaxConvBatch];
+    for (int i = 0; i < n; ++i) {
+        rdm_status st = conv_bwd_params(&a[i], &ps[i]);
+        if (st != RDM_OK) return st;
+    }
+    return from_cuda(launch_conv_bwd_many(ps, n, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 static bool ska_dim_ok(int d) { return d == 64 || d == 128; }

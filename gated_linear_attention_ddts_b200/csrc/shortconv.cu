@@ -21,6 +21,7 @@
 // then shared memory) before one float32 atomic per value and head.
 #include <algorithm>
 
+#include "conv_launch.h"
 #include "launch.h"
 #include "rdm_common.cuh"
 #include "tc_ptx.cuh"
@@ -137,6 +138,19 @@ __device__ __forceinline__ ConvTile conv_tile_of(const ConvParams& p, int g) {
     return c;
 }
 
+// The problems of one launch: problem i owns global tiles [tile0[i], tile0[i+1]).
+struct ConvBatch {
+    ConvParams p[kMaxConvBatch];
+    int tile0[kMaxConvBatch + 1];
+    int n;
+    int stage;  // elements per ring stage: the largest of the problems'
+};
+__device__ __forceinline__ int conv_problem(const ConvBatch& m, int g) {
+    int i = 0;
+    while (i + 1 < m.n && g >= m.tile0[i + 1]) ++i;
+    return i;
+}
+
 // Thread 0: bulk copy of the in-sequence rows [max(lo, 0), min(hi, T)) of
 // sequence bh into dst, whose row 0 is token lo (the rows of one (b, h) are
 // contiguous in HBM).  Returns the bytes it will deliver on `bar`.
@@ -201,20 +215,22 @@ __device__ void drain_stages(uint64_t* full, int k, int g, int g1, const ConvPar
 // (4096 elements) give every block several, so that the first tiles' work
 // overlaps the later tiles' copies.
 template <typename T, int W, bool SILU>
-__global__ void __launch_bounds__(kThreads, 4) conv_fwd_kernel(const ConvParams p) {
+__global__ void __launch_bounds__(kThreads, 4) conv_fwd_kernel(const __grid_constant__ ConvBatch m) {
     constexpr int N = Vec<T>::N, RUN = kConvFwdRun;
     extern __shared__ __align__(128) uint8_t conv_smem[];
     __shared__ uint64_t full[kConvStages];
-    const int CG = p.D / N;
-    const int total = p.B * p.H * ((p.T + p.tile - 1) / p.tile);
+    const int total = m.tile0[m.n];
     // a contiguous run of tiles per block (same sequence, mostly the same head);
     // the runs of the blocks differ by at most one tile
     const int g0 = (int)((long long)blockIdx.x * total / gridDim.x);
     const int g1 = (int)((long long)(blockIdx.x + 1) * total / gridDim.x);
-    const size_t stage = (size_t)(p.tile + W - 1) * p.D;  // elements per ring stage
+    const size_t stage = (size_t)m.stage;
     T* ring = reinterpret_cast<T*>(conv_smem);
+    const ConvParams& p0 = m.p[0];  // status word, wait bound and test hook (shared)
     auto issue = [&](int g, int s) {
-        const ConvTile c = conv_tile_of(p, g);
+        const int pi = conv_problem(m, g);
+        const ConvParams& p = m.p[pi];
+        const ConvTile c = conv_tile_of(p, g - m.tile0[pi]);
         mbar_expect_tx(&full[s], (uint32_t)((size_t)(c.t1 - max(c.t0 - (W - 1), 0)) * p.D * sizeof(T)));
         if (p.withhold) return;  // test hook: the stage never fills, its wait runs out
         copy_rows<T>(p, static_cast<const T*>(p.x), c.bh, c.t0 - (W - 1), c.t1, ring + s * stage, &full[s]);
@@ -226,15 +242,19 @@ __global__ void __launch_bounds__(kThreads, 4) conv_fwd_kernel(const ConvParams 
             if (g0 + s < g1) issue(g0 + s, s);
     }
     __syncthreads();
-    const int cg = threadIdx.x % CG, run = threadIdx.x / CG, c0 = cg * N;
     float wv[W][N], bv[N];
-    int cur_h = -1;
+    int cur_p = -1, cur_h = -1;
     int k = 0;
     for (int g = g0; g < g1; ++g, ++k) {
         const int s = k % kConvStages;
-        const ConvTile c = conv_tile_of(p, g);
+        const int pi = conv_problem(m, g);
+        const ConvParams& p = m.p[pi];
+        const ConvTile c = conv_tile_of(p, g - m.tile0[pi]);
+        const int CG = p.D / N;
+        const int cg = threadIdx.x % CG, run = threadIdx.x / CG, c0 = cg * N;
         const int lo = c.t0 - (W - 1);
-        if (c.h != cur_h) {  // consecutive tiles mostly share the head
+        if (pi != cur_p || c.h != cur_h) {  // consecutive tiles mostly share the head
+            cur_p = pi;
             cur_h = c.h;
 #pragma unroll
             for (int e = 0; e < N; ++e) {
@@ -243,8 +263,8 @@ __global__ void __launch_bounds__(kThreads, 4) conv_fwd_kernel(const ConvParams 
                 bv[e] = p.bias ? __ldg(p.bias + (size_t)c.h * p.D + c0 + e) : 0.0f;
             }
         }
-        if (!stage_ready(&full[s], (k / kConvStages) & 1, p)) {
-            drain_stages<kConvStages>(full, k, g, g1, p);
+        if (!stage_ready(&full[s], (k / kConvStages) & 1, p0)) {
+            drain_stages<kConvStages>(full, k, g, g1, p0);
             return;
         }
         T* xs = ring + s * stage;
@@ -338,23 +358,24 @@ __device__ __forceinline__ void dz_row(const ConvParams& p, int bh, int t, int c
 // per value for each run of tiles of one head.
 constexpr int kConvBwdRun = 8;
 template <typename T, int W, bool SILU>
-__global__ void __launch_bounds__(kThreads, 2) conv_bwd_kernel(const ConvParams p) {
+__global__ void __launch_bounds__(kThreads, 2) conv_bwd_kernel(const __grid_constant__ ConvBatch m) {
     constexpr int N = Vec<T>::N, RUN = kConvBwdRun;
     extern __shared__ __align__(128) uint8_t conv_smem[];
     __shared__ uint64_t full[kConvBwdStages];
-    const int TT = p.tile;
-    const int total = p.B * p.H * ((p.T + TT - 1) / TT);
+    const int total = m.tile0[m.n];
     // contiguous runs of tiles that differ by at most one tile between blocks
     const int g0 = (int)((long long)blockIdx.x * total / gridDim.x);
     const int g1 = (int)((long long)(blockIdx.x + 1) * total / gridDim.x);
-    const size_t xrows = TT + 2 * (W - 1), yrows = TT + W - 1;
-    const size_t stage = (xrows + yrows) * p.D;  // elements per ring stage
+    const size_t stage = (size_t)m.stage;  // elements per ring stage
     T* ring = reinterpret_cast<T*>(conv_smem);
     float* s_red = reinterpret_cast<float*>(ring + kConvBwdStages * stage);  // [warps][D (W + 1)]
-    const int CG = p.D / N;
+    const ConvParams& p0 = m.p[0];  // status word, wait bound and test hook (shared)
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    // a ring stage holds x of tokens [t0 - (W-1), t1 + W - 1), then dy of [t0, t1 + W - 1)
     auto issue = [&](int g, int s) {
-        const ConvTile c = conv_tile_of(p, g);
+        const int pi = conv_problem(m, g);
+        const ConvParams& p = m.p[pi];
+        const ConvTile c = conv_tile_of(p, g - m.tile0[pi]);
         const int lo = c.t0 - (W - 1), hi = c.t1 + W - 1;
         const size_t bx = (size_t)(min(hi, p.T) - max(lo, 0)) * p.D * sizeof(T);
         const size_t by = (size_t)(min(hi, p.T) - c.t0) * p.D * sizeof(T);
@@ -362,7 +383,8 @@ __global__ void __launch_bounds__(kThreads, 2) conv_bwd_kernel(const ConvParams 
         if (p.withhold) return;  // test hook: the stage never fills, its wait runs out
         T* st = ring + s * stage;
         copy_rows<T>(p, static_cast<const T*>(p.x), c.bh, lo, hi, st, &full[s]);
-        copy_rows<T>(p, static_cast<const T*>(p.dy), c.bh, c.t0, hi, st + xrows * p.D, &full[s]);
+        copy_rows<T>(p, static_cast<const T*>(p.dy), c.bh, c.t0, hi, st + (size_t)(p.tile + 2 * (W - 1)) * p.D,
+                     &full[s]);
     };
     if (threadIdx.x == 0) {
         for (int s = 0; s < kConvBwdStages; ++s) mbar_init(&full[s], 1);
@@ -371,14 +393,14 @@ __global__ void __launch_bounds__(kThreads, 2) conv_bwd_kernel(const ConvParams 
             if (g0 + s < g1) issue(g0 + s, s);
     }
     __syncthreads();
-    const int cg = threadIdx.x % CG, r0 = threadIdx.x / CG, c0 = cg * N;
-    const int tout0 = p.T - (W - 1);  // first token copied into the carried-out state
-    const int DW1 = p.D * (W + 1);
     float wv[W][N], bv[N], aw[W][N], ab[N];
-    // weight and bias gradients summed over the block's tiles of head h: lanes
-    // holding the same channels (cg, cg + CG, ...) by shuffles, one slot per
-    // warp in shared memory, a sum over the warps, one float32 atomic per value
-    auto flush = [&](int h) {
+    // weight and bias gradients summed over the block's tiles of head h of
+    // problem pi: lanes holding the same channels (cg, cg + CG, ...) by shuffles,
+    // one slot per warp in shared memory, a sum over the warps, one float32
+    // atomic per value
+    auto flush = [&](int pi, int h) {
+        const ConvParams& p = m.p[pi];
+        const int CG = p.D / N, cg = threadIdx.x % CG, DW1 = p.D * (W + 1);
 #pragma unroll
         for (int e = 0; e < N; ++e) {
 #pragma unroll
@@ -401,14 +423,20 @@ __global__ void __launch_bounds__(kThreads, 2) conv_bwd_kernel(const ConvParams 
         }
         __syncthreads();  // s_red read before it is written again
     };
-    int cur_h = -1;
+    int cur_p = -1, cur_h = -1;
     int k = 0;
     for (int g = g0; g < g1; ++g, ++k) {
         const int s = k % kConvBwdStages;
-        const ConvTile c = conv_tile_of(p, g);
+        const int pi = conv_problem(m, g);
+        const ConvParams& p = m.p[pi];
+        const ConvTile c = conv_tile_of(p, g - m.tile0[pi]);
+        const int CG = p.D / N;
+        const int cg = threadIdx.x % CG, r0 = threadIdx.x / CG, c0 = cg * N;
+        const int tout0 = p.T - (W - 1);  // first token copied into the carried-out state
         const int lo = c.t0 - (W - 1);
-        if (c.h != cur_h) {  // block-uniform
-            if (cur_h >= 0) flush(cur_h);
+        if (pi != cur_p || c.h != cur_h) {  // block-uniform
+            if (cur_p >= 0) flush(cur_p, cur_h);
+            cur_p = pi;
             cur_h = c.h;
 #pragma unroll
             for (int e = 0; e < N; ++e) {
@@ -421,12 +449,12 @@ __global__ void __launch_bounds__(kThreads, 2) conv_bwd_kernel(const ConvParams 
                 ab[e] = 0.0f;
             }
         }
-        if (!stage_ready(&full[s], (k / kConvBwdStages) & 1, p)) {
-            drain_stages<kConvBwdStages>(full, k, g, g1, p);
+        if (!stage_ready(&full[s], (k / kConvBwdStages) & 1, p0)) {
+            drain_stages<kConvBwdStages>(full, k, g, g1, p0);
             return;
         }
         T* xs = ring + s * stage;
-        const T* dys = xs + xrows * p.D;
+        const T* dys = xs + (size_t)(p.tile + 2 * (W - 1)) * p.D;
         if (W > 1 && lo < 0) fill_state_rows<T, W>(p, c.bh, lo, xs);
         const int ta = c.t0 + r0 * RUN, tb = min(ta + RUN, c.t1);
         if (ta < c.t1) {
@@ -503,7 +531,7 @@ __global__ void __launch_bounds__(kThreads, 2) conv_bwd_kernel(const ConvParams 
         __syncthreads();  // stage s fully read: refill it
         if (threadIdx.x == 0 && g + kConvBwdStages < g1) issue(g + kConvBwdStages, s);
     }
-    if (cur_h >= 0) flush(cur_h);
+    if (cur_p >= 0) flush(cur_p, cur_h);
 }
 
 // gradient of the carried-in state: dxs[s] = sum_i w_i dz[s-(W-1)+i] over tokens
@@ -550,101 +578,129 @@ __global__ void conv_state_grad_kernel(ConvParams p) {
 int conv_tile(const ConvParams& p) { return kConvFwdRun * kThreads / (p.D / Vec<float>::N); }
 int conv_tile_bwd(const ConvParams& p) { return kConvBwdRun * kThreads / (p.D / Vec<float>::N); }
 
-template <typename T, int W>
-size_t fwd_smem(const ConvParams& p) {
-    return (size_t)kConvStages * (p.tile + W - 1) * p.D * sizeof(T);
-}
-
-template <typename T, int W>
-size_t bwd_smem(const ConvParams& p) {
-    const size_t stage = (size_t)(2 * p.tile + 3 * (W - 1)) * p.D * sizeof(T);
-    return kConvBwdStages * stage + (size_t)(kThreads / 32) * p.D * (W + 1) * 4;
+// The batch of a launch: tiles of each problem, their index space, the largest
+// ring stage.  Returns the number of tiles.
+template <int W>
+int make_batch(ConvBatch& m, const ConvParams* ps, int n, bool bwd, size_t elem) {
+    m.n = n;
+    int total = 0;
+    size_t stage = 0;
+    for (int i = 0; i < n; ++i) {
+        ConvParams p = ps[i];
+        p.tile = bwd ? conv_tile_bwd(p) : conv_tile(p);
+        m.p[i] = p;
+        m.tile0[i] = total;
+        if (p.T > 0) total += p.B * p.H * ((p.T + p.tile - 1) / p.tile);
+        const size_t rows = bwd ? (size_t)2 * p.tile + 3 * (W - 1) : (size_t)p.tile + W - 1;
+        stage = std::max(stage, rows * p.D);
+    }
+    m.tile0[n] = total;
+    // keep every stage 128-byte aligned (bulk copies need 16)
+    const size_t q = 128 / elem;
+    m.stage = (int)((stage + q - 1) / q * q);
+    return total;
 }
 
 // Persistent grid: `per_sm` blocks per SM, or fewer when there are fewer tiles.
-unsigned conv_grid(const ConvParams& p, int per_sm) {
-    const long long tiles = (long long)p.B * p.H * ((p.T + p.tile - 1) / p.tile);
+unsigned conv_grid(int tiles, int per_sm) {
     const long long cap = (long long)per_sm * sm_count();
     return (unsigned)(tiles < cap ? tiles : cap);
 }
 
 template <typename T, int W>
-cudaError_t fwd_tw(const ConvParams& p0, cudaStream_t s) {
-    ConvParams p = p0;
-    p.tile = conv_tile(p);
-    if (p.T > 0) {
-        const size_t smem = fwd_smem<T, W>(p);
-        auto kern = p.silu ? conv_fwd_kernel<T, W, true> : conv_fwd_kernel<T, W, false>;
+cudaError_t fwd_tw(const ConvParams* ps, int n, cudaStream_t s) {
+    ConvBatch m;
+    const int tiles = make_batch<W>(m, ps, n, false, sizeof(T));
+    if (tiles > 0) {
+        const size_t smem = (size_t)kConvStages * m.stage * sizeof(T);
+        auto kern = ps[0].silu ? conv_fwd_kernel<T, W, true> : conv_fwd_kernel<T, W, false>;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        kern<<<conv_grid(p, 4), kThreads, smem, s>>>(p);
+        kern<<<conv_grid(tiles, 4), kThreads, smem, s>>>(m);
     }
-    if (p.xs_out && W > 1) {
-        const size_t n = (size_t)p.B * p.H * (W - 1) * p.D;
-        conv_state_kernel<T><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(p);
+    for (int i = 0; i < n; ++i) {
+        const ConvParams& p = ps[i];
+        if (p.xs_out && W > 1) {
+            const size_t ne = (size_t)p.B * p.H * (W - 1) * p.D;
+            conv_state_kernel<T><<<(unsigned)((ne + 255) / 256), 256, 0, s>>>(p);
+        }
     }
     return cudaGetLastError();
 }
 
 template <typename T, int W>
-cudaError_t bwd_tw(const ConvParams& p0, cudaStream_t s) {
-    ConvParams p = p0;
-    p.tile = conv_tile_bwd(p);
-    cudaError_t e = cudaMemsetAsync(p.dw, 0, (size_t)p.H * p.D * W * sizeof(float), s);
-    if (e == cudaSuccess && p.dbias) e = cudaMemsetAsync(p.dbias, 0, (size_t)p.H * p.D * sizeof(float), s);
-    if (e != cudaSuccess) return e;
-    if (p.T > 0) {
-        const size_t smem = bwd_smem<T, W>(p);
-        auto kern = p.silu ? conv_bwd_kernel<T, W, true> : conv_bwd_kernel<T, W, false>;
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+cudaError_t bwd_tw(const ConvParams* ps, int n, cudaStream_t s) {
+    for (int i = 0; i < n; ++i) {
+        const ConvParams& p = ps[i];
+        cudaError_t e = cudaMemsetAsync(p.dw, 0, (size_t)p.H * p.D * W * sizeof(float), s);
+        if (e == cudaSuccess && p.dbias) e = cudaMemsetAsync(p.dbias, 0, (size_t)p.H * p.D * sizeof(float), s);
         if (e != cudaSuccess) return e;
-        kern<<<conv_grid(p, 2), kThreads, smem, s>>>(p);
+    }
+    ConvBatch m;
+    const int tiles = make_batch<W>(m, ps, n, true, sizeof(T));
+    if (tiles > 0) {
+        int dmax = 0;
+        for (int i = 0; i < n; ++i) dmax = std::max(dmax, ps[i].D);
+        const size_t smem = (size_t)kConvBwdStages * m.stage * sizeof(T) +
+                            (size_t)(kThreads / 32) * dmax * (W + 1) * 4;
+        auto kern = ps[0].silu ? conv_bwd_kernel<T, W, true> : conv_bwd_kernel<T, W, false>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        kern<<<conv_grid(tiles, 2), kThreads, smem, s>>>(m);
     }
     if constexpr (W > 1) {
-        if (p.dxs) {
-            const size_t n = (size_t)p.B * p.H * (W - 1) * (p.D / Vec<T>::N);
-            conv_state_grad_kernel<T, W><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(p);
+        for (int i = 0; i < n; ++i) {
+            const ConvParams& p = ps[i];
+            if (p.dxs && p.B * p.H > 0) {
+                const size_t ne = (size_t)p.B * p.H * (W - 1) * (p.D / Vec<T>::N);
+                conv_state_grad_kernel<T, W><<<(unsigned)((ne + 255) / 256), 256, 0, s>>>(p);
+            }
         }
     }
     return cudaGetLastError();
 }
 
 template <typename T>
-cudaError_t fwd_t(const ConvParams& p, cudaStream_t s) {
-    switch (p.W) {
-        case 1: return fwd_tw<T, 1>(p, s);
-        case 2: return fwd_tw<T, 2>(p, s);
-        case 3: return fwd_tw<T, 3>(p, s);
-        case 4: return fwd_tw<T, 4>(p, s);
+cudaError_t fwd_t(const ConvParams* ps, int n, cudaStream_t s) {
+    switch (ps[0].W) {
+        case 1: return fwd_tw<T, 1>(ps, n, s);
+        case 2: return fwd_tw<T, 2>(ps, n, s);
+        case 3: return fwd_tw<T, 3>(ps, n, s);
+        case 4: return fwd_tw<T, 4>(ps, n, s);
     }
     return cudaErrorInvalidValue;
 }
 
 template <typename T>
-cudaError_t bwd_t(const ConvParams& p, cudaStream_t s) {
-    switch (p.W) {
-        case 1: return bwd_tw<T, 1>(p, s);
-        case 2: return bwd_tw<T, 2>(p, s);
-        case 3: return bwd_tw<T, 3>(p, s);
-        case 4: return bwd_tw<T, 4>(p, s);
+cudaError_t bwd_t(const ConvParams* ps, int n, cudaStream_t s) {
+    switch (ps[0].W) {
+        case 1: return bwd_tw<T, 1>(ps, n, s);
+        case 2: return bwd_tw<T, 2>(ps, n, s);
+        case 3: return bwd_tw<T, 3>(ps, n, s);
+        case 4: return bwd_tw<T, 4>(ps, n, s);
     }
     return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
-cudaError_t launch_conv_fwd(const ConvParams& p, cudaStream_t s) {
-    if (p.B * p.H == 0) return cudaSuccess;
-    return p.bf16 ? fwd_t<__nv_bfloat16>(p, s) : fwd_t<float>(p, s);
+cudaError_t launch_conv_fwd_many(const ConvParams* ps, int n, cudaStream_t s) {
+    if (n < 1 || n > kMaxConvBatch) return cudaErrorInvalidValue;
+    return ps[0].bf16 ? fwd_t<__nv_bfloat16>(ps, n, s) : fwd_t<float>(ps, n, s);
 }
 
-cudaError_t launch_conv_bwd(const ConvParams& p, cudaStream_t s) {
-    if (p.B * p.H == 0) {  // no tokens anywhere: the weight gradients are zero
-        cudaError_t e = cudaMemsetAsync(p.dw, 0, (size_t)p.H * p.D * p.W * sizeof(float), s);
-        if (e == cudaSuccess && p.dbias) e = cudaMemsetAsync(p.dbias, 0, (size_t)p.H * p.D * sizeof(float), s);
-        return e;
-    }
-    return p.bf16 ? bwd_t<__nv_bfloat16>(p, s) : bwd_t<float>(p, s);
+cudaError_t launch_conv_bwd_many(const ConvParams* ps, int n, cudaStream_t s) {
+    if (n < 1 || n > kMaxConvBatch) return cudaErrorInvalidValue;
+    // a problem without tokens (B*H == 0 or T == 0) still gets its weight
+    // gradients zeroed by the memsets
+    return ps[0].bf16 ? bwd_t<__nv_bfloat16>(ps, n, s) : bwd_t<float>(ps, n, s);
 }
+
+cudaError_t launch_conv_fwd(const ConvParams& p, cudaStream_t s) {
+    if (p.B * p.H == 0) return cudaSuccess;
+    return launch_conv_fwd_many(&p, 1, s);
+}
+
+cudaError_t launch_conv_bwd(const ConvParams& p, cudaStream_t s) { return launch_conv_bwd_many(&p, 1, s); }
 
 }  // namespace rdm

@@ -338,6 +338,16 @@ typedef struct {
 
 rdm_status rdm_shortconv_bwd(const rdm_shortconv_bwd_args *args, rdm_stream_t stream);
 
+/* Several independent ShortConv problems in one launch (the q, k and v
+ * convolutions of a layer, say): args[0 .. n-1], 1 <= n <= 4, each exactly as
+ * for rdm_shortconv_fwd / rdm_shortconv_bwd (own B, H, T, D, pointers), all with
+ * the same dtype, W and silu (else RDM_ERR_INVALID_ARG; nothing is launched
+ * when any problem fails its checks).  Their tiles share the persistent
+ * blocks of one kernel, so the launch pays one ramp and one tail for all of
+ * them.  The single-problem calls above are these with n = 1. */
+rdm_status rdm_shortconv_fwd_many(const rdm_shortconv_args *args, int n, rdm_stream_t stream);
+rdm_status rdm_shortconv_bwd_many(const rdm_shortconv_bwd_args *args, int n, rdm_stream_t stream);
+
 /* ------------------------------------------------------------------ SW-SKA
  * Sliding-window shared-key attention, the attention half of the Rodimus+
  * block (Rodimus* digest.lyk-ai.com summary, "Method", Rodimus+ bullets: a

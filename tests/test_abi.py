@@ -169,3 +169,29 @@ def test_ska_fwd_validation(lib, kw, status):
     (dict(v=(1 << 20) + 2), 1), (dict(o=None), 1)])
 def test_ska_decode_validation(lib, kw, status):
     assert lib.rdm_ska_decode(ctypes.byref(_ska_dec(**kw)), None) == status
+
+
+def _conv(**kw):
+    from gated_linear_attention_ddts_b200._binding import RDM_BF16, ConvArgs
+    a = dict(B=1, H=2, T=64, D=64, W=4, dtype=RDM_BF16, silu=1, x=4096, weight=8192, bias=None,
+             state_in=None, y=12288, state_out=None)
+    a.update(kw)
+    return ConvArgs(a["B"], a["H"], a["T"], a["D"], a["W"], a["dtype"], a["silu"], a["x"], a["weight"],
+                    a["bias"], a["state_in"], a["y"], a["state_out"])
+
+
+def test_shortconv_many_validation(lib):
+    """The batched ShortConv calls refuse n outside [1, 4], problems of
+    different kinds (dtype, W, SiLU) and any problem that fails its own checks,
+    before any CUDA call."""
+    from gated_linear_attention_ddts_b200._binding import (RDM_ERR_INVALID_ARG, RDM_ERR_UNSUPPORTED,
+                                                           ConvArgs)
+    two = (ConvArgs * 2)(_conv(), _conv(D=128))
+    assert lib.rdm_shortconv_fwd_many(two, 0, None) == RDM_ERR_INVALID_ARG
+    assert lib.rdm_shortconv_fwd_many(two, 5, None) == RDM_ERR_INVALID_ARG
+    assert lib.rdm_shortconv_fwd_many(None, 1, None) == RDM_ERR_INVALID_ARG
+    for bad in (dict(W=3), dict(silu=0), dict(dtype=0)):
+        mixed = (ConvArgs * 2)(_conv(), _conv(**bad))
+        assert lib.rdm_shortconv_fwd_many(mixed, 2, None) == RDM_ERR_INVALID_ARG, bad
+    assert lib.rdm_shortconv_fwd_many((ConvArgs * 2)(_conv(), _conv(D=48)), 2, None) == RDM_ERR_UNSUPPORTED
+    assert lib.rdm_shortconv_fwd_many((ConvArgs * 2)(_conv(), _conv(y=12290)), 2, None) == RDM_ERR_INVALID_ARG

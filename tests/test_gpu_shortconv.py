@@ -78,3 +78,44 @@ def test_shortconv_full_size_layer_tensor(cuda_ok):
     assert_close(s, s_ref, 2e-2, "workload 1 shortconv state")
     for n in ("dx", "dw", "dbias"):
         assert_close(gr[n], ref[n], 2e-2, f"workload 1 shortconv {n}")
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("silu", [False, True])
+def test_shortconv_many_in_one_launch(cuda_ok, dtype, silu):
+    """Problems of different shapes (D 16, 64, 128 and 32; ragged T; one
+    without tokens; with and without bias and carried state) in one batched
+    forward and one batched backward, each against the oracle, and equal to the
+    single-problem calls."""
+    W = 4
+    shapes = [(2, 3, 37, 16, True, True), (1, 2, 300, 64, False, True), (2, 1, 129, 128, True, False),
+              (1, 1, 0, 32, False, True)]
+    probs, refs = [], []
+    for i, (B, H, T, D, state, bias) in enumerate(shapes):
+        x, w, b, xs = conv_inputs(B, H, T, D, W, dtype, seed=500 + i, state=state, bias=bias)
+        gy = torch.randn(B, H, T, D, generator=torch.Generator().manual_seed(600 + i)).to(dtype)
+        gso = torch.randn(B, H, W - 1, D, generator=torch.Generator().manual_seed(700 + i)).to(dtype)
+        probs.append(dict(x=x, w=w, b=b, xs=xs, gy=gy, gso=gso))
+        refs.append((oracle.shortconv_fwd(x, w, b, xs, silu=silu), oracle.shortconv_bwd(x, w, b, xs, gy, gso, silu=silu)))
+    d = [{k: cuda(v) for k, v in pr.items()} for pr in probs]
+    outs = rdm.rdm_shortconv_fwd_many(
+        [dict(x=q["x"], weight=q["w"], bias=q["b"], state_in=q["xs"], return_state=True) for q in d], silu=silu)
+    grads = rdm.rdm_shortconv_bwd_many(
+        [dict(x=q["x"], weight=q["w"], bias=q["b"], state_in=q["xs"], grad_y=q["gy"], grad_state_out=q["gso"])
+         for q in d], silu=silu)
+    torch.cuda.synchronize()
+    tol = TOL[dtype]
+    for i, ((y, so), gr, ((y_ref, so_ref), ref)) in enumerate(zip(outs, grads, refs)):
+        assert_close(y, y_ref, tol, f"batched shortconv y, problem {i}")
+        assert_close(so, so_ref, tol, f"batched shortconv state out, problem {i}")
+        assert_close(gr["dx"], ref["dx"], tol, f"batched shortconv dx, problem {i}")
+        assert_close(gr["dw"], ref["dw"], tol, f"batched shortconv dw, problem {i}")
+        if probs[i]["b"] is not None:
+            assert_close(gr["dbias"], ref["dbias"], tol, f"batched shortconv dbias, problem {i}")
+        if probs[i]["xs"] is not None:
+            assert_close(gr["dxs"], ref["dxs"], tol, f"batched shortconv d state in, problem {i}")
+        # the single-problem call gives the same forward bits
+        q = d[i]
+        y1, _ = rdm.rdm_shortconv_fwd(q["x"], q["w"], q["b"], q["xs"], silu=silu)
+        torch.cuda.synchronize()
+        assert torch.equal(y1, y), f"batched vs single forward, problem {i}"
