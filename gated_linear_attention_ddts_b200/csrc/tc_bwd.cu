@@ -320,6 +320,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 for (int ks = 0; ks < C / 16; ++ks)
                     mma_bf16(tmem + K::COL_DR, sdesc(q + ks * 256, 128, kQK),
                              sdesc(d + ks * 256, 128, 1024), id_r, ks > 0);
+                // and with Qt's bf16 remainder: R (hence dS_0 and the segment carries)
+                // to ~16 mantissa bits
+#pragma unroll
+                for (int ks = 0; ks < C / 16; ++ks)
+                    mma_bf16(tmem + K::COL_DR, sdesc(ql + ks * 256, 128, kQK),
+                             sdesc(d + ks * 256, 128, 1024), id_r, 1);
                 if (i2 == 0 && last_seg && p.dST) {
                     // Kt^T Vh of the last chunk, for S_T (only the final-state gradient needs it)
 #pragma unroll
