@@ -350,6 +350,22 @@ def run_extras(rdm, dev, pk, K):
                                  ncu_counters("tc_bwd_kernel", BWD_SRC, 3)),
         "roofline_step": roofline(fb + bwd_bytes(w), chunk_flops_fwd(w) + chunk_flops_bwd(w),
                                   msf + msb, pk, None)}
+    # the same backward with one chunk of every 16th head too wide for one decay
+    # reference (g scaled up 40x there): those heads are recomputed whole by the
+    # exact CUDA-core backward, which this line prices
+    gw = x["g"].float()
+    gw[:, ::16, 64 * 20:64 * 21] *= 40.0
+    x["g"] = gw.clamp(min=0.05).to(torch.bfloat16)
+    del gw
+    fwd()
+    tw = time_steps(bwd, max(3, K // 8), 2)
+    msw = statistics.mean(tw)
+    out["training_bwd_wide_heads"] = {
+        "workload": w.name + ", one chunk in every 16th head too wide for one reference",
+        "value": w.B * w.T / (msw / 1e3), "unit": "tokens/s", "ms_per_step": msw,
+        "ms_bwd_without": msb, "wide_heads": w.B * ((w.H + 15) // 16),
+        # backward kernel + the two exact re-run kernels
+        "gpu_launches_per_step": 3}
     del x, o, saved, grads, ws, wsf
     # headline forward with the feedthrough o_t += d (.) v_t (same algorithmic
     # bytes plus d; v is re-read from L2 in the store stage)

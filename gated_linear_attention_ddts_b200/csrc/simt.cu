@@ -7,8 +7,9 @@
 // (Rodimus*, digest.lyk-ai.com summary "Method" for the gates; diagonal decay
 // along d_k per the paperhub.cn rebuttal "Efficient Parallelization" bullet.)
 //
-// Backward, exact reverse mode organised in two sweeps per (b,h), thread i
-// owning row i of the state or of its gradient:
+// Backward, exact reverse mode organised in two sweeps per (b,h), each run by a
+// cluster of blocks that split the state's columns, thread i owning row i of
+// its block's columns of the state or of its gradient:
 //   sweep F (forward in t):  S_t, dq_t = S_t dO_t, and q_t*dq_t kept in scratch;
 //   sweep R (reverse in t):  dS_t = q_t dO_t^T + diag(alpha_{t+1}) dS_{t+1},
 //                            dkhat_t = dS_t vhat_t, dvhat_t = dS_t^T khat_t.
@@ -16,6 +17,8 @@
 //   dG_u = q_u*dq_u - khat_u*dkhat_u  (+ rowsum(dS_T o S_T) at u = T),
 // which follows from S_t = sum_s diag(exp(G_t - G_s)) khat_s vhat_s^T + diag(exp(G_t)) S_0
 // with G_t the running sum of log alpha.
+#include <cooperative_groups.h>
+
 #include "launch.h"
 #include "rdm_common.cuh"
 
@@ -89,169 +92,338 @@ __global__ void __launch_bounds__(128) simt_fwd_kernel(SeqParams p) {
 }
 
 // ------------------------------------------------ backward, forward sweep F
+// The state's columns are split over a cluster of DV / kCB blocks: the
+// recurrences of dS and S act column by column, so each block runs its kCB
+// columns for every row on its own.  Only the row sums over all columns (dq_t
+// here, dkhat_t in sweep R) need the whole cluster; each block writes its
+// partial sums of a tile of tokens into its shared memory, and after one cluster
+// barrier per tile the block that owns a row adds the partials of every block
+// through distributed shared memory.
+constexpr int kCB = 16;      // state columns per block
+constexpr int kMaxRows = 128;
+
+template <int DV>
+__device__ __forceinline__ int owner_rows(int dk) {
+    constexpr int NCB = DV / kCB;
+    return (dk + NCB - 1) / NCB;
+}
+
+// out[tt] = sum over the cluster's blocks r of their s_part[.][tt][row] (`mine`
+// points at this block's element for tt = 0; tokens are kMaxRows apart).  All
+// NCB * kTile distributed shared-memory loads are issued before any sum is used.
+template <int NCB>
+__device__ __forceinline__ void cluster_row_sums(cooperative_groups::cluster_group& cl,
+                                                 float* mine, float (&out)[kTile]) {
+#pragma unroll
+    for (int tt = 0; tt < kTile; ++tt) out[tt] = 0.0f;
+#pragma unroll
+    for (int r = 0; r < NCB; ++r) {
+        const float* part = cl.map_shared_rank(mine, r);
+#pragma unroll
+        for (int tt = 0; tt < kTile; ++tt) out[tt] += part[tt * kMaxRows];
+    }
+}
+
 template <typename T, int DV>
 __global__ void __launch_bounds__(128) simt_bwd_fsweep(BwdParams p, float* qdq, float* fin,
                                                        const int* only) {
-    const int bh = blockIdx.x;
+    constexpr int NCB = DV / kCB;
+    namespace cg = cooperative_groups;
+    cg::cluster_group cl = cg::this_cluster();
+    const int rank = (int)cl.block_rank(), bh = blockIdx.x / NCB;
     if (only && only[bh] == 0) return;  // head already handled by the tensor-core path
-    const int T_ = p.T, dk = p.dk;
+    const int T_ = p.T, dk = p.dk, c0 = rank * kCB;
     const bool act = (int)threadIdx.x < dk;  // block padded to whole warps
     const int i = act ? threadIdx.x : 0;      // row of the state owned by this thread
-    __shared__ float s_vh[kTile][DV], s_do[kTile][DV];
+    const bool own = act && i / owner_rows<DV>(dk) == rank;  // this block finishes row i
+    __shared__ float s_vh[kTile][kCB], s_do[kTile][kCB], s_part[2][kTile][kMaxRows], s_fin[kMaxRows];
 
     const T* q = static_cast<const T*>(p.q) + (size_t)bh * T_ * dk;
     const T* k = static_cast<const T*>(p.k) + (size_t)bh * T_ * dk;
     const T* g = static_cast<const T*>(p.g) + (size_t)bh * T_ * dk;
     const T* tau = static_cast<const T*>(p.tau) + (size_t)bh * T_ * dk;
-    const T* v = static_cast<const T*>(p.v) + (size_t)bh * T_ * DV;
-    const T* beta = static_cast<const T*>(p.beta) + (size_t)bh * T_ * DV;
-    const T* dO = static_cast<const T*>(p.dO) + (size_t)bh * T_ * DV;
+    const T* v = static_cast<const T*>(p.v) + (size_t)bh * T_ * DV + c0;
+    const T* beta = static_cast<const T*>(p.beta) + (size_t)bh * T_ * DV + c0;
+    const T* dO = static_cast<const T*>(p.dO) + (size_t)bh * T_ * DV + c0;
     T* dq = static_cast<T*>(p.dq) + (size_t)bh * T_ * dk;
     float* qdq_bh = qdq + (size_t)bh * T_ * dk;
 
-    float s[DV];
+    float s[kCB];
 #pragma unroll
-    for (int j = 0; j < DV; ++j) s[j] = p.S0 ? p.S0[((size_t)bh * dk + i) * DV + j] : 0.0f;
+    for (int j = 0; j < kCB; ++j)
+        s[j] = (act && p.S0) ? p.S0[((size_t)bh * dk + i) * DV + c0 + j] : 0.0f;
 
-    for (int t0 = 0; t0 < T_; t0 += kTile) {
+    int buf = 0;
+    for (int t0 = 0; t0 < T_; t0 += kTile, buf ^= 1) {
         const int nt = min(kTile, T_ - t0);
-        for (int idx = threadIdx.x; idx < nt * DV; idx += blockDim.x) {
-            const int tt = idx / DV, j = idx % DV;
+        // tokens past the end of a partial tile are staged as zeros
+        for (int idx = threadIdx.x; idx < kTile * kCB; idx += blockDim.x) {
+            const int tt = idx / kCB, j = idx % kCB;
             const size_t off = (size_t)(t0 + tt) * DV + j;
-            const float bb = ldf(beta + off);
-            s_vh[tt][j] = (p.preact ? sigmoid_acc(bb) : bb) * ldf(v + off);
-            s_do[tt][j] = ldf(dO + off);
+            float vh = 0.0f, d_o = 0.0f;
+            if (tt < nt) {
+                const float bb = ldf(beta + off);
+                vh = (p.preact ? sigmoid_acc(bb) : bb) * ldf(v + off);
+                d_o = ldf(dO + off);
+            }
+            s_vh[tt][j] = vh;
+            s_do[tt][j] = d_o;
+        }
+        // this row's gates, key and query for the whole tile, loaded at once (the
+        // loads of a tile overlap instead of one latency per token)
+        float rg[kTile], rt[kTile], rk[kTile], rq[kTile];
+#pragma unroll
+        for (int tt = 0; tt < kTile; ++tt) {
+            const size_t off = (size_t)(t0 + (tt < nt ? tt : 0)) * dk + i;
+            rg[tt] = ldf(g + off);
+            rt[tt] = ldf(tau + off);
+            rk[tt] = ldf(k + off);
+            rq[tt] = ldf(q + off);
+        }
+        if (p.preact) {
+#pragma unroll
+            for (int tt = 0; tt < kTile; ++tt) {
+                rg[tt] = softplus_acc(rg[tt]);
+                rt[tt] = sigmoid_acc(rt[tt]);
+            }
         }
         __syncthreads();
-        for (int tt = 0; tt < nt; ++tt) {
-            const size_t off = (size_t)(t0 + tt) * dk + i;
-            float gg = ldf(g + off), ta = ldf(tau + off);
-            if (p.preact) {
-                gg = softplus_acc(gg);
-                ta = sigmoid_acc(ta);
-            }
-            const float al = alpha(gg, ta), kh = alpha_hat(gg, ta) * ldf(k + off);
-            float acc = 0.0f;
+        // the tile's tokens as one straight run (a token past the end of a partial
+        // tile leaves the state as it is: alpha 1, khat 0), so the compiler can
+        // overlap the gate arithmetic of one token with the updates of another
 #pragma unroll
-            for (int j = 0; j < DV; ++j) {
+        for (int tt = 0; tt < kTile; ++tt) {
+            const bool live = tt < nt;
+            const float gg = rg[tt], ta = rt[tt];
+            const float al = live ? alpha(gg, ta) : 1.0f;
+            const float kh = live ? alpha_hat(gg, ta) * rk[tt] : 0.0f;
+            float a0 = 0.0f, a1 = 0.0f;
+#pragma unroll
+            for (int j = 0; j < kCB; j += 2) {
                 s[j] = fmaf(al, s[j], kh * s_vh[tt][j]);
-                acc = fmaf(s[j], s_do[tt][j], acc);
+                s[j + 1] = fmaf(al, s[j + 1], kh * s_vh[tt][j + 1]);
+                a0 = fmaf(s[j], s_do[tt][j], a0);
+                a1 = fmaf(s[j + 1], s_do[tt][j + 1], a1);
             }
-            if (act) {
-                stf(dq + off, acc);
-                qdq_bh[off] = ldf(q + off) * acc;
+            if (act) s_part[buf][tt][i] = a0 + a1;
+        }
+        // the partials of this tile are complete in every block of the cluster (the
+        // barrier also orders this block's staging buffers before the next tile);
+        // s_part alternates by tile, so the next tile's partial sums go to the
+        // other buffer while the owners still read this one
+        cl.sync();
+        if (own) {
+            // every block's partials of the tile, all read before the first store
+            float dqv[kTile];
+            cluster_row_sums<NCB>(cl, &s_part[buf][0][i], dqv);
+#pragma unroll
+            for (int tt = 0; tt < kTile; ++tt) {
+                if (tt >= nt) break;
+                const size_t off = (size_t)(t0 + tt) * dk + i;
+                stf(dq + off, dqv[tt]);
+                qdq_bh[off] = rq[tt] * dqv[tt];
             }
         }
-        __syncthreads();
     }
+    // rowsum(dS_T o S_T), the decay gradient's term at u = T
     float f = 0.0f;
-    if (p.dST) {
+    if (act && p.dST) {
 #pragma unroll
-        for (int j = 0; j < DV; ++j) f = fmaf(p.dST[((size_t)bh * dk + i) * DV + j], s[j], f);
+        for (int j = 0; j < kCB; ++j) f = fmaf(p.dST[((size_t)bh * dk + i) * DV + c0 + j], s[j], f);
     }
-    if (act) fin[(size_t)bh * dk + i] = f;
+    if (act) s_fin[i] = f;
+    cl.sync();
+    if (own) {
+        float acc = 0.0f;
+#pragma unroll
+        for (int r = 0; r < NCB; ++r) acc += *cl.map_shared_rank(&s_fin[i], r);
+        fin[(size_t)bh * dk + i] = acc;
+    }
+    cl.sync();  // no block leaves while another still reads its shared memory
 }
 
 // ------------------------------------------------ backward, reverse sweep R
 template <typename T, int DV>
 __global__ void __launch_bounds__(128) simt_bwd_rsweep(BwdParams p, const float* qdq,
                                                        const float* fin, const int* only) {
-    const int bh = blockIdx.x;
+    constexpr int NCB = DV / kCB;
+    static_assert(kCB == 16, "the column reduce-scatter below takes four halving rounds");
+    namespace cg = cooperative_groups;
+    cg::cluster_group cl = cg::this_cluster();
+    const int rank = (int)cl.block_rank(), bh = blockIdx.x / NCB;
     if (only && only[bh] == 0) return;
-    const int T_ = p.T, dk = p.dk;
+    const int T_ = p.T, dk = p.dk, c0 = rank * kCB;
     // the block is padded to whole warps; rows past d_k carry zeros
     const bool act = (int)threadIdx.x < dk;
     const int i = act ? threadIdx.x : 0;
+    const bool own = act && i / owner_rows<DV>(dk) == rank;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x / 32;
-    __shared__ float s_vh[kTile][DV], s_do[kTile][DV], s_red[4][DV];
+    __shared__ float s_vh[kTile][kCB], s_do[kTile][kCB], s_b[kTile][kCB], s_v[kTile][kCB];
+    __shared__ float s_part[2][kTile][kMaxRows], s_red[kTile][4][kCB];
 
     const T* q = static_cast<const T*>(p.q) + (size_t)bh * T_ * dk;
     const T* k = static_cast<const T*>(p.k) + (size_t)bh * T_ * dk;
     const T* g = static_cast<const T*>(p.g) + (size_t)bh * T_ * dk;
     const T* tau = static_cast<const T*>(p.tau) + (size_t)bh * T_ * dk;
-    const T* v = static_cast<const T*>(p.v) + (size_t)bh * T_ * DV;
-    const T* beta = static_cast<const T*>(p.beta) + (size_t)bh * T_ * DV;
-    const T* dO = static_cast<const T*>(p.dO) + (size_t)bh * T_ * DV;
+    const T* v = static_cast<const T*>(p.v) + (size_t)bh * T_ * DV + c0;
+    const T* beta = static_cast<const T*>(p.beta) + (size_t)bh * T_ * DV + c0;
+    const T* dO = static_cast<const T*>(p.dO) + (size_t)bh * T_ * DV + c0;
     T* dk_ = static_cast<T*>(p.dk_) + (size_t)bh * T_ * dk;
     T* dg = static_cast<T*>(p.dg) + (size_t)bh * T_ * dk;
     T* dtau = static_cast<T*>(p.dtau) + (size_t)bh * T_ * dk;
-    T* dv_ = static_cast<T*>(p.dv_) + (size_t)bh * T_ * DV;
-    T* dbeta = static_cast<T*>(p.dbeta) + (size_t)bh * T_ * DV;
+    T* dv_ = static_cast<T*>(p.dv_) + (size_t)bh * T_ * DV + c0;
+    T* dbeta = static_cast<T*>(p.dbeta) + (size_t)bh * T_ * DV + c0;
     const float* qdq_bh = qdq + (size_t)bh * T_ * dk;
+    const float* dfeed = p.dfeed ? p.dfeed + (size_t)(bh % p.H) * DV + c0 : nullptr;
 
-    float ds[DV];
+    float ds[kCB];
 #pragma unroll
-    for (int j = 0; j < DV; ++j)
-        ds[j] = (act && p.dST) ? p.dST[((size_t)bh * dk + i) * DV + j] : 0.0f;
-    float a_next = 1.0f;                  // alpha_{t+1,i}
-    float da = fin[(size_t)bh * dk + i];  // running sum of dG over u >= t
+    for (int j = 0; j < kCB; ++j)
+        ds[j] = (act && p.dST) ? p.dST[((size_t)bh * dk + i) * DV + c0 + j] : 0.0f;
+    float a_next = 1.0f;                            // alpha_{t+1,i}
+    float da = own ? fin[(size_t)bh * dk + i] : 0.0f;  // running sum of dG over u >= t
 
-    for (int t1 = T_; t1 > 0; t1 -= kTile) {
+    int buf = 0;
+    for (int t1 = T_; t1 > 0; t1 -= kTile, buf ^= 1) {
         const int t0 = max(0, t1 - kTile), nt = t1 - t0;
-        for (int idx = threadIdx.x; idx < nt * DV; idx += blockDim.x) {
-            const int tt = idx / DV, j = idx % DV;
+        // tokens past the end of a partial tile are staged as zeros
+        for (int idx = threadIdx.x; idx < kTile * kCB; idx += blockDim.x) {
+            const int tt = idx / kCB, j = idx % kCB;
             const size_t off = (size_t)(t0 + tt) * DV + j;
-            const float bb = ldf(beta + off);
-            s_vh[tt][j] = (p.preact ? sigmoid_acc(bb) : bb) * ldf(v + off);
-            s_do[tt][j] = ldf(dO + off);
+            float bb = 0.0f, vv = 0.0f, d_o = 0.0f;
+            if (tt < nt) {
+                const float b_in = ldf(beta + off);
+                bb = p.preact ? sigmoid_acc(b_in) : b_in;
+                vv = ldf(v + off);
+                d_o = ldf(dO + off);
+            }
+            s_b[tt][j] = bb;
+            s_v[tt][j] = vv;
+            s_vh[tt][j] = bb * vv;
+            s_do[tt][j] = d_o;
+        }
+        // this row's gates, key and query for the whole tile, loaded at once; the
+        // gates are activated in place, and log2(g) and alpha_hat are kept for the
+        // owner's scan below
+        float rg[kTile], rt[kTile], rk[kTile], rq[kTile], rlg[kTile], rah[kTile];
+#pragma unroll
+        for (int tt = 0; tt < kTile; ++tt) {
+            const size_t off = (size_t)(t0 + (tt < nt ? tt : 0)) * dk + i;
+            rg[tt] = ldf(g + off);
+            rt[tt] = ldf(tau + off);
+            rk[tt] = ldf(k + off);
+            rq[tt] = ldf(q + off);
+        }
+        if (p.preact) {
+#pragma unroll
+            for (int tt = 0; tt < kTile; ++tt) {
+                rg[tt] = softplus_acc(rg[tt]);
+                rt[tt] = sigmoid_acc(rt[tt]);
+            }
         }
         __syncthreads();
-        for (int tt = nt - 1; tt >= 0; --tt) {
-            const size_t off = (size_t)(t0 + tt) * dk + i;
-            const float g_in = ldf(g + off), t_in = ldf(tau + off), kk = ldf(k + off);
-            const float gg = p.preact ? softplus_acc(g_in) : g_in;
-            const float ta = p.preact ? sigmoid_acc(t_in) : t_in;
-            // chain factors to the pre-activations: softplus' = sigmoid, sigmoid' = s (1 - s)
-            const float cg = p.preact ? sigmoid_acc(g_in) : 1.0f;
-            const float ct = p.preact ? ta * (1.0f - ta) : 1.0f;
-            const float qi = act ? ldf(q + off) : 0.0f;
-            const float al = alpha(gg, ta), ah = alpha_hat(gg, ta);
-            const float kh = act ? ah * kk : 0.0f;
-            float dkh = 0.0f;
+        // the tile's tokens as one straight run, as in sweep F (a token past the end
+        // of a partial tile leaves dS as it is: factor 1, no q dO^T term)
 #pragma unroll
-            for (int j = 0; j < DV; ++j) {
-                ds[j] = fmaf(a_next, ds[j], qi * s_do[tt][j]);
-                dkh = fmaf(ds[j], s_vh[tt][j], dkh);
-            }
-            // dvhat_j = sum_i dS_ij khat_i : warp shuffles, then across warps
+        for (int tt = kTile - 1; tt >= 0; --tt) {
+            const bool live = tt < nt;
+            const float gg = rg[tt], ta = rt[tt];
+            // alpha_hat = g^tau with 0^0 = 1 and 0^tau = 0 (log2(0) = -inf)
+            rlg[tt] = log2f(gg);
+            rah[tt] = ta == 0.0f ? 1.0f : exp2f(ta * rlg[tt]);
+            const float f = live ? a_next : 1.0f;
+            const float qi = act ? rq[tt] : 0.0f;
+            const float kh = act ? rah[tt] * rk[tt] : 0.0f;
+            float d0 = 0.0f, d1 = 0.0f;
 #pragma unroll
-            for (int j = 0; j < DV; ++j) {
-                float x = ds[j] * kh;
-                x += __shfl_xor_sync(0xffffffffu, x, 16);
-                x += __shfl_xor_sync(0xffffffffu, x, 8);
-                x += __shfl_xor_sync(0xffffffffu, x, 4);
-                x += __shfl_xor_sync(0xffffffffu, x, 2);
-                x += __shfl_xor_sync(0xffffffffu, x, 1);
-                if (lane == 0) s_red[warp][j] = x;
+            for (int j = 0; j < kCB; j += 2) {
+                ds[j] = fmaf(f, ds[j], qi * s_do[tt][j]);
+                ds[j + 1] = fmaf(f, ds[j + 1], qi * s_do[tt][j + 1]);
+                d0 = fmaf(ds[j], s_vh[tt][j], d0);
+                d1 = fmaf(ds[j + 1], s_vh[tt][j + 1], d1);
             }
-            da += qdq_bh[off] - kh * dkh;
-            const float dah = kk * dkh;
-            const float dah_dg = ta == 0.0f ? 0.0f : ta * exp2f((ta - 1.0f) * log2f(gg));
-            const float dah_dtau = ah == 0.0f ? 0.0f : ah * logf(gg);
-            if (act) {
-                stf(dk_ + off, ah * dkh);
-                stf(dg + off, cg * (-ta * da + dah_dg * dah));
-                stf(dtau + off, ct * (-gg * da + dah_dtau * dah));
+            if (act) s_part[buf][tt][i] = d0 + d1;  // this block's share of dkhat_{t,i}
+            // dvhat_j = sum_i dS_ij khat_i over this warp's rows: a reduce-scatter
+            // (each halving round sends half of the lane's partial sums to the lane
+            // `o` apart and adds the other half it receives), after which lanes
+            // 2c and 2c+1 both hold column c's sum; the warps' sums meet below
+            float x[kCB / 2];
+            const bool up0 = (lane & 16) != 0;
+            int col = up0 ? kCB / 2 : 0;
+#pragma unroll
+            for (int j = 0; j < kCB / 2; ++j) {
+                const float lo = ds[j] * kh, hi = ds[j + kCB / 2] * kh;
+                x[j] = (up0 ? hi : lo) + __shfl_xor_sync(0xffffffffu, up0 ? lo : hi, 16);
             }
-            a_next = al;
-            __syncthreads();
-            for (int j = threadIdx.x; j < DV; j += blockDim.x) {
-                float dvh = 0.0f;
-                for (int w = 0; w < nwarps; ++w) dvh += s_red[w][j];
-                const size_t ov = (size_t)(t0 + tt) * DV + j;
-                const float b_in = ldf(beta + ov);
-                const float bb = p.preact ? sigmoid_acc(b_in) : b_in;
-                const float df = p.dfeed ? p.dfeed[(size_t)(bh % p.H) * DV + j] * ldf(dO + ov) : 0.0f;
-                stf(dv_ + ov, fmaf(bb, dvh, df));
-                stf(dbeta + ov, (p.preact ? bb * (1.0f - bb) : 1.0f) * ldf(v + ov) * dvh);
+#pragma unroll
+            for (int r = 1; r < 4; ++r) {
+                const int o = 16 >> r, h = (kCB >> r) / 2;
+                const bool up = (lane & o) != 0;
+#pragma unroll
+                for (int j = 0; j < h; ++j) {
+                    const float send = up ? x[j] : x[j + h];
+                    const float keep = up ? x[j + h] : x[j];
+                    x[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+                }
+                if (up) col += h;
             }
-            __syncthreads();
+            x[0] += __shfl_xor_sync(0xffffffffu, x[0], 1);
+            if ((lane & 1) == 0) s_red[tt][warp][col] = x[0];
+            if (live) a_next = alpha(gg, ta);
         }
+        // every block's dkhat partials and this block's dvhat partials of the tile
+        // are complete (s_part alternates by tile, as in sweep F)
+        cl.sync();
+        for (int idx = threadIdx.x; idx < nt * kCB; idx += blockDim.x) {
+            const int tt = idx / kCB, j = idx % kCB;
+            float dvh = 0.0f;
+            for (int w = 0; w < nwarps; ++w) dvh += s_red[tt][w][j];
+            const size_t ov = (size_t)(t0 + tt) * DV + j;
+            const float bb = s_b[tt][j];
+            const float df = dfeed ? dfeed[j] * s_do[tt][j] : 0.0f;
+            stf(dv_ + ov, fmaf(bb, dvh, df));
+            stf(dbeta + ov, (p.preact ? bb * (1.0f - bb) : 1.0f) * s_v[tt][j] * dvh);
+        }
+        if (own) {
+            // the owner's reverse scan of the decay gradient over the tile
+            float rqd[kTile], dkv[kTile];
+#pragma unroll
+            for (int tt = 0; tt < kTile; ++tt)
+                rqd[tt] = qdq_bh[(size_t)(t0 + (tt < nt ? tt : 0)) * dk + i];
+            cluster_row_sums<NCB>(cl, &s_part[buf][0][i], dkv);
+#pragma unroll
+            for (int tt = kTile - 1; tt >= 0; --tt) {
+                const bool live = tt < nt;
+                const float dkh = dkv[tt], gg = rg[tt], ta = rt[tt], kk = rk[tt];
+                const float ah = rah[tt], lg = rlg[tt];
+                // chain factors to the pre-activations: softplus' = sigmoid, which is
+                // 1 - e^-g of the activated g; sigmoid' = s (1 - s)
+                const float cg_ = p.preact ? -expm1f(-gg) : 1.0f;
+                const float ct = p.preact ? ta * (1.0f - ta) : 1.0f;
+                if (live) da += rqd[tt] - ah * kk * dkh;
+                const float dah = kk * dkh;
+                // d alpha_hat / d g = tau g^(tau - 1), which is tau alpha_hat / g while
+                // alpha_hat is a normal number (then g > 0); d alpha_hat / d tau =
+                // alpha_hat ln g
+                const float dah_dg = ta == 0.0f ? 0.0f
+                                     : ah >= 1.17549435e-38f ? ta * ah / gg
+                                                              : ta * exp2f((ta - 1.0f) * lg);
+                const float dah_dtau = ah == 0.0f ? 0.0f : ah * (lg * kLn2);
+                if (live) {
+                    const size_t off = (size_t)(t0 + tt) * dk + i;
+                    stf(dk_ + off, ah * dkh);
+                    stf(dg + off, cg_ * (-ta * da + dah_dg * dah));
+                    stf(dtau + off, ct * (-gg * da + dah_dtau * dah));
+                }
+            }
+        }
+        __syncthreads();  // the staging buffers and s_red are free for the next tile
     }
     if (act && p.dS0) {
 #pragma unroll
-        for (int j = 0; j < DV; ++j) p.dS0[((size_t)bh * dk + i) * DV + j] = a_next * ds[j];
+        for (int j = 0; j < kCB; ++j) p.dS0[((size_t)bh * dk + i) * DV + c0 + j] = a_next * ds[j];
     }
+    cl.sync();  // no block leaves while another still reads its shared memory
 }
 
 template <typename T>
@@ -269,12 +441,24 @@ cudaError_t fwd_t(const SeqParams& p, cudaStream_t s) {
 
 template <typename T, int DV>
 cudaError_t bwd_tv(const BwdParams& p, float* qdq, float* fin, const int* only, cudaStream_t s) {
-    const int grid = p.B * p.H, block = (p.dk + 31) / 32 * 32;
-    simt_bwd_fsweep<T, DV><<<grid, block, 0, s>>>(p, qdq, fin, only);
-    cudaError_t e = cudaGetLastError();
+    // one cluster of DV / kCB blocks per (b,h)
+    constexpr int NCB = DV / kCB;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(p.B * p.H * NCB));
+    cfg.blockDim = dim3((unsigned)((p.dk + 31) / 32 * 32));
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = NCB;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, simt_bwd_fsweep<T, DV>, p, qdq, fin, only);
     if (e != cudaSuccess) return e;
-    simt_bwd_rsweep<T, DV><<<grid, block, 0, s>>>(p, qdq, fin, only);
-    return cudaGetLastError();
+    return cudaLaunchKernelEx(&cfg, simt_bwd_rsweep<T, DV>, p, static_cast<const float*>(qdq),
+                              static_cast<const float*>(fin), only);
 }
 
 template <typename T>
