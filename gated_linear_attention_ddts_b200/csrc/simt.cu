@@ -98,7 +98,8 @@ __global__ void __launch_bounds__(128) simt_fwd_kernel(SeqParams p) {
 // here, dkhat_t in sweep R) need the whole cluster; each block writes its
 // partial sums of a tile of tokens into its shared memory, and after one cluster
 // barrier per tile the block that owns a row adds the partials of every block
-// through distributed shared memory.
+// through distributed shared memory.  The inputs of a tile are fetched one tile
+// ahead with asynchronous copies, so their latency overlaps the tile before.
 constexpr int kCB = 16;      // state columns per block
 constexpr int kMaxRows = 128;
 
@@ -124,6 +125,95 @@ __device__ __forceinline__ void cluster_row_sums(cooperative_groups::cluster_gro
     }
 }
 
+// 16-byte global -> shared copies that complete asynchronously (cp.async), in
+// per-thread commit groups
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+    const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;\n" ::: "memory");
+}
+// waits until at most the newest of this thread's groups is still in flight
+__device__ __forceinline__ void cp_async_wait_prev() {
+    asm volatile("cp.async.wait_group 1;\n" ::: "memory");
+}
+
+// One stage of the tile pipeline in dynamic shared memory, inputs as stored:
+// the rows [kTile][dk] of g, tau, k, q, in sweep R the rows of q*dq (float32),
+// then the block's columns [kTile][kCB] of beta, v, dO.  Every part is a
+// multiple of 16 bytes (dk >= 16).
+template <typename T>
+struct SweepStage {
+    T* row[4];
+    float* qdq;
+    T* col[3];
+};
+
+template <typename T>
+__host__ __device__ __forceinline__ size_t sweep_stage_bytes(int dk, bool with_qdq) {
+    return (size_t)4 * kTile * dk * sizeof(T) + (with_qdq ? (size_t)kTile * dk * 4 : 0) +
+           (size_t)3 * kTile * kCB * sizeof(T);
+}
+
+template <typename T>
+__device__ __forceinline__ SweepStage<T> sweep_stage(unsigned char* base, int dk, bool with_qdq) {
+    SweepStage<T> s;
+    const size_t rb = (size_t)kTile * dk * sizeof(T), cb = (size_t)kTile * kCB * sizeof(T);
+#pragma unroll
+    for (int a = 0; a < 4; ++a) s.row[a] = reinterpret_cast<T*>(base + a * rb);
+    unsigned char* p = base + 4 * rb;
+    s.qdq = with_qdq ? reinterpret_cast<float*>(p) : nullptr;
+    if (with_qdq) p += (size_t)kTile * dk * 4;
+#pragma unroll
+    for (int a = 0; a < 3; ++a) s.col[a] = reinterpret_cast<T*>(p + a * cb);
+    return s;
+}
+
+// Starts the copies of tokens [t0, t0 + nt) into stage `st` (the rows of a tile
+// are contiguous in [T][dk]; the block's kCB columns of a token are kCB * size
+// bytes of [T][DV]) and closes one commit group; the rest of a partial tile is
+// zero-filled with plain stores.  All addresses are 16-byte aligned: the
+// pointers are, and every offset is a multiple of 16 * dk, DV or kCB elements.
+template <typename T, int DV>
+__device__ __forceinline__ void sweep_fetch(const SweepStage<T>& st, const T* const (&rows)[4],
+                                            const float* qdq_bh, const T* const (&cols)[3], int t0,
+                                            int nt, int dk) {
+    const size_t roff = (size_t)t0 * dk;
+    const int rchunks = nt * dk * (int)sizeof(T) / 16;
+    for (int c = threadIdx.x; c < rchunks; c += blockDim.x) {
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+            cp_async16(reinterpret_cast<char*>(st.row[a]) + c * 16,
+                       reinterpret_cast<const char*>(rows[a] + roff) + c * 16);
+    }
+    if (st.qdq) {
+        for (int c = threadIdx.x; c < nt * dk / 4; c += blockDim.x)
+            cp_async16(st.qdq + c * 4, qdq_bh + roff + c * 4);
+    }
+    constexpr int cpt = kCB * (int)sizeof(T) / 16;  // 16-byte pieces of one token's columns
+    for (int c = threadIdx.x; c < nt * cpt; c += blockDim.x) {
+        const int tt = c / cpt, part = c % cpt;
+        const size_t off = (size_t)(t0 + tt) * DV;
+#pragma unroll
+        for (int a = 0; a < 3; ++a)
+            cp_async16(reinterpret_cast<char*>(st.col[a] + tt * kCB) + part * 16,
+                       reinterpret_cast<const char*>(cols[a] + off) + part * 16);
+    }
+    cp_async_commit();
+    if (nt < kTile) {
+        for (int e = nt * dk + threadIdx.x; e < kTile * dk; e += blockDim.x) {
+#pragma unroll
+            for (int a = 0; a < 4; ++a) stf(st.row[a] + e, 0.0f);
+            if (st.qdq) st.qdq[e] = 0.0f;
+        }
+        for (int e = nt * kCB + threadIdx.x; e < kTile * kCB; e += blockDim.x) {
+#pragma unroll
+            for (int a = 0; a < 3; ++a) stf(st.col[a] + e, 0.0f);
+        }
+    }
+}
+
 template <typename T, int DV>
 __global__ void __launch_bounds__(128) simt_bwd_fsweep(BwdParams p, float* qdq, float* fin,
                                                        const int* only) {
@@ -137,48 +227,49 @@ __global__ void __launch_bounds__(128) simt_bwd_fsweep(BwdParams p, float* qdq, 
     const int i = act ? threadIdx.x : 0;      // row of the state owned by this thread
     const bool own = act && i / owner_rows<DV>(dk) == rank;  // this block finishes row i
     __shared__ float s_vh[kTile][kCB], s_do[kTile][kCB], s_part[2][kTile][kMaxRows], s_fin[kMaxRows];
+    extern __shared__ __align__(16) unsigned char s_stage[];
 
-    const T* q = static_cast<const T*>(p.q) + (size_t)bh * T_ * dk;
-    const T* k = static_cast<const T*>(p.k) + (size_t)bh * T_ * dk;
-    const T* g = static_cast<const T*>(p.g) + (size_t)bh * T_ * dk;
-    const T* tau = static_cast<const T*>(p.tau) + (size_t)bh * T_ * dk;
-    const T* v = static_cast<const T*>(p.v) + (size_t)bh * T_ * DV + c0;
-    const T* beta = static_cast<const T*>(p.beta) + (size_t)bh * T_ * DV + c0;
-    const T* dO = static_cast<const T*>(p.dO) + (size_t)bh * T_ * DV + c0;
-    T* dq = static_cast<T*>(p.dq) + (size_t)bh * T_ * dk;
-    float* qdq_bh = qdq + (size_t)bh * T_ * dk;
+    const size_t rbase = (size_t)bh * T_ * dk, cbase = (size_t)bh * T_ * DV + c0;
+    const T* const rows[4] = {static_cast<const T*>(p.g) + rbase, static_cast<const T*>(p.tau) + rbase,
+                              static_cast<const T*>(p.k) + rbase, static_cast<const T*>(p.q) + rbase};
+    const T* const cols[3] = {static_cast<const T*>(p.beta) + cbase, static_cast<const T*>(p.v) + cbase,
+                              static_cast<const T*>(p.dO) + cbase};
+    T* dq = static_cast<T*>(p.dq) + rbase;
+    float* qdq_bh = qdq + rbase;
+    const size_t sbytes = sweep_stage_bytes<T>(dk, false);
 
     float s[kCB];
 #pragma unroll
     for (int j = 0; j < kCB; ++j)
         s[j] = (act && p.S0) ? p.S0[((size_t)bh * dk + i) * DV + c0 + j] : 0.0f;
 
-    int buf = 0;
-    for (int t0 = 0; t0 < T_; t0 += kTile, buf ^= 1) {
-        const int nt = min(kTile, T_ - t0);
-        // tokens past the end of a partial tile are staged as zeros
+    const int ntiles = (T_ + kTile - 1) / kTile;
+    if (ntiles > 0)
+        sweep_fetch<T, DV>(sweep_stage<T>(s_stage, dk, false), rows, nullptr, cols, 0, min(kTile, T_), dk);
+    for (int n = 0; n < ntiles; ++n) {
+        const int t0 = n * kTile, nt = min(kTile, T_ - t0), buf = n & 1;
+        const SweepStage<T> cur = sweep_stage<T>(s_stage + buf * sbytes, dk, false);
+        if (n + 1 < ntiles)
+            sweep_fetch<T, DV>(sweep_stage<T>(s_stage + (buf ^ 1) * sbytes, dk, false), rows, nullptr,
+                               cols, t0 + kTile,
+                               min(kTile, T_ - t0 - kTile), dk);
+        else
+            cp_async_commit();
+        cp_async_wait_prev();
+        __syncthreads();  // this tile's stage is complete and visible
         for (int idx = threadIdx.x; idx < kTile * kCB; idx += blockDim.x) {
-            const int tt = idx / kCB, j = idx % kCB;
-            const size_t off = (size_t)(t0 + tt) * DV + j;
-            float vh = 0.0f, d_o = 0.0f;
-            if (tt < nt) {
-                const float bb = ldf(beta + off);
-                vh = (p.preact ? sigmoid_acc(bb) : bb) * ldf(v + off);
-                d_o = ldf(dO + off);
-            }
-            s_vh[tt][j] = vh;
-            s_do[tt][j] = d_o;
+            const float bb = ldf(cur.col[0] + idx);
+            s_vh[idx / kCB][idx % kCB] = (p.preact ? sigmoid_acc(bb) : bb) * ldf(cur.col[1] + idx);
+            s_do[idx / kCB][idx % kCB] = ldf(cur.col[2] + idx);
         }
-        // this row's gates, key and query for the whole tile, loaded at once (the
-        // loads of a tile overlap instead of one latency per token)
+        // this row's gates, key and query for the whole tile (zeros past the end)
         float rg[kTile], rt[kTile], rk[kTile], rq[kTile];
 #pragma unroll
         for (int tt = 0; tt < kTile; ++tt) {
-            const size_t off = (size_t)(t0 + (tt < nt ? tt : 0)) * dk + i;
-            rg[tt] = ldf(g + off);
-            rt[tt] = ldf(tau + off);
-            rk[tt] = ldf(k + off);
-            rq[tt] = ldf(q + off);
+            rg[tt] = ldf(cur.row[0] + tt * dk + i);
+            rt[tt] = ldf(cur.row[1] + tt * dk + i);
+            rk[tt] = ldf(cur.row[2] + tt * dk + i);
+            rq[tt] = ldf(cur.row[3] + tt * dk + i);
         }
         if (p.preact) {
 #pragma unroll
@@ -260,21 +351,21 @@ __global__ void __launch_bounds__(128) simt_bwd_rsweep(BwdParams p, const float*
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x / 32;
     __shared__ float s_vh[kTile][kCB], s_do[kTile][kCB], s_b[kTile][kCB], s_v[kTile][kCB];
     __shared__ float s_part[2][kTile][kMaxRows], s_red[kTile][4][kCB];
+    extern __shared__ __align__(16) unsigned char s_stage[];
 
-    const T* q = static_cast<const T*>(p.q) + (size_t)bh * T_ * dk;
-    const T* k = static_cast<const T*>(p.k) + (size_t)bh * T_ * dk;
-    const T* g = static_cast<const T*>(p.g) + (size_t)bh * T_ * dk;
-    const T* tau = static_cast<const T*>(p.tau) + (size_t)bh * T_ * dk;
-    const T* v = static_cast<const T*>(p.v) + (size_t)bh * T_ * DV + c0;
-    const T* beta = static_cast<const T*>(p.beta) + (size_t)bh * T_ * DV + c0;
-    const T* dO = static_cast<const T*>(p.dO) + (size_t)bh * T_ * DV + c0;
-    T* dk_ = static_cast<T*>(p.dk_) + (size_t)bh * T_ * dk;
-    T* dg = static_cast<T*>(p.dg) + (size_t)bh * T_ * dk;
-    T* dtau = static_cast<T*>(p.dtau) + (size_t)bh * T_ * dk;
-    T* dv_ = static_cast<T*>(p.dv_) + (size_t)bh * T_ * DV + c0;
-    T* dbeta = static_cast<T*>(p.dbeta) + (size_t)bh * T_ * DV + c0;
-    const float* qdq_bh = qdq + (size_t)bh * T_ * dk;
+    const size_t rbase = (size_t)bh * T_ * dk, cbase = (size_t)bh * T_ * DV + c0;
+    const T* const rows[4] = {static_cast<const T*>(p.g) + rbase, static_cast<const T*>(p.tau) + rbase,
+                              static_cast<const T*>(p.k) + rbase, static_cast<const T*>(p.q) + rbase};
+    const T* const cols[3] = {static_cast<const T*>(p.beta) + cbase, static_cast<const T*>(p.v) + cbase,
+                              static_cast<const T*>(p.dO) + cbase};
+    T* dk_ = static_cast<T*>(p.dk_) + rbase;
+    T* dg = static_cast<T*>(p.dg) + rbase;
+    T* dtau = static_cast<T*>(p.dtau) + rbase;
+    T* dv_ = static_cast<T*>(p.dv_) + cbase;
+    T* dbeta = static_cast<T*>(p.dbeta) + cbase;
+    const float* qdq_bh = qdq + rbase;
     const float* dfeed = p.dfeed ? p.dfeed + (size_t)(bh % p.H) * DV + c0 : nullptr;
+    const size_t sbytes = sweep_stage_bytes<T>(dk, true);
 
     float ds[kCB];
 #pragma unroll
@@ -283,36 +374,41 @@ __global__ void __launch_bounds__(128) simt_bwd_rsweep(BwdParams p, const float*
     float a_next = 1.0f;                            // alpha_{t+1,i}
     float da = own ? fin[(size_t)bh * dk + i] : 0.0f;  // running sum of dG over u >= t
 
-    int buf = 0;
-    for (int t1 = T_; t1 > 0; t1 -= kTile, buf ^= 1) {
-        const int t0 = max(0, t1 - kTile), nt = t1 - t0;
-        // tokens past the end of a partial tile are staged as zeros
+    // tile n holds tokens [t1 - kTile, t1) with t1 = T - n kTile (the last one
+    // processed may be partial)
+    const int ntiles = (T_ + kTile - 1) / kTile;
+    if (ntiles > 0)
+        sweep_fetch<T, DV>(sweep_stage<T>(s_stage, dk, true), rows, qdq_bh, cols, max(0, T_ - kTile),
+                           min(kTile, T_), dk);
+    for (int n = 0; n < ntiles; ++n) {
+        const int t1 = T_ - n * kTile, t0 = max(0, t1 - kTile), nt = t1 - t0, buf = n & 1;
+        const SweepStage<T> cur = sweep_stage<T>(s_stage + buf * sbytes, dk, true);
+        if (n + 1 < ntiles)
+            sweep_fetch<T, DV>(sweep_stage<T>(s_stage + (buf ^ 1) * sbytes, dk, true), rows, qdq_bh,
+                               cols, max(0, t0 - kTile), min(kTile, t0), dk);
+        else
+            cp_async_commit();
+        cp_async_wait_prev();
+        __syncthreads();  // this tile's stage is complete and visible
         for (int idx = threadIdx.x; idx < kTile * kCB; idx += blockDim.x) {
             const int tt = idx / kCB, j = idx % kCB;
-            const size_t off = (size_t)(t0 + tt) * DV + j;
-            float bb = 0.0f, vv = 0.0f, d_o = 0.0f;
-            if (tt < nt) {
-                const float b_in = ldf(beta + off);
-                bb = p.preact ? sigmoid_acc(b_in) : b_in;
-                vv = ldf(v + off);
-                d_o = ldf(dO + off);
-            }
+            const float b_in = ldf(cur.col[0] + idx), vv = ldf(cur.col[1] + idx);
+            const float bb = p.preact ? sigmoid_acc(b_in) : b_in;
             s_b[tt][j] = bb;
             s_v[tt][j] = vv;
             s_vh[tt][j] = bb * vv;
-            s_do[tt][j] = d_o;
+            s_do[tt][j] = ldf(cur.col[2] + idx);
         }
-        // this row's gates, key and query for the whole tile, loaded at once; the
-        // gates are activated in place, and log2(g) and alpha_hat are kept for the
-        // owner's scan below
+        // this row's gates, key and query for the whole tile (zeros past the end);
+        // the gates are activated in place, and log2(g) and alpha_hat are kept for
+        // the owner's scan below
         float rg[kTile], rt[kTile], rk[kTile], rq[kTile], rlg[kTile], rah[kTile];
 #pragma unroll
         for (int tt = 0; tt < kTile; ++tt) {
-            const size_t off = (size_t)(t0 + (tt < nt ? tt : 0)) * dk + i;
-            rg[tt] = ldf(g + off);
-            rt[tt] = ldf(tau + off);
-            rk[tt] = ldf(k + off);
-            rq[tt] = ldf(q + off);
+            rg[tt] = ldf(cur.row[0] + tt * dk + i);
+            rt[tt] = ldf(cur.row[1] + tt * dk + i);
+            rk[tt] = ldf(cur.row[2] + tt * dk + i);
+            rq[tt] = ldf(cur.row[3] + tt * dk + i);
         }
         if (p.preact) {
 #pragma unroll
@@ -388,8 +484,7 @@ __global__ void __launch_bounds__(128) simt_bwd_rsweep(BwdParams p, const float*
             // the owner's reverse scan of the decay gradient over the tile
             float rqd[kTile], dkv[kTile];
 #pragma unroll
-            for (int tt = 0; tt < kTile; ++tt)
-                rqd[tt] = qdq_bh[(size_t)(t0 + (tt < nt ? tt : 0)) * dk + i];
+            for (int tt = 0; tt < kTile; ++tt) rqd[tt] = cur.qdq[tt * dk + i];
             cluster_row_sums<NCB>(cl, &s_part[buf][0][i], dkv);
 #pragma unroll
             for (int tt = kTile - 1; tt >= 0; --tt) {
@@ -443,10 +538,18 @@ template <typename T, int DV>
 cudaError_t bwd_tv(const BwdParams& p, float* qdq, float* fin, const int* only, cudaStream_t s) {
     // one cluster of DV / kCB blocks per (b,h)
     constexpr int NCB = DV / kCB;
+    // two pipeline stages of dynamic shared memory (sweep R's carry q*dq too)
+    const size_t smf = 2 * sweep_stage_bytes<T>(p.dk, false), smr = 2 * sweep_stage_bytes<T>(p.dk, true);
+    cudaError_t e = cudaFuncSetAttribute(simt_bwd_fsweep<T, DV>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smf);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(simt_bwd_rsweep<T, DV>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smr);
+    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(p.B * p.H * NCB));
     cfg.blockDim = dim3((unsigned)((p.dk + 31) / 32 * 32));
-    cfg.dynamicSmemBytes = 0;
+    cfg.dynamicSmemBytes = smf;
     cfg.stream = s;
     cudaLaunchAttribute at[1];
     at[0].id = cudaLaunchAttributeClusterDimension;
@@ -455,8 +558,9 @@ cudaError_t bwd_tv(const BwdParams& p, float* qdq, float* fin, const int* only, 
     at[0].val.clusterDim.z = 1;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, simt_bwd_fsweep<T, DV>, p, qdq, fin, only);
+    e = cudaLaunchKernelEx(&cfg, simt_bwd_fsweep<T, DV>, p, qdq, fin, only);
     if (e != cudaSuccess) return e;
+    cfg.dynamicSmemBytes = smr;
     return cudaLaunchKernelEx(&cfg, simt_bwd_rsweep<T, DV>, p, static_cast<const float*>(qdq),
                               static_cast<const float*>(fin), only);
 }
