@@ -18,6 +18,7 @@
 // which follows from S_t = sum_s diag(exp(G_t - G_s)) khat_s vhat_s^T + diag(exp(G_t)) S_0
 // with G_t the running sum of log alpha.
 #include <cooperative_groups.h>
+#include <type_traits>
 
 #include "launch.h"
 #include "rdm_common.cuh"
@@ -123,6 +124,18 @@ __device__ __forceinline__ void cluster_row_sums(cooperative_groups::cluster_gro
 #pragma unroll
         for (int tt = 0; tt < kTile; ++tt) out[tt] += part[tt * kMaxRows];
     }
+}
+
+__host__ __device__ __forceinline__ int ntiles_of(int T) { return (T + kTile - 1) / kTile; }
+
+// the two halves of a cluster barrier: arrive (releasing this thread's earlier
+// writes, shared memory included) and wait (acquiring those of every thread
+// that arrived); every thread of every block takes both
+__device__ __forceinline__ void cluster_arrive() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+    asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
 }
 
 // 16-byte global -> shared copies that complete asynchronously (cp.async), in
@@ -243,27 +256,27 @@ __global__ void __launch_bounds__(128) simt_bwd_fsweep(BwdParams p, float* qdq, 
     for (int j = 0; j < kCB; ++j)
         s[j] = (act && p.S0) ? p.S0[((size_t)bh * dk + i) * DV + c0 + j] : 0.0f;
 
-    const int ntiles = (T_ + kTile - 1) / kTile;
-    if (ntiles > 0)
-        sweep_fetch<T, DV>(sweep_stage<T>(s_stage, dk, false), rows, nullptr, cols, 0, min(kTile, T_), dk);
-    for (int n = 0; n < ntiles; ++n) {
-        const int t0 = n * kTile, nt = min(kTile, T_ - t0), buf = n & 1;
-        const SweepStage<T> cur = sweep_stage<T>(s_stage + buf * sbytes, dk, false);
-        if (n + 1 < ntiles)
-            sweep_fetch<T, DV>(sweep_stage<T>(s_stage + (buf ^ 1) * sbytes, dk, false), rows, nullptr,
-                               cols, t0 + kTile,
-                               min(kTile, T_ - t0 - kTile), dk);
-        else
+    // Tile n: its stage was fetched while tile n - 1 ran; it is unpacked into
+    // s_vh, s_do and this row's registers before the cluster waits for the
+    // partial sums of tile n - 1, so that wait overlaps the unpacking.
+    float rg[kTile], rt[kTile], rk[kTile], rq[kTile];
+    auto fetch = [&](int m) {  // starts tile m's copies (an empty group past the end)
+        if (m < ntiles_of(T_)) {
+            const int tm = m * kTile;
+            sweep_fetch<T, DV>(sweep_stage<T>(s_stage + (m & 1) * sbytes, dk, false), rows, nullptr,
+                               cols, tm, min(kTile, T_ - tm), dk);
+        } else {
             cp_async_commit();
-        cp_async_wait_prev();
-        __syncthreads();  // this tile's stage is complete and visible
+        }
+    };
+    auto unpack = [&](int m) {  // after tile m's copies are complete and visible
+        const SweepStage<T> cur = sweep_stage<T>(s_stage + (m & 1) * sbytes, dk, false);
         for (int idx = threadIdx.x; idx < kTile * kCB; idx += blockDim.x) {
             const float bb = ldf(cur.col[0] + idx);
             s_vh[idx / kCB][idx % kCB] = (p.preact ? sigmoid_acc(bb) : bb) * ldf(cur.col[1] + idx);
             s_do[idx / kCB][idx % kCB] = ldf(cur.col[2] + idx);
         }
         // this row's gates, key and query for the whole tile (zeros past the end)
-        float rg[kTile], rt[kTile], rk[kTile], rq[kTile];
 #pragma unroll
         for (int tt = 0; tt < kTile; ++tt) {
             rg[tt] = ldf(cur.row[0] + tt * dk + i);
@@ -278,7 +291,18 @@ __global__ void __launch_bounds__(128) simt_bwd_fsweep(BwdParams p, float* qdq, 
                 rt[tt] = sigmoid_acc(rt[tt]);
             }
         }
+    };
+    const int ntiles = ntiles_of(T_);
+    if (ntiles > 0) {
+        fetch(0);
+        fetch(1);
+        cp_async_wait_prev();
         __syncthreads();
+        unpack(0);
+        __syncthreads();
+    }
+    for (int n = 0; n < ntiles; ++n) {
+        const int t0 = n * kTile, nt = min(kTile, T_ - t0), buf = n & 1;
         // the tile's tokens as one straight run (a token past the end of a partial
         // tile leaves the state as it is: alpha 1, khat 0), so the compiler can
         // overlap the gate arithmetic of one token with the updates of another
@@ -298,11 +322,21 @@ __global__ void __launch_bounds__(128) simt_bwd_fsweep(BwdParams p, float* qdq, 
             }
             if (act) s_part[buf][tt][i] = a0 + a1;
         }
-        // the partials of this tile are complete in every block of the cluster (the
-        // barrier also orders this block's staging buffers before the next tile);
-        // s_part alternates by tile, so the next tile's partial sums go to the
-        // other buffer while the owners still read this one
-        cl.sync();
+        // this block's partials of the tile are written (s_part alternates by tile:
+        // a block writes tile n + 2 into this buffer only after every block has
+        // arrived after tile n + 1, that is, after its owners read tile n)
+        cluster_arrive();
+        float rqo[kTile];
+#pragma unroll
+        for (int tt = 0; tt < kTile; ++tt) rqo[tt] = rq[tt];
+        if (n + 1 < ntiles) {
+            fetch(n + 2);  // into the stage tile n came from, unpacked before its run
+            cp_async_wait_prev();
+            __syncthreads();  // tile n + 1's stage is visible; tile n's run is over
+            unpack(n + 1);
+            __syncthreads();
+        }
+        cluster_wait();  // every block's partials of tile n are written
         if (own) {
             // every block's partials of the tile, all read before the first store
             float dqv[kTile];
@@ -312,7 +346,7 @@ __global__ void __launch_bounds__(128) simt_bwd_fsweep(BwdParams p, float* qdq, 
                 if (tt >= nt) break;
                 const size_t off = (size_t)(t0 + tt) * dk + i;
                 stf(dq + off, dqv[tt]);
-                qdq_bh[off] = rq[tt] * dqv[tt];
+                qdq_bh[off] = rqo[tt] * dqv[tt];
             }
         }
     }
@@ -467,9 +501,10 @@ __global__ void __launch_bounds__(128) simt_bwd_rsweep(BwdParams p, const float*
             if ((lane & 1) == 0) s_red[tt][warp][col] = x[0];
             if (live) a_next = alpha(gg, ta);
         }
-        // every block's dkhat partials and this block's dvhat partials of the tile
-        // are complete (s_part alternates by tile, as in sweep F)
-        cl.sync();
+        // this block's dkhat partials of the tile are written (s_part alternates by
+        // tile, as in sweep F); the dvhat outputs need only this block's partials
+        cluster_arrive();
+        __syncthreads();
         for (int idx = threadIdx.x; idx < nt * kCB; idx += blockDim.x) {
             const int tt = idx / kCB, j = idx % kCB;
             float dvh = 0.0f;
@@ -480,37 +515,46 @@ __global__ void __launch_bounds__(128) simt_bwd_rsweep(BwdParams p, const float*
             stf(dv_ + ov, fmaf(bb, dvh, df));
             stf(dbeta + ov, (p.preact ? bb * (1.0f - bb) : 1.0f) * s_v[tt][j] * dvh);
         }
+        cluster_wait();  // every block's dkhat partials of the tile are written
         if (own) {
             // the owner's reverse scan of the decay gradient over the tile
             float rqd[kTile], dkv[kTile];
 #pragma unroll
             for (int tt = 0; tt < kTile; ++tt) rqd[tt] = cur.qdq[tt * dk + i];
             cluster_row_sums<NCB>(cl, &s_part[buf][0][i], dkv);
+            // a whole tile runs without a test per token (a partial one is the last)
+            auto scan = [&](auto whole) {
+                constexpr bool kWhole = decltype(whole)::value;
 #pragma unroll
-            for (int tt = kTile - 1; tt >= 0; --tt) {
-                const bool live = tt < nt;
-                const float dkh = dkv[tt], gg = rg[tt], ta = rt[tt], kk = rk[tt];
-                const float ah = rah[tt], lg = rlg[tt];
-                // chain factors to the pre-activations: softplus' = sigmoid, which is
-                // 1 - e^-g of the activated g; sigmoid' = s (1 - s)
-                const float cg_ = p.preact ? -expm1f(-gg) : 1.0f;
-                const float ct = p.preact ? ta * (1.0f - ta) : 1.0f;
-                if (live) da += rqd[tt] - ah * kk * dkh;
-                const float dah = kk * dkh;
-                // d alpha_hat / d g = tau g^(tau - 1), which is tau alpha_hat / g while
-                // alpha_hat is a normal number (then g > 0); d alpha_hat / d tau =
-                // alpha_hat ln g
-                const float dah_dg = ta == 0.0f ? 0.0f
-                                     : ah >= 1.17549435e-38f ? ta * ah / gg
-                                                              : ta * exp2f((ta - 1.0f) * lg);
-                const float dah_dtau = ah == 0.0f ? 0.0f : ah * (lg * kLn2);
-                if (live) {
-                    const size_t off = (size_t)(t0 + tt) * dk + i;
-                    stf(dk_ + off, ah * dkh);
-                    stf(dg + off, cg_ * (-ta * da + dah_dg * dah));
-                    stf(dtau + off, ct * (-gg * da + dah_dtau * dah));
+                for (int tt = kTile - 1; tt >= 0; --tt) {
+                    const bool live = kWhole || tt < nt;
+                    const float dkh = dkv[tt], gg = rg[tt], ta = rt[tt], kk = rk[tt];
+                    const float ah = rah[tt], lg = rlg[tt];
+                    // chain factors to the pre-activations: softplus' = sigmoid, which
+                    // is 1 - e^-g of the activated g; sigmoid' = s (1 - s)
+                    const float cg_ = p.preact ? -expm1f(-gg) : 1.0f;
+                    const float ct = p.preact ? ta * (1.0f - ta) : 1.0f;
+                    if (live) da += rqd[tt] - ah * kk * dkh;
+                    const float dah = kk * dkh;
+                    // d alpha_hat / d g = tau g^(tau - 1), which is tau alpha_hat / g
+                    // while alpha_hat is a normal number (then g > 0); d alpha_hat /
+                    // d tau = alpha_hat ln g
+                    const float dah_dg = ta == 0.0f ? 0.0f
+                                         : ah >= 1.17549435e-38f ? __fdividef(ta * ah, gg)
+                                                                  : ta * exp2f((ta - 1.0f) * lg);
+                    const float dah_dtau = ah == 0.0f ? 0.0f : ah * (lg * kLn2);
+                    if (live) {
+                        const size_t off = (size_t)(t0 + tt) * dk + i;
+                        stf(dk_ + off, ah * dkh);
+                        stf(dg + off, cg_ * (-ta * da + dah_dg * dah));
+                        stf(dtau + off, ct * (-gg * da + dah_dtau * dah));
+                    }
                 }
-            }
+            };
+            if (nt == kTile)
+                scan(std::true_type{});
+            else
+                scan(std::false_type{});
         }
         __syncthreads();  // the staging buffers and s_red are free for the next tile
     }
