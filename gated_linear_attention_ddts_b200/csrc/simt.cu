@@ -8,8 +8,8 @@
 // along d_k per the paperhub.cn rebuttal "Efficient Parallelization" bullet.)
 //
 // Backward, exact reverse mode organised in two sweeps per (b,h), each run by a
-// cluster of blocks that split the state's columns, thread i owning row i of
-// its block's columns of the state or of its gradient:
+// cluster of blocks that split the state's columns, threads 2i and 2i+1 owning
+// row i of their block's columns of the state or of its gradient:
 //   sweep F (forward in t):  S_t, dq_t = S_t dO_t, and q_t*dq_t kept in scratch;
 //   sweep R (reverse in t):  dS_t = q_t dO_t^T + diag(alpha_{t+1}) dS_{t+1},
 //                            dkhat_t = dS_t vhat_t, dvhat_t = dS_t^T khat_t.
@@ -102,6 +102,7 @@ __global__ void __launch_bounds__(128) simt_fwd_kernel(SeqParams p) {
 // through distributed shared memory.  The inputs of a tile are fetched one tile
 // ahead with asynchronous copies, so their latency overlaps the tile before.
 constexpr int kCB = 16;      // state columns per block
+constexpr int kCH = kCB / 2;  // state columns per thread (two threads a row)
 constexpr int kMaxRows = 128;
 
 template <int DV>
@@ -228,7 +229,7 @@ __device__ __forceinline__ void sweep_fetch(const SweepStage<T>& st, const T* co
 }
 
 template <typename T, int DV>
-__global__ void __launch_bounds__(128) simt_bwd_fsweep(BwdParams p, float* qdq, float* fin,
+__global__ void __launch_bounds__(256) simt_bwd_fsweep(BwdParams p, float* qdq, float* fin,
                                                        const int* only) {
     constexpr int NCB = DV / kCB;
     namespace cg = cooperative_groups;
@@ -236,9 +237,11 @@ __global__ void __launch_bounds__(128) simt_bwd_fsweep(BwdParams p, float* qdq, 
     const int rank = (int)cl.block_rank(), bh = blockIdx.x / NCB;
     if (only && only[bh] == 0) return;  // head already handled by the tensor-core path
     const int T_ = p.T, dk = p.dk, c0 = rank * kCB;
-    const bool act = (int)threadIdx.x < dk;  // block padded to whole warps
-    const int i = act ? threadIdx.x : 0;      // row of the state owned by this thread
-    const bool own = act && i / owner_rows<DV>(dk) == rank;  // this block finishes row i
+    // two threads a row: thread 2i + h runs columns c0 + 8h ... c0 + 8h + 7 of row i
+    // (the block has 2 d_k threads)
+    const int i = threadIdx.x >> 1, cb = (threadIdx.x & 1) * kCH;
+    const bool act = i < dk;
+    const bool own = act && cb == 0 && i / owner_rows<DV>(dk) == rank;  // this block finishes row i
     __shared__ float s_vh[kTile][kCB], s_do[kTile][kCB], s_part[2][kTile][kMaxRows], s_fin[kMaxRows];
     extern __shared__ __align__(16) unsigned char s_stage[];
 
@@ -251,10 +254,10 @@ __global__ void __launch_bounds__(128) simt_bwd_fsweep(BwdParams p, float* qdq, 
     float* qdq_bh = qdq + rbase;
     const size_t sbytes = sweep_stage_bytes<T>(dk, false);
 
-    float s[kCB];
+    float s[kCH];
 #pragma unroll
-    for (int j = 0; j < kCB; ++j)
-        s[j] = (act && p.S0) ? p.S0[((size_t)bh * dk + i) * DV + c0 + j] : 0.0f;
+    for (int j = 0; j < kCH; ++j)
+        s[j] = (act && p.S0) ? p.S0[((size_t)bh * dk + i) * DV + c0 + cb + j] : 0.0f;
 
     // Tile n: its stage was fetched while tile n - 1 ran; it is unpacked into
     // s_vh, s_do and this row's registers before the cluster waits for the
@@ -314,13 +317,15 @@ __global__ void __launch_bounds__(128) simt_bwd_fsweep(BwdParams p, float* qdq, 
             const float kh = live ? alpha_hat(gg, ta) * rk[tt] : 0.0f;
             float a0 = 0.0f, a1 = 0.0f;
 #pragma unroll
-            for (int j = 0; j < kCB; j += 2) {
-                s[j] = fmaf(al, s[j], kh * s_vh[tt][j]);
-                s[j + 1] = fmaf(al, s[j + 1], kh * s_vh[tt][j + 1]);
-                a0 = fmaf(s[j], s_do[tt][j], a0);
-                a1 = fmaf(s[j + 1], s_do[tt][j + 1], a1);
+            for (int j = 0; j < kCH; j += 2) {
+                s[j] = fmaf(al, s[j], kh * s_vh[tt][cb + j]);
+                s[j + 1] = fmaf(al, s[j + 1], kh * s_vh[tt][cb + j + 1]);
+                a0 = fmaf(s[j], s_do[tt][cb + j], a0);
+                a1 = fmaf(s[j + 1], s_do[tt][cb + j + 1], a1);
             }
-            if (act) s_part[buf][tt][i] = a0 + a1;
+            float a = a0 + a1;
+            a += __shfl_xor_sync(0xffffffffu, a, 1);  // the row's other half
+            if (act && cb == 0) s_part[buf][tt][i] = a;
         }
         // this block's partials of the tile are written (s_part alternates by tile:
         // a block writes tile n + 2 into this buffer only after every block has
@@ -354,9 +359,11 @@ __global__ void __launch_bounds__(128) simt_bwd_fsweep(BwdParams p, float* qdq, 
     float f = 0.0f;
     if (act && p.dST) {
 #pragma unroll
-        for (int j = 0; j < kCB; ++j) f = fmaf(p.dST[((size_t)bh * dk + i) * DV + c0 + j], s[j], f);
+        for (int j = 0; j < kCH; ++j)
+            f = fmaf(p.dST[((size_t)bh * dk + i) * DV + c0 + cb + j], s[j], f);
     }
-    if (act) s_fin[i] = f;
+    f += __shfl_xor_sync(0xffffffffu, f, 1);
+    if (act && cb == 0) s_fin[i] = f;
     cl.sync();
     if (own) {
         float acc = 0.0f;
@@ -369,22 +376,22 @@ __global__ void __launch_bounds__(128) simt_bwd_fsweep(BwdParams p, float* qdq, 
 
 // ------------------------------------------------ backward, reverse sweep R
 template <typename T, int DV>
-__global__ void __launch_bounds__(128) simt_bwd_rsweep(BwdParams p, const float* qdq,
+__global__ void __launch_bounds__(256) simt_bwd_rsweep(BwdParams p, const float* qdq,
                                                        const float* fin, const int* only) {
     constexpr int NCB = DV / kCB;
-    static_assert(kCB == 16, "the column reduce-scatter below takes four halving rounds");
+    static_assert(kCH == 8, "the column reduce-scatter below takes three halving rounds");
     namespace cg = cooperative_groups;
     cg::cluster_group cl = cg::this_cluster();
     const int rank = (int)cl.block_rank(), bh = blockIdx.x / NCB;
     if (only && only[bh] == 0) return;
     const int T_ = p.T, dk = p.dk, c0 = rank * kCB;
-    // the block is padded to whole warps; rows past d_k carry zeros
-    const bool act = (int)threadIdx.x < dk;
-    const int i = act ? threadIdx.x : 0;
-    const bool own = act && i / owner_rows<DV>(dk) == rank;
+    // two threads a row, as in sweep F
+    const int i = threadIdx.x >> 1, cb = (threadIdx.x & 1) * kCH;
+    const bool act = i < dk;
+    const bool own = act && cb == 0 && i / owner_rows<DV>(dk) == rank;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x / 32;
     __shared__ float s_vh[kTile][kCB], s_do[kTile][kCB], s_b[kTile][kCB], s_v[kTile][kCB];
-    __shared__ float s_part[2][kTile][kMaxRows], s_red[kTile][4][kCB];
+    __shared__ float s_part[2][kTile][kMaxRows], s_red[kTile][8][kCB];
     extern __shared__ __align__(16) unsigned char s_stage[];
 
     const size_t rbase = (size_t)bh * T_ * dk, cbase = (size_t)bh * T_ * DV + c0;
@@ -401,10 +408,10 @@ __global__ void __launch_bounds__(128) simt_bwd_rsweep(BwdParams p, const float*
     const float* dfeed = p.dfeed ? p.dfeed + (size_t)(bh % p.H) * DV + c0 : nullptr;
     const size_t sbytes = sweep_stage_bytes<T>(dk, true);
 
-    float ds[kCB];
+    float ds[kCH];
 #pragma unroll
-    for (int j = 0; j < kCB; ++j)
-        ds[j] = (act && p.dST) ? p.dST[((size_t)bh * dk + i) * DV + c0 + j] : 0.0f;
+    for (int j = 0; j < kCH; ++j)
+        ds[j] = (act && p.dST) ? p.dST[((size_t)bh * dk + i) * DV + c0 + cb + j] : 0.0f;
     float a_next = 1.0f;                            // alpha_{t+1,i}
     float da = own ? fin[(size_t)bh * dk + i] : 0.0f;  // running sum of dG over u >= t
 
@@ -466,28 +473,31 @@ __global__ void __launch_bounds__(128) simt_bwd_rsweep(BwdParams p, const float*
             const float kh = act ? rah[tt] * rk[tt] : 0.0f;
             float d0 = 0.0f, d1 = 0.0f;
 #pragma unroll
-            for (int j = 0; j < kCB; j += 2) {
-                ds[j] = fmaf(f, ds[j], qi * s_do[tt][j]);
-                ds[j + 1] = fmaf(f, ds[j + 1], qi * s_do[tt][j + 1]);
-                d0 = fmaf(ds[j], s_vh[tt][j], d0);
-                d1 = fmaf(ds[j + 1], s_vh[tt][j + 1], d1);
+            for (int j = 0; j < kCH; j += 2) {
+                ds[j] = fmaf(f, ds[j], qi * s_do[tt][cb + j]);
+                ds[j + 1] = fmaf(f, ds[j + 1], qi * s_do[tt][cb + j + 1]);
+                d0 = fmaf(ds[j], s_vh[tt][cb + j], d0);
+                d1 = fmaf(ds[j + 1], s_vh[tt][cb + j + 1], d1);
             }
-            if (act) s_part[buf][tt][i] = d0 + d1;  // this block's share of dkhat_{t,i}
-            // dvhat_j = sum_i dS_ij khat_i over this warp's rows: a reduce-scatter
-            // (each halving round sends half of the lane's partial sums to the lane
-            // `o` apart and adds the other half it receives), after which lanes
-            // 2c and 2c+1 both hold column c's sum; the warps' sums meet below
-            float x[kCB / 2];
+            float d = d0 + d1;
+            d += __shfl_xor_sync(0xffffffffu, d, 1);  // the row's other half
+            if (act && cb == 0) s_part[buf][tt][i] = d;  // this block's share of dkhat_{t,i}
+            // dvhat_j = sum_i dS_ij khat_i over the warp's 16 rows (lanes of one
+            // parity): a reduce-scatter over lane bits 4, 3, 2 (each halving round
+            // sends half of the lane's partial sums to the lane `o` apart and adds
+            // the other half it receives), then a plain sum over bit 1, after which
+            // lanes l and l ^ 2 both hold column cb + col; the warps meet below
+            float x[kCH / 2];
             const bool up0 = (lane & 16) != 0;
-            int col = up0 ? kCB / 2 : 0;
+            int col = up0 ? kCH / 2 : 0;
 #pragma unroll
-            for (int j = 0; j < kCB / 2; ++j) {
-                const float lo = ds[j] * kh, hi = ds[j + kCB / 2] * kh;
+            for (int j = 0; j < kCH / 2; ++j) {
+                const float lo = ds[j] * kh, hi = ds[j + kCH / 2] * kh;
                 x[j] = (up0 ? hi : lo) + __shfl_xor_sync(0xffffffffu, up0 ? lo : hi, 16);
             }
 #pragma unroll
-            for (int r = 1; r < 4; ++r) {
-                const int o = 16 >> r, h = (kCB >> r) / 2;
+            for (int r = 1; r < 3; ++r) {
+                const int o = 16 >> r, h = (kCH >> r) / 2;
                 const bool up = (lane & o) != 0;
 #pragma unroll
                 for (int j = 0; j < h; ++j) {
@@ -497,8 +507,8 @@ __global__ void __launch_bounds__(128) simt_bwd_rsweep(BwdParams p, const float*
                 }
                 if (up) col += h;
             }
-            x[0] += __shfl_xor_sync(0xffffffffu, x[0], 1);
-            if ((lane & 1) == 0) s_red[tt][warp][col] = x[0];
+            x[0] += __shfl_xor_sync(0xffffffffu, x[0], 2);
+            if ((lane & 2) == 0) s_red[tt][warp][cb + col] = x[0];
             if (live) a_next = alpha(gg, ta);
         }
         // this block's dkhat partials of the tile are written (s_part alternates by
@@ -560,7 +570,7 @@ __global__ void __launch_bounds__(128) simt_bwd_rsweep(BwdParams p, const float*
     }
     if (act && p.dS0) {
 #pragma unroll
-        for (int j = 0; j < kCB; ++j) p.dS0[((size_t)bh * dk + i) * DV + c0 + j] = a_next * ds[j];
+        for (int j = 0; j < kCH; ++j) p.dS0[((size_t)bh * dk + i) * DV + c0 + cb + j] = a_next * ds[j];
     }
     cl.sync();  // no block leaves while another still reads its shared memory
 }
@@ -592,7 +602,7 @@ cudaError_t bwd_tv(const BwdParams& p, float* qdq, float* fin, const int* only, 
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(p.B * p.H * NCB));
-    cfg.blockDim = dim3((unsigned)((p.dk + 31) / 32 * 32));
+    cfg.blockDim = dim3((unsigned)(2 * p.dk));  // two threads a row
     cfg.dynamicSmemBytes = smf;
     cfg.stream = s;
     cudaLaunchAttribute at[1];
