@@ -1,14 +1,16 @@
 #!/usr/bin/env python
 """Small launches of each kernel, the command that profiler captures wrap.
 
-    python profile_kernels.py fwd1|fwd1pre|fwd1feed|fwd1lr|fwd2|fwdbwd3|decode4|conv1|ska1|ska4
+    python profile_kernels.py fwd1|fwd1pre|fwd1feed|fwd1lr|fwd2|fwdbwd3|bwdwide3|decode4|conv1|ska1|ska4
 
 One workload per call: the mode draws its inputs on the device, runs the
 kernel(s) three times and synchronises.  fwd1 is the 130M-scale layer forward
 (B8 H6 T2048 d_k64 d_v128), fwd1pre the same with the gates passed before
 their activations, fwd2 the long-context forward (B1 H16 T32768 d_k=d_v=128),
 fwdbwd3 the training forward (saving chunk states) and backward (B4 H16 T4096
-d_k64 d_v128), decode4 four steps of the batched decode (B256 H16 d_k64 d_v128;
+d_k64 d_v128), bwdwide3 the same with one chunk of every 16th head too wide for
+one decay reference (g scaled by 40 there; the exact backward recomputes those
+heads), decode4 four steps of the batched decode (B256 H16 d_k64 d_v128;
 only 4 steps of inputs are drawn instead of 1024, the kernel is the same),
 fwd1feed the 130M-scale layer forward with the feedthrough, fwd1lr the same
 layer with the gates passed before their activations and a rank-16 beta_hat, conv1 the
@@ -71,9 +73,13 @@ def main(mode: str) -> int:
             pos = torch.full((B,), 1000, dtype=torch.int32, device="cuda")
             for _ in range(3):
                 rdm.rdm_ska_decode(q, k, v, kc, vc, pos)
-    elif mode == "fwdbwd3":
+    elif mode in ("fwdbwd3", "bwdwide3"):
         w = WORKLOADS[3]
         x = draw_workload(w, device="cuda")
+        if mode == "bwdwide3":
+            gw = x["g"].float()
+            gw[:, ::16, 64 * 20:64 * 21] *= 40.0
+            x["g"] = gw.clamp(min=0.05).to(torch.bfloat16)
         saved = torch.empty(rdm.rdm_ddts_saved_states_size(w.B, w.H, w.T, w.dk, w.dv, 64) // 4,
                             device="cuda")
         for _ in range(3):

@@ -54,7 +54,8 @@ def test_simt_forward_shapes(cuda_ok, dtype, dk, dv, T):
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-@pytest.mark.parametrize("dk,dv,T", [(16, 32, 9), (64, 128, 70), (128, 32, 33)])
+@pytest.mark.parametrize("dk,dv,T", [(16, 32, 9), (64, 128, 70), (128, 32, 33), (32, 16, 48),
+                                     (128, 128, 40)])
 def test_simt_backward(cuda_ok, dtype, dk, dv, T):
     x = draw_sequence(1, 2, T, dk, dv, dtype, seed=200 + T, s0_std=0.1, with_dO=True)
     dST = torch.randn(1, 2, dk, dv, generator=torch.Generator().manual_seed(5)) * 0.1
