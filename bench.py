@@ -101,6 +101,7 @@ BWD_SRC = ["tc_bwd.cu"] + _DEV_HDR
 DECODE_SRC = ["decode.cu", "rdm_common.cuh", "launch.h"]
 SKA_SRC = ["ska.cu", "ska_launch.h"] + _DEV_HDR
 CONV_SRC = ["shortconv.cu", "conv_launch.h"] + _DEV_HDR
+SIMT_SRC = ["simt.cu", "rdm_common.cuh", "launch.h"]
 
 
 def src_sha(*names):
@@ -365,7 +366,12 @@ def run_extras(rdm, dev, pk, K):
         "value": w.B * w.T / (msw / 1e3), "unit": "tokens/s", "ms_per_step": msw,
         "ms_bwd_without": msb, "wide_heads": w.B * ((w.H + 15) // 16),
         # backward kernel + the two exact re-run kernels
-        "gpu_launches_per_step": 3}
+        "gpu_launches_per_step": 3,
+        # the backward's algorithmic bytes over the whole step: the recomputed heads
+        # are latency-bound token-serial sweeps, not a bandwidth problem
+        "roofline": roofline(bwd_bytes(w), chunk_flops_bwd(w), msw, pk, None),
+        "ncu_exact_sweeps": {"reverse": ncu_counters("simt_bwd_rsweep", SIMT_SRC, "wide3"),
+                             "forward": ncu_counters("simt_bwd_fsweep", SIMT_SRC, "wide3")}}
     del x, o, saved, grads, ws, wsf
     # headline forward with the feedthrough o_t += d (.) v_t (same algorithmic
     # bytes plus d; v is re-read from L2 in the store stage)
