@@ -10,7 +10,7 @@
 // Backward, exact reverse mode organised in two sweeps per (b,h), each run by a
 // cluster of blocks that split the state's columns, threads 2i and 2i+1 owning
 // row i of their block's columns of the state or of its gradient:
-//   sweep F (forward in t):  S_t, dq_t = S_t dO_t, and q_t*dq_t kept in scratch;
+//   sweep F (forward in t):  S_t, dq_t = S_t dO_t (kept in float32 scratch too);
 //   sweep R (reverse in t):  dS_t = q_t dO_t^T + diag(alpha_{t+1}) dS_{t+1},
 //                            dkhat_t = dS_t vhat_t, dvhat_t = dS_t^T khat_t.
 // The decay gradient uses d(log alpha_t) = sum_{u>=t} dG_u with
@@ -154,31 +154,31 @@ __device__ __forceinline__ void cp_async_wait_prev() {
 }
 
 // One stage of the tile pipeline in dynamic shared memory, inputs as stored:
-// the rows [kTile][dk] of g, tau, k, q, in sweep R the rows of q*dq (float32),
+// the rows [kTile][dk] of g, tau, k, q, in sweep R the rows of dq (float32),
 // then the block's columns [kTile][kCB] of beta, v, dO.  Every part is a
 // multiple of 16 bytes (dk >= 16).
 template <typename T>
 struct SweepStage {
     T* row[4];
-    float* qdq;
+    float* dqf;
     T* col[3];
 };
 
 template <typename T>
-__host__ __device__ __forceinline__ size_t sweep_stage_bytes(int dk, bool with_qdq) {
-    return (size_t)4 * kTile * dk * sizeof(T) + (with_qdq ? (size_t)kTile * dk * 4 : 0) +
+__host__ __device__ __forceinline__ size_t sweep_stage_bytes(int dk, bool with_dq) {
+    return (size_t)4 * kTile * dk * sizeof(T) + (with_dq ? (size_t)kTile * dk * 4 : 0) +
            (size_t)3 * kTile * kCB * sizeof(T);
 }
 
 template <typename T>
-__device__ __forceinline__ SweepStage<T> sweep_stage(unsigned char* base, int dk, bool with_qdq) {
+__device__ __forceinline__ SweepStage<T> sweep_stage(unsigned char* base, int dk, bool with_dq) {
     SweepStage<T> s;
     const size_t rb = (size_t)kTile * dk * sizeof(T), cb = (size_t)kTile * kCB * sizeof(T);
 #pragma unroll
     for (int a = 0; a < 4; ++a) s.row[a] = reinterpret_cast<T*>(base + a * rb);
     unsigned char* p = base + 4 * rb;
-    s.qdq = with_qdq ? reinterpret_cast<float*>(p) : nullptr;
-    if (with_qdq) p += (size_t)kTile * dk * 4;
+    s.dqf = with_dq ? reinterpret_cast<float*>(p) : nullptr;
+    if (with_dq) p += (size_t)kTile * dk * 4;
 #pragma unroll
     for (int a = 0; a < 3; ++a) s.col[a] = reinterpret_cast<T*>(p + a * cb);
     return s;
@@ -191,7 +191,7 @@ __device__ __forceinline__ SweepStage<T> sweep_stage(unsigned char* base, int dk
 // pointers are, and every offset is a multiple of 16 * dk, DV or kCB elements.
 template <typename T, int DV>
 __device__ __forceinline__ void sweep_fetch(const SweepStage<T>& st, const T* const (&rows)[4],
-                                            const float* qdq_bh, const T* const (&cols)[3], int t0,
+                                            const float* dqf_bh, const T* const (&cols)[3], int t0,
                                             int nt, int dk) {
     const size_t roff = (size_t)t0 * dk;
     const int rchunks = nt * dk * (int)sizeof(T) / 16;
@@ -201,9 +201,9 @@ __device__ __forceinline__ void sweep_fetch(const SweepStage<T>& st, const T* co
             cp_async16(reinterpret_cast<char*>(st.row[a]) + c * 16,
                        reinterpret_cast<const char*>(rows[a] + roff) + c * 16);
     }
-    if (st.qdq) {
+    if (st.dqf) {
         for (int c = threadIdx.x; c < nt * dk / 4; c += blockDim.x)
-            cp_async16(st.qdq + c * 4, qdq_bh + roff + c * 4);
+            cp_async16(st.dqf + c * 4, dqf_bh + roff + c * 4);
     }
     constexpr int cpt = kCB * (int)sizeof(T) / 16;  // 16-byte pieces of one token's columns
     for (int c = threadIdx.x; c < nt * cpt; c += blockDim.x) {
@@ -219,7 +219,7 @@ __device__ __forceinline__ void sweep_fetch(const SweepStage<T>& st, const T* co
         for (int e = nt * dk + threadIdx.x; e < kTile * dk; e += blockDim.x) {
 #pragma unroll
             for (int a = 0; a < 4; ++a) stf(st.row[a] + e, 0.0f);
-            if (st.qdq) st.qdq[e] = 0.0f;
+            if (st.dqf) st.dqf[e] = 0.0f;
         }
         for (int e = nt * kCB + threadIdx.x; e < kTile * kCB; e += blockDim.x) {
 #pragma unroll
@@ -229,7 +229,7 @@ __device__ __forceinline__ void sweep_fetch(const SweepStage<T>& st, const T* co
 }
 
 template <typename T, int DV>
-__global__ void __launch_bounds__(256) simt_bwd_fsweep(BwdParams p, float* qdq, float* fin,
+__global__ void __launch_bounds__(256) simt_bwd_fsweep(BwdParams p, float* dqf, float* fin,
                                                        const int* only) {
     constexpr int NCB = DV / kCB;
     namespace cg = cooperative_groups;
@@ -241,7 +241,7 @@ __global__ void __launch_bounds__(256) simt_bwd_fsweep(BwdParams p, float* qdq, 
     // (the block has 2 d_k threads)
     const int i = threadIdx.x >> 1, cb = (threadIdx.x & 1) * kCH;
     const bool act = i < dk;
-    const bool own = act && cb == 0 && i / owner_rows<DV>(dk) == rank;  // this block finishes row i
+    const int rows_pb = owner_rows<DV>(dk), r0 = rank * rows_pb;  // rows this block finishes
     __shared__ float s_vh[kTile][kCB], s_do[kTile][kCB], s_part[2][kTile][kMaxRows], s_fin[kMaxRows];
     extern __shared__ __align__(16) unsigned char s_stage[];
 
@@ -251,8 +251,12 @@ __global__ void __launch_bounds__(256) simt_bwd_fsweep(BwdParams p, float* qdq, 
     const T* const cols[3] = {static_cast<const T*>(p.beta) + cbase, static_cast<const T*>(p.v) + cbase,
                               static_cast<const T*>(p.dO) + cbase};
     T* dq = static_cast<T*>(p.dq) + rbase;
-    float* qdq_bh = qdq + rbase;
+    float* dqf_bh = dqf + rbase;
     const size_t sbytes = sweep_stage_bytes<T>(dk, false);
+    // the tile's gates as the token loop uses them, [kTile][dk]: alpha and
+    // khat = alpha_hat k (1 and 0 past the end of a partial tile)
+    float* s_al = reinterpret_cast<float*>(s_stage + 2 * sbytes);
+    float* s_kh = s_al + kTile * dk;
 
     float s[kCH];
 #pragma unroll
@@ -260,9 +264,8 @@ __global__ void __launch_bounds__(256) simt_bwd_fsweep(BwdParams p, float* qdq, 
         s[j] = (act && p.S0) ? p.S0[((size_t)bh * dk + i) * DV + c0 + cb + j] : 0.0f;
 
     // Tile n: its stage was fetched while tile n - 1 ran; it is unpacked into
-    // s_vh, s_do and this row's registers before the cluster waits for the
-    // partial sums of tile n - 1, so that wait overlaps the unpacking.
-    float rg[kTile], rt[kTile], rk[kTile], rq[kTile];
+    // s_vh, s_do and the gate arrays before the cluster waits for the partial
+    // sums of tile n - 1, so that wait overlaps the unpacking.
     auto fetch = [&](int m) {  // starts tile m's copies (an empty group past the end)
         if (m < ntiles_of(T_)) {
             const int tm = m * kTile;
@@ -274,25 +277,22 @@ __global__ void __launch_bounds__(256) simt_bwd_fsweep(BwdParams p, float* qdq, 
     };
     auto unpack = [&](int m) {  // after tile m's copies are complete and visible
         const SweepStage<T> cur = sweep_stage<T>(s_stage + (m & 1) * sbytes, dk, false);
+        const int nt_m = min(kTile, T_ - m * kTile);
         for (int idx = threadIdx.x; idx < kTile * kCB; idx += blockDim.x) {
             const float bb = ldf(cur.col[0] + idx);
             s_vh[idx / kCB][idx % kCB] = (p.preact ? sigmoid_acc(bb) : bb) * ldf(cur.col[1] + idx);
             s_do[idx / kCB][idx % kCB] = ldf(cur.col[2] + idx);
         }
-        // this row's gates, key and query for the whole tile (zeros past the end)
-#pragma unroll
-        for (int tt = 0; tt < kTile; ++tt) {
-            rg[tt] = ldf(cur.row[0] + tt * dk + i);
-            rt[tt] = ldf(cur.row[1] + tt * dk + i);
-            rk[tt] = ldf(cur.row[2] + tt * dk + i);
-            rq[tt] = ldf(cur.row[3] + tt * dk + i);
-        }
-        if (p.preact) {
-#pragma unroll
-            for (int tt = 0; tt < kTile; ++tt) {
-                rg[tt] = softplus_acc(rg[tt]);
-                rt[tt] = sigmoid_acc(rt[tt]);
+        // the gate arithmetic of every (token, row) once, spread over the block
+        for (int e = threadIdx.x; e < kTile * dk; e += blockDim.x) {
+            float gg = ldf(cur.row[0] + e), ta = ldf(cur.row[1] + e);
+            if (p.preact) {
+                gg = softplus_acc(gg);
+                ta = sigmoid_acc(ta);
             }
+            const bool live = e / dk < nt_m;
+            s_al[e] = live ? alpha(gg, ta) : 1.0f;
+            s_kh[e] = live ? alpha_hat(gg, ta) * ldf(cur.row[2] + e) : 0.0f;
         }
     };
     const int ntiles = ntiles_of(T_);
@@ -307,14 +307,10 @@ __global__ void __launch_bounds__(256) simt_bwd_fsweep(BwdParams p, float* qdq, 
     for (int n = 0; n < ntiles; ++n) {
         const int t0 = n * kTile, nt = min(kTile, T_ - t0), buf = n & 1;
         // the tile's tokens as one straight run (a token past the end of a partial
-        // tile leaves the state as it is: alpha 1, khat 0), so the compiler can
-        // overlap the gate arithmetic of one token with the updates of another
+        // tile leaves the state as it is: alpha 1, khat 0)
 #pragma unroll
         for (int tt = 0; tt < kTile; ++tt) {
-            const bool live = tt < nt;
-            const float gg = rg[tt], ta = rt[tt];
-            const float al = live ? alpha(gg, ta) : 1.0f;
-            const float kh = live ? alpha_hat(gg, ta) * rk[tt] : 0.0f;
+            const float al = s_al[tt * dk + i], kh = s_kh[tt * dk + i];
             float a0 = 0.0f, a1 = 0.0f;
 #pragma unroll
             for (int j = 0; j < kCH; j += 2) {
@@ -329,11 +325,8 @@ __global__ void __launch_bounds__(256) simt_bwd_fsweep(BwdParams p, float* qdq, 
         }
         // this block's partials of the tile are written (s_part alternates by tile:
         // a block writes tile n + 2 into this buffer only after every block has
-        // arrived after tile n + 1, that is, after its owners read tile n)
+        // arrived after tile n + 1, that is, after it read tile n's sums)
         cluster_arrive();
-        float rqo[kTile];
-#pragma unroll
-        for (int tt = 0; tt < kTile; ++tt) rqo[tt] = rq[tt];
         if (n + 1 < ntiles) {
             fetch(n + 2);  // into the stage tile n came from, unpacked before its run
             cp_async_wait_prev();
@@ -342,16 +335,17 @@ __global__ void __launch_bounds__(256) simt_bwd_fsweep(BwdParams p, float* qdq, 
             __syncthreads();
         }
         cluster_wait();  // every block's partials of tile n are written
-        if (own) {
-            // every block's partials of the tile, all read before the first store
-            float dqv[kTile];
-            cluster_row_sums<NCB>(cl, &s_part[buf][0][i], dqv);
+        // dq of this block's rows, one (row, token) a thread: the sum of every
+        // block's partial through distributed shared memory
+        for (int it = threadIdx.x; it < rows_pb * kTile; it += blockDim.x) {
+            const int row = r0 + it / kTile, tt = it % kTile;
+            if (row < dk && tt < nt) {
+                float acc = 0.0f;
 #pragma unroll
-            for (int tt = 0; tt < kTile; ++tt) {
-                if (tt >= nt) break;
-                const size_t off = (size_t)(t0 + tt) * dk + i;
-                stf(dq + off, dqv[tt]);
-                qdq_bh[off] = rqo[tt] * dqv[tt];
+                for (int r = 0; r < NCB; ++r) acc += *cl.map_shared_rank(&s_part[buf][tt][row], r);
+                const size_t off = (size_t)(t0 + tt) * dk + row;
+                stf(dq + off, acc);
+                dqf_bh[off] = acc;
             }
         }
     }
@@ -365,18 +359,18 @@ __global__ void __launch_bounds__(256) simt_bwd_fsweep(BwdParams p, float* qdq, 
     f += __shfl_xor_sync(0xffffffffu, f, 1);
     if (act && cb == 0) s_fin[i] = f;
     cl.sync();
-    if (own) {
+    for (int row = r0 + threadIdx.x; row < min(dk, r0 + rows_pb); row += blockDim.x) {
         float acc = 0.0f;
 #pragma unroll
-        for (int r = 0; r < NCB; ++r) acc += *cl.map_shared_rank(&s_fin[i], r);
-        fin[(size_t)bh * dk + i] = acc;
+        for (int r = 0; r < NCB; ++r) acc += *cl.map_shared_rank(&s_fin[row], r);
+        fin[(size_t)bh * dk + row] = acc;
     }
     cl.sync();  // no block leaves while another still reads its shared memory
 }
 
 // ------------------------------------------------ backward, reverse sweep R
 template <typename T, int DV>
-__global__ void __launch_bounds__(256) simt_bwd_rsweep(BwdParams p, const float* qdq,
+__global__ void __launch_bounds__(256) simt_bwd_rsweep(BwdParams p, const float* dqf,
                                                        const float* fin, const int* only) {
     constexpr int NCB = DV / kCB;
     static_assert(kCH == 8, "the column reduce-scatter below takes three halving rounds");
@@ -388,10 +382,11 @@ __global__ void __launch_bounds__(256) simt_bwd_rsweep(BwdParams p, const float*
     // two threads a row, as in sweep F
     const int i = threadIdx.x >> 1, cb = (threadIdx.x & 1) * kCH;
     const bool act = i < dk;
-    const bool own = act && cb == 0 && i / owner_rows<DV>(dk) == rank;
+    const int rows_pb = owner_rows<DV>(dk), r0 = rank * rows_pb;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x / 32;
     __shared__ float s_vh[kTile][kCB], s_do[kTile][kCB], s_b[kTile][kCB], s_v[kTile][kCB];
     __shared__ float s_part[2][kTile][kMaxRows], s_red[kTile][8][kCB];
+    __shared__ float s_da[kMaxRows];  // decay-gradient carry of this block's rows
     extern __shared__ __align__(16) unsigned char s_stage[];
 
     const size_t rbase = (size_t)bh * T_ * dk, cbase = (size_t)bh * T_ * DV + c0;
@@ -404,28 +399,38 @@ __global__ void __launch_bounds__(256) simt_bwd_rsweep(BwdParams p, const float*
     T* dtau = static_cast<T*>(p.dtau) + rbase;
     T* dv_ = static_cast<T*>(p.dv_) + cbase;
     T* dbeta = static_cast<T*>(p.dbeta) + cbase;
-    const float* qdq_bh = qdq + rbase;
+    const float* dqf_bh = dqf + rbase;
     const float* dfeed = p.dfeed ? p.dfeed + (size_t)(bh % p.H) * DV + c0 : nullptr;
     const size_t sbytes = sweep_stage_bytes<T>(dk, true);
+    // the tile's gates, [kTile][dk] each: alpha and khat = alpha_hat k for the
+    // token loop (1 and 0 past the end of a partial tile), and for the scan the
+    // activated g and tau, alpha_hat and log2 g
+    float* s_al = reinterpret_cast<float*>(s_stage + 2 * sbytes);
+    float* s_kh = s_al + kTile * dk;
+    float* s_gg = s_kh + kTile * dk;
+    float* s_ta = s_gg + kTile * dk;
+    float* s_ah = s_ta + kTile * dk;
+    float* s_lg = s_ah + kTile * dk;
 
     float ds[kCH];
 #pragma unroll
     for (int j = 0; j < kCH; ++j)
         ds[j] = (act && p.dST) ? p.dST[((size_t)bh * dk + i) * DV + c0 + cb + j] : 0.0f;
-    float a_next = 1.0f;                            // alpha_{t+1,i}
-    float da = own ? fin[(size_t)bh * dk + i] : 0.0f;  // running sum of dG over u >= t
+    float a_next = 1.0f;  // alpha_{t+1,i}
+    for (int rl = threadIdx.x; rl < rows_pb; rl += blockDim.x)
+        s_da[rl] = r0 + rl < dk ? fin[(size_t)bh * dk + r0 + rl] : 0.0f;
 
     // tile n holds tokens [t1 - kTile, t1) with t1 = T - n kTile (the last one
     // processed may be partial)
-    const int ntiles = (T_ + kTile - 1) / kTile;
+    const int ntiles = ntiles_of(T_);
     if (ntiles > 0)
-        sweep_fetch<T, DV>(sweep_stage<T>(s_stage, dk, true), rows, qdq_bh, cols, max(0, T_ - kTile),
+        sweep_fetch<T, DV>(sweep_stage<T>(s_stage, dk, true), rows, dqf_bh, cols, max(0, T_ - kTile),
                            min(kTile, T_), dk);
     for (int n = 0; n < ntiles; ++n) {
         const int t1 = T_ - n * kTile, t0 = max(0, t1 - kTile), nt = t1 - t0, buf = n & 1;
         const SweepStage<T> cur = sweep_stage<T>(s_stage + buf * sbytes, dk, true);
         if (n + 1 < ntiles)
-            sweep_fetch<T, DV>(sweep_stage<T>(s_stage + (buf ^ 1) * sbytes, dk, true), rows, qdq_bh,
+            sweep_fetch<T, DV>(sweep_stage<T>(s_stage + (buf ^ 1) * sbytes, dk, true), rows, dqf_bh,
                                cols, max(0, t0 - kTile), min(kTile, t0), dk);
         else
             cp_async_commit();
@@ -440,23 +445,23 @@ __global__ void __launch_bounds__(256) simt_bwd_rsweep(BwdParams p, const float*
             s_vh[tt][j] = bb * vv;
             s_do[tt][j] = ldf(cur.col[2] + idx);
         }
-        // this row's gates, key and query for the whole tile (zeros past the end);
-        // the gates are activated in place, and log2(g) and alpha_hat are kept for
-        // the owner's scan below
-        float rg[kTile], rt[kTile], rk[kTile], rq[kTile], rlg[kTile], rah[kTile];
-#pragma unroll
-        for (int tt = 0; tt < kTile; ++tt) {
-            rg[tt] = ldf(cur.row[0] + tt * dk + i);
-            rt[tt] = ldf(cur.row[1] + tt * dk + i);
-            rk[tt] = ldf(cur.row[2] + tt * dk + i);
-            rq[tt] = ldf(cur.row[3] + tt * dk + i);
-        }
-        if (p.preact) {
-#pragma unroll
-            for (int tt = 0; tt < kTile; ++tt) {
-                rg[tt] = softplus_acc(rg[tt]);
-                rt[tt] = sigmoid_acc(rt[tt]);
+        // the gate arithmetic of every (token, row) once, spread over the block
+        for (int e = threadIdx.x; e < kTile * dk; e += blockDim.x) {
+            float gg = ldf(cur.row[0] + e), ta = ldf(cur.row[1] + e);
+            if (p.preact) {
+                gg = softplus_acc(gg);
+                ta = sigmoid_acc(ta);
             }
+            const bool live = e / dk < nt;
+            // alpha_hat = g^tau with 0^0 = 1 and 0^tau = 0 (log2(0) = -inf)
+            const float lg = log2f(gg);
+            const float ah = ta == 0.0f ? 1.0f : exp2f(ta * lg);
+            s_al[e] = live ? alpha(gg, ta) : 1.0f;
+            s_kh[e] = live ? ah * ldf(cur.row[2] + e) : 0.0f;
+            s_gg[e] = gg;
+            s_ta[e] = ta;
+            s_ah[e] = ah;
+            s_lg[e] = lg;
         }
         __syncthreads();
         // the tile's tokens as one straight run, as in sweep F (a token past the end
@@ -464,13 +469,9 @@ __global__ void __launch_bounds__(256) simt_bwd_rsweep(BwdParams p, const float*
 #pragma unroll
         for (int tt = kTile - 1; tt >= 0; --tt) {
             const bool live = tt < nt;
-            const float gg = rg[tt], ta = rt[tt];
-            // alpha_hat = g^tau with 0^0 = 1 and 0^tau = 0 (log2(0) = -inf)
-            rlg[tt] = log2f(gg);
-            rah[tt] = ta == 0.0f ? 1.0f : exp2f(ta * rlg[tt]);
             const float f = live ? a_next : 1.0f;
-            const float qi = act ? rq[tt] : 0.0f;
-            const float kh = act ? rah[tt] * rk[tt] : 0.0f;
+            const float qi = act ? ldf(cur.row[3] + tt * dk + i) : 0.0f;
+            const float kh = act ? s_kh[tt * dk + i] : 0.0f;
             float d0 = 0.0f, d1 = 0.0f;
 #pragma unroll
             for (int j = 0; j < kCH; j += 2) {
@@ -509,7 +510,7 @@ __global__ void __launch_bounds__(256) simt_bwd_rsweep(BwdParams p, const float*
             }
             x[0] += __shfl_xor_sync(0xffffffffu, x[0], 2);
             if ((lane & 2) == 0) s_red[tt][warp][cb + col] = x[0];
-            if (live) a_next = alpha(gg, ta);
+            if (live) a_next = s_al[tt * dk + i];
         }
         // this block's dkhat partials of the tile are written (s_part alternates by
         // tile, as in sweep F); the dvhat outputs need only this block's partials
@@ -526,47 +527,52 @@ __global__ void __launch_bounds__(256) simt_bwd_rsweep(BwdParams p, const float*
             stf(dbeta + ov, (p.preact ? bb * (1.0f - bb) : 1.0f) * s_v[tt][j] * dvh);
         }
         cluster_wait();  // every block's dkhat partials of the tile are written
-        if (own) {
-            // the owner's reverse scan of the decay gradient over the tile
-            float rqd[kTile], dkv[kTile];
+        // The decay gradient of this block's rows, one (row, token) a thread: the
+        // 16 tokens of a row are 16 consecutive lanes (the block has 2 d_k threads
+        // and rows_pb * kTile = 16 d_k / NCB items, so every thread takes the same
+        // number of passes and whole warps shuffle).  d log alpha_t is the row's
+        // carry (every later tile) plus the suffix sum over the tile's tokens u >= t
+        // of dG_u = q_u dq_u - khat_u dkhat_u.
+        for (int it = threadIdx.x; it < rows_pb * kTile; it += blockDim.x) {
+            const int rl = it / kTile, row = min(r0 + rl, dk - 1), tt = it % kTile;
+            const bool live = tt < nt && r0 + rl < dk;
+            const int e = tt * dk + row;
+            float dkh = 0.0f;
 #pragma unroll
-            for (int tt = 0; tt < kTile; ++tt) rqd[tt] = cur.qdq[tt * dk + i];
-            cluster_row_sums<NCB>(cl, &s_part[buf][0][i], dkv);
-            // a whole tile runs without a test per token (a partial one is the last)
-            auto scan = [&](auto whole) {
-                constexpr bool kWhole = decltype(whole)::value;
+            for (int r = 0; r < NCB; ++r) dkh += *cl.map_shared_rank(&s_part[buf][tt][row], r);
+            const float kk = ldf(cur.row[2] + e), ah = s_ah[e];
+            const float dG = live ? ldf(cur.row[3] + e) * cur.dqf[e] - ah * kk * dkh : 0.0f;
+            const float carry = s_da[rl];
+            float sfx = dG;
 #pragma unroll
-                for (int tt = kTile - 1; tt >= 0; --tt) {
-                    const bool live = kWhole || tt < nt;
-                    const float dkh = dkv[tt], gg = rg[tt], ta = rt[tt], kk = rk[tt];
-                    const float ah = rah[tt], lg = rlg[tt];
-                    // chain factors to the pre-activations: softplus' = sigmoid, which
-                    // is 1 - e^-g of the activated g; sigmoid' = s (1 - s)
-                    const float cg_ = p.preact ? -expm1f(-gg) : 1.0f;
-                    const float ct = p.preact ? ta * (1.0f - ta) : 1.0f;
-                    if (live) da += rqd[tt] - ah * kk * dkh;
-                    const float dah = kk * dkh;
-                    // d alpha_hat / d g = tau g^(tau - 1), which is tau alpha_hat / g
-                    // while alpha_hat is a normal number (then g > 0); d alpha_hat /
-                    // d tau = alpha_hat ln g
-                    const float dah_dg = ta == 0.0f ? 0.0f
-                                         : ah >= 1.17549435e-38f ? __fdividef(ta * ah, gg)
-                                                                  : ta * exp2f((ta - 1.0f) * lg);
-                    const float dah_dtau = ah == 0.0f ? 0.0f : ah * (lg * kLn2);
-                    if (live) {
-                        const size_t off = (size_t)(t0 + tt) * dk + i;
-                        stf(dk_ + off, ah * dkh);
-                        stf(dg + off, cg_ * (-ta * da + dah_dg * dah));
-                        stf(dtau + off, ct * (-gg * da + dah_dtau * dah));
-                    }
-                }
-            };
-            if (nt == kTile)
-                scan(std::true_type{});
-            else
-                scan(std::false_type{});
+            for (int o = 1; o < kTile; o <<= 1) {
+                const float y = __shfl_down_sync(0xffffffffu, sfx, o, kTile);
+                if (tt + o < kTile) sfx += y;
+            }
+            const float da = carry + sfx;
+            const float gg = s_gg[e], ta = s_ta[e], lg = s_lg[e];
+            // chain factors to the pre-activations: softplus' = sigmoid, which is
+            // 1 - e^-g of the activated g; sigmoid' = s (1 - s)
+            const float cg_ = p.preact ? -expm1f(-gg) : 1.0f;
+            const float ct = p.preact ? ta * (1.0f - ta) : 1.0f;
+            const float dah = kk * dkh;
+            // d alpha_hat / d g = tau g^(tau - 1), which is tau alpha_hat / g while
+            // alpha_hat is a normal number (then g > 0); d alpha_hat / d tau =
+            // alpha_hat ln g
+            const float dah_dg = ta == 0.0f ? 0.0f
+                                 : ah >= 1.17549435e-38f ? __fdividef(ta * ah, gg)
+                                                          : ta * exp2f((ta - 1.0f) * lg);
+            const float dah_dtau = ah == 0.0f ? 0.0f : ah * (lg * kLn2);
+            if (live) {
+                const size_t off = (size_t)(t0 + tt) * dk + row;
+                stf(dk_ + off, ah * dkh);
+                stf(dg + off, cg_ * (-ta * da + dah_dg * dah));
+                stf(dtau + off, ct * (-gg * da + dah_dtau * dah));
+            }
+            __syncwarp();  // every lane of the row has read the carry
+            if (tt == 0) s_da[rl] = carry + sfx;  // the whole tile's sum
         }
-        __syncthreads();  // the staging buffers and s_red are free for the next tile
+        __syncthreads();  // the staging buffers, gate arrays and s_red are free for the next tile
     }
     if (act && p.dS0) {
 #pragma unroll
@@ -589,11 +595,14 @@ cudaError_t fwd_t(const SeqParams& p, cudaStream_t s) {
 }
 
 template <typename T, int DV>
-cudaError_t bwd_tv(const BwdParams& p, float* qdq, float* fin, const int* only, cudaStream_t s) {
+cudaError_t bwd_tv(const BwdParams& p, float* dqf, float* fin, const int* only, cudaStream_t s) {
     // one cluster of DV / kCB blocks per (b,h)
     constexpr int NCB = DV / kCB;
-    // two pipeline stages of dynamic shared memory (sweep R's carry q*dq too)
-    const size_t smf = 2 * sweep_stage_bytes<T>(p.dk, false), smr = 2 * sweep_stage_bytes<T>(p.dk, true);
+    // two pipeline stages of dynamic shared memory (sweep R's carry dq too), then
+    // the tile's gate arrays (two in sweep F, six in sweep R)
+    const size_t ga = (size_t)kTile * p.dk * 4;
+    const size_t smf = 2 * sweep_stage_bytes<T>(p.dk, false) + 2 * ga;
+    const size_t smr = 2 * sweep_stage_bytes<T>(p.dk, true) + 6 * ga;
     cudaError_t e = cudaFuncSetAttribute(simt_bwd_fsweep<T, DV>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smf);
     if (e == cudaSuccess)
@@ -612,20 +621,20 @@ cudaError_t bwd_tv(const BwdParams& p, float* qdq, float* fin, const int* only, 
     at[0].val.clusterDim.z = 1;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, simt_bwd_fsweep<T, DV>, p, qdq, fin, only);
+    e = cudaLaunchKernelEx(&cfg, simt_bwd_fsweep<T, DV>, p, dqf, fin, only);
     if (e != cudaSuccess) return e;
     cfg.dynamicSmemBytes = smr;
-    return cudaLaunchKernelEx(&cfg, simt_bwd_rsweep<T, DV>, p, static_cast<const float*>(qdq),
+    return cudaLaunchKernelEx(&cfg, simt_bwd_rsweep<T, DV>, p, static_cast<const float*>(dqf),
                               static_cast<const float*>(fin), only);
 }
 
 template <typename T>
-cudaError_t bwd_t(const BwdParams& p, float* qdq, float* fin, const int* only, cudaStream_t s) {
+cudaError_t bwd_t(const BwdParams& p, float* dqf, float* fin, const int* only, cudaStream_t s) {
     switch (p.dv) {
-        case 16: return bwd_tv<T, 16>(p, qdq, fin, only, s);
-        case 32: return bwd_tv<T, 32>(p, qdq, fin, only, s);
-        case 64: return bwd_tv<T, 64>(p, qdq, fin, only, s);
-        case 128: return bwd_tv<T, 128>(p, qdq, fin, only, s);
+        case 16: return bwd_tv<T, 16>(p, dqf, fin, only, s);
+        case 32: return bwd_tv<T, 32>(p, dqf, fin, only, s);
+        case 64: return bwd_tv<T, 64>(p, dqf, fin, only, s);
+        case 128: return bwd_tv<T, 128>(p, dqf, fin, only, s);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -637,7 +646,7 @@ cudaError_t launch_simt_fwd(const SeqParams& p, cudaStream_t s) {
     return p.bf16 ? fwd_t<__nv_bfloat16>(p, s) : fwd_t<float>(p, s);
 }
 
-// scratch: q*dq for every (b,h,t,i) and the final-state term per (b,h,i), float32
+// scratch: dq for every (b,h,t,i) and the final-state term per (b,h,i), float32
 size_t simt_bwd_workspace(const BwdParams& p) {
     const size_t rows = (size_t)p.B * p.H * p.dk;
     const size_t a = ((rows * (size_t)p.T * 4) + 255) / 256 * 256;
@@ -648,9 +657,9 @@ static cudaError_t simt_bwd(const BwdParams& p, const int* only, cudaStream_t s)
     if (p.B * p.H == 0) return cudaSuccess;
     const size_t rows = (size_t)p.B * p.H * p.dk;
     const size_t a = ((rows * (size_t)p.T * 4) + 255) / 256 * 256;
-    float* qdq = static_cast<float*>(p.ws);
+    float* dqf = static_cast<float*>(p.ws);
     float* fin = reinterpret_cast<float*>(static_cast<char*>(p.ws) + a);
-    return p.bf16 ? bwd_t<__nv_bfloat16>(p, qdq, fin, only, s) : bwd_t<float>(p, qdq, fin, only, s);
+    return p.bf16 ? bwd_t<__nv_bfloat16>(p, dqf, fin, only, s) : bwd_t<float>(p, dqf, fin, only, s);
 }
 
 cudaError_t launch_simt_bwd(const BwdParams& p, cudaStream_t s) { return simt_bwd(p, nullptr, s); }
