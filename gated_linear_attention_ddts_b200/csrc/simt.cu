@@ -8,7 +8,7 @@
 // along d_k per the paperhub.cn rebuttal "Efficient Parallelization" bullet.)
 //
 // Backward, exact reverse mode organised in two sweeps per (b,h), each run by a
-// cluster of blocks that split the state's columns, threads 2i and 2i+1 owning
+// cluster of blocks that split the state's columns, threads 4i ... 4i+3 owning
 // row i of their block's columns of the state or of its gradient:
 //   sweep F (forward in t):  S_t, dq_t = S_t dO_t (kept in float32 scratch too);
 //   sweep R (reverse in t):  dS_t = q_t dO_t^T + diag(alpha_{t+1}) dS_{t+1},
@@ -102,7 +102,8 @@ __global__ void __launch_bounds__(128) simt_fwd_kernel(SeqParams p) {
 // through distributed shared memory.  The inputs of a tile are fetched one tile
 // ahead with asynchronous copies, so their latency overlaps the tile before.
 constexpr int kCB = 16;      // state columns per block
-constexpr int kCH = kCB / 2;  // state columns per thread (two threads a row)
+constexpr int kTPR = 4;        // threads a row
+constexpr int kCH = kCB / kTPR;  // state columns per thread
 constexpr int kMaxRows = 128;
 
 template <int DV>
@@ -229,7 +230,7 @@ __device__ __forceinline__ void sweep_fetch(const SweepStage<T>& st, const T* co
 }
 
 template <typename T, int DV>
-__global__ void __launch_bounds__(256) simt_bwd_fsweep(BwdParams p, float* dqf, float* fin,
+__global__ void __launch_bounds__(512) simt_bwd_fsweep(BwdParams p, float* dqf, float* fin,
                                                        const int* only) {
     constexpr int NCB = DV / kCB;
     namespace cg = cooperative_groups;
@@ -237,9 +238,9 @@ __global__ void __launch_bounds__(256) simt_bwd_fsweep(BwdParams p, float* dqf, 
     const int rank = (int)cl.block_rank(), bh = blockIdx.x / NCB;
     if (only && only[bh] == 0) return;  // head already handled by the tensor-core path
     const int T_ = p.T, dk = p.dk, c0 = rank * kCB;
-    // two threads a row: thread 2i + h runs columns c0 + 8h ... c0 + 8h + 7 of row i
-    // (the block has 2 d_k threads)
-    const int i = threadIdx.x >> 1, cb = (threadIdx.x & 1) * kCH;
+    // four threads a row: thread 4i + h runs columns c0 + 4h ... c0 + 4h + 3 of
+    // row i (the block has 4 d_k threads)
+    const int i = threadIdx.x / kTPR, cb = (threadIdx.x % kTPR) * kCH;
     const bool act = i < dk;
     const int rows_pb = owner_rows<DV>(dk), r0 = rank * rows_pb;  // rows this block finishes
     __shared__ float s_vh[kTile][kCB], s_do[kTile][kCB], s_part[2][kTile][kMaxRows], s_fin[kMaxRows];
@@ -320,7 +321,8 @@ __global__ void __launch_bounds__(256) simt_bwd_fsweep(BwdParams p, float* dqf, 
                 a1 = fmaf(s[j + 1], s_do[tt][cb + j + 1], a1);
             }
             float a = a0 + a1;
-            a += __shfl_xor_sync(0xffffffffu, a, 1);  // the row's other half
+            a += __shfl_xor_sync(0xffffffffu, a, 1);  // the row's other columns
+            a += __shfl_xor_sync(0xffffffffu, a, 2);
             if (act && cb == 0) s_part[buf][tt][i] = a;
         }
         // this block's partials of the tile are written (s_part alternates by tile:
@@ -357,6 +359,7 @@ __global__ void __launch_bounds__(256) simt_bwd_fsweep(BwdParams p, float* dqf, 
             f = fmaf(p.dST[((size_t)bh * dk + i) * DV + c0 + cb + j], s[j], f);
     }
     f += __shfl_xor_sync(0xffffffffu, f, 1);
+    f += __shfl_xor_sync(0xffffffffu, f, 2);
     if (act && cb == 0) s_fin[i] = f;
     cl.sync();
     for (int row = r0 + threadIdx.x; row < min(dk, r0 + rows_pb); row += blockDim.x) {
@@ -370,22 +373,22 @@ __global__ void __launch_bounds__(256) simt_bwd_fsweep(BwdParams p, float* dqf, 
 
 // ------------------------------------------------ backward, reverse sweep R
 template <typename T, int DV>
-__global__ void __launch_bounds__(256) simt_bwd_rsweep(BwdParams p, const float* dqf,
+__global__ void __launch_bounds__(512) simt_bwd_rsweep(BwdParams p, const float* dqf,
                                                        const float* fin, const int* only) {
     constexpr int NCB = DV / kCB;
-    static_assert(kCH == 8, "the column reduce-scatter below takes three halving rounds");
+    static_assert(kCH == 4 && kTPR == 4, "the column reduce-scatter below takes two halving rounds");
     namespace cg = cooperative_groups;
     cg::cluster_group cl = cg::this_cluster();
     const int rank = (int)cl.block_rank(), bh = blockIdx.x / NCB;
     if (only && only[bh] == 0) return;
     const int T_ = p.T, dk = p.dk, c0 = rank * kCB;
-    // two threads a row, as in sweep F
-    const int i = threadIdx.x >> 1, cb = (threadIdx.x & 1) * kCH;
+    // four threads a row, as in sweep F
+    const int i = threadIdx.x / kTPR, cb = (threadIdx.x % kTPR) * kCH;
     const bool act = i < dk;
     const int rows_pb = owner_rows<DV>(dk), r0 = rank * rows_pb;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x / 32;
     __shared__ float s_vh[kTile][kCB], s_do[kTile][kCB], s_b[kTile][kCB], s_v[kTile][kCB];
-    __shared__ float s_part[2][kTile][kMaxRows], s_red[kTile][8][kCB];
+    __shared__ float s_part[2][kTile][kMaxRows], s_red[kTile][16][kCB];
     __shared__ float s_da[kMaxRows];  // decay-gradient carry of this block's rows
     extern __shared__ __align__(16) unsigned char s_stage[];
 
@@ -481,13 +484,14 @@ __global__ void __launch_bounds__(256) simt_bwd_rsweep(BwdParams p, const float*
                 d1 = fmaf(ds[j + 1], s_vh[tt][cb + j + 1], d1);
             }
             float d = d0 + d1;
-            d += __shfl_xor_sync(0xffffffffu, d, 1);  // the row's other half
+            d += __shfl_xor_sync(0xffffffffu, d, 1);  // the row's other columns
+            d += __shfl_xor_sync(0xffffffffu, d, 2);
             if (act && cb == 0) s_part[buf][tt][i] = d;  // this block's share of dkhat_{t,i}
-            // dvhat_j = sum_i dS_ij khat_i over the warp's 16 rows (lanes of one
-            // parity): a reduce-scatter over lane bits 4, 3, 2 (each halving round
+            // dvhat_j = sum_i dS_ij khat_i over the warp's 8 rows (lanes with the same
+            // l mod 4): a reduce-scatter over lane bits 4, 3 (each halving round
             // sends half of the lane's partial sums to the lane `o` apart and adds
-            // the other half it receives), then a plain sum over bit 1, after which
-            // lanes l and l ^ 2 both hold column cb + col; the warps meet below
+            // the other half it receives), then a plain sum over bit 2, after which
+            // lanes l and l ^ 4 both hold column cb + col; the warps meet below
             float x[kCH / 2];
             const bool up0 = (lane & 16) != 0;
             int col = up0 ? kCH / 2 : 0;
@@ -497,7 +501,7 @@ __global__ void __launch_bounds__(256) simt_bwd_rsweep(BwdParams p, const float*
                 x[j] = (up0 ? hi : lo) + __shfl_xor_sync(0xffffffffu, up0 ? lo : hi, 16);
             }
 #pragma unroll
-            for (int r = 1; r < 3; ++r) {
+            for (int r = 1; r < 2; ++r) {
                 const int o = 16 >> r, h = (kCH >> r) / 2;
                 const bool up = (lane & o) != 0;
 #pragma unroll
@@ -508,8 +512,8 @@ __global__ void __launch_bounds__(256) simt_bwd_rsweep(BwdParams p, const float*
                 }
                 if (up) col += h;
             }
-            x[0] += __shfl_xor_sync(0xffffffffu, x[0], 2);
-            if ((lane & 2) == 0) s_red[tt][warp][cb + col] = x[0];
+            x[0] += __shfl_xor_sync(0xffffffffu, x[0], 4);
+            if ((lane & 4) == 0) s_red[tt][warp][cb + col] = x[0];
             if (live) a_next = s_al[tt * dk + i];
         }
         // this block's dkhat partials of the tile are written (s_part alternates by
@@ -528,9 +532,8 @@ __global__ void __launch_bounds__(256) simt_bwd_rsweep(BwdParams p, const float*
         }
         cluster_wait();  // every block's dkhat partials of the tile are written
         // The decay gradient of this block's rows, one (row, token) a thread: the
-        // 16 tokens of a row are 16 consecutive lanes (the block has 2 d_k threads
-        // and rows_pb * kTile = 16 d_k / NCB items, so every thread takes the same
-        // number of passes and whole warps shuffle).  d log alpha_t is the row's
+        // 16 tokens of a row are 16 consecutive lanes (rows_pb * kTile = 16 d_k / NCB
+        // items, a multiple of 32, so whole warps take a pass and shuffle).  d log alpha_t is the row's
         // carry (every later tile) plus the suffix sum over the tile's tokens u >= t
         // of dG_u = q_u dq_u - khat_u dkhat_u.
         for (int it = threadIdx.x; it < rows_pb * kTile; it += blockDim.x) {
@@ -611,7 +614,7 @@ cudaError_t bwd_tv(const BwdParams& p, float* dqf, float* fin, const int* only, 
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(p.B * p.H * NCB));
-    cfg.blockDim = dim3((unsigned)(2 * p.dk));  // two threads a row
+    cfg.blockDim = dim3((unsigned)(kTPR * p.dk));
     cfg.dynamicSmemBytes = smf;
     cfg.stream = s;
     cudaLaunchAttribute at[1];
