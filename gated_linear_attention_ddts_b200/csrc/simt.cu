@@ -102,8 +102,8 @@ __global__ void __launch_bounds__(128) simt_fwd_kernel(SeqParams p) {
 // through distributed shared memory.  The inputs of a tile are fetched one tile
 // ahead with asynchronous copies, so their latency overlaps the tile before.
 constexpr int kCB = 16;      // state columns per block
-constexpr int kTPR = 4;        // threads a row
-constexpr int kCH = kCB / kTPR;  // state columns per thread
+// Threads a row, TPR (a template parameter: 8 for d_k <= 64, 4 for d_k = 128,
+// so a block has at most 512 threads), each running CH = kCB / TPR columns.
 constexpr int kMaxRows = 128;
 
 template <int DV>
@@ -229,18 +229,18 @@ __device__ __forceinline__ void sweep_fetch(const SweepStage<T>& st, const T* co
     }
 }
 
-template <typename T, int DV>
+template <typename T, int DV, int TPR>
 __global__ void __launch_bounds__(512) simt_bwd_fsweep(BwdParams p, float* dqf, float* fin,
                                                        const int* only) {
-    constexpr int NCB = DV / kCB;
+    constexpr int NCB = DV / kCB, CH = kCB / TPR;
     namespace cg = cooperative_groups;
     cg::cluster_group cl = cg::this_cluster();
     const int rank = (int)cl.block_rank(), bh = blockIdx.x / NCB;
     if (only && only[bh] == 0) return;  // head already handled by the tensor-core path
     const int T_ = p.T, dk = p.dk, c0 = rank * kCB;
-    // four threads a row: thread 4i + h runs columns c0 + 4h ... c0 + 4h + 3 of
-    // row i (the block has 4 d_k threads)
-    const int i = threadIdx.x / kTPR, cb = (threadIdx.x % kTPR) * kCH;
+    // TPR threads a row: thread TPR i + h runs columns c0 + CH h ... c0 + CH (h + 1) - 1
+    // of row i (the block has TPR d_k threads)
+    const int i = threadIdx.x / TPR, cb = (threadIdx.x % TPR) * CH;
     const bool act = i < dk;
     const int rows_pb = owner_rows<DV>(dk), r0 = rank * rows_pb;  // rows this block finishes
     __shared__ float s_vh[kTile][kCB], s_do[kTile][kCB], s_part[2][kTile][kMaxRows], s_fin[kMaxRows];
@@ -259,9 +259,9 @@ __global__ void __launch_bounds__(512) simt_bwd_fsweep(BwdParams p, float* dqf, 
     float* s_al = reinterpret_cast<float*>(s_stage + 2 * sbytes);
     float* s_kh = s_al + kTile * dk;
 
-    float s[kCH];
+    float s[CH];
 #pragma unroll
-    for (int j = 0; j < kCH; ++j)
+    for (int j = 0; j < CH; ++j)
         s[j] = (act && p.S0) ? p.S0[((size_t)bh * dk + i) * DV + c0 + cb + j] : 0.0f;
 
     // Tile n: its stage was fetched while tile n - 1 ran; it is unpacked into
@@ -314,15 +314,15 @@ __global__ void __launch_bounds__(512) simt_bwd_fsweep(BwdParams p, float* dqf, 
             const float al = s_al[tt * dk + i], kh = s_kh[tt * dk + i];
             float a0 = 0.0f, a1 = 0.0f;
 #pragma unroll
-            for (int j = 0; j < kCH; j += 2) {
+            for (int j = 0; j < CH; j += 2) {
                 s[j] = fmaf(al, s[j], kh * s_vh[tt][cb + j]);
                 s[j + 1] = fmaf(al, s[j + 1], kh * s_vh[tt][cb + j + 1]);
                 a0 = fmaf(s[j], s_do[tt][cb + j], a0);
                 a1 = fmaf(s[j + 1], s_do[tt][cb + j + 1], a1);
             }
             float a = a0 + a1;
-            a += __shfl_xor_sync(0xffffffffu, a, 1);  // the row's other columns
-            a += __shfl_xor_sync(0xffffffffu, a, 2);
+#pragma unroll
+            for (int o = 1; o < TPR; o <<= 1) a += __shfl_xor_sync(0xffffffffu, a, o);  // the row's other columns
             if (act && cb == 0) s_part[buf][tt][i] = a;
         }
         // this block's partials of the tile are written (s_part alternates by tile:
@@ -355,11 +355,11 @@ __global__ void __launch_bounds__(512) simt_bwd_fsweep(BwdParams p, float* dqf, 
     float f = 0.0f;
     if (act && p.dST) {
 #pragma unroll
-        for (int j = 0; j < kCH; ++j)
+        for (int j = 0; j < CH; ++j)
             f = fmaf(p.dST[((size_t)bh * dk + i) * DV + c0 + cb + j], s[j], f);
     }
-    f += __shfl_xor_sync(0xffffffffu, f, 1);
-    f += __shfl_xor_sync(0xffffffffu, f, 2);
+#pragma unroll
+    for (int o = 1; o < TPR; o <<= 1) f += __shfl_xor_sync(0xffffffffu, f, o);
     if (act && cb == 0) s_fin[i] = f;
     cl.sync();
     for (int row = r0 + threadIdx.x; row < min(dk, r0 + rows_pb); row += blockDim.x) {
@@ -372,18 +372,18 @@ __global__ void __launch_bounds__(512) simt_bwd_fsweep(BwdParams p, float* dqf, 
 }
 
 // ------------------------------------------------ backward, reverse sweep R
-template <typename T, int DV>
+template <typename T, int DV, int TPR>
 __global__ void __launch_bounds__(512) simt_bwd_rsweep(BwdParams p, const float* dqf,
                                                        const float* fin, const int* only) {
-    constexpr int NCB = DV / kCB;
-    static_assert(kCH == 4 && kTPR == 4, "the column reduce-scatter below takes two halving rounds");
+    constexpr int NCB = DV / kCB, CH = kCB / TPR;
+    static_assert(TPR == 4 || TPR == 8, "the column reduce-scatter below takes CH = 4 or 2");
     namespace cg = cooperative_groups;
     cg::cluster_group cl = cg::this_cluster();
     const int rank = (int)cl.block_rank(), bh = blockIdx.x / NCB;
     if (only && only[bh] == 0) return;
     const int T_ = p.T, dk = p.dk, c0 = rank * kCB;
-    // four threads a row, as in sweep F
-    const int i = threadIdx.x / kTPR, cb = (threadIdx.x % kTPR) * kCH;
+    // TPR threads a row, as in sweep F
+    const int i = threadIdx.x / TPR, cb = (threadIdx.x % TPR) * CH;
     const bool act = i < dk;
     const int rows_pb = owner_rows<DV>(dk), r0 = rank * rows_pb;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x / 32;
@@ -415,9 +415,9 @@ __global__ void __launch_bounds__(512) simt_bwd_rsweep(BwdParams p, const float*
     float* s_ah = s_ta + kTile * dk;
     float* s_lg = s_ah + kTile * dk;
 
-    float ds[kCH];
+    float ds[CH];
 #pragma unroll
-    for (int j = 0; j < kCH; ++j)
+    for (int j = 0; j < CH; ++j)
         ds[j] = (act && p.dST) ? p.dST[((size_t)bh * dk + i) * DV + c0 + cb + j] : 0.0f;
     float a_next = 1.0f;  // alpha_{t+1,i}
     for (int rl = threadIdx.x; rl < rows_pb; rl += blockDim.x)
@@ -477,43 +477,37 @@ __global__ void __launch_bounds__(512) simt_bwd_rsweep(BwdParams p, const float*
             const float kh = act ? s_kh[tt * dk + i] : 0.0f;
             float d0 = 0.0f, d1 = 0.0f;
 #pragma unroll
-            for (int j = 0; j < kCH; j += 2) {
+            for (int j = 0; j < CH; j += 2) {
                 ds[j] = fmaf(f, ds[j], qi * s_do[tt][cb + j]);
                 ds[j + 1] = fmaf(f, ds[j + 1], qi * s_do[tt][cb + j + 1]);
                 d0 = fmaf(ds[j], s_vh[tt][cb + j], d0);
                 d1 = fmaf(ds[j + 1], s_vh[tt][cb + j + 1], d1);
             }
             float d = d0 + d1;
-            d += __shfl_xor_sync(0xffffffffu, d, 1);  // the row's other columns
-            d += __shfl_xor_sync(0xffffffffu, d, 2);
-            if (act && cb == 0) s_part[buf][tt][i] = d;  // this block's share of dkhat_{t,i}
-            // dvhat_j = sum_i dS_ij khat_i over the warp's 8 rows (lanes with the same
-            // l mod 4): a reduce-scatter over lane bits 4, 3 (each halving round
-            // sends half of the lane's partial sums to the lane `o` apart and adds
-            // the other half it receives), then a plain sum over bit 2, after which
-            // lanes l and l ^ 4 both hold column cb + col; the warps meet below
-            float x[kCH / 2];
-            const bool up0 = (lane & 16) != 0;
-            int col = up0 ? kCH / 2 : 0;
 #pragma unroll
-            for (int j = 0; j < kCH / 2; ++j) {
-                const float lo = ds[j] * kh, hi = ds[j + kCH / 2] * kh;
+            for (int o = 1; o < TPR; o <<= 1) d += __shfl_xor_sync(0xffffffffu, d, o);  // the row's other columns
+            if (act && cb == 0) s_part[buf][tt][i] = d;  // this block's share of dkhat_{t,i}
+            // dvhat_j = sum_i dS_ij khat_i over the warp's 32 / TPR rows (lanes with
+            // the same l mod TPR): a reduce-scatter over the top lane bits (each
+            // halving round sends half of the lane's partial sums to the lane `o`
+            // apart and adds the other half it receives: bits 4, 3 for CH = 4, bit 4
+            // for CH = 2), then a plain sum over the next bit (TPR), after which
+            // lanes l and l ^ TPR both hold column cb + col; the warps meet below
+            float x[CH / 2];
+            const bool up0 = (lane & 16) != 0;
+            int col = up0 ? CH / 2 : 0;
+#pragma unroll
+            for (int j = 0; j < CH / 2; ++j) {
+                const float lo = ds[j] * kh, hi = ds[j + CH / 2] * kh;
                 x[j] = (up0 ? hi : lo) + __shfl_xor_sync(0xffffffffu, up0 ? lo : hi, 16);
             }
-#pragma unroll
-            for (int r = 1; r < 2; ++r) {
-                const int o = 16 >> r, h = (kCH >> r) / 2;
-                const bool up = (lane & o) != 0;
-#pragma unroll
-                for (int j = 0; j < h; ++j) {
-                    const float send = up ? x[j] : x[j + h];
-                    const float keep = up ? x[j + h] : x[j];
-                    x[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-                }
-                if (up) col += h;
+            if constexpr (CH == 4) {
+                const bool up = (lane & 8) != 0;
+                x[0] = (up ? x[1] : x[0]) + __shfl_xor_sync(0xffffffffu, up ? x[0] : x[1], 8);
+                if (up) col += 1;
             }
-            x[0] += __shfl_xor_sync(0xffffffffu, x[0], 4);
-            if ((lane & 4) == 0) s_red[tt][warp][cb + col] = x[0];
+            x[0] += __shfl_xor_sync(0xffffffffu, x[0], TPR);
+            if ((lane & TPR) == 0) s_red[tt][warp][cb + col] = x[0];
             if (live) a_next = s_al[tt * dk + i];
         }
         // this block's dkhat partials of the tile are written (s_part alternates by
@@ -579,7 +573,7 @@ __global__ void __launch_bounds__(512) simt_bwd_rsweep(BwdParams p, const float*
     }
     if (act && p.dS0) {
 #pragma unroll
-        for (int j = 0; j < kCH; ++j) p.dS0[((size_t)bh * dk + i) * DV + c0 + cb + j] = a_next * ds[j];
+        for (int j = 0; j < CH; ++j) p.dS0[((size_t)bh * dk + i) * DV + c0 + cb + j] = a_next * ds[j];
     }
     cl.sync();  // no block leaves while another still reads its shared memory
 }
@@ -597,8 +591,8 @@ cudaError_t fwd_t(const SeqParams& p, cudaStream_t s) {
     return cudaGetLastError();
 }
 
-template <typename T, int DV>
-cudaError_t bwd_tv(const BwdParams& p, float* dqf, float* fin, const int* only, cudaStream_t s) {
+template <typename T, int DV, int TPR>
+cudaError_t bwd_tvr(const BwdParams& p, float* dqf, float* fin, const int* only, cudaStream_t s) {
     // one cluster of DV / kCB blocks per (b,h)
     constexpr int NCB = DV / kCB;
     // two pipeline stages of dynamic shared memory (sweep R's carry dq too), then
@@ -606,15 +600,15 @@ cudaError_t bwd_tv(const BwdParams& p, float* dqf, float* fin, const int* only, 
     const size_t ga = (size_t)kTile * p.dk * 4;
     const size_t smf = 2 * sweep_stage_bytes<T>(p.dk, false) + 2 * ga;
     const size_t smr = 2 * sweep_stage_bytes<T>(p.dk, true) + 6 * ga;
-    cudaError_t e = cudaFuncSetAttribute(simt_bwd_fsweep<T, DV>,
+    cudaError_t e = cudaFuncSetAttribute(simt_bwd_fsweep<T, DV, TPR>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smf);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(simt_bwd_rsweep<T, DV>,
+        e = cudaFuncSetAttribute(simt_bwd_rsweep<T, DV, TPR>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smr);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(p.B * p.H * NCB));
-    cfg.blockDim = dim3((unsigned)(kTPR * p.dk));
+    cfg.blockDim = dim3((unsigned)(TPR * p.dk));
     cfg.dynamicSmemBytes = smf;
     cfg.stream = s;
     cudaLaunchAttribute at[1];
@@ -624,11 +618,16 @@ cudaError_t bwd_tv(const BwdParams& p, float* dqf, float* fin, const int* only, 
     at[0].val.clusterDim.z = 1;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, simt_bwd_fsweep<T, DV>, p, dqf, fin, only);
+    e = cudaLaunchKernelEx(&cfg, simt_bwd_fsweep<T, DV, TPR>, p, dqf, fin, only);
     if (e != cudaSuccess) return e;
     cfg.dynamicSmemBytes = smr;
-    return cudaLaunchKernelEx(&cfg, simt_bwd_rsweep<T, DV>, p, static_cast<const float*>(dqf),
+    return cudaLaunchKernelEx(&cfg, simt_bwd_rsweep<T, DV, TPR>, p, static_cast<const float*>(dqf),
                               static_cast<const float*>(fin), only);
+}
+
+template <typename T, int DV>
+cudaError_t bwd_tv(const BwdParams& p, float* dqf, float* fin, const int* only, cudaStream_t s) {
+    return p.dk <= 64 ? bwd_tvr<T, DV, 8>(p, dqf, fin, only, s) : bwd_tvr<T, DV, 4>(p, dqf, fin, only, s);
 }
 
 template <typename T>
