@@ -119,3 +119,29 @@ def test_workload3_backward_sampled(cuda_ok):
         ref = oracle.bwd(*(xs[n] for n in SEQ), xs["S0"], xs["dO"])
         for n in GR:
             assert_close(gr[n][b:b + 1, h:h + 1], ref[n], TOL, f"head ({b},{h}) {n}")
+
+
+@pytest.mark.parametrize("dv", [64, 128])
+def test_tc_backward_wide_decay_preact_feedthrough(cuda_ok, dv):
+    """A wide head under gates passed before their activations and with the
+    feedthrough: the exact re-run then activates g, tau and beta itself, takes
+    the chain factors to the pre-activations and adds the feedthrough's term to
+    dv."""
+    from tests.test_gpu_feedthrough import feed_weights
+    T = 64 * 3 + 17
+    x = draw_sequence(1, 3, T, 64, dv, torch.bfloat16, seed=31 + dv, s0_std=0.1, with_dO=True,
+                      preact=True)
+    g = x["g"].float()
+    g[:, 1, 70:110] = g[:, 1, 70:110] * 4.0 + 12.0  # softplus ~ 12: one chunk of head 1 is wide
+    x["g"] = g.to(torch.bfloat16)
+    d = feed_weights(3, dv, 31 + dv)
+    dST = 0.1 * torch.randn(1, 3, 64, dv, generator=torch.Generator().manual_seed(dv))
+    dx = {n: (t.cuda() if t is not None else None) for n, t in x.items()}
+    gr = rdm.rdm_ddts_bwd(*(dx[n] for n in SEQ), dx["S0"], dx["dO"], dST.cuda(), impl="tc",
+                          gates="preact", feedthrough=d.cuda())
+    torch.cuda.synchronize()
+    assert rdm.rdm_ddts_sync_status() == rdm.RDM_OK
+    ref = oracle.bwd(*(x[n] for n in SEQ), x["S0"], x["dO"], dST, preact=True, d=d)
+    for n in GR:
+        assert_close(gr[n], ref[n], TOL, f"wide head, preact, feedthrough: {n}")
+    assert_close(gr["dfeed"], ref["dd"], TOL, "wide head: grad of the feedthrough weights")
