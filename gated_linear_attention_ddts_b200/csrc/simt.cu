@@ -8,8 +8,9 @@
 // along d_k per the paperhub.cn rebuttal "Efficient Parallelization" bullet.)
 //
 // Backward, exact reverse mode organised in two sweeps per (b,h), each run by a
-// cluster of blocks that split the state's columns, threads 4i ... 4i+3 owning
-// row i of their block's columns of the state or of its gradient:
+// cluster of blocks that split the state's columns, TPR consecutive threads (8,
+// or 4 at d_k = 128) owning row i of their block's columns of the state or of
+// its gradient:
 //   sweep F (forward in t):  S_t, dq_t = S_t dO_t (kept in float32 scratch too);
 //   sweep R (reverse in t):  dS_t = q_t dO_t^T + diag(alpha_{t+1}) dS_{t+1},
 //                            dkhat_t = dS_t vhat_t, dvhat_t = dS_t^T khat_t.
@@ -99,8 +100,10 @@ __global__ void __launch_bounds__(128) simt_fwd_kernel(SeqParams p) {
 // here, dkhat_t in sweep R) need the whole cluster; each block writes its
 // partial sums of a tile of tokens into its shared memory, and after one cluster
 // barrier per tile the block that owns a row adds the partials of every block
-// through distributed shared memory.  The inputs of a tile are fetched one tile
-// ahead with asynchronous copies, so their latency overlaps the tile before.
+// through distributed shared memory, one (row, token) a thread.  The inputs of a
+// tile are fetched one tile ahead with asynchronous copies, so their latency
+// overlaps the tile before, and the tile's gate arithmetic is done once per
+// (token, row) by the whole block before its token loop.
 constexpr int kCB = 16;      // state columns per block
 // Threads a row, TPR (a template parameter: 8 for d_k <= 64, 4 for d_k = 128,
 // so a block has at most 512 threads), each running CH = kCB / TPR columns.
@@ -110,22 +113,6 @@ template <int DV>
 __device__ __forceinline__ int owner_rows(int dk) {
     constexpr int NCB = DV / kCB;
     return (dk + NCB - 1) / NCB;
-}
-
-// out[tt] = sum over the cluster's blocks r of their s_part[.][tt][row] (`mine`
-// points at this block's element for tt = 0; tokens are kMaxRows apart).  All
-// NCB * kTile distributed shared-memory loads are issued before any sum is used.
-template <int NCB>
-__device__ __forceinline__ void cluster_row_sums(cooperative_groups::cluster_group& cl,
-                                                 float* mine, float (&out)[kTile]) {
-#pragma unroll
-    for (int tt = 0; tt < kTile; ++tt) out[tt] = 0.0f;
-#pragma unroll
-    for (int r = 0; r < NCB; ++r) {
-        const float* part = cl.map_shared_rank(mine, r);
-#pragma unroll
-        for (int tt = 0; tt < kTile; ++tt) out[tt] += part[tt * kMaxRows];
-    }
 }
 
 __host__ __device__ __forceinline__ int ntiles_of(int T) { return (T + kTile - 1) / kTile; }
