@@ -117,6 +117,25 @@ __device__ __forceinline__ int owner_rows(int dk) {
 
 __host__ __device__ __forceinline__ int ntiles_of(int T) { return (T + kTile - 1) / kTile; }
 
+// Sequence segments of the sweeps.  A head's tokens are cut into P segments of
+// seg_len tokens (a multiple of kTile; the last one may be shorter), run by P
+// clusters side by side.  Both recurrences are affine across a segment:
+//   sweep F:  S_out = diag(e^L) S_in + S_loc,
+//   sweep R:  C_out = diag(e^L) C_in + C_loc,  C = alpha_{t+1} o dS_{t+1} at a cut,
+// with L the sum of log alpha over the segment's tokens and S_loc, C_loc the
+// results from a zero start.  So a pass computes S_loc / C_loc and L of every
+// segment (mode kSegLocal), and the full pass (kSegFull) of a segment folds the
+// maps before it (F) or after it (R) onto S_0 / dS_T and runs from there.  The decay-gradient carry into segment j from later segments,
+// fin + sum over later segments of their dG totals, is added afterwards to dg
+// and dtau of segment j by a fix-up launch.  P = 1 is the plain sweep.
+enum { kSegWhole = 0, kSegLocal = 1, kSegFull = 2 };
+struct SimtSeg {
+    int P, seg_len, mode;
+    float* Sx;   // [B H][P][d_k][d_v]: S_loc (sweep F), then C_loc (sweep R)
+    float* La;   // [B H][P][d_k]: sum of log alpha over the segment
+    float* tot;  // [B H][P][d_k]: the segment's sum of dG (sweep R)
+};
+
 // the two halves of a cluster barrier: arrive (releasing this thread's earlier
 // writes, shared memory included) and wait (acquiring those of every thread
 // that arrived); every thread of every block takes both
@@ -216,15 +235,18 @@ __device__ __forceinline__ void sweep_fetch(const SweepStage<T>& st, const T* co
     }
 }
 
+// Sweep F of head bh, segment sj, by this cluster.
 template <typename T, int DV, int TPR>
-__global__ void __launch_bounds__(512) simt_bwd_fsweep(BwdParams p, float* dqf, float* fin,
-                                                       const int* only) {
+__device__ __forceinline__ void fsweep_head(const BwdParams& p, float* dqf, float* fin,
+                                            const SimtSeg& sg, int bh, int sj) {
     constexpr int NCB = DV / kCB, CH = kCB / TPR;
     namespace cg = cooperative_groups;
     cg::cluster_group cl = cg::this_cluster();
-    const int rank = (int)cl.block_rank(), bh = blockIdx.x / NCB;
-    if (only && only[bh] == 0) return;  // head already handled by the tensor-core path
+    const int rank = (int)cl.block_rank(), cid = bh * sg.P + sj;
+    if (sg.mode == kSegLocal && sj == sg.P - 1) return;  // the last segment's map is never used
+    const bool local = sg.mode == kSegLocal;
     const int T_ = p.T, dk = p.dk, c0 = rank * kCB;
+    const int sa = sj * sg.seg_len, sb = min(T_, sa + sg.seg_len);  // this segment's tokens
     // TPR threads a row: thread TPR i + h runs columns c0 + CH h ... c0 + CH (h + 1) - 1
     // of row i (the block has TPR d_k threads)
     const int i = threadIdx.x / TPR, cb = (threadIdx.x % TPR) * CH;
@@ -245,27 +267,41 @@ __global__ void __launch_bounds__(512) simt_bwd_fsweep(BwdParams p, float* dqf, 
     // khat = alpha_hat k (1 and 0 past the end of a partial tile)
     float* s_al = reinterpret_cast<float*>(s_stage + 2 * sbytes);
     float* s_kh = s_al + kTile * dk;
+    float* s_la = s_kh + kTile * dk;  // log alpha (0 past the end), for a local pass
+    float* Sx = sg.Sx + ((size_t)cid * dk + i) * DV + c0 + cb;  // this thread's part of the segment's slot
 
-    float s[CH];
+    // the segment's entry state: zero for a local pass, else S_0 folded through
+    // the maps of the segments before this one (S_in(j+1) = diag(e^{L_j}) S_in(j)
+    // + S_loc(j); none for the whole sequence or the first segment)
+    float s[CH], lsum = 0.0f;
 #pragma unroll
     for (int j = 0; j < CH; ++j)
-        s[j] = (act && p.S0) ? p.S0[((size_t)bh * dk + i) * DV + c0 + cb + j] : 0.0f;
+        s[j] = !act || local || !p.S0 ? 0.0f : p.S0[((size_t)bh * dk + i) * DV + c0 + cb + j];
+    if (act && !local) {
+        for (int jj = 0; jj < sj; ++jj) {
+            const size_t slot = (size_t)bh * sg.P + jj;
+            const float e = expf(sg.La[slot * dk + i]);
+            const float* loc = sg.Sx + (slot * dk + i) * DV + c0 + cb;
+#pragma unroll
+            for (int j = 0; j < CH; ++j) s[j] = fmaf(e, s[j], loc[j]);
+        }
+    }
 
     // Tile n: its stage was fetched while tile n - 1 ran; it is unpacked into
     // s_vh, s_do and the gate arrays before the cluster waits for the partial
     // sums of tile n - 1, so that wait overlaps the unpacking.
     auto fetch = [&](int m) {  // starts tile m's copies (an empty group past the end)
-        if (m < ntiles_of(T_)) {
-            const int tm = m * kTile;
+        if (m < ntiles_of(sb - sa)) {
+            const int tm = sa + m * kTile;
             sweep_fetch<T, DV>(sweep_stage<T>(s_stage + (m & 1) * sbytes, dk, false), rows, nullptr,
-                               cols, tm, min(kTile, T_ - tm), dk);
+                               cols, tm, min(kTile, sb - tm), dk);
         } else {
             cp_async_commit();
         }
     };
     auto unpack = [&](int m) {  // after tile m's copies are complete and visible
         const SweepStage<T> cur = sweep_stage<T>(s_stage + (m & 1) * sbytes, dk, false);
-        const int nt_m = min(kTile, T_ - m * kTile);
+        const int nt_m = min(kTile, sb - sa - m * kTile);
         for (int idx = threadIdx.x; idx < kTile * kCB; idx += blockDim.x) {
             const float bb = ldf(cur.col[0] + idx);
             s_vh[idx / kCB][idx % kCB] = (p.preact ? sigmoid_acc(bb) : bb) * ldf(cur.col[1] + idx);
@@ -281,9 +317,10 @@ __global__ void __launch_bounds__(512) simt_bwd_fsweep(BwdParams p, float* dqf, 
             const bool live = e / dk < nt_m;
             s_al[e] = live ? alpha(gg, ta) : 1.0f;
             s_kh[e] = live ? alpha_hat(gg, ta) * ldf(cur.row[2] + e) : 0.0f;
+            s_la[e] = live ? log_alpha(gg, ta) : 0.0f;
         }
     };
-    const int ntiles = ntiles_of(T_);
+    const int ntiles = ntiles_of(sb - sa);
     if (ntiles > 0) {
         fetch(0);
         fetch(1);
@@ -293,7 +330,25 @@ __global__ void __launch_bounds__(512) simt_bwd_fsweep(BwdParams p, float* dqf, 
         __syncthreads();
     }
     for (int n = 0; n < ntiles; ++n) {
-        const int t0 = n * kTile, nt = min(kTile, T_ - t0), buf = n & 1;
+        const int t0 = sa + n * kTile, nt = min(kTile, sb - t0), buf = n & 1;
+        if (local) {
+            // the segment's map only: the state from zero and the sum of log alpha
+#pragma unroll
+            for (int tt = 0; tt < kTile; ++tt) {
+                const float al = s_al[tt * dk + i], kh = s_kh[tt * dk + i];
+                lsum += s_la[tt * dk + i];
+#pragma unroll
+                for (int j = 0; j < CH; ++j) s[j] = fmaf(al, s[j], kh * s_vh[tt][cb + j]);
+            }
+            if (n + 1 < ntiles) {
+                fetch(n + 2);
+                cp_async_wait_prev();
+                __syncthreads();
+                unpack(n + 1);
+                __syncthreads();
+            }
+            continue;
+        }
         // the tile's tokens as one straight run (a token past the end of a partial
         // tile leaves the state as it is: alpha 1, khat 0)
 #pragma unroll
@@ -338,6 +393,18 @@ __global__ void __launch_bounds__(512) simt_bwd_fsweep(BwdParams p, float* dqf, 
             }
         }
     }
+    if (local) {  // the segment's map: S_loc (this thread's columns) and L (its row)
+        if (act) {
+#pragma unroll
+            for (int j = 0; j < CH; ++j) Sx[j] = s[j];
+            if (cb == 0) sg.La[(size_t)cid * dk + i] = lsum;
+        }
+        return;
+    }
+    if (sj != sg.P - 1) {
+        cl.sync();  // no block leaves while another still reads its shared memory
+        return;
+    }
     // rowsum(dS_T o S_T), the decay gradient's term at u = T
     float f = 0.0f;
     if (act && p.dST) {
@@ -359,16 +426,19 @@ __global__ void __launch_bounds__(512) simt_bwd_fsweep(BwdParams p, float* dqf, 
 }
 
 // ------------------------------------------------ backward, reverse sweep R
+// Sweep R of head bh, segment sj, by this cluster.
 template <typename T, int DV, int TPR>
-__global__ void __launch_bounds__(512) simt_bwd_rsweep(BwdParams p, const float* dqf,
-                                                       const float* fin, const int* only) {
+__device__ __forceinline__ void rsweep_head(const BwdParams& p, const float* dqf, const float* fin,
+                                            const SimtSeg& sg, int bh, int sj) {
     constexpr int NCB = DV / kCB, CH = kCB / TPR;
     static_assert(TPR == 4 || TPR == 8, "the column reduce-scatter below takes CH = 4 or 2");
     namespace cg = cooperative_groups;
     cg::cluster_group cl = cg::this_cluster();
-    const int rank = (int)cl.block_rank(), bh = blockIdx.x / NCB;
-    if (only && only[bh] == 0) return;
+    const int rank = (int)cl.block_rank(), cid = bh * sg.P + sj;
+    if (sg.mode == kSegLocal && sj == 0) return;  // the first segment's map is never used
+    const bool local = sg.mode == kSegLocal;
     const int T_ = p.T, dk = p.dk, c0 = rank * kCB;
+    const int sa = sj * sg.seg_len, sb = min(T_, sa + sg.seg_len);  // this segment's tokens
     // TPR threads a row, as in sweep F
     const int i = threadIdx.x / TPR, cb = (threadIdx.x % TPR) * CH;
     const bool act = i < dk;
@@ -402,26 +472,43 @@ __global__ void __launch_bounds__(512) simt_bwd_rsweep(BwdParams p, const float*
     float* s_ah = s_ta + kTile * dk;
     float* s_lg = s_ah + kTile * dk;
 
-    float ds[CH];
+    float* Sx = sg.Sx + ((size_t)cid * dk + i) * DV + c0 + cb;  // this thread's part of the segment's slot
+
+    // the gradient flowing in at the segment's end: zero for a local pass, else
+    // dS_T (alpha_{T+1} taken as 1) folded through the maps of the segments after
+    // this one (C_in(j-1) = diag(e^{L_j}) C_in(j) + C_loc(j))
+    float ds[CH], lsum = 0.0f;
 #pragma unroll
     for (int j = 0; j < CH; ++j)
-        ds[j] = (act && p.dST) ? p.dST[((size_t)bh * dk + i) * DV + c0 + cb + j] : 0.0f;
+        ds[j] = !act || local || !p.dST ? 0.0f : p.dST[((size_t)bh * dk + i) * DV + c0 + cb + j];
+    if (act && !local) {
+        for (int jj = sg.P - 1; jj > sj; --jj) {
+            const size_t slot = (size_t)bh * sg.P + jj;
+            const float e = expf(sg.La[slot * dk + i]);
+            const float* loc = sg.Sx + (slot * dk + i) * DV + c0 + cb;
+#pragma unroll
+            for (int j = 0; j < CH; ++j) ds[j] = fmaf(e, ds[j], loc[j]);
+        }
+    }
     float a_next = 1.0f;  // alpha_{t+1,i}
+    // the carry fin + later segments' dG enters the last segment here; the other
+    // segments' carries are added by the fix-up launch
+    const bool last = sj == sg.P - 1;
     for (int rl = threadIdx.x; rl < rows_pb; rl += blockDim.x)
-        s_da[rl] = r0 + rl < dk ? fin[(size_t)bh * dk + r0 + rl] : 0.0f;
+        s_da[rl] = r0 + rl < dk && last ? fin[(size_t)bh * dk + r0 + rl] : 0.0f;
 
-    // tile n holds tokens [t1 - kTile, t1) with t1 = T - n kTile (the last one
+    // tile n holds tokens [t1 - kTile, t1) with t1 = sb - n kTile (the last one
     // processed may be partial)
-    const int ntiles = ntiles_of(T_);
+    const int ntiles = ntiles_of(sb - sa);
     if (ntiles > 0)
-        sweep_fetch<T, DV>(sweep_stage<T>(s_stage, dk, true), rows, dqf_bh, cols, max(0, T_ - kTile),
-                           min(kTile, T_), dk);
+        sweep_fetch<T, DV>(sweep_stage<T>(s_stage, dk, true), rows, dqf_bh, cols, max(sa, sb - kTile),
+                           min(kTile, sb - sa), dk);
     for (int n = 0; n < ntiles; ++n) {
-        const int t1 = T_ - n * kTile, t0 = max(0, t1 - kTile), nt = t1 - t0, buf = n & 1;
+        const int t1 = sb - n * kTile, t0 = max(sa, t1 - kTile), nt = t1 - t0, buf = n & 1;
         const SweepStage<T> cur = sweep_stage<T>(s_stage + buf * sbytes, dk, true);
         if (n + 1 < ntiles)
             sweep_fetch<T, DV>(sweep_stage<T>(s_stage + (buf ^ 1) * sbytes, dk, true), rows, dqf_bh,
-                               cols, max(0, t0 - kTile), min(kTile, t0), dk);
+                               cols, max(sa, t0 - kTile), min(kTile, t0 - sa), dk);
         else
             cp_async_commit();
         cp_async_wait_prev();
@@ -454,6 +541,23 @@ __global__ void __launch_bounds__(512) simt_bwd_rsweep(BwdParams p, const float*
             s_lg[e] = lg;
         }
         __syncthreads();
+        if (local) {
+            // the segment's map only: dS from zero and the sum of log alpha
+#pragma unroll
+            for (int tt = kTile - 1; tt >= 0; --tt) {
+                const bool live = tt < nt;
+                const float f = live ? a_next : 1.0f;
+                const float qi = act ? ldf(cur.row[3] + tt * dk + i) : 0.0f;
+#pragma unroll
+                for (int j = 0; j < CH; ++j) ds[j] = fmaf(f, ds[j], qi * s_do[tt][cb + j]);
+                if (live) {
+                    lsum += log_alpha(s_gg[tt * dk + i], s_ta[tt * dk + i]);
+                    a_next = s_al[tt * dk + i];
+                }
+            }
+            __syncthreads();  // the staging buffers and gate arrays are free for the next tile
+            continue;
+        }
         // the tile's tokens as one straight run, as in sweep F (a token past the end
         // of a partial tile leaves dS as it is: factor 1, no q dO^T term)
 #pragma unroll
@@ -558,9 +662,23 @@ __global__ void __launch_bounds__(512) simt_bwd_rsweep(BwdParams p, const float*
         }
         __syncthreads();  // the staging buffers, gate arrays and s_red are free for the next tile
     }
-    if (act && p.dS0) {
+    if (local) {  // the segment's map: C_loc = alpha_{first} o dS_{first} and L
+        if (act) {
+#pragma unroll
+            for (int j = 0; j < CH; ++j) Sx[j] = a_next * ds[j];
+            if (cb == 0) sg.La[(size_t)cid * dk + i] = lsum;
+        }
+        return;
+    }
+    if (act && p.dS0 && sj == 0) {
 #pragma unroll
         for (int j = 0; j < CH; ++j) p.dS0[((size_t)bh * dk + i) * DV + c0 + cb + j] = a_next * ds[j];
+    }
+    if (sg.mode == kSegFull) {  // the segment's sum of dG, for the carries of earlier segments
+        for (int rl = threadIdx.x; rl < rows_pb; rl += blockDim.x)
+            if (r0 + rl < dk)
+                sg.tot[(size_t)cid * dk + r0 + rl] =
+                    s_da[rl] - (last ? fin[(size_t)bh * dk + r0 + rl] : 0.0f);
     }
     cl.sync();  // no block leaves while another still reads its shared memory
 }
@@ -578,55 +696,165 @@ cudaError_t fwd_t(const SeqParams& p, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+// Programmatic dependent launch: a launch of the chain below may start while
+// the one before it is finishing (its blocks then wait in chain_enter until that
+// grid has completed and its writes are visible); a block lets the next launch
+// start once it is done (chain_leave), so the waiting blocks never hold an SM
+// that a working block of this launch could use.
+__device__ __forceinline__ void chain_enter() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void chain_leave() {
+    asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+
+// The sweep kernels: cluster c takes segment c % P of the heads slot, slot +
+// slots, ... (slot = c / P) of `list` (list[0] heads, then their indices; every
+// head when list is null).  The tensor-core backward lists only the heads it
+// flagged, so a few slots cover them and the launch stays small.
 template <typename T, int DV, int TPR>
-cudaError_t bwd_tvr(const BwdParams& p, float* dqf, float* fin, const int* only, cudaStream_t s) {
-    // one cluster of DV / kCB blocks per (b,h)
+__global__ void __launch_bounds__(512) simt_bwd_fsweep(const BwdParams p, float* dqf, float* fin,
+                                                       const int* list, int slots, const SimtSeg sg) {
+    chain_enter();
+    const int c = blockIdx.x / (DV / kCB), slot = c / sg.P, sj = c % sg.P;
+    const int nheads = list ? list[0] : p.B * p.H;
+    for (int q = slot; q < nheads; q += slots) {
+        fsweep_head<T, DV, TPR>(p, dqf, fin, sg, list ? list[1 + q] : q, sj);
+        __syncthreads();
+    }
+    chain_leave();
+}
+
+template <typename T, int DV, int TPR>
+__global__ void __launch_bounds__(512) simt_bwd_rsweep(const BwdParams p, const float* dqf,
+                                                       const float* fin, const int* list, int slots,
+                                                       const SimtSeg sg) {
+    chain_enter();
+    const int c = blockIdx.x / (DV / kCB), slot = c / sg.P, sj = c % sg.P;
+    const int nheads = list ? list[0] : p.B * p.H;
+    for (int q = slot; q < nheads; q += slots) {
+        rsweep_head<T, DV, TPR>(p, dqf, fin, sg, list ? list[1 + q] : q, sj);
+        __syncthreads();
+    }
+    chain_leave();
+}
+
+// list[0] = the number of flagged heads, list[1..] their indices (one block).
+__global__ void simt_flag_list(const int* flags, int BH, int* list) {
+    __shared__ int n;
+    if (threadIdx.x == 0) n = 0;
+    __syncthreads();
+    for (int bh = threadIdx.x; bh < BH; bh += blockDim.x)
+        if (flags[bh] != 0) list[1 + atomicAdd(&n, 1)] = bh;
+    __syncthreads();
+    if (threadIdx.x == 0) list[0] = n;
+}
+
+// One sweep launch (F when `rev` is false, R when true) in the segment mode of `sg`.
+template <typename T, int DV, int TPR>
+cudaError_t bwd_tvr(const BwdParams& p, float* dqf, float* fin, const int* list, int slots,
+                    const SimtSeg& sg, bool rev, cudaStream_t s) {
+    // one cluster of DV / kCB blocks per (b,h) and segment
     constexpr int NCB = DV / kCB;
     // two pipeline stages of dynamic shared memory (sweep R's carry dq too), then
-    // the tile's gate arrays (two in sweep F, six in sweep R)
+    // the tile's gate arrays (three in sweep F, six in sweep R)
     const size_t ga = (size_t)kTile * p.dk * 4;
-    const size_t smf = 2 * sweep_stage_bytes<T>(p.dk, false) + 2 * ga;
-    const size_t smr = 2 * sweep_stage_bytes<T>(p.dk, true) + 6 * ga;
-    cudaError_t e = cudaFuncSetAttribute(simt_bwd_fsweep<T, DV, TPR>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smf);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(simt_bwd_rsweep<T, DV, TPR>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smr);
+    const size_t sm = rev ? 2 * sweep_stage_bytes<T>(p.dk, true) + 6 * ga
+                          : 2 * sweep_stage_bytes<T>(p.dk, false) + 3 * ga;
+    cudaError_t e = rev ? cudaFuncSetAttribute(simt_bwd_rsweep<T, DV, TPR>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm)
+                        : cudaFuncSetAttribute(simt_bwd_fsweep<T, DV, TPR>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(p.B * p.H * NCB));
+    cfg.gridDim = dim3((unsigned)(slots * sg.P * NCB));
     cfg.blockDim = dim3((unsigned)(TPR * p.dk));
-    cfg.dynamicSmemBytes = smf;
+    cfg.dynamicSmemBytes = sm;
     cfg.stream = s;
-    cudaLaunchAttribute at[1];
+    cudaLaunchAttribute at[2];
     at[0].id = cudaLaunchAttributeClusterDimension;
     at[0].val.clusterDim.x = NCB;
     at[0].val.clusterDim.y = 1;
     at[0].val.clusterDim.z = 1;
+    at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = at;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, simt_bwd_fsweep<T, DV, TPR>, p, dqf, fin, only);
-    if (e != cudaSuccess) return e;
-    cfg.dynamicSmemBytes = smr;
-    return cudaLaunchKernelEx(&cfg, simt_bwd_rsweep<T, DV, TPR>, p, static_cast<const float*>(dqf),
-                              static_cast<const float*>(fin), only);
+    cfg.numAttrs = 2;
+    if (rev)
+        return cudaLaunchKernelEx(&cfg, simt_bwd_rsweep<T, DV, TPR>, p, static_cast<const float*>(dqf),
+                                  static_cast<const float*>(fin), list, slots, sg);
+    return cudaLaunchKernelEx(&cfg, simt_bwd_fsweep<T, DV, TPR>, p, dqf, fin, list, slots, sg);
 }
 
 template <typename T, int DV>
-cudaError_t bwd_tv(const BwdParams& p, float* dqf, float* fin, const int* only, cudaStream_t s) {
-    return p.dk <= 64 ? bwd_tvr<T, DV, 8>(p, dqf, fin, only, s) : bwd_tvr<T, DV, 4>(p, dqf, fin, only, s);
+cudaError_t bwd_tv(const BwdParams& p, float* dqf, float* fin, const int* list, int slots,
+                   const SimtSeg& sg, bool rev, cudaStream_t s) {
+    return p.dk <= 64 ? bwd_tvr<T, DV, 8>(p, dqf, fin, list, slots, sg, rev, s)
+                      : bwd_tvr<T, DV, 4>(p, dqf, fin, list, slots, sg, rev, s);
 }
 
 template <typename T>
-cudaError_t bwd_t(const BwdParams& p, float* dqf, float* fin, const int* only, cudaStream_t s) {
+cudaError_t bwd_t(const BwdParams& p, float* dqf, float* fin, const int* list, int slots,
+                  const SimtSeg& sg, bool rev, cudaStream_t s) {
     switch (p.dv) {
-        case 16: return bwd_tv<T, 16>(p, dqf, fin, only, s);
-        case 32: return bwd_tv<T, 32>(p, dqf, fin, only, s);
-        case 64: return bwd_tv<T, 64>(p, dqf, fin, only, s);
-        case 128: return bwd_tv<T, 128>(p, dqf, fin, only, s);
+        case 16: return bwd_tv<T, 16>(p, dqf, fin, list, slots, sg, rev, s);
+        case 32: return bwd_tv<T, 32>(p, dqf, fin, list, slots, sg, rev, s);
+        case 64: return bwd_tv<T, 64>(p, dqf, fin, list, slots, sg, rev, s);
+        case 128: return bwd_tv<T, 128>(p, dqf, fin, list, slots, sg, rev, s);
         default: return cudaErrorInvalidValue;
     }
 }
+
+// The fix-up launch: blocks [slot * kFixBlocks, (slot + 1) * kFixBlocks) take the
+// heads slot, slot + slots, ... of the list (as the sweeps do).
+constexpr int kFixBlocks = 16;
+
+__device__ __forceinline__ int listed_heads(const int* list, int BH) { return list ? list[0] : BH; }
+__device__ __forceinline__ int listed_head(const int* list, int q) { return list ? list[1 + q] : q; }
+
+// dg and dtau of every segment but the last, plus the decay-gradient carry into
+// it: fin + the dG sums of all later segments (d log alpha grows by that carry
+// at every token of the segment).  One thread per
+// (t, i) of the head.
+template <typename T>
+__global__ void simt_carry_fix(const BwdParams p, const SimtSeg sg, const float* fin,
+                               const int* list, int slots) {
+    chain_enter();
+    const int dk = p.dk;
+    const int n = min(p.T, (sg.P - 1) * sg.seg_len) * dk;
+    for (int q = blockIdx.x / kFixBlocks; q < listed_heads(list, p.B * p.H); q += slots) {
+        const int bh = listed_head(list, q);
+        for (int e = (blockIdx.x % kFixBlocks) * blockDim.x + threadIdx.x; e < n;
+             e += kFixBlocks * blockDim.x) {
+            const int i = e % dk, t = e / dk;
+            float carry = fin[(size_t)bh * dk + i];
+            for (int j = t / sg.seg_len + 1; j < sg.P; ++j)
+                carry += sg.tot[((size_t)bh * sg.P + j) * dk + i];
+            const size_t off = ((size_t)bh * p.T + t) * dk + i;
+            const float g_in = ldf(static_cast<const T*>(p.g) + off);
+            const float t_in = ldf(static_cast<const T*>(p.tau) + off);
+            const float gg = p.preact ? softplus_acc(g_in) : g_in;
+            const float ta = p.preact ? sigmoid_acc(t_in) : t_in;
+            const float cg = p.preact ? sigmoid_acc(g_in) : 1.0f;
+            const float ct = p.preact ? ta * (1.0f - ta) : 1.0f;
+            T* dg = static_cast<T*>(p.dg) + off;
+            T* dtau = static_cast<T*>(p.dtau) + off;
+            stf(dg, ldf(dg) - cg * ta * carry);
+            stf(dtau, ldf(dtau) - ct * gg * carry);
+        }
+    }
+}
+
+// Segments of the exact backward: P = min(8, T / 512) for T >= 1024 (segments of
+// at least 512 tokens), seg_len a whole number of tiles; the count actually used
+// is the number of non-empty segments.
+void simt_segments(int T, int* P, int* seg_len) {
+    const int want = T >= 1024 ? min(8, T / 512) : 1;
+    const int tiles = ntiles_of(T);
+    const int len = max(1, (tiles + want - 1) / want) * kTile;
+    *P = max(1, (T + len - 1) / len);
+    *seg_len = *P > 1 ? len : max(T, 1);
+}
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
 }  // namespace
 
@@ -635,20 +863,83 @@ cudaError_t launch_simt_fwd(const SeqParams& p, cudaStream_t s) {
     return p.bf16 ? fwd_t<__nv_bfloat16>(p, s) : fwd_t<float>(p, s);
 }
 
-// scratch: dq for every (b,h,t,i) and the final-state term per (b,h,i), float32
+// scratch, float32: dq for every (b,h,t,i), the final-state term per (b,h,i), the
+// flagged-head list (int32) and, with segments, the segments' state slots [B H][P][d_k][d_v], their sums of log
+// alpha and of dG [B H][P][d_k]
 size_t simt_bwd_workspace(const BwdParams& p) {
+    int P, len;
+    simt_segments(p.T, &P, &len);
     const size_t rows = (size_t)p.B * p.H * p.dk;
-    const size_t a = ((rows * (size_t)p.T * 4) + 255) / 256 * 256;
-    return a + rows * 4;
+    size_t w = align256(rows * (size_t)p.T * 4) + align256(rows * 4) +
+               align256((size_t)(p.B * p.H + 1) * 4);  // the flagged-head list
+    if (P > 1) w += align256(rows * P * (size_t)p.dv * 4) + 2 * align256(rows * P * 4);
+    return w;
 }
 
-static cudaError_t simt_bwd(const BwdParams& p, const int* only, cudaStream_t s) {
+// heads a launch of the flagged re-run covers side by side (more flagged heads
+// run in turn)
+constexpr int kFlaggedSlots = 8;
+
+static cudaError_t simt_bwd(const BwdParams& p, const int* flags, cudaStream_t s) {
     if (p.B * p.H == 0) return cudaSuccess;
-    const size_t rows = (size_t)p.B * p.H * p.dk;
-    const size_t a = ((rows * (size_t)p.T * 4) + 255) / 256 * 256;
-    float* dqf = static_cast<float*>(p.ws);
-    float* fin = reinterpret_cast<float*>(static_cast<char*>(p.ws) + a);
-    return p.bf16 ? bwd_t<__nv_bfloat16>(p, dqf, fin, only, s) : bwd_t<float>(p, dqf, fin, only, s);
+    int P, len;
+    simt_segments(p.T, &P, &len);
+    const int BH = p.B * p.H;
+    const size_t rows = (size_t)BH * p.dk;
+    char* w = static_cast<char*>(p.ws);
+    float* dqf = reinterpret_cast<float*>(w);
+    w += align256(rows * (size_t)p.T * 4);
+    float* fin = reinterpret_cast<float*>(w);
+    w += align256(rows * 4);
+    int* list = nullptr;
+    int slots = BH;
+    if (flags) {  // the flagged heads, listed on the device
+        list = reinterpret_cast<int*>(w);
+        w += align256((size_t)(BH + 1) * 4);
+        slots = BH < kFlaggedSlots ? BH : kFlaggedSlots;
+        simt_flag_list<<<1, 256, 0, s>>>(flags, BH, list);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    SimtSeg sg = {P, len, kSegWhole, nullptr, nullptr, nullptr};
+    auto sweep = [&](bool rev) {
+        return p.bf16 ? bwd_t<__nv_bfloat16>(p, dqf, fin, list, slots, sg, rev, s)
+                      : bwd_t<float>(p, dqf, fin, list, slots, sg, rev, s);
+    };
+    if (P == 1) {
+        cudaError_t e = sweep(false);
+        return e != cudaSuccess ? e : sweep(true);
+    }
+    sg.Sx = reinterpret_cast<float*>(w);
+    w += align256(rows * P * (size_t)p.dv * 4);
+    sg.La = reinterpret_cast<float*>(w);
+    w += align256(rows * P * 4);
+    sg.tot = reinterpret_cast<float*>(w);
+    const unsigned fgrid = (unsigned)(slots * kFixBlocks);
+    cudaError_t e;
+    // local maps of sweep F, full passes (each folding the maps before it), the
+    // same for sweep R, then the decay-gradient carries
+    sg.mode = kSegLocal;
+    if ((e = sweep(false)) != cudaSuccess) return e;
+    sg.mode = kSegFull;
+    if ((e = sweep(false)) != cudaSuccess) return e;
+    sg.mode = kSegLocal;
+    if ((e = sweep(true)) != cudaSuccess) return e;
+    sg.mode = kSegFull;
+    if ((e = sweep(true)) != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(fgrid);
+    cfg.blockDim = dim3(256);
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return p.bf16 ? cudaLaunchKernelEx(&cfg, simt_carry_fix<__nv_bfloat16>, p, sg,
+                                       static_cast<const float*>(fin), static_cast<const int*>(list), slots)
+                  : cudaLaunchKernelEx(&cfg, simt_carry_fix<float>, p, sg, static_cast<const float*>(fin),
+                                       static_cast<const int*>(list), slots);
 }
 
 cudaError_t launch_simt_bwd(const BwdParams& p, cudaStream_t s) { return simt_bwd(p, nullptr, s); }

@@ -115,3 +115,21 @@ def test_empty_sequence(cuda_ok):
 
 def test_sync_status_clean(cuda_ok):
     assert rdm.rdm_ddts_sync_status() == rdm.RDM_OK
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("dk,dv,T", [(16, 32, 1024 + 37), (64, 128, 2100)])
+def test_simt_backward_segmented(cuda_ok, dtype, dk, dv, T):
+    """Sequences of 1024 tokens and more run the exact backward in segments (two
+    and four here): local maps, folds, full passes and the carry fix-up."""
+    x = draw_sequence(1, 2, T, dk, dv, dtype, seed=250 + T, s0_std=0.1, with_dO=True)
+    dST = torch.randn(1, 2, dk, dv, generator=torch.Generator().manual_seed(6)) * 0.1
+    d = dev_inputs(x)
+    gr = rdm.rdm_ddts_bwd(d["q"], d["k"], d["v"], d["g"], d["tau"], d["beta"], d["S0"],
+                          d["dO"], dST.cuda(), impl="simt")
+    torch.cuda.synchronize()
+    assert rdm.rdm_ddts_sync_status() == rdm.RDM_OK
+    ref = oracle.bwd(x["q"], x["k"], x["v"], x["g"], x["tau"], x["beta"], x["S0"], x["dO"],
+                     dST)
+    for n in ("dq", "dk", "dv", "dg", "dtau", "dbeta", "dS0"):
+        assert_close(gr[n], ref[n], TOL[dtype], f"segmented {n}")

@@ -145,3 +145,48 @@ def test_tc_backward_wide_decay_preact_feedthrough(cuda_ok, dv):
     for n in GR:
         assert_close(gr[n], ref[n], TOL, f"wide head, preact, feedthrough: {n}")
     assert_close(gr["dfeed"], ref["dd"], TOL, "wide head: grad of the feedthrough weights")
+
+
+def test_tc_backward_wide_decay_long(cuda_ok):
+    """A wide head in a sequence long enough for the exact re-run to go in
+    segments, with gates passed before their activations and the feedthrough."""
+    from tests.test_gpu_feedthrough import feed_weights
+    T = 1024 + 300
+    x = draw_sequence(1, 2, T, 64, 128, torch.bfloat16, seed=41, s0_std=0.1, with_dO=True,
+                      preact=True)
+    g = x["g"].float()
+    g[:, 0, 700:760] = g[:, 0, 700:760] * 4.0 + 12.0
+    x["g"] = g.to(torch.bfloat16)
+    d = feed_weights(2, 128, 41)
+    dST = 0.1 * torch.randn(1, 2, 64, 128, generator=torch.Generator().manual_seed(41))
+    dx = {n: (t.cuda() if t is not None else None) for n, t in x.items()}
+    gr = rdm.rdm_ddts_bwd(*(dx[n] for n in SEQ), dx["S0"], dx["dO"], dST.cuda(), impl="tc",
+                          gates="preact", feedthrough=d.cuda())
+    torch.cuda.synchronize()
+    assert rdm.rdm_ddts_sync_status() == rdm.RDM_OK
+    ref = oracle.bwd(*(x[n] for n in SEQ), x["S0"], x["dO"], dST, preact=True, d=d)
+    for n in GR:
+        assert_close(gr[n], ref[n], TOL, f"long wide head: {n}")
+
+
+def test_workload3_backward_wide_heads_sampled(cuda_ok):
+    """The bench's wide-heads backward (every 16th head with one chunk's g x40,
+    re-run exactly in 8 segments of 512 tokens): a wide and a plain head against
+    the oracle."""
+    w = WORKLOADS[3]
+    x = draw_workload(w, device="cuda")
+    gw = x["g"].float()
+    gw[:, ::16, 64 * 20:64 * 21] *= 40.0
+    x["g"] = gw.clamp(min=0.05).to(torch.bfloat16)
+    del gw
+    saved = torch.empty(rdm.rdm_ddts_saved_states_size(w.B, w.H, w.T, w.dk, w.dv, 64) // 4,
+                        device="cuda")
+    rdm.rdm_ddts_fwd(*(x[n] for n in SEQ), x["S0"], saved_states=saved)
+    gr = rdm.rdm_ddts_bwd(*(x[n] for n in SEQ), x["S0"], x["dO"], None, saved)
+    torch.cuda.synchronize()
+    assert rdm.rdm_ddts_sync_status() == rdm.RDM_OK
+    for (b, h) in [(1, 0), (2, 5)]:
+        xs = {n: x[n][b:b + 1, h:h + 1].cpu() for n in SEQ + ("dO", "S0")}
+        ref = oracle.bwd(*(xs[n] for n in SEQ), xs["S0"], xs["dO"])
+        for n in GR:
+            assert_close(gr[n][b:b + 1, h:h + 1], ref[n], TOL, f"wide-heads workload ({b},{h}) {n}")
