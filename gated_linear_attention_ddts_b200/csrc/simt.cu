@@ -805,7 +805,7 @@ cudaError_t bwd_t(const BwdParams& p, float* dqf, float* fin, const int* list, i
 
 // The fix-up launch: blocks [slot * kFixBlocks, (slot + 1) * kFixBlocks) take the
 // heads slot, slot + slots, ... of the list (as the sweeps do).
-constexpr int kFixBlocks = 16;
+constexpr int kFixBlocks = 128;
 
 __device__ __forceinline__ int listed_heads(const int* list, int BH) { return list ? list[0] : BH; }
 __device__ __forceinline__ int listed_head(const int* list, int q) { return list ? list[1 + q] : q; }
