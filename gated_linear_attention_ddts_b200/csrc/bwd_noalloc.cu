@@ -1,8 +1,9 @@
 // bwd_noalloc.cu -- rdm_ddts_bwd_noalloc: the backward for callers that cannot
 // allocate device memory at the point of the call.
 //
-// The exact CUDA-core backward needs float32 scratch (q*dq for every token and
-// channel, plus one row per head).  rdm_ddts_bwd takes that scratch from the
+// The exact CUDA-core backward needs float32 scratch (dq for every token and
+// channel, one row per head and, for long sequences, the maps of its sequence
+// segments).  rdm_ddts_bwd takes that scratch from the
 // caller.  This variant takes it from a fixed array compiled into the library
 // instead, so a caller with no allocator at hand -- for example a serving
 // process whose device memory was carved up once at start-up and may not grow,

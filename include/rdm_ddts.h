@@ -242,8 +242,11 @@ size_t rdm_ddts_bwd_workspace_size(const rdm_bwd_args *args);
  *     relying on the no-allocation guarantee and before any stream capture.
  *     The address is looked up again on every call (it is cheap once the
  *     module is loaded), so it stays right across cudaDeviceReset.
- *   - Problems needing more scratch than 16 MiB (B*H*T*d_k*4 + B*H*d_k*4
- *     bytes) return RDM_ERR_WORKSPACE and launch nothing.
+ *   - Problems needing more scratch than 16 MiB return RDM_ERR_WORKSPACE
+ *     and launch nothing.  The figure is rdm_ddts_bwd_workspace_size with
+ *     impl = RDM_IMPL_SIMT: B*H*T*d_k*4 + B*H*d_k*4 + 4*(B*H+1) bytes (each
+ *     part rounded up to 256), plus, when T >= 1024 (the sweeps then run in
+ *     P = min(8, T/512) sequence segments), B*H*P*d_k*(d_v+2)*4 bytes.
  *   - All calls share the one array and it keeps whatever the last call left;
  *     nothing in it has to start at zero (each call writes every scratch
  *     element before reading it).  Calls whose kernels overlap on the GPU

@@ -195,3 +195,25 @@ def test_shortconv_many_validation(lib):
         assert lib.rdm_shortconv_fwd_many(mixed, 2, None) == RDM_ERR_INVALID_ARG, bad
     assert lib.rdm_shortconv_fwd_many((ConvArgs * 2)(_conv(), _conv(D=48)), 2, None) == RDM_ERR_UNSUPPORTED
     assert lib.rdm_shortconv_fwd_many((ConvArgs * 2)(_conv(), _conv(y=12290)), 2, None) == RDM_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("B,H,T,dk,dv", [(1, 1, 8, 64, 64), (2, 3, 1000, 32, 128),
+                                         (1, 2, 1024 + 37, 16, 32), (4, 16, 4096, 64, 128),
+                                         (1, 1, 9000, 128, 16)])
+def test_simt_workspace_size(lib, B, H, T, dk, dv):
+    """The exact backward's scratch as the header states it: dq, one row a head,
+    the flagged-head list and, from T = 1024 on, the maps of P = min(8, T/512)
+    sequence segments (each part rounded up to 256 bytes)."""
+    def up(x):
+        return (x + 255) // 256 * 256
+    P = min(8, T // 512) if T >= 1024 else 1
+    if P > 1:  # segments of whole 16-token tiles; the count actually used
+        tiles = (T + 15) // 16
+        seg = -(-tiles // P) * 16
+        P = -(-T // seg)
+    rows = B * H * dk
+    want = up(rows * T * 4) + up(rows * 4) + up((B * H + 1) * 4)
+    if P > 1:
+        want += up(rows * P * dv * 4) + 2 * up(rows * P * 4)
+    a = _bwd_args(B=B, H=H, T=T, dk=dk, dv=dv, impl=1)
+    assert lib.rdm_ddts_bwd_workspace_size(ctypes.byref(a)) == want
