@@ -125,9 +125,10 @@ __host__ __device__ __forceinline__ int ntiles_of(int T) { return (T + kTile - 1
 // with L the sum of log alpha over the segment's tokens and S_loc, C_loc the
 // results from a zero start.  So a pass computes S_loc / C_loc and L of every
 // segment (mode kSegLocal), and the full pass (kSegFull) of a segment folds the
-// maps before it (F) or after it (R) onto S_0 / dS_T and runs from there.  The decay-gradient carry into segment j from later segments,
-// fin + sum over later segments of their dG totals, is added afterwards to dg
-// and dtau of segment j by a fix-up launch.  P = 1 is the plain sweep.
+// maps before it (F) or after it (R) onto S_0 / dS_T and runs from there.  The
+// decay-gradient carry into segment j from later segments, fin + the sum of
+// their dG totals, is added afterwards to dg and dtau of segment j by a fix-up
+// launch.  P = 1 is the plain sweep.
 enum { kSegWhole = 0, kSegLocal = 1, kSegFull = 2 };
 struct SimtSeg {
     int P, seg_len, mode;
@@ -364,7 +365,8 @@ __device__ __forceinline__ void fsweep_head(const BwdParams& p, float* dqf, floa
             }
             float a = a0 + a1;
 #pragma unroll
-            for (int o = 1; o < TPR; o <<= 1) a += __shfl_xor_sync(0xffffffffu, a, o);  // the row's other columns
+            // the row's other columns
+            for (int o = 1; o < TPR; o <<= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
             if (act && cb == 0) s_part[buf][tt][i] = a;
         }
         // this block's partials of the tile are written (s_part alternates by tile:
@@ -576,7 +578,8 @@ __device__ __forceinline__ void rsweep_head(const BwdParams& p, const float* dqf
             }
             float d = d0 + d1;
 #pragma unroll
-            for (int o = 1; o < TPR; o <<= 1) d += __shfl_xor_sync(0xffffffffu, d, o);  // the row's other columns
+            // the row's other columns
+            for (int o = 1; o < TPR; o <<= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
             if (act && cb == 0) s_part[buf][tt][i] = d;  // this block's share of dkhat_{t,i}
             // dvhat_j = sum_i dS_ij khat_i over the warp's 32 / TPR rows (lanes with
             // the same l mod TPR): a reduce-scatter over the top lane bits (each
@@ -863,9 +866,9 @@ cudaError_t launch_simt_fwd(const SeqParams& p, cudaStream_t s) {
     return p.bf16 ? fwd_t<__nv_bfloat16>(p, s) : fwd_t<float>(p, s);
 }
 
-// scratch, float32: dq for every (b,h,t,i), the final-state term per (b,h,i), the
-// flagged-head list (int32) and, with segments, the segments' state slots [B H][P][d_k][d_v], their sums of log
-// alpha and of dG [B H][P][d_k]
+// scratch, float32: dq for every (b,h,t,i), the final-state term per (b,h,i),
+// the flagged-head list (int32) and, with segments, the segments' state slots
+// [B H][P][d_k][d_v], their sums of log alpha and of dG [B H][P][d_k]
 size_t simt_bwd_workspace(const BwdParams& p) {
     int P, len;
     simt_segments(p.T, &P, &len);
