@@ -13,9 +13,13 @@ exchange), time is the max over ranks and `value` counts all ranks' tokens.
 
 At N = 1 the same line also carries, under "workloads", the long-context
 forward (B=1, H=16, T=32768, d_k=d_v=128, S_T returned), the training
-forward+backward (B=4, H=16, T=4096, d_k=64, d_v=128) and the batched decode
-(B=256, H=16, d_k=64, d_v=128, 1024 steps in one CUDA graph), each with the
-roofline of its kernels, and the fp64 oracle timed on the host cores.
+forward+backward (B=4, H=16, T=4096, d_k=64, d_v=128), the same backward with
+every 16th head given one chunk too wide for one decay reference (those heads
+are recomputed by the exact CUDA-core backward), the batched decode (B=256,
+H=16, d_k=64, d_v=128, 1024 steps in one CUDA graph), the forward variants
+(gates before their activations, rank-16 beta_hat, feedthrough), ShortConv
+and SW-SKA, each with the roofline of its kernels, and the fp64 oracle timed on
+the host cores.
 
 `--impl reference` times the fp64 CPU oracle (the only reference: the pages
 publish no implementation) on bounded samples of the headline workload.
