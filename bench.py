@@ -346,9 +346,10 @@ def run_extras(rdm, dev, pk, K):
     out["training_fwd_bwd"] = {
         "workload": w.name, "value": w.B * w.T / ((msf + msb) / 1e3), "unit": "tokens/s",
         "ms_per_step": msf + msb, "ms_fwd": msf, "ms_bwd": msb,
-        # forward kernel; backward kernel + the two exact re-run kernels (they exit at
-        # once for heads the tensor-core kernel handled)
-        "gpu_launches_per_step": 4,
+        # forward kernel; backward kernel, the flagged-head list and the exact
+        # re-run (local and full passes of both sweeps over 8 segments, the carry
+        # fix-up: small grids that exit at once when no head is flagged)
+        "gpu_launches_per_step": 8,
         "roofline_fwd": roofline(fb, chunk_flops_fwd(w), msf, pk,
                                  ncu_counters("tc_fwd_kernel", FWD_SRC, 3)),
         "roofline_bwd": roofline(bwd_bytes(w), chunk_flops_bwd(w), msb, pk,
@@ -369,8 +370,8 @@ def run_extras(rdm, dev, pk, K):
         "workload": w.name + ", one chunk in every 16th head too wide for one reference",
         "value": w.B * w.T / (msw / 1e3), "unit": "tokens/s", "ms_per_step": msw,
         "ms_bwd_without": msb, "wide_heads": w.B * ((w.H + 15) // 16),
-        # backward kernel + the two exact re-run kernels
-        "gpu_launches_per_step": 3,
+        # backward kernel, the flagged-head list and the five exact re-run launches
+        "gpu_launches_per_step": 7,
         # the backward's algorithmic bytes over the whole step: the recomputed heads
         # are latency-bound token-serial sweeps, not a bandwidth problem
         "roofline": roofline(bwd_bytes(w), chunk_flops_bwd(w), msw, pk, None),
